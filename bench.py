@@ -1,0 +1,418 @@
+#!/usr/bin/env python
+"""Benchmark of the looped nGPT hot path on B200.
+
+Workload: the 4B-shaped model (d=2560, vocab 131072, 20 q-heads x 128, 4 KV
+heads, SwiGLU 10240, 16 + 40 + 16 physical layers, window 4096) in bf16 with
+seeded random weights; batch 1, a 2560-token uniform-random prompt, then
+greedy decode at k=2 with the last-loop KV cache.  One "step" is one decode
+step (every row of the hot path: embed, the input block, k passes of the
+recurrent block with re-injection, the output block, the LM head and the
+argmax).  The decode steps stream ~11.2 GB of weights each, far above the
+126 MB L2, so no flush is needed between steps.
+
+Default: 1 GPU.  Under torchrun each rank runs an independent replica (the
+path shards over sequences with no exchange), so scaling is weak; the time is
+the max over ranks.  --impl reference times the oracle on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode tokens/s at k=1/2/4 (last-loop KV), % HBM roofline; prefill TFLOP/s"
+
+
+def peaks():
+    try:
+        p = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", 1400.0)), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------- algorithmic work
+def weight_bytes(shape, k):
+    """Weight bytes one decode step streams at loop count k (bf16)."""
+    d, q, kv, f = shape.d_model, shape.q_dim, shape.kv_dim, shape.d_ff
+    attn = (q + 2 * kv) * d + d * q
+    mlp = 3 * f * d
+    def block(n):
+        return (n // 2) * attn + (n - n // 2) * mlp
+    per = block(shape.n_in) + k * block(shape.n_rec) + block(shape.n_out)
+    return 2 * (per + shape.vocab * d + d)  # + LM head + one embedding row
+
+
+def kv_read_bytes(shape, k, ctx):
+    """KV bytes one decode step at context ctx reads (all attention
+    applications; each key is K+V of every KV head)."""
+    per_key = 2 * shape.kv_dim * 2
+    tot = 0
+    j = 0
+    for l in range(shape.n_layers):
+        if l % 2:
+            continue
+        full = (j % shape.full_every) == shape.full_phase
+        j += 1
+        rec = shape.n_in <= l < shape.n_in + shape.n_rec
+        keys = ctx if full else min(ctx, shape.swa_window)
+        tot += (k if rec else 1) * keys * per_key
+    return tot
+
+
+def proj_flops(shape, k, tokens):
+    return 2 * tokens * (weight_bytes(shape, k) / 2 - shape.vocab * shape.d_model - shape.d_model)
+
+
+def attn_flops_prefill(shape, k, T):
+    pairs_full = T * (T + 1) // 2
+    W = shape.swa_window
+    pairs_swa = sum(min(p + 1, W) for p in range(T))
+    per = 4 * shape.n_heads * shape.head_dim
+    tot = 0
+    j = 0
+    for l in range(shape.n_layers):
+        if l % 2:
+            continue
+        full = (j % shape.full_every) == shape.full_phase
+        j += 1
+        rec = shape.n_in <= l < shape.n_in + shape.n_rec
+        tot += (k if rec else 1) * (pairs_full if full else pairs_swa) * per
+    return tot
+
+
+# ---------------------------------------------------------------- clocks
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        try:
+            self.p.wait(5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        rows = [r.split(", ") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm = [float(r[1]) for r in rows if len(r) >= 9 and r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if len(r) >= 9 and r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows if len(r) >= 9 for i in range(4) if r[5 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max(i.get("num_threads", 1) for i in threadpool_info()) or (os.cpu_count() or 1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def host_mem_gb():
+    try:
+        for line in open("/proc/meminfo"):
+            if line.startswith("MemAvailable"):
+                return int(line.split()[1]) / 1e6
+    except Exception:
+        pass
+    return 0.0
+
+
+def oracle_decode_rate(shape, weights, k, mode, prompt_len, steps, seed=1):
+    """Oracle (float32 on the host) decode tokens/s on a bounded sample:
+    prefill a short prompt, then time `steps` greedy decode steps."""
+    import oracle as O
+    m = O.Model(shape, weights, dtype=np.float32)
+    prompt = __import__("synth").make_prompt(seed, prompt_len, shape.vocab)
+    cache = O.Cache(m, prompt_len + steps + 2)
+    lg = O.forward_chunk(m, cache, prompt, k, mode)
+    tok = int(np.argmax(lg[-1]))
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        lg = O.forward_chunk(m, cache, [tok], k, mode)
+        tok = int(np.argmax(lg[-1]))
+    dt = time.perf_counter() - t0
+    return steps / dt, dt
+
+
+# ---------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--prompt", type=int, default=2560)
+    ap.add_argument("--k", type=int, default=2)
+    ap.add_argument("--mode", default="last_loop", choices=["last_loop", "per_loop"])
+    ap.add_argument("--no-aux", action="store_true", help="skip the k sweep, e2e and CPU baseline legs")
+    ap.add_argument("--profile-steps", type=int, default=3)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    import synth
+    shape = synth.DORY_4B
+    workload = f"dory4b_bf16_batch1_prompt{args.prompt}_decode_k{args.k}_{args.mode}"
+    hbm, tc, tc_sus, peak_src = peaks()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        run_reference(args, shape, workload)
+        return
+
+    import torch
+    import looped_ngpt_lm_b200 as dory
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+
+    w_np = synth.make_weights(shape, 1)
+    dw = dory.DeviceWeights(shape, w_np)
+    if rank != 0 or args.no_aux:
+        del w_np
+        w_np = None
+    max_seq = args.prompt + args.warmup + args.steps + 64
+    cfg = dory.make_config(shape, max_batch=1, max_seq=max_seq, k_max=4, gamma_max=4, max_chunk=args.prompt)
+    h = dory.Handle(cfg, dw, dory.LAST_LOOP if args.mode == "last_loop" else dory.PER_LOOP)
+    mode = dory.MODES[args.mode]
+    stream = torch.cuda.current_stream()
+    prompt = torch.tensor(synth.make_prompt(1, args.prompt, shape.vocab), dtype=torch.int32, device="cuda")
+
+    def barrier():
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- prefill (timed on its own: projection + attention TFLOP/s)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    pre_ms = []
+    for rep in range(2):
+        h.reset()
+        barrier()
+        a, b = ev(), ev()
+        a.record(stream)
+        first = h.prefill([0], prompt, [args.prompt], args.k, mode)
+        b.record(stream)
+        torch.cuda.synchronize()
+        pre_ms.append(a.elapsed_time(b))
+    h.synchronize()
+    pre_ms = max_over_ranks(min(pre_ms))
+    pf = proj_flops(shape, args.k, args.prompt)
+    af = attn_flops_prefill(shape, args.k, args.prompt)
+
+    # ---- decode: warm-up, then exactly K timed steps
+    bufs = [torch.empty(1, dtype=torch.int32, device="cuda") for _ in range(2)]
+    tok = first
+    for i in range(args.warmup):
+        tok = h.decode_step([0], tok, args.k, mode, next_tokens=bufs[i % 2])
+    barrier()
+    clocks = Clocks(local)
+    clocks.start()
+    t0, t1 = ev(), ev()
+    t0.record(stream)
+    for i in range(args.steps):
+        tok = h.decode_step([0], tok, args.k, mode, next_tokens=bufs[i % 2])
+    t1.record(stream)
+    barrier()
+    clk = clocks.stop()
+    h.synchronize()
+    dec_ms = max_over_ranks(t0.elapsed_time(t1))
+    ms_step = dec_ms / args.steps
+    value = world * args.steps / (dec_ms / 1e3)
+    ctx_mid = args.prompt + args.warmup + args.steps // 2
+    step_bytes = weight_bytes(shape, args.k) + kv_read_bytes(shape, args.k, ctx_mid)
+
+    # ---- per-kernel timing (CUDA events around every launch, same stream)
+    h.profile_reset()
+    h.set_option(dory.OPT_PROFILE, 1)
+    for i in range(args.profile_steps):
+        tok = h.decode_step([0], tok, args.k, mode, next_tokens=bufs[i % 2])
+    prof = h.profile_read()
+    h.set_option(dory.OPT_PROFILE, 0)
+    launches_per_step = sum(v["launches"] for v in prof.values()) / args.profile_steps
+    gemm = {n: v for n, v in prof.items() if n.startswith("gemm")}
+    g_ms = sum(v["ms"] for v in gemm.values())
+    g_bytes = sum(v["bytes"] for v in gemm.values())
+    g_launch = sum(v["launches"] for v in gemm.values())
+    tot_ms = sum(v["ms"] for v in prof.values())
+    achieved = g_bytes / (g_ms / 1e3) / 1e9 if g_ms > 0 else 0.0
+    roofline = {"bound": "hbm", "kernel": "gemm (decode projections + LM head)", "achieved": round(achieved, 1),
+                "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4), "peak_source": peak_src,
+                "traffic": None, "bytes_per_launch": round(g_bytes / max(g_launch, 1)),
+                "avg_launch_us": round(1e3 * g_ms / max(g_launch, 1), 2),
+                "share_of_step": round(g_ms / tot_ms, 4) if tot_ms else None}
+    kernel_share = {n: round(v["ms"] / tot_ms, 4) for n, v in sorted(prof.items(), key=lambda kv: -kv[1]["ms"])}
+
+    aux = {}
+    e2e = None
+    cpu = None
+    if not args.no_aux and world == 1:
+        # ---- k sweep (short runs, same context)
+        sweep = {}
+        for kk in (1, 2, 4):
+            n = 32
+            a, b = ev(), ev()
+            for i in range(3):
+                tok = h.decode_step([0], tok, kk, mode, next_tokens=bufs[i % 2])
+            torch.cuda.synchronize()
+            a.record(stream)
+            for i in range(n):
+                tok = h.decode_step([0], tok, kk, mode, next_tokens=bufs[i % 2])
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / n
+            ctx = h.seq_len(0)
+            by = weight_bytes(shape, kk) + kv_read_bytes(shape, kk, ctx)
+            sweep[f"k{kk}"] = {"tokens_per_s": round(1e3 / ms, 2), "ms_per_token": round(ms, 4),
+                               "hbm_frac_of_measured": round(by / (ms / 1e3) / 1e9 / hbm, 4),
+                               "bytes_per_token": by, "ctx": ctx}
+        aux["decode_k_sweep_last_loop" if args.mode == "last_loop" else "decode_k_sweep"] = sweep
+        # ---- end to end: every step copies its input token from pinned host
+        # memory and reads the chosen token back, through the public API
+        pin_in = torch.empty(1, dtype=torch.int32).pin_memory()
+        pin_out = torch.empty(1, dtype=torch.int32).pin_memory()
+        d_in = torch.empty(1, dtype=torch.int32, device="cuda")
+        pin_in[0] = int(tok[0])
+        n = min(args.steps, 100)
+        torch.cuda.synchronize()
+        a, b = ev(), ev()
+        a.record(stream)
+        for i in range(n):
+            d_in.copy_(pin_in, non_blocking=True)
+            out = h.decode_step([0], d_in, args.k, mode, next_tokens=bufs[i % 2])
+            pin_out.copy_(out, non_blocking=True)
+            stream.synchronize()
+            pin_in[0] = pin_out[0]
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b)
+        e2e = {"value": round(n / (e_ms / 1e3), 2), "unit": "tokens/s", "h2d_bytes_per_step": 4,
+               "d2h_bytes_per_step": 4, "steps": n,
+               "note": "host-driven greedy loop: pinned H2D of the input token, decode step, D2H of the choice, sync"}
+        # ---- CPU oracle baseline (bounded sample)
+        if rank == 0 and w_np is not None:
+            if host_mem_gb() > 40:
+                rate, secs = oracle_decode_rate(shape, w_np, args.k, args.mode, 8, 3)
+                cpu = {"value": round(rate, 4), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                       "sample": f"float32 oracle, 4B shape, 8-token prompt then 3 greedy decode steps at "
+                                 f"k={args.k} {args.mode} ({secs:.1f} s timed)"}
+            else:
+                cpu = {"value": None, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                       "sample": f"skipped: {host_mem_gb():.0f} GB host memory available, the fp32 oracle needs ~40"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded N(0,1) weights with L2-normalised rows (bf16), uniform random prompt ids",
+            "config": {"workload": workload, "model": "looped nGPT 4B-shaped", "global_batch": world,
+                       "seq_len": args.prompt, "k": args.k, "cache_mode": args.mode,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2: each step streams ~11 GB of weights"},
+            "hbm": {"bytes_per_step": step_bytes, "achieved_GBs": round(step_bytes / (ms_step / 1e3) / 1e9, 1),
+                    "frac_of_measured": round(step_bytes / (ms_step / 1e3) / 1e9 / hbm, 4),
+                    "frac_of_8TBs": round(step_bytes / (ms_step / 1e3) / 8e12, 4)},
+            "prefill": {"tokens": args.prompt, "ms": round(pre_ms, 3),
+                        "proj_tflops": round(pf / (pre_ms / 1e3) / 1e12, 2),
+                        "total_tflops": round((pf + af) / (pre_ms / 1e3) / 1e12, 2),
+                        "proj_frac_of_measured_bf16": round(pf / (pre_ms / 1e3) / 1e12 / tc, 4)},
+            "roofline": roofline,
+            "kernel_share": kernel_share,
+            "gpu_launches": int(round(launches_per_step * args.steps)),
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        line.update(aux)
+        print(json.dumps(line))
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args, shape, workload):
+    """Reference arm: the oracle on the host cores, one decode step per step,
+    on a bounded sample (8-token prompt; steps capped to keep the run short)."""
+    import synth
+    w = synth.make_weights(shape, 1)
+    if host_mem_gb() < 40:
+        print(json.dumps({"impl": "reference", "unavailable": "the float32 oracle of the 4B shape needs ~40 GB of host memory"}))
+        return
+    import oracle as O
+    m = O.Model(shape, w, dtype=np.float32)
+    del w
+    prompt = synth.make_prompt(1, 8, shape.vocab)
+    steps = min(args.steps, 4)
+    warm = min(args.warmup, 1)
+    cache = O.Cache(m, 8 + steps + warm + 2)
+    lg = O.forward_chunk(m, cache, prompt, args.k, args.mode)
+    tok = int(np.argmax(lg[-1]))
+    for _ in range(warm):
+        tok = int(np.argmax(O.forward_chunk(m, cache, [tok], args.k, args.mode)[-1]))
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        tok = int(np.argmax(O.forward_chunk(m, cache, [tok], args.k, args.mode)[-1]))
+    dt = time.perf_counter() - t0
+    v = steps / dt
+    sample = f"float32 oracle, 4B shape, 8-token prompt, {steps} timed greedy decode steps at k={args.k} {args.mode}"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "tokens/s", "n_gpus": 1,
+        "steps": steps, "warmup": warm, "ms_per_step": round(1e3 * dt / steps, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": workload, "model": "looped nGPT 4B-shaped", "global_batch": 1, "seq_len": 8},
+        "cpu_baseline": {"value": round(v, 4), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(v, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,232 @@
+/*
+ * dory.h -- C ABI of the looped normalized-GPT inference library (libdory.so).
+ *
+ * The library runs the per-token forward of a looped nGPT language model on
+ * one NVIDIA B200 (sm_100a): an input block run once, a shared recurrent block
+ * run k times with the input re-injected every loop, an output block and an
+ * LM head, over a KV cache in last-loop or per-loop mode.
+ *
+ * Sources (web pages about Dory1.0-4B; section names translated):
+ *   [digest]  onedev.kr/papers/1692 "Dory1.0-4B는 반복 횟수로 추론 연산과
+ *             정확도를 조절한다": "How it works" (block split, recurrence
+ *             s0=x, u_t=N(s_{t-1}+x), s_t=N(F(u_t)), 72/112/192 layer
+ *             applications, 36 MLP / 27 sliding-window / 9 full attention
+ *             layers), "Premises & limits" (last-loop KV caching and its
+ *             final-loop mismatch; self-speculative decoding with draft k=1,
+ *             verify k=4, gamma=4, KV and activation reuse).
+ *   [news]    lucasainews.com "NVIDIA, 루프 구조 4B 모델 Dory1.0-4B 4가지
+ *             정밀도로 공개": "Looped structure" (input re-injected every loop),
+ *             "How to run" (loop count 1..4 chosen at inference; the
+ *             recurrent KV cache mode switch last_loop / per-loop).
+ *   [review]  blog.secrett2633.cloud "[논문리뷰] Dory1.0-4B: A Looped
+ *             Normalized-GPT", "1. Key Terms" (nGPT: L2-normalised states;
+ *             last-loop KV caching keeps the footprint of one loop).
+ *
+ * Conventions for every entry point:
+ *   - Return DORY_OK or an error status; dory_last_error() gives the message.
+ *   - Arguments are validated before any work is queued: an error leaves the
+ *     handle and its caches unchanged.
+ *   - Pointers marked "device" are CUDA device pointers, "host" are host
+ *     pointers.  The caller owns every buffer it passes; the library keeps no
+ *     pointer past the call except the weights and workspace given to
+ *     dory_create, which must outlive the handle.
+ *   - Work is queued on the caller's stream (a cudaStream_t passed as
+ *     dory_stream; NULL is the legacy default stream) and returns before it
+ *     finishes, except where a function says it synchronises.
+ *   - The library never allocates device memory: all device state lives in
+ *     the caller-provided workspace.
+ *   - A handle is not thread-safe; use one host thread per handle.
+ */
+#ifndef DORY_H
+#define DORY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct dory_handle dory_handle;
+typedef void* dory_stream; /* cudaStream_t */
+
+typedef enum {
+  DORY_OK = 0,
+  DORY_ERR_INVALID_ARG = 1, /* bad pointer, size, k, gamma, seq id, ... */
+  DORY_ERR_CAPACITY = 2,    /* request exceeds max_seq / max_chunk / max_batch */
+  DORY_ERR_STATE = 3,       /* call not allowed in the sequence's current state */
+  DORY_ERR_WORKSPACE = 4,   /* workspace too small or misaligned */
+  DORY_ERR_CUDA = 5,        /* a CUDA runtime call failed */
+  DORY_ERR_TIMEOUT = 6,     /* a device-side bounded wait gave up */
+  DORY_ERR_UNSUPPORTED = 7  /* valid but not supported by this build */
+} dory_status;
+
+/* Recurrent-block KV cache mode ([digest] "Premises & limits"; [news] "How to run").
+ * LAST_LOOP: one slot per attention layer; every loop overwrites it, so a
+ *            token's cached K/V are those of its final loop and the cache size
+ *            does not depend on k.  Queries in loop t < k of a later token see
+ *            the final-loop K/V of earlier tokens.
+ * PER_LOOP:  each recurrent attention layer keeps one slot per loop; loop t
+ *            reads and writes slot t.  Cache size grows with k. */
+typedef enum { DORY_LAST_LOOP = 0, DORY_PER_LOOP = 1 } dory_cache_mode;
+
+typedef enum { DORY_F32 = 0, DORY_BF16 = 1 } dory_dtype;
+
+/* Model shape and capacity.  Layer counts are physical layers: physical layers
+ * alternate attention and MLP, attention first; attention layer j (counted
+ * over the whole stack) is full causal when j % full_every == full_phase and
+ * sliding-window (keys p-W < j <= p) otherwise ([digest] "How it works":
+ * attention interleaved 3:1).  Weights and the KV cache are stored in dtype;
+ * hidden states are fp32; GEMMs accumulate in fp32. */
+typedef struct {
+  int32_t d_model, vocab, n_heads, head_dim, n_kv_heads, d_ff;
+  int32_t n_in, n_rec, n_out;     /* physical layers of the input, recurrent, output blocks */
+  int32_t swa_window;             /* W */
+  int32_t full_every, full_phase; /* 4, 3 for the 3:1 interleave */
+  int32_t dtype;                  /* dory_dtype */
+  int32_t max_batch;              /* number of sequence slots (seq ids 0..max_batch-1) */
+  int32_t max_seq;                /* positions per sequence */
+  int32_t k_max;                  /* largest loop count a call may use (1..4) */
+  int32_t gamma_max;              /* largest speculative draft length (0 disables) */
+  int32_t max_chunk;              /* most new tokens in one forward, summed over the batch */
+} dory_config;
+
+/* Device weight pointers, BORROWED (must outlive the handle).  All matrices
+ * are row-major [out, in] in dtype.  The per-layer arrays are HOST arrays of
+ * n_in+n_rec+n_out device pointers (copied at dory_create); entries for the
+ * other layer kind are ignored.
+ *   embed   [vocab, d]         token embedding (rows are used as given)
+ *   lm_head [vocab, d]         untied LM head: logits = s . lm_head^T
+ *   w_qkv   [q + 2 kv, d]      rows 0..q-1 = W_q, then W_k, then W_v
+ *                              (q = n_heads*head_dim, kv = n_kv_heads*head_dim)
+ *   w_o     [d, q]
+ *   w_gu    [2 d_ff, d]        rows 0..d_ff-1 = W_gate, then W_up
+ *   w_down  [d, d_ff]
+ * The MLP is W_down (silu(W_gate h) * (W_up h)); attention head h reads KV
+ * head h / (n_heads / n_kv_heads); the softmax scale is 1/sqrt(head_dim). */
+typedef struct {
+  const void* embed;
+  const void* lm_head;
+  const void* const* w_qkv;
+  const void* const* w_o;
+  const void* const* w_gu;
+  const void* const* w_down;
+} dory_weights;
+
+typedef struct {
+  int64_t steps;    /* verify passes */
+  int64_t drafted;  /* draft tokens proposed */
+  int64_t accepted; /* draft tokens accepted */
+} dory_spec_stats;
+
+/* Bytes of device workspace dory_create needs for this configuration.
+ * alloc_mode PER_LOOP reserves k_max slots for every recurrent attention
+ * layer (and still serves LAST_LOOP calls); LAST_LOOP reserves one. */
+dory_status dory_workspace_size(const dory_config* cfg, dory_cache_mode alloc_mode, size_t* bytes);
+
+/* Create a handle over caller-owned device memory.  workspace: device
+ * pointer, 256-byte aligned, ws_bytes >= dory_workspace_size().  The
+ * workspace is not cleared here; call dory_reset(h, -1, stream) before the
+ * first prefill.  Host-only: queues no device work. */
+dory_status dory_create(const dory_config* cfg, const dory_weights* w, dory_cache_mode alloc_mode,
+                        void* workspace, size_t ws_bytes, dory_handle** out);
+
+dory_status dory_destroy(dory_handle* h);
+
+/* Empty sequence `seq` (or all sequences when seq == -1): its length becomes 0
+ * and its cache mode and loop count are forgotten. */
+dory_status dory_reset(dory_handle* h, int32_t seq, dory_stream stream);
+
+/* Prefill: append lens[i] tokens to sequence seq_ids[i] for i < batch, as one
+ * forward chunk per sequence at loop count k, and choose the next token of
+ * each sequence (greedy, lowest id on ties).
+ *   seq_ids      host int32[batch], distinct, in [0, max_batch)
+ *   tokens       device int32[sum(lens)], the sequences' tokens concatenated
+ *   lens         host int32[batch], each >= 1; sum(lens) <= max_chunk
+ *   k            1..k_max
+ *   mode         fixed per sequence from its first prefill; per_loop
+ *                sequences must keep the same k in every later call
+ *   last_logits  device float[batch, vocab] or NULL: logits of each
+ *                sequence's last new position
+ *   next_tokens  device int32[batch]
+ * Within a chunk, loop t of every position writes its loop-t K/V and attends
+ * to the chunk's loop-t K/V plus the cached K/V of earlier calls. */
+dory_status dory_prefill(dory_handle* h, int32_t batch, const int32_t* seq_ids, const int32_t* tokens,
+                         const int32_t* lens, int32_t k, dory_cache_mode mode, float* last_logits,
+                         int32_t* next_tokens, dory_stream stream);
+
+/* One decode step: append tokens_in[i] to sequence seq_ids[i] and choose its
+ * next token.  seq_ids host int32[batch]; tokens_in device int32[batch];
+ * logits device float[batch, vocab] or NULL; next_tokens device int32[batch]. */
+dory_status dory_decode_step(dory_handle* h, int32_t batch, const int32_t* seq_ids, const int32_t* tokens_in,
+                             int32_t k, dory_cache_mode mode, float* logits, int32_t* next_tokens,
+                             dory_stream stream);
+
+/* Self-speculative greedy decoding ([digest] "Premises & limits"): each step
+ * drafts gamma tokens one at a time at k_draft, verifies the chunk
+ * [pending, d_1..d_gamma] at k_verify reusing the drafts' input-block output,
+ * loop-1 state and K/V, accepts the longest prefix the verifier agrees with
+ * plus the verifier's own next token, and rolls the cache back to the
+ * accepted length.  Steps repeat until every sequence has max_new tokens.
+ *   last_tokens  device int32[batch]: each sequence's pending token (the
+ *                token chosen by its prefill or last decode, not yet in the cache)
+ *   out_tokens   device int32[batch, max_new]; out_len device int32[batch]
+ *   stats        host, may be NULL
+ * k_draft must be 1 (loop-1 reuse); gamma in 1..gamma_max; k_verify in 1..k_max.
+ * Needs len + max_new + 2*gamma + 1 <= max_seq for every sequence (a sequence
+ * that finishes first keeps drafting from its frozen length while the others
+ * continue).  Synchronises the stream after every verify step to test for
+ * completion.
+ * In PER_LOOP mode the output equals plain k_verify greedy decoding. */
+dory_status dory_spec_decode(dory_handle* h, int32_t batch, const int32_t* seq_ids, const int32_t* last_tokens,
+                             int32_t k_draft, int32_t k_verify, int32_t gamma, dory_cache_mode mode,
+                             int32_t max_new, int32_t* out_tokens, int32_t* out_len, dory_spec_stats* stats,
+                             dory_stream stream);
+
+/* KV bytes one sequence of ctx tokens holds at loop count k in `mode` (the
+ * positions a future query can still read: the last W for a sliding-window
+ * layer, all for a full layer).  Host only. */
+dory_status dory_kv_bytes(const dory_handle* h, int32_t k, dory_cache_mode mode, int64_t ctx, int64_t* bytes);
+
+/* Committed length of a sequence as known to the host (exact after every
+ * call returns; dory_spec_decode synchronises before returning). */
+dory_status dory_seq_len(const dory_handle* h, int32_t seq, int32_t* len);
+
+/* Copy fp32 rows of the last forward pass's states into device dst[rows, d]:
+ * which = 0: x (input-block output), 1: s_k (final loop state),
+ * 2: output-block result.  rows = the last call's chunk rows. */
+dory_status dory_read_state(dory_handle* h, int32_t which, float* dst, int32_t rows, dory_stream stream);
+
+/* Copy a sequence's cached K and V of physical attention layer `layer`, slot
+ * `slot` (0 unless PER_LOOP recurrent: loop t -> slot t-1), positions
+ * [pos0, pos0+n) into device k_dst/v_dst [n, n_kv_heads, head_dim] (dtype).
+ * Positions must still be retained (ring slots of sliding-window layers). */
+dory_status dory_read_kv(dory_handle* h, int32_t layer, int32_t slot, int32_t seq, int32_t pos0, int32_t n,
+                         void* k_dst, void* v_dst, dory_stream stream);
+
+/* Synchronise `stream` and report device-side errors (DORY_ERR_TIMEOUT when
+ * a bounded wait in a kernel gave up; the handle stays usable). */
+dory_status dory_synchronize(dory_handle* h, dory_stream stream);
+
+/* Options. */
+enum {
+  DORY_OPT_CUDA_GRAPHS = 1, /* 1 (default): replay captured decode steps */
+  DORY_OPT_PROFILE = 2,     /* 1: time every launch with CUDA events (slow) */
+  DORY_OPT_GEMM_IMPL = 3    /* bf16 GEMM: 0 auto, 1 SIMT reference kernel, 2 tcgen05 */
+};
+dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value);
+
+/* Per-kernel launch statistics gathered while DORY_OPT_PROFILE is on:
+ * fills up to n entries of names (host char[n][48]), launches, total_ms and
+ * algorithmic bytes; returns the number of kernels in *count. */
+dory_status dory_profile_read(dory_handle* h, int32_t n, char (*names)[48], int64_t* launches,
+                              double* total_ms, double* bytes, int32_t* count);
+dory_status dory_profile_reset(dory_handle* h);
+
+/* Message of the last failed call on this host thread ("" if none). */
+const char* dory_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DORY_H */

@@ -1,0 +1,276 @@
+"""Python binding of libdory.so (the looped nGPT C ABI declared in include/dory.h).
+
+Argument marshalling only: every step of the forward runs in the library's
+CUDA kernels.  PyTorch supplies device memory and streams.  Importing this
+package fails loudly when the compiled library is missing; there is no CPU
+fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdory.so")
+
+LAST_LOOP = 0
+PER_LOOP = 1
+F32 = 0
+BF16 = 1
+MODES = {"last_loop": LAST_LOOP, "per_loop": PER_LOOP, LAST_LOOP: LAST_LOOP, PER_LOOP: PER_LOOP}
+
+OPT_CUDA_GRAPHS = 1
+OPT_PROFILE = 2
+OPT_GEMM_IMPL = 3
+
+STATUS = {0: "DORY_OK", 1: "DORY_ERR_INVALID_ARG", 2: "DORY_ERR_CAPACITY", 3: "DORY_ERR_STATE",
+          4: "DORY_ERR_WORKSPACE", 5: "DORY_ERR_CUDA", 6: "DORY_ERR_TIMEOUT", 7: "DORY_ERR_UNSUPPORTED"}
+
+# Every entry point include/dory.h declares.
+SYMBOLS = ["dory_workspace_size", "dory_create", "dory_destroy", "dory_reset", "dory_prefill",
+           "dory_decode_step", "dory_spec_decode", "dory_kv_bytes", "dory_seq_len", "dory_read_state",
+           "dory_read_kv", "dory_synchronize", "dory_set_option", "dory_profile_read", "dory_profile_reset",
+           "dory_last_error"]
+
+
+class DoryError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class Config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "d_model", "vocab", "n_heads", "head_dim", "n_kv_heads", "d_ff", "n_in", "n_rec", "n_out",
+        "swa_window", "full_every", "full_phase", "dtype", "max_batch", "max_seq", "k_max", "gamma_max",
+        "max_chunk")]
+
+
+class Weights(ctypes.Structure):
+    _fields_ = [("embed", ctypes.c_void_p), ("lm_head", ctypes.c_void_p),
+                ("w_qkv", ctypes.POINTER(ctypes.c_void_p)), ("w_o", ctypes.POINTER(ctypes.c_void_p)),
+                ("w_gu", ctypes.POINTER(ctypes.c_void_p)), ("w_down", ctypes.POINTER(ctypes.c_void_p))]
+
+
+class SpecStats(ctypes.Structure):
+    _fields_ = [("steps", ctypes.c_int64), ("drafted", ctypes.c_int64), ("accepted", ctypes.c_int64)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python looped_ngpt_lm_b200/build.py`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    IP = ctypes.POINTER(ctypes.c_int32)
+    sig = {
+        "dory_workspace_size": [ctypes.POINTER(Config), I32, ctypes.POINTER(SZ)],
+        "dory_create": [ctypes.POINTER(Config), ctypes.POINTER(Weights), I32, P, SZ, ctypes.POINTER(P)],
+        "dory_destroy": [P],
+        "dory_reset": [P, I32, P],
+        "dory_prefill": [P, I32, IP, P, IP, I32, I32, P, P, P],
+        "dory_decode_step": [P, I32, IP, P, I32, I32, P, P, P],
+        "dory_spec_decode": [P, I32, IP, P, I32, I32, I32, I32, I32, P, P, ctypes.POINTER(SpecStats), P],
+        "dory_kv_bytes": [P, I32, I32, I64, ctypes.POINTER(I64)],
+        "dory_seq_len": [P, I32, IP],
+        "dory_read_state": [P, I32, P, I32, P],
+        "dory_read_kv": [P, I32, I32, I32, I32, I32, P, P, P],
+        "dory_synchronize": [P, P],
+        "dory_set_option": [P, I32, I64],
+        "dory_profile_read": [P, I32, P, ctypes.POINTER(I64), ctypes.POINTER(ctypes.c_double),
+                              ctypes.POINTER(ctypes.c_double), IP],
+        "dory_profile_reset": [P],
+    }
+    for name, args in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = ctypes.c_int
+    lib.dory_last_error.argtypes = []
+    lib.dory_last_error.restype = ctypes.c_char_p
+    return lib
+
+
+lib = _load()
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        raise DoryError(status, lib.dory_last_error().decode())
+
+
+def make_config(shape, max_batch=1, max_seq=256, k_max=4, gamma_max=4, max_chunk=None) -> Config:
+    """C config for a synth.Shape plus capacity."""
+    return Config(shape.d_model, shape.vocab, shape.n_heads, shape.head_dim, shape.n_kv_heads, shape.d_ff,
+                  shape.n_in, shape.n_rec, shape.n_out, shape.swa_window, shape.full_every, shape.full_phase,
+                  BF16 if shape.dtype == "bf16" else F32, max_batch, max_seq, k_max, gamma_max,
+                  max_chunk if max_chunk is not None else max_seq)
+
+
+def _ptr(t) -> int:
+    return t.data_ptr() if t is not None else None
+
+
+def _stream(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class DeviceWeights:
+    """Model weights in device memory, packed into the C ABI's layout
+    (q|k|v rows stacked into w_qkv, gate|up rows into w_gu)."""
+
+    def __init__(self, shape, weights: dict, device="cuda"):
+        import torch
+        self.shape = shape
+        self.bf16 = shape.dtype == "bf16"
+
+        def up(a):
+            if self.bf16:
+                t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+            else:
+                t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+            return t.to(device, non_blocking=False)
+
+        self.tensors = {"embed": up(weights["embed"]), "lm_head": up(weights["lm_head"])}
+        L = shape.n_layers
+        self.qkv, self.o, self.gu, self.down = [None] * L, [None] * L, [None] * L, [None] * L
+        for l in range(L):
+            if f"L{l}.wq" in weights:
+                self.qkv[l] = up(np.concatenate([weights[f"L{l}.wq"], weights[f"L{l}.wk"], weights[f"L{l}.wv"]]))
+                self.o[l] = up(weights[f"L{l}.wo"])
+            else:
+                self.gu[l] = up(np.concatenate([weights[f"L{l}.wg"], weights[f"L{l}.wu"]]))
+                self.down[l] = up(weights[f"L{l}.wdown"])
+        arr = ctypes.c_void_p * L
+        self._qkv = arr(*[_ptr(t) for t in self.qkv])
+        self._o = arr(*[_ptr(t) for t in self.o])
+        self._gu = arr(*[_ptr(t) for t in self.gu])
+        self._down = arr(*[_ptr(t) for t in self.down])
+        self.c = Weights(self.tensors["embed"].data_ptr(), self.tensors["lm_head"].data_ptr(),
+                         self._qkv, self._o, self._gu, self._down)
+
+
+def workspace_size(cfg: Config, alloc_mode=LAST_LOOP) -> int:
+    n = ctypes.c_size_t()
+    _check(lib.dory_workspace_size(ctypes.byref(cfg), MODES[alloc_mode], ctypes.byref(n)))
+    return n.value
+
+
+class Handle:
+    """One dory_handle over a torch-allocated workspace."""
+
+    def __init__(self, cfg: Config, weights: DeviceWeights, alloc_mode=LAST_LOOP, device="cuda"):
+        import torch
+        self.cfg = cfg
+        self.weights = weights
+        self.alloc_mode = MODES[alloc_mode]
+        nbytes = workspace_size(cfg, self.alloc_mode)
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        h = ctypes.c_void_p()
+        _check(lib.dory_create(ctypes.byref(cfg), ctypes.byref(weights.c), self.alloc_mode,
+                               ctypes.c_void_p(self.workspace.data_ptr()), nbytes, ctypes.byref(h)))
+        self.h = h
+        self.reset()
+
+    def close(self):
+        if self.h:
+            lib.dory_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @staticmethod
+    def _ids(seq_ids):
+        a = (ctypes.c_int32 * len(seq_ids))(*[int(s) for s in seq_ids])
+        return a
+
+    def reset(self, seq=-1, stream=None):
+        _check(lib.dory_reset(self.h, seq, _stream(stream)))
+
+    def set_option(self, opt, value):
+        _check(lib.dory_set_option(self.h, opt, int(value)))
+
+    def prefill(self, seq_ids, tokens, lens, k, mode, logits=None, next_tokens=None, stream=None):
+        import torch
+        ids = self._ids(seq_ids)
+        ln = (ctypes.c_int32 * len(lens))(*[int(x) for x in lens])
+        if next_tokens is None:
+            next_tokens = torch.empty(len(seq_ids), dtype=torch.int32, device=tokens.device)
+        _check(lib.dory_prefill(self.h, len(seq_ids), ids, ctypes.c_void_p(tokens.data_ptr()), ln, k, MODES[mode],
+                                ctypes.c_void_p(_ptr(logits)), ctypes.c_void_p(next_tokens.data_ptr()),
+                                _stream(stream)))
+        return next_tokens
+
+    def decode_step(self, seq_ids, tokens_in, k, mode, logits=None, next_tokens=None, stream=None):
+        import torch
+        ids = self._ids(seq_ids)
+        if next_tokens is None:
+            next_tokens = torch.empty(len(seq_ids), dtype=torch.int32, device=tokens_in.device)
+        _check(lib.dory_decode_step(self.h, len(seq_ids), ids, ctypes.c_void_p(tokens_in.data_ptr()), k,
+                                    MODES[mode], ctypes.c_void_p(_ptr(logits)),
+                                    ctypes.c_void_p(next_tokens.data_ptr()), _stream(stream)))
+        return next_tokens
+
+    def spec_decode(self, seq_ids, last_tokens, k_draft, k_verify, gamma, mode, max_new, stream=None):
+        import torch
+        ids = self._ids(seq_ids)
+        B = len(seq_ids)
+        out = torch.zeros((B, max_new), dtype=torch.int32, device=last_tokens.device)
+        out_len = torch.zeros(B, dtype=torch.int32, device=last_tokens.device)
+        st = SpecStats()
+        _check(lib.dory_spec_decode(self.h, B, ids, ctypes.c_void_p(last_tokens.data_ptr()), k_draft, k_verify,
+                                    gamma, MODES[mode], max_new, ctypes.c_void_p(out.data_ptr()),
+                                    ctypes.c_void_p(out_len.data_ptr()), ctypes.byref(st), _stream(stream)))
+        return out, out_len, {"steps": st.steps, "drafted": st.drafted, "accepted": st.accepted}
+
+    def kv_bytes(self, k, mode, ctx) -> int:
+        n = ctypes.c_int64()
+        _check(lib.dory_kv_bytes(self.h, k, MODES[mode], ctx, ctypes.byref(n)))
+        return n.value
+
+    def seq_len(self, seq) -> int:
+        n = ctypes.c_int32()
+        _check(lib.dory_seq_len(self.h, seq, ctypes.byref(n)))
+        return n.value
+
+    def read_state(self, which, rows, stream=None):
+        import torch
+        out = torch.empty((rows, self.cfg.d_model), dtype=torch.float32, device=self.workspace.device)
+        sel = {"x": 0, "s": 1, "out": 2}[which] if isinstance(which, str) else which
+        _check(lib.dory_read_state(self.h, sel, ctypes.c_void_p(out.data_ptr()), rows, _stream(stream)))
+        return out
+
+    def read_kv(self, layer, slot, seq, pos0, n, stream=None):
+        import torch
+        dt = torch.bfloat16 if self.cfg.dtype == BF16 else torch.float32
+        k = torch.empty((n, self.cfg.n_kv_heads, self.cfg.head_dim), dtype=dt, device=self.workspace.device)
+        v = torch.empty_like(k)
+        _check(lib.dory_read_kv(self.h, layer, slot, seq, pos0, n, ctypes.c_void_p(k.data_ptr()),
+                                ctypes.c_void_p(v.data_ptr()), _stream(stream)))
+        return k, v
+
+    def synchronize(self, stream=None):
+        _check(lib.dory_synchronize(self.h, _stream(stream)))
+
+    def profile_reset(self):
+        _check(lib.dory_profile_reset(self.h))
+
+    def profile_read(self):
+        n = 64
+        names = (ctypes.c_char * 48 * n)()
+        launches = (ctypes.c_int64 * n)()
+        ms = (ctypes.c_double * n)()
+        by = (ctypes.c_double * n)()
+        cnt = ctypes.c_int32()
+        _check(lib.dory_profile_read(self.h, n, ctypes.cast(names, ctypes.c_void_p), launches, ms, by,
+                                     ctypes.byref(cnt)))
+        out = {}
+        for i in range(min(cnt.value, n)):
+            out[bytes(names[i]).split(b"\0")[0].decode()] = {"launches": launches[i], "ms": ms[i], "bytes": by[i]}
+        return out

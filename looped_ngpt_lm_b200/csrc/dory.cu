@@ -1,0 +1,843 @@
+// Host runner and C ABI of the looped nGPT library.
+//
+// The forward of one chunk of new tokens follows the recurrence of the
+// Dory1.0-4B digest (onedev.kr/papers/1692, "How it works"): the input block
+// runs once, the shared recurrent block runs k times on u_t = N(s_{t-1} + x)
+// with s_0 = x and s_t = N(F(u_t)), then the output block and the LM head
+// run on s_k.  Every physical layer updates h <- N(h + sublayer(h)).  The KV
+// cache follows the same digest's "Premises & limits": in last-loop mode a
+// recurrent attention layer has one slot that every loop overwrites; in
+// per-loop mode loop t has its own slot.
+//
+// All device state lives in the caller's workspace; nothing here allocates
+// device memory.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "dory.h"
+#include "gemm_tc.cuh"
+#include "kernels.cuh"
+
+using namespace dory;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+dory_status fail(dory_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+dory_status fail(dory_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+#define CK(expr)                                                                                  \
+  do {                                                                                            \
+    cudaError_t e_ = (expr);                                                                      \
+    if (e_ != cudaSuccess) return fail(DORY_ERR_CUDA, "%s: %s", #expr, cudaGetErrorString(e_)); \
+  } while (0)
+
+// Bump allocator over the workspace (or a size counter when base == nullptr).
+struct Carve {
+  char* base;
+  size_t off = 0;
+  template <typename P>
+  P* take(size_t bytes) {
+    off = (off + 255) & ~(size_t)255;
+    P* p = base ? (P*)(base + off) : nullptr;
+    off += bytes;
+    return p;
+  }
+};
+
+struct AttnLayer {
+  int layer;      // physical layer index
+  bool full;      // full causal (else sliding window)
+  bool rec;       // in the recurrent block
+  int cap;        // positions held: ring size (window) or max_seq (full)
+  int nslots;     // 1, or k_max for per-loop recurrent layers
+  char* K[8];
+  char* V[8];
+};
+
+struct ProfRec {
+  int name;
+  double bytes;
+  cudaEvent_t a, b;
+};
+
+}  // namespace
+
+struct dory_handle {
+  dory_config c{};
+  int alloc_mode = 0;
+  bool bf16 = false;
+  int esz = 4;
+  int L = 0, q_dim = 0, kv_dim = 0, qkv_dim = 0, slack = 0, M_max = 0, head_max = 0, nb_max = 0;
+  const void* embed = nullptr;
+  const void* head = nullptr;
+  std::vector<const void*> w_qkv, w_o, w_gu, w_down;
+  std::vector<int> attn_of;
+  std::vector<AttnLayer> attn;
+
+  // device buffers (inside the workspace)
+  char* ws = nullptr;
+  size_t ws_bytes = 0;
+  int *seq_len = nullptr, *err = nullptr, *seq_ids = nullptr, *tokens = nullptr, *next = nullptr;
+  int *cu = nullptr, *head_rows = nullptr;
+  RowMeta meta{};
+  float *h = nullptr, *x = nullptr, *s = nullptr, *q = nullptr, *part_qkv = nullptr, *part_y = nullptr,
+        *part_gu = nullptr, *attn_part = nullptr, *logits = nullptr;
+  void *hop = nullptr, *ao = nullptr, *act = nullptr, *kscr = nullptr, *vscr = nullptr, *hop_head = nullptr;
+  size_t part_rows = 0;
+  float *stash_x = nullptr, *stash_s = nullptr;
+  int *drafts = nullptr, *pending = nullptr, *vtok = nullptr, *out_len = nullptr, *all_done = nullptr;
+  unsigned long long* accepted = nullptr;
+
+  // host state
+  std::vector<int> len, mode, kfix;  // per sequence; mode -1 = empty
+  std::vector<int> ids_on_device;     // seq ids last uploaded to seq_ids
+  int last_rows = 0;
+  bool graphs = true, profile = false;
+  int gemm_impl = 0;
+  std::vector<std::string> prof_names;
+  std::vector<ProfRec> prof_recs;
+  std::vector<cudaEvent_t> ev_pool;
+  size_t ev_used = 0;
+
+  template <typename T>
+  T* hop_t() const { return (T*)hop; }
+};
+
+namespace {
+
+// ------------------------------------------------------------------ layout
+bool layer_is_attn(int l) { return l % 2 == 0; }
+
+dory_status check_config(const dory_config* c) {
+  if (!c) return fail(DORY_ERR_INVALID_ARG, "config is NULL");
+  if (c->d_model <= 0 || c->vocab <= 0 || c->n_heads <= 0 || c->head_dim <= 0 || c->n_kv_heads <= 0 ||
+      c->d_ff <= 0)
+    return fail(DORY_ERR_INVALID_ARG, "non-positive model dimension");
+  if (c->n_in < 0 || c->n_rec <= 0 || c->n_out < 0) return fail(DORY_ERR_INVALID_ARG, "bad block sizes");
+  if (c->n_heads % c->n_kv_heads) return fail(DORY_ERR_INVALID_ARG, "n_heads %% n_kv_heads != 0");
+  if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128)
+    return fail(DORY_ERR_UNSUPPORTED, "head_dim must be 32, 64 or 128");
+  int G = c->n_heads / c->n_kv_heads;
+  if (!(G == 1 || G == 2 || G == 4 || G == 5 || (G == 8 && c->head_dim <= 64)))
+    return fail(DORY_ERR_UNSUPPORTED, "query heads per KV head must be 1, 2, 4, 5 or 8");
+  if (c->d_model > 4096) return fail(DORY_ERR_UNSUPPORTED, "d_model > 4096");
+  if (c->d_model % 8 || c->d_ff % 8) return fail(DORY_ERR_UNSUPPORTED, "d_model and d_ff must be multiples of 8");
+  if (c->swa_window <= 0) return fail(DORY_ERR_INVALID_ARG, "swa_window must be >= 1");
+  if (c->full_every <= 0 || c->full_phase < 0) return fail(DORY_ERR_INVALID_ARG, "bad full-attention pattern");
+  if (c->dtype != DORY_F32 && c->dtype != DORY_BF16) return fail(DORY_ERR_INVALID_ARG, "bad dtype");
+  if (c->max_batch <= 0 || c->max_seq <= 0 || c->max_chunk <= 0) return fail(DORY_ERR_INVALID_ARG, "bad capacity");
+  if (c->k_max < 1 || c->k_max > 8) return fail(DORY_ERR_INVALID_ARG, "k_max must be in 1..8");
+  if (c->gamma_max < 0 || c->gamma_max > 16) return fail(DORY_ERR_INVALID_ARG, "gamma_max must be in 0..16");
+  return DORY_OK;
+}
+
+// Fill the handle's layout; with h->ws == nullptr only sizes are computed.
+size_t layout(dory_handle* h) {
+  const dory_config& c = h->c;
+  Carve cv{h->ws};
+  h->bf16 = c.dtype == DORY_BF16;
+  h->esz = h->bf16 ? 2 : 4;
+  h->L = c.n_in + c.n_rec + c.n_out;
+  h->q_dim = c.n_heads * c.head_dim;
+  h->kv_dim = c.n_kv_heads * c.head_dim;
+  h->qkv_dim = h->q_dim + 2 * h->kv_dim;
+  // sliding-window rings keep W + slack positions so that speculative writes
+  // past the accepted length never evict a key a later query still needs
+  h->slack = ((c.gamma_max + 1 + 15) / 16) * 16;
+  h->M_max = std::max(c.max_chunk, c.max_batch * (c.gamma_max + 1));
+  h->head_max = std::max(c.max_batch * (c.gamma_max + 1), c.max_batch);
+  h->nb_max = (c.max_seq + ATTN_BK - 1) / ATTN_BK + 1;
+  const int M = h->M_max;
+  const size_t e = h->esz;
+
+  h->attn.clear();
+  h->attn_of.assign(h->L, -1);
+  int j = 0;
+  for (int l = 0; l < h->L; ++l) {
+    if (!layer_is_attn(l)) continue;
+    AttnLayer a{};
+    a.layer = l;
+    a.full = (j % c.full_every) == c.full_phase;
+    a.rec = l >= c.n_in && l < c.n_in + c.n_rec;
+    a.cap = a.full ? c.max_seq : std::min(c.max_seq, c.swa_window + h->slack);
+    a.nslots = (h->alloc_mode == DORY_PER_LOOP && a.rec) ? c.k_max : 1;
+    size_t bytes = (size_t)c.max_batch * c.n_kv_heads * a.cap * c.head_dim * e;
+    for (int s = 0; s < a.nslots; ++s) {
+      a.K[s] = cv.take<char>(bytes);
+      a.V[s] = cv.take<char>(bytes);
+    }
+    h->attn_of[l] = (int)h->attn.size();
+    h->attn.push_back(a);
+    ++j;
+  }
+  const int d = c.d_model;
+  h->seq_len = cv.take<int>(sizeof(int) * c.max_batch);
+  h->err = cv.take<int>(sizeof(int) * 4);
+  h->seq_ids = cv.take<int>(sizeof(int) * M);
+  h->tokens = cv.take<int>(sizeof(int) * M);
+  h->next = cv.take<int>(sizeof(int) * M);
+  h->cu = cv.take<int>(sizeof(int) * (c.max_batch + 1));
+  h->head_rows = cv.take<int>(sizeof(int) * h->head_max);
+  h->meta.seq = cv.take<int>(sizeof(int) * M);
+  h->meta.pos = cv.take<int>(sizeof(int) * M);
+  h->meta.p0 = cv.take<int>(sizeof(int) * M);
+  h->meta.base = cv.take<int>(sizeof(int) * M);
+  h->meta.pend = cv.take<int>(sizeof(int) * M);
+  h->h = cv.take<float>(sizeof(float) * M * d);
+  h->x = cv.take<float>(sizeof(float) * M * d);
+  h->s = cv.take<float>(sizeof(float) * M * d);
+  h->q = cv.take<float>(sizeof(float) * M * h->q_dim);
+  h->hop = cv.take<char>(e * M * std::max(d, 1));
+  h->ao = cv.take<char>(e * M * h->q_dim);
+  h->act = cv.take<char>(e * M * c.d_ff);
+  h->kscr = cv.take<char>(e * M * h->kv_dim);
+  h->vscr = cv.take<char>(e * M * h->kv_dim);
+  h->hop_head = cv.take<char>(e * h->head_max * d);
+  h->part_rows = (size_t)M * kMaxSplitK;
+  h->part_qkv = cv.take<float>(sizeof(float) * h->part_rows * h->qkv_dim);
+  h->part_y = cv.take<float>(sizeof(float) * h->part_rows * d);
+  h->part_gu = cv.take<float>(sizeof(float) * h->part_rows * 2 * c.d_ff);
+  h->attn_part = cv.take<float>(sizeof(float) * (size_t)M * c.n_heads * h->nb_max * (c.head_dim + 2));
+  h->logits = cv.take<float>(sizeof(float) * (size_t)h->head_max * c.vocab * kMaxSplitK);
+  const int gc = c.gamma_max + 1;
+  h->stash_x = cv.take<float>(sizeof(float) * (size_t)c.max_batch * gc * d);
+  h->stash_s = cv.take<float>(sizeof(float) * (size_t)c.max_batch * gc * d);
+  h->drafts = cv.take<int>(sizeof(int) * c.max_batch * gc);
+  h->pending = cv.take<int>(sizeof(int) * c.max_batch);
+  h->vtok = cv.take<int>(sizeof(int) * c.max_batch * gc);
+  h->out_len = cv.take<int>(sizeof(int) * c.max_batch);
+  h->all_done = cv.take<int>(sizeof(int) * 4);
+  h->accepted = cv.take<unsigned long long>(sizeof(unsigned long long) * 2);
+  return cv.off + 256;
+}
+
+// ------------------------------------------------------------------ profiling
+struct Scope {
+  dory_handle* H;
+  cudaStream_t st;
+  ProfRec rec{};
+  bool on;
+  Scope(dory_handle* h, cudaStream_t s, const char* name, double bytes) : H(h), st(s), on(h->profile) {
+    if (!on) return;
+    int id = -1;
+    for (size_t i = 0; i < H->prof_names.size(); ++i)
+      if (H->prof_names[i] == name) id = (int)i;
+    if (id < 0) {
+      id = (int)H->prof_names.size();
+      H->prof_names.push_back(name);
+    }
+    rec.name = id;
+    rec.bytes = bytes;
+    rec.a = event();
+    rec.b = event();
+    cudaEventRecord(rec.a, st);
+  }
+  cudaEvent_t event() {
+    if (H->ev_used == H->ev_pool.size()) {
+      cudaEvent_t e;
+      cudaEventCreate(&e);
+      H->ev_pool.push_back(e);
+    }
+    return H->ev_pool[H->ev_used++];
+  }
+  ~Scope() {
+    if (!on) return;
+    cudaEventRecord(rec.b, st);
+    H->prof_recs.push_back(rec);
+  }
+};
+
+// ------------------------------------------------------------------ forward pieces
+template <typename T>
+struct Fwd {
+  dory_handle* H;
+  cudaStream_t st;
+  int M;        // chunk rows
+  int max_ctx;  // bound on (position + 1) of every row
+  bool direct;  // K/V of the chunk go straight into the cache
+  int mode;     // dory_cache_mode
+};
+
+KVView kv_view(dory_handle* H, int l, int loop, int mode) {
+  AttnLayer& a = H->attn[H->attn_of[l]];
+  int slot = (mode == DORY_PER_LOOP && a.rec && loop >= 1) ? loop - 1 : 0;
+  KVView v;
+  v.K = a.K[slot];
+  v.V = a.V[slot];
+  v.cap = a.cap;
+  v.window = a.full ? 0 : H->c.swa_window;
+  v.limit = H->c.max_seq;
+  v.err = H->err;
+  return v;
+}
+
+template <typename T>
+dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, const void* W, float* Y, int ldy,
+                 int* S_out, size_t* ps_out, const char* name) {
+  dory_handle* H = f.H;
+  double bytes = (double)N * K * sizeof(T) + (double)M * K * sizeof(T) + (double)M * N * 4;
+  Scope sc(H, f.st, name, bytes);
+  *S_out = 1;
+  *ps_out = 0;
+  if constexpr (sizeof(T) == 2) {
+    if (H->gemm_impl != 1) {
+      int S = 1;
+      size_t ps = 0;
+      cudaError_t e = launch_gemm_tc(M, N, K, (const bf16*)X, ldx, (const bf16*)W, Y, ldy, H->part_rows,
+                                     H->err, &S, &ps, f.st);
+      if (e == cudaSuccess) {
+        *S_out = S;
+        *ps_out = ps;
+        return DORY_OK;
+      }
+      if (e != cudaErrorNotSupported) return fail(DORY_ERR_CUDA, "%s: %s", name, cudaGetErrorString(e));
+      if (H->gemm_impl == 2) return fail(DORY_ERR_UNSUPPORTED, "%s: shape not supported by tcgen05 GEMM", name);
+    }
+  }
+  CK(launch_gemm_simt<T>(M, N, K, X, ldx, (const T*)W, Y, ldy, f.st));
+  return DORY_OK;
+}
+
+#define RET(x)                          \
+  do {                                  \
+    dory_status r_ = (x);               \
+    if (r_ != DORY_OK) return r_;       \
+  } while (0)
+
+template <typename T>
+dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop) {
+  dory_handle* H = f.H;
+  const dory_config& c = H->c;
+  const int M = f.M, d = c.d_model;
+  for (int l = l0; l < l1; ++l) {
+    int S;
+    size_t ps;
+    if (layer_is_attn(l)) {
+      KVView kv = kv_view(H, l, loop, f.mode);
+      RET(gemm<T>(f, M, H->qkv_dim, d, H->hop_t<T>(), d, H->w_qkv[l], H->part_qkv, H->qkv_dim, &S, &ps, "gemm_qkv"));
+      {
+        Scope sc(H, f.st, "qkv_post", 0);
+        CK(launch_qkv_post<T>(M, c.n_heads, c.n_kv_heads, c.head_dim, H->part_qkv, S, ps, H->q, (T*)H->kscr,
+                              (T*)H->vscr, f.direct, kv, H->meta, c.max_batch, f.st));
+      }
+      {
+        Scope sc(H, f.st, "attention", 0);
+        CK(launch_attention<T>(M, c.n_heads, c.n_kv_heads, c.head_dim, H->q, (const T*)H->kscr,
+                               (const T*)H->vscr, !f.direct, kv, H->meta, f.max_ctx, H->attn_part, (T*)H->ao,
+                               f.st));
+      }
+      if (!f.direct) {
+        Scope sc(H, f.st, "kv_commit", 0);
+        CK(launch_kv_commit<T>(M, c.n_kv_heads, c.head_dim, (const T*)H->kscr, (const T*)H->vscr, kv, H->meta,
+                               f.st));
+      }
+      RET(gemm<T>(f, M, d, H->q_dim, (const T*)H->ao, H->q_dim, H->w_o[l], H->part_y, d, &S, &ps, "gemm_o"));
+    } else {
+      RET(gemm<T>(f, M, 2 * c.d_ff, d, H->hop_t<T>(), d, H->w_gu[l], H->part_gu, 2 * c.d_ff, &S, &ps,
+                  "gemm_gate_up"));
+      {
+        Scope sc(H, f.st, "swiglu", 0);
+        CK(launch_swiglu<T>(M, c.d_ff, H->part_gu, S, ps, (T*)H->act, f.st));
+      }
+      RET(gemm<T>(f, M, d, c.d_ff, (const T*)H->act, c.d_ff, H->w_down[l], H->part_y, d, &S, &ps, "gemm_down"));
+    }
+    Scope sc(H, f.st, "addnorm", 0);
+    CK(launch_addnorm<T>(M, d, H->h, H->part_y, S, ps, d, H->hop_t<T>(), f.st));
+  }
+  return DORY_OK;
+}
+
+// Embed + input block; x <- h.
+template <typename T>
+dory_status input_block(const Fwd<T>& f, const int* tokens) {
+  dory_handle* H = f.H;
+  const dory_config& c = H->c;
+  {
+    Scope sc(H, f.st, "embed", 0);
+    CK(launch_embed<T>(f.M, c.d_model, c.vocab, tokens, (const T*)H->embed, H->h, H->hop_t<T>(), H->err, f.st));
+  }
+  RET(run_layers<T>(f, 0, c.n_in, 0));
+  CK(cudaMemcpyAsync(H->x, H->h, sizeof(float) * f.M * c.d_model, cudaMemcpyDeviceToDevice, f.st));
+  return DORY_OK;
+}
+
+// Loops t0..k of the recurrent block; on entry h holds x (t0 == 1) or s
+// holds s_{t0-1} (t0 > 1).  Leaves s_k in h and s.  If stash_col >= 0, s_1
+// is written to the stash (rows_per_seq rps).
+template <typename T>
+dory_status loops(const Fwd<T>& f, int t0, int k, int stash_col, int rps) {
+  dory_handle* H = f.H;
+  const dory_config& c = H->c;
+  const int d = c.d_model, gc = c.gamma_max + 1;
+  for (int t = t0; t <= k; ++t) {
+    // entry: u_t = N(s_{t-1} + x); s_0 = x; s_{t-1} = N(h) after loop t-1
+    int src = (t == 1) ? 0 : (t == t0 ? 2 : 1);
+    float* save = (t > 1 && t - 1 == 1 && stash_col >= 0) ? H->stash_s : nullptr;
+    {
+      Scope sc(H, f.st, "reinject", 0);
+      CK(launch_reinject<T>(f.M, d, H->h, H->x, src, H->s, true, H->hop_t<T>(), save, rps, gc,
+                            stash_col < 0 ? 0 : stash_col, f.st));
+    }
+    RET(run_layers<T>(f, c.n_in, c.n_in + c.n_rec, t));
+  }
+  // exit: s_k = N(h) (or s_k = s when no loop ran here)
+  float* save = (k == 1 && stash_col >= 0) ? H->stash_s : nullptr;
+  Scope sc(H, f.st, "reinject", 0);
+  if (t0 > k) {
+    CK(launch_reinject<T>(f.M, d, H->h, H->x, 2, H->s, false, H->hop_t<T>(), nullptr, 1, 1, 0, f.st));
+  } else {
+    CK(launch_reinject<T>(f.M, d, H->h, H->x, 1, nullptr, false, H->hop_t<T>(), save, rps, gc,
+                          stash_col < 0 ? 0 : stash_col, f.st));
+  }
+  CK(cudaMemcpyAsync(H->s, H->h, sizeof(float) * f.M * d, cudaMemcpyDeviceToDevice, f.st));
+  return DORY_OK;
+}
+
+// Output block on h, then LM head + argmax on `nrows` rows (all rows when
+// rows == nullptr, else the listed rows).  Choices go to `choice`.
+template <typename T>
+dory_status output_and_head(const Fwd<T>& f, int nrows, const int* rows, float* logits_out, int* choice) {
+  dory_handle* H = f.H;
+  const dory_config& c = H->c;
+  const int d = c.d_model;
+  RET(run_layers<T>(f, c.n_in + c.n_rec, H->L, 0));
+  const T* X = H->hop_t<T>();
+  if (rows) {
+    Scope sc(H, f.st, "gather", 0);
+    CK(launch_gather_rows<T>(nrows, d, rows, H->hop_t<T>(), (T*)H->hop_head, f.st));
+    X = (const T*)H->hop_head;
+  }
+  float* lg = logits_out ? logits_out : H->logits;
+  int S;
+  size_t ps;
+  RET(gemm<T>(f, nrows, c.vocab, d, X, d, H->head, lg, c.vocab, &S, &ps, "gemm_lm_head"));
+  if (S != 1) return fail(DORY_ERR_CUDA, "LM head GEMM must not split K");
+  Scope sc(H, f.st, "argmax", 0);
+  CK(launch_argmax(nrows, c.vocab, lg, choice, f.st));
+  return DORY_OK;
+}
+
+dory_status upload_ids(dory_handle* H, const int32_t* ids, int n, cudaStream_t st) {
+  if ((int)H->ids_on_device.size() == n && std::equal(ids, ids + n, H->ids_on_device.begin())) return DORY_OK;
+  CK(cudaMemcpyAsync(H->seq_ids, ids, sizeof(int) * n, cudaMemcpyHostToDevice, st));
+  H->ids_on_device.assign(ids, ids + n);
+  return DORY_OK;
+}
+
+dory_status check_seqs(dory_handle* H, int batch, const int32_t* seq_ids, int k, int mode) {
+  const dory_config& c = H->c;
+  if (batch <= 0 || batch > c.max_batch) return fail(DORY_ERR_INVALID_ARG, "batch %d outside 1..%d", batch, c.max_batch);
+  if (!seq_ids) return fail(DORY_ERR_INVALID_ARG, "seq_ids is NULL");
+  if (k < 1 || k > c.k_max) return fail(DORY_ERR_INVALID_ARG, "k=%d outside 1..%d", k, c.k_max);
+  if (mode != DORY_LAST_LOOP && mode != DORY_PER_LOOP) return fail(DORY_ERR_INVALID_ARG, "bad cache mode");
+  if (mode == DORY_PER_LOOP && H->alloc_mode != DORY_PER_LOOP)
+    return fail(DORY_ERR_STATE, "per_loop call on a handle allocated for last_loop");
+  for (int i = 0; i < batch; ++i) {
+    int sq = seq_ids[i];
+    if (sq < 0 || sq >= c.max_batch) return fail(DORY_ERR_INVALID_ARG, "seq id %d outside 0..%d", sq, c.max_batch - 1);
+    for (int j = 0; j < i; ++j)
+      if (seq_ids[j] == sq) return fail(DORY_ERR_INVALID_ARG, "seq id %d repeated", sq);
+    if (H->mode[sq] >= 0 && H->mode[sq] != mode)
+      return fail(DORY_ERR_STATE, "sequence %d was started in the other cache mode", sq);
+    if (mode == DORY_PER_LOOP && H->mode[sq] >= 0 && H->kfix[sq] != k)
+      return fail(DORY_ERR_STATE, "per_loop sequence %d was started at k=%d, not %d", sq, H->kfix[sq], k);
+  }
+  return DORY_OK;
+}
+
+void mark_started(dory_handle* H, int batch, const int32_t* seq_ids, int k, int mode) {
+  for (int i = 0; i < batch; ++i) {
+    int sq = seq_ids[i];
+    if (H->mode[sq] < 0) {
+      H->mode[sq] = mode;
+      H->kfix[sq] = k;
+    }
+  }
+}
+
+template <typename T>
+dory_status prefill_t(dory_handle* H, int batch, const int32_t* seq_ids, const int32_t* tokens, const int32_t* lens,
+                      int k, int mode, float* last_logits, int32_t* next_tokens, cudaStream_t st) {
+  const dory_config& c = H->c;
+  std::vector<int> cu(batch + 1, 0), rows(batch);
+  int max_ctx = 0;
+  for (int i = 0; i < batch; ++i) {
+    cu[i + 1] = cu[i] + lens[i];
+    rows[i] = cu[i + 1] - 1;
+    max_ctx = std::max(max_ctx, H->len[seq_ids[i]] + lens[i]);
+  }
+  const int M = cu[batch];
+  RET(upload_ids(H, seq_ids, batch, st));
+  CK(cudaMemcpyAsync(H->cu, cu.data(), sizeof(int) * (batch + 1), cudaMemcpyHostToDevice, st));
+  CK(cudaMemcpyAsync(H->head_rows, rows.data(), sizeof(int) * batch, cudaMemcpyHostToDevice, st));
+  CK(launch_plan_ragged(batch, M, H->cu, H->seq_ids, H->seq_len, H->meta, st));
+  int max_len = *std::max_element(lens, lens + batch);
+  Fwd<T> f{H, st, M, max_ctx, max_len <= H->slack + 1, mode};
+  RET(input_block<T>(f, tokens));
+  RET(loops<T>(f, 1, k, -1, 1));
+  RET(output_and_head<T>(f, batch, H->head_rows, last_logits, next_tokens));
+  CK(launch_advance_ragged(batch, H->seq_ids, H->cu, H->seq_len, st));
+  for (int i = 0; i < batch; ++i) H->len[seq_ids[i]] += lens[i];
+  H->last_rows = M;
+  return DORY_OK;
+}
+
+template <typename T>
+dory_status decode_t(dory_handle* H, int batch, const int32_t* seq_ids, const int32_t* tokens_in, int k, int mode,
+                     float* logits, int32_t* next_tokens, cudaStream_t st) {
+  int max_ctx = 0;
+  for (int i = 0; i < batch; ++i) max_ctx = std::max(max_ctx, H->len[seq_ids[i]] + 1);
+  RET(upload_ids(H, seq_ids, batch, st));
+  CK(launch_plan_uniform(batch, 1, 0, H->seq_ids, H->seq_len, H->meta, st));
+  Fwd<T> f{H, st, batch, max_ctx, true, mode};
+  RET(input_block<T>(f, tokens_in));
+  RET(loops<T>(f, 1, k, -1, 1));
+  RET(output_and_head<T>(f, batch, nullptr, logits, next_tokens));
+  CK(launch_advance(batch, H->seq_ids, H->seq_len, 1, st));
+  for (int i = 0; i < batch; ++i) H->len[seq_ids[i]] += 1;
+  H->last_rows = batch;
+  return DORY_OK;
+}
+
+template <typename T>
+dory_status spec_t(dory_handle* H, int B, const int32_t* seq_ids, const int32_t* last_tokens, int kv_, int gamma,
+                   int mode, int max_new, int32_t* out_tokens, int32_t* out_len, dory_spec_stats* stats,
+                   cudaStream_t st) {
+  const dory_config& c = H->c;
+  const int gc = c.gamma_max + 1;
+  int max_ctx = 0;
+  for (int i = 0; i < B; ++i) max_ctx = std::max(max_ctx, H->len[seq_ids[i]] + max_new + 2 * gamma + 1);
+  RET(upload_ids(H, seq_ids, B, st));
+  CK(cudaMemcpyAsync(H->pending, last_tokens, sizeof(int) * B, cudaMemcpyDeviceToDevice, st));
+  CK(cudaMemsetAsync(out_len, 0, sizeof(int) * B, st));
+  CK(cudaMemsetAsync(H->accepted, 0, sizeof(unsigned long long), st));
+  int64_t steps = 0;
+  for (;;) {
+    // drafts: y0, d1..d_{gamma-1} at k = 1, one token per sequence each
+    for (int i = 0; i < gamma; ++i) {
+      CK(launch_plan_uniform(B, 1, i, H->seq_ids, H->seq_len, H->meta, st));
+      Fwd<T> f{H, st, B, max_ctx, true, mode};
+      const int* tok = i == 0 ? H->pending : H->drafts + (i - 1) * B;
+      RET(input_block<T>(f, tok));
+      CK(launch_stash_copy(B, c.d_model, H->x, H->stash_x, 1, gc, i, 0, st));
+      RET(loops<T>(f, 1, 1, i, 1));
+      RET(output_and_head<T>(f, B, nullptr, nullptr, H->drafts + i * B));
+    }
+    // d_gamma: input block and loop 1 only
+    {
+      CK(launch_plan_uniform(B, 1, gamma, H->seq_ids, H->seq_len, H->meta, st));
+      Fwd<T> f{H, st, B, max_ctx, true, mode};
+      RET(input_block<T>(f, H->drafts + (gamma - 1) * B));
+      CK(launch_stash_copy(B, c.d_model, H->x, H->stash_x, 1, gc, gamma, 0, st));
+      Scope sc(H, st, "reinject", 0);
+      CK(launch_reinject<T>(B, c.d_model, H->h, H->x, 0, nullptr, true, H->hop_t<T>(), nullptr, 1, 1, 0, st));
+      RET(run_layers<T>(f, c.n_in, c.n_in + c.n_rec, 1));
+      CK(launch_reinject<T>(B, c.d_model, H->h, H->x, 1, nullptr, false, H->hop_t<T>(), H->stash_s, 1, gc, gamma,
+                            st));
+    }
+    // verify [y0, d1..d_gamma] at k_verify from the stashed x and s_1
+    {
+      const int rps = gamma + 1, M = B * rps;
+      CK(launch_plan_uniform(B, rps, 0, H->seq_ids, H->seq_len, H->meta, st));
+      Fwd<T> f{H, st, M, max_ctx, true, mode};
+      CK(launch_stash_copy(M, c.d_model, H->x, H->stash_x, rps, gc, 0, 1, st));
+      CK(launch_stash_copy(M, c.d_model, H->s, H->stash_s, rps, gc, 0, 1, st));
+      RET(loops<T>(f, 2, kv_, -1, rps));
+      RET(output_and_head<T>(f, M, nullptr, nullptr, H->vtok));
+      CK(launch_spec_accept(B, gamma, B, H->seq_ids, H->seq_len, H->drafts, H->vtok, H->pending, out_tokens, out_len,
+                            max_new, H->accepted, H->all_done, st));
+      H->last_rows = M;
+    }
+    ++steps;
+    int done = 0;
+    CK(cudaMemcpyAsync(&done, H->all_done, sizeof(int), cudaMemcpyDeviceToHost, st));
+    CK(cudaStreamSynchronize(st));
+    if (done) break;
+    if (steps > (int64_t)max_new + 1) return fail(DORY_ERR_STATE, "speculative loop did not finish");
+  }
+  std::vector<int> lens(c.max_batch);
+  CK(cudaMemcpyAsync(lens.data(), H->seq_len, sizeof(int) * c.max_batch, cudaMemcpyDeviceToHost, st));
+  unsigned long long acc = 0;
+  CK(cudaMemcpyAsync(&acc, H->accepted, sizeof(acc), cudaMemcpyDeviceToHost, st));
+  CK(cudaStreamSynchronize(st));
+  for (int i = 0; i < B; ++i) H->len[seq_ids[i]] = lens[seq_ids[i]];
+  if (stats) {
+    stats->steps = steps;
+    stats->drafted = steps * gamma * B;
+    stats->accepted = (int64_t)acc;
+  }
+  return DORY_OK;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+const char* dory_last_error(void) { return g_last_error.c_str(); }
+
+dory_status dory_workspace_size(const dory_config* cfg, dory_cache_mode alloc_mode, size_t* bytes) {
+  RET(check_config(cfg));
+  if (!bytes) return fail(DORY_ERR_INVALID_ARG, "bytes is NULL");
+  if (alloc_mode != DORY_LAST_LOOP && alloc_mode != DORY_PER_LOOP) return fail(DORY_ERR_INVALID_ARG, "bad alloc mode");
+  dory_handle tmp;
+  tmp.c = *cfg;
+  tmp.alloc_mode = alloc_mode;
+  *bytes = layout(&tmp);
+  return DORY_OK;
+}
+
+dory_status dory_create(const dory_config* cfg, const dory_weights* w, dory_cache_mode alloc_mode, void* workspace,
+                        size_t ws_bytes, dory_handle** out) {
+  RET(check_config(cfg));
+  if (!w || !out || !workspace) return fail(DORY_ERR_INVALID_ARG, "NULL argument");
+  if ((uintptr_t)workspace % 256) return fail(DORY_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  size_t need = 0;
+  RET(dory_workspace_size(cfg, alloc_mode, &need));
+  if (ws_bytes < need) return fail(DORY_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);
+  const int L = cfg->n_in + cfg->n_rec + cfg->n_out;
+  if (!w->embed || !w->lm_head || !w->w_qkv || !w->w_o || !w->w_gu || !w->w_down)
+    return fail(DORY_ERR_INVALID_ARG, "NULL weight pointer");
+  for (int l = 0; l < L; ++l) {
+    bool ok = layer_is_attn(l) ? (w->w_qkv[l] && w->w_o[l]) : (w->w_gu[l] && w->w_down[l]);
+    if (!ok) return fail(DORY_ERR_INVALID_ARG, "layer %d: NULL weight", l);
+  }
+  dory_handle* H = new dory_handle();
+  H->c = *cfg;
+  H->alloc_mode = alloc_mode;
+  H->ws = (char*)workspace;
+  H->ws_bytes = ws_bytes;
+  layout(H);
+  H->embed = w->embed;
+  H->head = w->lm_head;
+  H->w_qkv.assign(w->w_qkv, w->w_qkv + L);
+  H->w_o.assign(w->w_o, w->w_o + L);
+  H->w_gu.assign(w->w_gu, w->w_gu + L);
+  H->w_down.assign(w->w_down, w->w_down + L);
+  H->len.assign(cfg->max_batch, 0);
+  H->mode.assign(cfg->max_batch, -1);
+  H->kfix.assign(cfg->max_batch, 0);
+  *out = H;
+  return DORY_OK;
+}
+
+dory_status dory_destroy(dory_handle* h) {
+  if (!h) return fail(DORY_ERR_INVALID_ARG, "NULL handle");
+  for (auto e : h->ev_pool) cudaEventDestroy(e);
+  delete h;
+  return DORY_OK;
+}
+
+dory_status dory_reset(dory_handle* h, int32_t seq, dory_stream stream) {
+  if (!h) return fail(DORY_ERR_INVALID_ARG, "NULL handle");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (seq == -1) {
+    CK(cudaMemsetAsync(h->seq_len, 0, sizeof(int) * h->c.max_batch, st));
+    CK(cudaMemsetAsync(h->err, 0, sizeof(int) * 4, st));
+    std::fill(h->len.begin(), h->len.end(), 0);
+    std::fill(h->mode.begin(), h->mode.end(), -1);
+    return DORY_OK;
+  }
+  if (seq < 0 || seq >= h->c.max_batch) return fail(DORY_ERR_INVALID_ARG, "seq %d out of range", seq);
+  CK(cudaMemsetAsync(h->seq_len + seq, 0, sizeof(int), st));
+  h->len[seq] = 0;
+  h->mode[seq] = -1;
+  return DORY_OK;
+}
+
+dory_status dory_prefill(dory_handle* h, int32_t batch, const int32_t* seq_ids, const int32_t* tokens,
+                         const int32_t* lens, int32_t k, dory_cache_mode mode, float* last_logits,
+                         int32_t* next_tokens, dory_stream stream) {
+  if (!h) return fail(DORY_ERR_INVALID_ARG, "NULL handle");
+  RET(check_seqs(h, batch, seq_ids, k, mode));
+  if (!tokens || !lens || !next_tokens) return fail(DORY_ERR_INVALID_ARG, "NULL argument");
+  int64_t total = 0;
+  for (int i = 0; i < batch; ++i) {
+    if (lens[i] < 1) return fail(DORY_ERR_INVALID_ARG, "lens[%d] = %d < 1", i, lens[i]);
+    total += lens[i];
+    if ((int64_t)h->len[seq_ids[i]] + lens[i] > h->c.max_seq)
+      return fail(DORY_ERR_CAPACITY, "sequence %d would exceed max_seq", seq_ids[i]);
+  }
+  if (total > h->c.max_chunk) return fail(DORY_ERR_CAPACITY, "%lld tokens > max_chunk %d", (long long)total, h->c.max_chunk);
+  dory_status r = h->bf16 ? prefill_t<bf16>(h, batch, seq_ids, tokens, lens, k, mode, last_logits, next_tokens,
+                                             (cudaStream_t)stream)
+                          : prefill_t<float>(h, batch, seq_ids, tokens, lens, k, mode, last_logits, next_tokens,
+                                             (cudaStream_t)stream);
+  if (r == DORY_OK) mark_started(h, batch, seq_ids, k, mode);
+  return r;
+}
+
+dory_status dory_decode_step(dory_handle* h, int32_t batch, const int32_t* seq_ids, const int32_t* tokens_in,
+                             int32_t k, dory_cache_mode mode, float* logits, int32_t* next_tokens,
+                             dory_stream stream) {
+  if (!h) return fail(DORY_ERR_INVALID_ARG, "NULL handle");
+  RET(check_seqs(h, batch, seq_ids, k, mode));
+  if (!tokens_in || !next_tokens) return fail(DORY_ERR_INVALID_ARG, "NULL argument");
+  for (int i = 0; i < batch; ++i)
+    if (h->len[seq_ids[i]] + 1 > h->c.max_seq)
+      return fail(DORY_ERR_CAPACITY, "sequence %d would exceed max_seq", seq_ids[i]);
+  dory_status r = h->bf16 ? decode_t<bf16>(h, batch, seq_ids, tokens_in, k, mode, logits, next_tokens,
+                                            (cudaStream_t)stream)
+                          : decode_t<float>(h, batch, seq_ids, tokens_in, k, mode, logits, next_tokens,
+                                            (cudaStream_t)stream);
+  if (r == DORY_OK) mark_started(h, batch, seq_ids, k, mode);
+  return r;
+}
+
+dory_status dory_spec_decode(dory_handle* h, int32_t batch, const int32_t* seq_ids, const int32_t* last_tokens,
+                             int32_t k_draft, int32_t k_verify, int32_t gamma, dory_cache_mode mode, int32_t max_new,
+                             int32_t* out_tokens, int32_t* out_len, dory_spec_stats* stats, dory_stream stream) {
+  if (!h) return fail(DORY_ERR_INVALID_ARG, "NULL handle");
+  RET(check_seqs(h, batch, seq_ids, k_verify, mode));
+  if (k_draft != 1) return fail(DORY_ERR_UNSUPPORTED, "k_draft must be 1 (loop-1 reuse)");
+  if (gamma < 1 || gamma > h->c.gamma_max) return fail(DORY_ERR_INVALID_ARG, "gamma %d outside 1..%d", gamma, h->c.gamma_max);
+  if (max_new < 1) return fail(DORY_ERR_INVALID_ARG, "max_new must be >= 1");
+  if (!last_tokens || !out_tokens || !out_len) return fail(DORY_ERR_INVALID_ARG, "NULL argument");
+  if (batch * (gamma + 1) > h->M_max) return fail(DORY_ERR_CAPACITY, "batch*(gamma+1) exceeds chunk capacity");
+  for (int i = 0; i < batch; ++i) {
+    int sq = seq_ids[i];
+    if (h->mode[sq] < 0) return fail(DORY_ERR_STATE, "sequence %d has no prefill", sq);
+    // a sequence that finishes first stays frozen at <= len + max_new + gamma
+    // committed positions while the others continue, and each later step
+    // still writes gamma positions past its length
+    if ((int64_t)h->len[sq] + max_new + 2 * gamma + 1 > h->c.max_seq)
+      return fail(DORY_ERR_CAPACITY, "sequence %d: len + max_new + 2*gamma + 1 exceeds max_seq", sq);
+  }
+  return h->bf16 ? spec_t<bf16>(h, batch, seq_ids, last_tokens, k_verify, gamma, mode, max_new, out_tokens, out_len,
+                                stats, (cudaStream_t)stream)
+                 : spec_t<float>(h, batch, seq_ids, last_tokens, k_verify, gamma, mode, max_new, out_tokens, out_len,
+                                 stats, (cudaStream_t)stream);
+}
+
+dory_status dory_kv_bytes(const dory_handle* h, int32_t k, dory_cache_mode mode, int64_t ctx, int64_t* bytes) {
+  if (!h || !bytes) return fail(DORY_ERR_INVALID_ARG, "NULL argument");
+  if (k < 1 || ctx < 0) return fail(DORY_ERR_INVALID_ARG, "bad k or ctx");
+  int64_t total = 0;
+  for (const AttnLayer& a : h->attn) {
+    int64_t keep = a.full ? ctx : std::min<int64_t>(ctx, h->c.swa_window);
+    int slots = (mode == DORY_PER_LOOP && a.rec) ? k : 1;
+    total += keep * 2 * h->kv_dim * h->esz * slots;
+  }
+  *bytes = total;
+  return DORY_OK;
+}
+
+dory_status dory_seq_len(const dory_handle* h, int32_t seq, int32_t* len) {
+  if (!h || !len) return fail(DORY_ERR_INVALID_ARG, "NULL argument");
+  if (seq < 0 || seq >= h->c.max_batch) return fail(DORY_ERR_INVALID_ARG, "seq out of range");
+  *len = h->len[seq];
+  return DORY_OK;
+}
+
+dory_status dory_read_state(dory_handle* h, int32_t which, float* dst, int32_t rows, dory_stream stream) {
+  if (!h || !dst) return fail(DORY_ERR_INVALID_ARG, "NULL argument");
+  if (rows < 1 || rows > h->last_rows) return fail(DORY_ERR_INVALID_ARG, "rows %d outside 1..%d", rows, h->last_rows);
+  const float* src = which == 0 ? h->x : which == 1 ? h->s : which == 2 ? h->h : nullptr;
+  if (!src) return fail(DORY_ERR_INVALID_ARG, "bad state selector");
+  CK(cudaMemcpyAsync(dst, src, sizeof(float) * rows * h->c.d_model, cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
+  return DORY_OK;
+}
+
+dory_status dory_read_kv(dory_handle* h, int32_t layer, int32_t slot, int32_t seq, int32_t pos0, int32_t n,
+                         void* k_dst, void* v_dst, dory_stream stream) {
+  if (!h || !k_dst || !v_dst) return fail(DORY_ERR_INVALID_ARG, "NULL argument");
+  if (layer < 0 || layer >= h->L || h->attn_of[layer] < 0) return fail(DORY_ERR_INVALID_ARG, "not an attention layer");
+  const AttnLayer& a = h->attn[h->attn_of[layer]];
+  if (slot < 0 || slot >= a.nslots) return fail(DORY_ERR_INVALID_ARG, "slot out of range");
+  if (seq < 0 || seq >= h->c.max_batch || pos0 < 0 || n < 1 || pos0 + n > h->len[seq])
+    return fail(DORY_ERR_INVALID_ARG, "positions outside the sequence");
+  if (!a.full && pos0 < h->len[seq] - a.cap) return fail(DORY_ERR_INVALID_ARG, "positions no longer in the ring");
+  const int hd = h->c.head_dim, KV = h->c.n_kv_heads;
+  const size_t row = (size_t)hd * h->esz;
+  cudaStream_t st = (cudaStream_t)stream;
+  for (int i = 0; i < n; ++i) {
+    int p = pos0 + i;
+    for (int g = 0; g < KV; ++g) {
+      size_t src = (((size_t)seq * KV + g) * a.cap + (p % a.cap)) * row;
+      size_t dst = ((size_t)i * KV + g) * row;
+      CK(cudaMemcpyAsync((char*)k_dst + dst, a.K[slot] + src, row, cudaMemcpyDeviceToDevice, st));
+      CK(cudaMemcpyAsync((char*)v_dst + dst, a.V[slot] + src, row, cudaMemcpyDeviceToDevice, st));
+    }
+  }
+  return DORY_OK;
+}
+
+dory_status dory_synchronize(dory_handle* h, dory_stream stream) {
+  if (!h) return fail(DORY_ERR_INVALID_ARG, "NULL handle");
+  int err[4] = {0, 0, 0, 0};
+  CK(cudaMemcpyAsync(err, h->err, sizeof err, cudaMemcpyDeviceToHost, (cudaStream_t)stream));
+  CK(cudaStreamSynchronize((cudaStream_t)stream));
+  if (err[0] != DEV_ERR_NONE) {
+    CK(cudaMemsetAsync(h->err, 0, sizeof(int) * 4, (cudaStream_t)stream));
+    if (err[0] == DEV_ERR_TIMEOUT) return fail(DORY_ERR_TIMEOUT, "a device-side wait timed out");
+    if (err[0] == DEV_ERR_BAD_TOKEN) return fail(DORY_ERR_INVALID_ARG, "a token id was outside [0, vocab)");
+    if (err[0] == DEV_ERR_BAD_INDEX) return fail(DORY_ERR_CAPACITY, "a cache position was outside max_seq");
+    return fail(DORY_ERR_CUDA, "device error code %d", err[0]);
+  }
+  return DORY_OK;
+}
+
+dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value) {
+  if (!h) return fail(DORY_ERR_INVALID_ARG, "NULL handle");
+  switch (opt) {
+    case DORY_OPT_CUDA_GRAPHS: h->graphs = value != 0; return DORY_OK;
+    case DORY_OPT_PROFILE: h->profile = value != 0; return DORY_OK;
+    case DORY_OPT_GEMM_IMPL:
+      if (value < 0 || value > 2) return fail(DORY_ERR_INVALID_ARG, "bad GEMM impl");
+      h->gemm_impl = (int)value;
+      return DORY_OK;
+  }
+  return fail(DORY_ERR_INVALID_ARG, "unknown option %d", opt);
+}
+
+dory_status dory_profile_reset(dory_handle* h) {
+  if (!h) return fail(DORY_ERR_INVALID_ARG, "NULL handle");
+  h->prof_recs.clear();
+  h->ev_used = 0;
+  return DORY_OK;
+}
+
+dory_status dory_profile_read(dory_handle* h, int32_t n, char (*names)[48], int64_t* launches, double* total_ms,
+                              double* bytes, int32_t* count) {
+  if (!h || !count) return fail(DORY_ERR_INVALID_ARG, "NULL argument");
+  CK(cudaDeviceSynchronize());
+  const size_t K = h->prof_names.size();
+  std::vector<int64_t> cnt(K, 0);
+  std::vector<double> ms(K, 0.0), by(K, 0.0);
+  for (auto& r : h->prof_recs) {
+    float t = 0.f;
+    CK(cudaEventElapsedTime(&t, r.a, r.b));
+    cnt[r.name] += 1;
+    ms[r.name] += t;
+    by[r.name] += r.bytes;
+  }
+  *count = (int32_t)K;
+  for (int i = 0; i < (int)K && i < n; ++i) {
+    if (names) {
+      strncpy(names[i], h->prof_names[i].c_str(), 47);
+      names[i][47] = 0;
+    }
+    if (launches) launches[i] = cnt[i];
+    if (total_ms) total_ms[i] = ms[i];
+    if (bytes) bytes[i] = by[i];
+  }
+  return DORY_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,21 @@
+// bf16 GEMM on the 5th-generation tensor cores (tcgen05 + TMEM, TMA-fed).
+#pragma once
+
+#include "common.cuh"
+
+namespace dory {
+
+// Largest split-K factor the GEMM may choose; callers size partial buffers
+// for kMaxSplitK slices.
+constexpr int kMaxSplitK = 8;
+
+// Y = X . W^T for X [M, K] (row stride ldx) and W [N, K], both bf16, fp32
+// accumulation.  Writes S partial products to Y + s * (*part_stride)
+// (row stride ldy); the consumer adds them in order s = 0..S-1.  The split
+// and the per-element accumulation order depend only on (N, K), never on M.
+// part_rows: rows available per slice (>= M).  Returns cudaErrorNotSupported
+// for shapes the kernel does not handle (the caller falls back).
+cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf16* W, float* Y, int ldy,
+                           size_t part_rows, int* err, int* S, size_t* part_stride, cudaStream_t st);
+
+}  // namespace dory

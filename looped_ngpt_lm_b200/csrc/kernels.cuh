@@ -1,0 +1,113 @@
+// Launchers of the looped nGPT kernels.  Every launcher queues work on
+// `stream` and returns the launch status; none allocates memory.
+#pragma once
+
+#include "common.cuh"
+
+namespace dory {
+
+// Per-row metadata of one forward chunk (device arrays of n_rows entries).
+//   seq  : sequence slot of the row
+//   pos  : absolute position of the row's token
+//   p0   : first position of this sequence's rows in the chunk
+//   base : chunk row index of this sequence's first row
+//   pend : p0 + (rows of this sequence in the chunk)
+struct RowMeta {
+  int* seq;
+  int* pos;
+  int* p0;
+  int* base;
+  int* pend;
+};
+
+// One attention layer's cache for one slot: K, V of shape
+// [max_batch][n_kv][cap][head_dim] in the storage type.  window == 0 means
+// full causal attention, otherwise keys p-window < j <= p.  Position j lives
+// at index j % cap (a ring for sliding-window layers, cap >= max_seq for full).
+struct KVView {
+  void* K;
+  void* V;
+  int cap;
+  int window;
+  int limit;  // max_seq: positions >= limit are rejected (error word set)
+  int* err;   // device error word
+};
+
+// ---- chunk planning (device-side row metadata) ---------------------------
+cudaError_t launch_plan_uniform(int n_seq, int rows_per_seq, int pos_offset, const int* seq_ids,
+                                const int* seq_len, RowMeta m, cudaStream_t st);
+cudaError_t launch_plan_ragged(int n_seq, int n_rows, const int* cu_rows, const int* seq_ids,
+                               const int* seq_len, RowMeta m, cudaStream_t st);
+cudaError_t launch_advance(int n_seq, const int* seq_ids, int* seq_len, int delta, cudaStream_t st);
+// seq_len[seq_ids[b]] += cu[b+1] - cu[b]
+cudaError_t launch_advance_ragged(int n_seq, const int* seq_ids, const int* cu, int* seq_len, cudaStream_t st);
+
+// ---- elementwise / normalisation -----------------------------------------
+template <typename T>
+cudaError_t launch_embed(int M, int d, int vocab, const int* tokens, const T* E, float* h, T* hop,
+                         int* err, cudaStream_t st);
+// h <- N(h + sum_{s<S} y[s]) ; hop <- (T)h.  y[s] = y + s*part_stride, rows of ldy.
+template <typename T>
+cudaError_t launch_addnorm(int M, int d, float* h, const float* y, int S, size_t part_stride, int ldy,
+                           T* hop, cudaStream_t st);
+// Loop boundary.  s_src: 0 -> s = x ; 1 -> s = N(h) ; 2 -> s = s_in.
+// If make_u: out = N(s + x), else out = s.  h <- out, hop <- (T)out.
+// If s_save: s_save <- s.  stash rows: when stash_x/stash_s are given, row r
+// also copies x / s into stash[(r / rps) * stash_cols + r % rps + col0].
+template <typename T>
+cudaError_t launch_reinject(int M, int d, float* h, const float* x, int s_src, const float* s_in,
+                            bool make_u, T* hop, float* stash_s, int rps, int stash_cols, int col0,
+                            cudaStream_t st);
+// Copy rows between the x/s state and the speculative stash (dir 0: state ->
+// stash, 1: stash -> state).
+cudaError_t launch_stash_copy(int M, int d, float* state, float* stash, int rps, int stash_cols, int col0,
+                              int dir, cudaStream_t st);
+
+// Split q/k/v out of the QKV projection (sum of S partials).  q -> fp32 q_out
+// [M, H*hd]; k, v rounded to T -> scratch [M, KV*hd] (direct == false) or
+// straight into the cache at pos % cap (direct == true).
+template <typename T>
+cudaError_t launch_qkv_post(int M, int H, int KV, int hd, const float* qkv, int S, size_t part_stride,
+                            float* q_out, T* kscr, T* vscr, bool direct, KVView kv, RowMeta m,
+                            int max_batch, cudaStream_t st);
+
+// GQA attention over the cache (+ chunk scratch), split over absolute key
+// blocks of ATTN_BK positions, then merged in block order.
+constexpr int ATTN_BK = 256;
+template <typename T>
+cudaError_t launch_attention(int M, int H, int KV, int hd, const float* q, const T* kscr, const T* vscr,
+                             bool inchunk_scratch, KVView kv, RowMeta m, int max_ctx, float* part,
+                             T* out, cudaStream_t st);
+// Copy chunk K/V from scratch into the cache (positions >= pend - cap).
+template <typename T>
+cudaError_t launch_kv_commit(int M, int KV, int hd, const T* kscr, const T* vscr, KVView kv, RowMeta m,
+                             cudaStream_t st);
+
+// act[m, i] = silu(sum_s g) * sum_s u, g = column i, u = column dff + i.
+template <typename T>
+cudaError_t launch_swiglu(int M, int dff, const float* gu, int S, size_t part_stride, T* act,
+                          cudaStream_t st);
+
+template <typename T>
+cudaError_t launch_gather_rows(int R, int d, const int* rows, const T* src, T* dst, cudaStream_t st);
+
+// Y[m, n] = sum_k X[m, k] W[n, k] with fp32 accumulation in increasing k
+// (identical for every M).  X rows of ldx elements, Y rows of ldy floats.
+template <typename T>
+cudaError_t launch_gemm_simt(int M, int N, int K, const T* X, int ldx, const T* W, float* Y, int ldy,
+                             cudaStream_t st);
+
+// Greedy choice per row (largest logit, lowest id on ties).
+cudaError_t launch_argmax(int R, int V, const float* logits, int* out, cudaStream_t st);
+
+// Speculative acceptance for B sequences.  drafts[i * dstride + b] = d_{i+1},
+// vtok [B, gamma+1] verifier choices.  Appends accepted tokens to out
+// [B, max_new] at out_len, sets seq_len = p0 + n + 1 and pending = a_n for
+// unfinished sequences; adds n to *accepted (device int64).
+cudaError_t launch_spec_accept(int B, int gamma, int dstride, const int* seq_ids, int* seq_len,
+                               const int* drafts, const int* vtok, int* pending, int* out, int* out_len,
+                               int max_new, unsigned long long* accepted, int* all_done, cudaStream_t st);
+
+cudaError_t launch_fill_i32(int n, int* p, int v, cudaStream_t st);
+
+}  // namespace dory

@@ -1,0 +1,700 @@
+// CUDA-core kernels of the looped nGPT forward: planning, embedding, the nGPT
+// residual+L2-norm, loop re-injection, QKV split and KV-cache writes, GQA
+// attention over ring/linear caches, SwiGLU, argmax, speculative acceptance,
+// and a reference SIMT GEMM (fp32 storage, or bf16 before the tensor-core
+// path takes over).
+//
+// Every reduction here runs in a fixed order that depends only on the row's
+// own data and absolute positions, never on how many rows share a launch, so
+// a row computes bit-identical results alone or inside a larger chunk.
+#include <float.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace dory {
+
+// ------------------------------------------------------------------ planning
+__global__ void k_plan_uniform(int n_rows, int rps, int pos_offset, const int* seq_ids, const int* seq_len,
+                               RowMeta m) {
+  int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= n_rows) return;
+  int b = r / rps, i = r % rps;
+  int seq = seq_ids[b];
+  int p0 = seq_len[seq] + pos_offset;
+  m.seq[r] = seq;
+  m.pos[r] = p0 + i;
+  m.p0[r] = p0;
+  m.base[r] = b * rps;
+  m.pend[r] = p0 + rps;
+}
+
+cudaError_t launch_plan_uniform(int n_seq, int rps, int pos_offset, const int* seq_ids, const int* seq_len,
+                                RowMeta m, cudaStream_t st) {
+  int n = n_seq * rps;
+  k_plan_uniform<<<(n + 127) / 128, 128, 0, st>>>(n, rps, pos_offset, seq_ids, seq_len, m);
+  return cudaGetLastError();
+}
+
+__global__ void k_plan_ragged(int n_seq, const int* cu, const int* seq_ids, const int* seq_len, RowMeta m) {
+  int b = blockIdx.x;
+  int seq = seq_ids[b];
+  int r0 = cu[b], r1 = cu[b + 1];
+  int p0 = seq_len[seq];
+  for (int r = r0 + threadIdx.x; r < r1; r += blockDim.x) {
+    m.seq[r] = seq;
+    m.pos[r] = p0 + (r - r0);
+    m.p0[r] = p0;
+    m.base[r] = r0;
+    m.pend[r] = p0 + (r1 - r0);
+  }
+}
+
+cudaError_t launch_plan_ragged(int n_seq, int n_rows, const int* cu, const int* seq_ids, const int* seq_len,
+                               RowMeta m, cudaStream_t st) {
+  (void)n_rows;
+  k_plan_ragged<<<n_seq, 128, 0, st>>>(n_seq, cu, seq_ids, seq_len, m);
+  return cudaGetLastError();
+}
+
+__global__ void k_advance(int n_seq, const int* seq_ids, int* seq_len, int delta) {
+  int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < n_seq) seq_len[seq_ids[b]] += delta;
+}
+
+cudaError_t launch_advance(int n_seq, const int* seq_ids, int* seq_len, int delta, cudaStream_t st) {
+  k_advance<<<(n_seq + 127) / 128, 128, 0, st>>>(n_seq, seq_ids, seq_len, delta);
+  return cudaGetLastError();
+}
+
+__global__ void k_advance_ragged(int n_seq, const int* seq_ids, const int* cu, int* seq_len) {
+  int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < n_seq) seq_len[seq_ids[b]] += cu[b + 1] - cu[b];
+}
+
+cudaError_t launch_advance_ragged(int n_seq, const int* seq_ids, const int* cu, int* seq_len, cudaStream_t st) {
+  k_advance_ragged<<<(n_seq + 127) / 128, 128, 0, st>>>(n_seq, seq_ids, cu, seq_len);
+  return cudaGetLastError();
+}
+
+__global__ void k_fill_i32(int n, int* p, int v) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) p[i] = v;
+}
+
+cudaError_t launch_fill_i32(int n, int* p, int v, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  k_fill_i32<<<(n + 255) / 256, 256, 0, st>>>(n, p, v);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ embedding
+template <typename T>
+__global__ void k_embed(int d, int vocab, const int* tokens, const T* E, float* h, T* hop, int* err) {
+  int r = blockIdx.x;
+  int tok = tokens[r];
+  if (tok < 0 || tok >= vocab) {
+    if (threadIdx.x == 0) set_error(err, DEV_ERR_BAD_TOKEN);
+    tok = 0;
+  }
+  const T* src = E + (size_t)tok * d;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    T v = src[i];
+    h[(size_t)r * d + i] = to_f(v);
+    hop[(size_t)r * d + i] = v;
+  }
+}
+
+template <typename T>
+cudaError_t launch_embed(int M, int d, int vocab, const int* tokens, const T* E, float* h, T* hop, int* err,
+                         cudaStream_t st) {
+  k_embed<T><<<M, 256, 0, st>>>(d, vocab, tokens, E, h, hop, err);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ add + norm
+// One 256-thread block per row; thread t owns elements t, t+256, ...
+template <typename T>
+__global__ void k_addnorm(int d, float* h, const float* y, int S, size_t ps, int ldy, T* hop) {
+  __shared__ float red[33];
+  const int r = blockIdx.x;
+  float* hr = h + (size_t)r * d;
+  float v[16];  // d <= 16 * 256
+  float ss = 0.f;
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    int i = threadIdx.x + c * 256;
+    v[c] = 0.f;
+    if (i < d) {
+      float acc = 0.f;
+      for (int s = 0; s < S; ++s) acc += y[s * ps + (size_t)r * ldy + i];
+      v[c] = hr[i] + acc;
+      ss += v[c] * v[c];
+    }
+  }
+  ss = block_sum(ss, red);
+  const float inv = 1.f / fmaxf(sqrtf(ss), 1e-12f);
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    int i = threadIdx.x + c * 256;
+    if (i < d) {
+      float o = v[c] * inv;
+      hr[i] = o;
+      hop[(size_t)r * d + i] = from_f<T>(o);
+    }
+  }
+}
+
+template <typename T>
+cudaError_t launch_addnorm(int M, int d, float* h, const float* y, int S, size_t ps, int ldy, T* hop,
+                           cudaStream_t st) {
+  if (d > 16 * 256) return cudaErrorInvalidValue;
+  k_addnorm<T><<<M, 256, 0, st>>>(d, h, y, S, ps, ldy, hop);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ loop boundary
+template <typename T>
+__global__ void k_reinject(int d, float* h, const float* x, int s_src, const float* s_in, bool make_u, T* hop,
+                           float* stash_s, int rps, int scols, int col0) {
+  __shared__ float red[33];
+  const int r = blockIdx.x;
+  float* hr = h + (size_t)r * d;
+  const float* xr = x + (size_t)r * d;
+  float sv[16];
+  float ss = 0.f;
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    int i = threadIdx.x + c * 256;
+    sv[c] = 0.f;
+    if (i < d) {
+      sv[c] = s_src == 0 ? xr[i] : (s_src == 1 ? hr[i] : s_in[(size_t)r * d + i]);
+      ss += sv[c] * sv[c];
+    }
+  }
+  if (s_src == 1) {  // s = N(h)
+    ss = block_sum(ss, red);
+    const float inv = 1.f / fmaxf(sqrtf(ss), 1e-12f);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) sv[c] *= inv;
+  }
+  if (stash_s) {
+    size_t srow = (size_t)((r / rps) * scols + r % rps + col0) * d;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      int i = threadIdx.x + c * 256;
+      if (i < d) stash_s[srow + i] = sv[c];
+    }
+  }
+  if (make_u) {  // u = N(s + x)
+    float uu = 0.f;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      int i = threadIdx.x + c * 256;
+      if (i < d) {
+        sv[c] += xr[i];
+        uu += sv[c] * sv[c];
+      }
+    }
+    uu = block_sum(uu, red);
+    const float inv = 1.f / fmaxf(sqrtf(uu), 1e-12f);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) sv[c] *= inv;
+  }
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    int i = threadIdx.x + c * 256;
+    if (i < d) {
+      hr[i] = sv[c];
+      hop[(size_t)r * d + i] = from_f<T>(sv[c]);
+    }
+  }
+}
+
+template <typename T>
+cudaError_t launch_reinject(int M, int d, float* h, const float* x, int s_src, const float* s_in, bool make_u,
+                            T* hop, float* stash_s, int rps, int scols, int col0, cudaStream_t st) {
+  if (d > 16 * 256) return cudaErrorInvalidValue;
+  k_reinject<T><<<M, 256, 0, st>>>(d, h, x, s_src, s_in, make_u, hop, stash_s, rps, scols, col0);
+  return cudaGetLastError();
+}
+
+__global__ void k_stash_copy(int d, float* state, float* stash, int rps, int scols, int col0, int dir) {
+  const int r = blockIdx.x;
+  size_t srow = (size_t)((r / rps) * scols + r % rps + col0) * d;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    if (dir == 0)
+      stash[srow + i] = state[(size_t)r * d + i];
+    else
+      state[(size_t)r * d + i] = stash[srow + i];
+  }
+}
+
+cudaError_t launch_stash_copy(int M, int d, float* state, float* stash, int rps, int scols, int col0, int dir,
+                              cudaStream_t st) {
+  k_stash_copy<<<M, 256, 0, st>>>(d, state, stash, rps, scols, col0, dir);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ QKV split
+template <typename T>
+__global__ void k_qkv_post(int H, int KV, int hd, const float* qkv, int S, size_t ps, float* q_out, T* kscr,
+                           T* vscr, bool direct, KVView kv, RowMeta m, int max_batch) {
+  const int r = blockIdx.x;
+  const int qd = H * hd, kvd = KV * hd, ld = qd + 2 * kvd;
+  const float* src = qkv + (size_t)r * ld;
+  const int seq = m.seq[r], pos = m.pos[r];
+  if (pos < 0 || pos >= kv.limit) {
+    if (threadIdx.x == 0) set_error(kv.err, DEV_ERR_BAD_INDEX);
+    return;
+  }
+  const size_t ring = (size_t)(pos % kv.cap);
+  for (int i = threadIdx.x; i < ld; i += blockDim.x) {
+    float a = 0.f;
+    for (int s = 0; s < S; ++s) a += src[s * ps + i];
+    if (i < qd) {
+      q_out[(size_t)r * qd + i] = a;
+    } else {
+      int j = i - qd;
+      bool is_v = j >= kvd;
+      if (is_v) j -= kvd;
+      T val = from_f<T>(a);
+      if (direct) {
+        int g = j / hd, e = j % hd;
+        size_t off = (((size_t)seq * KV + g) * kv.cap + ring) * hd + e;
+        (is_v ? (T*)kv.V : (T*)kv.K)[off] = val;
+      } else {
+        (is_v ? vscr : kscr)[(size_t)r * kvd + j] = val;
+      }
+    }
+  }
+  (void)max_batch;
+}
+
+template <typename T>
+cudaError_t launch_qkv_post(int M, int H, int KV, int hd, const float* qkv, int S, size_t ps, float* q_out,
+                            T* kscr, T* vscr, bool direct, KVView kv, RowMeta m, int max_batch, cudaStream_t st) {
+  k_qkv_post<T><<<M, 256, 0, st>>>(H, KV, hd, qkv, S, ps, q_out, kscr, vscr, direct, kv, m, max_batch);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ attention
+// Block (row r, kv head g, key block b): 4 warps; each warp is 4 groups of 8
+// lanes; group s of warp w takes keys kb + 4w + s + 16i; each lane of a group
+// holds hd/8 dimensions.  Per group: online softmax (base-2) over its keys for
+// the G query heads that share kv head g; groups are merged by a fixed xor
+// tree, warps in index order.  Partial result: m, l, acc[hd] per head.
+template <typename T, int HD, int G>
+__global__ void __launch_bounds__(128) k_attn_partial(int KV, const float* __restrict__ q, const T* kscr,
+                                                      const T* vscr, bool inchunk_scratch, KVView kv, RowMeta m,
+                                                      float* __restrict__ part, int nb_max, float scale_log2) {
+  constexpr int DL = HD / 8;  // dims per lane
+  __shared__ float sm_m[4][G], sm_l[4][G];
+  __shared__ float sm_acc[4][G][HD];
+  const int r = blockIdx.x / KV, g = blockIdx.x % KV;
+  const int pos = m.pos[r], seq = m.seq[r], p0 = m.p0[r], base = m.base[r];
+  if (pos < 0 || pos >= kv.limit) {
+    if (threadIdx.x == 0 && blockIdx.y == 0) set_error(kv.err, DEV_ERR_BAD_INDEX);
+    return;
+  }
+  const int lo = kv.window > 0 ? max(0, pos - kv.window + 1) : 0;
+  const int nb_row = pos / ATTN_BK - lo / ATTN_BK + 1;
+  if (nb_row > nb_max) {
+    if (threadIdx.x == 0 && blockIdx.y == 0) set_error(kv.err, DEV_ERR_BAD_INDEX);
+    return;
+  }
+  if ((int)blockIdx.y >= nb_row) return;
+  const int ab = lo / ATTN_BK + blockIdx.y;
+  const int klo = max(lo, ab * ATTN_BK), khi = min(pos, ab * ATTN_BK + ATTN_BK - 1);
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, sg = lane >> 3, dl = lane & 7;
+  const int H = KV * G;
+  const int qd = H * HD, kvd = KV * HD;
+
+  float qv[G][DL];
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int e = 0; e < DL; ++e) qv[h][e] = q[(size_t)r * qd + (g * G + h) * HD + dl * DL + e] * scale_log2;
+
+  float mx[G], ls[G], acc[G][DL];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    mx[h] = -FLT_MAX;
+    ls[h] = 0.f;
+#pragma unroll
+    for (int e = 0; e < DL; ++e) acc[h][e] = 0.f;
+  }
+  const T* Kc = (const T*)kv.K + ((size_t)seq * KV + g) * kv.cap * HD;
+  const T* Vc = (const T*)kv.V + ((size_t)seq * KV + g) * kv.cap * HD;
+  const int kb = ab * ATTN_BK;
+  for (int jq = kb + 4 * w; jq <= khi; jq += 16) {
+    const int j = jq + sg;
+    const bool valid = j >= klo && j <= khi;
+    float kf[DL], vf[DL];
+    if (valid) {
+      const T *kp, *vp;
+      if (inchunk_scratch && j >= p0) {
+        size_t row = (size_t)(base + (j - p0));
+        kp = kscr + row * kvd + g * HD;
+        vp = vscr + row * kvd + g * HD;
+      } else {
+        size_t idx = (size_t)(j % kv.cap) * HD;
+        kp = Kc + idx;
+        vp = Vc + idx;
+      }
+#pragma unroll
+      for (int e = 0; e < DL; ++e) {
+        kf[e] = to_f(kp[dl * DL + e]);
+        vf[e] = to_f(vp[dl * DL + e]);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < DL; ++e) kf[e] = vf[e] = 0.f;
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float sdot = 0.f;
+#pragma unroll
+      for (int e = 0; e < DL; ++e) sdot += qv[h][e] * kf[e];
+      sdot += __shfl_xor_sync(0xffffffffu, sdot, 1);
+      sdot += __shfl_xor_sync(0xffffffffu, sdot, 2);
+      sdot += __shfl_xor_sync(0xffffffffu, sdot, 4);
+      if (valid) {
+        float mn = fmaxf(mx[h], sdot);
+        float corr = exp2f(mx[h] - mn);
+        float p = exp2f(sdot - mn);
+        ls[h] = ls[h] * corr + p;
+#pragma unroll
+        for (int e = 0; e < DL; ++e) acc[h][e] = acc[h][e] * corr + p * vf[e];
+        mx[h] = mn;
+      }
+    }
+  }
+  // merge the 4 groups of the warp (xor 8, then 16)
+#pragma unroll
+  for (int off = 8; off <= 16; off <<= 1) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float om = __shfl_xor_sync(0xffffffffu, mx[h], off);
+      float ol = __shfl_xor_sync(0xffffffffu, ls[h], off);
+      float mn = fmaxf(mx[h], om);
+      float ca = (mx[h] == -FLT_MAX) ? 0.f : exp2f(mx[h] - mn);
+      float cb = (om == -FLT_MAX) ? 0.f : exp2f(om - mn);
+      ls[h] = ls[h] * ca + ol * cb;
+#pragma unroll
+      for (int e = 0; e < DL; ++e) {
+        float oa = __shfl_xor_sync(0xffffffffu, acc[h][e], off);
+        acc[h][e] = acc[h][e] * ca + oa * cb;
+      }
+      mx[h] = mn;
+    }
+  }
+  if (sg == 0) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      if (dl == 0) {
+        sm_m[w][h] = mx[h];
+        sm_l[w][h] = ls[h];
+      }
+#pragma unroll
+      for (int e = 0; e < DL; ++e) sm_acc[w][h][dl * DL + e] = acc[h][e];
+    }
+  }
+  __syncthreads();
+  // merge warps 0..3 in order; thread t handles (head, dim) pairs
+  for (int idx = threadIdx.x; idx < G * (HD + 2); idx += blockDim.x) {
+    const int h = idx / (HD + 2), c = idx % (HD + 2);
+    float M = -FLT_MAX;
+#pragma unroll
+    for (int ww = 0; ww < 4; ++ww) M = fmaxf(M, sm_m[ww][h]);
+    float val = 0.f;
+    if (c == 0) {
+      val = M;
+    } else {
+#pragma unroll
+      for (int ww = 0; ww < 4; ++ww) {
+        float sc = sm_m[ww][h] == -FLT_MAX ? 0.f : exp2f(sm_m[ww][h] - M);
+        val += (c == 1 ? sm_l[ww][h] : sm_acc[ww][h][c - 2]) * sc;
+      }
+    }
+    const int head = g * G + h;
+    part[(((size_t)r * H + head) * nb_max + blockIdx.y) * (HD + 2) + c] = val;
+  }
+}
+
+// One warp per (row, head): merge the row's key blocks in order.
+template <typename T, int HD>
+__global__ void k_attn_combine(int H, const float* __restrict__ part, int nb_max, KVView kv, RowMeta m, T* out) {
+  const int r = blockIdx.x, head = blockIdx.y * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (head >= H) return;
+  const int lane = threadIdx.x & 31;
+  const int pos = m.pos[r];
+  const int lo = kv.window > 0 ? max(0, pos - kv.window + 1) : 0;
+  const int nb = pos / ATTN_BK - lo / ATTN_BK + 1;
+  constexpr int DPL0 = HD / 32;
+  if (pos < 0 || pos >= kv.limit || nb > nb_max) {  // rejected by the partial kernel
+#pragma unroll
+    for (int e = 0; e < DPL0; ++e) out[(size_t)r * H * HD + head * HD + lane * DPL0 + e] = from_f<T>(0.f);
+    return;
+  }
+  const float* pr = part + ((size_t)r * H + head) * nb_max * (HD + 2);
+  float M = -FLT_MAX;
+  for (int b = 0; b < nb; ++b) M = fmaxf(M, pr[b * (HD + 2)]);
+  constexpr int DPL = HD / 32;
+  float L = 0.f, acc[DPL];
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+  for (int b = 0; b < nb; ++b) {
+    const float* pb = pr + b * (HD + 2);
+    float sc = exp2f(pb[0] - M);
+    L += pb[1] * sc;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) acc[e] += pb[2 + lane * DPL + e] * sc;
+  }
+  const float inv = 1.f / L;
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) out[(size_t)r * H * HD + head * HD + lane * DPL + e] = from_f<T>(acc[e] * inv);
+}
+
+template <typename T, int HD, int G>
+static cudaError_t attn_dispatch(int M, int KV, const float* q, const T* kscr, const T* vscr, bool sc, KVView kv,
+                                 RowMeta m, int nb, float* part, T* out, cudaStream_t st) {
+  const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
+  dim3 grid(M * KV, nb);
+  k_attn_partial<T, HD, G><<<grid, 128, 0, st>>>(KV, q, kscr, vscr, sc, kv, m, part, nb, scale_log2);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int H = KV * G;
+  dim3 g2(M, (H + 3) / 4);
+  k_attn_combine<T, HD><<<g2, 128, 0, st>>>(H, part, nb, kv, m, out);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_attention(int M, int H, int KV, int hd, const float* q, const T* kscr, const T* vscr,
+                             bool sc, KVView kv, RowMeta m, int max_ctx, float* part, T* out, cudaStream_t st) {
+  int span = kv.window > 0 ? min(max_ctx, kv.window) : max_ctx;
+  int nb = (span + ATTN_BK - 1) / ATTN_BK + 1;
+  const int G = H / KV;
+#define DORY_ATTN_CASE(HDV, GV) \
+  if (hd == HDV && G == GV) return attn_dispatch<T, HDV, GV>(M, KV, q, kscr, vscr, sc, kv, m, nb, part, out, st);
+  DORY_ATTN_CASE(32, 1) DORY_ATTN_CASE(32, 2) DORY_ATTN_CASE(32, 4) DORY_ATTN_CASE(32, 5) DORY_ATTN_CASE(32, 8)
+  DORY_ATTN_CASE(64, 1) DORY_ATTN_CASE(64, 2) DORY_ATTN_CASE(64, 4) DORY_ATTN_CASE(64, 5) DORY_ATTN_CASE(64, 8)
+  DORY_ATTN_CASE(128, 1) DORY_ATTN_CASE(128, 2) DORY_ATTN_CASE(128, 4) DORY_ATTN_CASE(128, 5)
+#undef DORY_ATTN_CASE
+  return cudaErrorInvalidValue;
+}
+
+template <typename T>
+__global__ void k_kv_commit(int KV, int hd, const T* kscr, const T* vscr, KVView kv, RowMeta m) {
+  const int r = blockIdx.x;
+  const int pos = m.pos[r], pend = m.pend[r], seq = m.seq[r];
+  if (pos < pend - kv.cap) return;  // overwritten later in this chunk
+  if (pos < 0 || pos >= kv.limit) {
+    if (threadIdx.x == 0) set_error(kv.err, DEV_ERR_BAD_INDEX);
+    return;
+  }
+  const int kvd = KV * hd;
+  const size_t ring = (size_t)(pos % kv.cap);
+  for (int j = threadIdx.x; j < kvd; j += blockDim.x) {
+    int g = j / hd, e = j % hd;
+    size_t off = (((size_t)seq * KV + g) * kv.cap + ring) * hd + e;
+    ((T*)kv.K)[off] = kscr[(size_t)r * kvd + j];
+    ((T*)kv.V)[off] = vscr[(size_t)r * kvd + j];
+  }
+}
+
+template <typename T>
+cudaError_t launch_kv_commit(int M, int KV, int hd, const T* kscr, const T* vscr, KVView kv, RowMeta m,
+                             cudaStream_t st) {
+  k_kv_commit<T><<<M, 128, 0, st>>>(KV, hd, kscr, vscr, kv, m);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ SwiGLU
+template <typename T>
+__global__ void k_swiglu(int dff, const float* gu, int S, size_t ps, T* act) {
+  const int r = blockIdx.y;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= dff) return;
+  const float* row = gu + (size_t)r * 2 * dff;
+  float g = 0.f, u = 0.f;
+  for (int s = 0; s < S; ++s) {
+    g += row[s * ps + i];
+    u += row[s * ps + dff + i];
+  }
+  float a = g / (1.f + expf(-g)) * u;
+  act[(size_t)r * dff + i] = from_f<T>(a);
+}
+
+template <typename T>
+cudaError_t launch_swiglu(int M, int dff, const float* gu, int S, size_t ps, T* act, cudaStream_t st) {
+  dim3 grid((dff + 255) / 256, M);
+  k_swiglu<T><<<grid, 256, 0, st>>>(dff, gu, S, ps, act);
+  return cudaGetLastError();
+}
+
+template <typename T>
+__global__ void k_gather_rows(int d, const int* rows, const T* src, T* dst) {
+  const int r = blockIdx.x;
+  const T* s = src + (size_t)rows[r] * d;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) dst[(size_t)r * d + i] = s[i];
+}
+
+template <typename T>
+cudaError_t launch_gather_rows(int R, int d, const int* rows, const T* src, T* dst, cudaStream_t st) {
+  k_gather_rows<T><<<R, 256, 0, st>>>(d, rows, src, dst);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ SIMT GEMM
+// 64 (m) x 64 (n) tile per 256-thread block, k tile 16; each thread 4x4
+// outputs accumulated in increasing k.
+template <typename T>
+__global__ void __launch_bounds__(256) k_gemm_simt(int M, int N, int K, const T* __restrict__ X, int ldx,
+                                                   const T* __restrict__ W, float* __restrict__ Y, int ldy) {
+  __shared__ float xs[16][64 + 4];
+  __shared__ float ws[16][64 + 4];
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    for (int i = threadIdx.x; i < 64 * 16; i += 256) {
+      int rr = i / 16, kk = i % 16;
+      int gm = m0 + rr, gn = n0 + rr, gk = k0 + kk;
+      xs[kk][rr] = (gm < M && gk < K) ? to_f(X[(size_t)gm * ldx + gk]) : 0.f;
+      ws[kk][rr] = (gn < N && gk < K) ? to_f(W[(size_t)gn * K + gk]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = xs[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = ws[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    int gm = m0 + ty * 4 + i;
+    if (gm >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      int gn = n0 + tx * 4 + j;
+      if (gn < N) Y[(size_t)gm * ldy + gn] = acc[i][j];
+    }
+  }
+}
+
+template <typename T>
+cudaError_t launch_gemm_simt(int M, int N, int K, const T* X, int ldx, const T* W, float* Y, int ldy,
+                             cudaStream_t st) {
+  dim3 grid((N + 63) / 64, (M + 63) / 64);
+  k_gemm_simt<T><<<grid, 256, 0, st>>>(M, N, K, X, ldx, W, Y, ldy);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ argmax
+// One block per row; per-thread running (max, lowest index), then a fixed
+// tree.  max with lowest-index ties is order independent.
+__global__ void k_argmax(int V, const float* logits, int* out) {
+  __shared__ float sv[32];
+  __shared__ int si[32];
+  const float* row = logits + (size_t)blockIdx.x * V;
+  float best = -FLT_MAX;
+  int bi = 0x7fffffff;
+  for (int i = threadIdx.x; i < V; i += blockDim.x) {
+    float v = row[i];
+    if (v > best) {
+      best = v;
+      bi = i;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    float ov = __shfl_xor_sync(0xffffffffu, best, o);
+    int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (ov > best || (ov == best && oi < bi)) {
+      best = ov;
+      bi = oi;
+    }
+  }
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    sv[w] = best;
+    si[w] = bi;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int i = 1; i < (int)(blockDim.x >> 5); ++i)
+      if (sv[i] > best || (sv[i] == best && si[i] < bi)) {
+        best = sv[i];
+        bi = si[i];
+      }
+    out[blockIdx.x] = bi;
+  }
+}
+
+cudaError_t launch_argmax(int R, int V, const float* logits, int* out, cudaStream_t st) {
+  k_argmax<<<R, 1024, 0, st>>>(V, logits, out);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ speculative acceptance
+__global__ void k_spec_accept(int B, int gamma, int dstride, const int* seq_ids, int* seq_len, const int* drafts,
+                              const int* vtok, int* pending, int* out, int* out_len, int max_new,
+                              unsigned long long* accepted, int* all_done) {
+  __shared__ int n_unfinished;
+  if (threadIdx.x == 0) n_unfinished = 0;
+  __syncthreads();
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    int ol = out_len[b];
+    if (ol >= max_new) continue;  // finished: cache and length stay frozen
+    const int* a = vtok + b * (gamma + 1);
+    int n = 0;
+    while (n < gamma && a[n] == drafts[n * dstride + b]) ++n;
+    for (int i = 0; i < n && ol < max_new; ++i) out[b * max_new + ol++] = drafts[i * dstride + b];
+    if (ol < max_new) out[b * max_new + ol++] = a[n];
+    out_len[b] = ol;
+    seq_len[seq_ids[b]] += n + 1;
+    pending[b] = a[n];
+    atomicAdd(accepted, (unsigned long long)n);
+    if (ol < max_new) atomicAdd(&n_unfinished, 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) *all_done = (n_unfinished == 0);
+}
+
+cudaError_t launch_spec_accept(int B, int gamma, int dstride, const int* seq_ids, int* seq_len, const int* drafts,
+                               const int* vtok, int* pending, int* out, int* out_len, int max_new,
+                               unsigned long long* accepted, int* all_done, cudaStream_t st) {
+  k_spec_accept<<<1, 256, 0, st>>>(B, gamma, dstride, seq_ids, seq_len, drafts, vtok, pending, out, out_len, max_new,
+                                   accepted, all_done);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ instantiations
+#define DORY_INST(T)                                                                                              \
+  template cudaError_t launch_embed<T>(int, int, int, const int*, const T*, float*, T*, int*, cudaStream_t);      \
+  template cudaError_t launch_addnorm<T>(int, int, float*, const float*, int, size_t, int, T*, cudaStream_t);     \
+  template cudaError_t launch_reinject<T>(int, int, float*, const float*, int, const float*, bool, T*, float*,    \
+                                          int, int, int, cudaStream_t);                                           \
+  template cudaError_t launch_qkv_post<T>(int, int, int, int, const float*, int, size_t, float*, T*, T*, bool,    \
+                                          KVView, RowMeta, int, cudaStream_t);                                    \
+  template cudaError_t launch_attention<T>(int, int, int, int, const float*, const T*, const T*, bool, KVView,    \
+                                           RowMeta, int, float*, T*, cudaStream_t);                               \
+  template cudaError_t launch_kv_commit<T>(int, int, int, const T*, const T*, KVView, RowMeta, cudaStream_t);     \
+  template cudaError_t launch_swiglu<T>(int, int, const float*, int, size_t, T*, cudaStream_t);                   \
+  template cudaError_t launch_gather_rows<T>(int, int, const int*, const T*, T*, cudaStream_t);                   \
+  template cudaError_t launch_gemm_simt<T>(int, int, int, const T*, int, const T*, float*, int, cudaStream_t);
+DORY_INST(float)
+DORY_INST(bf16)
+#undef DORY_INST
+
+}  // namespace dory

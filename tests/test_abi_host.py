@@ -1,0 +1,135 @@
+"""C-ABI checks that need no GPU: exported symbols, workspace sizing, KV byte
+accounting against the oracle, and argument validation (which runs before
+any device work, so a fake workspace address is enough)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle as O
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+dory = pytest.importorskip("looped_ngpt_lm_b200")
+lib = dory.lib
+FAKE_WS = 1 << 40  # never dereferenced: validation fails before any launch
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "dory.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dory_[a-z_]+)\s*\(", src)))
+
+
+def test_every_declared_function_is_exported():
+    names = header_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(dory.SYMBOLS) == names
+
+
+def cfg_for(shape, **kw):
+    args = dict(max_batch=2, max_seq=128, k_max=4, gamma_max=4, max_chunk=96)
+    args.update(kw)
+    return dory.make_config(shape, **args)
+
+
+def fake_handle(shape, alloc=dory.PER_LOOP, **kw):
+    cfg = cfg_for(shape, **kw)
+    n = dory.workspace_size(cfg, alloc)
+    L = shape.n_layers
+    arr = ctypes.c_void_p * L
+    fake = arr(*([FAKE_WS] * L))
+    w = dory.Weights(FAKE_WS, FAKE_WS, fake, fake, fake, fake)
+    h = ctypes.c_void_p()
+    st = lib.dory_create(ctypes.byref(cfg), ctypes.byref(w), alloc, ctypes.c_void_p(FAKE_WS), n, ctypes.byref(h))
+    assert st == 0, lib.dory_last_error()
+    return h, cfg, (cfg, w, fake)
+
+
+def test_workspace_grows_with_per_loop_slots():
+    a = dory.workspace_size(cfg_for(synth.TINY), dory.LAST_LOOP)
+    b = dory.workspace_size(cfg_for(synth.TINY), dory.PER_LOOP)
+    c = dory.workspace_size(cfg_for(synth.TINY, k_max=2), dory.PER_LOOP)
+    assert 0 < a < c < b
+
+
+def test_4b_workspace_is_kv_dominated_and_fits():
+    cfg = cfg_for(synth.DORY_4B, max_batch=1, max_seq=2560 + 300 + 16, max_chunk=2560)
+    n = dory.workspace_size(cfg, dory.LAST_LOOP)
+    assert n < 16e9
+
+
+@pytest.mark.parametrize("shape", [synth.TINY, synth.DORY_4B])
+def test_kv_bytes_match_oracle(shape):
+    h, cfg, keep = fake_handle(shape, max_seq=8192, max_chunk=64)
+    m = O.Model(shape, {})
+    esz = 2 if shape.dtype == "bf16" else 4
+    for mode, cmode in ((O.LAST_LOOP, dory.LAST_LOOP), (O.PER_LOOP, dory.PER_LOOP)):
+        for k in (1, 2, 4):
+            for ctx in (1, 15, 16, 17, 100, 5000):
+                n = ctypes.c_int64()
+                assert lib.dory_kv_bytes(h, k, cmode, ctx, ctypes.byref(n)) == 0
+                assert n.value == O.kv_bytes(m, k, mode, ctx, esz), (mode, k, ctx)
+    lib.dory_destroy(h)
+
+
+def status_name(s):
+    return dory.STATUS[s]
+
+
+def test_argument_validation():
+    h, cfg, keep = fake_handle(synth.TINY, alloc=dory.LAST_LOOP)
+    ids = (ctypes.c_int32 * 2)(0, 1)
+    lens = (ctypes.c_int32 * 2)(4, 4)
+    tok = ctypes.c_void_p(FAKE_WS)
+    nt = ctypes.c_void_p(FAKE_WS)
+    P = lambda *a: status_name(lib.dory_prefill(h, *a))
+    assert P(2, ids, tok, lens, 0, 0, None, nt, None) == "DORY_ERR_INVALID_ARG"       # k = 0
+    assert P(2, ids, tok, lens, 5, 0, None, nt, None) == "DORY_ERR_INVALID_ARG"       # k > k_max
+    assert P(2, ids, tok, lens, 2, 1, None, nt, None) == "DORY_ERR_STATE"             # per_loop on last_loop handle
+    assert P(3, ids, tok, lens, 2, 0, None, nt, None) == "DORY_ERR_INVALID_ARG"       # batch > max_batch
+    dup = (ctypes.c_int32 * 2)(1, 1)
+    assert P(2, dup, tok, lens, 2, 0, None, nt, None) == "DORY_ERR_INVALID_ARG"       # repeated id
+    bad = (ctypes.c_int32 * 2)(0, 7)
+    assert P(2, bad, tok, lens, 2, 0, None, nt, None) == "DORY_ERR_INVALID_ARG"       # id out of range
+    big = (ctypes.c_int32 * 2)(60, 60)
+    assert P(2, ids, tok, big, 2, 0, None, nt, None) == "DORY_ERR_CAPACITY"           # > max_chunk
+    zero = (ctypes.c_int32 * 2)(0, 3)
+    assert P(2, ids, tok, zero, 2, 0, None, nt, None) == "DORY_ERR_INVALID_ARG"       # empty sequence
+    over = (ctypes.c_int32 * 1)(129)
+    assert P(1, ids, tok, over, 2, 0, None, nt, None) == "DORY_ERR_CAPACITY"          # > max_seq
+    S = lambda *a: status_name(lib.dory_spec_decode(h, *a))
+    out = ctypes.c_void_p(FAKE_WS)
+    assert S(1, ids, tok, 2, 4, 4, 0, 8, out, out, None, None) == "DORY_ERR_UNSUPPORTED"  # k_draft != 1
+    assert S(1, ids, tok, 1, 4, 5, 0, 8, out, out, None, None) == "DORY_ERR_INVALID_ARG"  # gamma > gamma_max
+    assert S(1, ids, tok, 1, 4, 4, 0, 8, out, out, None, None) == "DORY_ERR_STATE"        # no prefill yet
+    D = lambda *a: status_name(lib.dory_decode_step(h, *a))
+    assert D(1, ids, tok, 9, 0, None, nt, None) == "DORY_ERR_INVALID_ARG"
+    assert D(1, ids, None, 2, 0, None, nt, None) == "DORY_ERR_INVALID_ARG"
+    assert lib.dory_set_option(h, 99, 1) == 1
+    n = ctypes.c_int32()
+    assert lib.dory_seq_len(h, 0, ctypes.byref(n)) == 0 and n.value == 0
+    assert lib.dory_read_state(h, 0, ctypes.c_void_p(FAKE_WS), 1, None) == 1  # nothing computed yet
+    assert b"rows" in lib.dory_last_error()
+    lib.dory_destroy(h)
+
+
+def test_create_rejects_bad_workspace_and_config():
+    cfg = cfg_for(synth.TINY)
+    n = dory.workspace_size(cfg, dory.LAST_LOOP)
+    L = synth.TINY.n_layers
+    fake = (ctypes.c_void_p * L)(*([FAKE_WS] * L))
+    w = dory.Weights(FAKE_WS, FAKE_WS, fake, fake, fake, fake)
+    h = ctypes.c_void_p()
+    assert lib.dory_create(ctypes.byref(cfg), ctypes.byref(w), 0, ctypes.c_void_p(FAKE_WS), n - 1,
+                           ctypes.byref(h)) == 4
+    assert lib.dory_create(ctypes.byref(cfg), ctypes.byref(w), 0, ctypes.c_void_p(FAKE_WS + 8), n,
+                           ctypes.byref(h)) == 4
+    bad = dory.make_config(synth.TINY.with_(head_dim=48))
+    assert lib.dory_workspace_size(ctypes.byref(bad), 0, ctypes.byref(ctypes.c_size_t())) == 7
+    bad = dory.make_config(synth.TINY.with_(n_kv_heads=3))
+    assert lib.dory_workspace_size(ctypes.byref(bad), 0, ctypes.byref(ctypes.c_size_t())) == 1

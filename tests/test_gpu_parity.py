@@ -1,0 +1,204 @@
+"""CUDA path against the oracle on the tiny configurations (GPU).
+
+Tolerances: the tiny fp32 model must match the oracle within 1e-4 (max abs
+logit error); bf16 models must keep final-state cosine >= 0.999, logits
+relative L2 error <= 2e-2 and greedy tokens identical (near ties excepted,
+see gpu_util.check_tokens) over the decode steps.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA GPU", allow_module_level=True)
+
+import looped_ngpt_lm_b200 as dory  # noqa: E402
+from gpu_util import MODES, check_tokens, cosine_rows, gpu_generate, make, rel_l2  # noqa: E402
+
+F32_TOL = 1e-4
+CAP = dict(max_batch=4, max_seq=160, k_max=4, gamma_max=4, max_chunk=128)
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    w, dw, h = make(synth.TINY, **CAP)
+    return O.Model(synth.TINY, w), dw, h
+
+
+@pytest.fixture(scope="module")
+def tiny_bf16():
+    w, dw, h = make(synth.TINY_BF16, **CAP)
+    return O.Model(synth.TINY_BF16, w), dw, h
+
+
+@pytest.fixture(scope="module")
+def prompt():
+    return synth.make_prompt(0, 64, synth.TINY.vocab)
+
+
+@pytest.mark.parametrize("k", [1, 2, 4])
+@pytest.mark.parametrize("mode", ["last_loop", "per_loop"])
+def test_tiny_f32_matches_oracle(tiny, prompt, k, mode):
+    model, _, h = tiny
+    h.reset()
+    om, cm = MODES[mode]
+    toks, lg = gpu_generate(h, prompt, 17, k, cm)
+    _, ora = O.generate(model, prompt, 17, k, om, forced=toks[:-1])
+    err = np.abs(lg - ora).max()
+    assert err <= F32_TOL, err
+    check_tokens(toks, ora, 2 * F32_TOL)
+
+
+@pytest.mark.parametrize("k", [1, 2, 4])
+@pytest.mark.parametrize("mode", ["last_loop", "per_loop"])
+def test_tiny_bf16_matches_oracle(tiny_bf16, prompt, k, mode):
+    model, _, h = tiny_bf16
+    h.reset()
+    om, cm = MODES[mode]
+    toks, lg = gpu_generate(h, prompt, 17, k, cm)
+    _, ora = O.generate(model, prompt, 17, k, om, forced=toks[:-1])
+    errs = [rel_l2(lg[i], ora[i]) for i in range(len(toks))]
+    assert max(errs) <= 2e-2, errs
+    tol = 4 * max(float(np.abs(lg[i] - ora[i]).max()) for i in range(len(toks)))
+    check_tokens(toks, ora, tol)
+    # final state of the prompt: rerun the prefill and read s_k for every row
+    h.reset()
+    tok = torch.tensor(prompt, dtype=torch.int32, device="cuda")
+    h.prefill([0], tok, [len(prompt)], k, cm)
+    s_gpu = h.read_state("s", len(prompt)).cpu().numpy()
+    tr = {}
+    O.forward_chunk(model, O.Cache(model, 128), prompt, k, om, trace=tr)
+    assert cosine_rows(s_gpu, tr["s"][-1]).min() >= 0.999
+
+
+def test_states_are_unit_norm(tiny, prompt):
+    model, _, h = tiny
+    h.reset()
+    tok = torch.tensor(prompt, dtype=torch.int32, device="cuda")
+    h.prefill([0], tok, [64], 2, dory.LAST_LOOP)
+    for which in ("x", "s", "out"):
+        n = torch.linalg.norm(h.read_state(which, 64), dim=-1)
+        assert torch.all((n - 1).abs() < 1e-5), which
+
+
+def test_k1_modes_identical_on_gpu(tiny, prompt):
+    _, _, h = tiny
+    h.reset()
+    a = gpu_generate(h, prompt, 6, 1, dory.LAST_LOOP, seq=0)
+    b = gpu_generate(h, prompt, 6, 1, dory.PER_LOOP, seq=1)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_input_block_kv_independent_of_k_and_mode(tiny, prompt):
+    _, _, h = tiny
+    h.reset()
+    tok = torch.tensor(prompt[:40], dtype=torch.int32, device="cuda")
+    runs = [(0, 1, dory.LAST_LOOP), (1, 4, dory.LAST_LOOP), (2, 2, dory.PER_LOOP)]
+    for seq, k, m in runs:
+        h.prefill([seq], tok, [40], k, m)
+    ref = h.read_kv(0, 0, 0, 24, 16)  # layer 0 (input block, window 16): last 16 positions
+    for seq, _, _ in runs[1:]:
+        kv = h.read_kv(0, 0, seq, 24, 16)
+        assert torch.equal(kv[0], ref[0]) and torch.equal(kv[1], ref[1])
+
+
+def test_ragged_batch_prefill_and_batched_decode(tiny):
+    model, _, h = tiny
+    h.reset()
+    prompts = [synth.make_prompt(s, n, synth.TINY.vocab) for s, n in ((1, 13), (2, 40), (3, 1))]
+    ids = [2, 0, 3]
+    tok = torch.tensor(np.concatenate(prompts), dtype=torch.int32, device="cuda")
+    V = synth.TINY.vocab
+    lg = torch.empty((3, V), device="cuda")
+    nxt = h.prefill(ids, tok, [len(p) for p in prompts], 2, dory.PER_LOOP, logits=lg)
+    steps = [(nxt.cpu().numpy().copy(), lg.cpu().numpy().copy())]
+    for _ in range(5):
+        nxt = h.decode_step(ids, nxt, 2, dory.PER_LOOP, logits=lg)
+        steps.append((nxt.cpu().numpy().copy(), lg.cpu().numpy().copy()))
+    for b, p in enumerate(prompts):
+        toks = np.array([s[0][b] for s in steps])
+        gl = np.stack([s[1][b] for s in steps])
+        _, ora = O.generate(model, p, 6, 2, O.PER_LOOP, forced=toks[:-1])
+        assert np.abs(gl - ora).max() <= F32_TOL
+        check_tokens(toks, ora, 2 * F32_TOL)
+
+
+@pytest.mark.parametrize("mode", ["last_loop", "per_loop"])
+def test_chunked_prefill(tiny, prompt, mode):
+    """Prompt in three calls (the middle one longer than the window ring)."""
+    model, _, h = tiny
+    h.reset()
+    om, cm = MODES[mode]
+    chunks = [5, 45, 14]
+    lg = torch.empty((1, synth.TINY.vocab), device="cuda")
+    off = 0
+    for c in chunks:
+        tok = torch.tensor(prompt[off:off + c], dtype=torch.int32, device="cuda")
+        h.prefill([0], tok, [c], 4, cm, logits=lg)
+        off += c
+    cache = O.Cache(model, 80)
+    off = 0
+    for c in chunks:
+        ora = O.forward_chunk(model, cache, prompt[off:off + c], 4, om)
+        off += c
+    assert np.abs(lg.cpu().numpy()[0] - ora[-1]).max() <= F32_TOL
+
+
+@pytest.mark.parametrize("mode", ["last_loop", "per_loop"])
+@pytest.mark.parametrize("gamma", [1, 4])
+def test_spec_decode_tiny(tiny, prompt, mode, gamma):
+    model, _, h = tiny
+    om, cm = MODES[mode]
+    n_new = 24
+    # plain k=4 greedy on sequence 0; speculative on sequence 1
+    h.reset()
+    plain, _ = gpu_generate(h, prompt[:48], n_new, 4, cm, seq=0)
+    tok = torch.tensor(prompt[:48], dtype=torch.int32, device="cuda")
+    first = h.prefill([1], tok, [48], 4, cm)
+    out, out_len, st = h.spec_decode([1], first, 1, 4, gamma, cm, n_new - 1)
+    spec = np.concatenate([[int(first[0])], out[0].cpu().numpy()])
+    assert int(out_len[0]) == n_new - 1
+    assert st["steps"] >= 1 and 0 <= st["accepted"] <= st["drafted"]
+    ora, ost = O.spec_generate(model, prompt[:48], n_new, 1, 4, gamma, om)
+    if mode == "per_loop":
+        assert np.array_equal(spec, plain)  # token-identical to plain k=4 decoding
+    assert np.array_equal(spec, ora), (spec, ora)
+    assert h.seq_len(1) >= 48 + n_new - 1
+
+
+def test_spec_decode_batched(tiny):
+    model, _, h = tiny
+    h.reset()
+    prompts = [synth.make_prompt(10 + b, 20 + 7 * b, synth.TINY.vocab) for b in range(3)]
+    ids = [3, 1, 0]
+    tok = torch.tensor(np.concatenate(prompts), dtype=torch.int32, device="cuda")
+    first = h.prefill(ids, tok, [len(p) for p in prompts], 4, dory.PER_LOOP)
+    out, out_len, st = h.spec_decode(ids, first, 1, 4, 4, dory.PER_LOOP, 12)
+    for b, p in enumerate(prompts):
+        ref, _ = O.generate(model, p, 13, 4, O.PER_LOOP)
+        got = np.concatenate([[int(first[b])], out[b].cpu().numpy()])
+        assert np.array_equal(got, ref)
+
+
+def test_state_errors(tiny, prompt):
+    _, _, h = tiny
+    h.reset()
+    tok = torch.tensor(prompt[:8], dtype=torch.int32, device="cuda")
+    h.prefill([0], tok, [8], 2, dory.PER_LOOP)
+    with pytest.raises(dory.DoryError) as e:
+        h.prefill([0], tok, [8], 2, dory.LAST_LOOP)
+    assert e.value.status == 3
+    with pytest.raises(dory.DoryError) as e:
+        h.decode_step([0], tok[:1], 4, dory.PER_LOOP)
+    assert e.value.status == 3
+    bad = torch.tensor([synth.TINY.vocab + 5], dtype=torch.int32, device="cuda")
+    h.decode_step([0], bad, 2, dory.PER_LOOP)
+    with pytest.raises(dory.DoryError) as e:
+        h.synchronize()
+    assert e.value.status == 1
+    h.synchronize()  # the error word was cleared
