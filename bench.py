@@ -211,7 +211,7 @@ def main():
     if rank != 0 or args.no_aux:
         del w_np
         w_np = None
-    max_seq = args.prompt + args.warmup + args.steps + 64
+    max_seq = args.prompt + args.warmup + args.steps + args.profile_steps + 512
     cfg = dory.make_config(shape, max_batch=1, max_seq=max_seq, k_max=4, gamma_max=4, max_chunk=args.prompt)
     h = dory.Handle(cfg, dw, dory.LAST_LOOP if args.mode == "last_loop" else dory.PER_LOOP)
     mode = dory.MODES[args.mode]

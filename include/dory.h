@@ -204,6 +204,20 @@ dory_status dory_read_state(dory_handle* h, int32_t which, float* dst, int32_t r
 dory_status dory_read_kv(dory_handle* h, int32_t layer, int32_t slot, int32_t seq, int32_t pos0, int32_t n,
                          void* k_dst, void* v_dst, dory_stream stream);
 
+/* Projection GEMM on its own (the kernel every projection of the forward
+ * uses): Y_s = X . W^T partial products for X [M, K], W [N, K] bf16 (device,
+ * row-major, 16-byte aligned) with fp32 accumulation.  Y (device) must hold
+ * 8 * M * N floats: the result is *splits slices Y[s][M][N] whose in-order
+ * sum s = 0..*splits-1 is the product.  batch_hint selects the split the
+ * decode path uses for that many sequences; invariant != 0 makes each row's
+ * arithmetic independent of M.  impl: 0 auto, 1 SIMT kernel, 2 tcgen05 only
+ * (DORY_ERR_CUDA if the shape is unsupported).  err_word (device int, may be
+ * NULL) receives DORY_ERR_TIMEOUT-class codes from bounded waits.  Queues work
+ * on `stream`; no handle needed. */
+dory_status dory_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* X, const void* W, float* Y,
+                           int32_t batch_hint, int32_t invariant, int32_t impl, int32_t* splits, int32_t* err_word,
+                           dory_stream stream);
+
 /* Synchronise `stream` and report device-side errors (DORY_ERR_TIMEOUT when
  * a bounded wait in a kernel gave up; the handle stays usable). */
 dory_status dory_synchronize(dory_handle* h, dory_stream stream);

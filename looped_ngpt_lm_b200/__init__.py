@@ -32,7 +32,7 @@ STATUS = {0: "DORY_OK", 1: "DORY_ERR_INVALID_ARG", 2: "DORY_ERR_CAPACITY", 3: "D
 SYMBOLS = ["dory_workspace_size", "dory_create", "dory_destroy", "dory_reset", "dory_prefill",
            "dory_decode_step", "dory_spec_decode", "dory_kv_bytes", "dory_seq_len", "dory_read_state",
            "dory_read_kv", "dory_synchronize", "dory_set_option", "dory_profile_read", "dory_profile_reset",
-           "dory_last_error"]
+           "dory_last_error", "dory_gemm_bf16"]
 
 
 class DoryError(RuntimeError):
@@ -81,6 +81,7 @@ def _load() -> ctypes.CDLL:
         "dory_profile_read": [P, I32, P, ctypes.POINTER(I64), ctypes.POINTER(ctypes.c_double),
                               ctypes.POINTER(ctypes.c_double), IP],
         "dory_profile_reset": [P],
+        "dory_gemm_bf16": [I32, I32, I32, P, P, P, I32, I32, I32, IP, P, P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -150,6 +151,24 @@ class DeviceWeights:
         self._down = arr(*[_ptr(t) for t in self.down])
         self.c = Weights(self.tensors["embed"].data_ptr(), self.tensors["lm_head"].data_ptr(),
                          self._qkv, self._o, self._gu, self._down)
+
+
+def gemm_bf16(X, W, batch_hint=1, invariant=True, impl=0, err=None, stream=None):
+    """Y = X . W^T through dory_gemm_bf16 (X [M, K], W [N, K] bf16 CUDA
+    tensors).  Returns (Y fp32 [M, N], splits); Y is the in-order sum of the
+    kernel's split-K slices."""
+    import torch
+    M, K = X.shape
+    N = W.shape[0]
+    Y = torch.empty((8, M, N), dtype=torch.float32, device=X.device)
+    s = ctypes.c_int32()
+    _check(lib.dory_gemm_bf16(M, N, K, ctypes.c_void_p(X.data_ptr()), ctypes.c_void_p(W.data_ptr()),
+                              ctypes.c_void_p(Y.data_ptr()), batch_hint, int(invariant), impl, ctypes.byref(s),
+                              ctypes.c_void_p(_ptr(err)), _stream(stream)))
+    out = Y[0].clone()
+    for i in range(1, s.value):
+        out += Y[i]
+    return out, s.value
 
 
 def workspace_size(cfg: Config, alloc_mode=LAST_LOOP) -> int:

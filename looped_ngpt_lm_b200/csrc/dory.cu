@@ -209,10 +209,10 @@ size_t layout(dory_handle* h) {
   h->kscr = cv.take<char>(e * M * h->kv_dim);
   h->vscr = cv.take<char>(e * M * h->kv_dim);
   h->hop_head = cv.take<char>(e * h->head_max * d);
-  h->part_rows = (size_t)M * kMaxSplitK;
-  h->part_qkv = cv.take<float>(sizeof(float) * h->part_rows * h->qkv_dim);
-  h->part_y = cv.take<float>(sizeof(float) * h->part_rows * d);
-  h->part_gu = cv.take<float>(sizeof(float) * h->part_rows * 2 * c.d_ff);
+  h->part_rows = (size_t)M;  // rows per split slice; kMaxSplitK slices each
+  h->part_qkv = cv.take<float>(sizeof(float) * kMaxSplitK * h->part_rows * h->qkv_dim);
+  h->part_y = cv.take<float>(sizeof(float) * kMaxSplitK * h->part_rows * d);
+  h->part_gu = cv.take<float>(sizeof(float) * kMaxSplitK * h->part_rows * 2 * c.d_ff);
   h->attn_part = cv.take<float>(sizeof(float) * (size_t)M * c.n_heads * h->nb_max * (c.head_dim + 2));
   h->logits = cv.take<float>(sizeof(float) * (size_t)h->head_max * c.vocab * kMaxSplitK);
   const int gc = c.gamma_max + 1;
@@ -272,6 +272,9 @@ struct Fwd {
   int max_ctx;  // bound on (position + 1) of every row
   bool direct;  // K/V of the chunk go straight into the cache
   int mode;     // dory_cache_mode
+  int k;        // loop count of this pass (last loop = k)
+  int batch;    // sequences in the call (selects the GEMM split)
+  bool invariant;  // decode / speculative rows: GEMM arithmetic independent of M
 };
 
 KVView kv_view(dory_handle* H, int l, int loop, int mode) {
@@ -287,9 +290,11 @@ KVView kv_view(dory_handle* H, int l, int loop, int mode) {
   return v;
 }
 
+// Y (and, when the tensor-core kernel splits K, the slices after it) must
+// hold kMaxSplitK slices of part_rows rows of ldy floats.
 template <typename T>
 dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, const void* W, float* Y, int ldy,
-                 int* S_out, size_t* ps_out, const char* name) {
+                 size_t part_rows, int* S_out, size_t* ps_out, const char* name) {
   dory_handle* H = f.H;
   double bytes = (double)N * K * sizeof(T) + (double)M * K * sizeof(T) + (double)M * N * 4;
   Scope sc(H, f.st, name, bytes);
@@ -299,8 +304,8 @@ dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, cons
     if (H->gemm_impl != 1) {
       int S = 1;
       size_t ps = 0;
-      cudaError_t e = launch_gemm_tc(M, N, K, (const bf16*)X, ldx, (const bf16*)W, Y, ldy, H->part_rows,
-                                     H->err, &S, &ps, f.st);
+      cudaError_t e = launch_gemm_tc(M, N, K, (const bf16*)X, ldx, (const bf16*)W, Y, ldy, part_rows,
+                                     H->err, f.batch, f.invariant, &S, &ps, f.st);
       if (e == cudaSuccess) {
         *S_out = S;
         *ps_out = ps;
@@ -330,7 +335,7 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop) {
     size_t ps;
     if (layer_is_attn(l)) {
       KVView kv = kv_view(H, l, loop, f.mode);
-      RET(gemm<T>(f, M, H->qkv_dim, d, H->hop_t<T>(), d, H->w_qkv[l], H->part_qkv, H->qkv_dim, &S, &ps, "gemm_qkv"));
+      RET(gemm<T>(f, M, H->qkv_dim, d, H->hop_t<T>(), d, H->w_qkv[l], H->part_qkv, H->qkv_dim, H->M_max, &S, &ps, "gemm_qkv"));
       {
         Scope sc(H, f.st, "qkv_post", 0);
         CK(launch_qkv_post<T>(M, c.n_heads, c.n_kv_heads, c.head_dim, H->part_qkv, S, ps, H->q, (T*)H->kscr,
@@ -342,20 +347,27 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop) {
                                (const T*)H->vscr, !f.direct, kv, H->meta, f.max_ctx, H->attn_part, (T*)H->ao,
                                f.st));
       }
-      if (!f.direct) {
+      // Deferred writes (chunks longer than the ring slack): a last-loop
+      // recurrent layer shares one slot across loops, so the chunk's keys are
+      // committed only after the final loop -- committing loop t earlier
+      // would overwrite ring entries of earlier positions that loop t+1 of
+      // this chunk still reads.
+      const bool rec = H->attn[H->attn_of[l]].rec;
+      if (!f.direct && (!rec || f.mode == DORY_PER_LOOP || loop == f.k)) {
         Scope sc(H, f.st, "kv_commit", 0);
         CK(launch_kv_commit<T>(M, c.n_kv_heads, c.head_dim, (const T*)H->kscr, (const T*)H->vscr, kv, H->meta,
                                f.st));
       }
-      RET(gemm<T>(f, M, d, H->q_dim, (const T*)H->ao, H->q_dim, H->w_o[l], H->part_y, d, &S, &ps, "gemm_o"));
+      RET(gemm<T>(f, M, d, H->q_dim, (const T*)H->ao, H->q_dim, H->w_o[l], H->part_y, d, H->M_max, &S, &ps, "gemm_o"));
     } else {
-      RET(gemm<T>(f, M, 2 * c.d_ff, d, H->hop_t<T>(), d, H->w_gu[l], H->part_gu, 2 * c.d_ff, &S, &ps,
-                  "gemm_gate_up"));
+      RET(gemm<T>(f, M, 2 * c.d_ff, d, H->hop_t<T>(), d, H->w_gu[l], H->part_gu, 2 * c.d_ff, H->M_max,
+                  &S, &ps, "gemm_gate_up"));
       {
         Scope sc(H, f.st, "swiglu", 0);
         CK(launch_swiglu<T>(M, c.d_ff, H->part_gu, S, ps, (T*)H->act, f.st));
       }
-      RET(gemm<T>(f, M, d, c.d_ff, (const T*)H->act, c.d_ff, H->w_down[l], H->part_y, d, &S, &ps, "gemm_down"));
+      RET(gemm<T>(f, M, d, c.d_ff, (const T*)H->act, c.d_ff, H->w_down[l], H->part_y, d, H->M_max, &S, &ps,
+                  "gemm_down"));
     }
     Scope sc(H, f.st, "addnorm", 0);
     CK(launch_addnorm<T>(M, d, H->h, H->part_y, S, ps, d, H->hop_t<T>(), f.st));
@@ -423,11 +435,16 @@ dory_status output_and_head(const Fwd<T>& f, int nrows, const int* rows, float* 
     CK(launch_gather_rows<T>(nrows, d, rows, H->hop_t<T>(), (T*)H->hop_head, f.st));
     X = (const T*)H->hop_head;
   }
-  float* lg = logits_out ? logits_out : H->logits;
+  // partial slices live in the internal logits buffer (kMaxSplitK slices
+  // of head_max rows); a split result is reduced into the output in order
   int S;
   size_t ps;
-  RET(gemm<T>(f, nrows, c.vocab, d, X, d, H->head, lg, c.vocab, &S, &ps, "gemm_lm_head"));
-  if (S != 1) return fail(DORY_ERR_CUDA, "LM head GEMM must not split K");
+  RET(gemm<T>(f, nrows, c.vocab, d, X, d, H->head, H->logits, c.vocab, H->head_max, &S, &ps, "gemm_lm_head"));
+  float* lg = logits_out ? logits_out : H->logits;
+  if (S != 1 || lg != H->logits) {
+    Scope sc(H, f.st, "split_reduce", 0);
+    CK(launch_split_reduce(nrows, c.vocab, H->logits, S, ps, lg, f.st));
+  }
   Scope sc(H, f.st, "argmax", 0);
   CK(launch_argmax(nrows, c.vocab, lg, choice, f.st));
   return DORY_OK;
@@ -488,7 +505,7 @@ dory_status prefill_t(dory_handle* H, int batch, const int32_t* seq_ids, const i
   CK(cudaMemcpyAsync(H->head_rows, rows.data(), sizeof(int) * batch, cudaMemcpyHostToDevice, st));
   CK(launch_plan_ragged(batch, M, H->cu, H->seq_ids, H->seq_len, H->meta, st));
   int max_len = *std::max_element(lens, lens + batch);
-  Fwd<T> f{H, st, M, max_ctx, max_len <= H->slack + 1, mode};
+  Fwd<T> f{H, st, M, max_ctx, max_len <= H->slack + 1, mode, k, batch, false};
   RET(input_block<T>(f, tokens));
   RET(loops<T>(f, 1, k, -1, 1));
   RET(output_and_head<T>(f, batch, H->head_rows, last_logits, next_tokens));
@@ -505,7 +522,7 @@ dory_status decode_t(dory_handle* H, int batch, const int32_t* seq_ids, const in
   for (int i = 0; i < batch; ++i) max_ctx = std::max(max_ctx, H->len[seq_ids[i]] + 1);
   RET(upload_ids(H, seq_ids, batch, st));
   CK(launch_plan_uniform(batch, 1, 0, H->seq_ids, H->seq_len, H->meta, st));
-  Fwd<T> f{H, st, batch, max_ctx, true, mode};
+  Fwd<T> f{H, st, batch, max_ctx, true, mode, k, batch, true};
   RET(input_block<T>(f, tokens_in));
   RET(loops<T>(f, 1, k, -1, 1));
   RET(output_and_head<T>(f, batch, nullptr, logits, next_tokens));
@@ -532,7 +549,7 @@ dory_status spec_t(dory_handle* H, int B, const int32_t* seq_ids, const int32_t*
     // drafts: y0, d1..d_{gamma-1} at k = 1, one token per sequence each
     for (int i = 0; i < gamma; ++i) {
       CK(launch_plan_uniform(B, 1, i, H->seq_ids, H->seq_len, H->meta, st));
-      Fwd<T> f{H, st, B, max_ctx, true, mode};
+      Fwd<T> f{H, st, B, max_ctx, true, mode, 1, B, true};
       const int* tok = i == 0 ? H->pending : H->drafts + (i - 1) * B;
       RET(input_block<T>(f, tok));
       CK(launch_stash_copy(B, c.d_model, H->x, H->stash_x, 1, gc, i, 0, st));
@@ -542,7 +559,7 @@ dory_status spec_t(dory_handle* H, int B, const int32_t* seq_ids, const int32_t*
     // d_gamma: input block and loop 1 only
     {
       CK(launch_plan_uniform(B, 1, gamma, H->seq_ids, H->seq_len, H->meta, st));
-      Fwd<T> f{H, st, B, max_ctx, true, mode};
+      Fwd<T> f{H, st, B, max_ctx, true, mode, 1, B, true};
       RET(input_block<T>(f, H->drafts + (gamma - 1) * B));
       CK(launch_stash_copy(B, c.d_model, H->x, H->stash_x, 1, gc, gamma, 0, st));
       Scope sc(H, st, "reinject", 0);
@@ -555,7 +572,7 @@ dory_status spec_t(dory_handle* H, int B, const int32_t* seq_ids, const int32_t*
     {
       const int rps = gamma + 1, M = B * rps;
       CK(launch_plan_uniform(B, rps, 0, H->seq_ids, H->seq_len, H->meta, st));
-      Fwd<T> f{H, st, M, max_ctx, true, mode};
+      Fwd<T> f{H, st, M, max_ctx, true, mode, kv_, B, true};
       CK(launch_stash_copy(M, c.d_model, H->x, H->stash_x, rps, gc, 0, 1, st));
       CK(launch_stash_copy(M, c.d_model, H->s, H->stash_s, rps, gc, 0, 1, st));
       RET(loops<T>(f, 2, kv_, -1, rps));
@@ -775,6 +792,27 @@ dory_status dory_read_kv(dory_handle* h, int32_t layer, int32_t slot, int32_t se
       CK(cudaMemcpyAsync((char*)v_dst + dst, a.V[slot] + src, row, cudaMemcpyDeviceToDevice, st));
     }
   }
+  return DORY_OK;
+}
+
+dory_status dory_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* X, const void* W, float* Y,
+                           int32_t batch_hint, int32_t invariant, int32_t impl, int32_t* splits, int32_t* err_word,
+                           dory_stream stream) {
+  if (M < 1 || N < 1 || K < 1 || !X || !W || !Y || !splits) return fail(DORY_ERR_INVALID_ARG, "bad GEMM arguments");
+  cudaStream_t st = (cudaStream_t)stream;
+  *splits = 1;
+  if (impl != 1) {
+    int S = 1;
+    size_t ps = 0;
+    cudaError_t e = launch_gemm_tc(M, N, K, (const bf16*)X, K, (const bf16*)W, Y, N, (size_t)M, err_word,
+                                   batch_hint < 1 ? 1 : batch_hint, invariant != 0, &S, &ps, st);
+    if (e == cudaSuccess) {
+      *splits = S;
+      return DORY_OK;
+    }
+    if (e != cudaErrorNotSupported || impl == 2) return fail(DORY_ERR_CUDA, "tcgen05 GEMM: %s", cudaGetErrorString(e));
+  }
+  CK(launch_gemm_simt<bf16>(M, N, K, (const bf16*)X, K, (const bf16*)W, Y, N, st));
   return DORY_OK;
 }
 

@@ -1,12 +1,505 @@
+// bf16 GEMM on the sm_100a tensor cores: tcgen05.mma with fp32 accumulators
+// in TMEM, operands staged in shared memory by TMA.
+//
+// Y[m, n] = sum_k X[m, k] W[n, k].  The weight matrix is the MMA's A operand
+// (128-row tiles, K-major, 128-byte swizzle) and the tokens are the MMA's N
+// dimension, so a decode step with one token still fills the 128-lane
+// datapath with weights and the kernel streams W at HBM speed.
+//
+// A work unit is (128-row weight tile, token tile, K split).  Each CTA is
+// persistent and takes units blockIdx.x, blockIdx.x + gridDim.x, ...:
+//   warp 0 (one lane)  TMA producer: A and B tiles into a STAGES-deep ring
+//   warp 1 (one lane)  MMA issuer: 4 K-steps of 16 per 64-wide k-block;
+//                      accumulators double-buffered in TMEM
+//   warps 2..5         epilogue: tcgen05.ld -> registers -> fp32 global
+// Decode tiles use GN = 16 tokens per MMA instruction and loop over NG groups;
+// the prefill tile uses one N = 256 instruction.
+//
+// Every mbarrier wait is bounded (about a second); on expiry the kernel sets
+// the device error word, stops issuing work, waits (bounded) for its own
+// copies in flight, frees its TMEM and returns.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+#include <unordered_map>
+
 #include "gemm_tc.cuh"
 
 namespace dory {
 
-cudaError_t launch_gemm_tc(int, int, int, const bf16*, int, const bf16*, float*, int, size_t, int*, int* S,
-                           size_t* ps, cudaStream_t) {
-  *S = 1;
-  *ps = 0;
-  return cudaErrorNotSupported;
+namespace {
+
+constexpr int BK = 64;            // k elements per stage (128 bytes of bf16: one swizzle row)
+constexpr int BM = 128;           // weight rows per tile (MMA M)
+constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at 2 GHz
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait; false when this CTA has given up (timeout here or elsewhere).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (;;) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      *abort_flag = 1;
+      set_error(err, DEV_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// Bounded wait used during teardown: ignores the abort flag.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > kWaitCycles) return false;
+  return true;
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                            uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 bytes, 8-row core-matrix groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFF) >> 4);  // start address
+  d |= (uint64_t)1 << 16;                   // leading-dimension offset (unused with swizzle)
+  d |= (uint64_t)(1024 >> 4) << 32;         // stride-dimension offset: 8 rows x 128 B
+  d |= (uint64_t)1 << 46;                   // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;                   // 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor: bf16 x bf16 -> fp32, both operands K-major, M = 128.
+__host__ __device__ constexpr uint32_t idesc_bf16(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <int NG, int GN>
+struct Tile {
+  static constexpr int MT = NG * GN;                   // tokens per unit
+  static constexpr int A_BYTES = BM * BK * 2;          // 16 KB
+  static constexpr int B_BYTES = MT * BK * 2;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (200 * 1024) / STAGE > 12 ? 12 : (200 * 1024) / STAGE;
+  static constexpr int ACC = MT;                       // TMEM columns per accumulator
+  static constexpr int TMEM_COLS = 2 * ACC <= 32 ? 32 : 2 * ACC <= 64 ? 64 : 2 * ACC <= 128 ? 128 : 2 * ACC <= 256 ? 256 : 512;
+  static constexpr int SMEM = STAGES * STAGE + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+struct UnitMap {
+  int n_tiles, m_tiles, S, KB, units;
+  __device__ __forceinline__ void decode(int u, int& nt, int& mt, int& s, int& kb0, int& kb1) const {
+    s = u % S;
+    int t = u / S;
+    mt = t % m_tiles;
+    nt = t / m_tiles;
+    kb0 = s * KB / S;
+    kb1 = (s + 1) * KB / S;
+  }
+};
+
+template <int NG, int GN>
+__global__ void __launch_bounds__(192, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, float* Y, int ldy,
+              size_t part_stride, int M, UnitMap um, int* err) {
+  using TL = Tile<NG, GN>;
+  constexpr int STAGES = TL::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* full = (uint64_t*)(smem + STAGES * TL::STAGE);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 4);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&mapA) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&mapB) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TL::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer
+      const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < um.units && ok; u += gridDim.x) {
+        int nt, mt, s, kb0, kb1;
+        um.decode(u, nt, mt, s, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          ++issued;
+          uint8_t* sa = smem + stage * TL::STAGE;
+          mbar_expect_tx(&full[stage], TL::STAGE);
+          tma_load_2d(sa, &mapA, &full[stage], kb * BK, nt * BM, pol_w);
+          tma_load_2d(sa + TL::A_BYTES, &mapB, &full[stage], kb * BK, mt * TL::MT, pol_x);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // drain: every issued copy must land before this CTA may exit.  The
+      // last min(issued, STAGES) stages are the ones that can be in flight;
+      // walk back over them and wait for their fill (bounded).
+      int st = stage;
+      uint32_t ph = phase;
+      for (int i = 0; i < STAGES && i < issued; ++i) {
+        if (st == 0) {
+          st = STAGES;
+          ph ^= 1;
+        }
+        --st;
+        mbar_wait_drain(&full[st], ph);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer
+      constexpr uint32_t IDESC = idesc_bf16(GN);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < um.units && ok; u += gridDim.x) {
+        int nt, mt, s, kb0, kb1;
+        um.decode(u, nt, mt, s, kb0, kb1);
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, err)) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + acc * TL::ACC;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * TL::STAGE);
+          const uint64_t adesc = sw128_desc(sa);
+          const uint64_t bdesc = sw128_desc(sa + TL::A_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+#pragma unroll
+            for (int g = 0; g < NG; ++g) {
+              // +32 bytes per K-step of 16 inside the swizzled row; group g
+              // starts GN rows (GN * 128 bytes) further into the B tile
+              umma(d0 + g * GN, adesc + 2 * kk, bdesc + 2 * kk + (uint64_t)(g * GN * 128 >> 4), IDESC,
+                   (kb > kb0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      // all MMAs issued by this thread have completed once mma_done fires
+      umma_commit(mma_done);
+      mbar_wait_drain(mma_done, 0);
+    }
+  } else {
+    // ---------------- epilogue: warps 2..5 own TMEM lanes 32*(warp%4) ..
+    const int lane_base = 32 * (warp & 3);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int u = blockIdx.x; u < um.units; u += gridDim.x) {
+      int nt, mt, s, kb0, kb1;
+      um.decode(u, nt, mt, s, kb0, kb1);
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, err)) break;
+      tc_fence_after();
+      const int n = nt * BM + lane_base + lane;
+      float* out = Y + (size_t)s * part_stride + n;
+      const int m_base = mt * TL::MT;
+#pragma unroll 1
+      for (int c = 0; c < TL::MT; c += 16) {
+        if (m_base + c >= M) break;
+        float v[16];
+        tmem_ld16(tmem_base + ((uint32_t)lane_base << 16) + acc * TL::ACC + c, v);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int m = m_base + c + j;
+          if (m < M) out[(size_t)m * ldy] = v[j];
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TL::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map over rows x cols (row stride in elements), box of
+// BK columns x box_rows rows, 128-byte swizzle; rows past the end read zeros.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint64_t stride, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {stride * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct MapKey {
+  const void* p;
+  int rows, cols;
+  bool operator==(const MapKey& o) const { return p == o.p && rows == o.rows && cols == o.cols; }
+};
+struct MapKeyHash {
+  size_t operator()(const MapKey& k) const { return std::hash<const void*>()(k.p) ^ ((size_t)k.rows << 20) ^ k.cols; }
+};
+
+std::mutex g_map_mu;
+std::unordered_map<MapKey, CUtensorMap, MapKeyHash> g_wmaps;
+
+bool weight_map(CUtensorMap* m, const void* W, int N, int K) {
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  MapKey key{W, N, K};
+  auto it = g_wmaps.find(key);
+  if (it != g_wmaps.end()) {
+    *m = it->second;
+    return true;
+  }
+  if (!make_map(m, W, N, K, K, BM)) return false;
+  g_wmaps.emplace(key, *m);
+  return true;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int NG, int GN>
+cudaError_t run(const CUtensorMap& ma, const bf16* X, int ldx, int M, int K, float* Y, int ldy, size_t ps,
+                UnitMap um, int* err, cudaStream_t st) {
+  using TL = Tile<NG, GN>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<NG, GN>, cudaFuncAttributeMaxDynamicSharedMemorySize, TL::SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  CUtensorMap mb;
+  if (!make_map(&mb, X, M, K, ldx, TL::MT)) return cudaErrorInvalidValue;
+  int grid = um.units < sm_count() ? um.units : sm_count();
+  k_gemm_tc<NG, GN><<<grid, 192, TL::SMEM, st>>>(ma, mb, Y, ldy, ps, M, um, err);
+  return cudaGetLastError();
+}
+
+// Split factor for the decode tiles: chosen from (N, K, batch) only, never
+// from M, so a row's accumulation grouping is the same at every M.  Model:
+// each round of units runs at the slower of HBM (all units of the round
+// share it) and one SM's own streaming rate; partial sums cost HBM traffic.
+int choose_split(int N, int K, int batch) {
+  const double hbm = 6.5e12, sm_bw = 1.2e11;
+  const int tiles = N / BM, KB = K / BK, sms = sm_count();
+  const double rows = 5.0 * batch;  // decode / verify rows this batch size produces
+  int best = 1;
+  double best_t = 1e30;
+  for (int S = 1; S <= kMaxSplitK && S <= KB; ++S) {
+    const int U = tiles * S;
+    const double ubytes = (double)BM * ((KB + S - 1) / S) * BK * 2;
+    double t = 0;
+    for (int left = U; left > 0; left -= sms) {
+      const int in_round = left < sms ? left : sms;
+      t += fmax(in_round * ubytes / hbm, ubytes / sm_bw);
+    }
+    t += S * rows * N * 8.0 / hbm;
+    if (t < best_t * 0.98) {
+      best_t = t;
+      best = S;
+    }
+  }
+  return best;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf16* W, float* Y, int ldy,
+                           size_t part_rows, int* err, int batch, bool invariant, int* S_out, size_t* ps_out,
+                           cudaStream_t st) {
+  *S_out = 1;
+  *ps_out = 0;
+  if (M <= 0 || N % BM || K % BK || ldx % 8 || (size_t)M > part_rows || ((uintptr_t)X & 15) || ((uintptr_t)W & 15))
+    return cudaErrorNotSupported;
+  CUtensorMap ma;
+  if (!weight_map(&ma, W, N, K)) return cudaErrorNotSupported;
+  UnitMap um;
+  um.n_tiles = N / BM;
+  um.KB = K / BK;
+  if (invariant || M <= 128) {
+    // decode / verify: 16-token MMA groups, split chosen from (N, K, batch)
+    const int S = choose_split(N, K, batch);
+    const size_t ps = part_rows * (size_t)ldy;
+    um.S = S;
+    int NG = M <= 16 ? 1 : M <= 32 ? 2 : M <= 64 ? 4 : 8;
+    const int MT = 16 * NG;
+    um.m_tiles = (M + MT - 1) / MT;
+    um.units = um.n_tiles * um.m_tiles * S;
+    *S_out = S;
+    *ps_out = ps;
+    switch (NG) {
+      case 1: return run<1, 16>(ma, X, ldx, M, K, Y, ldy, ps, um, err, st);
+      case 2: return run<2, 16>(ma, X, ldx, M, K, Y, ldy, ps, um, err, st);
+      case 4: return run<4, 16>(ma, X, ldx, M, K, Y, ldy, ps, um, err, st);
+      default: return run<8, 16>(ma, X, ldx, M, K, Y, ldy, ps, um, err, st);
+    }
+  }
+  // prefill: 128 x 256 tiles, no split
+  um.S = 1;
+  um.m_tiles = (M + 255) / 256;
+  um.units = um.n_tiles * um.m_tiles;
+  return run<1, 256>(ma, X, ldx, M, K, Y, ldy, 0, um, err, st);
 }
 
 }  // namespace dory

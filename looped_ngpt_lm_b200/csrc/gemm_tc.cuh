@@ -11,11 +11,14 @@ constexpr int kMaxSplitK = 8;
 
 // Y = X . W^T for X [M, K] (row stride ldx) and W [N, K], both bf16, fp32
 // accumulation.  Writes S partial products to Y + s * (*part_stride)
-// (row stride ldy); the consumer adds them in order s = 0..S-1.  The split
-// and the per-element accumulation order depend only on (N, K), never on M.
-// part_rows: rows available per slice (>= M).  Returns cudaErrorNotSupported
-// for shapes the kernel does not handle (the caller falls back).
+// (row stride ldy); the consumer adds them in order s = 0..S-1.
+// invariant (or M <= 128): 16-token MMA groups and a split chosen from
+// (N, K, batch) only, so each row's result is bit-identical for every M;
+// otherwise 128 x 256 tiles without split.  part_rows: rows available per
+// slice (>= M).  Returns cudaErrorNotSupported for shapes the kernel does not
+// handle (N % 128, K % 64, unaligned pointers).
 cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf16* W, float* Y, int ldy,
-                           size_t part_rows, int* err, int* S, size_t* part_stride, cudaStream_t st);
+                           size_t part_rows, int* err, int batch, bool invariant, int* S, size_t* part_stride,
+                           cudaStream_t st);
 
 }  // namespace dory

@@ -110,4 +110,7 @@ cudaError_t launch_spec_accept(int B, int gamma, int dstride, const int* seq_ids
 
 cudaError_t launch_fill_i32(int n, int* p, int v, cudaStream_t st);
 
+// out[m, n] = sum_{s<S} part[s * ps + m * N + n] in order s = 0..S-1 (out may alias part).
+cudaError_t launch_split_reduce(int M, int N, const float* part, int S, size_t ps, float* out, cudaStream_t st);
+
 }  // namespace dory

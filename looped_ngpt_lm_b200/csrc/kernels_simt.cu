@@ -88,6 +88,22 @@ cudaError_t launch_fill_i32(int n, int* p, int v, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+__global__ void k_split_reduce(size_t total, const float* part, int S, size_t ps, float* out) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    float a = 0.f;
+    for (int s = 0; s < S; ++s) a += part[s * ps + i];
+    out[i] = a;
+  }
+}
+
+cudaError_t launch_split_reduce(int M, int N, const float* part, int S, size_t ps, float* out, cudaStream_t st) {
+  size_t total = (size_t)M * N;
+  int blocks = (int)((total + 255) / 256);
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  k_split_reduce<<<blocks, 256, 0, st>>>(total, part, S, ps, out);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ embedding
 template <typename T>
 __global__ void k_embed(int d, int vocab, const int* tokens, const T* E, float* h, T* hop, int* err) {
