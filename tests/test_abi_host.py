@@ -20,7 +20,7 @@ FAKE_WS = 1 << 40  # never dereferenced: validation fails before any launch
 def header_functions():
     src = open(os.path.join(ROOT, "include", "dory.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(dory_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(dory_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_every_declared_function_is_exported():
