@@ -226,7 +226,8 @@ dory_status dory_synchronize(dory_handle* h, dory_stream stream);
 enum {
   DORY_OPT_CUDA_GRAPHS = 1, /* 1 (default): replay captured decode steps */
   DORY_OPT_PROFILE = 2,     /* 1: time every launch with CUDA events (slow) */
-  DORY_OPT_GEMM_IMPL = 3    /* bf16 GEMM: 0 auto, 1 SIMT reference kernel, 2 tcgen05 */
+  DORY_OPT_GEMM_IMPL = 3,   /* bf16 GEMM: 0 auto, 1 SIMT reference kernel, 2 tcgen05 */
+  DORY_OPT_PDL = 4          /* 1 (default): programmatic dependent launches (process-wide) */
 };
 dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value);
 

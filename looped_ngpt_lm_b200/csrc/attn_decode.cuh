@@ -1,0 +1,19 @@
+// Fused GQA attention for decode and speculative chunks.
+#pragma once
+
+#include "kernels.cuh"
+
+namespace dory {
+
+constexpr int DEC_BK = 128;  // keys per block (absolute-position aligned)
+
+// Attention of M rows whose K/V go straight into the cache.  qkv: the QKV
+// projection's S split-K partial slices (slice stride ps floats, rows of
+// q_dim + 2 kv_dim).  part: [M, H, nb_cap, hd + 2] scratch; counters:
+// [M * KV] zeros (left zero on return).  out: [M, H * hd] in the storage type.
+template <typename T>
+cudaError_t launch_attn_decode(int M, int H, int KV, int hd, const float* qkv, int S, size_t ps, KVView kv,
+                               RowMeta m, int max_ctx, float* part, int nb_cap, unsigned* counters, T* out,
+                               cudaStream_t st);
+
+}  // namespace dory

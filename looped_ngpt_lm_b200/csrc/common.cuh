@@ -63,3 +63,36 @@ __device__ __forceinline__ void set_error(int* err, int code) {
 }
 
 }  // namespace dory
+
+namespace dory {
+
+// Programmatic dependent launch.  Every kernel of the forward is launched
+// with programmatic stream serialization allowed, so it may start while its
+// predecessor in the stream is still running.  pdl_wait() blocks until the
+// predecessor grid has completed and its memory is visible; a kernel calls it
+// before touching anything an earlier kernel writes or reads.  pdl_trigger()
+// lets the next kernel in the stream start early (it still waits in its own
+// pdl_wait()).  Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Host switch for programmatic launches (tests can turn it off).
+extern bool g_pdl;
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                          Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = g_pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+}  // namespace dory

@@ -21,8 +21,13 @@
 #include <vector>
 
 #include "dory.h"
+#include "attn_decode.cuh"
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
+
+namespace dory {
+bool g_pdl = true;
+}
 
 using namespace dory;
 
@@ -103,6 +108,8 @@ struct dory_handle {
   float *stash_x = nullptr, *stash_s = nullptr;
   int *drafts = nullptr, *pending = nullptr, *vtok = nullptr, *out_len = nullptr, *all_done = nullptr;
   unsigned long long* accepted = nullptr;
+  unsigned* attn_counters = nullptr;  // [M_max * n_kv], zero between launches
+  int nb_cap = 0;                     // key blocks per row the partial buffer holds
 
   // host state
   std::vector<int> len, mode, kfix;  // per sequence; mode -1 = empty
@@ -114,6 +121,12 @@ struct dory_handle {
   std::vector<ProfRec> prof_recs;
   std::vector<cudaEvent_t> ev_pool;
   size_t ev_used = 0;
+  struct Graph {
+    long long key;
+    int seen;
+    cudaGraphExec_t exec;
+  };
+  std::vector<Graph> graphs_cache;
 
   template <typename T>
   T* hop_t() const { return (T*)hop; }
@@ -163,6 +176,7 @@ size_t layout(dory_handle* h) {
   h->M_max = std::max(c.max_chunk, c.max_batch * (c.gamma_max + 1));
   h->head_max = std::max(c.max_batch * (c.gamma_max + 1), c.max_batch);
   h->nb_max = (c.max_seq + ATTN_BK - 1) / ATTN_BK + 1;
+  h->nb_cap = std::max(h->nb_max, (c.max_seq + DEC_BK - 1) / DEC_BK + 1);
   const int M = h->M_max;
   const size_t e = h->esz;
 
@@ -213,7 +227,8 @@ size_t layout(dory_handle* h) {
   h->part_qkv = cv.take<float>(sizeof(float) * kMaxSplitK * h->part_rows * h->qkv_dim);
   h->part_y = cv.take<float>(sizeof(float) * kMaxSplitK * h->part_rows * d);
   h->part_gu = cv.take<float>(sizeof(float) * kMaxSplitK * h->part_rows * 2 * c.d_ff);
-  h->attn_part = cv.take<float>(sizeof(float) * (size_t)M * c.n_heads * h->nb_max * (c.head_dim + 2));
+  h->attn_part = cv.take<float>(sizeof(float) * (size_t)M * c.n_heads * h->nb_cap * (c.head_dim + 2));
+  h->attn_counters = cv.take<unsigned>(sizeof(unsigned) * (size_t)M * c.n_kv_heads);
   h->logits = cv.take<float>(sizeof(float) * (size_t)h->head_max * c.vocab * kMaxSplitK);
   const int gc = c.gamma_max + 1;
   h->stash_x = cv.take<float>(sizeof(float) * (size_t)c.max_batch * gc * d);
@@ -325,8 +340,10 @@ dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, cons
     if (r_ != DORY_OK) return r_;       \
   } while (0)
 
+// Apply physical layers l0..l1-1.  copy_last (if not NULL) also receives the
+// result of the last layer.
 template <typename T>
-dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop) {
+dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop, float* copy_last = nullptr) {
   dory_handle* H = f.H;
   const dory_config& c = H->c;
   const int M = f.M, d = c.d_model;
@@ -336,27 +353,33 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop) {
     if (layer_is_attn(l)) {
       KVView kv = kv_view(H, l, loop, f.mode);
       RET(gemm<T>(f, M, H->qkv_dim, d, H->hop_t<T>(), d, H->w_qkv[l], H->part_qkv, H->qkv_dim, H->M_max, &S, &ps, "gemm_qkv"));
-      {
-        Scope sc(H, f.st, "qkv_post", 0);
-        CK(launch_qkv_post<T>(M, c.n_heads, c.n_kv_heads, c.head_dim, H->part_qkv, S, ps, H->q, (T*)H->kscr,
-                              (T*)H->vscr, f.direct, kv, H->meta, c.max_batch, f.st));
-      }
-      {
-        Scope sc(H, f.st, "attention", 0);
-        CK(launch_attention<T>(M, c.n_heads, c.n_kv_heads, c.head_dim, H->q, (const T*)H->kscr,
-                               (const T*)H->vscr, !f.direct, kv, H->meta, f.max_ctx, H->attn_part, (T*)H->ao,
-                               f.st));
-      }
-      // Deferred writes (chunks longer than the ring slack): a last-loop
-      // recurrent layer shares one slot across loops, so the chunk's keys are
-      // committed only after the final loop -- committing loop t earlier
-      // would overwrite ring entries of earlier positions that loop t+1 of
-      // this chunk still reads.
-      const bool rec = H->attn[H->attn_of[l]].rec;
-      if (!f.direct && (!rec || f.mode == DORY_PER_LOOP || loop == f.k)) {
-        Scope sc(H, f.st, "kv_commit", 0);
-        CK(launch_kv_commit<T>(M, c.n_kv_heads, c.head_dim, (const T*)H->kscr, (const T*)H->vscr, kv, H->meta,
-                               f.st));
+      if (f.direct) {
+        // fused: q from the partials, own K/V into the cache, split-KV attention
+        Scope sc(H, f.st, "attn_decode", 0);
+        CK(launch_attn_decode<T>(M, c.n_heads, c.n_kv_heads, c.head_dim, H->part_qkv, S, ps, kv, H->meta, f.max_ctx,
+                                 H->attn_part, H->nb_cap, H->attn_counters, (T*)H->ao, f.st));
+      } else {
+        // long chunks: K/V into scratch, attention, then the cache commit
+        {
+          Scope sc(H, f.st, "qkv_post", 0);
+          CK(launch_qkv_post<T>(M, c.n_heads, c.n_kv_heads, c.head_dim, H->part_qkv, S, ps, H->q, (T*)H->kscr,
+                                (T*)H->vscr, false, kv, H->meta, c.max_batch, f.st));
+        }
+        {
+          Scope sc(H, f.st, "attention", 0);
+          CK(launch_attention<T>(M, c.n_heads, c.n_kv_heads, c.head_dim, H->q, (const T*)H->kscr,
+                                 (const T*)H->vscr, true, kv, H->meta, f.max_ctx, H->attn_part, (T*)H->ao, f.st));
+        }
+        // A last-loop recurrent layer shares one slot across loops, so the
+        // chunk's keys are committed only after the final loop: committing
+        // loop t earlier would overwrite ring entries of earlier positions
+        // that loop t+1 of this chunk still reads.
+        const bool rec = H->attn[H->attn_of[l]].rec;
+        if (!rec || f.mode == DORY_PER_LOOP || loop == f.k) {
+          Scope sc(H, f.st, "kv_commit", 0);
+          CK(launch_kv_commit<T>(M, c.n_kv_heads, c.head_dim, (const T*)H->kscr, (const T*)H->vscr, kv, H->meta,
+                                 f.st));
+        }
       }
       RET(gemm<T>(f, M, d, H->q_dim, (const T*)H->ao, H->q_dim, H->w_o[l], H->part_y, d, H->M_max, &S, &ps, "gemm_o"));
     } else {
@@ -370,7 +393,7 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop) {
                   "gemm_down"));
     }
     Scope sc(H, f.st, "addnorm", 0);
-    CK(launch_addnorm<T>(M, d, H->h, H->part_y, S, ps, d, H->hop_t<T>(), f.st));
+    CK(launch_addnorm<T>(M, d, H->h, H->part_y, S, ps, d, H->hop_t<T>(), l == l1 - 1 ? copy_last : nullptr, f.st));
   }
   return DORY_OK;
 }
@@ -382,10 +405,10 @@ dory_status input_block(const Fwd<T>& f, const int* tokens) {
   const dory_config& c = H->c;
   {
     Scope sc(H, f.st, "embed", 0);
-    CK(launch_embed<T>(f.M, c.d_model, c.vocab, tokens, (const T*)H->embed, H->h, H->hop_t<T>(), H->err, f.st));
+    CK(launch_embed<T>(f.M, c.d_model, c.vocab, tokens, (const T*)H->embed, H->h, H->hop_t<T>(),
+                       c.n_in == 0 ? H->x : nullptr, H->err, f.st));
   }
-  RET(run_layers<T>(f, 0, c.n_in, 0));
-  CK(cudaMemcpyAsync(H->x, H->h, sizeof(float) * f.M * c.d_model, cudaMemcpyDeviceToDevice, f.st));
+  RET(run_layers<T>(f, 0, c.n_in, 0, H->x));
   return DORY_OK;
 }
 
@@ -408,16 +431,17 @@ dory_status loops(const Fwd<T>& f, int t0, int k, int stash_col, int rps) {
     }
     RET(run_layers<T>(f, c.n_in, c.n_in + c.n_rec, t));
   }
-  // exit: s_k = N(h) (or s_k = s when no loop ran here)
-  float* save = (k == 1 && stash_col >= 0) ? H->stash_s : nullptr;
+  // exit: s_k = N(h) (or s_k = s when no loop ran here); s_k is kept in s,
+  // or in the speculative stash when a stash column is given
   Scope sc(H, f.st, "reinject", 0);
   if (t0 > k) {
     CK(launch_reinject<T>(f.M, d, H->h, H->x, 2, H->s, false, H->hop_t<T>(), nullptr, 1, 1, 0, f.st));
+  } else if (stash_col >= 0 && k == 1) {
+    CK(launch_reinject<T>(f.M, d, H->h, H->x, 1, nullptr, false, H->hop_t<T>(), H->stash_s, rps, gc, stash_col,
+                          f.st));
   } else {
-    CK(launch_reinject<T>(f.M, d, H->h, H->x, 1, nullptr, false, H->hop_t<T>(), save, rps, gc,
-                          stash_col < 0 ? 0 : stash_col, f.st));
+    CK(launch_reinject<T>(f.M, d, H->h, H->x, 1, nullptr, false, H->hop_t<T>(), H->s, 1, 1, 0, f.st));
   }
-  CK(cudaMemcpyAsync(H->s, H->h, sizeof(float) * f.M * d, cudaMemcpyDeviceToDevice, f.st));
   return DORY_OK;
 }
 
@@ -516,17 +540,66 @@ dory_status prefill_t(dory_handle* H, int batch, const int32_t* seq_ids, const i
 }
 
 template <typename T>
-dory_status decode_t(dory_handle* H, int batch, const int32_t* seq_ids, const int32_t* tokens_in, int k, int mode,
-                     float* logits, int32_t* next_tokens, cudaStream_t st) {
-  int max_ctx = 0;
-  for (int i = 0; i < batch; ++i) max_ctx = std::max(max_ctx, H->len[seq_ids[i]] + 1);
-  RET(upload_ids(H, seq_ids, batch, st));
+dory_status decode_body(dory_handle* H, int batch, const int32_t* tokens_in, int k, int mode, int max_ctx,
+                        float* logits, int32_t* next_tokens, cudaStream_t st) {
   CK(launch_plan_uniform(batch, 1, 0, H->seq_ids, H->seq_len, H->meta, st));
   Fwd<T> f{H, st, batch, max_ctx, true, mode, k, batch, true};
   RET(input_block<T>(f, tokens_in));
   RET(loops<T>(f, 1, k, -1, 1));
   RET(output_and_head<T>(f, batch, nullptr, logits, next_tokens));
   CK(launch_advance(batch, H->seq_ids, H->seq_len, 1, st));
+  return DORY_OK;
+}
+
+// Decode steps without logits replay a CUDA graph of the whole step (captured
+// on the second call with the same batch, k and mode; the first call also
+// initialises the kernels' attributes outside any capture).  Inputs are copied
+// into the handle's buffers first, outputs copied out after, so the graph only
+// touches workspace memory; attention grids are sized for max_seq.
+template <typename T>
+dory_status decode_t(dory_handle* H, int batch, const int32_t* seq_ids, const int32_t* tokens_in, int k, int mode,
+                     float* logits, int32_t* next_tokens, cudaStream_t st) {
+  int max_ctx = 0;
+  for (int i = 0; i < batch; ++i) max_ctx = std::max(max_ctx, H->len[seq_ids[i]] + 1);
+  RET(upload_ids(H, seq_ids, batch, st));
+  const bool use_graph = H->graphs && !H->profile && logits == nullptr;
+  if (!use_graph) {
+    RET(decode_body<T>(H, batch, tokens_in, k, mode, max_ctx, logits, next_tokens, st));
+  } else {
+    const long long key = ((long long)batch << 16) | (k << 4) | mode;
+    dory_handle::Graph* g = nullptr;
+    for (auto& e : H->graphs_cache)
+      if (e.key == key) g = &e;
+    if (!g) {
+      H->graphs_cache.push_back({key, 0, nullptr});
+      g = &H->graphs_cache.back();
+    }
+    CK(cudaMemcpyAsync(H->tokens, tokens_in, sizeof(int) * batch, cudaMemcpyDeviceToDevice, st));
+    if (!g->exec && g->seen == 0) {
+      g->seen = 1;
+      RET(decode_body<T>(H, batch, H->tokens, k, mode, H->c.max_seq, nullptr, H->next, st));
+    } else {
+      if (!g->exec) {
+        cudaGraph_t graph = nullptr;
+        CK(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
+        dory_status r = decode_body<T>(H, batch, H->tokens, k, mode, H->c.max_seq, nullptr, H->next, st);
+        cudaError_t e = cudaStreamEndCapture(st, &graph);
+        if (r != DORY_OK) {
+          if (graph) cudaGraphDestroy(graph);
+          return r;
+        }
+        if (e != cudaSuccess) return fail(DORY_ERR_CUDA, "graph capture: %s", cudaGetErrorString(e));
+        e = cudaGraphInstantiate(&g->exec, graph, 0);
+        cudaGraphDestroy(graph);
+        if (e != cudaSuccess) {
+          g->exec = nullptr;
+          return fail(DORY_ERR_CUDA, "graph instantiate: %s", cudaGetErrorString(e));
+        }
+      }
+      CK(cudaGraphLaunch(g->exec, st));
+    }
+    CK(cudaMemcpyAsync(next_tokens, H->next, sizeof(int) * batch, cudaMemcpyDeviceToDevice, st));
+  }
   for (int i = 0; i < batch; ++i) H->len[seq_ids[i]] += 1;
   H->last_rows = batch;
   return DORY_OK;
@@ -657,6 +730,8 @@ dory_status dory_create(const dory_config* cfg, const dory_weights* w, dory_cach
 dory_status dory_destroy(dory_handle* h) {
   if (!h) return fail(DORY_ERR_INVALID_ARG, "NULL handle");
   for (auto e : h->ev_pool) cudaEventDestroy(e);
+  for (auto& g : h->graphs_cache)
+    if (g.exec) cudaGraphExecDestroy(g.exec);
   delete h;
   return DORY_OK;
 }
@@ -667,6 +742,7 @@ dory_status dory_reset(dory_handle* h, int32_t seq, dory_stream stream) {
   if (seq == -1) {
     CK(cudaMemsetAsync(h->seq_len, 0, sizeof(int) * h->c.max_batch, st));
     CK(cudaMemsetAsync(h->err, 0, sizeof(int) * 4, st));
+    CK(cudaMemsetAsync(h->attn_counters, 0, sizeof(unsigned) * (size_t)h->M_max * h->c.n_kv_heads, st));
     std::fill(h->len.begin(), h->len.end(), 0);
     std::fill(h->mode.begin(), h->mode.end(), -1);
     return DORY_OK;
@@ -836,6 +912,7 @@ dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value) {
   switch (opt) {
     case DORY_OPT_CUDA_GRAPHS: h->graphs = value != 0; return DORY_OK;
     case DORY_OPT_PROFILE: h->profile = value != 0; return DORY_OK;
+    case DORY_OPT_PDL: dory::g_pdl = value != 0; return DORY_OK;
     case DORY_OPT_GEMM_IMPL:
       if (value < 0 || value > 2) return fail(DORY_ERR_INVALID_ARG, "bad GEMM impl");
       h->gemm_impl = (int)value;

@@ -220,31 +220,50 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  if (threadIdx.x == 0) pdl_trigger();
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer
       const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
-      int stage = 0, issued = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; u < um.units && ok; u += gridDim.x) {
-        int nt, mt, s, kb0, kb1;
-        um.decode(u, nt, mt, s, kb0, kb1);
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, err)) {
-            ok = false;
-            break;
-          }
-          ++issued;
-          uint8_t* sa = smem + stage * TL::STAGE;
-          mbar_expect_tx(&full[stage], TL::STAGE);
-          tma_load_2d(sa, &mapA, &full[stage], kb * BK, nt * BM, pol_w);
-          tma_load_2d(sa + TL::A_BYTES, &mapB, &full[stage], kb * BK, mt * TL::MT, pol_x);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1;
-          }
+      // (u, kb) items of this CTA in order
+      int u = blockIdx.x, nt = 0, mt = 0, s = 0, kb = 0, kb1 = 0;
+      if (u < um.units) um.decode(u, nt, mt, s, kb, kb1);
+      auto next = [&]() {
+        if (++kb >= kb1) {
+          u += gridDim.x;
+          if (u < um.units) um.decode(u, nt, mt, s, kb, kb1);
         }
+      };
+      // Weights do not depend on earlier kernels: fill the first stages with
+      // A tiles before waiting for the predecessor grid, then add B.
+      int pre_kb[STAGES], pre_mt[STAGES];
+      int npre = 0;
+      while (npre < STAGES && u < um.units) {
+        uint8_t* sa = smem + npre * TL::STAGE;
+        mbar_expect_tx(&full[npre], TL::STAGE);
+        tma_load_2d(sa, &mapA, &full[npre], kb * BK, nt * BM, pol_w);
+        pre_kb[npre] = kb;
+        pre_mt[npre] = mt;
+        ++npre;
+        next();
+      }
+      pdl_wait();
+      for (int i = 0; i < npre; ++i)
+        tma_load_2d(smem + i * TL::STAGE + TL::A_BYTES, &mapB, &full[i], pre_kb[i] * BK, pre_mt[i] * TL::MT, pol_x);
+      int stage = npre % STAGES, issued = npre;
+      uint32_t phase = npre == STAGES ? 1u : 0u;
+      while (u < um.units) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, err)) break;
+        ++issued;
+        uint8_t* sa = smem + stage * TL::STAGE;
+        mbar_expect_tx(&full[stage], TL::STAGE);
+        tma_load_2d(sa, &mapA, &full[stage], kb * BK, nt * BM, pol_w);
+        tma_load_2d(sa + TL::A_BYTES, &mapB, &full[stage], kb * BK, mt * TL::MT, pol_x);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+        next();
       }
       // drain: every issued copy must land before this CTA may exit.  The
       // last min(issued, STAGES) stages are the ones that can be in flight;
@@ -261,6 +280,7 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else if (warp == 1) {
+    pdl_wait();
     if (lane == 0) {
       // ---------------- MMA issuer
       constexpr uint32_t IDESC = idesc_bf16(GN);
@@ -311,6 +331,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ---------------- epilogue: warps 2..5 own TMEM lanes 32*(warp%4) ..
+    pdl_wait();
     const int lane_base = 32 * (warp & 3);
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -432,8 +453,7 @@ cudaError_t run(const CUtensorMap& ma, const bf16* X, int ldx, int M, int K, flo
   CUtensorMap mb;
   if (!make_map(&mb, X, M, K, ldx, TL::MT)) return cudaErrorInvalidValue;
   int grid = um.units < sm_count() ? um.units : sm_count();
-  k_gemm_tc<NG, GN><<<grid, 192, TL::SMEM, st>>>(ma, mb, Y, ldy, ps, M, um, err);
-  return cudaGetLastError();
+  return launch(k_gemm_tc<NG, GN>, dim3(grid), dim3(192), TL::SMEM, st, ma, mb, Y, ldy, ps, M, um, err);
 }
 
 // Split factor for the decode tiles: chosen from (N, K, batch) only, never

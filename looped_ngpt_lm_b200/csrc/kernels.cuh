@@ -43,13 +43,15 @@ cudaError_t launch_advance(int n_seq, const int* seq_ids, int* seq_len, int delt
 cudaError_t launch_advance_ragged(int n_seq, const int* seq_ids, const int* cu, int* seq_len, cudaStream_t st);
 
 // ---- elementwise / normalisation -----------------------------------------
+// h <- E[token] (fp32), hop <- E[token]; x (if not NULL) <- the same rows.
 template <typename T>
-cudaError_t launch_embed(int M, int d, int vocab, const int* tokens, const T* E, float* h, T* hop,
+cudaError_t launch_embed(int M, int d, int vocab, const int* tokens, const T* E, float* h, T* hop, float* x,
                          int* err, cudaStream_t st);
-// h <- N(h + sum_{s<S} y[s]) ; hop <- (T)h.  y[s] = y + s*part_stride, rows of ldy.
+// h <- N(h + sum_{s<S} y[s]) ; hop <- (T)h ; copy_out (if not NULL) <- h.
+// y[s] = y + s*part_stride, rows of ldy.  S <= kMaxSplitK.
 template <typename T>
 cudaError_t launch_addnorm(int M, int d, float* h, const float* y, int S, size_t part_stride, int ldy,
-                           T* hop, cudaStream_t st);
+                           T* hop, float* copy_out, cudaStream_t st);
 // Loop boundary.  s_src: 0 -> s = x ; 1 -> s = N(h) ; 2 -> s = s_in.
 // If make_u: out = N(s + x), else out = s.  h <- out, hop <- (T)out.
 // If s_save: s_save <- s.  stash rows: when stash_x/stash_s are given, row r

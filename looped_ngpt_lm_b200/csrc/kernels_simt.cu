@@ -11,12 +11,17 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "gemm_tc.cuh"
 
 namespace dory {
+
+constexpr int kMaxSplit = kMaxSplitK;
 
 // ------------------------------------------------------------------ planning
 __global__ void k_plan_uniform(int n_rows, int rps, int pos_offset, const int* seq_ids, const int* seq_len,
                                RowMeta m) {
+  pdl_wait();
+  pdl_trigger();
   int r = blockIdx.x * blockDim.x + threadIdx.x;
   if (r >= n_rows) return;
   int b = r / rps, i = r % rps;
@@ -32,11 +37,13 @@ __global__ void k_plan_uniform(int n_rows, int rps, int pos_offset, const int* s
 cudaError_t launch_plan_uniform(int n_seq, int rps, int pos_offset, const int* seq_ids, const int* seq_len,
                                 RowMeta m, cudaStream_t st) {
   int n = n_seq * rps;
-  k_plan_uniform<<<(n + 127) / 128, 128, 0, st>>>(n, rps, pos_offset, seq_ids, seq_len, m);
+  launch(k_plan_uniform, (n + 127) / 128, 128, 0, st, n, rps, pos_offset, seq_ids, seq_len, m);
   return cudaGetLastError();
 }
 
 __global__ void k_plan_ragged(int n_seq, const int* cu, const int* seq_ids, const int* seq_len, RowMeta m) {
+  pdl_wait();
+  pdl_trigger();
   int b = blockIdx.x;
   int seq = seq_ids[b];
   int r0 = cu[b], r1 = cu[b + 1];
@@ -53,42 +60,50 @@ __global__ void k_plan_ragged(int n_seq, const int* cu, const int* seq_ids, cons
 cudaError_t launch_plan_ragged(int n_seq, int n_rows, const int* cu, const int* seq_ids, const int* seq_len,
                                RowMeta m, cudaStream_t st) {
   (void)n_rows;
-  k_plan_ragged<<<n_seq, 128, 0, st>>>(n_seq, cu, seq_ids, seq_len, m);
+  launch(k_plan_ragged, n_seq, 128, 0, st, n_seq, cu, seq_ids, seq_len, m);
   return cudaGetLastError();
 }
 
 __global__ void k_advance(int n_seq, const int* seq_ids, int* seq_len, int delta) {
+  pdl_wait();
+  pdl_trigger();
   int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < n_seq) seq_len[seq_ids[b]] += delta;
 }
 
 cudaError_t launch_advance(int n_seq, const int* seq_ids, int* seq_len, int delta, cudaStream_t st) {
-  k_advance<<<(n_seq + 127) / 128, 128, 0, st>>>(n_seq, seq_ids, seq_len, delta);
+  launch(k_advance, (n_seq + 127) / 128, 128, 0, st, n_seq, seq_ids, seq_len, delta);
   return cudaGetLastError();
 }
 
 __global__ void k_advance_ragged(int n_seq, const int* seq_ids, const int* cu, int* seq_len) {
+  pdl_wait();
+  pdl_trigger();
   int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < n_seq) seq_len[seq_ids[b]] += cu[b + 1] - cu[b];
 }
 
 cudaError_t launch_advance_ragged(int n_seq, const int* seq_ids, const int* cu, int* seq_len, cudaStream_t st) {
-  k_advance_ragged<<<(n_seq + 127) / 128, 128, 0, st>>>(n_seq, seq_ids, cu, seq_len);
+  launch(k_advance_ragged, (n_seq + 127) / 128, 128, 0, st, n_seq, seq_ids, cu, seq_len);
   return cudaGetLastError();
 }
 
 __global__ void k_fill_i32(int n, int* p, int v) {
+  pdl_wait();
+  pdl_trigger();
   int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) p[i] = v;
 }
 
 cudaError_t launch_fill_i32(int n, int* p, int v, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
-  k_fill_i32<<<(n + 255) / 256, 256, 0, st>>>(n, p, v);
+  launch(k_fill_i32, (n + 255) / 256, 256, 0, st, n, p, v);
   return cudaGetLastError();
 }
 
 __global__ void k_split_reduce(size_t total, const float* part, int S, size_t ps, float* out) {
+  pdl_wait();
+  pdl_trigger();
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
     float a = 0.f;
     for (int s = 0; s < S; ++s) a += part[s * ps + i];
@@ -100,13 +115,15 @@ cudaError_t launch_split_reduce(int M, int N, const float* part, int S, size_t p
   size_t total = (size_t)M * N;
   int blocks = (int)((total + 255) / 256);
   if (blocks > 148 * 16) blocks = 148 * 16;
-  k_split_reduce<<<blocks, 256, 0, st>>>(total, part, S, ps, out);
+  launch(k_split_reduce, blocks, 256, 0, st, total, part, S, ps, out);
   return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ embedding
 template <typename T>
-__global__ void k_embed(int d, int vocab, const int* tokens, const T* E, float* h, T* hop, int* err) {
+__global__ void k_embed(int d, int vocab, const int* tokens, const T* E, float* h, T* hop, float* x, int* err) {
+  pdl_wait();
+  pdl_trigger();
   int r = blockIdx.x;
   int tok = tokens[r];
   if (tok < 0 || tok >= vocab) {
@@ -118,32 +135,45 @@ __global__ void k_embed(int d, int vocab, const int* tokens, const T* E, float* 
     T v = src[i];
     h[(size_t)r * d + i] = to_f(v);
     hop[(size_t)r * d + i] = v;
+    if (x) x[(size_t)r * d + i] = to_f(v);
   }
 }
 
 template <typename T>
-cudaError_t launch_embed(int M, int d, int vocab, const int* tokens, const T* E, float* h, T* hop, int* err,
-                         cudaStream_t st) {
-  k_embed<T><<<M, 256, 0, st>>>(d, vocab, tokens, E, h, hop, err);
+cudaError_t launch_embed(int M, int d, int vocab, const int* tokens, const T* E, float* h, T* hop, float* x,
+                         int* err, cudaStream_t st) {
+  launch(k_embed<T>, M, 256, 0, st, d, vocab, tokens, E, h, hop, x, err);
   return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ add + norm
-// One 256-thread block per row; thread t owns elements t, t+256, ...
+// One 512-thread block per row; thread t owns elements t, t+512, ...; the S
+// partial loads are independent (unrolled, predicated) so they overlap.
+constexpr int AN_THREADS = 512;
+constexpr int AN_CPT = 8;  // d <= 4096
 template <typename T>
-__global__ void k_addnorm(int d, float* h, const float* y, int S, size_t ps, int ldy, T* hop) {
+__global__ void __launch_bounds__(AN_THREADS) k_addnorm(int d, float* h, const float* __restrict__ y, int S,
+                                                        size_t ps, int ldy, T* hop, float* copy_out) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[33];
   const int r = blockIdx.x;
   float* hr = h + (size_t)r * d;
-  float v[16];  // d <= 16 * 256
+  const float* yr = y + (size_t)r * ldy;
+  float v[AN_CPT];
   float ss = 0.f;
 #pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    int i = threadIdx.x + c * 256;
+  for (int c = 0; c < AN_CPT; ++c) {
+    const int i = threadIdx.x + c * AN_THREADS;
     v[c] = 0.f;
     if (i < d) {
+      float p[kMaxSplit];
+#pragma unroll
+      for (int s = 0; s < kMaxSplit; ++s) p[s] = s < S ? __ldcg(yr + s * ps + i) : 0.f;
       float acc = 0.f;
-      for (int s = 0; s < S; ++s) acc += y[s * ps + (size_t)r * ldy + i];
+#pragma unroll
+      for (int s = 0; s < kMaxSplit; ++s)
+        if (s < S) acc += p[s];
       v[c] = hr[i] + acc;
       ss += v[c] * v[c];
     }
@@ -151,28 +181,30 @@ __global__ void k_addnorm(int d, float* h, const float* y, int S, size_t ps, int
   ss = block_sum(ss, red);
   const float inv = 1.f / fmaxf(sqrtf(ss), 1e-12f);
 #pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    int i = threadIdx.x + c * 256;
+  for (int c = 0; c < AN_CPT; ++c) {
+    const int i = threadIdx.x + c * AN_THREADS;
     if (i < d) {
-      float o = v[c] * inv;
+      const float o = v[c] * inv;
       hr[i] = o;
       hop[(size_t)r * d + i] = from_f<T>(o);
+      if (copy_out) copy_out[(size_t)r * d + i] = o;
     }
   }
 }
 
 template <typename T>
 cudaError_t launch_addnorm(int M, int d, float* h, const float* y, int S, size_t ps, int ldy, T* hop,
-                           cudaStream_t st) {
-  if (d > 16 * 256) return cudaErrorInvalidValue;
-  k_addnorm<T><<<M, 256, 0, st>>>(d, h, y, S, ps, ldy, hop);
-  return cudaGetLastError();
+                           float* copy_out, cudaStream_t st) {
+  if (d > AN_CPT * AN_THREADS || S > kMaxSplit) return cudaErrorInvalidValue;
+  return launch(k_addnorm<T>, dim3(M), dim3(AN_THREADS), 0, st, d, h, y, S, ps, ldy, hop, copy_out);
 }
 
 // ------------------------------------------------------------------ loop boundary
 template <typename T>
 __global__ void k_reinject(int d, float* h, const float* x, int s_src, const float* s_in, bool make_u, T* hop,
                            float* stash_s, int rps, int scols, int col0) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[33];
   const int r = blockIdx.x;
   float* hr = h + (size_t)r * d;
@@ -231,11 +263,13 @@ template <typename T>
 cudaError_t launch_reinject(int M, int d, float* h, const float* x, int s_src, const float* s_in, bool make_u,
                             T* hop, float* stash_s, int rps, int scols, int col0, cudaStream_t st) {
   if (d > 16 * 256) return cudaErrorInvalidValue;
-  k_reinject<T><<<M, 256, 0, st>>>(d, h, x, s_src, s_in, make_u, hop, stash_s, rps, scols, col0);
+  launch(k_reinject<T>, M, 256, 0, st, d, h, x, s_src, s_in, make_u, hop, stash_s, rps, scols, col0);
   return cudaGetLastError();
 }
 
 __global__ void k_stash_copy(int d, float* state, float* stash, int rps, int scols, int col0, int dir) {
+  pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x;
   size_t srow = (size_t)((r / rps) * scols + r % rps + col0) * d;
   for (int i = threadIdx.x; i < d; i += blockDim.x) {
@@ -248,7 +282,7 @@ __global__ void k_stash_copy(int d, float* state, float* stash, int rps, int sco
 
 cudaError_t launch_stash_copy(int M, int d, float* state, float* stash, int rps, int scols, int col0, int dir,
                               cudaStream_t st) {
-  k_stash_copy<<<M, 256, 0, st>>>(d, state, stash, rps, scols, col0, dir);
+  launch(k_stash_copy, M, 256, 0, st, d, state, stash, rps, scols, col0, dir);
   return cudaGetLastError();
 }
 
@@ -256,6 +290,8 @@ cudaError_t launch_stash_copy(int M, int d, float* state, float* stash, int rps,
 template <typename T>
 __global__ void k_qkv_post(int H, int KV, int hd, const float* qkv, int S, size_t ps, float* q_out, T* kscr,
                            T* vscr, bool direct, KVView kv, RowMeta m, int max_batch) {
+  pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x;
   const int qd = H * hd, kvd = KV * hd, ld = qd + 2 * kvd;
   const float* src = qkv + (size_t)r * ld;
@@ -290,7 +326,7 @@ __global__ void k_qkv_post(int H, int KV, int hd, const float* qkv, int S, size_
 template <typename T>
 cudaError_t launch_qkv_post(int M, int H, int KV, int hd, const float* qkv, int S, size_t ps, float* q_out,
                             T* kscr, T* vscr, bool direct, KVView kv, RowMeta m, int max_batch, cudaStream_t st) {
-  k_qkv_post<T><<<M, 256, 0, st>>>(H, KV, hd, qkv, S, ps, q_out, kscr, vscr, direct, kv, m, max_batch);
+  launch(k_qkv_post<T>, M, 256, 0, st, H, KV, hd, qkv, S, ps, q_out, kscr, vscr, direct, kv, m, max_batch);
   return cudaGetLastError();
 }
 
@@ -304,6 +340,8 @@ template <typename T, int HD, int G>
 __global__ void __launch_bounds__(128) k_attn_partial(int KV, const float* __restrict__ q, const T* kscr,
                                                       const T* vscr, bool inchunk_scratch, KVView kv, RowMeta m,
                                                       float* __restrict__ part, int nb_max, float scale_log2) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int DL = HD / 8;  // dims per lane
   __shared__ float sm_m[4][G], sm_l[4][G];
   __shared__ float sm_acc[4][G][HD];
@@ -441,6 +479,8 @@ __global__ void __launch_bounds__(128) k_attn_partial(int KV, const float* __res
 // One warp per (row, head): merge the row's key blocks in order.
 template <typename T, int HD>
 __global__ void k_attn_combine(int H, const float* __restrict__ part, int nb_max, KVView kv, RowMeta m, T* out) {
+  pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x, head = blockIdx.y * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (head >= H) return;
   const int lane = threadIdx.x & 31;
@@ -477,12 +517,12 @@ static cudaError_t attn_dispatch(int M, int KV, const float* q, const T* kscr, c
                                  RowMeta m, int nb, float* part, T* out, cudaStream_t st) {
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   dim3 grid(M * KV, nb);
-  k_attn_partial<T, HD, G><<<grid, 128, 0, st>>>(KV, q, kscr, vscr, sc, kv, m, part, nb, scale_log2);
+  launch(k_attn_partial<T, HD, G>, grid, 128, 0, st, KV, q, kscr, vscr, sc, kv, m, part, nb, scale_log2);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int H = KV * G;
   dim3 g2(M, (H + 3) / 4);
-  k_attn_combine<T, HD><<<g2, 128, 0, st>>>(H, part, nb, kv, m, out);
+  launch(k_attn_combine<T, HD>, g2, 128, 0, st, H, part, nb, kv, m, out);
   return cudaGetLastError();
 }
 
@@ -503,6 +543,8 @@ cudaError_t launch_attention(int M, int H, int KV, int hd, const float* q, const
 
 template <typename T>
 __global__ void k_kv_commit(int KV, int hd, const T* kscr, const T* vscr, KVView kv, RowMeta m) {
+  pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x;
   const int pos = m.pos[r], pend = m.pend[r], seq = m.seq[r];
   if (pos < pend - kv.cap) return;  // overwritten later in this chunk
@@ -523,13 +565,15 @@ __global__ void k_kv_commit(int KV, int hd, const T* kscr, const T* vscr, KVView
 template <typename T>
 cudaError_t launch_kv_commit(int M, int KV, int hd, const T* kscr, const T* vscr, KVView kv, RowMeta m,
                              cudaStream_t st) {
-  k_kv_commit<T><<<M, 128, 0, st>>>(KV, hd, kscr, vscr, kv, m);
+  launch(k_kv_commit<T>, M, 128, 0, st, KV, hd, kscr, vscr, kv, m);
   return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ SwiGLU
 template <typename T>
 __global__ void k_swiglu(int dff, const float* gu, int S, size_t ps, T* act) {
+  pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.y;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= dff) return;
@@ -546,12 +590,14 @@ __global__ void k_swiglu(int dff, const float* gu, int S, size_t ps, T* act) {
 template <typename T>
 cudaError_t launch_swiglu(int M, int dff, const float* gu, int S, size_t ps, T* act, cudaStream_t st) {
   dim3 grid((dff + 255) / 256, M);
-  k_swiglu<T><<<grid, 256, 0, st>>>(dff, gu, S, ps, act);
+  launch(k_swiglu<T>, grid, 256, 0, st, dff, gu, S, ps, act);
   return cudaGetLastError();
 }
 
 template <typename T>
 __global__ void k_gather_rows(int d, const int* rows, const T* src, T* dst) {
+  pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x;
   const T* s = src + (size_t)rows[r] * d;
   for (int i = threadIdx.x; i < d; i += blockDim.x) dst[(size_t)r * d + i] = s[i];
@@ -559,7 +605,7 @@ __global__ void k_gather_rows(int d, const int* rows, const T* src, T* dst) {
 
 template <typename T>
 cudaError_t launch_gather_rows(int R, int d, const int* rows, const T* src, T* dst, cudaStream_t st) {
-  k_gather_rows<T><<<R, 256, 0, st>>>(d, rows, src, dst);
+  launch(k_gather_rows<T>, R, 256, 0, st, d, rows, src, dst);
   return cudaGetLastError();
 }
 
@@ -569,6 +615,8 @@ cudaError_t launch_gather_rows(int R, int d, const int* rows, const T* src, T* d
 template <typename T>
 __global__ void __launch_bounds__(256) k_gemm_simt(int M, int N, int K, const T* __restrict__ X, int ldx,
                                                    const T* __restrict__ W, float* __restrict__ Y, int ldy) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float xs[16][64 + 4];
   __shared__ float ws[16][64 + 4];
   const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
@@ -612,7 +660,7 @@ template <typename T>
 cudaError_t launch_gemm_simt(int M, int N, int K, const T* X, int ldx, const T* W, float* Y, int ldy,
                              cudaStream_t st) {
   dim3 grid((N + 63) / 64, (M + 63) / 64);
-  k_gemm_simt<T><<<grid, 256, 0, st>>>(M, N, K, X, ldx, W, Y, ldy);
+  launch(k_gemm_simt<T>, grid, 256, 0, st, M, N, K, X, ldx, W, Y, ldy);
   return cudaGetLastError();
 }
 
@@ -620,6 +668,8 @@ cudaError_t launch_gemm_simt(int M, int N, int K, const T* X, int ldx, const T* 
 // One block per row; per-thread running (max, lowest index), then a fixed
 // tree.  max with lowest-index ties is order independent.
 __global__ void k_argmax(int V, const float* logits, int* out) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float sv[32];
   __shared__ int si[32];
   const float* row = logits + (size_t)blockIdx.x * V;
@@ -658,7 +708,7 @@ __global__ void k_argmax(int V, const float* logits, int* out) {
 }
 
 cudaError_t launch_argmax(int R, int V, const float* logits, int* out, cudaStream_t st) {
-  k_argmax<<<R, 1024, 0, st>>>(V, logits, out);
+  launch(k_argmax, R, 1024, 0, st, V, logits, out);
   return cudaGetLastError();
 }
 
@@ -666,6 +716,8 @@ cudaError_t launch_argmax(int R, int V, const float* logits, int* out, cudaStrea
 __global__ void k_spec_accept(int B, int gamma, int dstride, const int* seq_ids, int* seq_len, const int* drafts,
                               const int* vtok, int* pending, int* out, int* out_len, int max_new,
                               unsigned long long* accepted, int* all_done) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int n_unfinished;
   if (threadIdx.x == 0) n_unfinished = 0;
   __syncthreads();
@@ -690,15 +742,17 @@ __global__ void k_spec_accept(int B, int gamma, int dstride, const int* seq_ids,
 cudaError_t launch_spec_accept(int B, int gamma, int dstride, const int* seq_ids, int* seq_len, const int* drafts,
                                const int* vtok, int* pending, int* out, int* out_len, int max_new,
                                unsigned long long* accepted, int* all_done, cudaStream_t st) {
-  k_spec_accept<<<1, 256, 0, st>>>(B, gamma, dstride, seq_ids, seq_len, drafts, vtok, pending, out, out_len, max_new,
+  launch(k_spec_accept, 1, 256, 0, st, B, gamma, dstride, seq_ids, seq_len, drafts, vtok, pending, out, out_len, max_new,
                                    accepted, all_done);
   return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ instantiations
 #define DORY_INST(T)                                                                                              \
-  template cudaError_t launch_embed<T>(int, int, int, const int*, const T*, float*, T*, int*, cudaStream_t);      \
-  template cudaError_t launch_addnorm<T>(int, int, float*, const float*, int, size_t, int, T*, cudaStream_t);     \
+  template cudaError_t launch_embed<T>(int, int, int, const int*, const T*, float*, T*, float*, int*,            \
+                                       cudaStream_t);                                                             \
+  template cudaError_t launch_addnorm<T>(int, int, float*, const float*, int, size_t, int, T*, float*,            \
+                                         cudaStream_t);                                                           \
   template cudaError_t launch_reinject<T>(int, int, float*, const float*, int, const float*, bool, T*, float*,    \
                                           int, int, int, cudaStream_t);                                           \
   template cudaError_t launch_qkv_post<T>(int, int, int, int, const float*, int, size_t, float*, T*, T*, bool,    \

@@ -202,3 +202,32 @@ def test_state_errors(tiny, prompt):
         h.synchronize()
     assert e.value.status == 1
     h.synchronize()  # the error word was cleared
+
+
+@pytest.mark.parametrize("graphs,pdl", [(0, 0), (1, 0), (1, 1)])
+def test_graph_and_pdl_paths_agree(tiny_bf16, prompt, graphs, pdl):
+    """Eager launches, CUDA-graph replay and programmatic dependent launches
+    must produce the same bits."""
+    _, _, h = tiny_bf16
+
+    def run():
+        h.reset()
+        tok = torch.tensor(prompt[:40], dtype=torch.int32, device="cuda")
+        nxt = h.prefill([0], tok, [40], 2, dory.LAST_LOOP)
+        toks = [int(nxt[0])]
+        for _ in range(6):
+            nxt = h.decode_step([0], nxt, 2, dory.LAST_LOOP)
+            toks.append(int(nxt[0]))
+        return toks, h.read_state("s", 1).cpu()
+
+    h.set_option(dory.OPT_CUDA_GRAPHS, 0)
+    h.set_option(dory.OPT_PDL, 0)
+    ref = run()
+    h.set_option(dory.OPT_CUDA_GRAPHS, graphs)
+    h.set_option(dory.OPT_PDL, pdl)
+    got = run()
+    got2 = run()  # a second pass replays the captured graph
+    h.set_option(dory.OPT_PDL, 1)
+    h.set_option(dory.OPT_CUDA_GRAPHS, 1)
+    assert got[0] == ref[0] and got2[0] == ref[0]
+    assert torch.equal(got[1], ref[1]) and torch.equal(got2[1], ref[1])
