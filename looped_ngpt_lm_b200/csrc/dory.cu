@@ -127,6 +127,7 @@ struct dory_handle {
     cudaGraphExec_t exec;
   };
   std::vector<Graph> graphs_cache;
+  cudaStream_t cap_stream = nullptr;  // private stream used only to record graphs
 
   template <typename T>
   T* hop_t() const { return (T*)hop; }
@@ -580,10 +581,14 @@ dory_status decode_t(dory_handle* H, int batch, const int32_t* seq_ids, const in
       RET(decode_body<T>(H, batch, H->tokens, k, mode, H->c.max_seq, nullptr, H->next, st));
     } else {
       if (!g->exec) {
+        // record on a private stream (the caller's may be the legacy default
+        // stream, which cannot be captured); nothing runs while recording
+        if (!H->cap_stream) CK(cudaStreamCreateWithFlags(&H->cap_stream, cudaStreamNonBlocking));
+        cudaStream_t cs = H->cap_stream;
         cudaGraph_t graph = nullptr;
-        CK(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
-        dory_status r = decode_body<T>(H, batch, H->tokens, k, mode, H->c.max_seq, nullptr, H->next, st);
-        cudaError_t e = cudaStreamEndCapture(st, &graph);
+        CK(cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal));
+        dory_status r = decode_body<T>(H, batch, H->tokens, k, mode, H->c.max_seq, nullptr, H->next, cs);
+        cudaError_t e = cudaStreamEndCapture(cs, &graph);
         if (r != DORY_OK) {
           if (graph) cudaGraphDestroy(graph);
           return r;
@@ -732,6 +737,7 @@ dory_status dory_destroy(dory_handle* h) {
   for (auto e : h->ev_pool) cudaEventDestroy(e);
   for (auto& g : h->graphs_cache)
     if (g.exec) cudaGraphExecDestroy(g.exec);
+  if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
   delete h;
   return DORY_OK;
 }
