@@ -172,12 +172,21 @@ def main():
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--gemm-impl", dest="gemm_variant", type=int, default=2,
+                    help="--kernel gemm: 2 tcgen05 (default stages), 3 tcgen05 one sub-tile per stage, 1 SIMT")
     ap.add_argument("--prompt", type=int, default=2560)
     ap.add_argument("--k", type=int, default=2)
     ap.add_argument("--mode", default="last_loop", choices=["last_loop", "per_loop"])
     ap.add_argument("--no-aux", action="store_true", help="skip the k sweep, e2e and CPU baseline legs")
     ap.add_argument("--profile-steps", type=int, default=3)
+    ap.add_argument("--kernel", default=None, choices=["gemm"],
+                    help="time one kernel alone instead of the decode step (prints its own JSON line)")
+    ap.add_argument("--shape", default="qkv,o,gate_up,down,lm_head", help="GEMM shapes for --kernel gemm")
+    ap.add_argument("--m", type=int, default=1, help="token rows for --kernel gemm")
     args = ap.parse_args()
+    if args.kernel == "gemm":
+        gemm_probe(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
 
@@ -376,6 +385,46 @@ def main():
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def gemm_probe(args):
+    """Decode-projection GEMMs of the 4B shape at M token rows, each timed
+    alone with CUDA events over launches that rotate through enough weight
+    copies (> 4x L2) that every launch streams its weights from HBM."""
+    import torch
+    import looped_ngpt_lm_b200 as dory
+    import synth
+    s = synth.DORY_4B
+    shapes = {"qkv": (s.q_dim + 2 * s.kv_dim, s.d_model), "o": (s.d_model, s.q_dim),
+              "gate_up": (2 * s.d_ff, s.d_model), "down": (s.d_model, s.d_ff), "lm_head": (s.vocab, s.d_model)}
+    hbm = peaks()[0]
+    out = {}
+    for name in args.shape.split(","):
+        N, K = shapes[name]
+        wbytes = N * K * 2
+        copies = max(2, -(-512_000_000 // wbytes))
+        g = torch.Generator(device="cuda").manual_seed(0)
+        Ws = [(torch.randn((N, K), generator=g, device="cuda") * 0.02).to(torch.bfloat16) for _ in range(copies)]
+        X = torch.randn((args.m, K), generator=g, device="cuda").to(torch.bfloat16)
+        Y = torch.empty((8, args.m, N), dtype=torch.float32, device="cuda")
+        S = 1
+        for i in range(3):
+            S = dory.gemm_bf16_into(X, Ws[i % copies], Y, 1, True, args.gemm_variant)
+        torch.cuda.synchronize()
+        iters = max(30, 3 * copies)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for i in range(iters):
+            dory.gemm_bf16_into(X, Ws[i % copies], Y, 1, True, args.gemm_variant)
+        b.record()
+        torch.cuda.synchronize()
+        us = 1e3 * a.elapsed_time(b) / iters
+        by = wbytes + args.m * K * 2 + S * args.m * N * 4
+        out[name] = {"N": N, "K": K, "splits": S, "us": round(us, 2), "GBs": round(by / us / 1e3, 1),
+                     "frac_of_measured": round(by / us / 1e3 / hbm, 4)}
+        del Ws
+    print(json.dumps({"kernel": "gemm_tc", "impl": args.gemm_variant, "m": args.m, "results": out,
+                      "note": "back-to-back launches (no PDL overlap), weights cold in L2"}))
 
 
 def run_reference(args, shape, workload):

@@ -211,7 +211,8 @@ dory_status dory_read_kv(dory_handle* h, int32_t layer, int32_t slot, int32_t se
  * sum s = 0..*splits-1 is the product.  batch_hint selects the split the
  * decode path uses for that many sequences; invariant != 0 makes each row's
  * arithmetic independent of M.  impl: 0 auto, 1 SIMT kernel, 2 tcgen05 only
- * (DORY_ERR_CUDA if the shape is unsupported).  err_word (device int, may be
+ * (DORY_ERR_CUDA if the shape is unsupported), 3 tcgen05 with one 64-column
+ * sub-tile per pipeline stage (comparison variant).  err_word (device int, may be
  * NULL) receives DORY_ERR_TIMEOUT-class codes from bounded waits.  Queues work
  * on `stream`; no handle needed. */
 dory_status dory_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* X, const void* W, float* Y,

@@ -172,6 +172,18 @@ def gemm_bf16(X, W, batch_hint=1, invariant=True, impl=0, err=None, stream=None)
     return out, s.value
 
 
+def gemm_bf16_into(X, W, Y, batch_hint=1, invariant=True, impl=0, err=None, stream=None) -> int:
+    """dory_gemm_bf16 into a caller buffer Y (fp32, >= 8*M*N); returns the
+    number of split slices."""
+    M, K = X.shape
+    N = W.shape[0]
+    s = ctypes.c_int32()
+    _check(lib.dory_gemm_bf16(M, N, K, ctypes.c_void_p(X.data_ptr()), ctypes.c_void_p(W.data_ptr()),
+                              ctypes.c_void_p(Y.data_ptr()), batch_hint, int(invariant), impl, ctypes.byref(s),
+                              ctypes.c_void_p(_ptr(err)), _stream(stream)))
+    return s.value
+
+
 def workspace_size(cfg: Config, alloc_mode=LAST_LOOP) -> int:
     n = ctypes.c_size_t()
     _check(lib.dory_workspace_size(ctypes.byref(cfg), MODES[alloc_mode], ctypes.byref(n)))

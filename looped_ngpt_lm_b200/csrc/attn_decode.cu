@@ -20,6 +20,7 @@
 #include <float.h>
 
 #include "attn_decode.cuh"
+#include "gemm_tc.cuh"
 
 namespace dory {
 
@@ -44,6 +45,18 @@ __device__ __forceinline__ void load_raw(const T* p, RowBuf<T, DL>& b) {
     static_assert(BYTES == 8, "row slice must be 8 or a multiple of 16 bytes");
     *reinterpret_cast<uint2*>(b.v) = *reinterpret_cast<const uint2*>(p);
   }
+}
+
+// In-order sum of a value's S split-K slices (independent, predicated loads).
+__device__ __forceinline__ float sum_splits(const float* p, int S, size_t ps) {
+  float v[kMaxSplitK];
+#pragma unroll
+  for (int s = 0; s < kMaxSplitK; ++s) v[s] = s < S ? __ldcg(p + s * ps) : 0.f;
+  float a = 0.f;
+#pragma unroll
+  for (int s = 0; s < kMaxSplitK; ++s)
+    if (s < S) a += v[s];
+  return a;
 }
 
 template <typename T, int HD, int G>
@@ -80,12 +93,14 @@ __global__ void __launch_bounds__(256) k_attn_decode(int KV, const float* __rest
   const int H = KV * G, qd = H * HD, kvd = KV * HD, ld = qd + 2 * kvd;
   const int tid = threadIdx.x;
 
-  for (int idx = tid; idx < G * HD; idx += blockDim.x) {
-    const int h = idx / HD, d = idx % HD;
-    const float* src = qkv + (size_t)r * ld + (g * G + h) * HD + d;
-    float a = 0.f;
-    for (int s = 0; s < S; ++s) a += src[s * ps];
-    q_sm[h][d] = a * scale_log2;
+  constexpr int QPT = (G * HD + 255) / 256;  // q values per thread
+#pragma unroll
+  for (int c = 0; c < QPT; ++c) {
+    const int idx = tid + c * 256;
+    if (idx < G * HD) {
+      const int h = idx / HD, d = idx % HD;
+      q_sm[h][d] = sum_splits(qkv + (size_t)r * ld + (g * G + h) * HD + d, S, ps) * scale_log2;
+    }
   }
   T* Kc = (T*)kv.K + ((size_t)seq * KV + g) * kv.cap * HD;
   T* Vc = (T*)kv.V + ((size_t)seq * KV + g) * kv.cap * HD;
@@ -94,9 +109,7 @@ __global__ void __launch_bounds__(256) k_attn_decode(int KV, const float* __rest
     for (int idx = tid; idx < 2 * HD; idx += blockDim.x) {
       const int d = idx % HD;
       const bool is_v = idx >= HD;
-      const float* src = qkv + (size_t)r * ld + qd + (is_v ? kvd : 0) + g * HD + d;
-      float a = 0.f;
-      for (int s = 0; s < S; ++s) a += src[s * ps];
+      const float a = sum_splits(qkv + (size_t)r * ld + qd + (is_v ? kvd : 0) + g * HD + d, S, ps);
       (is_v ? Vc : Kc)[slot + d] = from_f<T>(a);
     }
   }
@@ -132,13 +145,8 @@ __global__ void __launch_bounds__(256) k_attn_decode(int KV, const float* __rest
         const float* src = qkv + (size_t)(base + (j - p0)) * ld + qd + g * HD + dl * DL;
 #pragma unroll
         for (int e = 0; e < DL; ++e) {
-          float a = 0.f, b = 0.f;
-          for (int s = 0; s < S; ++s) {
-            a += src[s * ps + e];
-            b += src[s * ps + kvd + e];
-          }
-          kr[it].v[e] = from_f<T>(a);
-          vr[it].v[e] = from_f<T>(b);
+          kr[it].v[e] = from_f<T>(sum_splits(src + e, S, ps));
+          vr[it].v[e] = from_f<T>(sum_splits(src + kvd + e, S, ps));
         }
       }
     } else {
@@ -224,21 +232,63 @@ __global__ void __launch_bounds__(256) k_attn_decode(int KV, const float* __rest
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  for (int idx = tid; idx < G * HD; idx += blockDim.x) {
-    const int h = idx / HD, d = idx % HD;
-    const float* pr = part + ((size_t)r * H + g * G + h) * nb_max * (HD + 2);
-    float M = -FLT_MAX, L = 0.f, a = 0.f;
-    for (int b = 0; b < nb_row; ++b) {
-      const float* pb = pr + b * (HD + 2);
-      const float mb = __ldcg(pb), lb = __ldcg(pb + 1), ab_ = __ldcg(pb + 2 + d);
-      const float mn = fmaxf(M, mb);
-      const float ca = M == -FLT_MAX ? 0.f : exp2f(M - mn);
-      const float cb = exp2f(mb - mn);
-      L = L * ca + lb * cb;
-      a = a * ca + ab_ * cb;
-      M = mn;
+  // merge: (1) all threads fetch every block's (m, l) into shared memory;
+  // (2) per head, the max M and 1/L = 1 / sum_b l_b 2^(m_b - M); (3) block
+  // weights 2^(m_b - M); (4) every (head, dim) output sums its blocks with
+  // independent loads.  Block order fixes the summation order.
+  float* sm_mb = &sm_acc[0][0][0];  // reused: [G][nb_row] m, then weights
+  float* sm_lb = sm_mb + G * nb_row;  // [G][nb_row] l
+  float* sm_hd = sm_lb + G * nb_row;  // [G] M, then [G] 1/L
+  const size_t hstride = (size_t)nb_max * (HD + 2);
+  const float* pr0 = part + ((size_t)r * H + g * G) * hstride;
+  for (int idx = tid; idx < G * nb_row; idx += blockDim.x) {
+    const int h = idx / nb_row, b = idx % nb_row;
+    sm_mb[idx] = __ldcg(pr0 + h * hstride + b * (HD + 2));
+    sm_lb[idx] = __ldcg(pr0 + h * hstride + b * (HD + 2) + 1);
+  }
+  __syncthreads();
+  if (tid < G) {
+    float M = -FLT_MAX;
+    for (int b = 0; b < nb_row; ++b) M = fmaxf(M, sm_mb[tid * nb_row + b]);
+    float L = 0.f;
+    for (int b = 0; b < nb_row; ++b) L += sm_lb[tid * nb_row + b] * exp2f(sm_mb[tid * nb_row + b] - M);
+    sm_hd[tid] = M;
+    sm_hd[G + tid] = 1.f / L;
+  }
+  __syncthreads();
+  for (int idx = tid; idx < G * nb_row; idx += blockDim.x) sm_mb[idx] = exp2f(sm_mb[idx] - sm_hd[idx / nb_row]);
+  __syncthreads();
+  const float* wts = sm_mb;
+  constexpr int OPT = (G * HD + 255) / 256;  // outputs per thread
+  constexpr int BB = 8;                      // blocks per batch of loads
+  float o[OPT];
+#pragma unroll
+  for (int c = 0; c < OPT; ++c) o[c] = 0.f;
+  for (int b0 = 0; b0 < nb_row; b0 += BB) {
+    float v[OPT][BB];
+#pragma unroll
+    for (int c = 0; c < OPT; ++c) {
+      const int idx = tid + c * 256;
+      const int h = idx / HD, d = idx % HD;
+#pragma unroll
+      for (int j = 0; j < BB; ++j)
+        v[c][j] = (idx < G * HD && b0 + j < nb_row) ? __ldcg(pr0 + h * hstride + (b0 + j) * (HD + 2) + 2 + d) : 0.f;
     }
-    out[(size_t)r * qd + (g * G + h) * HD + d] = from_f<T>(a / L);
+#pragma unroll
+    for (int c = 0; c < OPT; ++c) {
+      const int h = min((tid + c * 256) / HD, G - 1);
+#pragma unroll
+      for (int j = 0; j < BB; ++j)
+        if (b0 + j < nb_row) o[c] += v[c][j] * wts[h * nb_row + b0 + j];
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < OPT; ++c) {
+    const int idx = tid + c * 256;
+    if (idx < G * HD) {
+      const int h = idx / HD, d = idx % HD;
+      out[(size_t)r * qd + (g * G + h) * HD + d] = from_f<T>(o[c] * sm_hd[G + h]);
+    }
   }
   if (tid == 0) counters[r * KV + g] = 0u;
 }
@@ -248,7 +298,8 @@ cudaError_t dispatch(int M, int KV, const float* qkv, int S, size_t ps, KVView k
                      float* part, int nb_cap, unsigned* counters, T* out, cudaStream_t st) {
   const int span = kv.window > 0 ? min(max_ctx, kv.window) : max_ctx;
   const int nb = (span + DEC_BK - 1) / DEC_BK + 1;
-  if (nb > nb_cap) return cudaErrorInvalidValue;
+  // the merge keeps 2 * G * nb + 2 * G floats in the 8 * G * HD float buffer
+  if (nb > nb_cap || 2 * nb + 2 > 8 * HD) return cudaErrorInvalidValue;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   return launch(k_attn_decode<T, HD, G>, dim3(M * KV, nb), dim3(256), 0, st, KV, qkv, S, ps, kv, m, part, nb,
                 counters, out, scale_log2);

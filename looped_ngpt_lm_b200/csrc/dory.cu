@@ -109,6 +109,7 @@ struct dory_handle {
   int *drafts = nullptr, *pending = nullptr, *vtok = nullptr, *out_len = nullptr, *all_done = nullptr;
   unsigned long long* accepted = nullptr;
   unsigned* attn_counters = nullptr;  // [M_max * n_kv], zero between launches
+  unsigned* tile_counters = nullptr;  // [kTileCounters], zero between launches
   int nb_cap = 0;                     // key blocks per row the partial buffer holds
 
   // host state
@@ -230,6 +231,7 @@ size_t layout(dory_handle* h) {
   h->part_gu = cv.take<float>(sizeof(float) * kMaxSplitK * h->part_rows * 2 * c.d_ff);
   h->attn_part = cv.take<float>(sizeof(float) * (size_t)M * c.n_heads * h->nb_cap * (c.head_dim + 2));
   h->attn_counters = cv.take<unsigned>(sizeof(unsigned) * (size_t)M * c.n_kv_heads);
+  h->tile_counters = cv.take<unsigned>(sizeof(unsigned) * kTileCounters);
   h->logits = cv.take<float>(sizeof(float) * (size_t)h->head_max * c.vocab * kMaxSplitK);
   const int gc = c.gamma_max + 1;
   h->stash_x = cv.take<float>(sizeof(float) * (size_t)c.max_batch * gc * d);
@@ -321,7 +323,7 @@ dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, cons
       int S = 1;
       size_t ps = 0;
       cudaError_t e = launch_gemm_tc(M, N, K, (const bf16*)X, ldx, (const bf16*)W, Y, ldy, part_rows,
-                                     H->err, f.batch, f.invariant, &S, &ps, f.st);
+                                     H->err, f.batch, f.invariant, &S, &ps, f.st, 0, H->tile_counters);
       if (e == cudaSuccess) {
         *S_out = S;
         *ps_out = ps;
@@ -749,6 +751,7 @@ dory_status dory_reset(dory_handle* h, int32_t seq, dory_stream stream) {
     CK(cudaMemsetAsync(h->seq_len, 0, sizeof(int) * h->c.max_batch, st));
     CK(cudaMemsetAsync(h->err, 0, sizeof(int) * 4, st));
     CK(cudaMemsetAsync(h->attn_counters, 0, sizeof(unsigned) * (size_t)h->M_max * h->c.n_kv_heads, st));
+    CK(cudaMemsetAsync(h->tile_counters, 0, sizeof(unsigned) * kTileCounters, st));
     std::fill(h->len.begin(), h->len.end(), 0);
     std::fill(h->mode.begin(), h->mode.end(), -1);
     return DORY_OK;
@@ -887,12 +890,12 @@ dory_status dory_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* X, const
     int S = 1;
     size_t ps = 0;
     cudaError_t e = launch_gemm_tc(M, N, K, (const bf16*)X, K, (const bf16*)W, Y, N, (size_t)M, err_word,
-                                   batch_hint < 1 ? 1 : batch_hint, invariant != 0, &S, &ps, st);
+                                   batch_hint < 1 ? 1 : batch_hint, invariant != 0, &S, &ps, st, impl == 3 ? 1 : 0);
     if (e == cudaSuccess) {
       *splits = S;
       return DORY_OK;
     }
-    if (e != cudaErrorNotSupported || impl == 2) return fail(DORY_ERR_CUDA, "tcgen05 GEMM: %s", cudaGetErrorString(e));
+    if (e != cudaErrorNotSupported || impl >= 2) return fail(DORY_ERR_CUDA, "tcgen05 GEMM: %s", cudaGetErrorString(e));
   }
   CK(launch_gemm_simt<bf16>(M, N, K, (const bf16*)X, K, (const bf16*)W, Y, N, st));
   return DORY_OK;

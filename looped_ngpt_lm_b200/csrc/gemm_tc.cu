@@ -150,35 +150,42 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-template <int NG, int GN>
+// KSUB 64-column sub-tiles per pipeline stage: a stage reads KSUB*128
+// contiguous bytes of every weight row.
+template <int NG, int GN, int KSUB>
 struct Tile {
   static constexpr int MT = NG * GN;                   // tokens per unit
-  static constexpr int A_BYTES = BM * BK * 2;          // 16 KB
-  static constexpr int B_BYTES = MT * BK * 2;
+  static constexpr int A_SUB = BM * BK * 2;            // 16 KB per sub-tile
+  static constexpr int B_SUB = MT * BK * 2;
+  static constexpr int A_BYTES = KSUB * A_SUB;
+  static constexpr int B_BYTES = KSUB * B_SUB;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (200 * 1024) / STAGE > 12 ? 12 : (200 * 1024) / STAGE;
+  static constexpr int STAGES = (216 * 1024) / STAGE > 12 ? 12 : (216 * 1024) / STAGE;
   static constexpr int ACC = MT;                       // TMEM columns per accumulator
   static constexpr int TMEM_COLS = 2 * ACC <= 32 ? 32 : 2 * ACC <= 64 ? 64 : 2 * ACC <= 128 ? 128 : 2 * ACC <= 256 ? 256 : 512;
   static constexpr int SMEM = STAGES * STAGE + 1024 /*align*/ + 256 /*barriers*/;
 };
 
+// Units are (n tile, m tile, split).  Split boundaries are placed on groups
+// of `gran` stages (KBg groups in all) so they fall on the same K columns
+// whatever the stage width: a row's split-K grouping never depends on M.
 struct UnitMap {
-  int n_tiles, m_tiles, S, KB, units;
+  int n_tiles, m_tiles, S, KBg, gran, units;
   __device__ __forceinline__ void decode(int u, int& nt, int& mt, int& s, int& kb0, int& kb1) const {
     s = u % S;
     int t = u / S;
     mt = t % m_tiles;
     nt = t / m_tiles;
-    kb0 = s * KB / S;
-    kb1 = (s + 1) * KB / S;
+    kb0 = (s * KBg / S) * gran;
+    kb1 = ((s + 1) * KBg / S) * gran;
   }
 };
 
-template <int NG, int GN>
+template <int NG, int GN, int KSUB>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, float* Y, int ldy,
-              size_t part_stride, int M, UnitMap um, int* err) {
-  using TL = Tile<NG, GN>;
+              size_t part_stride, int M, UnitMap um, unsigned* tile_counters, int* err) {
+  using TL = Tile<NG, GN, KSUB>;
   constexpr int STAGES = TL::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -189,6 +196,7 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* mma_done = tempty + 2;
   uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  volatile int* last_flag = (volatile int*)(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -241,7 +249,9 @@ __global__ void __launch_bounds__(192, 1)
       while (npre < STAGES && u < um.units) {
         uint8_t* sa = smem + npre * TL::STAGE;
         mbar_expect_tx(&full[npre], TL::STAGE);
-        tma_load_2d(sa, &mapA, &full[npre], kb * BK, nt * BM, pol_w);
+#pragma unroll
+        for (int q = 0; q < KSUB; ++q)
+          tma_load_2d(sa + q * TL::A_SUB, &mapA, &full[npre], (kb * KSUB + q) * BK, nt * BM, pol_w);
         pre_kb[npre] = kb;
         pre_mt[npre] = mt;
         ++npre;
@@ -249,7 +259,10 @@ __global__ void __launch_bounds__(192, 1)
       }
       pdl_wait();
       for (int i = 0; i < npre; ++i)
-        tma_load_2d(smem + i * TL::STAGE + TL::A_BYTES, &mapB, &full[i], pre_kb[i] * BK, pre_mt[i] * TL::MT, pol_x);
+#pragma unroll
+        for (int q = 0; q < KSUB; ++q)
+          tma_load_2d(smem + i * TL::STAGE + TL::A_BYTES + q * TL::B_SUB, &mapB, &full[i], (pre_kb[i] * KSUB + q) * BK,
+                      pre_mt[i] * TL::MT, pol_x);
       int stage = npre % STAGES, issued = npre;
       uint32_t phase = npre == STAGES ? 1u : 0u;
       while (u < um.units) {
@@ -257,8 +270,12 @@ __global__ void __launch_bounds__(192, 1)
         ++issued;
         uint8_t* sa = smem + stage * TL::STAGE;
         mbar_expect_tx(&full[stage], TL::STAGE);
-        tma_load_2d(sa, &mapA, &full[stage], kb * BK, nt * BM, pol_w);
-        tma_load_2d(sa + TL::A_BYTES, &mapB, &full[stage], kb * BK, mt * TL::MT, pol_x);
+#pragma unroll
+        for (int q = 0; q < KSUB; ++q) {
+          tma_load_2d(sa + q * TL::A_SUB, &mapA, &full[stage], (kb * KSUB + q) * BK, nt * BM, pol_w);
+          tma_load_2d(sa + TL::A_BYTES + q * TL::B_SUB, &mapB, &full[stage], (kb * KSUB + q) * BK, mt * TL::MT,
+                      pol_x);
+        }
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1;
@@ -300,16 +317,19 @@ __global__ void __launch_bounds__(192, 1)
           }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * TL::STAGE);
-          const uint64_t adesc = sw128_desc(sa);
-          const uint64_t bdesc = sw128_desc(sa + TL::A_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
+          for (int q = 0; q < KSUB; ++q) {
+            const uint64_t adesc = sw128_desc(sa + q * TL::A_SUB);
+            const uint64_t bdesc = sw128_desc(sa + TL::A_BYTES + q * TL::B_SUB);
 #pragma unroll
-            for (int g = 0; g < NG; ++g) {
-              // +32 bytes per K-step of 16 inside the swizzled row; group g
-              // starts GN rows (GN * 128 bytes) further into the B tile
-              umma(d0 + g * GN, adesc + 2 * kk, bdesc + 2 * kk + (uint64_t)(g * GN * 128 >> 4), IDESC,
-                   (kb > kb0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BK / 16; ++kk) {
+#pragma unroll
+              for (int g = 0; g < NG; ++g) {
+                // +32 bytes per K-step of 16 inside the swizzled row; group g
+                // starts GN rows (GN * 128 bytes) further into the B tile
+                umma(d0 + g * GN, adesc + 2 * kk, bdesc + 2 * kk + (uint64_t)(g * GN * 128 >> 4), IDESC,
+                     (kb > kb0 || q > 0 || kk > 0) ? 1u : 0u);
+              }
             }
           }
           umma_commit(&empty[stage]);
@@ -357,6 +377,36 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (um.S > 1 && tile_counters) {
+        // split-K: the last split of this tile to finish adds all slices in
+        // order s = 0..S-1 and leaves the sum in slice 0
+        __threadfence();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (warp == 2 && lane == 0) {
+          const unsigned prev = atomicAdd(&tile_counters[nt * um.m_tiles + mt], 1u);
+          *last_flag = prev == (unsigned)(um.S - 1);
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (*last_flag) {
+          __threadfence();
+          const int m_end = min(M, m_base + TL::MT);
+          for (int m0 = m_base; m0 < m_end; m0 += 4) {
+            float acc4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int q = 0; q < kMaxSplitK; ++q) {
+              if (q < um.S) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                  if (m0 + j < m_end) acc4[j] += __ldcg(Y + (size_t)q * part_stride + (size_t)(m0 + j) * ldy + n);
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              if (m0 + j < m_end) Y[(size_t)(m0 + j) * ldy + n] = acc4[j];
+          }
+          if (warp == 2 && lane == 0) tile_counters[nt * um.m_tiles + mt] = 0u;
+        }
+      }
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
@@ -440,40 +490,41 @@ int sm_count() {
   return n;
 }
 
-template <int NG, int GN>
+template <int NG, int GN, int KSUB>
 cudaError_t run(const CUtensorMap& ma, const bf16* X, int ldx, int M, int K, float* Y, int ldy, size_t ps,
-                UnitMap um, int* err, cudaStream_t st) {
-  using TL = Tile<NG, GN>;
+                UnitMap um, unsigned* tile_counters, int* err, cudaStream_t st) {
+  using TL = Tile<NG, GN, KSUB>;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<NG, GN>, cudaFuncAttributeMaxDynamicSharedMemorySize, TL::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<NG, GN, KSUB>, cudaFuncAttributeMaxDynamicSharedMemorySize, TL::SMEM);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   CUtensorMap mb;
   if (!make_map(&mb, X, M, K, ldx, TL::MT)) return cudaErrorInvalidValue;
   int grid = um.units < sm_count() ? um.units : sm_count();
-  return launch(k_gemm_tc<NG, GN>, dim3(grid), dim3(192), TL::SMEM, st, ma, mb, Y, ldy, ps, M, um, err);
+  return launch(k_gemm_tc<NG, GN, KSUB>, dim3(grid), dim3(192), TL::SMEM, st, ma, mb, Y, ldy, ps, M, um,
+                tile_counters, err);
 }
 
 // Split factor for the decode tiles: chosen from (N, K, batch) only, never
-// from M, so a row's accumulation grouping is the same at every M.  Model:
-// each round of units runs at the slower of HBM (all units of the round
-// share it) and one SM's own streaming rate; partial sums cost HBM traffic.
-int choose_split(int N, int K, int batch) {
-  const double hbm = 6.5e12, sm_bw = 1.2e11;
-  const int tiles = N / BM, KB = K / BK, sms = sm_count();
+// from M, so a row's accumulation grouping is the same at every M.  Units are
+// dealt round-robin to one CTA per SM; the model charges the larger of the
+// whole GEMM at HBM speed and the busiest CTA at one SM's streaming rate,
+// plus the partial sums' HBM traffic.
+int choose_split(int N, int K, int batch, int kstages) {
+  const double hbm = 6.5e12, sm_bw = 5.5e10;
+  const int tiles = N / BM, sms = sm_count();
   const double rows = 5.0 * batch;  // decode / verify rows this batch size produces
+  const double stage_bytes = (double)BM * (K / kstages) * 2;
   int best = 1;
   double best_t = 1e30;
-  for (int S = 1; S <= kMaxSplitK && S <= KB; ++S) {
+  for (int S = 1; S <= kMaxSplitK && S <= kstages; ++S) {
     const int U = tiles * S;
-    const double ubytes = (double)BM * ((KB + S - 1) / S) * BK * 2;
-    double t = 0;
-    for (int left = U; left > 0; left -= sms) {
-      const int in_round = left < sms ? left : sms;
-      t += fmax(in_round * ubytes / hbm, ubytes / sm_bw);
-    }
+    // busiest CTA: ceil(U / sms) units, the largest of which has ceil(KB / S) stages
+    const int per_cta = (U + sms - 1) / sms;
+    const double busiest = per_cta * (double)((kstages + S - 1) / S) * stage_bytes;
+    double t = fmax(tiles * (double)kstages * stage_bytes / hbm, busiest / sm_bw);
     t += S * rows * N * 8.0 / hbm;
     if (t < best_t * 0.98) {
       best_t = t;
@@ -487,7 +538,7 @@ int choose_split(int N, int K, int batch) {
 
 cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf16* W, float* Y, int ldy,
                            size_t part_rows, int* err, int batch, bool invariant, int* S_out, size_t* ps_out,
-                           cudaStream_t st) {
+                           cudaStream_t st, int variant, unsigned* tile_counters) {
   *S_out = 1;
   *ps_out = 0;
   if (M <= 0 || N % BM || K % BK || ldx % 8 || (size_t)M > part_rows || ((uintptr_t)X & 15) || ((uintptr_t)W & 15))
@@ -496,30 +547,44 @@ cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf
   if (!weight_map(&ma, W, N, K)) return cudaErrorNotSupported;
   UnitMap um;
   um.n_tiles = N / BM;
-  um.KB = K / BK;
   if (invariant || M <= 128) {
-    // decode / verify: 16-token MMA groups, split chosen from (N, K, batch)
-    const int S = choose_split(N, K, batch);
+    // decode / verify: 16-token MMA groups, split chosen from (N, K, batch).
+    // Stages span 4 sub-tiles (512 contiguous bytes per weight row) when K
+    // allows; variant 1 forces one sub-tile per stage.
+    int NG = M <= 16 ? 1 : M <= 32 ? 2 : M <= 64 ? 4 : 8;
+    const bool g256 = K % (4 * BK) == 0;  // split on 256-column groups
+    const int ksub = (variant == 1 || !g256) ? 1 : (NG >= 8 ? 1 : (NG >= 2 ? 2 : 4));
+    um.KBg = g256 ? K / (4 * BK) : K / BK;
+    um.gran = g256 ? 4 / ksub : 1;
+    const int S = choose_split(N, K, batch, um.KBg);
+    if (S > um.KBg) return cudaErrorNotSupported;
     const size_t ps = part_rows * (size_t)ldy;
     um.S = S;
-    int NG = M <= 16 ? 1 : M <= 32 ? 2 : M <= 64 ? 4 : 8;
     const int MT = 16 * NG;
     um.m_tiles = (M + MT - 1) / MT;
     um.units = um.n_tiles * um.m_tiles * S;
-    *S_out = S;
-    *ps_out = ps;
+    unsigned* tc = (S > 1 && tile_counters && um.n_tiles * um.m_tiles <= kTileCounters) ? tile_counters : nullptr;
+    *S_out = tc ? 1 : S;  // reduced in the kernel: one slice for the consumer
+    *ps_out = tc ? 0 : ps;
+    if (ksub == 4) return run<1, 16, 4>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st);
+    if (ksub == 2) {
+      if (NG == 2) return run<2, 16, 2>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st);
+      return run<4, 16, 2>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st);
+    }
     switch (NG) {
-      case 1: return run<1, 16>(ma, X, ldx, M, K, Y, ldy, ps, um, err, st);
-      case 2: return run<2, 16>(ma, X, ldx, M, K, Y, ldy, ps, um, err, st);
-      case 4: return run<4, 16>(ma, X, ldx, M, K, Y, ldy, ps, um, err, st);
-      default: return run<8, 16>(ma, X, ldx, M, K, Y, ldy, ps, um, err, st);
+      case 1: return run<1, 16, 1>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st);
+      case 2: return run<2, 16, 1>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st);
+      case 4: return run<4, 16, 1>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st);
+      default: return run<8, 16, 1>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st);
     }
   }
   // prefill: 128 x 256 tiles, no split
+  um.KBg = K / BK;
+  um.gran = 1;
   um.S = 1;
   um.m_tiles = (M + 255) / 256;
   um.units = um.n_tiles * um.m_tiles;
-  return run<1, 256>(ma, X, ldx, M, K, Y, ldy, 0, um, err, st);
+  return run<1, 256, 1>(ma, X, ldx, M, K, Y, ldy, 0, um, nullptr, err, st);
 }
 
 }  // namespace dory

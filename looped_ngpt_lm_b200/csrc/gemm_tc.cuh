@@ -8,6 +8,9 @@ namespace dory {
 // Largest split-K factor the GEMM may choose; callers size partial buffers
 // for kMaxSplitK slices.
 constexpr int kMaxSplitK = 8;
+// Device counters a split GEMM needs (one per output tile; zero between
+// launches, and left zero by every launch).
+constexpr int kTileCounters = 4096;
 
 // Y = X . W^T for X [M, K] (row stride ldx) and W [N, K], both bf16, fp32
 // accumulation.  Writes S partial products to Y + s * (*part_stride)
@@ -16,9 +19,12 @@ constexpr int kMaxSplitK = 8;
 // (N, K, batch) only, so each row's result is bit-identical for every M;
 // otherwise 128 x 256 tiles without split.  part_rows: rows available per
 // slice (>= M).  Returns cudaErrorNotSupported for shapes the kernel does not
-// handle (N % 128, K % 64, unaligned pointers).
+// handle (N % 128, K % 64, unaligned pointers).  variant 1 forces one
+// 64-column sub-tile per pipeline stage (for comparisons).  With
+// tile_counters (kTileCounters zeros), the last split of each output tile
+// adds the slices in order s = 0..S-1 inside the kernel and *S is 1.
 cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf16* W, float* Y, int ldy,
                            size_t part_rows, int* err, int batch, bool invariant, int* S, size_t* part_stride,
-                           cudaStream_t st);
+                           cudaStream_t st, int variant = 0, unsigned* tile_counters = nullptr);
 
 }  // namespace dory

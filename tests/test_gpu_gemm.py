@@ -56,3 +56,13 @@ def test_rows_bit_identical_across_M(N, K, batch):
         full, s2 = dory.gemm_bf16(Xm, W, batch_hint=batch, invariant=True, impl=2)
         assert s1 == s2
         assert torch.equal(full[at], alone[0]), (M, at)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 2560, 10240), (3, 20480, 2560), (40, 3584, 2560)])
+def test_stage_width_does_not_change_bits(M, N, K):
+    """One 64-column sub-tile per stage (impl 3) and the default wide stages
+    (impl 2) accumulate the same K-steps in the same order."""
+    X, W = operands(M, N, K, 3)
+    a, s1 = dory.gemm_bf16(X, W, batch_hint=1, invariant=True, impl=2)
+    b, s2 = dory.gemm_bf16(X, W, batch_hint=1, invariant=True, impl=3)
+    assert s1 == s2 and torch.equal(a, b)
