@@ -323,7 +323,7 @@ dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, cons
       int S = 1;
       size_t ps = 0;
       cudaError_t e = launch_gemm_tc(M, N, K, (const bf16*)X, ldx, (const bf16*)W, Y, ldy, part_rows,
-                                     H->err, f.batch, f.invariant, &S, &ps, f.st, 0, H->tile_counters);
+                                     H->err, f.batch, f.invariant, &S, &ps, f.st, 0, nullptr);
       if (e == cudaSuccess) {
         *S_out = S;
         *ps_out = ps;

@@ -33,6 +33,11 @@ namespace {
 constexpr int BK = 64;            // k elements per stage (128 bytes of bf16: one swizzle row)
 constexpr int BM = 128;           // weight rows per tile (MMA M)
 constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at 2 GHz
+// Decode tiles: 64-column sub-tiles per stage and the shared-memory budget of
+// the stage ring (a budget near 100 KB lets the next GEMM's CTA co-reside and
+// prefetch its weights while this one drains).
+constexpr int kDecodeKsub = 4;
+constexpr int kDecodeBudget = 216 * 1024;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -152,7 +157,7 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 
 // KSUB 64-column sub-tiles per pipeline stage: a stage reads KSUB*128
 // contiguous bytes of every weight row.
-template <int NG, int GN, int KSUB>
+template <int NG, int GN, int KSUB, int BUDGET = 216 * 1024>
 struct Tile {
   static constexpr int MT = NG * GN;                   // tokens per unit
   static constexpr int A_SUB = BM * BK * 2;            // 16 KB per sub-tile
@@ -160,7 +165,7 @@ struct Tile {
   static constexpr int A_BYTES = KSUB * A_SUB;
   static constexpr int B_BYTES = KSUB * B_SUB;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (216 * 1024) / STAGE > 12 ? 12 : (216 * 1024) / STAGE;
+  static constexpr int STAGES = BUDGET / STAGE > 12 ? 12 : (BUDGET / STAGE < 1 ? 1 : BUDGET / STAGE);
   static constexpr int ACC = MT;                       // TMEM columns per accumulator
   static constexpr int TMEM_COLS = 2 * ACC <= 32 ? 32 : 2 * ACC <= 64 ? 64 : 2 * ACC <= 128 ? 128 : 2 * ACC <= 256 ? 256 : 512;
   static constexpr int SMEM = STAGES * STAGE + 1024 /*align*/ + 256 /*barriers*/;
@@ -181,11 +186,11 @@ struct UnitMap {
   }
 };
 
-template <int NG, int GN, int KSUB>
+template <int NG, int GN, int KSUB, int BUDGET>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, float* Y, int ldy,
               size_t part_stride, int M, UnitMap um, unsigned* tile_counters, int* err) {
-  using TL = Tile<NG, GN, KSUB>;
+  using TL = Tile<NG, GN, KSUB, BUDGET>;
   constexpr int STAGES = TL::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -490,20 +495,21 @@ int sm_count() {
   return n;
 }
 
-template <int NG, int GN, int KSUB>
+template <int NG, int GN, int KSUB, int BUDGET = kDecodeBudget>
 cudaError_t run(const CUtensorMap& ma, const bf16* X, int ldx, int M, int K, float* Y, int ldy, size_t ps,
                 UnitMap um, unsigned* tile_counters, int* err, cudaStream_t st) {
-  using TL = Tile<NG, GN, KSUB>;
+  using TL = Tile<NG, GN, KSUB, BUDGET>;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<NG, GN, KSUB>, cudaFuncAttributeMaxDynamicSharedMemorySize, TL::SMEM);
+    cudaError_t e =
+        cudaFuncSetAttribute(k_gemm_tc<NG, GN, KSUB, BUDGET>, cudaFuncAttributeMaxDynamicSharedMemorySize, TL::SMEM);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   CUtensorMap mb;
   if (!make_map(&mb, X, M, K, ldx, TL::MT)) return cudaErrorInvalidValue;
   int grid = um.units < sm_count() ? um.units : sm_count();
-  return launch(k_gemm_tc<NG, GN, KSUB>, dim3(grid), dim3(192), TL::SMEM, st, ma, mb, Y, ldy, ps, M, um,
+  return launch(k_gemm_tc<NG, GN, KSUB, BUDGET>, dim3(grid), dim3(192), TL::SMEM, st, ma, mb, Y, ldy, ps, M, um,
                 tile_counters, err);
 }
 
@@ -553,7 +559,7 @@ cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf
     // allows; variant 1 forces one sub-tile per stage.
     int NG = M <= 16 ? 1 : M <= 32 ? 2 : M <= 64 ? 4 : 8;
     const bool g256 = K % (4 * BK) == 0;  // split on 256-column groups
-    const int ksub = (variant == 1 || !g256) ? 1 : (NG >= 8 ? 1 : (NG >= 2 ? 2 : 4));
+    const int ksub = (variant == 1 || !g256) ? 1 : (NG >= 8 ? 1 : (NG >= 2 ? 2 : kDecodeKsub));
     um.KBg = g256 ? K / (4 * BK) : K / BK;
     um.gran = g256 ? 4 / ksub : 1;
     const int S = choose_split(N, K, batch, um.KBg);
@@ -566,17 +572,22 @@ cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf
     unsigned* tc = (S > 1 && tile_counters && um.n_tiles * um.m_tiles <= kTileCounters) ? tile_counters : nullptr;
     *S_out = tc ? 1 : S;  // reduced in the kernel: one slice for the consumer
     *ps_out = tc ? 0 : ps;
-    if (ksub == 4) return run<1, 16, 4>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st);
-    if (ksub == 2) {
-      if (NG == 2) return run<2, 16, 2>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st);
-      return run<4, 16, 2>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st);
+#define DORY_RUN(NGV, KS) return run<NGV, 16, KS>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st)
+    if (NG == 1) {
+      if (ksub == 4) DORY_RUN(1, 4);
+      if (ksub == 2) DORY_RUN(1, 2);
+      DORY_RUN(1, 1);
     }
-    switch (NG) {
-      case 1: return run<1, 16, 1>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st);
-      case 2: return run<2, 16, 1>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st);
-      case 4: return run<4, 16, 1>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st);
-      default: return run<8, 16, 1>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st);
+    if (NG == 2) {
+      if (ksub == 2) DORY_RUN(2, 2);
+      DORY_RUN(2, 1);
     }
+    if (NG == 4) {
+      if (ksub == 2) DORY_RUN(4, 2);
+      DORY_RUN(4, 1);
+    }
+    DORY_RUN(8, 1);
+#undef DORY_RUN
   }
   // prefill: 128 x 256 tiles, no split
   um.KBg = K / BK;
@@ -584,7 +595,7 @@ cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf
   um.S = 1;
   um.m_tiles = (M + 255) / 256;
   um.units = um.n_tiles * um.m_tiles;
-  return run<1, 256, 1>(ma, X, ldx, M, K, Y, ldy, 0, um, nullptr, err, st);
+  return run<1, 256, 1, 200 * 1024>(ma, X, ldx, M, K, Y, ldy, 0, um, nullptr, err, st);
 }
 
 }  // namespace dory
