@@ -219,6 +219,24 @@ dory_status dory_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* X, const
                            int32_t batch_hint, int32_t invariant, int32_t impl, int32_t* splits, int32_t* err_word,
                            dory_stream stream);
 
+/* Projection GEMM for callers that cannot allocate device memory (no
+ * counterpart on the pages: this is a library convenience).  Some callers
+ * cannot hand dory_gemm_bf16 its 8 * M * N-float partial buffer: code running
+ * while a CUDA graph is recorded (cudaMalloc is not allowed there), servers
+ * whose device memory is one arena owned by someone else, real-time paths
+ * that forbid allocation.  This variant keeps the split-K partial sums in an
+ * 8 MiB array built into the library (held on every GPU that loads it, until
+ * exit) and writes the finished product Y = X . W^T [M, N] fp32 (device).
+ * X [M, K], W [N, K] bf16 device pointers, 16-byte aligned, N % 128 == 0,
+ * K % 64 == 0; 8 * M * N <= 2097152 or DORY_ERR_CAPACITY (checked before any
+ * work).  It calls no allocator.  The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture.  All calls share the array:
+ * calls whose kernels overlap on the GPU (other streams or threads) corrupt
+ * each other's results, so serialise them.  Queues work on `stream`. */
+dory_status dory_gemm_bf16_noalloc(int32_t M, int32_t N, int32_t K, const void* X, const void* W, float* Y,
+                                   int32_t batch_hint, dory_stream stream);
+
 /* Synchronise `stream` and report device-side errors (DORY_ERR_TIMEOUT when
  * a bounded wait in a kernel gave up; the handle stays usable). */
 dory_status dory_synchronize(dory_handle* h, dory_stream stream);

@@ -33,7 +33,7 @@ STATUS = {0: "DORY_OK", 1: "DORY_ERR_INVALID_ARG", 2: "DORY_ERR_CAPACITY", 3: "D
 SYMBOLS = ["dory_workspace_size", "dory_create", "dory_destroy", "dory_reset", "dory_prefill",
            "dory_decode_step", "dory_spec_decode", "dory_kv_bytes", "dory_seq_len", "dory_read_state",
            "dory_read_kv", "dory_synchronize", "dory_set_option", "dory_profile_read", "dory_profile_reset",
-           "dory_last_error", "dory_gemm_bf16"]
+           "dory_last_error", "dory_gemm_bf16", "dory_gemm_bf16_noalloc"]
 
 
 class DoryError(RuntimeError):
@@ -83,6 +83,7 @@ def _load() -> ctypes.CDLL:
                               ctypes.POINTER(ctypes.c_double), IP],
         "dory_profile_reset": [P],
         "dory_gemm_bf16": [I32, I32, I32, P, P, P, I32, I32, I32, IP, P, P],
+        "dory_gemm_bf16_noalloc": [I32, I32, I32, P, P, P, I32, P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)

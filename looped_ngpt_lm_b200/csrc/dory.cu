@@ -46,6 +46,15 @@ dory_status fail(dory_status s, const char* fmt, ...) {
   return s;
 }
 
+}  // namespace
+
+namespace dory {
+// Lets other translation units of the library report through dory_last_error().
+void set_last_error(const char* msg) { g_last_error = msg; }
+}  // namespace dory
+
+namespace {
+
 #define CK(expr)                                                                                  \
   do {                                                                                            \
     cudaError_t e_ = (expr);                                                                      \
