@@ -183,6 +183,8 @@ def main():
                     help="time one kernel alone instead of the decode step (prints its own JSON line)")
     ap.add_argument("--shape", default="qkv,o,gate_up,down,lm_head", help="GEMM shapes for --kernel gemm")
     ap.add_argument("--m", type=int, default=1, help="token rows for --kernel gemm")
+    ap.add_argument("--layers", default=None,
+                    help="I,R,O physical layers (a narrower model of the same width, for small profiling captures)")
     args = ap.parse_args()
     if args.kernel == "gemm":
         gemm_probe(args)
@@ -197,6 +199,10 @@ def main():
     import synth
     shape = synth.DORY_4B
     workload = f"dory4b_bf16_batch1_prompt{args.prompt}_decode_k{args.k}_{args.mode}"
+    if args.layers:
+        n_in, n_rec, n_out = (int(v) for v in args.layers.split(","))
+        shape = shape.with_(name="dory4b_cut", n_in=n_in, n_rec=n_rec, n_out=n_out)
+        workload += f"_layers{n_in}-{n_rec}-{n_out}"
     hbm, tc, tc_sus, peak_src = peaks()
 
     if args.impl == "reference":

@@ -22,6 +22,7 @@
 
 #include "dory.h"
 #include "attn_decode.cuh"
+#include "attn_prefill.cuh"
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
 
@@ -109,6 +110,9 @@ struct dory_handle {
   size_t ws_bytes = 0;
   int *seq_len = nullptr, *err = nullptr, *seq_ids = nullptr, *tokens = nullptr, *next = nullptr;
   int *cu = nullptr, *head_rows = nullptr;
+  int2* tiles = nullptr;  // prefill attention tiles (64 rows of one sequence)
+  int tiles_cap = 0;
+  void* qh = nullptr;     // bf16 pre-scaled queries of long chunks
   RowMeta meta{};
   float *h = nullptr, *x = nullptr, *s = nullptr, *q = nullptr, *part_qkv = nullptr, *part_y = nullptr,
         *part_gu = nullptr, *attn_part = nullptr, *logits = nullptr;
@@ -125,7 +129,7 @@ struct dory_handle {
   std::vector<int> len, mode, kfix;  // per sequence; mode -1 = empty
   std::vector<int> ids_on_device;     // seq ids last uploaded to seq_ids
   int last_rows = 0;
-  bool graphs = true, profile = false;
+  bool graphs = true, profile = false, prefill_tc = true;
   int gemm_impl = 0;
   std::vector<std::string> prof_names;
   std::vector<ProfRec> prof_recs;
@@ -219,6 +223,9 @@ size_t layout(dory_handle* h) {
   h->next = cv.take<int>(sizeof(int) * M);
   h->cu = cv.take<int>(sizeof(int) * (c.max_batch + 1));
   h->head_rows = cv.take<int>(sizeof(int) * h->head_max);
+  h->tiles_cap = M / 64 + c.max_batch + 1;
+  h->tiles = cv.take<int2>(sizeof(int2) * h->tiles_cap);
+  h->qh = cv.take<char>(2 * (size_t)M * h->q_dim);
   h->meta.seq = cv.take<int>(sizeof(int) * M);
   h->meta.pos = cv.take<int>(sizeof(int) * M);
   h->meta.p0 = cv.take<int>(sizeof(int) * M);
@@ -302,6 +309,7 @@ struct Fwd {
   int k;        // loop count of this pass (last loop = k)
   int batch;    // sequences in the call (selects the GEMM split)
   bool invariant;  // decode / speculative rows: GEMM arithmetic independent of M
+  int n_tiles = 0;  // > 0: long-chunk attention on the tensor cores over H->tiles
 };
 
 KVView kv_view(dory_handle* H, int l, int loop, int mode) {
@@ -372,12 +380,17 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop, float* copy_la
                                  H->attn_part, H->nb_cap, H->attn_counters, (T*)H->ao, f.st));
       } else {
         // long chunks: K/V into scratch, attention, then the cache commit
+        const bool tc = f.n_tiles > 0;
         {
           Scope sc(H, f.st, "qkv_post", 0);
           CK(launch_qkv_post<T>(M, c.n_heads, c.n_kv_heads, c.head_dim, H->part_qkv, S, ps, H->q, (T*)H->kscr,
-                                (T*)H->vscr, false, kv, H->meta, c.max_batch, f.st));
+                                (T*)H->vscr, false, kv, H->meta, c.max_batch, tc ? (bf16*)H->qh : nullptr, f.st));
         }
-        {
+        if (tc) {
+          Scope sc(H, f.st, "attn_prefill", 0);
+          CK(launch_attn_prefill(f.n_tiles, H->tiles, c.n_heads, c.n_kv_heads, c.head_dim, (const bf16*)H->qh,
+                                 (const bf16*)H->kscr, (const bf16*)H->vscr, kv, H->meta, (bf16*)H->ao, f.st));
+        } else {
           Scope sc(H, f.st, "attention", 0);
           CK(launch_attention<T>(M, c.n_heads, c.n_kv_heads, c.head_dim, H->q, (const T*)H->kscr,
                                  (const T*)H->vscr, true, kv, H->meta, f.max_ctx, H->attn_part, (T*)H->ao, f.st));
@@ -542,6 +555,13 @@ dory_status prefill_t(dory_handle* H, int batch, const int32_t* seq_ids, const i
   CK(launch_plan_ragged(batch, M, H->cu, H->seq_ids, H->seq_len, H->meta, st));
   int max_len = *std::max_element(lens, lens + batch);
   Fwd<T> f{H, st, M, max_ctx, max_len <= H->slack + 1, mode, k, batch, false};
+  if (!f.direct && H->bf16 && attn_prefill_supported(c.head_dim) && H->prefill_tc) {
+    std::vector<int2> tl(H->tiles_cap);
+    const int n = prefill_tiles(batch, cu.data(), tl.data(), H->tiles_cap);
+    if (n < 0) return fail(DORY_ERR_CAPACITY, "too many prefill attention tiles");
+    CK(cudaMemcpyAsync(H->tiles, tl.data(), sizeof(int2) * n, cudaMemcpyHostToDevice, st));
+    f.n_tiles = n;
+  }
   RET(input_block<T>(f, tokens));
   RET(loops<T>(f, 1, k, -1, 1));
   RET(output_and_head<T>(f, batch, H->head_rows, last_logits, next_tokens));
@@ -931,6 +951,7 @@ dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value) {
     case DORY_OPT_CUDA_GRAPHS: h->graphs = value != 0; return DORY_OK;
     case DORY_OPT_PROFILE: h->profile = value != 0; return DORY_OK;
     case DORY_OPT_PDL: dory::g_pdl = value != 0; return DORY_OK;
+    case DORY_OPT_PREFILL_TC: h->prefill_tc = value != 0; return DORY_OK;
     case DORY_OPT_GEMM_IMPL:
       if (value < 0 || value > 2) return fail(DORY_ERR_INVALID_ARG, "bad GEMM impl");
       h->gemm_impl = (int)value;

@@ -66,12 +66,13 @@ cudaError_t launch_stash_copy(int M, int d, float* state, float* stash, int rps,
                               int dir, cudaStream_t st);
 
 // Split q/k/v out of the QKV projection (sum of S partials).  q -> fp32 q_out
-// [M, H*hd]; k, v rounded to T -> scratch [M, KV*hd] (direct == false) or
-// straight into the cache at pos % cap (direct == true).
+// [M, H*hd] (and, when qh is not NULL, bf16 q * log2(e)/sqrt(hd) into qh);
+// k, v rounded to T -> scratch [M, KV*hd] (direct == false) or straight into
+// the cache at pos % cap (direct == true).
 template <typename T>
 cudaError_t launch_qkv_post(int M, int H, int KV, int hd, const float* qkv, int S, size_t part_stride,
                             float* q_out, T* kscr, T* vscr, bool direct, KVView kv, RowMeta m,
-                            int max_batch, cudaStream_t st);
+                            int max_batch, bf16* qh, cudaStream_t st);
 
 // GQA attention over the cache (+ chunk scratch), split over absolute key
 // blocks of ATTN_BK positions, then merged in block order.

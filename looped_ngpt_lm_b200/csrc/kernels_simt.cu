@@ -289,7 +289,7 @@ cudaError_t launch_stash_copy(int M, int d, float* state, float* stash, int rps,
 // ------------------------------------------------------------------ QKV split
 template <typename T>
 __global__ void k_qkv_post(int H, int KV, int hd, const float* qkv, int S, size_t ps, float* q_out, T* kscr,
-                           T* vscr, bool direct, KVView kv, RowMeta m, int max_batch) {
+                           T* vscr, bool direct, KVView kv, RowMeta m, int max_batch, bf16* qh, float qscale) {
   pdl_wait();
   pdl_trigger();
   const int r = blockIdx.x;
@@ -306,6 +306,7 @@ __global__ void k_qkv_post(int H, int KV, int hd, const float* qkv, int S, size_
     for (int s = 0; s < S; ++s) a += src[s * ps + i];
     if (i < qd) {
       q_out[(size_t)r * qd + i] = a;
+      if (qh) qh[(size_t)r * qd + i] = __float2bfloat16_rn(a * qscale);
     } else {
       int j = i - qd;
       bool is_v = j >= kvd;
@@ -325,8 +326,11 @@ __global__ void k_qkv_post(int H, int KV, int hd, const float* qkv, int S, size_
 
 template <typename T>
 cudaError_t launch_qkv_post(int M, int H, int KV, int hd, const float* qkv, int S, size_t ps, float* q_out,
-                            T* kscr, T* vscr, bool direct, KVView kv, RowMeta m, int max_batch, cudaStream_t st) {
-  launch(k_qkv_post<T>, M, 256, 0, st, H, KV, hd, qkv, S, ps, q_out, kscr, vscr, direct, kv, m, max_batch);
+                            T* kscr, T* vscr, bool direct, KVView kv, RowMeta m, int max_batch, bf16* qh,
+                            cudaStream_t st) {
+  const float qscale = 1.4426950408889634f / sqrtf((float)hd);
+  launch(k_qkv_post<T>, M, 256, 0, st, H, KV, hd, qkv, S, ps, q_out, kscr, vscr, direct, kv, m, max_batch, qh,
+         qscale);
   return cudaGetLastError();
 }
 
@@ -756,7 +760,7 @@ cudaError_t launch_spec_accept(int B, int gamma, int dstride, const int* seq_ids
   template cudaError_t launch_reinject<T>(int, int, float*, const float*, int, const float*, bool, T*, float*,    \
                                           int, int, int, cudaStream_t);                                           \
   template cudaError_t launch_qkv_post<T>(int, int, int, int, const float*, int, size_t, float*, T*, T*, bool,    \
-                                          KVView, RowMeta, int, cudaStream_t);                                    \
+                                          KVView, RowMeta, int, bf16*, cudaStream_t);                             \
   template cudaError_t launch_attention<T>(int, int, int, int, const float*, const T*, const T*, bool, KVView,    \
                                            RowMeta, int, float*, T*, cudaStream_t);                               \
   template cudaError_t launch_kv_commit<T>(int, int, int, const T*, const T*, KVView, RowMeta, cudaStream_t);     \

@@ -9,6 +9,7 @@ from .inputs import (  # noqa: F401
     TINY,
     TINY_BF16,
     DORY_4B,
+    SMALL128,
     SHAPES,
     layer_kinds,
     weight_specs,

@@ -80,7 +80,11 @@ TINY_BF16 = TINY.with_(name="tiny_bf16", dtype="bf16")
 # SwiGLU 10240, 16 + 40 + 16 physical layers, window 4096.
 DORY_4B = Shape("dory4b", 2560, 131072, 20, 128, 4, 10240, 16, 40, 16, 4096, dtype="bf16")
 
-SHAPES = {s.name: s for s in (TINY, TINY_BF16, DORY_4B)}
+# Small bf16 shape with 128-wide heads (the 4B head shape) and a short window,
+# so long chunks and ring wrap-around reach the bf16 attention kernels cheaply.
+SMALL128 = Shape("small128", 512, 2048, 4, 128, 1, 1024, 2, 4, 2, 32, dtype="bf16")
+
+SHAPES = {s.name: s for s in (TINY, TINY_BF16, DORY_4B, SMALL128)}
 
 
 def layer_kinds(shape: Shape) -> list[str]:
