@@ -1,22 +1,26 @@
 // Fused GQA attention for decode and speculative chunks (K/V written straight
 // into the cache).
 //
-// One block per (row, KV head g, absolute key block of DEC_BK positions):
-//   1. q of the G query heads that share KV head g = in-order sum of the QKV
-//      projection's split-K partials (scaled by log2(e)/sqrt(head_dim));
-//   2. the block holding the row's own position writes the row's K and V
-//      (same partial sums, rounded to the storage type) into the cache slot;
-//   3. keys of earlier calls come from the cache (ring index j % cap); keys of
-//      this chunk are rebuilt from the partials with the same arithmetic, so
-//      they equal what the cache will hold;
-//   4. base-2 online softmax over the block's keys: 8 warps x 4 groups of 8
+// One 256-thread block per (row, KV head g, absolute key block of DEC_BK
+// positions):
+//   1. stage the block's cached keys and values in shared memory with cp.async
+//      (every byte in flight at once from a short rolled loop); keys of this
+//      chunk are rebuilt from the QKV projection's split-K partials with the
+//      same in-order sums and rounding the cache write uses;
+//   2. q of the G query heads sharing KV head g = in-order partial sums,
+//      scaled by log2(e)/sqrt(head_dim); the block holding the row's own
+//      position writes the row's K and V into the cache slot;
+//   3. base-2 online softmax over the block's keys: 8 warps x 4 groups of 8
 //      lanes, one key per group, head_dim/8 dimensions per lane; groups merge
 //      by a fixed xor tree, warps in index order;
-//   5. the block stores (m, l, acc[head_dim]) per head; the last block of the
-//      (row, g) pair to finish (device counter) merges all blocks in block
-//      order and writes the attention output.
-// Block boundaries are absolute positions, so a row computes the same bits
-// whether it is decoded alone or verified inside a speculative chunk.
+//   4. the block stores (m, l, -, -, acc[head_dim]) per head (rows padded to
+//      16 bytes); the last block of the (row, g) pair to finish (device
+//      counter) merges every block's partial in block order, after copying
+//      them into shared memory when they fit.
+// Loops stay rolled: each block runs its code once, so a compact body keeps
+// the instruction cache warm.  Block boundaries are absolute positions, so a
+// row computes the same bits whether it is decoded alone or verified inside a
+// speculative chunk.
 #include <float.h>
 
 #include "attn_decode.cuh"
@@ -26,28 +30,15 @@ namespace dory {
 
 namespace {
 
-// A row slice of DL elements kept in the storage type until it is used.
-template <typename T, int DL>
-struct RowBuf {
-  T v[DL];
-};
+constexpr int NW = 8;  // warps per block
 
-// Vector load of DL consecutive elements (16-byte pieces; 8 bytes for 4 bf16).
-template <typename T, int DL>
-__device__ __forceinline__ void load_raw(const T* p, RowBuf<T, DL>& b) {
-  constexpr int BYTES = DL * (int)sizeof(T);
-  if constexpr (BYTES % 16 == 0) {
-    const uint4* src = reinterpret_cast<const uint4*>(p);
-    uint4* dst = reinterpret_cast<uint4*>(b.v);
-#pragma unroll
-    for (int i = 0; i < BYTES / 16; ++i) dst[i] = src[i];
-  } else {
-    static_assert(BYTES == 8, "row slice must be 8 or a multiple of 16 bytes");
-    *reinterpret_cast<uint2*>(b.v) = *reinterpret_cast<const uint2*>(p);
-  }
+__device__ __forceinline__ uint32_t saddr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void cp16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 
-// In-order sum of a value's S split-K slices (independent, predicated loads).
+// In-order sum of a value's S split-K slices.
 __device__ __forceinline__ float sum_splits(const float* p, int S, size_t ps) {
   float v[kMaxSplitK];
 #pragma unroll
@@ -60,17 +51,24 @@ __device__ __forceinline__ float sum_splits(const float* p, int S, size_t ps) {
 }
 
 template <typename T, int HD, int G>
+struct DecSmem {
+  T k[DEC_BK][HD];
+  T v[DEC_BK][HD];
+  float q[G][HD];
+  float wm[NW][G], wl[NW][G];
+  float wacc[NW][G][HD];
+  int last;
+};
+
+template <typename T, int HD, int G>
 __global__ void __launch_bounds__(256) k_attn_decode(int KV, const float* __restrict__ qkv, int S, size_t ps,
                                                      KVView kv, RowMeta m, float* __restrict__ part, int nb_max,
                                                      unsigned* __restrict__ counters, T* __restrict__ out,
                                                      float scale_log2) {
-  constexpr int DL = HD / 8;
-  constexpr int NW = 8;
-  constexpr int KPI = NW * 4;  // keys per iteration
-  __shared__ float q_sm[G][HD];
-  __shared__ float sm_m[NW][G], sm_l[NW][G];
-  __shared__ float sm_acc[NW][G][HD];
-  __shared__ int s_last;
+  constexpr int DL = HD / 8;                    // dimensions per lane
+  constexpr int CH = HD * (int)sizeof(T) / 16;  // 16-byte chunks per row
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  DecSmem<T, HD, G>& sm = *reinterpret_cast<DecSmem<T, HD, G>*>(smem_raw);
 
   pdl_wait();
   pdl_trigger();
@@ -87,95 +85,90 @@ __global__ void __launch_bounds__(256) k_attn_decode(int KV, const float* __rest
     return;
   }
   if ((int)blockIdx.y >= nb_row) return;
-  const int ab = lo / DEC_BK + blockIdx.y;
-  const int kb = ab * DEC_BK;
+  const int kb = (lo / DEC_BK + blockIdx.y) * DEC_BK;
   const int klo = max(lo, kb), khi = min(pos, kb + DEC_BK - 1);
   const int H = KV * G, qd = H * HD, kvd = KV * HD, ld = qd + 2 * kvd;
   const int tid = threadIdx.x;
-
-  constexpr int QPT = (G * HD + 255) / 256;  // q values per thread
-#pragma unroll
-  for (int c = 0; c < QPT; ++c) {
-    const int idx = tid + c * 256;
-    if (idx < G * HD) {
-      const int h = idx / HD, d = idx % HD;
-      q_sm[h][d] = sum_splits(qkv + (size_t)r * ld + (g * G + h) * HD + d, S, ps) * scale_log2;
-    }
-  }
   T* Kc = (T*)kv.K + ((size_t)seq * KV + g) * kv.cap * HD;
   T* Vc = (T*)kv.V + ((size_t)seq * KV + g) * kv.cap * HD;
-  if (khi == pos) {  // this block holds the row's own key: write it to the cache
+
+  // 1. cached keys -> shared memory (all copies in flight), chunk keys rebuilt
+  const int cache_hi = min(khi, p0 - 1);  // last cached key of this block
+  for (int i = tid; i < (cache_hi - klo + 1) * CH; i += blockDim.x) {
+    const int jj = i / CH, c = i % CH;
+    const size_t src = (size_t)((klo + jj) % kv.cap) * HD;
+    cp16(saddr(&sm.k[klo - kb + jj][0]) + c * 16, (const uint8_t*)(Kc + src) + c * 16);
+    cp16(saddr(&sm.v[klo - kb + jj][0]) + c * 16, (const uint8_t*)(Vc + src) + c * 16);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  const int jc0 = max(klo, p0);  // first key of this chunk in the block
+  for (int i = tid; i < (khi - jc0 + 1) * HD; i += blockDim.x) {
+    const int jj = i / HD, d = i % HD;
+    const float* src = qkv + (size_t)(base + (jc0 + jj - p0)) * ld + qd + g * HD + d;
+    sm.k[jc0 - kb + jj][d] = from_f<T>(sum_splits(src, S, ps));
+    sm.v[jc0 - kb + jj][d] = from_f<T>(sum_splits(src + kvd, S, ps));
+  }
+  // 2. q for the G heads; the own key goes to the cache
+  for (int i = tid; i < G * HD; i += blockDim.x) {
+    const int h = i / HD, d = i % HD;
+    sm.q[h][d] = sum_splits(qkv + (size_t)r * ld + (g * G + h) * HD + d, S, ps) * scale_log2;
+  }
+  if (khi == pos) {
     const size_t slot = (size_t)(pos % kv.cap) * HD;
-    for (int idx = tid; idx < 2 * HD; idx += blockDim.x) {
-      const int d = idx % HD;
-      const bool is_v = idx >= HD;
+    for (int i = tid; i < 2 * HD; i += blockDim.x) {
+      const int d = i % HD;
+      const bool is_v = i >= HD;
       const float a = sum_splits(qkv + (size_t)r * ld + qd + (is_v ? kvd : 0) + g * HD + d, S, ps);
       (is_v ? Vc : Kc)[slot + d] = from_f<T>(a);
     }
   }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
 
+  // 3. online softmax over the block's keys
   const int w = tid >> 5, lane = tid & 31, sg = lane >> 3, dl = lane & 7;
-  float qv[G][DL];
-#pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int e = 0; e < DL; ++e) qv[h][e] = q_sm[h][dl * DL + e];
-  float mx[G], ls[G], acc[G][DL];
+  float qv[G][DL], mx[G], ls[G], acc[G][DL];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
     mx[h] = -FLT_MAX;
     ls[h] = 0.f;
 #pragma unroll
-    for (int e = 0; e < DL; ++e) acc[h][e] = 0.f;
-  }
-  constexpr int ITER = DEC_BK / KPI;
-  RowBuf<T, DL> kr[ITER], vr[ITER];
-  bool valid[ITER];
-#pragma unroll
-  for (int it = 0; it < ITER; ++it) {
-    const int j = kb + it * KPI + w * 4 + sg;
-    valid[it] = j >= klo && j <= khi;
-    if (valid[it]) {
-      if (j < p0) {
-        const size_t idx = (size_t)(j % kv.cap) * HD + dl * DL;
-        load_raw<T, DL>(Kc + idx, kr[it]);
-        load_raw<T, DL>(Vc + idx, vr[it]);
-      } else {  // key of this chunk: rebuild it from the projection partials
-        const float* src = qkv + (size_t)(base + (j - p0)) * ld + qd + g * HD + dl * DL;
-#pragma unroll
-        for (int e = 0; e < DL; ++e) {
-          kr[it].v[e] = from_f<T>(sum_splits(src + e, S, ps));
-          vr[it].v[e] = from_f<T>(sum_splits(src + kvd + e, S, ps));
-        }
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < DL; ++e) kr[it].v[e] = vr[it].v[e] = from_f<T>(0.f);
+    for (int e = 0; e < DL; ++e) {
+      qv[h][e] = sm.q[h][dl * DL + e];
+      acc[h][e] = 0.f;
     }
   }
+#pragma unroll 1
+  for (int jq = kb + 4 * w; jq <= khi; jq += 4 * NW) {
+    const int j = jq + sg;
+    const bool valid = j >= klo && j <= khi;
+    const int row = valid ? j - kb : 0;
+    float kf[DL], vf[DL];
 #pragma unroll
-  for (int it = 0; it < ITER; ++it) {
+    for (int e = 0; e < DL; ++e) {
+      kf[e] = to_f(sm.k[row][dl * DL + e]);
+      vf[e] = to_f(sm.v[row][dl * DL + e]);
+    }
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       float sdot = 0.f;
 #pragma unroll
-      for (int e = 0; e < DL; ++e) sdot += qv[h][e] * to_f(kr[it].v[e]);
+      for (int e = 0; e < DL; ++e) sdot += qv[h][e] * kf[e];
       sdot += __shfl_xor_sync(0xffffffffu, sdot, 1);
       sdot += __shfl_xor_sync(0xffffffffu, sdot, 2);
       sdot += __shfl_xor_sync(0xffffffffu, sdot, 4);
-      if (valid[it]) {
+      if (valid) {
         const float mn = fmaxf(mx[h], sdot);
         const float corr = exp2f(mx[h] - mn);
         const float p = exp2f(sdot - mn);
         ls[h] = ls[h] * corr + p;
 #pragma unroll
-        for (int e = 0; e < DL; ++e) acc[h][e] = acc[h][e] * corr + p * to_f(vr[it].v[e]);
+        for (int e = 0; e < DL; ++e) acc[h][e] = acc[h][e] * corr + p * vf[e];
         mx[h] = mn;
       }
     }
   }
-#pragma unroll
+#pragma unroll 1
   for (int off = 8; off <= 16; off <<= 1) {
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -197,98 +190,71 @@ __global__ void __launch_bounds__(256) k_attn_decode(int KV, const float* __rest
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       if (dl == 0) {
-        sm_m[w][h] = mx[h];
-        sm_l[w][h] = ls[h];
+        sm.wm[w][h] = mx[h];
+        sm.wl[w][h] = ls[h];
       }
 #pragma unroll
-      for (int e = 0; e < DL; ++e) sm_acc[w][h][dl * DL + e] = acc[h][e];
+      for (int e = 0; e < DL; ++e) sm.wacc[w][h][dl * DL + e] = acc[h][e];
     }
   }
   __syncthreads();
-  for (int idx = tid; idx < G * (HD + 2); idx += blockDim.x) {
-    const int h = idx / (HD + 2), c = idx % (HD + 2);
+  constexpr int PE = HD + 4;  // partial entry: m, l, 2 pad, acc[HD]
+  const size_t hstride = (size_t)nb_max * PE;
+  float* pr0 = part + ((size_t)r * H + g * G) * hstride;
+  for (int i = tid; i < G * (HD + 2); i += blockDim.x) {
+    const int h = i / (HD + 2), c = i % (HD + 2);
     float M = -FLT_MAX;
-#pragma unroll
-    for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, sm_m[ww][h]);
-    float val = 0.f;
-    if (c == 0) {
-      val = M;
-    } else {
-#pragma unroll
+    for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, sm.wm[ww][h]);
+    float val = M;
+    if (c > 0) {
+      val = 0.f;
       for (int ww = 0; ww < NW; ++ww) {
-        const float sc = sm_m[ww][h] == -FLT_MAX ? 0.f : exp2f(sm_m[ww][h] - M);
-        val += (c == 1 ? sm_l[ww][h] : sm_acc[ww][h][c - 2]) * sc;
+        const float sc = sm.wm[ww][h] == -FLT_MAX ? 0.f : exp2f(sm.wm[ww][h] - M);
+        val += (c == 1 ? sm.wl[ww][h] : sm.wacc[ww][h][c - 2]) * sc;
       }
     }
-    part[(((size_t)r * H + g * G + h) * nb_max + blockIdx.y) * (HD + 2) + c] = val;
+    pr0[h * hstride + blockIdx.y * PE + (c < 2 ? c : c + 2)] = val;
   }
-  // last block of this (row, g) merges every block in order
+
+  // 4. the last block of this (row, g) merges all blocks in order
   __threadfence();
   __syncthreads();
-  if (tid == 0) {
-    const unsigned prev = atomicAdd(&counters[r * KV + g], 1u);
-    s_last = prev == (unsigned)(nb_row - 1);
-  }
+  if (tid == 0) sm.last = atomicAdd(&counters[r * KV + g], 1u) == (unsigned)(nb_row - 1);
   __syncthreads();
-  if (!s_last) return;
+  if (!sm.last) return;
   __threadfence();
-  // merge: (1) all threads fetch every block's (m, l) into shared memory;
-  // (2) per head, the max M and 1/L = 1 / sum_b l_b 2^(m_b - M); (3) block
-  // weights 2^(m_b - M); (4) every (head, dim) output sums its blocks with
-  // independent loads.  Block order fixes the summation order.
-  float* sm_mb = &sm_acc[0][0][0];  // reused: [G][nb_row] m, then weights
-  float* sm_lb = sm_mb + G * nb_row;  // [G][nb_row] l
-  float* sm_hd = sm_lb + G * nb_row;  // [G] M, then [G] 1/L
-  const size_t hstride = (size_t)nb_max * (HD + 2);
-  const float* pr0 = part + ((size_t)r * H + g * G) * hstride;
-  for (int idx = tid; idx < G * nb_row; idx += blockDim.x) {
-    const int h = idx / nb_row, b = idx % nb_row;
-    sm_mb[idx] = __ldcg(pr0 + h * hstride + b * (HD + 2));
-    sm_lb[idx] = __ldcg(pr0 + h * hstride + b * (HD + 2) + 1);
+  // every block's partial -> shared memory (reusing the key/value buffers)
+  // when they fit, else read them from L2
+  const bool in_smem = (size_t)G * nb_row * PE * 4 <= sizeof(sm.k) + sizeof(sm.v);
+  const float* pb = pr0;
+  size_t pstride = hstride;
+  if (in_smem) {
+    float* dst = reinterpret_cast<float*>(&sm.k[0][0]);  // [G][nb_row][PE]
+    const int nrow4 = nb_row * PE / 4;                   // 16-byte pieces per head
+    for (int i = tid; i < G * nrow4; i += blockDim.x) {
+      const int h = i / nrow4, c = i % nrow4;
+      cp16(saddr(dst + (size_t)h * nb_row * PE) + c * 16, pr0 + h * hstride + c * 4);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    pb = dst;
+    pstride = (size_t)nb_row * PE;
   }
   __syncthreads();
-  if (tid < G) {
+  // shared memory: plain loads; global (other blocks' writes): L2 loads
+  auto ldp = [&](const float* p) { return in_smem ? *p : __ldcg(p); };
+  for (int i = tid; i < G * HD; i += blockDim.x) {
+    const int h = i / HD, d = i % HD;
+    const float* ph = pb + h * pstride;
     float M = -FLT_MAX;
-    for (int b = 0; b < nb_row; ++b) M = fmaxf(M, sm_mb[tid * nb_row + b]);
-    float L = 0.f;
-    for (int b = 0; b < nb_row; ++b) L += sm_lb[tid * nb_row + b] * exp2f(sm_mb[tid * nb_row + b] - M);
-    sm_hd[tid] = M;
-    sm_hd[G + tid] = 1.f / L;
-  }
-  __syncthreads();
-  for (int idx = tid; idx < G * nb_row; idx += blockDim.x) sm_mb[idx] = exp2f(sm_mb[idx] - sm_hd[idx / nb_row]);
-  __syncthreads();
-  const float* wts = sm_mb;
-  constexpr int OPT = (G * HD + 255) / 256;  // outputs per thread
-  constexpr int BB = 8;                      // blocks per batch of loads
-  float o[OPT];
-#pragma unroll
-  for (int c = 0; c < OPT; ++c) o[c] = 0.f;
-  for (int b0 = 0; b0 < nb_row; b0 += BB) {
-    float v[OPT][BB];
-#pragma unroll
-    for (int c = 0; c < OPT; ++c) {
-      const int idx = tid + c * 256;
-      const int h = idx / HD, d = idx % HD;
-#pragma unroll
-      for (int j = 0; j < BB; ++j)
-        v[c][j] = (idx < G * HD && b0 + j < nb_row) ? __ldcg(pr0 + h * hstride + (b0 + j) * (HD + 2) + 2 + d) : 0.f;
+    for (int b = 0; b < nb_row; ++b) M = fmaxf(M, ldp(ph + b * PE));
+    float L = 0.f, a = 0.f;
+    for (int b = 0; b < nb_row; ++b) {
+      const float wgt = exp2f(ldp(ph + b * PE) - M);
+      L += ldp(ph + b * PE + 1) * wgt;
+      a += ldp(ph + b * PE + 4 + d) * wgt;
     }
-#pragma unroll
-    for (int c = 0; c < OPT; ++c) {
-      const int h = min((tid + c * 256) / HD, G - 1);
-#pragma unroll
-      for (int j = 0; j < BB; ++j)
-        if (b0 + j < nb_row) o[c] += v[c][j] * wts[h * nb_row + b0 + j];
-    }
-  }
-#pragma unroll
-  for (int c = 0; c < OPT; ++c) {
-    const int idx = tid + c * 256;
-    if (idx < G * HD) {
-      const int h = idx / HD, d = idx % HD;
-      out[(size_t)r * qd + (g * G + h) * HD + d] = from_f<T>(o[c] * sm_hd[G + h]);
-    }
+    out[(size_t)r * qd + (g * G + h) * HD + d] = from_f<T>(a / L);
   }
   if (tid == 0) counters[r * KV + g] = 0u;
 }
@@ -298,10 +264,16 @@ cudaError_t dispatch(int M, int KV, const float* qkv, int S, size_t ps, KVView k
                      float* part, int nb_cap, unsigned* counters, T* out, cudaStream_t st) {
   const int span = kv.window > 0 ? min(max_ctx, kv.window) : max_ctx;
   const int nb = (span + DEC_BK - 1) / DEC_BK + 1;
-  // the merge keeps 2 * G * nb + 2 * G floats in the 8 * G * HD float buffer
-  if (nb > nb_cap || 2 * nb + 2 > 8 * HD) return cudaErrorInvalidValue;
+  constexpr int SMEM = (int)sizeof(DecSmem<T, HD, G>);
+  if (nb > nb_cap) return cudaErrorInvalidValue;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_attn_decode<T, HD, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
-  return launch(k_attn_decode<T, HD, G>, dim3(M * KV, nb), dim3(256), 0, st, KV, qkv, S, ps, kv, m, part, nb,
+  return launch(k_attn_decode<T, HD, G>, dim3(M * KV, nb), dim3(256), SMEM, st, KV, qkv, S, ps, kv, m, part, nb,
                 counters, out, scale_log2);
 }
 

@@ -9,7 +9,7 @@ constexpr int DEC_BK = 128;  // keys per block (absolute-position aligned)
 
 // Attention of M rows whose K/V go straight into the cache.  qkv: the QKV
 // projection's S split-K partial slices (slice stride ps floats, rows of
-// q_dim + 2 kv_dim).  part: [M, H, nb_cap, hd + 2] scratch; counters:
+// q_dim + 2 kv_dim).  part: [M, H, nb_cap, hd + 4] scratch; counters:
 // [M * KV] zeros (left zero on return).  out: [M, H * hd] in the storage type.
 template <typename T>
 cudaError_t launch_attn_decode(int M, int H, int KV, int hd, const float* qkv, int S, size_t ps, KVView kv,

@@ -245,7 +245,7 @@ size_t layout(dory_handle* h) {
   h->part_qkv = cv.take<float>(sizeof(float) * kMaxSplitK * h->part_rows * h->qkv_dim);
   h->part_y = cv.take<float>(sizeof(float) * kMaxSplitK * h->part_rows * d);
   h->part_gu = cv.take<float>(sizeof(float) * kMaxSplitK * h->part_rows * 2 * c.d_ff);
-  h->attn_part = cv.take<float>(sizeof(float) * (size_t)M * c.n_heads * h->nb_cap * (c.head_dim + 2));
+  h->attn_part = cv.take<float>(sizeof(float) * (size_t)M * c.n_heads * h->nb_cap * (c.head_dim + 4));
   h->attn_counters = cv.take<unsigned>(sizeof(unsigned) * (size_t)M * c.n_kv_heads);
   h->tile_counters = cv.take<unsigned>(sizeof(unsigned) * kTileCounters);
   h->logits = cv.take<float>(sizeof(float) * (size_t)h->head_max * c.vocab * kMaxSplitK);
