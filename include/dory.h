@@ -247,7 +247,8 @@ enum {
   DORY_OPT_PROFILE = 2,     /* 1: time every launch with CUDA events (slow) */
   DORY_OPT_GEMM_IMPL = 3,   /* bf16 GEMM: 0 auto, 1 SIMT reference kernel, 2 tcgen05 */
   DORY_OPT_PDL = 4,         /* 1 (default): programmatic dependent launches (process-wide) */
-  DORY_OPT_PREFILL_TC = 5   /* 1 (default): bf16 long-chunk attention on the tensor cores; 0: CUDA cores */
+  DORY_OPT_PREFILL_TC = 5,  /* 1 (default): bf16 long-chunk attention on the tensor cores; 0: CUDA cores */
+  DORY_OPT_ATTN_CLUSTER = 6 /* 1 (default): decode attention as 16-block clusters (process-wide) */
 };
 dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value);
 

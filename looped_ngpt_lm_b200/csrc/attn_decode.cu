@@ -32,6 +32,12 @@ namespace {
 
 constexpr int NW = 8;  // warps per block
 
+}  // namespace
+
+bool g_attn_cluster = true;
+
+namespace {
+
 __device__ __forceinline__ uint32_t saddr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
 __device__ __forceinline__ void cp16(uint32_t dst, const void* src) {
@@ -259,9 +265,270 @@ __global__ void __launch_bounds__(256) k_attn_decode(int KV, const float* __rest
   if (tid == 0) counters[r * KV + g] = 0u;
 }
 
+// ---------------------------------------------------------------------------
+// Cluster variant: one cluster of CS blocks per (row, KV head).  The row's key
+// range [lo, pos] is cut into CS equal parts (a function of the row's own
+// positions only, so decode and verify rows get identical partitions); each
+// block streams its part through shared memory in sub-chunks of DEC_BK keys;
+// the blocks' partials are merged in rank order by rank 0 through
+// distributed shared memory.  No global partials, fences or counters.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float dsmem_ld(const float* local, int rank) {
+  uint32_t a = saddr(local), ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+  return v;
+}
+
+template <typename T, int HD, int G>
+struct ClSmem {
+  T k[DEC_BK][HD];
+  T v[DEC_BK][HD];
+  float q[G][HD];
+  float wm[NW][G], wl[NW][G];
+  float wacc[NW][G][HD];
+  float part[G][HD + 2];   // this block's (m, l, acc) -- read by rank 0
+  float rw[16][G];         // rank 0: per-rank weights
+  float rinv[G];
+};
+
+template <typename T, int HD, int G, int CS>
+__global__ void __launch_bounds__(256) k_attn_decode_cl(int KV, const float* __restrict__ qkv, int S, size_t ps,
+                                                        KVView kv, RowMeta m, T* __restrict__ out,
+                                                        float scale_log2) {
+  constexpr int DL = HD / 8;
+  constexpr int CH = HD * (int)sizeof(T) / 16;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  ClSmem<T, HD, G>& sm = *reinterpret_cast<ClSmem<T, HD, G>*>(smem_raw);
+
+  pdl_wait();
+  pdl_trigger();
+  const int pair = blockIdx.x / CS, rank = blockIdx.x % CS;
+  const int r = pair / KV, g = pair % KV;
+  const int pos = m.pos[r], seq = m.seq[r], p0 = m.p0[r], base = m.base[r];
+  const bool row_ok = pos >= 0 && pos < kv.limit;
+  if (!row_ok && threadIdx.x == 0 && rank == 0) set_error(kv.err, DEV_ERR_BAD_INDEX);
+  const int lo = kv.window > 0 ? max(0, pos - kv.window + 1) : 0;
+  const int nk = pos - lo + 1, per = (nk + CS - 1) / CS;
+  const int klo = lo + rank * per, khi = row_ok ? min(pos, klo + per - 1) : klo - 1;  // empty when klo > khi
+  const int H = KV * G, qd = H * HD, kvd = KV * HD, ld = qd + 2 * kvd;
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, sg = lane >> 3, dl = lane & 7;
+  T* Kc = (T*)kv.K + ((size_t)seq * KV + g) * kv.cap * HD;
+  T* Vc = (T*)kv.V + ((size_t)seq * KV + g) * kv.cap * HD;
+
+  if (row_ok) {
+    for (int i = tid; i < G * HD; i += blockDim.x) {
+      const int h = i / HD, d = i % HD;
+      sm.q[h][d] = sum_splits(qkv + (size_t)r * ld + (g * G + h) * HD + d, S, ps) * scale_log2;
+    }
+    if (klo <= pos && pos <= khi) {  // this block holds the row's own key
+      const size_t slot = (size_t)(pos % kv.cap) * HD;
+      for (int i = tid; i < 2 * HD; i += blockDim.x) {
+        const int d = i % HD;
+        const bool is_v = i >= HD;
+        const float a = sum_splits(qkv + (size_t)r * ld + qd + (is_v ? kvd : 0) + g * HD + d, S, ps);
+        (is_v ? Vc : Kc)[slot + d] = from_f<T>(a);
+      }
+    }
+  }
+  __syncthreads();
+  float qv[G][DL], mx[G], ls[G], acc[G][DL];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    mx[h] = -FLT_MAX;
+    ls[h] = 0.f;
+#pragma unroll
+    for (int e = 0; e < DL; ++e) {
+      qv[h][e] = sm.q[h][dl * DL + e];
+      acc[h][e] = 0.f;
+    }
+  }
+#pragma unroll 1
+  for (int c0 = klo; c0 <= khi; c0 += DEC_BK) {
+    const int c1 = min(khi, c0 + DEC_BK - 1);
+    const int cache_hi = min(c1, p0 - 1);
+    for (int i = tid; i < (cache_hi - c0 + 1) * CH; i += blockDim.x) {
+      const int jj = i / CH, c = i % CH;
+      const size_t src = (size_t)((c0 + jj) % kv.cap) * HD;
+      cp16(saddr(&sm.k[jj][0]) + c * 16, (const uint8_t*)(Kc + src) + c * 16);
+      cp16(saddr(&sm.v[jj][0]) + c * 16, (const uint8_t*)(Vc + src) + c * 16);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    const int jc0 = max(c0, p0);
+    for (int i = tid; i < (c1 - jc0 + 1) * HD; i += blockDim.x) {
+      const int jj = i / HD, d = i % HD;
+      const float* src = qkv + (size_t)(base + (jc0 + jj - p0)) * ld + qd + g * HD + d;
+      sm.k[jc0 - c0 + jj][d] = from_f<T>(sum_splits(src, S, ps));
+      sm.v[jc0 - c0 + jj][d] = from_f<T>(sum_splits(src + kvd, S, ps));
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+#pragma unroll 1
+    for (int jq = c0 + 4 * w; jq <= c1; jq += 4 * NW) {
+      const int j = jq + sg;
+      const bool valid = j <= c1;
+      const int row = valid ? j - c0 : 0;
+      float kf[DL], vf[DL];
+#pragma unroll
+      for (int e = 0; e < DL; ++e) {
+        kf[e] = to_f(sm.k[row][dl * DL + e]);
+        vf[e] = to_f(sm.v[row][dl * DL + e]);
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float sdot = 0.f;
+#pragma unroll
+        for (int e = 0; e < DL; ++e) sdot += qv[h][e] * kf[e];
+        sdot += __shfl_xor_sync(0xffffffffu, sdot, 1);
+        sdot += __shfl_xor_sync(0xffffffffu, sdot, 2);
+        sdot += __shfl_xor_sync(0xffffffffu, sdot, 4);
+        if (valid) {
+          const float mn = fmaxf(mx[h], sdot);
+          const float corr = exp2f(mx[h] - mn);
+          const float p = exp2f(sdot - mn);
+          ls[h] = ls[h] * corr + p;
+#pragma unroll
+          for (int e = 0; e < DL; ++e) acc[h][e] = acc[h][e] * corr + p * vf[e];
+          mx[h] = mn;
+        }
+      }
+    }
+    __syncthreads();
+  }
+#pragma unroll 1
+  for (int off = 8; off <= 16; off <<= 1) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float om = __shfl_xor_sync(0xffffffffu, mx[h], off);
+      const float ol = __shfl_xor_sync(0xffffffffu, ls[h], off);
+      const float mn = fmaxf(mx[h], om);
+      const float ca = (mx[h] == -FLT_MAX) ? 0.f : exp2f(mx[h] - mn);
+      const float cb = (om == -FLT_MAX) ? 0.f : exp2f(om - mn);
+      ls[h] = ls[h] * ca + ol * cb;
+#pragma unroll
+      for (int e = 0; e < DL; ++e) {
+        const float oa = __shfl_xor_sync(0xffffffffu, acc[h][e], off);
+        acc[h][e] = acc[h][e] * ca + oa * cb;
+      }
+      mx[h] = mn;
+    }
+  }
+  if (sg == 0) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      if (dl == 0) {
+        sm.wm[w][h] = mx[h];
+        sm.wl[w][h] = ls[h];
+      }
+#pragma unroll
+      for (int e = 0; e < DL; ++e) sm.wacc[w][h][dl * DL + e] = acc[h][e];
+    }
+  }
+  __syncthreads();
+  // warps -> this block's partial (per-warp weights computed once per head)
+  if (tid < G) {
+    float M = -FLT_MAX;
+    for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, sm.wm[ww][tid]);
+    float L = 0.f;
+    for (int ww = 0; ww < NW; ++ww) {
+      const float sc = sm.wm[ww][tid] == -FLT_MAX ? 0.f : exp2f(sm.wm[ww][tid] - M);
+      sm.wm[ww][tid] = sc;  // now the warp's weight
+      L += sm.wl[ww][tid] * sc;
+    }
+    sm.part[tid][0] = M;
+    sm.part[tid][1] = L;
+  }
+  __syncthreads();
+  for (int i = tid; i < G * HD; i += blockDim.x) {
+    const int h = i / HD, d = i % HD;
+    float a = 0.f;
+    for (int ww = 0; ww < NW; ++ww) a += sm.wacc[ww][h][d] * sm.wm[ww][h];
+    sm.part[h][2 + d] = a;
+  }
+  cluster_sync();  // every block's partial is ready
+  if (rank == 0 && row_ok) {
+    if (tid < G) {
+      float M = -FLT_MAX;
+      for (int q = 0; q < CS; ++q) M = fmaxf(M, dsmem_ld(&sm.part[tid][0], q));
+      float L = 0.f;
+      for (int q = 0; q < CS; ++q) {
+        const float mq = dsmem_ld(&sm.part[tid][0], q);
+        const float wq = mq == -FLT_MAX ? 0.f : exp2f(mq - M);
+        sm.rw[q][tid] = wq;
+        L += dsmem_ld(&sm.part[tid][1], q) * wq;
+      }
+      sm.rinv[tid] = 1.f / L;
+    }
+    __syncthreads();
+    for (int i = tid; i < G * HD; i += blockDim.x) {
+      const int h = i / HD, d = i % HD;
+      float a = 0.f;
+      for (int q = 0; q < CS; ++q) a += dsmem_ld(&sm.part[h][2 + d], q) * sm.rw[q][h];
+      out[(size_t)r * qd + (g * G + h) * HD + d] = from_f<T>(a * sm.rinv[h]);
+    }
+  }
+  cluster_sync();  // rank 0 has read every partial; blocks may exit
+}
+
+template <typename T, int HD, int G>
+cudaError_t dispatch_cl(int M, int KV, const float* qkv, int S, size_t ps, KVView kv, RowMeta m, T* out,
+                        cudaStream_t st) {
+  constexpr int CS = 16;
+  constexpr int SMEM = (int)sizeof(ClSmem<T, HD, G>);
+  static int state = 0;  // 0 unknown, 1 usable, -1 not schedulable here
+  if (state == 0) {
+    auto kern = k_attn_decode_cl<T, HD, G, CS>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+      cudaGetLastError();
+      state = -1;
+    } else {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(CS);
+      cfg.blockDim = dim3(256);
+      cfg.dynamicSmemBytes = SMEM;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = CS;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      int n = 0;
+      state = (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0) ? 1 : -1;
+      cudaGetLastError();
+    }
+  }
+  if (state < 0) return cudaErrorNotSupported;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(M * KV * CS);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = CS;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = g_pdl ? 1 : 0;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
+  return cudaLaunchKernelEx(&cfg, k_attn_decode_cl<T, HD, G, CS>, KV, qkv, S, ps, kv, m, out, scale_log2);
+}
+
 template <typename T, int HD, int G>
 cudaError_t dispatch(int M, int KV, const float* qkv, int S, size_t ps, KVView kv, RowMeta m, int max_ctx,
                      float* part, int nb_cap, unsigned* counters, T* out, cudaStream_t st) {
+  if (g_attn_cluster) {
+    cudaError_t e = dispatch_cl<T, HD, G>(M, KV, qkv, S, ps, kv, m, out, st);
+    if (e != cudaErrorNotSupported) return e;
+  }
   const int span = kv.window > 0 ? min(max_ctx, kv.window) : max_ctx;
   const int nb = (span + DEC_BK - 1) / DEC_BK + 1;
   constexpr int SMEM = (int)sizeof(DecSmem<T, HD, G>);

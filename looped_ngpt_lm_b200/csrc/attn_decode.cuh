@@ -7,6 +7,10 @@ namespace dory {
 
 constexpr int DEC_BK = 128;  // keys per block (absolute-position aligned)
 
+// Use the cluster kernel (16 blocks per row and KV head, merged through
+// distributed shared memory) when the device can schedule it.
+extern bool g_attn_cluster;
+
 // Attention of M rows whose K/V go straight into the cache.  qkv: the QKV
 // projection's S split-K partial slices (slice stride ps floats, rows of
 // q_dim + 2 kv_dim).  part: [M, H, nb_cap, hd + 4] scratch; counters:

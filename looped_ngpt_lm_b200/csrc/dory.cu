@@ -952,6 +952,7 @@ dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value) {
     case DORY_OPT_PROFILE: h->profile = value != 0; return DORY_OK;
     case DORY_OPT_PDL: dory::g_pdl = value != 0; return DORY_OK;
     case DORY_OPT_PREFILL_TC: h->prefill_tc = value != 0; return DORY_OK;
+    case DORY_OPT_ATTN_CLUSTER: dory::g_attn_cluster = value != 0; return DORY_OK;
     case DORY_OPT_GEMM_IMPL:
       if (value < 0 || value > 2) return fail(DORY_ERR_INVALID_ARG, "bad GEMM impl");
       h->gemm_impl = (int)value;
