@@ -25,6 +25,7 @@
 
 #include "attn_decode.cuh"
 #include "gemm_tc.cuh"
+#include "warp_mma.cuh"
 
 namespace dory {
 
@@ -474,6 +475,274 @@ __global__ void __launch_bounds__(256) k_attn_decode_cl(int KV, const float* __r
   cluster_sync();  // rank 0 has read every partial; blocks may exit
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core variant (bf16, head_dim 64 or 128): the cluster layout above,
+// with each warp running 16-key steps on mma.sync.  The G query heads that
+// share the KV head are rows 0..G-1 of a 16-row A tile (rows G..15 are zero),
+// so S = Q K^T and O += P V cost 2 * head_dim / 8 MMAs per 16 keys.  Warps
+// take steps w, w + 8, ...; their states merge in warp order, then the
+// cluster's blocks merge in rank order through distributed shared memory.
+constexpr int TC_KC = 192;  // keys per shared-memory sub-chunk
+
+template <int HD, int G>
+struct TcSmem {
+  uint8_t q[16 * HD * 2];
+  uint8_t k[TC_KC * HD * 2];
+  uint8_t v[TC_KC * HD * 2];
+  float wm[NW][G], wl[NW][G];
+  float wacc[NW][G][HD];
+  float part[G][HD + 2];
+  float rw[16][G];
+  float rinv[G];
+};
+
+template <int HD, int G, int CS>
+__global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __restrict__ qkv, int S, size_t ps,
+                                                        KVView kv, RowMeta m, bf16* __restrict__ out,
+                                                        float scale_log2) {
+  using namespace wm;
+  constexpr int CH = HD / 8;  // 16-byte chunks per row
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  TcSmem<HD, G>& sm = *reinterpret_cast<TcSmem<HD, G>*>(smem_raw);
+
+  pdl_wait();
+  pdl_trigger();
+  const int pair = blockIdx.x / CS, rank = blockIdx.x % CS;
+  const int r = pair / KV, g = pair % KV;
+  const int pos = m.pos[r], seq = m.seq[r], p0 = m.p0[r], base = m.base[r];
+  const bool row_ok = pos >= 0 && pos < kv.limit;
+  if (!row_ok && threadIdx.x == 0 && rank == 0) set_error(kv.err, DEV_ERR_BAD_INDEX);
+  const int lo = kv.window > 0 ? max(0, pos - kv.window + 1) : 0;
+  const int nk = pos - lo + 1, per = (nk + CS - 1) / CS;
+  const int klo = lo + rank * per, khi = row_ok ? min(pos, klo + per - 1) : klo - 1;
+  const int H = KV * G, qd = H * HD, kvd = KV * HD, ld = qd + 2 * kvd;
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, gq = lane >> 2, tig = lane & 3;
+  const bf16* Kc = (const bf16*)kv.K + ((size_t)seq * KV + g) * kv.cap * HD;
+  const bf16* Vc = (const bf16*)kv.V + ((size_t)seq * KV + g) * kv.cap * HD;
+
+  // Q tile: rows 0..G-1 = the G heads (pre-scaled, bf16), rows G..15 zero
+  for (int i = tid; i < 16 * HD; i += blockDim.x) {
+    const int h = i / HD, d = i % HD;
+    float val = 0.f;
+    if (h < G && row_ok) val = sum_splits(qkv + (size_t)r * ld + (g * G + h) * HD + d, S, ps) * scale_log2;
+    *reinterpret_cast<bf16*>(sm.q + swz<HD>(h, d / 8) + (d % 8) * 2) = __float2bfloat16_rn(val);
+  }
+  if (row_ok && klo <= pos && pos <= khi) {  // this block holds the row's own key
+    bf16* Kw = (bf16*)kv.K + ((size_t)seq * KV + g) * kv.cap * HD;
+    bf16* Vw = (bf16*)kv.V + ((size_t)seq * KV + g) * kv.cap * HD;
+    const size_t slot = (size_t)(pos % kv.cap) * HD;
+    for (int i = tid; i < 2 * HD; i += blockDim.x) {
+      const int d = i % HD;
+      const bool is_v = i >= HD;
+      const float a = sum_splits(qkv + (size_t)r * ld + qd + (is_v ? kvd : 0) + g * HD + d, S, ps);
+      (is_v ? Vw : Kw)[slot + d] = __float2bfloat16_rn(a);
+    }
+  }
+  __syncthreads();
+  uint32_t qa[HD / 16][4];
+#pragma unroll
+  for (int kk = 0; kk < HD / 16; ++kk)
+    ldsm_x4(smem_addr(sm.q + swz<HD>(lane % 16, kk * 2 + lane / 16)), qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
+
+  float o[HD / 8][4];
+#pragma unroll
+  for (int i = 0; i < HD / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float mrow[2] = {-FLT_MAX, -FLT_MAX}, lrow[2] = {0.f, 0.f};
+
+#pragma unroll 1
+  for (int c0 = klo; c0 <= khi; c0 += TC_KC) {
+    const int c1 = min(khi, c0 + TC_KC - 1), n = c1 - c0 + 1, n16 = (n + 15) & ~15;
+    const int cache_hi = min(c1, p0 - 1);
+    for (int i = tid; i < n16 * CH; i += blockDim.x) {
+      const int jj = i / CH, c = i % CH, j = c0 + jj;
+      if (j <= cache_hi || jj >= n) {  // cached key, or zero padding up to 16 keys
+        const bool ok = jj < n;
+        const size_t src = (size_t)((ok ? j : c0) % kv.cap) * HD + c * 8;
+        cp_async16(smem_addr(sm.k + swz<HD>(jj, c)), Kc + src, ok);
+        cp_async16(smem_addr(sm.v + swz<HD>(jj, c)), Vc + src, ok);
+      }
+    }
+    cp_async_commit();
+    const int jc0 = max(c0, p0);
+    for (int i = tid; i < (c1 - jc0 + 1) * HD; i += blockDim.x) {
+      const int jj = i / HD, d = i % HD, row = jc0 - c0 + jj;
+      const float* src = qkv + (size_t)(base + (jc0 + jj - p0)) * ld + qd + g * HD + d;
+      *reinterpret_cast<bf16*>(sm.k + swz<HD>(row, d / 8) + (d % 8) * 2) =
+          __float2bfloat16_rn(sum_splits(src, S, ps));
+      *reinterpret_cast<bf16*>(sm.v + swz<HD>(row, d / 8) + (d % 8) * 2) =
+          __float2bfloat16_rn(sum_splits(src + kvd, S, ps));
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+#pragma unroll 1
+    for (int st = w; st * 16 < n; st += NW) {
+      float sc[2][4];
+#pragma unroll
+      for (int t = 0; t < 2; ++t) sc[t][0] = sc[t][1] = sc[t][2] = sc[t][3] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < HD / 16; ++kk) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(smem_addr(sm.k + swz<HD>(st * 16 + (lane % 8) + (lane / 16) * 8, kk * 2 + (lane / 8) % 2)), b0, b1,
+                b2, b3);
+        mma_bf16(sc[0], qa[kk], b0, b1);
+        mma_bf16(sc[1], qa[kk], b2, b3);
+      }
+      float mx[2] = {mrow[0], mrow[1]};
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int jl = st * 16 + t * 8 + 2 * tig + (e & 1);
+          if (jl >= n) sc[t][e] = -FLT_MAX;
+          mx[e >> 1] = fmaxf(mx[e >> 1], sc[t][e]);
+        }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 1));
+        mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 2));
+      }
+      float corr[2], rs[2] = {0.f, 0.f}, pv[2][4];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) corr[i] = mrow[i] == -FLT_MAX ? 0.f : exp2f(mrow[i] - mx[i]);
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          pv[t][e] = sc[t][e] == -FLT_MAX ? 0.f : exp2f(sc[t][e] - mx[e >> 1]);
+          rs[e >> 1] += pv[t][e];
+        }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        rs[i] += __shfl_xor_sync(0xffffffffu, rs[i], 1);
+        rs[i] += __shfl_xor_sync(0xffffffffu, rs[i], 2);
+        lrow[i] = lrow[i] * corr[i] + rs[i];
+        mrow[i] = mx[i];
+      }
+      const uint32_t pa[4] = {pack_bf16(pv[0][0], pv[0][1]), pack_bf16(pv[0][2], pv[0][3]),
+                              pack_bf16(pv[1][0], pv[1][1]), pack_bf16(pv[1][2], pv[1][3])};
+#pragma unroll
+      for (int i = 0; i < HD / 8; ++i) {
+        o[i][0] *= corr[0];
+        o[i][1] *= corr[0];
+        o[i][2] *= corr[1];
+        o[i][3] *= corr[1];
+      }
+#pragma unroll
+      for (int d = 0; d < HD / 16; ++d) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(smem_addr(sm.v + swz<HD>(st * 16 + (lane % 8) + ((lane / 8) % 2) * 8, d * 2 + lane / 16)), b0, b1,
+                  b2, b3);
+        mma_bf16(o[2 * d], pa, b0, b1);
+        mma_bf16(o[2 * d + 1], pa, b2, b3);
+      }
+    }
+    __syncthreads();
+  }
+  // this warp's rows 0..G-1 (held by lanes with gq < G, row gq) -> shared memory
+  if (gq < G) {
+    if (tig == 0) {
+      sm.wm[w][gq] = mrow[0];
+      sm.wl[w][gq] = lrow[0];
+    }
+#pragma unroll
+    for (int i = 0; i < HD / 8; ++i) {
+      sm.wacc[w][gq][i * 8 + 2 * tig] = o[i][0];
+      sm.wacc[w][gq][i * 8 + 2 * tig + 1] = o[i][1];
+    }
+  }
+  __syncthreads();
+  if (tid < G) {
+    float M = -FLT_MAX;
+    for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, sm.wm[ww][tid]);
+    float L = 0.f;
+    for (int ww = 0; ww < NW; ++ww) {
+      const float scw = sm.wm[ww][tid] == -FLT_MAX ? 0.f : exp2f(sm.wm[ww][tid] - M);
+      sm.wm[ww][tid] = scw;
+      L += sm.wl[ww][tid] * scw;
+    }
+    sm.part[tid][0] = M;
+    sm.part[tid][1] = L;
+  }
+  __syncthreads();
+  for (int i = tid; i < G * HD; i += blockDim.x) {
+    const int h = i / HD, d = i % HD;
+    float a = 0.f;
+    for (int ww = 0; ww < NW; ++ww) a += sm.wacc[ww][h][d] * sm.wm[ww][h];
+    sm.part[h][2 + d] = a;
+  }
+  cluster_sync();
+  if (rank == 0 && row_ok) {
+    if (tid < G) {
+      float M = -FLT_MAX;
+      for (int q = 0; q < CS; ++q) M = fmaxf(M, dsmem_ld(&sm.part[tid][0], q));
+      float L = 0.f;
+      for (int q = 0; q < CS; ++q) {
+        const float mq = dsmem_ld(&sm.part[tid][0], q);
+        const float wq = mq == -FLT_MAX ? 0.f : exp2f(mq - M);
+        sm.rw[q][tid] = wq;
+        L += dsmem_ld(&sm.part[tid][1], q) * wq;
+      }
+      sm.rinv[tid] = 1.f / L;
+    }
+    __syncthreads();
+    for (int i = tid; i < G * HD; i += blockDim.x) {
+      const int h = i / HD, d = i % HD;
+      float a = 0.f;
+      for (int q = 0; q < CS; ++q) a += dsmem_ld(&sm.part[h][2 + d], q) * sm.rw[q][h];
+      out[(size_t)r * qd + (g * G + h) * HD + d] = __float2bfloat16_rn(a * sm.rinv[h]);
+    }
+  }
+  cluster_sync();
+}
+
+template <int HD, int G>
+cudaError_t dispatch_tc(int M, int KV, const float* qkv, int S, size_t ps, KVView kv, RowMeta m, bf16* out,
+                        cudaStream_t st) {
+  constexpr int CS = 16;
+  constexpr int SMEM = (int)sizeof(TcSmem<HD, G>);
+  auto kern = k_attn_decode_tc<HD, G, CS>;
+  static int state = 0;
+  if (state == 0) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+      cudaGetLastError();
+      state = -1;
+    } else {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(CS);
+      cfg.blockDim = dim3(256);
+      cfg.dynamicSmemBytes = SMEM;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = CS;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      int n = 0;
+      state = (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0) ? 1 : -1;
+      cudaGetLastError();
+    }
+  }
+  if (state < 0) return cudaErrorNotSupported;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(M * KV * CS);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = CS;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = g_pdl ? 1 : 0;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
+  return cudaLaunchKernelEx(&cfg, kern, KV, qkv, S, ps, kv, m, out, scale_log2);
+}
+
 template <typename T, int HD, int G>
 cudaError_t dispatch_cl(int M, int KV, const float* qkv, int S, size_t ps, KVView kv, RowMeta m, T* out,
                         cudaStream_t st) {
@@ -525,6 +794,12 @@ cudaError_t dispatch_cl(int M, int KV, const float* qkv, int S, size_t ps, KVVie
 template <typename T, int HD, int G>
 cudaError_t dispatch(int M, int KV, const float* qkv, int S, size_t ps, KVView kv, RowMeta m, int max_ctx,
                      float* part, int nb_cap, unsigned* counters, T* out, cudaStream_t st) {
+  if constexpr (sizeof(T) == 2 && HD >= 64 && G <= 16) {
+    if (g_attn_cluster) {
+      cudaError_t e = dispatch_tc<HD, G>(M, KV, qkv, S, ps, kv, m, (bf16*)out, st);
+      if (e != cudaErrorNotSupported) return e;
+    }
+  }
   if (g_attn_cluster) {
     cudaError_t e = dispatch_cl<T, HD, G>(M, KV, qkv, S, ps, kv, m, out, st);
     if (e != cudaErrorNotSupported) return e;
