@@ -484,6 +484,12 @@ __global__ void __launch_bounds__(256) k_attn_decode_cl(int KV, const float* __r
 // cluster's blocks merge in rank order through distributed shared memory.
 constexpr int TC_KC = 192;  // keys per shared-memory sub-chunk
 
+__device__ __forceinline__ void dsmem_st(float* local, int rank, float v) {
+  uint32_t a = saddr(local), ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
+}
+
 template <int HD, int G>
 struct TcSmem {
   uint8_t q[16 * HD * 2];
@@ -492,6 +498,7 @@ struct TcSmem {
   float wm[NW][G], wl[NW][G];
   float wacc[NW][G][HD];
   float part[G][HD + 2];
+  float all[16][G][HD + 2];  // rank 0: every rank's partial, pushed by the ranks
   float rw[16][G];
   float rinv[G];
 };
@@ -521,8 +528,10 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
   const bf16* Vc = (const bf16*)kv.V + ((size_t)seq * KV + g) * kv.cap * HD;
 
   // Q tile: rows 0..G-1 = the G heads (pre-scaled, bf16), rows G..15 zero
-  for (int i = tid; i < 16 * HD; i += blockDim.x) {
-    const int h = i / HD, d = i % HD;
+  // (unrolled: every partial load of the tile is in flight at once)
+#pragma unroll
+  for (int it = 0; it < 16 * HD / 256; ++it) {
+    const int i = tid + it * 256, h = i / HD, d = i % HD;
     float val = 0.f;
     if (h < G && row_ok) val = sum_splits(qkv + (size_t)r * ld + (g * G + h) * HD + d, S, ps) * scale_log2;
     *reinterpret_cast<bf16*>(sm.q + swz<HD>(h, d / 8) + (d % 8) * 2) = __float2bfloat16_rn(val);
@@ -564,6 +573,7 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
     }
     cp_async_commit();
     const int jc0 = max(c0, p0);
+#pragma unroll 4
     for (int i = tid; i < (c1 - jc0 + 1) * HD; i += blockDim.x) {
       const int jj = i / HD, d = i % HD, row = jc0 - c0 + jj;
       const float* src = qkv + (size_t)(base + (jc0 + jj - p0)) * ld + qd + g * HD + d;
@@ -670,17 +680,23 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
     for (int ww = 0; ww < NW; ++ww) a += sm.wacc[ww][h][d] * sm.wm[ww][h];
     sm.part[h][2 + d] = a;
   }
-  cluster_sync();
+  __syncthreads();
+  // push this block's partial into rank 0's shared memory (stores only)
+  for (int i = tid; i < G * (HD + 2); i += blockDim.x) {
+    const int h = i / (HD + 2), c = i % (HD + 2);
+    dsmem_st(&sm.all[rank][h][c], 0, sm.part[h][c]);
+  }
+  cluster_sync();  // every partial has landed in rank 0
   if (rank == 0 && row_ok) {
     if (tid < G) {
       float M = -FLT_MAX;
-      for (int q = 0; q < CS; ++q) M = fmaxf(M, dsmem_ld(&sm.part[tid][0], q));
+      for (int q = 0; q < CS; ++q) M = fmaxf(M, sm.all[q][tid][0]);
       float L = 0.f;
       for (int q = 0; q < CS; ++q) {
-        const float mq = dsmem_ld(&sm.part[tid][0], q);
+        const float mq = sm.all[q][tid][0];
         const float wq = mq == -FLT_MAX ? 0.f : exp2f(mq - M);
         sm.rw[q][tid] = wq;
-        L += dsmem_ld(&sm.part[tid][1], q) * wq;
+        L += sm.all[q][tid][1] * wq;
       }
       sm.rinv[tid] = 1.f / L;
     }
@@ -688,11 +704,10 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
     for (int i = tid; i < G * HD; i += blockDim.x) {
       const int h = i / HD, d = i % HD;
       float a = 0.f;
-      for (int q = 0; q < CS; ++q) a += dsmem_ld(&sm.part[h][2 + d], q) * sm.rw[q][h];
+      for (int q = 0; q < CS; ++q) a += sm.all[q][h][2 + d] * sm.rw[q][h];
       out[(size_t)r * qd + (g * G + h) * HD + d] = __float2bfloat16_rn(a * sm.rinv[h]);
     }
   }
-  cluster_sync();
 }
 
 template <int HD, int G>
