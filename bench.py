@@ -354,9 +354,9 @@ def main():
         # ---- CPU oracle baseline (bounded sample)
         if rank == 0 and w_np is not None:
             if host_mem_gb() > 40:
-                rate, secs = oracle_decode_rate(shape, w_np, args.k, args.mode, 8, 3)
+                rate, secs = oracle_decode_rate(shape, w_np, args.k, args.mode, 8, 48)
                 cpu = {"value": round(rate, 4), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                       "sample": f"float32 oracle, 4B shape, 8-token prompt then 3 greedy decode steps at "
+                       "sample": f"float32 oracle, 4B shape, 8-token prompt then 48 greedy decode steps at "
                                  f"k={args.k} {args.mode} ({secs:.1f} s timed)"}
             else:
                 cpu = {"value": None, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
