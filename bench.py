@@ -173,7 +173,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--gemm-impl", dest="gemm_variant", type=int, default=2,
-                    help="--kernel gemm: 2 tcgen05 (default stages), 3 tcgen05 one sub-tile per stage, 1 SIMT")
+                    help="--kernel gemm: 2 tcgen05 (default stages), 3 tcgen05 one sub-tile per stage, "
+                         "4 tcgen05 with packed weights, 1 SIMT")
     ap.add_argument("--prompt", type=int, default=2560)
     ap.add_argument("--k", type=int, default=2)
     ap.add_argument("--mode", default="last_loop", choices=["last_loop", "per_loop"])
@@ -411,17 +412,26 @@ def gemm_probe(args):
         copies = max(2, -(-512_000_000 // wbytes))
         g = torch.Generator(device="cuda").manual_seed(0)
         Ws = [(torch.randn((N, K), generator=g, device="cuda") * 0.02).to(torch.bfloat16) for _ in range(copies)]
+        if args.gemm_variant == 4:  # packed tile layout
+            Ws = [dory.pack_weight_bf16(w) for w in Ws]
         X = torch.randn((args.m, K), generator=g, device="cuda").to(torch.bfloat16)
         Y = torch.empty((8, args.m, N), dtype=torch.float32, device="cuda")
         S = 1
         for i in range(3):
             S = dory.gemm_bf16_into(X, Ws[i % copies], Y, 1, True, args.gemm_variant)
         torch.cuda.synchronize()
+        # replay the launches from a CUDA graph so the host does not pace them
         iters = max(30, 3 * copies)
+        side = torch.cuda.Stream()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            for i in range(iters):
+                dory.gemm_bf16_into(X, Ws[i % copies], Y, 1, True, args.gemm_variant, stream=side)
+        graph.replay()
+        torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        for i in range(iters):
-            dory.gemm_bf16_into(X, Ws[i % copies], Y, 1, True, args.gemm_variant)
+        graph.replay()
         b.record()
         torch.cuda.synchronize()
         us = 1e3 * a.elapsed_time(b) / iters
@@ -430,7 +440,7 @@ def gemm_probe(args):
                      "frac_of_measured": round(by / us / 1e3 / hbm, 4)}
         del Ws
     print(json.dumps({"kernel": "gemm_tc", "impl": args.gemm_variant, "m": args.m, "results": out,
-                      "note": "back-to-back launches (no PDL overlap), weights cold in L2"}))
+                      "note": "graph-replayed back-to-back launches, weights cold in L2"}))
 
 
 def run_reference(args, shape, workload):

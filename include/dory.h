@@ -212,7 +212,8 @@ dory_status dory_read_kv(dory_handle* h, int32_t layer, int32_t slot, int32_t se
  * decode path uses for that many sequences; invariant != 0 makes each row's
  * arithmetic independent of M.  impl: 0 auto, 1 SIMT kernel, 2 tcgen05 only
  * (DORY_ERR_CUDA if the shape is unsupported), 3 tcgen05 with one 64-column
- * sub-tile per pipeline stage (comparison variant).  err_word (device int, may be
+ * sub-tile per pipeline stage (comparison variant), 4 tcgen05 with W in the
+ * packed tile layout of dory_pack_weight_bf16.  err_word (device int, may be
  * NULL) receives DORY_ERR_TIMEOUT-class codes from bounded waits.  Queues work
  * on `stream`; no handle needed. */
 dory_status dory_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* X, const void* W, float* Y,
@@ -236,6 +237,15 @@ dory_status dory_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* X, const
  * each other's results, so serialise them.  Queues work on `stream`. */
 dory_status dory_gemm_bf16_noalloc(int32_t M, int32_t N, int32_t K, const void* X, const void* W, float* Y,
                                    int32_t batch_hint, dory_stream stream);
+
+/* Repack a row-major [N, K] bf16 weight (device src, 16-byte aligned,
+ * N % 128 == 0, K % 64 == 0) into device dst (N*K*2 bytes, distinct from src)
+ * in the packed tile layout: 128-row x 64-column tiles, each stored as its
+ * 16 KB shared-memory image with 128-byte swizzle (row r's 16-byte chunk c at
+ * byte r*128 + (c XOR (r mod 8))*16), tile (n, k) at ((n*K/64) + k) * 16 KB.
+ * The tensor-core GEMM streams packed weights with one bulk copy per pipeline
+ * stage.  Queues work on `stream`. */
+dory_status dory_pack_weight_bf16(const void* src, void* dst, int32_t N, int32_t K, dory_stream stream);
 
 /* Synchronise `stream` and report device-side errors (DORY_ERR_TIMEOUT when
  * a bounded wait in a kernel gave up; the handle stays usable). */

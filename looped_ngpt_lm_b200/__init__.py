@@ -35,7 +35,7 @@ STATUS = {0: "DORY_OK", 1: "DORY_ERR_INVALID_ARG", 2: "DORY_ERR_CAPACITY", 3: "D
 SYMBOLS = ["dory_workspace_size", "dory_create", "dory_destroy", "dory_reset", "dory_prefill",
            "dory_decode_step", "dory_spec_decode", "dory_kv_bytes", "dory_seq_len", "dory_read_state",
            "dory_read_kv", "dory_synchronize", "dory_set_option", "dory_profile_read", "dory_profile_reset",
-           "dory_last_error", "dory_gemm_bf16", "dory_gemm_bf16_noalloc"]
+           "dory_last_error", "dory_gemm_bf16", "dory_gemm_bf16_noalloc", "dory_pack_weight_bf16"]
 
 
 class DoryError(RuntimeError):
@@ -86,6 +86,7 @@ def _load() -> ctypes.CDLL:
         "dory_profile_reset": [P],
         "dory_gemm_bf16": [I32, I32, I32, P, P, P, I32, I32, I32, IP, P, P],
         "dory_gemm_bf16_noalloc": [I32, I32, I32, P, P, P, I32, P],
+        "dory_pack_weight_bf16": [P, P, I32, I32, P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -185,6 +186,16 @@ def gemm_bf16_into(X, W, Y, batch_hint=1, invariant=True, impl=0, err=None, stre
                               ctypes.c_void_p(Y.data_ptr()), batch_hint, int(invariant), impl, ctypes.byref(s),
                               ctypes.c_void_p(_ptr(err)), _stream(stream)))
     return s.value
+
+
+def pack_weight_bf16(W, stream=None):
+    """Packed tile layout copy of a row-major [N, K] bf16 CUDA tensor."""
+    import torch
+    N, K = W.shape
+    out = torch.empty((N, K), dtype=torch.bfloat16, device=W.device)
+    _check(lib.dory_pack_weight_bf16(ctypes.c_void_p(W.data_ptr()), ctypes.c_void_p(out.data_ptr()), N, K,
+                                     _stream(stream)))
+    return out
 
 
 def workspace_size(cfg: Config, alloc_mode=LAST_LOOP) -> int:

@@ -919,7 +919,8 @@ dory_status dory_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* X, const
     int S = 1;
     size_t ps = 0;
     cudaError_t e = launch_gemm_tc(M, N, K, (const bf16*)X, K, (const bf16*)W, Y, N, (size_t)M, err_word,
-                                   batch_hint < 1 ? 1 : batch_hint, invariant != 0, &S, &ps, st, impl == 3 ? 1 : 0);
+                                   batch_hint < 1 ? 1 : batch_hint, invariant != 0, &S, &ps, st, impl == 3 ? 1 : 0,
+                                   nullptr, impl == 4);
     if (e == cudaSuccess) {
       *splits = S;
       return DORY_OK;
@@ -927,6 +928,14 @@ dory_status dory_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* X, const
     if (e != cudaErrorNotSupported || impl >= 2) return fail(DORY_ERR_CUDA, "tcgen05 GEMM: %s", cudaGetErrorString(e));
   }
   CK(launch_gemm_simt<bf16>(M, N, K, (const bf16*)X, K, (const bf16*)W, Y, N, st));
+  return DORY_OK;
+}
+
+dory_status dory_pack_weight_bf16(const void* src, void* dst, int32_t N, int32_t K, dory_stream stream) {
+  if (!src || !dst || N < 1 || K < 1) return fail(DORY_ERR_INVALID_ARG, "bad pack arguments");
+  if (N % 128 || K % 64) return fail(DORY_ERR_UNSUPPORTED, "packing needs N %% 128 == 0 and K %% 64 == 0");
+  if (((uintptr_t)src & 15) || ((uintptr_t)dst & 15)) return fail(DORY_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  CK(launch_pack_weight((const bf16*)src, dst, N, K, (cudaStream_t)stream));
   return DORY_OK;
 }
 

@@ -21,6 +21,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cstring>
 #include <mutex>
 #include <unordered_map>
 
@@ -94,6 +95,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
       " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
       "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+
+// Untiled bulk copy global -> shared (16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
 }
 
@@ -186,12 +196,24 @@ struct UnitMap {
   }
 };
 
-template <int NG, int GN, int KSUB, int BUDGET>
+// PACK: the weights are in the packed tile layout (see dory_pack_weight_bf16):
+// 128 x 64 tiles stored as their 16 KB swizzled shared-memory image, tiles
+// of one 128-row band consecutive along K, so a stage is one bulk copy.
+template <int NG, int GN, int KSUB, int BUDGET, bool PACK>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, float* Y, int ldy,
-              size_t part_stride, int M, UnitMap um, unsigned* tile_counters, int* err) {
+              size_t part_stride, int M, UnitMap um, unsigned* tile_counters, int* err, const uint8_t* Apack,
+              int k_tiles) {
   using TL = Tile<NG, GN, KSUB, BUDGET>;
   constexpr int STAGES = TL::STAGES;
+  auto load_a = [&](uint8_t* sa, uint64_t* bar, int nt, int kb, uint64_t pol) {
+    if constexpr (PACK) {
+      bulk_load(sa, Apack + ((size_t)nt * k_tiles + (size_t)kb * KSUB) * TL::A_SUB, TL::A_BYTES, bar, pol);
+    } else {
+#pragma unroll
+      for (int q = 0; q < KSUB; ++q) tma_load_2d(sa + q * TL::A_SUB, &mapA, bar, (kb * KSUB + q) * BK, nt * BM, pol);
+    }
+  };
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* full = (uint64_t*)(smem + STAGES * TL::STAGE);
@@ -219,7 +241,7 @@ __global__ void __launch_bounds__(192, 1)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == 0 && lane == 0) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(&mapA) : "memory");
+    if (!PACK) asm volatile("prefetch.tensormap [%0];" ::"l"(&mapA) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(&mapB) : "memory");
   }
   if (warp == 1) {
@@ -254,9 +276,7 @@ __global__ void __launch_bounds__(192, 1)
       while (npre < STAGES && u < um.units) {
         uint8_t* sa = smem + npre * TL::STAGE;
         mbar_expect_tx(&full[npre], TL::STAGE);
-#pragma unroll
-        for (int q = 0; q < KSUB; ++q)
-          tma_load_2d(sa + q * TL::A_SUB, &mapA, &full[npre], (kb * KSUB + q) * BK, nt * BM, pol_w);
+        load_a(sa, &full[npre], nt, kb, pol_w);
         pre_kb[npre] = kb;
         pre_mt[npre] = mt;
         ++npre;
@@ -275,12 +295,10 @@ __global__ void __launch_bounds__(192, 1)
         ++issued;
         uint8_t* sa = smem + stage * TL::STAGE;
         mbar_expect_tx(&full[stage], TL::STAGE);
+        load_a(sa, &full[stage], nt, kb, pol_w);
 #pragma unroll
-        for (int q = 0; q < KSUB; ++q) {
-          tma_load_2d(sa + q * TL::A_SUB, &mapA, &full[stage], (kb * KSUB + q) * BK, nt * BM, pol_w);
-          tma_load_2d(sa + TL::A_BYTES + q * TL::B_SUB, &mapB, &full[stage], (kb * KSUB + q) * BK, mt * TL::MT,
-                      pol_x);
-        }
+        for (int q = 0; q < KSUB; ++q)
+          tma_load_2d(sa + TL::A_BYTES + q * TL::B_SUB, &mapB, &full[stage], (kb * KSUB + q) * BK, mt * TL::MT, pol_x);
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1;
@@ -495,22 +513,22 @@ int sm_count() {
   return n;
 }
 
-template <int NG, int GN, int KSUB, int BUDGET = kDecodeBudget>
+template <int NG, int GN, int KSUB, int BUDGET = kDecodeBudget, bool PACK = false>
 cudaError_t run(const CUtensorMap& ma, const bf16* X, int ldx, int M, int K, float* Y, int ldy, size_t ps,
-                UnitMap um, unsigned* tile_counters, int* err, cudaStream_t st) {
+                UnitMap um, unsigned* tile_counters, int* err, cudaStream_t st, const void* Apack = nullptr) {
   using TL = Tile<NG, GN, KSUB, BUDGET>;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e =
-        cudaFuncSetAttribute(k_gemm_tc<NG, GN, KSUB, BUDGET>, cudaFuncAttributeMaxDynamicSharedMemorySize, TL::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<NG, GN, KSUB, BUDGET, PACK>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, TL::SMEM);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   CUtensorMap mb;
   if (!make_map(&mb, X, M, K, ldx, TL::MT)) return cudaErrorInvalidValue;
   int grid = um.units < sm_count() ? um.units : sm_count();
-  return launch(k_gemm_tc<NG, GN, KSUB, BUDGET>, dim3(grid), dim3(192), TL::SMEM, st, ma, mb, Y, ldy, ps, M, um,
-                tile_counters, err);
+  return launch(k_gemm_tc<NG, GN, KSUB, BUDGET, PACK>, dim3(grid), dim3(192), TL::SMEM, st, ma, mb, Y, ldy, ps, M,
+                um, tile_counters, err, (const uint8_t*)Apack, K / BK);
 }
 
 // Split factor for the decode tiles: chosen from (N, K, batch) only, never
@@ -540,17 +558,37 @@ int choose_split(int N, int K, int batch, int kstages) {
   return best;
 }
 
+__global__ void k_pack_weight(const bf16* __restrict__ src, uint8_t* __restrict__ dst, int N, int K) {
+  const size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;  // 16-byte chunk of the source
+  if (i >= (size_t)N * K / 8) return;
+  const int kc = K / 8;
+  const int n = (int)(i / kc), c8 = (int)(i % kc);
+  const int nt = n / BM, r = n % BM, kt = c8 / 8, c = c8 % 8;
+  const size_t off = ((size_t)nt * (K / BK) + kt) * (BM * BK * 2) + r * 128 + ((c ^ (r & 7)) << 4);
+  *reinterpret_cast<uint4*>(dst + off) = *reinterpret_cast<const uint4*>(src + (size_t)n * K + (size_t)c8 * 8);
+}
+
 }  // namespace
+
+cudaError_t launch_pack_weight(const bf16* W, void* dst, int N, int K, cudaStream_t st) {
+  if (N % BM || K % BK || ((uintptr_t)W & 15) || ((uintptr_t)dst & 15)) return cudaErrorInvalidValue;
+  const size_t chunks = (size_t)N * K / 8;
+  k_pack_weight<<<(unsigned)((chunks + 255) / 256), 256, 0, st>>>(W, (uint8_t*)dst, N, K);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf16* W, float* Y, int ldy,
                            size_t part_rows, int* err, int batch, bool invariant, int* S_out, size_t* ps_out,
-                           cudaStream_t st, int variant, unsigned* tile_counters) {
+                           cudaStream_t st, int variant, unsigned* tile_counters, bool packed) {
   *S_out = 1;
   *ps_out = 0;
   if (M <= 0 || N % BM || K % BK || ldx % 8 || (size_t)M > part_rows || ((uintptr_t)X & 15) || ((uintptr_t)W & 15))
     return cudaErrorNotSupported;
   CUtensorMap ma;
-  if (!weight_map(&ma, W, N, K)) return cudaErrorNotSupported;
+  if (packed)
+    memset(&ma, 0, sizeof ma);
+  else if (!weight_map(&ma, W, N, K))
+    return cudaErrorNotSupported;
   UnitMap um;
   um.n_tiles = N / BM;
   if (invariant || M <= 128) {
@@ -572,7 +610,9 @@ cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf
     unsigned* tc = (S > 1 && tile_counters && um.n_tiles * um.m_tiles <= kTileCounters) ? tile_counters : nullptr;
     *S_out = tc ? 1 : S;  // reduced in the kernel: one slice for the consumer
     *ps_out = tc ? 0 : ps;
-#define DORY_RUN(NGV, KS) return run<NGV, 16, KS>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st)
+#define DORY_RUN(NGV, KS)                                                                            \
+  return packed ? run<NGV, 16, KS, kDecodeBudget, true>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st, W) \
+                : run<NGV, 16, KS>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st)
     if (NG == 1) {
       if (ksub == 4) DORY_RUN(1, 4);
       if (ksub == 2) DORY_RUN(1, 2);
@@ -595,6 +635,7 @@ cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf
   um.S = 1;
   um.m_tiles = (M + 255) / 256;
   um.units = um.n_tiles * um.m_tiles;
+  if (packed) return run<1, 256, 1, 200 * 1024, true>(ma, X, ldx, M, K, Y, ldy, 0, um, nullptr, err, st, W);
   return run<1, 256, 1, 200 * 1024>(ma, X, ldx, M, K, Y, ldy, 0, um, nullptr, err, st);
 }
 

@@ -23,8 +23,17 @@ constexpr int kTileCounters = 4096;
 // 64-column sub-tile per pipeline stage (for comparisons).  With
 // tile_counters (kTileCounters zeros), the last split of each output tile
 // adds the slices in order s = 0..S-1 inside the kernel and *S is 1.
+// packed: W is in the packed tile layout below.
 cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf16* W, float* Y, int ldy,
                            size_t part_rows, int* err, int batch, bool invariant, int* S, size_t* part_stride,
-                           cudaStream_t st, int variant = 0, unsigned* tile_counters = nullptr);
+                           cudaStream_t st, int variant = 0, unsigned* tile_counters = nullptr,
+                           bool packed = false);
+
+// Repack a row-major [N, K] bf16 weight (N % 128 == 0, K % 64 == 0) into the
+// packed tile layout the tensor-core GEMM streams with bulk copies: 128 x 64
+// tiles, each stored as its 16 KB 128-byte-swizzled shared-memory image
+// (row r's 16-byte chunk c at r*128 + (c ^ (r % 8))*16), tile (n, k) at
+// ((n * K/64) + k) * 16 KB.  dst holds N*K*2 bytes.
+cudaError_t launch_pack_weight(const bf16* W, void* dst, int N, int K, cudaStream_t st);
 
 }  // namespace dory

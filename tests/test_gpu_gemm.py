@@ -66,3 +66,14 @@ def test_stage_width_does_not_change_bits(M, N, K):
     a, s1 = dory.gemm_bf16(X, W, batch_hint=1, invariant=True, impl=2)
     b, s2 = dory.gemm_bf16(X, W, batch_hint=1, invariant=True, impl=3)
     assert s1 == s2 and torch.equal(a, b)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 2560, 10240), (3, 3584, 2560), (20, 20480, 2560), (300, 1024, 512)])
+def test_packed_weights_same_bits(M, N, K):
+    """Weights in the packed tile layout (bulk copies) give the same bits as
+    row-major weights read through tensor maps."""
+    X, W = operands(M, N, K, 4)
+    Wp = dory.pack_weight_bf16(W)
+    a, s1 = dory.gemm_bf16(X, W, batch_hint=1, invariant=M <= 128, impl=2)
+    b, s2 = dory.gemm_bf16(X, Wp, batch_hint=1, invariant=M <= 128, impl=4)
+    assert s1 == s2 and torch.equal(a, b)
