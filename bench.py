@@ -130,6 +130,116 @@ class Clocks:
 
 
 # ---------------------------------------------------------------- CPU oracle
+def sweep_modes(dory, torch, shape, dw, args, prompt_len=128, n_new=256):
+    """Batch 1, 128-token prompt, greedy decode at k = 1/2/4 in both cache
+    modes: tokens/s, KV bytes per token, and how far last_loop logits drift
+    from per_loop logits on the same tokens (teacher-forced)."""
+    import synth
+    cfg = dory.make_config(shape, max_batch=2, max_seq=prompt_len + n_new + 8, k_max=4, gamma_max=4,
+                           max_chunk=prompt_len)
+    h = dory.Handle(cfg, dw, dory.PER_LOOP)
+    prompt = torch.tensor(synth.make_prompt(2, prompt_len, shape.vocab), dtype=torch.int32, device="cuda")
+    out = {}
+    for k in (1, 2, 4):
+        toks = {}
+        for mode in ("last_loop", "per_loop"):
+            md = dory.MODES[mode]
+            seq = 0 if mode == "last_loop" else 1
+            h.reset(seq)
+            t = h.prefill([seq], prompt, [prompt_len], k, md)
+            bufs = [torch.empty(1, dtype=torch.int32, device="cuda") for _ in range(2)]
+            for i in range(3):
+                t = h.decode_step([seq], t, k, md, next_tokens=bufs[i % 2])
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            n = n_new - 4
+            for i in range(n):
+                t = h.decode_step([seq], t, k, md, next_tokens=bufs[i % 2])
+            b.record()
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / n
+            ctx = h.seq_len(seq)
+            out[f"k{k}_{mode}"] = {"tokens_per_s": round(1e3 / ms, 2),
+                                   "kv_bytes_per_token": round(h.kv_bytes(k, md, ctx) / ctx, 1), "ctx": ctx}
+        # logits drift: replay one greedy last_loop run in both modes on the same tokens
+        lg = {m: [] for m in ("last_loop", "per_loop")}
+        tok_seq = []
+        for mode in ("last_loop", "per_loop"):
+            md = dory.MODES[mode]
+            seq = 0 if mode == "last_loop" else 1
+            h.reset(seq)
+            L = torch.empty((1, shape.vocab), device="cuda")
+            t = h.prefill([seq], prompt, [prompt_len], k, md, logits=L)
+            lg[mode].append(L[0].clone())
+            for i in range(31):
+                if mode == "last_loop":
+                    tok_seq.append(int(t[0]))
+                inp = torch.tensor([tok_seq[i]], dtype=torch.int32, device="cuda")
+                t = h.decode_step([seq], inp, k, md, logits=L)
+                lg[mode].append(L[0].clone())
+        A, B = torch.stack(lg["last_loop"]), torch.stack(lg["per_loop"])
+        drift = ((A - B).norm(dim=1) / B.norm(dim=1)).cpu()
+        agree = (A.argmax(1) == B.argmax(1)).float().mean().item()
+        out[f"k{k}_logits_drift"] = {"rel_l2_max": round(float(drift.max()), 5), "rel_l2_mean": round(float(drift.mean()), 5),
+                                     "argmax_agreement": round(agree, 4), "steps": int(A.shape[0])}
+    h.close()
+    return out
+
+
+def spec_leg(dory, torch, shape, dw, args, prompt_len=512, n_new=128, gamma=4):
+    """Self-speculative decoding (draft k=1, verify k=4, gamma=4, last_loop)
+    at batch 1, 4 and 16 against plain k=4 greedy decoding of the same
+    prompts: accepted draft tokens per verify step, output tokens/s, speed-up,
+    and agreement with the plain k=4 tokens."""
+    import synth
+    res = {}
+    for B in (1, 4, 16):
+        cfg = dory.make_config(shape, max_batch=2 * B, max_seq=prompt_len + n_new + 2 * gamma + 8, k_max=4,
+                               gamma_max=gamma, max_chunk=2 * B * prompt_len)
+        h = dory.Handle(cfg, dw, dory.LAST_LOOP)
+        prompts = [synth.make_prompt(100 + b, prompt_len, shape.vocab) for b in range(B)]
+        tok = torch.tensor(np.concatenate(prompts), dtype=torch.int32, device="cuda")
+        md = dory.LAST_LOOP
+        # plain k=4
+        ids = list(range(B))
+        first = h.prefill(ids, tok, [prompt_len] * B, 4, md)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t = first
+        plain = [t.clone()]
+        a.record()
+        for i in range(n_new - 1):
+            t = h.decode_step(ids, t, 4, md)
+            plain.append(t.clone())
+        b.record()
+        torch.cuda.synchronize()
+        plain_ms = a.elapsed_time(b)
+        plain_tok = torch.stack(plain, 1).cpu()
+        # speculative on other sequence slots
+        sids = list(range(B, 2 * B))
+        first = h.prefill(sids, tok, [prompt_len] * B, 4, md)
+        torch.cuda.synchronize()
+        a.record()
+        out, out_len, st = h.spec_decode(sids, first, 1, 4, gamma, md, n_new - 1)
+        b.record()
+        torch.cuda.synchronize()
+        spec_ms = a.elapsed_time(b)
+        spec_tok = torch.cat([first.cpu()[:, None], out.cpu()], 1)
+        agree = (spec_tok == plain_tok).float().mean().item()
+        res[f"batch{B}"] = {
+            "accepted_per_verify_step": round(st["accepted"] / max(st["steps"] * B, 1), 3),
+            "tokens_per_verify_step": round((B * (n_new - 1)) / max(st["steps"] * B, 1), 3),
+            "spec_tokens_per_s": round(B * (n_new - 1) / (spec_ms / 1e3), 1),
+            "plain_k4_tokens_per_s": round(B * (n_new - 1) / (plain_ms / 1e3), 1),
+            "speedup_vs_plain_k4": round(plain_ms / spec_ms, 3),
+            "token_agreement_with_plain_k4": round(agree, 4),
+        }
+        h.close()
+    res["workload"] = f"prompt {prompt_len}, {n_new} output tokens, gamma {gamma}, last_loop, greedy"
+    return res
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -362,6 +472,10 @@ def main():
             else:
                 cpu = {"value": None, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                        "sample": f"skipped: {host_mem_gb():.0f} GB host memory available, the fp32 oracle needs ~40"}
+
+    if not args.no_aux and world == 1:
+        aux["k_mode_sweep"] = sweep_modes(dory, torch, shape, dw, args)
+        aux["spec_decode"] = spec_leg(dory, torch, shape, dw, args)
 
     if rank == 0:
         line = {

@@ -117,7 +117,8 @@ struct dory_handle {
   float *h = nullptr, *x = nullptr, *s = nullptr, *q = nullptr, *part_qkv = nullptr, *part_y = nullptr,
         *part_gu = nullptr, *attn_part = nullptr, *logits = nullptr;
   void *hop = nullptr, *ao = nullptr, *act = nullptr, *kscr = nullptr, *vscr = nullptr, *hop_head = nullptr;
-  size_t part_rows = 0;
+  size_t part_rows = 0;      // rows of an unsplit GEMM output (prefill)
+  size_t part_rows_dec = 0;  // rows per split slice on the decode / speculative path
   float *stash_x = nullptr, *stash_s = nullptr;
   int *drafts = nullptr, *pending = nullptr, *vtok = nullptr, *out_len = nullptr, *all_done = nullptr;
   unsigned long long* accepted = nullptr;
@@ -241,10 +242,14 @@ size_t layout(dory_handle* h) {
   h->kscr = cv.take<char>(e * M * h->kv_dim);
   h->vscr = cv.take<char>(e * M * h->kv_dim);
   h->hop_head = cv.take<char>(e * h->head_max * d);
-  h->part_rows = (size_t)M;  // rows per split slice; kMaxSplitK slices each
-  h->part_qkv = cv.take<float>(sizeof(float) * kMaxSplitK * h->part_rows * h->qkv_dim);
-  h->part_y = cv.take<float>(sizeof(float) * kMaxSplitK * h->part_rows * d);
-  h->part_gu = cv.take<float>(sizeof(float) * kMaxSplitK * h->part_rows * 2 * c.d_ff);
+  // Split-K slices are used only by decode / speculative rows (at most
+  // max_batch * (gamma_max + 1)); long prefill chunks never split K.
+  h->part_rows_dec = (size_t)std::max(c.max_batch, c.max_batch * (c.gamma_max + 1));
+  h->part_rows = (size_t)M;
+  const size_t prow = std::max((size_t)kMaxSplitK * h->part_rows_dec, (size_t)M);
+  h->part_qkv = cv.take<float>(sizeof(float) * prow * h->qkv_dim);
+  h->part_y = cv.take<float>(sizeof(float) * prow * d);
+  h->part_gu = cv.take<float>(sizeof(float) * prow * 2 * c.d_ff);
   h->attn_part = cv.take<float>(sizeof(float) * (size_t)M * c.n_heads * h->nb_cap * (c.head_dim + 4));
   h->attn_counters = cv.take<unsigned>(sizeof(unsigned) * (size_t)M * c.n_kv_heads);
   h->tile_counters = cv.take<unsigned>(sizeof(unsigned) * kTileCounters);
@@ -325,6 +330,12 @@ KVView kv_view(dory_handle* H, int l, int loop, int mode) {
   return v;
 }
 
+// Rows per split slice of a GEMM output buffer for this pass.
+template <typename T>
+size_t prows(const Fwd<T>& f) {
+  return f.invariant ? f.H->part_rows_dec : f.H->part_rows;
+}
+
 // Y (and, when the tensor-core kernel splits K, the slices after it) must
 // hold kMaxSplitK slices of part_rows rows of ldy floats.
 template <typename T>
@@ -372,7 +383,7 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop, float* copy_la
     size_t ps;
     if (layer_is_attn(l)) {
       KVView kv = kv_view(H, l, loop, f.mode);
-      RET(gemm<T>(f, M, H->qkv_dim, d, H->hop_t<T>(), d, H->w_qkv[l], H->part_qkv, H->qkv_dim, H->M_max, &S, &ps, "gemm_qkv"));
+      RET(gemm<T>(f, M, H->qkv_dim, d, H->hop_t<T>(), d, H->w_qkv[l], H->part_qkv, H->qkv_dim, prows(f), &S, &ps, "gemm_qkv"));
       if (f.direct) {
         // fused: q from the partials, own K/V into the cache, split-KV attention
         Scope sc(H, f.st, "attn_decode", 0);
@@ -406,15 +417,15 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop, float* copy_la
                                  f.st));
         }
       }
-      RET(gemm<T>(f, M, d, H->q_dim, (const T*)H->ao, H->q_dim, H->w_o[l], H->part_y, d, H->M_max, &S, &ps, "gemm_o"));
+      RET(gemm<T>(f, M, d, H->q_dim, (const T*)H->ao, H->q_dim, H->w_o[l], H->part_y, d, prows(f), &S, &ps, "gemm_o"));
     } else {
-      RET(gemm<T>(f, M, 2 * c.d_ff, d, H->hop_t<T>(), d, H->w_gu[l], H->part_gu, 2 * c.d_ff, H->M_max,
+      RET(gemm<T>(f, M, 2 * c.d_ff, d, H->hop_t<T>(), d, H->w_gu[l], H->part_gu, 2 * c.d_ff, prows(f),
                   &S, &ps, "gemm_gate_up"));
       {
         Scope sc(H, f.st, "swiglu", 0);
         CK(launch_swiglu<T>(M, c.d_ff, H->part_gu, S, ps, (T*)H->act, f.st));
       }
-      RET(gemm<T>(f, M, d, c.d_ff, (const T*)H->act, c.d_ff, H->w_down[l], H->part_y, d, H->M_max, &S, &ps,
+      RET(gemm<T>(f, M, d, c.d_ff, (const T*)H->act, c.d_ff, H->w_down[l], H->part_y, d, prows(f), &S, &ps,
                   "gemm_down"));
     }
     Scope sc(H, f.st, "addnorm", 0);

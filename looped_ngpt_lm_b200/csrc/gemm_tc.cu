@@ -591,7 +591,7 @@ cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf
     return cudaErrorNotSupported;
   UnitMap um;
   um.n_tiles = N / BM;
-  if (invariant || M <= 128) {
+  if (invariant) {
     // decode / verify: 16-token MMA groups, split chosen from (N, K, batch).
     // Stages span 4 sub-tiles (512 contiguous bytes per weight row) when K
     // allows; variant 1 forces one sub-tile per stage.

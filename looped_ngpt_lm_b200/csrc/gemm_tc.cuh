@@ -15,9 +15,9 @@ constexpr int kTileCounters = 4096;
 // Y = X . W^T for X [M, K] (row stride ldx) and W [N, K], both bf16, fp32
 // accumulation.  Writes S partial products to Y + s * (*part_stride)
 // (row stride ldy); the consumer adds them in order s = 0..S-1.
-// invariant (or M <= 128): 16-token MMA groups and a split chosen from
-// (N, K, batch) only, so each row's result is bit-identical for every M;
-// otherwise 128 x 256 tiles without split.  part_rows: rows available per
+// invariant: 16-token MMA groups and a split chosen from (N, K, batch) only,
+// so each row's result is bit-identical for every M; otherwise 128 x 256
+// tiles without split.  part_rows: rows available per
 // slice (>= M).  Returns cudaErrorNotSupported for shapes the kernel does not
 // handle (N % 128, K % 64, unaligned pointers).  variant 1 forces one
 // 64-column sub-tile per pipeline stage (for comparisons).  With
