@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(256) k_attn_decode(int KV, const float* __rest
                                                      float scale_log2) {
   constexpr int DL = HD / 8;                    // dimensions per lane
   constexpr int CH = HD * (int)sizeof(T) / 16;  // 16-byte chunks per row
-  extern __shared__ __align__(16) uint8_t smem_raw[];
+  extern __shared__ __align__(128) uint8_t smem_raw[];
   DecSmem<T, HD, G>& sm = *reinterpret_cast<DecSmem<T, HD, G>*>(smem_raw);
 
   pdl_wait();
@@ -303,7 +303,7 @@ __global__ void __launch_bounds__(256) k_attn_decode_cl(int KV, const float* __r
                                                         float scale_log2) {
   constexpr int DL = HD / 8;
   constexpr int CH = HD * (int)sizeof(T) / 16;
-  extern __shared__ __align__(16) uint8_t smem_raw[];
+  extern __shared__ __align__(128) uint8_t smem_raw[];
   ClSmem<T, HD, G>& sm = *reinterpret_cast<ClSmem<T, HD, G>*>(smem_raw);
 
   pdl_wait();
