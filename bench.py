@@ -294,6 +294,9 @@ def main():
                     help="time one kernel alone instead of the decode step (prints its own JSON line)")
     ap.add_argument("--shape", default="qkv,o,gate_up,down,lm_head", help="GEMM shapes for --kernel gemm")
     ap.add_argument("--m", type=int, default=1, help="token rows for --kernel gemm")
+    ap.add_argument("--l2-lookahead-mb", dest="l2_mb", type=int, default=None,
+                    help="bytes of upcoming weights each decode GEMM prefetches into L2 (MiB; 0 = off; "
+                         "default: the library's)")
     ap.add_argument("--layers", default=None,
                     help="I,R,O physical layers (a narrower model of the same width, for small profiling captures)")
     args = ap.parse_args()
@@ -340,6 +343,8 @@ def main():
     max_seq = args.prompt + args.warmup + args.steps + args.profile_steps + 512
     cfg = dory.make_config(shape, max_batch=1, max_seq=max_seq, k_max=4, gamma_max=4, max_chunk=args.prompt)
     h = dory.Handle(cfg, dw, dory.LAST_LOOP if args.mode == "last_loop" else dory.PER_LOOP)
+    if args.l2_mb is not None:
+        h.set_option(dory.OPT_L2_LOOKAHEAD, args.l2_mb << 20)
     mode = dory.MODES[args.mode]
     stream = torch.cuda.current_stream()
     prompt = torch.tensor(synth.make_prompt(1, args.prompt, shape.vocab), dtype=torch.int32, device="cuda")

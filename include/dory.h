@@ -258,7 +258,12 @@ enum {
   DORY_OPT_GEMM_IMPL = 3,   /* bf16 GEMM: 0 auto, 1 SIMT reference kernel, 2 tcgen05 */
   DORY_OPT_PDL = 4,         /* 1 (default): programmatic dependent launches (process-wide) */
   DORY_OPT_PREFILL_TC = 5,  /* 1 (default): bf16 long-chunk attention on the tensor cores; 0: CUDA cores */
-  DORY_OPT_ATTN_CLUSTER = 6 /* 1 (default): decode attention as 16-block clusters (process-wide) */
+  DORY_OPT_ATTN_CLUSTER = 6, /* 1 (default): decode attention as 16-block clusters (process-wide) */
+  /* bf16 decode steps: bytes of upcoming weights each GEMM prefetches into L2
+   * past its own once its loads have landed (default 8 MiB; 0 turns the
+   * look-ahead off).  Changes only when HBM reads happen, never what is
+   * computed. */
+  DORY_OPT_L2_LOOKAHEAD = 7
 };
 dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value);
 

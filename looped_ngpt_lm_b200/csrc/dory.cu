@@ -125,6 +125,9 @@ struct dory_handle {
   unsigned* attn_counters = nullptr;  // [M_max * n_kv], zero between launches
   unsigned* tile_counters = nullptr;  // [kTileCounters], zero between launches
   int nb_cap = 0;                     // key blocks per row the partial buffer holds
+  // weight stream of a decode step at each loop count k (L2 look-ahead)
+  PfSeg* pf_segs = nullptr;           // [k_max][pf_nseg_max]
+  int pf_nseg_max = 0;
 
   // host state
   std::vector<int> len, mode, kfix;  // per sequence; mode -1 = empty
@@ -132,6 +135,11 @@ struct dory_handle {
   int last_rows = 0;
   bool graphs = true, profile = false, prefill_tc = true;
   int gemm_impl = 0;
+  unsigned long long pf_lead = 8ull << 20;   // 0: no L2 look-ahead
+  std::vector<std::vector<PfSeg>> pf_host;   // [k] -> stream of a k-loop decode step
+  std::vector<char> pf_uploaded;             // [k]
+  int pf_pos = -1;                           // next segment of the pass being issued; -1 off
+  unsigned long long pf_done = 0;            // stream bytes already handed out for prefetch
   std::vector<std::string> prof_names;
   std::vector<ProfRec> prof_recs;
   std::vector<cudaEvent_t> ev_pool;
@@ -263,6 +271,9 @@ size_t layout(dory_handle* h) {
   h->out_len = cv.take<int>(sizeof(int) * c.max_batch);
   h->all_done = cv.take<int>(sizeof(int) * 4);
   h->accepted = cv.take<unsigned long long>(sizeof(unsigned long long) * 2);
+  // two GEMMs per physical layer per application, plus the LM head
+  h->pf_nseg_max = 2 * (c.n_in + c.n_out + c.k_max * c.n_rec) + 1;
+  h->pf_segs = cv.take<PfSeg>(sizeof(PfSeg) * (size_t)c.k_max * h->pf_nseg_max);
   return cv.off + 256;
 }
 
@@ -315,6 +326,7 @@ struct Fwd {
   int batch;    // sequences in the call (selects the GEMM split)
   bool invariant;  // decode / speculative rows: GEMM arithmetic independent of M
   int n_tiles = 0;  // > 0: long-chunk attention on the tensor cores over H->tiles
+  int pf_k = 0;     // > 0: GEMMs follow the weight stream of a pf_k-loop decode step
 };
 
 KVView kv_view(dory_handle* H, int l, int loop, int mode) {
@@ -350,8 +362,32 @@ dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, cons
     if (H->gemm_impl != 1) {
       int S = 1;
       size_t ps = 0;
+      // L2 look-ahead while this GEMM is the next one of the weight stream
+      PfCtl pfc;
+      const PfCtl* pp = nullptr;
+      if (f.pf_k > 0 && H->pf_pos >= 0) {
+        const std::vector<PfSeg>& v = H->pf_host[f.pf_k];
+        if (H->pf_pos < (int)v.size() && v[H->pf_pos].p == (const char*)W) {
+          const unsigned long long end = v[H->pf_pos].off + v[H->pf_pos].bytes;
+          const unsigned long long total = v.back().off + v.back().bytes;
+          pfc.segs = H->pf_segs + (size_t)(f.pf_k - 1) * H->pf_nseg_max;
+          pfc.nseg = (int)v.size();
+          pfc.first = H->pf_pos + 1;
+          pfc.lo = std::max(H->pf_done, end);
+          pfc.hi = std::min(end + H->pf_lead, total);
+          if (pfc.lo < pfc.hi) {
+            // start the segment walk at the segment holding lo
+            while (pfc.first + 1 < pfc.nseg && v[pfc.first + 1].off <= pfc.lo) ++pfc.first;
+            H->pf_done = pfc.hi;
+            pp = &pfc;
+          }
+          ++H->pf_pos;
+        } else {
+          H->pf_pos = -1;  // the pass left the stream: no further look-ahead
+        }
+      }
       cudaError_t e = launch_gemm_tc(M, N, K, (const bf16*)X, ldx, (const bf16*)W, Y, ldy, part_rows,
-                                     H->err, f.batch, f.invariant, &S, &ps, f.st, 0, nullptr);
+                                     H->err, f.batch, f.invariant, &S, &ps, f.st, 0, nullptr, false, pp);
       if (e == cudaSuccess) {
         *S_out = S;
         *ps_out = ps;
@@ -419,9 +455,22 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop, float* copy_la
       }
       RET(gemm<T>(f, M, d, H->q_dim, (const T*)H->ao, H->q_dim, H->w_o[l], H->part_y, d, prows(f), &S, &ps, "gemm_o"));
     } else {
-      RET(gemm<T>(f, M, 2 * c.d_ff, d, H->hop_t<T>(), d, H->w_gu[l], H->part_gu, 2 * c.d_ff, prows(f),
-                  &S, &ps, "gemm_gate_up"));
-      {
+      bool fused = false;
+      if constexpr (sizeof(T) == 2) {
+        // long chunks: gate-up GEMM with SwiGLU in its epilogue
+        if (!f.invariant && H->gemm_impl != 1) {
+          Scope sc(H, f.st, "gemm_gate_up_glu", 4.0 * c.d_ff * d + 2.0 * M * d + 2.0 * M * c.d_ff);
+          cudaError_t e = launch_gemm_glu(M, c.d_ff, d, (const bf16*)H->hop, d, (const bf16*)H->w_gu[l],
+                                          (bf16*)H->act, H->err, f.st);
+          if (e == cudaSuccess)
+            fused = true;
+          else if (e != cudaErrorNotSupported)
+            return fail(DORY_ERR_CUDA, "gemm_gate_up_glu: %s", cudaGetErrorString(e));
+        }
+      }
+      if (!fused) {
+        RET(gemm<T>(f, M, 2 * c.d_ff, d, H->hop_t<T>(), d, H->w_gu[l], H->part_gu, 2 * c.d_ff, prows(f), &S, &ps,
+                    "gemm_gate_up"));
         Scope sc(H, f.st, "swiglu", 0);
         CK(launch_swiglu<T>(M, c.d_ff, H->part_gu, S, ps, (T*)H->act, f.st));
       }
@@ -582,11 +631,56 @@ dory_status prefill_t(dory_handle* H, int batch, const int32_t* seq_ids, const i
   return DORY_OK;
 }
 
+// The weights a k-loop decode step reads, in the order its GEMMs read them:
+// per physical layer QKV then O (attention) or gate-up then down (MLP); the
+// input block, k passes over the recurrent block, the output block, the LM
+// head.  Uploaded once per k (outside any graph capture).
+dory_status ensure_stream(dory_handle* H, int k, cudaStream_t st) {
+  if (H->pf_lead == 0 || !H->bf16 || H->gemm_impl == 1) return DORY_OK;
+  if ((int)H->pf_host.size() <= k) {
+    H->pf_host.resize(k + 1);
+    H->pf_uploaded.resize(k + 1, 0);
+  }
+  if (H->pf_uploaded[k]) return DORY_OK;
+  const dory_config& c = H->c;
+  const unsigned long long d = c.d_model, e = 2;
+  std::vector<PfSeg>& v = H->pf_host[k];
+  v.clear();
+  unsigned long long off = 0;
+  auto add = [&](const void* p, unsigned long long bytes) {
+    v.push_back({(const char*)p, off, bytes});
+    off += bytes;
+  };
+  auto layer = [&](int l) {
+    if (layer_is_attn(l)) {
+      add(H->w_qkv[l], (unsigned long long)H->qkv_dim * d * e);
+      add(H->w_o[l], d * H->q_dim * e);
+    } else {
+      add(H->w_gu[l], 2ull * c.d_ff * d * e);
+      add(H->w_down[l], d * c.d_ff * e);
+    }
+  };
+  for (int l = 0; l < c.n_in; ++l) layer(l);
+  for (int t = 1; t <= k; ++t)
+    for (int l = c.n_in; l < c.n_in + c.n_rec; ++l) layer(l);
+  for (int l = c.n_in + c.n_rec; l < H->L; ++l) layer(l);
+  add(H->head, (unsigned long long)c.vocab * d * e);
+  if ((int)v.size() > H->pf_nseg_max) return fail(DORY_ERR_STATE, "weight stream larger than its buffer");
+  CK(cudaMemcpyAsync(H->pf_segs + (size_t)(k - 1) * H->pf_nseg_max, v.data(), sizeof(PfSeg) * v.size(),
+                     cudaMemcpyHostToDevice, st));
+  H->pf_uploaded[k] = 1;
+  return DORY_OK;
+}
+
 template <typename T>
 dory_status decode_body(dory_handle* H, int batch, const int32_t* tokens_in, int k, int mode, int max_ctx,
                         float* logits, int32_t* next_tokens, cudaStream_t st) {
+  const bool pf = H->pf_lead > 0 && (int)H->pf_uploaded.size() > k && H->pf_uploaded[k];
+  H->pf_pos = pf ? 0 : -1;
+  H->pf_done = 0;
   CK(launch_plan_uniform(batch, 1, 0, H->seq_ids, H->seq_len, H->meta, st));
   Fwd<T> f{H, st, batch, max_ctx, true, mode, k, batch, true};
+  f.pf_k = pf ? k : 0;
   RET(input_block<T>(f, tokens_in));
   RET(loops<T>(f, 1, k, -1, 1));
   RET(output_and_head<T>(f, batch, nullptr, logits, next_tokens));
@@ -605,6 +699,7 @@ dory_status decode_t(dory_handle* H, int batch, const int32_t* seq_ids, const in
   int max_ctx = 0;
   for (int i = 0; i < batch; ++i) max_ctx = std::max(max_ctx, H->len[seq_ids[i]] + 1);
   RET(upload_ids(H, seq_ids, batch, st));
+  RET(ensure_stream(H, k, st));
   const bool use_graph = H->graphs && !H->profile && logits == nullptr;
   if (!use_graph) {
     RET(decode_body<T>(H, batch, tokens_in, k, mode, max_ctx, logits, next_tokens, st));
@@ -973,6 +1068,16 @@ dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value) {
     case DORY_OPT_PDL: dory::g_pdl = value != 0; return DORY_OK;
     case DORY_OPT_PREFILL_TC: h->prefill_tc = value != 0; return DORY_OK;
     case DORY_OPT_ATTN_CLUSTER: dory::g_attn_cluster = value != 0; return DORY_OK;
+    case DORY_OPT_L2_LOOKAHEAD:
+      if (value < 0 || value > (1ll << 40)) return fail(DORY_ERR_INVALID_ARG, "bad look-ahead");
+      if ((unsigned long long)value != h->pf_lead) {
+        // graphs captured with the old setting are dropped
+        for (auto& g : h->graphs_cache)
+          if (g.exec) cudaGraphExecDestroy(g.exec);
+        h->graphs_cache.clear();
+      }
+      h->pf_lead = (unsigned long long)value & ~127ull;
+      return DORY_OK;
     case DORY_OPT_GEMM_IMPL:
       if (value < 0 || value > 2) return fail(DORY_ERR_INVALID_ARG, "bad GEMM impl");
       h->gemm_impl = (int)value;

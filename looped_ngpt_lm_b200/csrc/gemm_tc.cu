@@ -119,6 +119,25 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
   return p;
 }
 
+// Prefetch this CTA's piece of the look-ahead range (see PfCtl) into L2;
+// called by all 32 lanes of one warp, each taking every 32nd 128-byte line.
+// Segment sizes and offsets are multiples of 128 bytes.
+__device__ void l2_look_ahead(const PfCtl& pf, int lane) {
+  const unsigned long long span = pf.hi - pf.lo;
+  const unsigned long long piece = ((span + gridDim.x - 1) / gridDim.x + 127) & ~127ull;
+  const unsigned long long a0 = pf.lo + piece * blockIdx.x;
+  const unsigned long long a1 = a0 + piece < pf.hi ? a0 + piece : pf.hi;
+  if (a0 >= a1) return;
+  for (int q = pf.first; q < pf.nseg && pf.segs[q].off < a1; ++q) {
+    const unsigned long long so = pf.segs[q].off, se = so + pf.segs[q].bytes;
+    if (se <= a0) continue;
+    const unsigned long long lo = a0 > so ? a0 : so, hi = a1 < se ? a1 : se;
+    const char* base = pf.segs[q].p - so;
+    for (unsigned long long a = (lo & ~127ull) + 128ull * lane; a < hi; a += 128ull * 32)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(base + a));
+  }
+}
+
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
 // 128 bytes, 8-row core-matrix groups 1024 bytes apart.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
@@ -167,16 +186,19 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 
 // KSUB 64-column sub-tiles per pipeline stage: a stage reads KSUB*128
 // contiguous bytes of every weight row.
-template <int NG, int GN, int KSUB, int BUDGET = 216 * 1024>
+// GLU: a unit's A operand is two 128-row tiles of one matrix, rows
+// [128 nt, +128) and [glu_rows + 128 nt, +128), with one accumulator each.
+template <int NG, int GN, int KSUB, int BUDGET = 216 * 1024, bool GLU = false>
 struct Tile {
   static constexpr int MT = NG * GN;                   // tokens per unit
   static constexpr int A_SUB = BM * BK * 2;            // 16 KB per sub-tile
   static constexpr int B_SUB = MT * BK * 2;
-  static constexpr int A_BYTES = KSUB * A_SUB;
+  static constexpr int NA = GLU ? 2 : 1;               // A tiles per unit
+  static constexpr int A_BYTES = NA * KSUB * A_SUB;
   static constexpr int B_BYTES = KSUB * B_SUB;
   static constexpr int STAGE = A_BYTES + B_BYTES;
   static constexpr int STAGES = BUDGET / STAGE > 12 ? 12 : (BUDGET / STAGE < 1 ? 1 : BUDGET / STAGE);
-  static constexpr int ACC = MT;                       // TMEM columns per accumulator
+  static constexpr int ACC = NA * MT;                  // TMEM columns per accumulator (pair)
   static constexpr int TMEM_COLS = 2 * ACC <= 32 ? 32 : 2 * ACC <= 64 ? 64 : 2 * ACC <= 128 ? 128 : 2 * ACC <= 256 ? 256 : 512;
   static constexpr int SMEM = STAGES * STAGE + 1024 /*align*/ + 256 /*barriers*/;
 };
@@ -199,12 +221,17 @@ struct UnitMap {
 // PACK: the weights are in the packed tile layout (see dory_pack_weight_bf16):
 // 128 x 64 tiles stored as their 16 KB swizzled shared-memory image, tiles
 // of one 128-row band consecutive along K, so a stage is one bulk copy.
-template <int NG, int GN, int KSUB, int BUDGET, bool PACK>
+//
+// GLU (prefill, no split): the epilogue writes act[m, j] = silu(g) * u as
+// bf16 (row stride ldy) from the pair of accumulators, where g and u are the
+// products with weight rows j and glu_rows + j: the SwiGLU of a concatenated
+// [gate; up] matrix, without its fp32 products ever reaching memory.
+template <int NG, int GN, int KSUB, int BUDGET, bool PACK, bool GLU = false>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, float* Y, int ldy,
               size_t part_stride, int M, UnitMap um, unsigned* tile_counters, int* err, const uint8_t* Apack,
-              int k_tiles) {
-  using TL = Tile<NG, GN, KSUB, BUDGET>;
+              int k_tiles, PfCtl pf, bf16* act, int glu_rows) {
+  using TL = Tile<NG, GN, KSUB, BUDGET, GLU>;
   constexpr int STAGES = TL::STAGES;
   auto load_a = [&](uint8_t* sa, uint64_t* bar, int nt, int kb, uint64_t pol) {
     if constexpr (PACK) {
@@ -212,6 +239,11 @@ __global__ void __launch_bounds__(192, 1)
     } else {
 #pragma unroll
       for (int q = 0; q < KSUB; ++q) tma_load_2d(sa + q * TL::A_SUB, &mapA, bar, (kb * KSUB + q) * BK, nt * BM, pol);
+      if constexpr (GLU) {
+#pragma unroll
+        for (int q = 0; q < KSUB; ++q)
+          tma_load_2d(sa + (KSUB + q) * TL::A_SUB, &mapA, bar, (kb * KSUB + q) * BK, glu_rows + nt * BM, pol);
+      }
     }
   };
   extern __shared__ uint8_t smem_raw[];
@@ -319,6 +351,8 @@ __global__ void __launch_bounds__(192, 1)
         mbar_wait_drain(&full[st], ph);
       }
     }
+    __syncwarp();
+    if (pf.lo < pf.hi && !*abort_flag) l2_look_ahead(pf, lane);
   } else if (warp == 1) {
     pdl_wait();
     if (lane == 0) {
@@ -352,6 +386,9 @@ __global__ void __launch_bounds__(192, 1)
                 // starts GN rows (GN * 128 bytes) further into the B tile
                 umma(d0 + g * GN, adesc + 2 * kk, bdesc + 2 * kk + (uint64_t)(g * GN * 128 >> 4), IDESC,
                      (kb > kb0 || q > 0 || kk > 0) ? 1u : 0u);
+                if constexpr (GLU)  // the up tile: KSUB sub-tiles further, its accumulator MT columns on
+                  umma(d0 + TL::MT + g * GN, adesc + 2 * kk + (uint64_t)(KSUB * TL::A_SUB >> 4),
+                       bdesc + 2 * kk + (uint64_t)(g * GN * 128 >> 4), IDESC, (kb > kb0 || q > 0 || kk > 0) ? 1u : 0u);
               }
             }
           }
@@ -391,10 +428,20 @@ __global__ void __launch_bounds__(192, 1)
         if (m_base + c >= M) break;
         float v[16];
         tmem_ld16(tmem_base + ((uint32_t)lane_base << 16) + acc * TL::ACC + c, v);
+        if constexpr (GLU) {
+          float w[16];
+          tmem_ld16(tmem_base + ((uint32_t)lane_base << 16) + acc * TL::ACC + TL::MT + c, w);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int m = m_base + c + j;
-          if (m < M) out[(size_t)m * ldy] = v[j];
+          for (int j = 0; j < 16; ++j) {
+            const int m = m_base + c + j;
+            if (m < M) act[(size_t)m * ldy + n] = __float2bfloat16_rn(v[j] / (1.f + expf(-v[j])) * w[j]);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int m = m_base + c + j;
+            if (m < M) out[(size_t)m * ldy] = v[j];
+          }
         }
       }
       tc_fence_before();
@@ -513,13 +560,14 @@ int sm_count() {
   return n;
 }
 
-template <int NG, int GN, int KSUB, int BUDGET = kDecodeBudget, bool PACK = false>
+template <int NG, int GN, int KSUB, int BUDGET = kDecodeBudget, bool PACK = false, bool GLU = false>
 cudaError_t run(const CUtensorMap& ma, const bf16* X, int ldx, int M, int K, float* Y, int ldy, size_t ps,
-                UnitMap um, unsigned* tile_counters, int* err, cudaStream_t st, const void* Apack = nullptr) {
-  using TL = Tile<NG, GN, KSUB, BUDGET>;
+                UnitMap um, unsigned* tile_counters, int* err, cudaStream_t st, const void* Apack = nullptr,
+                const PfCtl& pf = PfCtl{}, bf16* act = nullptr, int glu_rows = 0) {
+  using TL = Tile<NG, GN, KSUB, BUDGET, GLU>;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<NG, GN, KSUB, BUDGET, PACK>,
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<NG, GN, KSUB, BUDGET, PACK, GLU>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, TL::SMEM);
     if (e != cudaSuccess) return e;
     attr = true;
@@ -527,8 +575,8 @@ cudaError_t run(const CUtensorMap& ma, const bf16* X, int ldx, int M, int K, flo
   CUtensorMap mb;
   if (!make_map(&mb, X, M, K, ldx, TL::MT)) return cudaErrorInvalidValue;
   int grid = um.units < sm_count() ? um.units : sm_count();
-  return launch(k_gemm_tc<NG, GN, KSUB, BUDGET, PACK>, dim3(grid), dim3(192), TL::SMEM, st, ma, mb, Y, ldy, ps, M,
-                um, tile_counters, err, (const uint8_t*)Apack, K / BK);
+  return launch(k_gemm_tc<NG, GN, KSUB, BUDGET, PACK, GLU>, dim3(grid), dim3(192), TL::SMEM, st, ma, mb, Y, ldy,
+                ps, M, um, tile_counters, err, (const uint8_t*)Apack, K / BK, pf, act, glu_rows);
 }
 
 // Split factor for the decode tiles: chosen from (N, K, batch) only, never
@@ -570,6 +618,25 @@ __global__ void k_pack_weight(const bf16* __restrict__ src, uint8_t* __restrict_
 
 }  // namespace
 
+cudaError_t launch_gemm_glu(int M, int dff, int K, const bf16* X, int ldx, const bf16* Wgu, bf16* act,
+                            int* err, cudaStream_t st) {
+  if (M <= 0 || dff % BM || K % BK || ldx % 8 || ((uintptr_t)X & 15) || ((uintptr_t)Wgu & 15))
+    return cudaErrorNotSupported;
+  CUtensorMap ma;
+  if (!weight_map(&ma, Wgu, 2 * dff, K)) return cudaErrorNotSupported;
+  // 128 x 128 token tiles: the gate/up accumulator pair fills 256 TMEM
+  // columns, two pairs double-buffer the epilogue
+  UnitMap um;
+  um.n_tiles = dff / BM;
+  um.KBg = K / BK;
+  um.gran = 1;
+  um.S = 1;
+  um.m_tiles = (M + 127) / 128;
+  um.units = um.n_tiles * um.m_tiles;
+  return run<1, 128, 1, 200 * 1024, false, true>(ma, X, ldx, M, K, nullptr, dff, 0, um, nullptr, err, st, nullptr,
+                                                 PfCtl{}, act, dff);
+}
+
 cudaError_t launch_pack_weight(const bf16* W, void* dst, int N, int K, cudaStream_t st) {
   if (N % BM || K % BK || ((uintptr_t)W & 15) || ((uintptr_t)dst & 15)) return cudaErrorInvalidValue;
   const size_t chunks = (size_t)N * K / 8;
@@ -579,7 +646,7 @@ cudaError_t launch_pack_weight(const bf16* W, void* dst, int N, int K, cudaStrea
 
 cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf16* W, float* Y, int ldy,
                            size_t part_rows, int* err, int batch, bool invariant, int* S_out, size_t* ps_out,
-                           cudaStream_t st, int variant, unsigned* tile_counters, bool packed) {
+                           cudaStream_t st, int variant, unsigned* tile_counters, bool packed, const PfCtl* pf) {
   *S_out = 1;
   *ps_out = 0;
   if (M <= 0 || N % BM || K % BK || ldx % 8 || (size_t)M > part_rows || ((uintptr_t)X & 15) || ((uintptr_t)W & 15))
@@ -610,9 +677,10 @@ cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf
     unsigned* tc = (S > 1 && tile_counters && um.n_tiles * um.m_tiles <= kTileCounters) ? tile_counters : nullptr;
     *S_out = tc ? 1 : S;  // reduced in the kernel: one slice for the consumer
     *ps_out = tc ? 0 : ps;
-#define DORY_RUN(NGV, KS)                                                                            \
-  return packed ? run<NGV, 16, KS, kDecodeBudget, true>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st, W) \
-                : run<NGV, 16, KS>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st)
+    const PfCtl pfc = pf ? *pf : PfCtl{};
+#define DORY_RUN(NGV, KS)                                                                                 \
+  return packed ? run<NGV, 16, KS, kDecodeBudget, true>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st, W, pfc) \
+                : run<NGV, 16, KS>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st, nullptr, pfc)
     if (NG == 1) {
       if (ksub == 4) DORY_RUN(1, 4);
       if (ksub == 2) DORY_RUN(1, 2);

@@ -12,6 +12,25 @@ constexpr int kMaxSplitK = 8;
 // launches, and left zero by every launch).
 constexpr int kTileCounters = 4096;
 
+// Weight stream of one forward pass: the weight matrices in the order the
+// pass's GEMMs read them, each at a byte offset of one concatenated stream.
+struct PfSeg {
+  const char* p;
+  unsigned long long off, bytes;
+};
+
+// L2 look-ahead of one GEMM launch: the byte range [lo, hi) of the stream,
+// past this GEMM's own weights, that its CTAs prefetch into L2 once their
+// own loads have landed (CTA b takes the b-th of gridDim.x equal pieces).
+// The following attention, norms and the next GEMM's ramp-up then overlap
+// HBM reads of the weights that come next.  lo >= hi: off.
+struct PfCtl {
+  const PfSeg* segs = nullptr;
+  int nseg = 0;
+  int first = 0;  // a segment at or before the one holding lo
+  unsigned long long lo = 0, hi = 0;
+};
+
 // Y = X . W^T for X [M, K] (row stride ldx) and W [N, K], both bf16, fp32
 // accumulation.  Writes S partial products to Y + s * (*part_stride)
 // (row stride ldy); the consumer adds them in order s = 0..S-1.
@@ -23,11 +42,19 @@ constexpr int kTileCounters = 4096;
 // 64-column sub-tile per pipeline stage (for comparisons).  With
 // tile_counters (kTileCounters zeros), the last split of each output tile
 // adds the slices in order s = 0..S-1 inside the kernel and *S is 1.
-// packed: W is in the packed tile layout below.
+// packed: W is in the packed tile layout below.  pf: L2 look-ahead (decode
+// tiles only; ignored for prefill tiles).
 cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf16* W, float* Y, int ldy,
                            size_t part_rows, int* err, int batch, bool invariant, int* S, size_t* part_stride,
                            cudaStream_t st, int variant = 0, unsigned* tile_counters = nullptr,
-                           bool packed = false);
+                           bool packed = false, const PfCtl* pf = nullptr);
+
+// act[m, j] = silu(g) * u (bf16, row stride dff) with g = X[m] . Wgu[j] and
+// u = X[m] . Wgu[dff + j] for the concatenated [gate; up] weight Wgu
+// [2 dff, K]: the gate-up projection and SwiGLU of a long chunk in one
+// tensor-core GEMM (fp32 accumulation, no split).  dff % 128 == 0.
+cudaError_t launch_gemm_glu(int M, int dff, int K, const bf16* X, int ldx, const bf16* Wgu, bf16* act,
+                            int* err, cudaStream_t st);
 
 // Repack a row-major [N, K] bf16 weight (N % 128 == 0, K % 64 == 0) into the
 // packed tile layout the tensor-core GEMM streams with bulk copies: 128 x 64

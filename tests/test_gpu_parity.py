@@ -231,3 +231,30 @@ def test_graph_and_pdl_paths_agree(tiny_bf16, prompt, graphs, pdl):
     h.set_option(dory.OPT_CUDA_GRAPHS, 1)
     assert got[0] == ref[0] and got2[0] == ref[0]
     assert torch.equal(got[1], ref[1]) and torch.equal(got2[1], ref[1])
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("lead_mib", [1, 64])
+def test_l2_look_ahead_changes_no_bits(tiny_bf16, prompt, lead_mib):
+    """Prefetching upcoming weights into L2 only moves HBM reads earlier:
+    tokens and the final state are bit-identical with it off."""
+    _, _, h = tiny_bf16
+
+    def run():
+        h.reset()
+        tok = torch.tensor(prompt[:40], dtype=torch.int32, device="cuda")
+        nxt = h.prefill([0], tok, [40], 2, dory.LAST_LOOP)
+        toks = [int(nxt[0])]
+        for _ in range(6):
+            nxt = h.decode_step([0], nxt, 2, dory.LAST_LOOP)
+            toks.append(int(nxt[0]))
+        return toks, h.read_state("s", 1).cpu()
+
+    h.set_option(dory.OPT_L2_LOOKAHEAD, 0)
+    ref = run()
+    h.set_option(dory.OPT_L2_LOOKAHEAD, lead_mib << 20)
+    got = run()
+    got2 = run()  # graph replay
+    h.set_option(dory.OPT_L2_LOOKAHEAD, 8 << 20)
+    assert got[0] == ref[0] and got2[0] == ref[0]
+    assert torch.equal(got[1], ref[1]) and torch.equal(got2[1], ref[1])
