@@ -297,9 +297,18 @@ def main():
     ap.add_argument("--l2-lookahead-mb", dest="l2_mb", type=int, default=None,
                     help="bytes of upcoming weights each decode GEMM prefetches into L2 (MiB; 0 = off; "
                          "default: the library's)")
+    ap.add_argument("--batched", action="store_true",
+                    help="run the batched workload instead (--batch sequences of --prompt-batched tokens, "
+                         "chunked prefill, then --steps decode steps) and print its own JSON line")
+    ap.add_argument("--batch", type=int, default=64)
+    ap.add_argument("--prompt-batched", dest="prompt_batched", type=int, default=32768)
+    ap.add_argument("--chunk", type=int, default=8192, help="prefill chunk of the batched workload")
     ap.add_argument("--layers", default=None,
                     help="I,R,O physical layers (a narrower model of the same width, for small profiling captures)")
     args = ap.parse_args()
+    if args.batched:
+        batched_leg(args)
+        return
     if args.kernel == "gemm":
         gemm_probe(args)
         return
@@ -377,6 +386,18 @@ def main():
     pre_ms = max_over_ranks(min(pre_ms))
     pf = proj_flops(shape, args.k, args.prompt)
     af = attn_flops_prefill(shape, args.k, args.prompt)
+    # one more prefill with CUDA events around every launch: the projection
+    # GEMMs' and the attention kernel's own time
+    h.reset()
+    h.profile_reset()
+    h.set_option(dory.OPT_PROFILE, 1)
+    first = h.prefill([0], prompt, [args.prompt], args.k, mode)
+    torch.cuda.synchronize()
+    pprof = h.profile_read()
+    h.set_option(dory.OPT_PROFILE, 0)
+    h.profile_reset()
+    proj_ms = sum(v["ms"] for n, v in pprof.items() if n.startswith("gemm") and n != "gemm_lm_head")
+    attn_ms = sum(v["ms"] for n, v in pprof.items() if n.startswith("attn"))
 
     # ---- decode: warm-up, then exactly K timed steps
     bufs = [torch.empty(1, dtype=torch.int32, device="cuda") for _ in range(2)]
@@ -496,9 +517,15 @@ def main():
                     "frac_of_measured": round(step_bytes / (ms_step / 1e3) / 1e9 / hbm, 4),
                     "frac_of_8TBs": round(step_bytes / (ms_step / 1e3) / 8e12, 4)},
             "prefill": {"tokens": args.prompt, "ms": round(pre_ms, 3),
-                        "proj_tflops": round(pf / (pre_ms / 1e3) / 1e12, 2),
-                        "total_tflops": round((pf + af) / (pre_ms / 1e3) / 1e12, 2),
-                        "proj_frac_of_measured_bf16": round(pf / (pre_ms / 1e3) / 1e12 / tc, 4)},
+                        "wall_tflops": round((pf + af) / (pre_ms / 1e3) / 1e12, 2),
+                        "proj_tflops": round(pf / (proj_ms / 1e3) / 1e12, 2),
+                        "proj_frac_of_measured_bf16": round(pf / (proj_ms / 1e3) / 1e12 / tc, 4),
+                        "attn_tflops": round(af / (attn_ms / 1e3) / 1e12, 2),
+                        "proj_tflop": round(pf / 1e12, 3), "attn_tflop": round(af / 1e12, 3),
+                        "note": "proj/attn TFLOP/s: algorithmic FLOPs over the event-timed GEMM / attention "
+                                "kernels of one prefill; wall: all FLOPs over the whole prefill",
+                        "kernel_ms": {n: round(v["ms"], 3) for n, v in
+                                      sorted(pprof.items(), key=lambda kv: -kv[1]["ms"])}},
             "roofline": roofline,
             "kernel_share": kernel_share,
             "gpu_launches": int(round(launches_per_step * args.steps)),
@@ -511,6 +538,104 @@ def main():
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def batched_leg(args):
+    """64 sequences with 32768-token prompts at k=2, last-loop cache: chunked
+    prefill (TFLOP/s), then batched decode steps (aggregate tokens/s, HBM GB/s).
+    Prints one JSON line of its own."""
+    import torch
+    import synth
+    import looped_ngpt_lm_b200 as dory
+
+    hbm, tc, _, peak_src = peaks()
+    shape = synth.DORY_4B
+    B, P, k, chunk = args.batch, args.prompt_batched, 2, args.chunk
+    steps, warm = args.steps, max(args.warmup, 3)
+    torch.cuda.set_device(0)
+    w_np = synth.make_weights(shape, 1)
+    dw = dory.DeviceWeights(shape, w_np)
+    del w_np
+    cfg = dory.make_config(shape, max_batch=B, max_seq=P + steps + warm + 64, k_max=2, gamma_max=0,
+                           max_chunk=chunk)
+    h = dory.Handle(cfg, dw, dory.LAST_LOOP)
+    ws_gb = dory.workspace_size(cfg, dory.LAST_LOOP) / 1e9
+    prompts = torch.tensor(synth.make_prompt(1, B * P, shape.vocab), dtype=torch.int32).view(B, P).cuda()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    # kernel-level split of one sequence's chunked prefill (events around every launch)
+    h.reset()
+    h.profile_reset()
+    h.set_option(dory.OPT_PROFILE, 1)
+    for c0 in range(0, P, chunk):
+        n = min(chunk, P - c0)
+        h.prefill([0], prompts[0, c0:c0 + n], [n], k, dory.LAST_LOOP)
+    torch.cuda.synchronize()
+    pprof = h.profile_read()
+    h.set_option(dory.OPT_PROFILE, 0)
+    h.profile_reset()
+    pf1 = proj_flops(shape, k, P)
+    af1 = attn_flops_prefill(shape, k, P)
+    proj_ms = sum(v["ms"] for n_, v in pprof.items() if n_.startswith("gemm") and n_ != "gemm_lm_head")
+    attn_ms = sum(v["ms"] for n_, v in pprof.items() if n_.startswith("attn"))
+
+    # the whole batch, timed
+    h.reset()
+    torch.cuda.synchronize()
+    a, b = ev(), ev()
+    a.record()
+    last = torch.empty(B, dtype=torch.int32, device="cuda")
+    for s in range(B):
+        for c0 in range(0, P, chunk):
+            n = min(chunk, P - c0)
+            t = h.prefill([s], prompts[s, c0:c0 + n], [n], k, dory.LAST_LOOP)
+        last[s] = t[0]
+    b.record()
+    torch.cuda.synchronize()
+    h.synchronize()
+    pre_ms = a.elapsed_time(b)
+
+    ids = list(range(B))
+    bufs = [torch.empty(B, dtype=torch.int32, device="cuda") for _ in range(2)]
+    tok = last
+    for i in range(warm):
+        tok = h.decode_step(ids, tok, k, dory.LAST_LOOP, next_tokens=bufs[i % 2])
+    torch.cuda.synchronize()
+    clocks = Clocks(0)
+    clocks.start()
+    a, b = ev(), ev()
+    a.record()
+    for i in range(steps):
+        tok = h.decode_step(ids, tok, k, dory.LAST_LOOP, next_tokens=bufs[i % 2])
+    b.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    h.synchronize()
+    dec_ms = a.elapsed_time(b)
+    ctx_mid = P + warm + steps // 2
+    step_bytes = weight_bytes(shape, k) + B * kv_read_bytes(shape, k, ctx_mid)
+    ms_step = dec_ms / steps
+    line = {
+        "leg": "batched", "config": {"workload": f"dory4b_bf16_batch{B}_prompt{P}_decode{steps}_k2_last_loop",
+                                     "prefill_chunk": chunk, "workspace_GB": round(ws_gb, 2),
+                                     "data": "synthetic: seeded weights, uniform random prompt ids"},
+        "prefill": {"tokens": B * P, "s": round(pre_ms / 1e3, 3),
+                    "wall_tflops": round(B * (pf1 + af1) / (pre_ms / 1e3) / 1e12, 2),
+                    "proj_tflops": round(pf1 / (proj_ms / 1e3) / 1e12, 2),
+                    "proj_frac_of_measured_bf16": round(pf1 / (proj_ms / 1e3) / 1e12 / tc, 4),
+                    "attn_tflops": round(af1 / (attn_ms / 1e3) / 1e12, 2),
+                    "pflop": round(B * (pf1 + af1) / 1e15, 3),
+                    "kernel_ms_one_sequence": {n_: round(v["ms"], 2) for n_, v in
+                                               sorted(pprof.items(), key=lambda kv: -kv[1]["ms"])[:8]}},
+        "decode": {"steps": steps, "ms_per_step": round(ms_step, 3),
+                   "tokens_per_s": round(B * steps / (dec_ms / 1e3), 1),
+                   "bytes_per_step": step_bytes,
+                   "hbm_GBs": round(step_bytes / (ms_step / 1e3) / 1e9, 1),
+                   "hbm_frac_of_measured": round(step_bytes / (ms_step / 1e3) / 1e9 / hbm, 4)},
+        "peaks": {"hbm_GBs": hbm, "bf16_tflops": tc, "source": peak_src},
+        "clocks": clk,
+    }
+    print(json.dumps(line))
 
 
 def gemm_probe(args):

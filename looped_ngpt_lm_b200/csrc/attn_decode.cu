@@ -808,7 +808,7 @@ cudaError_t dispatch_cl(int M, int KV, const float* qkv, int S, size_t ps, KVVie
 
 template <typename T, int HD, int G>
 cudaError_t dispatch(int M, int KV, const float* qkv, int S, size_t ps, KVView kv, RowMeta m, int max_ctx,
-                     float* part, int nb_cap, unsigned* counters, T* out, cudaStream_t st) {
+                     float* part, int nb_cap, int part_rows, unsigned* counters, T* out, cudaStream_t st) {
   if constexpr (sizeof(T) == 2 && HD >= 64 && G <= 16) {
     if (g_attn_cluster) {
       cudaError_t e = dispatch_tc<HD, G>(M, KV, qkv, S, ps, kv, m, (bf16*)out, st);
@@ -822,7 +822,7 @@ cudaError_t dispatch(int M, int KV, const float* qkv, int S, size_t ps, KVView k
   const int span = kv.window > 0 ? min(max_ctx, kv.window) : max_ctx;
   const int nb = (span + DEC_BK - 1) / DEC_BK + 1;
   constexpr int SMEM = (int)sizeof(DecSmem<T, HD, G>);
-  if (nb > nb_cap) return cudaErrorInvalidValue;
+  if (nb > nb_cap || M > part_rows) return cudaErrorInvalidValue;
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(k_attn_decode<T, HD, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
@@ -838,11 +838,12 @@ cudaError_t dispatch(int M, int KV, const float* qkv, int S, size_t ps, KVView k
 
 template <typename T>
 cudaError_t launch_attn_decode(int M, int H, int KV, int hd, const float* qkv, int S, size_t ps, KVView kv,
-                               RowMeta m, int max_ctx, float* part, int nb_cap, unsigned* counters, T* out,
-                               cudaStream_t st) {
+                               RowMeta m, int max_ctx, float* part, int nb_cap, int part_rows, unsigned* counters,
+                               T* out, cudaStream_t st) {
   const int G = H / KV;
-#define DORY_DEC_CASE(HDV, GV) \
-  if (hd == HDV && G == GV) return dispatch<T, HDV, GV>(M, KV, qkv, S, ps, kv, m, max_ctx, part, nb_cap, counters, out, st);
+#define DORY_DEC_CASE(HDV, GV)                                                                                   \
+  if (hd == HDV && G == GV)                                                                                      \
+    return dispatch<T, HDV, GV>(M, KV, qkv, S, ps, kv, m, max_ctx, part, nb_cap, part_rows, counters, out, st);
   DORY_DEC_CASE(32, 1) DORY_DEC_CASE(32, 2) DORY_DEC_CASE(32, 4) DORY_DEC_CASE(32, 5) DORY_DEC_CASE(32, 8)
   DORY_DEC_CASE(64, 1) DORY_DEC_CASE(64, 2) DORY_DEC_CASE(64, 4) DORY_DEC_CASE(64, 5) DORY_DEC_CASE(64, 8)
   DORY_DEC_CASE(128, 1) DORY_DEC_CASE(128, 2) DORY_DEC_CASE(128, 4) DORY_DEC_CASE(128, 5)
@@ -851,8 +852,8 @@ cudaError_t launch_attn_decode(int M, int H, int KV, int hd, const float* qkv, i
 }
 
 template cudaError_t launch_attn_decode<float>(int, int, int, int, const float*, int, size_t, KVView, RowMeta, int,
-                                               float*, int, unsigned*, float*, cudaStream_t);
+                                               float*, int, int, unsigned*, float*, cudaStream_t);
 template cudaError_t launch_attn_decode<bf16>(int, int, int, int, const float*, int, size_t, KVView, RowMeta, int,
-                                              float*, int, unsigned*, bf16*, cudaStream_t);
+                                              float*, int, int, unsigned*, bf16*, cudaStream_t);
 
 }  // namespace dory

@@ -13,11 +13,13 @@ extern bool g_attn_cluster;
 
 // Attention of M rows whose K/V go straight into the cache.  qkv: the QKV
 // projection's S split-K partial slices (slice stride ps floats, rows of
-// q_dim + 2 kv_dim).  part: [M, H, nb_cap, hd + 4] scratch; counters:
-// [M * KV] zeros (left zero on return).  out: [M, H * hd] in the storage type.
+// q_dim + 2 kv_dim).  part: [part_rows, H, nb_cap, hd + 4] scratch, used
+// only when the cluster kernels cannot run (then M <= part_rows is
+// required); counters: [M * KV] zeros (left zero on return).  out: [M, H * hd]
+// in the storage type.
 template <typename T>
 cudaError_t launch_attn_decode(int M, int H, int KV, int hd, const float* qkv, int S, size_t ps, KVView kv,
-                               RowMeta m, int max_ctx, float* part, int nb_cap, unsigned* counters, T* out,
-                               cudaStream_t st);
+                               RowMeta m, int max_ctx, float* part, int nb_cap, int part_rows, unsigned* counters,
+                               T* out, cudaStream_t st);
 
 }  // namespace dory

@@ -125,6 +125,7 @@ struct dory_handle {
   unsigned* attn_counters = nullptr;  // [M_max * n_kv], zero between launches
   unsigned* tile_counters = nullptr;  // [kTileCounters], zero between launches
   int nb_cap = 0;                     // key blocks per row the partial buffer holds
+  int attn_rows = 0;                  // rows the partial buffer holds
   // weight stream of a decode step at each loop count k (L2 look-ahead)
   PfSeg* pf_segs = nullptr;           // [k_max][pf_nseg_max]
   int pf_nseg_max = 0;
@@ -258,7 +259,11 @@ size_t layout(dory_handle* h) {
   h->part_qkv = cv.take<float>(sizeof(float) * prow * h->qkv_dim);
   h->part_y = cv.take<float>(sizeof(float) * prow * d);
   h->part_gu = cv.take<float>(sizeof(float) * prow * 2 * c.d_ff);
-  h->attn_part = cv.take<float>(sizeof(float) * (size_t)M * c.n_heads * h->nb_cap * (c.head_dim + 4));
+  // split-KV partials: decode / verify rows at full context, or a slice of
+  // up to 256 chunk rows (the CUDA-core chunk attention runs in row slices)
+  h->attn_rows = std::min(M, std::max(c.max_batch * (c.gamma_max + 1), 256));
+  h->attn_part =
+      cv.take<float>(sizeof(float) * (size_t)h->attn_rows * c.n_heads * h->nb_cap * (c.head_dim + 4));
   h->attn_counters = cv.take<unsigned>(sizeof(unsigned) * (size_t)M * c.n_kv_heads);
   h->tile_counters = cv.take<unsigned>(sizeof(unsigned) * kTileCounters);
   h->logits = cv.take<float>(sizeof(float) * (size_t)h->head_max * c.vocab * kMaxSplitK);
@@ -424,7 +429,7 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop, float* copy_la
         // fused: q from the partials, own K/V into the cache, split-KV attention
         Scope sc(H, f.st, "attn_decode", 0);
         CK(launch_attn_decode<T>(M, c.n_heads, c.n_kv_heads, c.head_dim, H->part_qkv, S, ps, kv, H->meta, f.max_ctx,
-                                 H->attn_part, H->nb_cap, H->attn_counters, (T*)H->ao, f.st));
+                                 H->attn_part, H->nb_cap, H->attn_rows, H->attn_counters, (T*)H->ao, f.st));
       } else {
         // long chunks: K/V into scratch, attention, then the cache commit
         const bool tc = f.n_tiles > 0;
@@ -440,7 +445,8 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop, float* copy_la
         } else {
           Scope sc(H, f.st, "attention", 0);
           CK(launch_attention<T>(M, c.n_heads, c.n_kv_heads, c.head_dim, H->q, (const T*)H->kscr,
-                                 (const T*)H->vscr, true, kv, H->meta, f.max_ctx, H->attn_part, (T*)H->ao, f.st));
+                                 (const T*)H->vscr, true, kv, H->meta, f.max_ctx, H->attn_part, H->attn_rows,
+                                 (T*)H->ao, f.st));
         }
         // A last-loop recurrent layer shares one slot across loops, so the
         // chunk's keys are committed only after the final loop: committing
@@ -614,7 +620,9 @@ dory_status prefill_t(dory_handle* H, int batch, const int32_t* seq_ids, const i
   CK(cudaMemcpyAsync(H->head_rows, rows.data(), sizeof(int) * batch, cudaMemcpyHostToDevice, st));
   CK(launch_plan_ragged(batch, M, H->cu, H->seq_ids, H->seq_len, H->meta, st));
   int max_len = *std::max_element(lens, lens + batch);
-  Fwd<T> f{H, st, M, max_ctx, max_len <= H->slack + 1, mode, k, batch, false};
+  // short chunks write K/V straight into the cache (the decode attention,
+  // whose split-KV partials hold attn_rows rows)
+  Fwd<T> f{H, st, M, max_ctx, max_len <= H->slack + 1 && M <= H->attn_rows, mode, k, batch, false};
   if (!f.direct && H->bf16 && attn_prefill_supported(c.head_dim) && H->prefill_tc) {
     std::vector<int2> tl(H->tiles_cap);
     const int n = prefill_tiles(batch, cu.data(), tl.data(), H->tiles_cap);

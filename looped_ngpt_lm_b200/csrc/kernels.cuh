@@ -75,12 +75,13 @@ cudaError_t launch_qkv_post(int M, int H, int KV, int hd, const float* qkv, int 
                             int max_batch, bf16* qh, cudaStream_t st);
 
 // GQA attention over the cache (+ chunk scratch), split over absolute key
-// blocks of ATTN_BK positions, then merged in block order.
+// blocks of ATTN_BK positions, then merged in block order.  part holds the
+// block partials of part_rows rows; longer chunks run in row slices.
 constexpr int ATTN_BK = 256;
 template <typename T>
 cudaError_t launch_attention(int M, int H, int KV, int hd, const float* q, const T* kscr, const T* vscr,
                              bool inchunk_scratch, KVView kv, RowMeta m, int max_ctx, float* part,
-                             T* out, cudaStream_t st);
+                             int part_rows, T* out, cudaStream_t st);
 // Copy chunk K/V from scratch into the cache (positions >= pend - cap).
 template <typename T>
 cudaError_t launch_kv_commit(int M, int KV, int hd, const T* kscr, const T* vscr, KVView kv, RowMeta m,

@@ -532,17 +532,29 @@ static cudaError_t attn_dispatch(int M, int KV, const float* q, const T* kscr, c
 
 template <typename T>
 cudaError_t launch_attention(int M, int H, int KV, int hd, const float* q, const T* kscr, const T* vscr,
-                             bool sc, KVView kv, RowMeta m, int max_ctx, float* part, T* out, cudaStream_t st) {
+                             bool sc, KVView kv, RowMeta m, int max_ctx, float* part, int part_rows, T* out,
+                             cudaStream_t st) {
   int span = kv.window > 0 ? min(max_ctx, kv.window) : max_ctx;
   int nb = (span + ATTN_BK - 1) / ATTN_BK + 1;
   const int G = H / KV;
+  if (part_rows <= 0) return cudaErrorInvalidValue;
+  // rows are independent: long chunks run in slices of part_rows rows that
+  // reuse the partial buffer (chunk keys are addressed by m.base, absolute)
+  for (int r0 = 0; r0 < M; r0 += part_rows) {
+    const int n = min(part_rows, M - r0);
+    RowMeta ms{m.seq + r0, m.pos + r0, m.p0 + r0, m.base + r0, m.pend + r0};
+    const float* qs = q + (size_t)r0 * H * hd;
+    T* os = out + (size_t)r0 * H * hd;
+    cudaError_t e = cudaErrorInvalidValue;
 #define DORY_ATTN_CASE(HDV, GV) \
-  if (hd == HDV && G == GV) return attn_dispatch<T, HDV, GV>(M, KV, q, kscr, vscr, sc, kv, m, nb, part, out, st);
-  DORY_ATTN_CASE(32, 1) DORY_ATTN_CASE(32, 2) DORY_ATTN_CASE(32, 4) DORY_ATTN_CASE(32, 5) DORY_ATTN_CASE(32, 8)
-  DORY_ATTN_CASE(64, 1) DORY_ATTN_CASE(64, 2) DORY_ATTN_CASE(64, 4) DORY_ATTN_CASE(64, 5) DORY_ATTN_CASE(64, 8)
-  DORY_ATTN_CASE(128, 1) DORY_ATTN_CASE(128, 2) DORY_ATTN_CASE(128, 4) DORY_ATTN_CASE(128, 5)
+  if (hd == HDV && G == GV) e = attn_dispatch<T, HDV, GV>(n, KV, qs, kscr, vscr, sc, kv, ms, nb, part, os, st);
+    DORY_ATTN_CASE(32, 1) DORY_ATTN_CASE(32, 2) DORY_ATTN_CASE(32, 4) DORY_ATTN_CASE(32, 5) DORY_ATTN_CASE(32, 8)
+    DORY_ATTN_CASE(64, 1) DORY_ATTN_CASE(64, 2) DORY_ATTN_CASE(64, 4) DORY_ATTN_CASE(64, 5) DORY_ATTN_CASE(64, 8)
+    DORY_ATTN_CASE(128, 1) DORY_ATTN_CASE(128, 2) DORY_ATTN_CASE(128, 4) DORY_ATTN_CASE(128, 5)
 #undef DORY_ATTN_CASE
-  return cudaErrorInvalidValue;
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 template <typename T>
@@ -762,7 +774,7 @@ cudaError_t launch_spec_accept(int B, int gamma, int dstride, const int* seq_ids
   template cudaError_t launch_qkv_post<T>(int, int, int, int, const float*, int, size_t, float*, T*, T*, bool,    \
                                           KVView, RowMeta, int, bf16*, cudaStream_t);                             \
   template cudaError_t launch_attention<T>(int, int, int, int, const float*, const T*, const T*, bool, KVView,    \
-                                           RowMeta, int, float*, T*, cudaStream_t);                               \
+                                           RowMeta, int, float*, int, T*, cudaStream_t);                          \
   template cudaError_t launch_kv_commit<T>(int, int, int, const T*, const T*, KVView, RowMeta, cudaStream_t);     \
   template cudaError_t launch_swiglu<T>(int, int, const float*, int, size_t, T*, cudaStream_t);                   \
   template cudaError_t launch_gather_rows<T>(int, int, const int*, const T*, T*, cudaStream_t);                   \
