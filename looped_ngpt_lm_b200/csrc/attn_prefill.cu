@@ -65,16 +65,27 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
   return (uint32_t)(row * HD * 2 + ((chunk ^ (row & 7)) << 4));
 }
 
+// Base-2 exponential on the special-function unit (PTX ex2.approx.ftz:
+// subnormal results flush to zero).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Shared memory: two K and two V tiles; the Q tile is staged in the second
+// K tile and moved to registers before the first prefetch lands there.
 template <int HD>
-__global__ void __launch_bounds__(128) k_attn_prefill(int KV, int G, const bf16* __restrict__ qh,
+__global__ void __launch_bounds__(128, 3) k_attn_prefill(int KV, int G, const bf16* __restrict__ qh,
                                                       const bf16* __restrict__ kscr, const bf16* __restrict__ vscr,
                                                       KVView kv, RowMeta m, const int2* __restrict__ tiles,
                                                       bf16* __restrict__ out) {
   constexpr int CH = HD / 8;  // 16-byte chunks per row
   extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* sQ = smem;
-  uint8_t* sK = smem + QT * HD * 2;
+  static_assert(QT == KT, "the Q tile is staged in a K tile");
+  uint8_t* sK = smem;
   uint8_t* sV = sK + 2 * KT * HD * 2;
+  uint8_t* sQ = sK + KT * HD * 2;
   pdl_wait();
   pdl_trigger();
 
@@ -131,6 +142,7 @@ __global__ void __launch_bounds__(128) k_attn_prefill(int KV, int G, const bf16*
     const int row = warp * 16 + (lane % 16), ch = kk * 2 + lane / 16;
     ldsm_x4(smem_addr(sQ + swz<HD>(row, ch)), qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
   }
+  __syncthreads();  // every warp holds its Q fragments: the tile may be overwritten
   const int gq = lane >> 2, tig = lane & 3;
   // positions of this thread's two rows
   const int pr0 = pf + warp * 16 + gq, pr1 = pr0 + 8;
@@ -164,19 +176,28 @@ __global__ void __launch_bounds__(128) k_attn_prefill(int KV, int G, const bf16*
         mma_bf16(s[2 * n + 1], qa[kk], b2, b3);
       }
     }
-    // mask and online softmax (two rows per thread)
+    // mask and online softmax (two rows per thread).  A tile whose keys are
+    // all visible to all 16 rows of this warp (causal and window) skips the
+    // per-element mask.
+    const int wr0 = pf + warp * 16;  // positions of this warp's first and last rows
+    const bool open = kt + KT - 1 <= wr0 && (kv.window == 0 || kt >= wr0 + 15 - kv.window + 1);
     float mx[2] = {mrow[0], mrow[1]};
+    if (!open) {
 #pragma unroll
-    for (int n = 0; n < KT / 8; ++n) {
+      for (int n = 0; n < KT / 8; ++n) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int j = kt + n * 8 + 2 * tig + (e & 1);
-        const int pr = e < 2 ? pr0 : pr1, lo = e < 2 ? lo0 : lo1;
-        const bool ok = j <= pr && j >= lo && j >= 0;
-        s[n][e] = ok ? s[n][e] : -FLT_MAX;
-        mx[e >> 1] = fmaxf(mx[e >> 1], s[n][e]);
+        for (int e = 0; e < 4; ++e) {
+          const int j = kt + n * 8 + 2 * tig + (e & 1);
+          const int pr = e < 2 ? pr0 : pr1, lo = e < 2 ? lo0 : lo1;
+          const bool ok = j <= pr && j >= lo && j >= 0;
+          s[n][e] = ok ? s[n][e] : -FLT_MAX;
+        }
       }
     }
+#pragma unroll
+    for (int n = 0; n < KT / 8; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) mx[e >> 1] = fmaxf(mx[e >> 1], s[n][e]);
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 1));
@@ -184,14 +205,14 @@ __global__ void __launch_bounds__(128) k_attn_prefill(int KV, int G, const bf16*
     }
     float corr[2], rs[2] = {0.f, 0.f};
 #pragma unroll
-    for (int i = 0; i < 2; ++i) corr[i] = exp2f(mrow[i] - mx[i]);
+    for (int i = 0; i < 2; ++i) corr[i] = ex2(mrow[i] - mx[i]);
     uint32_t pa[KT / 16][4];
 #pragma unroll
     for (int n = 0; n < KT / 8; ++n) {
       float p[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        p[e] = s[n][e] == -FLT_MAX ? 0.f : exp2f(s[n][e] - mx[e >> 1]);
+        p[e] = (open || s[n][e] != -FLT_MAX) ? ex2(s[n][e] - mx[e >> 1]) : 0.f;
         rs[e >> 1] += p[e];
       }
       // C fragments of key tiles 2c, 2c+1 form the A fragment of k-chunk c
@@ -263,7 +284,7 @@ cudaError_t launch_attn_prefill(int n_tiles, const int2* tiles, int H, int KV, i
                                 cudaStream_t st) {
   const int G = H / KV;
   if (hd == 128) {
-    constexpr int SM = QT * 128 * 2 + 4 * KT * 128 * 2;
+    constexpr int SM = 4 * KT * 128 * 2;
     static bool attr = false;
     if (!attr) {
       cudaError_t e = cudaFuncSetAttribute(k_attn_prefill<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, SM);
@@ -273,7 +294,7 @@ cudaError_t launch_attn_prefill(int n_tiles, const int2* tiles, int H, int KV, i
     return launch(k_attn_prefill<128>, dim3(n_tiles, H), dim3(128), SM, st, KV, G, qh, kscr, vscr, kv, m, tiles, out);
   }
   if (hd == 64) {
-    constexpr int SM = QT * 64 * 2 + 4 * KT * 64 * 2;
+    constexpr int SM = 4 * KT * 64 * 2;
     static bool attr = false;
     if (!attr) {
       cudaError_t e = cudaFuncSetAttribute(k_attn_prefill<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, SM);
