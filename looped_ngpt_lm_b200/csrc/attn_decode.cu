@@ -482,7 +482,10 @@ __global__ void __launch_bounds__(256) k_attn_decode_cl(int KV, const float* __r
 // so S = Q K^T and O += P V cost 2 * head_dim / 8 MMAs per 16 keys.  Warps
 // take steps w, w + 8, ...; their states merge in warp order, then the
 // cluster's blocks merge in rank order through distributed shared memory.
-constexpr int TC_KC = 192;  // keys per shared-memory sub-chunk
+// A block's keys stream through two shared-memory chunks of TC_KC keys: the
+// first two are requested at once, and chunk i + 2 is requested as soon as
+// chunk i has been consumed.
+constexpr int TC_KC = 128;  // keys per shared-memory chunk (two chunks)
 
 __device__ __forceinline__ void dsmem_st(float* local, int rank, float v) {
   uint32_t a = saddr(local), ra;
@@ -490,18 +493,31 @@ __device__ __forceinline__ void dsmem_st(float* local, int rank, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
 }
 
-template <int HD, int G>
+template <int HD, int G, int CS>
 struct TcSmem {
   uint8_t q[16 * HD * 2];
-  uint8_t k[TC_KC * HD * 2];
-  uint8_t v[TC_KC * HD * 2];
+  uint8_t k[2][TC_KC * HD * 2];
+  uint8_t v[2][TC_KC * HD * 2];
   float wm[NW][G], wl[NW][G];
   float wacc[NW][G][HD];
   float part[G][HD + 2];
-  float all[16][G][HD + 2];  // rank 0: every rank's partial, pushed by the ranks
-  float rw[16][G];
+  float all[CS][G][HD + 2];  // rank 0: every rank's partial, pushed by the ranks
+  float rw[CS][G];
   float rinv[G];
 };
+
+// Cluster size of the tensor-core decode attention: the largest of 16, 8, 4
+// whose grid for `batch` sequences stays within about four waves of one
+// block per SM.  It depends on the number of sequences only (never on rows
+// per sequence), so plain decode and a speculative verify of the same
+// sequences split every row's keys identically.
+constexpr int kDecodeBlockBudget = 4 * 148;
+inline int decode_cluster_size(int batch, int KV) {
+  const int pairs = batch * KV;
+  if (pairs * 16 <= kDecodeBlockBudget) return 16;
+  if (pairs * 8 <= kDecodeBlockBudget) return 8;
+  return 4;
+}
 
 template <int HD, int G, int CS>
 __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __restrict__ qkv, int S, size_t ps,
@@ -510,10 +526,8 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
   using namespace wm;
   constexpr int CH = HD / 8;  // 16-byte chunks per row
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  TcSmem<HD, G>& sm = *reinterpret_cast<TcSmem<HD, G>*>(smem_raw);
+  TcSmem<HD, G, CS>& sm = *reinterpret_cast<TcSmem<HD, G, CS>*>(smem_raw);
 
-  pdl_wait();
-  pdl_trigger();
   const int pair = blockIdx.x / CS, rank = blockIdx.x % CS;
   const int r = pair / KV, g = pair % KV;
   const int pos = m.pos[r], seq = m.seq[r], p0 = m.p0[r], base = m.base[r];
@@ -526,6 +540,47 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, gq = lane >> 2, tig = lane & 3;
   const bf16* Kc = (const bf16*)kv.K + ((size_t)seq * KV + g) * kv.cap * HD;
   const bf16* Vc = (const bf16*)kv.V + ((size_t)seq * KV + g) * kv.cap * HD;
+
+  // chunk ci holds keys klo + ci * TC_KC .. in buffer ci & 1.  Cached keys
+  // (positions < p0) and the zero padding up to 16 keys come by cp.async;
+  // they were written by earlier calls and nothing in flight rewrites them
+  // (this chunk's positions map to ring slots no row here reads), so the
+  // first two chunks are requested before waiting for the QKV projection.
+  const int nchunk = khi >= klo ? (khi - klo) / TC_KC + 1 : 0;
+  auto issue_cached = [&](int ci) {
+    const int c0 = klo + ci * TC_KC, c1 = min(khi, c0 + TC_KC - 1), n = c1 - c0 + 1, n16 = (n + 15) & ~15;
+    const int cache_hi = min(c1, p0 - 1);
+    uint8_t* kb = sm.k[ci & 1];
+    uint8_t* vb = sm.v[ci & 1];
+    for (int i = tid; i < n16 * CH; i += blockDim.x) {
+      const int jj = i / CH, c = i % CH, j = c0 + jj;
+      if (j <= cache_hi || jj >= n) {
+        const bool ok = jj < n;
+        const size_t src = (size_t)((ok ? j : c0) % kv.cap) * HD + c * 8;
+        cp_async16(smem_addr(kb + swz<HD>(jj, c)), Kc + src, ok);
+        cp_async16(smem_addr(vb + swz<HD>(jj, c)), Vc + src, ok);
+      }
+    }
+    cp_async_commit();
+  };
+  // the chunk's own keys (positions >= p0), summed from the QKV partials
+  auto fill_new = [&](int ci) {
+    const int c0 = klo + ci * TC_KC, c1 = min(khi, c0 + TC_KC - 1);
+    const int jc0 = max(c0, p0);
+    uint8_t* kb = sm.k[ci & 1];
+    uint8_t* vb = sm.v[ci & 1];
+#pragma unroll 4
+    for (int i = tid; i < (c1 - jc0 + 1) * HD; i += blockDim.x) {
+      const int jj = i / HD, d = i % HD, row = jc0 - c0 + jj;
+      const float* src = qkv + (size_t)(base + (jc0 + jj - p0)) * ld + qd + g * HD + d;
+      *reinterpret_cast<bf16*>(kb + swz<HD>(row, d / 8) + (d % 8) * 2) = __float2bfloat16_rn(sum_splits(src, S, ps));
+      *reinterpret_cast<bf16*>(vb + swz<HD>(row, d / 8) + (d % 8) * 2) =
+          __float2bfloat16_rn(sum_splits(src + kvd, S, ps));
+    }
+  };
+  if (nchunk > 0) issue_cached(0);
+  if (nchunk > 1) issue_cached(1);
+  pdl_wait();
 
   // Q tile: rows 0..G-1 = the G heads (pre-scaled, bf16), rows G..15 zero
   // (unrolled: every partial load of the tile is in flight at once)
@@ -558,32 +613,22 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
   for (int i = 0; i < HD / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   float mrow[2] = {-FLT_MAX, -FLT_MAX}, lrow[2] = {0.f, 0.f};
 
+  if (nchunk > 0) fill_new(0);
+  if (nchunk > 1) fill_new(1);
+
 #pragma unroll 1
-  for (int c0 = klo; c0 <= khi; c0 += TC_KC) {
-    const int c1 = min(khi, c0 + TC_KC - 1), n = c1 - c0 + 1, n16 = (n + 15) & ~15;
-    const int cache_hi = min(c1, p0 - 1);
-    for (int i = tid; i < n16 * CH; i += blockDim.x) {
-      const int jj = i / CH, c = i % CH, j = c0 + jj;
-      if (j <= cache_hi || jj >= n) {  // cached key, or zero padding up to 16 keys
-        const bool ok = jj < n;
-        const size_t src = (size_t)((ok ? j : c0) % kv.cap) * HD + c * 8;
-        cp_async16(smem_addr(sm.k + swz<HD>(jj, c)), Kc + src, ok);
-        cp_async16(smem_addr(sm.v + swz<HD>(jj, c)), Vc + src, ok);
-      }
-    }
-    cp_async_commit();
-    const int jc0 = max(c0, p0);
-#pragma unroll 4
-    for (int i = tid; i < (c1 - jc0 + 1) * HD; i += blockDim.x) {
-      const int jj = i / HD, d = i % HD, row = jc0 - c0 + jj;
-      const float* src = qkv + (size_t)(base + (jc0 + jj - p0)) * ld + qd + g * HD + d;
-      *reinterpret_cast<bf16*>(sm.k + swz<HD>(row, d / 8) + (d % 8) * 2) =
-          __float2bfloat16_rn(sum_splits(src, S, ps));
-      *reinterpret_cast<bf16*>(sm.v + swz<HD>(row, d / 8) + (d % 8) * 2) =
-          __float2bfloat16_rn(sum_splits(src + kvd, S, ps));
-    }
-    cp_async_wait<0>();
+  for (int ci = 0; ci < nchunk; ++ci) {
+    const int c0 = klo + ci * TC_KC, n = min(khi, c0 + TC_KC - 1) - c0 + 1;
+    if (ci + 1 < nchunk)
+      cp_async_wait<1>();  // chunk ci landed; ci + 1 may be in flight
+    else
+      cp_async_wait<0>();
     __syncthreads();
+    // the O projection that follows may launch (and stream its weights)
+    // once this block's first keys have arrived, not before
+    if (ci == 0) pdl_trigger();
+    const uint8_t* kbuf = sm.k[ci & 1];
+    const uint8_t* vbuf = sm.v[ci & 1];
 #pragma unroll 1
     for (int st = w; st * 16 < n; st += NW) {
       float sc[2][4];
@@ -592,7 +637,7 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
 #pragma unroll
       for (int kk = 0; kk < HD / 16; ++kk) {
         uint32_t b0, b1, b2, b3;
-        ldsm_x4(smem_addr(sm.k + swz<HD>(st * 16 + (lane % 8) + (lane / 16) * 8, kk * 2 + (lane / 8) % 2)), b0, b1,
+        ldsm_x4(smem_addr(kbuf + swz<HD>(st * 16 + (lane % 8) + (lane / 16) * 8, kk * 2 + (lane / 8) % 2)), b0, b1,
                 b2, b3);
         mma_bf16(sc[0], qa[kk], b0, b1);
         mma_bf16(sc[1], qa[kk], b2, b3);
@@ -640,14 +685,19 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
 #pragma unroll
       for (int d = 0; d < HD / 16; ++d) {
         uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(smem_addr(sm.v + swz<HD>(st * 16 + (lane % 8) + ((lane / 8) % 2) * 8, d * 2 + lane / 16)), b0, b1,
+        ldsm_x4_t(smem_addr(vbuf + swz<HD>(st * 16 + (lane % 8) + ((lane / 8) % 2) * 8, d * 2 + lane / 16)), b0, b1,
                   b2, b3);
         mma_bf16(o[2 * d], pa, b0, b1);
         mma_bf16(o[2 * d + 1], pa, b2, b3);
       }
     }
-    __syncthreads();
+    __syncthreads();  // buffer ci & 1 is free
+    if (ci + 2 < nchunk) {
+      issue_cached(ci + 2);
+      fill_new(ci + 2);
+    }
   }
+  if (nchunk == 0) pdl_trigger();
   // this warp's rows 0..G-1 (held by lanes with gq < G, row gq) -> shared memory
   if (gq < G) {
     if (tig == 0) {
@@ -710,11 +760,10 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
   }
 }
 
-template <int HD, int G>
+template <int HD, int G, int CS>
 cudaError_t dispatch_tc(int M, int KV, const float* qkv, int S, size_t ps, KVView kv, RowMeta m, bf16* out,
                         cudaStream_t st) {
-  constexpr int CS = 16;
-  constexpr int SMEM = (int)sizeof(TcSmem<HD, G>);
+  constexpr int SMEM = (int)sizeof(TcSmem<HD, G, CS>);
   auto kern = k_attn_decode_tc<HD, G, CS>;
   static int state = 0;
   if (state == 0) {
@@ -808,10 +857,14 @@ cudaError_t dispatch_cl(int M, int KV, const float* qkv, int S, size_t ps, KVVie
 
 template <typename T, int HD, int G>
 cudaError_t dispatch(int M, int KV, const float* qkv, int S, size_t ps, KVView kv, RowMeta m, int max_ctx,
-                     float* part, int nb_cap, int part_rows, unsigned* counters, T* out, cudaStream_t st) {
+                     float* part, int nb_cap, int part_rows, unsigned* counters, T* out, int batch,
+                     cudaStream_t st) {
   if constexpr (sizeof(T) == 2 && HD >= 64 && G <= 16) {
     if (g_attn_cluster) {
-      cudaError_t e = dispatch_tc<HD, G>(M, KV, qkv, S, ps, kv, m, (bf16*)out, st);
+      const int cs = decode_cluster_size(batch, KV);
+      cudaError_t e = cs == 16  ? dispatch_tc<HD, G, 16>(M, KV, qkv, S, ps, kv, m, (bf16*)out, st)
+                      : cs == 8 ? dispatch_tc<HD, G, 8>(M, KV, qkv, S, ps, kv, m, (bf16*)out, st)
+                                : dispatch_tc<HD, G, 4>(M, KV, qkv, S, ps, kv, m, (bf16*)out, st);
       if (e != cudaErrorNotSupported) return e;
     }
   }
@@ -839,11 +892,12 @@ cudaError_t dispatch(int M, int KV, const float* qkv, int S, size_t ps, KVView k
 template <typename T>
 cudaError_t launch_attn_decode(int M, int H, int KV, int hd, const float* qkv, int S, size_t ps, KVView kv,
                                RowMeta m, int max_ctx, float* part, int nb_cap, int part_rows, unsigned* counters,
-                               T* out, cudaStream_t st) {
+                               T* out, int batch, cudaStream_t st) {
   const int G = H / KV;
 #define DORY_DEC_CASE(HDV, GV)                                                                                   \
   if (hd == HDV && G == GV)                                                                                      \
-    return dispatch<T, HDV, GV>(M, KV, qkv, S, ps, kv, m, max_ctx, part, nb_cap, part_rows, counters, out, st);
+    return dispatch<T, HDV, GV>(M, KV, qkv, S, ps, kv, m, max_ctx, part, nb_cap, part_rows, counters, out, batch, \
+                                st);
   DORY_DEC_CASE(32, 1) DORY_DEC_CASE(32, 2) DORY_DEC_CASE(32, 4) DORY_DEC_CASE(32, 5) DORY_DEC_CASE(32, 8)
   DORY_DEC_CASE(64, 1) DORY_DEC_CASE(64, 2) DORY_DEC_CASE(64, 4) DORY_DEC_CASE(64, 5) DORY_DEC_CASE(64, 8)
   DORY_DEC_CASE(128, 1) DORY_DEC_CASE(128, 2) DORY_DEC_CASE(128, 4) DORY_DEC_CASE(128, 5)
@@ -852,8 +906,8 @@ cudaError_t launch_attn_decode(int M, int H, int KV, int hd, const float* qkv, i
 }
 
 template cudaError_t launch_attn_decode<float>(int, int, int, int, const float*, int, size_t, KVView, RowMeta, int,
-                                               float*, int, int, unsigned*, float*, cudaStream_t);
+                                               float*, int, int, unsigned*, float*, int, cudaStream_t);
 template cudaError_t launch_attn_decode<bf16>(int, int, int, int, const float*, int, size_t, KVView, RowMeta, int,
-                                              float*, int, int, unsigned*, bf16*, cudaStream_t);
+                                              float*, int, int, unsigned*, bf16*, int, cudaStream_t);
 
 }  // namespace dory

@@ -16,10 +16,11 @@ extern bool g_attn_cluster;
 // q_dim + 2 kv_dim).  part: [part_rows, H, nb_cap, hd + 4] scratch, used
 // only when the cluster kernels cannot run (then M <= part_rows is
 // required); counters: [M * KV] zeros (left zero on return).  out: [M, H * hd]
-// in the storage type.
+// in the storage type.  batch: sequences in the call (rows may be several
+// per sequence); selects how many blocks share one row's keys.
 template <typename T>
 cudaError_t launch_attn_decode(int M, int H, int KV, int hd, const float* qkv, int S, size_t ps, KVView kv,
                                RowMeta m, int max_ctx, float* part, int nb_cap, int part_rows, unsigned* counters,
-                               T* out, cudaStream_t st);
+                               T* out, int batch, cudaStream_t st);
 
 }  // namespace dory

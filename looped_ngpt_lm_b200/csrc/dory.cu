@@ -429,7 +429,8 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop, float* copy_la
         // fused: q from the partials, own K/V into the cache, split-KV attention
         Scope sc(H, f.st, "attn_decode", 0);
         CK(launch_attn_decode<T>(M, c.n_heads, c.n_kv_heads, c.head_dim, H->part_qkv, S, ps, kv, H->meta, f.max_ctx,
-                                 H->attn_part, H->nb_cap, H->attn_rows, H->attn_counters, (T*)H->ao, f.st));
+                                 H->attn_part, H->nb_cap, H->attn_rows, H->attn_counters, (T*)H->ao, f.batch,
+                                 f.st));
       } else {
         // long chunks: K/V into scratch, attention, then the cache commit
         const bool tc = f.n_tiles > 0;
