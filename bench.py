@@ -33,6 +33,56 @@ sys.path.insert(0, ROOT)
 METRIC = "decode tokens/s at k=1/2/4 (last-loop KV), % HBM roofline; prefill TFLOP/s"
 
 
+class Ranks:
+    """Rank plumbing: one process per GPU under torchrun (RANK, WORLD_SIZE,
+    LOCAL_RANK, MASTER_* from the environment), process group over NCCL;
+    backend "gloo" keeps every tensor on the host (used by the CPU tests).
+    Every rank takes the same collective steps in the same order."""
+
+    def __init__(self, backend="nccl", timeout_s=300):
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = backend
+        self.dist = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+            self.dist = dist
+
+    def _sync(self):
+        if self.backend != "gloo":
+            import torch
+            torch.cuda.synchronize()
+
+    def barrier(self):
+        """Device work finished here and on every rank."""
+        self._sync()
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def max(self, x: float) -> float:
+        """Maximum of x over the ranks (device times: the slowest rank)."""
+        if self.dist is None:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device="cpu" if self.backend == "gloo" else "cuda")
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.dist is not None:
+            self.dist.barrier()
+            self.dist.destroy_process_group()
+            self.dist = None
+
+
+def job_throughput(world: int, units_per_rank: int, max_ms: float) -> float:
+    """Whole-job rate: the units every rank processed over the slowest rank's time."""
+    return world * units_per_rank / (max_ms / 1e3)
+
+
 def peaks():
     try:
         p = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
@@ -130,10 +180,12 @@ class Clocks:
 
 
 # ---------------------------------------------------------------- CPU oracle
-def sweep_modes(dory, torch, shape, dw, args, prompt_len=128, n_new=256):
+def sweep_modes(dory, torch, shape, dw, args, prompt_len=128, n_new=1024):
     """Batch 1, 128-token prompt, greedy decode at k = 1/2/4 in both cache
     modes: tokens/s, KV bytes per token, and how far last_loop logits drift
-    from per_loop logits on the same tokens (teacher-forced)."""
+    from per_loop logits on the same tokens (teacher-forced over all n_new
+    steps: the last_loop run's logits are kept on the device, then the
+    per_loop replay is compared step by step)."""
     import synth
     cfg = dory.make_config(shape, max_batch=2, max_seq=prompt_len + n_new + 8, k_max=4, gamma_max=4,
                            max_chunk=prompt_len)
@@ -163,31 +215,33 @@ def sweep_modes(dory, torch, shape, dw, args, prompt_len=128, n_new=256):
             out[f"k{k}_{mode}"] = {"tokens_per_s": round(1e3 / ms, 2),
                                    "kv_bytes_per_token": round(h.kv_bytes(k, md, ctx) / ctx, 1), "ctx": ctx}
         # logits drift: replay one greedy last_loop run in both modes on the same tokens
-        lg = {m: [] for m in ("last_loop", "per_loop")}
-        tok_seq = []
+        L = torch.empty((1, shape.vocab), device="cuda")
+        ref = torch.empty((n_new, shape.vocab), device="cuda")
+        tok_seq = torch.empty(n_new, dtype=torch.int32, device="cuda")
+        drift = torch.empty(n_new, device="cuda")
+        agree = torch.empty(n_new, device="cuda")
         for mode in ("last_loop", "per_loop"):
             md = dory.MODES[mode]
             seq = 0 if mode == "last_loop" else 1
             h.reset(seq)
-            L = torch.empty((1, shape.vocab), device="cuda")
             t = h.prefill([seq], prompt, [prompt_len], k, md, logits=L)
-            lg[mode].append(L[0].clone())
-            for i in range(31):
+            for i in range(n_new):
                 if mode == "last_loop":
-                    tok_seq.append(int(t[0]))
-                inp = torch.tensor([tok_seq[i]], dtype=torch.int32, device="cuda")
-                t = h.decode_step([seq], inp, k, md, logits=L)
-                lg[mode].append(L[0].clone())
-        A, B = torch.stack(lg["last_loop"]), torch.stack(lg["per_loop"])
-        drift = ((A - B).norm(dim=1) / B.norm(dim=1)).cpu()
-        agree = (A.argmax(1) == B.argmax(1)).float().mean().item()
+                    ref[i] = L[0]
+                    tok_seq[i] = t[0]
+                else:
+                    drift[i] = (L[0] - ref[i]).norm() / ref[i].norm()
+                    agree[i] = (L[0].argmax() == ref[i].argmax()).float()
+                if i + 1 < n_new:
+                    t = h.decode_step([seq], tok_seq[i:i + 1], k, md, logits=L)
+        drift, agree = drift.cpu(), float(agree.mean())
         out[f"k{k}_logits_drift"] = {"rel_l2_max": round(float(drift.max()), 5), "rel_l2_mean": round(float(drift.mean()), 5),
-                                     "argmax_agreement": round(agree, 4), "steps": int(A.shape[0])}
+                                     "argmax_agreement": round(agree, 4), "steps": n_new}
     h.close()
     return out
 
 
-def spec_leg(dory, torch, shape, dw, args, prompt_len=512, n_new=128, gamma=4):
+def spec_leg(dory, torch, shape, dw, args, prompt_len=512, n_new=512, gamma=4):
     """Self-speculative decoding (draft k=1, verify k=4, gamma=4, last_loop)
     at batch 1, 4 and 16 against plain k=4 greedy decoding of the same
     prompts: accepted draft tokens per verify step, output tokens/s, speed-up,
@@ -338,11 +392,7 @@ def main():
     import looped_ngpt_lm_b200 as dory
 
     torch.cuda.set_device(local)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    ranks = Ranks("nccl")
 
     w_np = synth.make_weights(shape, 1)
     dw = dory.DeviceWeights(shape, w_np)
@@ -358,17 +408,7 @@ def main():
     stream = torch.cuda.current_stream()
     prompt = torch.tensor(synth.make_prompt(1, args.prompt, shape.vocab), dtype=torch.int32, device="cuda")
 
-    def barrier():
-        torch.cuda.synchronize()
-        if dist is not None:
-            dist.barrier()
-
-    def max_over_ranks(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier, max_over_ranks = ranks.barrier, ranks.max
 
     # ---- prefill (timed on its own: projection + attention TFLOP/s)
     ev = lambda: torch.cuda.Event(enable_timing=True)
@@ -417,7 +457,7 @@ def main():
     h.synchronize()
     dec_ms = max_over_ranks(t0.elapsed_time(t1))
     ms_step = dec_ms / args.steps
-    value = world * args.steps / (dec_ms / 1e3)
+    value = job_throughput(world, args.steps, dec_ms)
     ctx_mid = args.prompt + args.warmup + args.steps // 2
     step_bytes = weight_bytes(shape, args.k) + kv_read_bytes(shape, args.k, ctx_mid)
 
@@ -535,9 +575,7 @@ def main():
         }
         line.update(aux)
         print(json.dumps(line))
-    if dist is not None:
-        dist.barrier()
-        dist.destroy_process_group()
+    ranks.close()
 
 
 def batched_leg(args):
