@@ -257,7 +257,8 @@ enum {
   DORY_OPT_PROFILE = 2,     /* 1: time every launch with CUDA events (slow) */
   DORY_OPT_GEMM_IMPL = 3,   /* bf16 GEMM: 0 auto, 1 SIMT reference kernel, 2 tcgen05 */
   DORY_OPT_PDL = 4,         /* 1 (default): programmatic dependent launches (process-wide) */
-  DORY_OPT_PREFILL_TC = 5,  /* 1 (default): bf16 long-chunk attention on the tensor cores; 0: CUDA cores */
+  DORY_OPT_PREFILL_TC = 5,  /* bf16 long-chunk attention: 2 (default) tcgen05 with TMEM accumulators for
+                               head_dim 128 (else as 1), 1 warp-level mma.sync, 0 CUDA cores */
   DORY_OPT_ATTN_CLUSTER = 6, /* 1 (default): decode attention as 16-block clusters (process-wide) */
   /* bf16 decode steps: bytes of upcoming weights each GEMM prefetches into L2
    * past its own once its loads have landed (default 8 MiB; 0 turns the

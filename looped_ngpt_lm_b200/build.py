@@ -9,7 +9,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdory.so")
-SOURCES = ["dory.cu", "kernels_simt.cu", "gemm_tc.cu", "attn_decode.cu", "attn_prefill.cu", "gemm_noalloc.cu"]
+SOURCES = ["dory.cu", "kernels_simt.cu", "gemm_tc.cu", "attn_decode.cu", "attn_prefill.cu", "attn_prefill_tc.cu",
+           "gemm_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -267,12 +267,12 @@ __global__ void __launch_bounds__(128, 3) k_attn_prefill(int KV, int G, const bf
 
 }  // namespace
 
-int prefill_tiles(int n_seq, const int* cu, int2* tiles, int cap) {
+int prefill_tiles(int n_seq, const int* cu, int2* tiles, int cap, int rows) {
   int n = 0;
   for (int b = 0; b < n_seq; ++b)
-    for (int r = cu[b]; r < cu[b + 1]; r += QT) {
+    for (int r = cu[b]; r < cu[b + 1]; r += rows) {
       if (n >= cap) return -1;
-      tiles[n++] = make_int2(r, r + QT < cu[b + 1] ? r + QT : cu[b + 1]);
+      tiles[n++] = make_int2(r, r + rows < cu[b + 1] ? r + rows : cu[b + 1]);
     }
   return n;
 }

@@ -5,16 +5,24 @@
 
 namespace dory {
 
-// Host: split each sequence's chunk rows [cu[b], cu[b+1]) into tiles of 64
-// rows (int2 {first, end}); returns the count, or -1 past `cap`.
-int prefill_tiles(int n_seq, const int* cu, int2* tiles, int cap);
+// Host: split each sequence's chunk rows [cu[b], cu[b+1]) into tiles of
+// `rows` rows (int2 {first, end}); returns the count, or -1 past `cap`.
+int prefill_tiles(int n_seq, const int* cu, int2* tiles, int cap, int rows = 64);
 bool attn_prefill_supported(int head_dim);
+// The tcgen05 kernel (S and O accumulators in TMEM): head_dim 128, tiles of
+// 128 rows.
+bool attn_prefill_tc_supported(int head_dim);
 
 // qh: [M, H*hd] bf16 queries pre-scaled by log2(e)/sqrt(hd); kscr/vscr: the
 // chunk's K/V [M, KV*hd]; keys before each sequence's chunk come from kv.
 // out: [M, H*hd] bf16.
+// launch_attn_prefill: warp-level mma.sync, 64-row tiles; launch_attn_prefill_tc:
+// tcgen05 with TMEM accumulators, 128-row tiles.
 cudaError_t launch_attn_prefill(int n_tiles, const int2* tiles, int H, int KV, int hd, const bf16* qh,
                                 const bf16* kscr, const bf16* vscr, KVView kv, RowMeta m, bf16* out,
                                 cudaStream_t st);
+cudaError_t launch_attn_prefill_tc(int n_tiles, const int2* tiles, int H, int KV, int hd, const bf16* qh,
+                                   const bf16* kscr, const bf16* vscr, KVView kv, RowMeta m, bf16* out,
+                                   cudaStream_t st);
 
 }  // namespace dory

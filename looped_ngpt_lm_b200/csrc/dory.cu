@@ -134,7 +134,8 @@ struct dory_handle {
   std::vector<int> len, mode, kfix;  // per sequence; mode -1 = empty
   std::vector<int> ids_on_device;     // seq ids last uploaded to seq_ids
   int last_rows = 0;
-  bool graphs = true, profile = false, prefill_tc = true;
+  bool graphs = true, profile = false;
+  int prefill_tc = 2;  // long-chunk attention: 2 tcgen05 (head_dim 128), 1 mma.sync, 0 CUDA cores
   int gemm_impl = 0;
   unsigned long long pf_lead = 8ull << 20;   // 0: no L2 look-ahead
   std::vector<std::vector<PfSeg>> pf_host;   // [k] -> stream of a k-loop decode step
@@ -331,6 +332,7 @@ struct Fwd {
   int batch;    // sequences in the call (selects the GEMM split)
   bool invariant;  // decode / speculative rows: GEMM arithmetic independent of M
   int n_tiles = 0;  // > 0: long-chunk attention on the tensor cores over H->tiles
+  bool tc5 = false; // ... by the tcgen05 kernel (128-row tiles)
   int pf_k = 0;     // > 0: GEMMs follow the weight stream of a pf_k-loop decode step
 };
 
@@ -441,8 +443,12 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop, float* copy_la
         }
         if (tc) {
           Scope sc(H, f.st, "attn_prefill", 0);
-          CK(launch_attn_prefill(f.n_tiles, H->tiles, c.n_heads, c.n_kv_heads, c.head_dim, (const bf16*)H->qh,
-                                 (const bf16*)H->kscr, (const bf16*)H->vscr, kv, H->meta, (bf16*)H->ao, f.st));
+          if (f.tc5)
+            CK(launch_attn_prefill_tc(f.n_tiles, H->tiles, c.n_heads, c.n_kv_heads, c.head_dim, (const bf16*)H->qh,
+                                      (const bf16*)H->kscr, (const bf16*)H->vscr, kv, H->meta, (bf16*)H->ao, f.st));
+          else
+            CK(launch_attn_prefill(f.n_tiles, H->tiles, c.n_heads, c.n_kv_heads, c.head_dim, (const bf16*)H->qh,
+                                   (const bf16*)H->kscr, (const bf16*)H->vscr, kv, H->meta, (bf16*)H->ao, f.st));
         } else {
           Scope sc(H, f.st, "attention", 0);
           CK(launch_attention<T>(M, c.n_heads, c.n_kv_heads, c.head_dim, H->q, (const T*)H->kscr,
@@ -625,8 +631,9 @@ dory_status prefill_t(dory_handle* H, int batch, const int32_t* seq_ids, const i
   // whose split-KV partials hold attn_rows rows)
   Fwd<T> f{H, st, M, max_ctx, max_len <= H->slack + 1 && M <= H->attn_rows, mode, k, batch, false};
   if (!f.direct && H->bf16 && attn_prefill_supported(c.head_dim) && H->prefill_tc) {
+    f.tc5 = H->prefill_tc >= 2 && attn_prefill_tc_supported(c.head_dim);
     std::vector<int2> tl(H->tiles_cap);
-    const int n = prefill_tiles(batch, cu.data(), tl.data(), H->tiles_cap);
+    const int n = prefill_tiles(batch, cu.data(), tl.data(), H->tiles_cap, f.tc5 ? 128 : 64);
     if (n < 0) return fail(DORY_ERR_CAPACITY, "too many prefill attention tiles");
     CK(cudaMemcpyAsync(H->tiles, tl.data(), sizeof(int2) * n, cudaMemcpyHostToDevice, st));
     f.n_tiles = n;
@@ -1075,7 +1082,10 @@ dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value) {
     case DORY_OPT_CUDA_GRAPHS: h->graphs = value != 0; return DORY_OK;
     case DORY_OPT_PROFILE: h->profile = value != 0; return DORY_OK;
     case DORY_OPT_PDL: dory::g_pdl = value != 0; return DORY_OK;
-    case DORY_OPT_PREFILL_TC: h->prefill_tc = value != 0; return DORY_OK;
+    case DORY_OPT_PREFILL_TC:
+      if (value < 0 || value > 2) return fail(DORY_ERR_INVALID_ARG, "bad prefill attention kernel");
+      h->prefill_tc = (int)value;
+      return DORY_OK;
     case DORY_OPT_ATTN_CLUSTER: dory::g_attn_cluster = value != 0; return DORY_OK;
     case DORY_OPT_L2_LOOKAHEAD:
       if (value < 0 || value > (1ll << 40)) return fail(DORY_ERR_INVALID_ARG, "bad look-ahead");

@@ -305,8 +305,10 @@ __global__ void k_qkv_post(int H, int KV, int hd, const float* qkv, int S, size_
     float a = 0.f;
     for (int s = 0; s < S; ++s) a += src[s * ps + i];
     if (i < qd) {
-      q_out[(size_t)r * qd + i] = a;
-      if (qh) qh[(size_t)r * qd + i] = __float2bfloat16_rn(a * qscale);
+      if (qh)  // the tensor-core attention reads only the scaled bf16 copy
+        qh[(size_t)r * qd + i] = __float2bfloat16_rn(a * qscale);
+      else
+        q_out[(size_t)r * qd + i] = a;
     } else {
       int j = i - qd;
       bool is_v = j >= kvd;
@@ -681,31 +683,45 @@ cudaError_t launch_gemm_simt(int M, int N, int K, const T* X, int ldx, const T* 
 }
 
 // ------------------------------------------------------------------ argmax
-// One block per row; per-thread running (max, lowest index), then a fixed
-// tree.  max with lowest-index ties is order independent.
-__global__ void k_argmax(int V, const float* logits, int* out) {
+// One block per row; per-thread running (max, lowest index) over 16-byte
+// loads (8 in flight per thread) when every row starts 16-byte aligned, then
+// a fixed tree.  max with lowest-index ties is order independent.
+constexpr int AM_THREADS = 1024;
+
+__device__ __forceinline__ void am_take(float v, int i, float& best, int& bi) {
+  if (v > best || (v == best && i < bi)) {
+    best = v;
+    bi = i;
+  }
+}
+
+__global__ void __launch_bounds__(AM_THREADS) k_argmax(int V, const float* logits, int* out, bool vec) {
   pdl_wait();
   pdl_trigger();
-  __shared__ float sv[32];
-  __shared__ int si[32];
-  const float* row = logits + (size_t)blockIdx.x * V;
+  __shared__ float sv[AM_THREADS / 32];
+  __shared__ int si[AM_THREADS / 32];
+  const float* x = logits + (size_t)blockIdx.x * V;
   float best = -FLT_MAX;
   int bi = 0x7fffffff;
-  for (int i = threadIdx.x; i < V; i += blockDim.x) {
-    float v = row[i];
-    if (v > best) {
-      best = v;
-      bi = i;
+  if (vec) {
+    const float4* x4 = reinterpret_cast<const float4*>(x);
+    const int n4 = V / 4;
+#pragma unroll 8
+    for (int i = threadIdx.x; i < n4; i += AM_THREADS) {
+      const float4 v = x4[i];
+      am_take(v.x, 4 * i, best, bi);
+      am_take(v.y, 4 * i + 1, best, bi);
+      am_take(v.z, 4 * i + 2, best, bi);
+      am_take(v.w, 4 * i + 3, best, bi);
     }
+  } else {
+    for (int i = threadIdx.x; i < V; i += AM_THREADS) am_take(x[i], i, best, bi);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    float ov = __shfl_xor_sync(0xffffffffu, best, o);
-    int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-    if (ov > best || (ov == best && oi < bi)) {
-      best = ov;
-      bi = oi;
-    }
+    const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    am_take(ov, oi, best, bi);
   }
   const int w = threadIdx.x >> 5;
   if ((threadIdx.x & 31) == 0) {
@@ -714,17 +730,14 @@ __global__ void k_argmax(int V, const float* logits, int* out) {
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    for (int i = 1; i < (int)(blockDim.x >> 5); ++i)
-      if (sv[i] > best || (sv[i] == best && si[i] < bi)) {
-        best = sv[i];
-        bi = si[i];
-      }
+    for (int i = 1; i < AM_THREADS / 32; ++i) am_take(sv[i], si[i], best, bi);
     out[blockIdx.x] = bi;
   }
 }
 
 cudaError_t launch_argmax(int R, int V, const float* logits, int* out, cudaStream_t st) {
-  launch(k_argmax, R, 1024, 0, st, V, logits, out);
+  const bool vec = (V & 3) == 0 && ((uintptr_t)logits & 15) == 0;
+  launch(k_argmax, R, AM_THREADS, 0, st, V, logits, out, vec);
   return cudaGetLastError();
 }
 
