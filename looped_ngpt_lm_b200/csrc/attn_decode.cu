@@ -487,6 +487,13 @@ __global__ void __launch_bounds__(256) k_attn_decode_cl(int KV, const float* __r
 // chunk i has been consumed.
 constexpr int TC_KC = 128;  // keys per shared-memory chunk (two chunks)
 
+// Base-2 exponential on the special-function unit (PTX ex2.approx.ftz).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ void dsmem_st(float* local, int rank, float v) {
   uint32_t a = saddr(local), ra;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
@@ -547,19 +554,24 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
   // (this chunk's positions map to ring slots no row here reads), so the
   // first two chunks are requested before waiting for the QKV projection.
   const int nchunk = khi >= klo ? (khi - klo) / TC_KC + 1 : 0;
+  // thread `tid` keeps chunk column tid % CH and rows tid / CH + RS * n; the
+  // ring slot of its row advances by RS (a division only when it wraps)
+  constexpr int RS = 256 / CH;
   auto issue_cached = [&](int ci) {
     const int c0 = klo + ci * TC_KC, c1 = min(khi, c0 + TC_KC - 1), n = c1 - c0 + 1, n16 = (n + 15) & ~15;
     const int cache_hi = min(c1, p0 - 1);
     uint8_t* kb = sm.k[ci & 1];
     uint8_t* vb = sm.v[ci & 1];
-    for (int i = tid; i < n16 * CH; i += blockDim.x) {
-      const int jj = i / CH, c = i % CH, j = c0 + jj;
-      if (j <= cache_hi || jj >= n) {
-        const bool ok = jj < n;
-        const size_t src = (size_t)((ok ? j : c0) % kv.cap) * HD + c * 8;
-        cp_async16(smem_addr(kb + swz<HD>(jj, c)), Kc + src, ok);
-        cp_async16(smem_addr(vb + swz<HD>(jj, c)), Vc + src, ok);
+    const int c = tid % CH;
+    int jj = tid / CH, slot = (c0 + jj) % kv.cap;
+    for (; jj < n16; jj += RS) {
+      if (c0 + jj <= cache_hi || jj >= n) {  // cached key, or zero padding up to 16 keys
+        const size_t src = (size_t)slot * HD + c * 8;
+        cp_async16(smem_addr(kb + swz<HD>(jj, c)), Kc + src, jj < n);
+        cp_async16(smem_addr(vb + swz<HD>(jj, c)), Vc + src, jj < n);
       }
+      slot += RS;
+      if (slot >= kv.cap) slot %= kv.cap;  // rare: only when the row wraps around the ring
     }
     cp_async_commit();
   };
@@ -658,12 +670,12 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
       }
       float corr[2], rs[2] = {0.f, 0.f}, pv[2][4];
 #pragma unroll
-      for (int i = 0; i < 2; ++i) corr[i] = mrow[i] == -FLT_MAX ? 0.f : exp2f(mrow[i] - mx[i]);
+      for (int i = 0; i < 2; ++i) corr[i] = mrow[i] == -FLT_MAX ? 0.f : ex2(mrow[i] - mx[i]);
 #pragma unroll
       for (int t = 0; t < 2; ++t)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          pv[t][e] = sc[t][e] == -FLT_MAX ? 0.f : exp2f(sc[t][e] - mx[e >> 1]);
+          pv[t][e] = sc[t][e] == -FLT_MAX ? 0.f : ex2(sc[t][e] - mx[e >> 1]);
           rs[e >> 1] += pv[t][e];
         }
 #pragma unroll
@@ -675,12 +687,14 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
       }
       const uint32_t pa[4] = {pack_bf16(pv[0][0], pv[0][1]), pack_bf16(pv[0][2], pv[0][3]),
                               pack_bf16(pv[1][0], pv[1][1]), pack_bf16(pv[1][2], pv[1][3])};
+      if (__any_sync(0xffffffffu, corr[0] != 1.f || corr[1] != 1.f)) {  // a row max moved
 #pragma unroll
-      for (int i = 0; i < HD / 8; ++i) {
-        o[i][0] *= corr[0];
-        o[i][1] *= corr[0];
-        o[i][2] *= corr[1];
-        o[i][3] *= corr[1];
+        for (int i = 0; i < HD / 8; ++i) {
+          o[i][0] *= corr[0];
+          o[i][1] *= corr[0];
+          o[i][2] *= corr[1];
+          o[i][3] *= corr[1];
+        }
       }
 #pragma unroll
       for (int d = 0; d < HD / 16; ++d) {
