@@ -688,6 +688,16 @@ dory_status ensure_stream(dory_handle* H, int k, cudaStream_t st) {
   return DORY_OK;
 }
 
+// Let the GEMMs of a pass follow the weight stream of a k-loop decode step
+// from its segment `pos` on (L2 look-ahead), when that stream is uploaded.
+template <typename T>
+void follow_stream(dory_handle* H, Fwd<T>& f, int k, int pos) {
+  const bool on = H->pf_lead > 0 && (int)H->pf_uploaded.size() > k && H->pf_uploaded[k];
+  f.pf_k = on ? k : 0;
+  H->pf_pos = on ? pos : -1;
+  H->pf_done = 0;
+}
+
 template <typename T>
 dory_status decode_body(dory_handle* H, int batch, const int32_t* tokens_in, int k, int mode, int max_ctx,
                         float* logits, int32_t* next_tokens, cudaStream_t st) {
@@ -772,6 +782,8 @@ dory_status spec_t(dory_handle* H, int B, const int32_t* seq_ids, const int32_t*
   int max_ctx = 0;
   for (int i = 0; i < B; ++i) max_ctx = std::max(max_ctx, H->len[seq_ids[i]] + max_new + 2 * gamma + 1);
   RET(upload_ids(H, seq_ids, B, st));
+  RET(ensure_stream(H, 1, st));
+  RET(ensure_stream(H, kv_, st));
   CK(cudaMemcpyAsync(H->pending, last_tokens, sizeof(int) * B, cudaMemcpyDeviceToDevice, st));
   CK(cudaMemsetAsync(out_len, 0, sizeof(int) * B, st));
   CK(cudaMemsetAsync(H->accepted, 0, sizeof(unsigned long long), st));
@@ -781,6 +793,7 @@ dory_status spec_t(dory_handle* H, int B, const int32_t* seq_ids, const int32_t*
     for (int i = 0; i < gamma; ++i) {
       CK(launch_plan_uniform(B, 1, i, H->seq_ids, H->seq_len, H->meta, st));
       Fwd<T> f{H, st, B, max_ctx, true, mode, 1, B, true};
+      follow_stream(H, f, 1, 0);  // a draft is a k = 1 step
       const int* tok = i == 0 ? H->pending : H->drafts + (i - 1) * B;
       RET(input_block<T>(f, tok));
       CK(launch_stash_copy(B, c.d_model, H->x, H->stash_x, 1, gc, i, 0, st));
@@ -791,6 +804,7 @@ dory_status spec_t(dory_handle* H, int B, const int32_t* seq_ids, const int32_t*
     {
       CK(launch_plan_uniform(B, 1, gamma, H->seq_ids, H->seq_len, H->meta, st));
       Fwd<T> f{H, st, B, max_ctx, true, mode, 1, B, true};
+      follow_stream(H, f, 1, 0);  // the first two blocks of a k = 1 step
       RET(input_block<T>(f, H->drafts + (gamma - 1) * B));
       CK(launch_stash_copy(B, c.d_model, H->x, H->stash_x, 1, gc, gamma, 0, st));
       Scope sc(H, st, "reinject", 0);
@@ -804,6 +818,7 @@ dory_status spec_t(dory_handle* H, int B, const int32_t* seq_ids, const int32_t*
       const int rps = gamma + 1, M = B * rps;
       CK(launch_plan_uniform(B, rps, 0, H->seq_ids, H->seq_len, H->meta, st));
       Fwd<T> f{H, st, M, max_ctx, true, mode, kv_, B, true};
+      follow_stream(H, f, kv_, 2 * (c.n_in + c.n_rec));  // a k_verify step from its loop 2 on
       CK(launch_stash_copy(M, c.d_model, H->x, H->stash_x, rps, gc, 0, 1, st));
       CK(launch_stash_copy(M, c.d_model, H->s, H->stash_s, rps, gc, 0, 1, st));
       RET(loops<T>(f, 2, kv_, -1, rps));
