@@ -259,7 +259,8 @@ enum {
   DORY_OPT_PDL = 4,         /* 1 (default): programmatic dependent launches (process-wide) */
   DORY_OPT_PREFILL_TC = 5,  /* bf16 long-chunk attention: 2 (default) tcgen05 with TMEM accumulators for
                                head_dim 128 (else as 1), 1 warp-level mma.sync, 0 CUDA cores */
-  DORY_OPT_ATTN_CLUSTER = 6, /* 1 (default): decode attention as 16-block clusters (process-wide) */
+  DORY_OPT_ATTN_CLUSTER = 6, /* 1 (default): decode attention as clusters of 16, 8 or 4 blocks per row and
+                                KV head, chosen from the number of sequences (process-wide) */
   /* bf16 decode steps: bytes of upcoming weights each GEMM prefetches into L2
    * past its own once its loads have landed (default 8 MiB; 0 turns the
    * look-ahead off).  Changes only when HBM reads happen, never what is

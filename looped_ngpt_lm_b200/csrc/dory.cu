@@ -123,7 +123,6 @@ struct dory_handle {
   int *drafts = nullptr, *pending = nullptr, *vtok = nullptr, *out_len = nullptr, *all_done = nullptr;
   unsigned long long* accepted = nullptr;
   unsigned* attn_counters = nullptr;  // [M_max * n_kv], zero between launches
-  unsigned* tile_counters = nullptr;  // [kTileCounters], zero between launches
   int nb_cap = 0;                     // key blocks per row the partial buffer holds
   int attn_rows = 0;                  // rows the partial buffer holds
   // weight stream of a decode step at each loop count k (L2 look-ahead)
@@ -266,7 +265,6 @@ size_t layout(dory_handle* h) {
   h->attn_part =
       cv.take<float>(sizeof(float) * (size_t)h->attn_rows * c.n_heads * h->nb_cap * (c.head_dim + 4));
   h->attn_counters = cv.take<unsigned>(sizeof(unsigned) * (size_t)M * c.n_kv_heads);
-  h->tile_counters = cv.take<unsigned>(sizeof(unsigned) * kTileCounters);
   h->logits = cv.take<float>(sizeof(float) * (size_t)h->head_max * c.vocab * kMaxSplitK);
   const int gc = c.gamma_max + 1;
   h->stash_x = cv.take<float>(sizeof(float) * (size_t)c.max_batch * gc * d);
@@ -394,7 +392,7 @@ dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, cons
         }
       }
       cudaError_t e = launch_gemm_tc(M, N, K, (const bf16*)X, ldx, (const bf16*)W, Y, ldy, part_rows,
-                                     H->err, f.batch, f.invariant, &S, &ps, f.st, 0, nullptr, false, pp);
+                                     H->err, f.batch, f.invariant, &S, &ps, f.st, 0, false, pp);
       if (e == cudaSuccess) {
         *S_out = S;
         *ps_out = ps;
@@ -917,7 +915,6 @@ dory_status dory_reset(dory_handle* h, int32_t seq, dory_stream stream) {
     CK(cudaMemsetAsync(h->seq_len, 0, sizeof(int) * h->c.max_batch, st));
     CK(cudaMemsetAsync(h->err, 0, sizeof(int) * 4, st));
     CK(cudaMemsetAsync(h->attn_counters, 0, sizeof(unsigned) * (size_t)h->M_max * h->c.n_kv_heads, st));
-    CK(cudaMemsetAsync(h->tile_counters, 0, sizeof(unsigned) * kTileCounters, st));
     std::fill(h->len.begin(), h->len.end(), 0);
     std::fill(h->mode.begin(), h->mode.end(), -1);
     return DORY_OK;
@@ -1057,7 +1054,7 @@ dory_status dory_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* X, const
     size_t ps = 0;
     cudaError_t e = launch_gemm_tc(M, N, K, (const bf16*)X, K, (const bf16*)W, Y, N, (size_t)M, err_word,
                                    batch_hint < 1 ? 1 : batch_hint, invariant != 0, &S, &ps, st, impl == 3 ? 1 : 0,
-                                   nullptr, impl == 4);
+                                   impl == 4);
     if (e == cudaSuccess) {
       *splits = S;
       return DORY_OK;

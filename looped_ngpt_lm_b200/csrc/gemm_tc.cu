@@ -136,7 +136,7 @@ struct UnitMap {
 template <int NG, int GN, int KSUB, int BUDGET, bool PACK, bool GLU = false>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, float* Y, int ldy,
-              size_t part_stride, int M, UnitMap um, unsigned* tile_counters, int* err, const uint8_t* Apack,
+              size_t part_stride, int M, UnitMap um, int* err, const uint8_t* Apack,
               int k_tiles, PfCtl pf, bf16* act, int glu_rows) {
   using TL = Tile<NG, GN, KSUB, BUDGET, GLU>;
   constexpr int STAGES = TL::STAGES;
@@ -162,7 +162,6 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* mma_done = tempty + 2;
   uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
-  volatile int* last_flag = (volatile int*)(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -354,36 +353,6 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
-      if (um.S > 1 && tile_counters) {
-        // split-K: the last split of this tile to finish adds all slices in
-        // order s = 0..S-1 and leaves the sum in slice 0
-        __threadfence();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (warp == 2 && lane == 0) {
-          const unsigned prev = atomicAdd(&tile_counters[nt * um.m_tiles + mt], 1u);
-          *last_flag = prev == (unsigned)(um.S - 1);
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (*last_flag) {
-          __threadfence();
-          const int m_end = min(M, m_base + TL::MT);
-          for (int m0 = m_base; m0 < m_end; m0 += 4) {
-            float acc4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int q = 0; q < kMaxSplitK; ++q) {
-              if (q < um.S) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                  if (m0 + j < m_end) acc4[j] += __ldcg(Y + (size_t)q * part_stride + (size_t)(m0 + j) * ldy + n);
-              }
-            }
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              if (m0 + j < m_end) Y[(size_t)(m0 + j) * ldy + n] = acc4[j];
-          }
-          if (warp == 2 && lane == 0) tile_counters[nt * um.m_tiles + mt] = 0u;
-        }
-      }
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
@@ -469,7 +438,7 @@ int sm_count() {
 
 template <int NG, int GN, int KSUB, int BUDGET = kDecodeBudget, bool PACK = false, bool GLU = false>
 cudaError_t run(const CUtensorMap& ma, const bf16* X, int ldx, int M, int K, float* Y, int ldy, size_t ps,
-                UnitMap um, unsigned* tile_counters, int* err, cudaStream_t st, const void* Apack = nullptr,
+                UnitMap um, int* err, cudaStream_t st, const void* Apack = nullptr,
                 const PfCtl& pf = PfCtl{}, bf16* act = nullptr, int glu_rows = 0) {
   using TL = Tile<NG, GN, KSUB, BUDGET, GLU>;
   static bool attr = false;
@@ -483,7 +452,7 @@ cudaError_t run(const CUtensorMap& ma, const bf16* X, int ldx, int M, int K, flo
   if (!make_map(&mb, X, M, K, ldx, TL::MT)) return cudaErrorInvalidValue;
   int grid = um.units < sm_count() ? um.units : sm_count();
   return launch(k_gemm_tc<NG, GN, KSUB, BUDGET, PACK, GLU>, dim3(grid), dim3(192), TL::SMEM, st, ma, mb, Y, ldy,
-                ps, M, um, tile_counters, err, (const uint8_t*)Apack, K / BK, pf, act, glu_rows);
+                ps, M, um, err, (const uint8_t*)Apack, K / BK, pf, act, glu_rows);
 }
 
 // Split factor for the decode tiles: chosen from (N, K, batch) only, never
@@ -494,7 +463,9 @@ cudaError_t run(const CUtensorMap& ma, const bf16* X, int ldx, int M, int K, flo
 int choose_split(int N, int K, int batch, int kstages) {
   const double hbm = 6.5e12, sm_bw = 5.5e10;
   const int tiles = N / BM, sms = sm_count();
-  const double rows = 5.0 * batch;  // decode / verify rows this batch size produces
+  // partial-sum traffic is charged for one row per sequence (plain decode);
+  // a speculative verify chunk has gamma + 1 rows per sequence and pays more
+  const double rows = batch;
   const double stage_bytes = (double)BM * (K / kstages) * 2;
   int best = 1;
   double best_t = 1e30;
@@ -540,7 +511,7 @@ cudaError_t launch_gemm_glu(int M, int dff, int K, const bf16* X, int ldx, const
   um.S = 1;
   um.m_tiles = (M + 127) / 128;
   um.units = um.n_tiles * um.m_tiles;
-  return run<1, 128, 1, 200 * 1024, false, true>(ma, X, ldx, M, K, nullptr, dff, 0, um, nullptr, err, st, nullptr,
+  return run<1, 128, 1, 200 * 1024, false, true>(ma, X, ldx, M, K, nullptr, dff, 0, um, err, st, nullptr,
                                                  PfCtl{}, act, dff);
 }
 
@@ -553,7 +524,7 @@ cudaError_t launch_pack_weight(const bf16* W, void* dst, int N, int K, cudaStrea
 
 cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf16* W, float* Y, int ldy,
                            size_t part_rows, int* err, int batch, bool invariant, int* S_out, size_t* ps_out,
-                           cudaStream_t st, int variant, unsigned* tile_counters, bool packed, const PfCtl* pf) {
+                           cudaStream_t st, int variant, bool packed, const PfCtl* pf) {
   *S_out = 1;
   *ps_out = 0;
   if (M <= 0 || N % BM || K % BK || ldx % 8 || (size_t)M > part_rows || ((uintptr_t)X & 15) || ((uintptr_t)W & 15))
@@ -581,13 +552,12 @@ cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf
     const int MT = 16 * NG;
     um.m_tiles = (M + MT - 1) / MT;
     um.units = um.n_tiles * um.m_tiles * S;
-    unsigned* tc = (S > 1 && tile_counters && um.n_tiles * um.m_tiles <= kTileCounters) ? tile_counters : nullptr;
-    *S_out = tc ? 1 : S;  // reduced in the kernel: one slice for the consumer
-    *ps_out = tc ? 0 : ps;
+    *S_out = S;
+    *ps_out = ps;
     const PfCtl pfc = pf ? *pf : PfCtl{};
 #define DORY_RUN(NGV, KS)                                                                                 \
-  return packed ? run<NGV, 16, KS, kDecodeBudget, true>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st, W, pfc) \
-                : run<NGV, 16, KS>(ma, X, ldx, M, K, Y, ldy, ps, um, tc, err, st, nullptr, pfc)
+  return packed ? run<NGV, 16, KS, kDecodeBudget, true>(ma, X, ldx, M, K, Y, ldy, ps, um, err, st, W, pfc) \
+                : run<NGV, 16, KS>(ma, X, ldx, M, K, Y, ldy, ps, um, err, st, nullptr, pfc)
     if (NG == 1) {
       if (ksub == 4) DORY_RUN(1, 4);
       if (ksub == 2) DORY_RUN(1, 2);
@@ -610,8 +580,8 @@ cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf
   um.S = 1;
   um.m_tiles = (M + 255) / 256;
   um.units = um.n_tiles * um.m_tiles;
-  if (packed) return run<1, 256, 1, 200 * 1024, true>(ma, X, ldx, M, K, Y, ldy, 0, um, nullptr, err, st, W);
-  return run<1, 256, 1, 200 * 1024>(ma, X, ldx, M, K, Y, ldy, 0, um, nullptr, err, st);
+  if (packed) return run<1, 256, 1, 200 * 1024, true>(ma, X, ldx, M, K, Y, ldy, 0, um, err, st, W);
+  return run<1, 256, 1, 200 * 1024>(ma, X, ldx, M, K, Y, ldy, 0, um, err, st);
 }
 
 }  // namespace dory

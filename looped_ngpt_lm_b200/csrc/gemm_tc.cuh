@@ -8,9 +8,6 @@ namespace dory {
 // Largest split-K factor the GEMM may choose; callers size partial buffers
 // for kMaxSplitK slices.
 constexpr int kMaxSplitK = 8;
-// Device counters a split GEMM needs (one per output tile; zero between
-// launches, and left zero by every launch).
-constexpr int kTileCounters = 4096;
 
 // Weight stream of one forward pass: the weight matrices in the order the
 // pass's GEMMs read them, each at a byte offset of one concatenated stream.
@@ -39,15 +36,12 @@ struct PfCtl {
 // tiles without split.  part_rows: rows available per
 // slice (>= M).  Returns cudaErrorNotSupported for shapes the kernel does not
 // handle (N % 128, K % 64, unaligned pointers).  variant 1 forces one
-// 64-column sub-tile per pipeline stage (for comparisons).  With
-// tile_counters (kTileCounters zeros), the last split of each output tile
-// adds the slices in order s = 0..S-1 inside the kernel and *S is 1.
+// 64-column sub-tile per pipeline stage (for comparisons).
 // packed: W is in the packed tile layout below.  pf: L2 look-ahead (decode
 // tiles only; ignored for prefill tiles).
 cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf16* W, float* Y, int ldy,
                            size_t part_rows, int* err, int batch, bool invariant, int* S, size_t* part_stride,
-                           cudaStream_t st, int variant = 0, unsigned* tile_counters = nullptr,
-                           bool packed = false, const PfCtl* pf = nullptr);
+                           cudaStream_t st, int variant = 0, bool packed = false, const PfCtl* pf = nullptr);
 
 // act[m, j] = silu(g) * u (bf16, row stride dff) with g = X[m] . Wgu[j] and
 // u = X[m] . Wgu[dff + j] for the concatenated [gate; up] weight Wgu
