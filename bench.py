@@ -294,6 +294,57 @@ def spec_leg(dory, torch, shape, dw, args, prompt_len=512, n_new=512, gamma=4):
     return res
 
 
+def mixed_leg(dory, torch, shape, dw, args, prompt_len=512, steps=32):
+    """Mixed-k batched decode at batch 16 (k = 4 for 4 sequences, 2 for 4, 1
+    for 8; last_loop): one dory_decode_step_mixed call per step, against the
+    same sequences decoded as three per-k groups (three graph-replayed
+    decode_step calls per step)."""
+    import synth
+    ks = [4] * 4 + [2] * 4 + [1] * 8
+    B = len(ks)
+    cfg = dory.make_config(shape, max_batch=2 * B, max_seq=prompt_len + 2 * steps + 16, k_max=4, gamma_max=4,
+                           max_chunk=B * prompt_len)
+    h = dory.Handle(cfg, dw, dory.LAST_LOOP)
+    md = dory.LAST_LOOP
+    prompts = [synth.make_prompt(200 + b, prompt_len, shape.vocab) for b in range(B)]
+    tok = torch.tensor(np.concatenate(prompts), dtype=torch.int32, device="cuda")
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    # mixed: sequences 0..B-1
+    ids = list(range(B))
+    t = h.prefill(ids, tok, [prompt_len] * B, 4, md)
+    for _ in range(3):
+        t = h.decode_step_mixed(ids, t, ks, md)
+    torch.cuda.synchronize()
+    a, b = ev(), ev()
+    a.record()
+    for _ in range(steps):
+        t = h.decode_step_mixed(ids, t, ks, md)
+    b.record()
+    torch.cuda.synchronize()
+    mixed_ms = a.elapsed_time(b) / steps
+    # grouped: sequences B..2B-1, one call per k group
+    groups = [(4, list(range(B, B + 4))), (2, list(range(B + 4, B + 8))), (1, list(range(B + 8, 2 * B)))]
+    t2 = h.prefill(list(range(B, 2 * B)), tok, [prompt_len] * B, 4, md)
+    cur = {k: t2[(g[0] - B):(g[0] - B) + len(g)].clone() for k, g in groups}
+    for _ in range(3):
+        for k, g in groups:
+            cur[k] = h.decode_step(g, cur[k], k, md)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(steps):
+        for k, g in groups:
+            cur[k] = h.decode_step(g, cur[k], k, md)
+    b.record()
+    torch.cuda.synchronize()
+    grouped_ms = a.elapsed_time(b) / steps
+    h.close()
+    return {"ks": ks, "mixed_tokens_per_s": round(B * 1e3 / mixed_ms, 1), "mixed_ms_per_step": round(mixed_ms, 3),
+            "grouped_tokens_per_s": round(B * 1e3 / grouped_ms, 1), "grouped_ms_per_step": round(grouped_ms, 3),
+            "speedup_vs_grouped": round(grouped_ms / mixed_ms, 3),
+            "workload": f"batch {B}, prompt {prompt_len}, {steps} steps, last_loop; mixed: one call per step "
+                        f"(eager launches); grouped: one graph-replayed call per k group"}
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -542,6 +593,7 @@ def main():
     if not args.no_aux and world == 1:
         aux["k_mode_sweep"] = sweep_modes(dory, torch, shape, dw, args)
         aux["spec_decode"] = spec_leg(dory, torch, shape, dw, args)
+        aux["mixed_k_decode"] = mixed_leg(dory, torch, shape, dw, args)
 
     if rank == 0:
         line = {

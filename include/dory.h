@@ -162,6 +162,19 @@ dory_status dory_decode_step(dory_handle* h, int32_t batch, const int32_t* seq_i
                              int32_t k, dory_cache_mode mode, float* logits, int32_t* next_tokens,
                              dory_stream stream);
 
+/* One decode step with a loop count per sequence: sequence seq_ids[i] runs
+ * ks[i] loops of the recurrent block.  ks host int32[batch], each in
+ * 1..k_max, non-increasing along the batch (sequences grouped by k): loop t
+ * runs on the sequences with ks[i] >= t only, so the ones that finish early
+ * skip the later loops.  Other arguments and errors as dory_decode_step; a
+ * per_loop sequence must keep the k of its first call.  The loop count is
+ * chosen per request at inference ([news] "How to run"); this call batches
+ * requests with different k.  Each sequence's result equals a decode step of
+ * that sequence at its own k, up to rounding. */
+dory_status dory_decode_step_mixed(dory_handle* h, int32_t batch, const int32_t* seq_ids, const int32_t* tokens_in,
+                                   const int32_t* ks, dory_cache_mode mode, float* logits, int32_t* next_tokens,
+                                   dory_stream stream);
+
 /* Self-speculative greedy decoding ([digest] "Premises & limits"): each step
  * drafts gamma tokens one at a time at k_draft, verifies the chunk
  * [pending, d_1..d_gamma] at k_verify reusing the drafts' input-block output,

@@ -34,7 +34,7 @@ STATUS = {0: "DORY_OK", 1: "DORY_ERR_INVALID_ARG", 2: "DORY_ERR_CAPACITY", 3: "D
 
 # Every entry point include/dory.h declares.
 SYMBOLS = ["dory_workspace_size", "dory_create", "dory_destroy", "dory_reset", "dory_prefill",
-           "dory_decode_step", "dory_spec_decode", "dory_kv_bytes", "dory_seq_len", "dory_read_state",
+           "dory_decode_step", "dory_decode_step_mixed", "dory_spec_decode", "dory_kv_bytes", "dory_seq_len", "dory_read_state",
            "dory_read_kv", "dory_synchronize", "dory_set_option", "dory_profile_read", "dory_profile_reset",
            "dory_last_error", "dory_gemm_bf16", "dory_gemm_bf16_noalloc", "dory_pack_weight_bf16"]
 
@@ -75,6 +75,7 @@ def _load() -> ctypes.CDLL:
         "dory_reset": [P, I32, P],
         "dory_prefill": [P, I32, IP, P, IP, I32, I32, P, P, P],
         "dory_decode_step": [P, I32, IP, P, I32, I32, P, P, P],
+        "dory_decode_step_mixed": [P, I32, IP, P, IP, I32, P, P, P],
         "dory_spec_decode": [P, I32, IP, P, I32, I32, I32, I32, I32, P, P, ctypes.POINTER(SpecStats), P],
         "dory_kv_bytes": [P, I32, I32, I64, ctypes.POINTER(I64)],
         "dory_seq_len": [P, I32, IP],
@@ -262,6 +263,18 @@ class Handle:
         _check(lib.dory_decode_step(self.h, len(seq_ids), ids, ctypes.c_void_p(tokens_in.data_ptr()), k,
                                     MODES[mode], ctypes.c_void_p(_ptr(logits)),
                                     ctypes.c_void_p(next_tokens.data_ptr()), _stream(stream)))
+        return next_tokens
+
+    def decode_step_mixed(self, seq_ids, tokens_in, ks, mode, logits=None, next_tokens=None, stream=None):
+        """One decode step with loop count ks[i] for sequence seq_ids[i] (ks non-increasing)."""
+        import torch
+        ids = self._ids(seq_ids)
+        karr = (ctypes.c_int32 * len(ks))(*ks)
+        if next_tokens is None:
+            next_tokens = torch.empty(len(seq_ids), dtype=torch.int32, device=tokens_in.device)
+        _check(lib.dory_decode_step_mixed(self.h, len(seq_ids), ids, ctypes.c_void_p(tokens_in.data_ptr()), karr,
+                                          MODES[mode], ctypes.c_void_p(_ptr(logits)),
+                                          ctypes.c_void_p(next_tokens.data_ptr()), _stream(stream)))
         return next_tokens
 
     def spec_decode(self, seq_ids, last_tokens, k_draft, k_verify, gamma, mode, max_new, stream=None):

@@ -771,6 +771,48 @@ dory_status decode_t(dory_handle* H, int batch, const int32_t* seq_ids, const in
   return DORY_OK;
 }
 
+// A decode step with a loop count per sequence; rows are ordered by
+// non-increasing k, so loop t runs on the prefix of rows whose k >= t.  Rows
+// that have finished keep their last output (and, in last-loop mode, their
+// own final-loop K/V); the exit normalisation s_k = N(h) covers every row.
+// The decode GEMMs are row-count invariant, so each row's arithmetic does
+// not depend on how many rows share a loop.
+template <typename T>
+dory_status decode_mixed_t(dory_handle* H, int batch, const int32_t* seq_ids, const int32_t* tokens_in,
+                           const int32_t* ks, int mode, float* logits, int32_t* next_tokens, cudaStream_t st) {
+  const dory_config& c = H->c;
+  int max_ctx = 0;
+  for (int i = 0; i < batch; ++i) max_ctx = std::max(max_ctx, H->len[seq_ids[i]] + 1);
+  const int kmax = ks[0], d = c.d_model;
+  RET(upload_ids(H, seq_ids, batch, st));
+  RET(ensure_stream(H, kmax, st));
+  CK(launch_plan_uniform(batch, 1, 0, H->seq_ids, H->seq_len, H->meta, st));
+  Fwd<T> f{H, st, batch, max_ctx, true, mode, kmax, batch, true};
+  follow_stream(H, f, kmax, 0);  // the same weights as a kmax-loop step
+  RET(input_block<T>(f, tokens_in));
+  for (int t = 1; t <= kmax; ++t) {
+    int rows = 0;
+    while (rows < batch && ks[rows] >= t) ++rows;
+    Fwd<T> g = f;
+    g.M = rows;
+    {
+      // u_t = N(s_{t-1} + x), s_0 = x, s_{t-1} = N(h)
+      Scope sc(H, st, "reinject", 0);
+      CK(launch_reinject<T>(rows, d, H->h, H->x, t == 1 ? 0 : 1, H->s, true, H->hop_t<T>(), nullptr, 1, 1, 0, st));
+    }
+    RET(run_layers<T>(g, c.n_in, c.n_in + c.n_rec, t));
+  }
+  {
+    Scope sc(H, st, "reinject", 0);
+    CK(launch_reinject<T>(batch, d, H->h, H->x, 1, nullptr, false, H->hop_t<T>(), H->s, 1, 1, 0, st));
+  }
+  RET(output_and_head<T>(f, batch, nullptr, logits, next_tokens));
+  CK(launch_advance(batch, H->seq_ids, H->seq_len, 1, st));
+  for (int i = 0; i < batch; ++i) H->len[seq_ids[i]] += 1;
+  H->last_rows = batch;
+  return DORY_OK;
+}
+
 template <typename T>
 dory_status spec_t(dory_handle* H, int B, const int32_t* seq_ids, const int32_t* last_tokens, int kv_, int gamma,
                    int mode, int max_new, int32_t* out_tokens, int32_t* out_len, dory_spec_stats* stats,
@@ -962,6 +1004,29 @@ dory_status dory_decode_step(dory_handle* h, int32_t batch, const int32_t* seq_i
                           : decode_t<float>(h, batch, seq_ids, tokens_in, k, mode, logits, next_tokens,
                                             (cudaStream_t)stream);
   if (r == DORY_OK) mark_started(h, batch, seq_ids, k, mode);
+  return r;
+}
+
+dory_status dory_decode_step_mixed(dory_handle* h, int32_t batch, const int32_t* seq_ids, const int32_t* tokens_in,
+                                   const int32_t* ks, dory_cache_mode mode, float* logits, int32_t* next_tokens,
+                                   dory_stream stream) {
+  if (!h) return fail(DORY_ERR_INVALID_ARG, "NULL handle");
+  if (!seq_ids || !ks || !tokens_in || !next_tokens) return fail(DORY_ERR_INVALID_ARG, "NULL argument");
+  if (batch <= 0 || batch > h->c.max_batch)
+    return fail(DORY_ERR_INVALID_ARG, "batch %d outside 1..%d", batch, h->c.max_batch);
+  for (int i = 0; i < batch; ++i) {
+    RET(check_seqs(h, 1, seq_ids + i, ks[i], mode));  // range, mode and per-loop k of each sequence
+    if (i > 0 && ks[i] > ks[i - 1]) return fail(DORY_ERR_INVALID_ARG, "k must not increase along the batch");
+    for (int j = 0; j < i; ++j)
+      if (seq_ids[j] == seq_ids[i]) return fail(DORY_ERR_INVALID_ARG, "seq id %d repeated", seq_ids[i]);
+    if (h->len[seq_ids[i]] + 1 > h->c.max_seq)
+      return fail(DORY_ERR_CAPACITY, "sequence %d would exceed max_seq", seq_ids[i]);
+  }
+  const cudaStream_t st = (cudaStream_t)stream;
+  dory_status r = h->bf16 ? decode_mixed_t<bf16>(h, batch, seq_ids, tokens_in, ks, mode, logits, next_tokens, st)
+                          : decode_mixed_t<float>(h, batch, seq_ids, tokens_in, ks, mode, logits, next_tokens, st);
+  if (r == DORY_OK)
+    for (int i = 0; i < batch; ++i) mark_started(h, 1, seq_ids + i, ks[i], mode);
   return r;
 }
 

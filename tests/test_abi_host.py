@@ -110,6 +110,14 @@ def test_argument_validation():
     D = lambda *a: status_name(lib.dory_decode_step(h, *a))
     assert D(1, ids, tok, 9, 0, None, nt, None) == "DORY_ERR_INVALID_ARG"
     assert D(1, ids, None, 2, 0, None, nt, None) == "DORY_ERR_INVALID_ARG"
+    X = lambda ks, mode=0: status_name(lib.dory_decode_step_mixed(h, len(ks), ids, tok, (ctypes.c_int32 * len(ks))(*ks),
+                                                                  mode, None, nt, None))
+    assert X([1, 2]) == "DORY_ERR_INVALID_ARG"      # k increases along the batch
+    assert X([5, 1]) == "DORY_ERR_INVALID_ARG"      # k > k_max
+    assert X([2, 0]) == "DORY_ERR_INVALID_ARG"      # k = 0
+    assert X([2, 1], 1) == "DORY_ERR_STATE"         # per_loop on a last_loop handle
+    assert status_name(lib.dory_decode_step_mixed(h, 2, dup, tok, (ctypes.c_int32 * 2)(2, 1), 0, None, nt,
+                                                  None)) == "DORY_ERR_INVALID_ARG"  # repeated id
     assert lib.dory_set_option(h, 99, 1) == 1
     n = ctypes.c_int32()
     assert lib.dory_seq_len(h, 0, ctypes.byref(n)) == 0 and n.value == 0
