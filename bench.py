@@ -345,6 +345,31 @@ def mixed_leg(dory, torch, shape, dw, args, prompt_len=512, steps=32):
                         f"(eager launches); grouped: one graph-replayed call per k group"}
 
 
+def sampling_leg(dory, torch, h, tok, args, mode, steps=64):
+    """Batch-1 decode at k = args.k with top-p sampling (temperature 1.0,
+    top-p 0.95, the released model's settings) against greedy choice, on the
+    bench's own handle and sequence."""
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    out = {}
+    bufs = [torch.empty(1, dtype=torch.int32, device="cuda") for _ in range(2)]
+    for name, T in (("greedy", 0.0), ("top_p_0.95_T_1.0", 1.0)):
+        h.set_sampling(T, 0.95 if T > 0 else 1.0, 1234)
+        for i in range(3):
+            tok = h.decode_step([0], tok, args.k, mode, next_tokens=bufs[i % 2])
+        torch.cuda.synchronize()
+        a, b = ev(), ev()
+        a.record()
+        for i in range(steps):
+            tok = h.decode_step([0], tok, args.k, mode, next_tokens=bufs[i % 2])
+        b.record()
+        torch.cuda.synchronize()
+        out[name] = {"tokens_per_s": round(steps * 1e3 / a.elapsed_time(b), 2),
+                     "ms_per_step": round(a.elapsed_time(b) / steps, 4)}
+    h.set_sampling(0.0, 1.0, 0)
+    out["sampler_ms_per_step"] = round(out["top_p_0.95_T_1.0"]["ms_per_step"] - out["greedy"]["ms_per_step"], 4)
+    return out, tok
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -557,6 +582,7 @@ def main():
                                "hbm_frac_of_measured": round(by / (ms / 1e3) / 1e9 / hbm, 4),
                                "bytes_per_token": by, "ctx": ctx}
         aux["decode_k_sweep_last_loop" if args.mode == "last_loop" else "decode_k_sweep"] = sweep
+        aux["sampling"], tok = sampling_leg(dory, torch, h, tok, args, mode)
         # ---- end to end: every step copies its input token from pinned host
         # memory and reads the chosen token back, through the public API
         pin_in = torch.empty(1, dtype=torch.int32).pin_memory()

@@ -282,6 +282,26 @@ enum {
 };
 dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value);
 
+/* Token choice of prefill and decode steps.  temperature 0 (default):
+ * greedy, lowest id on ties.  temperature > 0: top-p sampling ([news] "How
+ * to run" names temperature 1.0, top-p 0.95 for the released model): one
+ * Philox4x32-10 draw per new token (key = seed, counter = (sequence id,
+ * position of the new token, 0, 0)), integer nucleus masses
+ * q_i = floor(exp2((l_i - max) log2(e) / T) * 2^31), nucleus = tokens with
+ * q_i >= tau for the largest tau whose tail mass reaches ceil(top_p * sum q),
+ * token = first id at which the running nucleus mass exceeds
+ * floor(u * nucleus mass).  top_p in (0, 1].  Speculative decoding stays
+ * greedy (DORY_ERR_UNSUPPORTED while temperature > 0). */
+dory_status dory_set_sampling(dory_handle* h, float temperature, float top_p, uint64_t seed);
+
+/* The sampler alone: rows of device logits [rows, vocab] (fp32), draw of row
+ * i keyed by device seq[i], pos[i]; scratch device uint32[rows * vocab] (may
+ * alias logits, which are then overwritten); out device int32[rows].
+ * temperature > 0.  Queues work on `stream`. */
+dory_status dory_sample(const float* logits, int32_t rows, int32_t vocab, const int32_t* seq, const int32_t* pos,
+                        float temperature, float top_p, uint64_t seed, uint32_t* scratch, int32_t* out,
+                        dory_stream stream);
+
 /* Per-kernel launch statistics gathered while DORY_OPT_PROFILE is on:
  * fills up to n entries of names (host char[n][48]), launches, total_ms and
  * algorithmic bytes; returns the number of kernels in *count. */

@@ -36,7 +36,8 @@ STATUS = {0: "DORY_OK", 1: "DORY_ERR_INVALID_ARG", 2: "DORY_ERR_CAPACITY", 3: "D
 SYMBOLS = ["dory_workspace_size", "dory_create", "dory_destroy", "dory_reset", "dory_prefill",
            "dory_decode_step", "dory_decode_step_mixed", "dory_spec_decode", "dory_kv_bytes", "dory_seq_len", "dory_read_state",
            "dory_read_kv", "dory_synchronize", "dory_set_option", "dory_profile_read", "dory_profile_reset",
-           "dory_last_error", "dory_gemm_bf16", "dory_gemm_bf16_noalloc", "dory_pack_weight_bf16"]
+           "dory_last_error", "dory_gemm_bf16", "dory_gemm_bf16_noalloc", "dory_pack_weight_bf16",
+           "dory_set_sampling", "dory_sample"]
 
 
 class DoryError(RuntimeError):
@@ -89,6 +90,8 @@ def _load() -> ctypes.CDLL:
         "dory_gemm_bf16": [I32, I32, I32, P, P, P, I32, I32, I32, IP, P, P],
         "dory_gemm_bf16_noalloc": [I32, I32, I32, P, P, P, I32, P],
         "dory_pack_weight_bf16": [P, P, I32, I32, P],
+        "dory_set_sampling": [P, ctypes.c_float, ctypes.c_float, ctypes.c_uint64],
+        "dory_sample": [P, I32, I32, P, P, ctypes.c_float, ctypes.c_float, ctypes.c_uint64, P, P, P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -264,6 +267,10 @@ class Handle:
                                     MODES[mode], ctypes.c_void_p(_ptr(logits)),
                                     ctypes.c_void_p(next_tokens.data_ptr()), _stream(stream)))
         return next_tokens
+
+    def set_sampling(self, temperature: float, top_p: float = 1.0, seed: int = 0):
+        """temperature 0: greedy; > 0: top-p sampling with seeded per-token draws."""
+        _check(lib.dory_set_sampling(self.h, temperature, top_p, seed))
 
     def decode_step_mixed(self, seq_ids, tokens_in, ks, mode, logits=None, next_tokens=None, stream=None):
         """One decode step with loop count ks[i] for sequence seq_ids[i] (ks non-increasing)."""

@@ -137,6 +137,8 @@ struct dory_handle {
   int prefill_tc = 2;  // long-chunk attention: 2 tcgen05 (head_dim 128), 1 mma.sync, 0 CUDA cores
   int gemm_impl = 0;
   unsigned long long pf_lead = 8ull << 20;   // 0: no L2 look-ahead
+  float temperature = 0.f, top_p = 1.f;      // temperature 0: greedy
+  unsigned long long seed = 0;
   std::vector<std::vector<PfSeg>> pf_host;   // [k] -> stream of a k-loop decode step
   std::vector<char> pf_uploaded;             // [k]
   int pf_pos = -1;                           // next segment of the pass being issued; -1 off
@@ -564,6 +566,13 @@ dory_status output_and_head(const Fwd<T>& f, int nrows, const int* rows, float* 
   if (S != 1 || lg != H->logits) {
     Scope sc(H, f.st, "split_reduce", 0);
     CK(launch_split_reduce(nrows, c.vocab, H->logits, S, ps, lg, f.st));
+  }
+  if (H->temperature > 0.f) {
+    // the draw of head row i is keyed by the sequence and the new token's position
+    Scope sc(H, f.st, "sample", 0);
+    CK(launch_sample(nrows, c.vocab, lg, (uint32_t*)H->logits, rows, H->meta.seq, H->meta.pos, 1, H->temperature,
+                     H->top_p, H->seed, choice, f.st));
+    return DORY_OK;
   }
   Scope sc(H, f.st, "argmax", 0);
   CK(launch_argmax(nrows, c.vocab, lg, choice, f.st));
@@ -1036,6 +1045,7 @@ dory_status dory_spec_decode(dory_handle* h, int32_t batch, const int32_t* seq_i
   if (!h) return fail(DORY_ERR_INVALID_ARG, "NULL handle");
   RET(check_seqs(h, batch, seq_ids, k_verify, mode));
   if (k_draft != 1) return fail(DORY_ERR_UNSUPPORTED, "k_draft must be 1 (loop-1 reuse)");
+  if (h->temperature > 0.f) return fail(DORY_ERR_UNSUPPORTED, "speculative decoding is greedy only");
   if (gamma < 1 || gamma > h->c.gamma_max) return fail(DORY_ERR_INVALID_ARG, "gamma %d outside 1..%d", gamma, h->c.gamma_max);
   if (max_new < 1) return fail(DORY_ERR_INVALID_ARG, "max_new must be >= 1");
   if (!last_tokens || !out_tokens || !out_len) return fail(DORY_ERR_INVALID_ARG, "NULL argument");
@@ -1180,6 +1190,34 @@ dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value) {
       return DORY_OK;
   }
   return fail(DORY_ERR_INVALID_ARG, "unknown option %d", opt);
+}
+
+dory_status dory_set_sampling(dory_handle* h, float temperature, float top_p, uint64_t seed) {
+  if (!h) return fail(DORY_ERR_INVALID_ARG, "NULL handle");
+  if (!(temperature >= 0.f) || !(top_p > 0.f) || top_p > 1.f)
+    return fail(DORY_ERR_INVALID_ARG, "temperature must be >= 0 and top_p in (0, 1]");
+  if (temperature != h->temperature || top_p != h->top_p || seed != h->seed) {
+    // graphs captured with the old choice rule are dropped
+    for (auto& g : h->graphs_cache)
+      if (g.exec) cudaGraphExecDestroy(g.exec);
+    h->graphs_cache.clear();
+  }
+  h->temperature = temperature;
+  h->top_p = top_p;
+  h->seed = seed;
+  return DORY_OK;
+}
+
+dory_status dory_sample(const float* logits, int32_t rows, int32_t vocab, const int32_t* seq, const int32_t* pos,
+                        float temperature, float top_p, uint64_t seed, uint32_t* scratch, int32_t* out,
+                        dory_stream stream) {
+  if (!logits || !seq || !pos || !scratch || !out) return fail(DORY_ERR_INVALID_ARG, "NULL argument");
+  if (rows <= 0 || vocab <= 0) return fail(DORY_ERR_INVALID_ARG, "rows and vocab must be positive");
+  if (!(temperature > 0.f) || !(top_p > 0.f) || top_p > 1.f)
+    return fail(DORY_ERR_INVALID_ARG, "temperature must be > 0 and top_p in (0, 1]");
+  CK(launch_sample(rows, vocab, logits, scratch, nullptr, seq, pos, 0, temperature, top_p, seed, out,
+                   (cudaStream_t)stream));
+  return DORY_OK;
 }
 
 dory_status dory_profile_reset(dory_handle* h) {

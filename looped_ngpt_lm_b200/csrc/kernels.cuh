@@ -103,6 +103,12 @@ cudaError_t launch_gemm_simt(int M, int N, int K, const T* X, int ldx, const T* 
 
 // Greedy choice per row (largest logit, lowest id on ties).
 cudaError_t launch_argmax(int R, int V, const float* logits, int* out, cudaStream_t st);
+// Temperature / top-p sampling of R rows of V logits (see sample.cu): the
+// draw of row i uses counter (seq[m], pos[m] + pos_add) with m = rows ? rows[i]
+// : i; qbuf: [R, V] uint32 scratch (may alias the logits).  out: token ids.
+cudaError_t launch_sample(int R, int V, const float* logits, uint32_t* qbuf, const int* rows, const int* seq,
+                          const int* pos, int pos_add, float temperature, float top_p, unsigned long long seed,
+                          int* out, cudaStream_t st);
 
 // Speculative acceptance for B sequences.  drafts[i * dstride + b] = d_{i+1},
 // vtok [B, gamma+1] verifier choices.  Appends accepted tokens to out

@@ -68,7 +68,9 @@ def nucleus_threshold(q: np.ndarray, top_p: float) -> int:
 
 
 def sample(logits, temperature: float, top_p: float, seed: int, seq: int, pos: int) -> int:
-    """The token drawn for sequence `seq` at position `pos`."""
+    """The token drawn for sequence `seq` at position `pos`.  Temperature and
+    top_p are float32 parameters (rounded to float32 first)."""
+    temperature, top_p = float(np.float32(temperature)), float(np.float32(top_p))
     q = masses(logits, temperature)
     tau = nucleus_threshold(q, top_p)
     mass = np.where(q >= tau, q, 0)
