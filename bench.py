@@ -370,6 +370,70 @@ def sampling_leg(dory, torch, h, tok, args, mode, steps=64):
     return out, tok
 
 
+def mxfp8_leg(dory, torch, shape, dw, args, mode, bf16_sweep, steps=32):
+    """Batch-1 decode with MXFP8 weights (E4M3 codes, one E8M0 scale per 32
+    weights, quantised on the GPU from the bench's bf16 weights) at k = 1, 2,
+    4 on a handle of its own: prefill reads the exact bf16 dequantisation,
+    decode GEMMs the 8-bit copies.  Reports tokens/s, the speed-up over the
+    bf16 k sweep at the same context, and the GEMV's HBM roofline."""
+    import synth
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    mx = dory.MxWeights(dw)
+    cfg = dory.make_config(shape, max_batch=1, max_seq=args.prompt + 8 * steps + 64, k_max=4, gamma_max=4,
+                           max_chunk=args.prompt)
+    h = dory.Handle(cfg, mx.dequantised, dory.LAST_LOOP if args.mode == "last_loop" else dory.PER_LOOP)
+    h.attach_mxfp8(mx)
+    prompt = torch.tensor(synth.make_prompt(1, args.prompt, shape.vocab), dtype=torch.int32, device="cuda")
+    tok = h.prefill([0], prompt, [args.prompt], args.k, mode)
+    bufs = [torch.empty(1, dtype=torch.int32, device="cuda") for _ in range(2)]
+    out = {}
+    for kk in (1, 2, 4):
+        if args.mode == "per_loop" and kk != args.k:
+            continue
+        for i in range(3):
+            tok = h.decode_step([0], tok, kk, mode, next_tokens=bufs[i % 2])
+        torch.cuda.synchronize()
+        a, b = ev(), ev()
+        a.record()
+        for i in range(steps):
+            tok = h.decode_step([0], tok, kk, mode, next_tokens=bufs[i % 2])
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / steps
+        r = {"tokens_per_s": round(1e3 / ms, 2), "ms_per_token": round(ms, 4), "ctx": h.seq_len(0)}
+        ref = (bf16_sweep or {}).get(f"k{kk}")
+        if ref:
+            r["speedup_vs_bf16"] = round(r["tokens_per_s"] / ref["tokens_per_s"], 3)
+        out[f"k{kk}"] = r
+    # the GEMV's own time: CUDA events around every launch of two steps
+    h.profile_reset()
+    h.set_option(dory.OPT_PROFILE, 1)
+    for i in range(2):
+        tok = h.decode_step([0], tok, args.k, mode, next_tokens=bufs[i % 2])
+    prof = h.profile_read()
+    h.set_option(dory.OPT_PROFILE, 0)
+    gemv = {n: v for n, v in prof.items() if n.startswith("gemm")}
+    g_ms = sum(v["ms"] for v in gemv.values())
+    g_bytes = sum(v["bytes"] for v in gemv.values())
+    g_launch = sum(v["launches"] for v in gemv.values())
+    tot_ms = sum(v["ms"] for v in prof.values())
+    hbm = peaks()[0]
+    achieved = g_bytes / (g_ms / 1e3) / 1e9 if g_ms > 0 else 0.0
+    out["gemv_roofline"] = {"bound": "hbm", "kernel": "k_mx_gemv (decode projections + LM head, MXFP8)",
+                            "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                            "frac": round(achieved / hbm, 4), "bytes_per_launch": round(g_bytes / max(g_launch, 1)),
+                            "avg_launch_us": round(1e3 * g_ms / max(g_launch, 1), 2),
+                            "share_of_step": round(g_ms / tot_ms, 4) if tot_ms else None}
+    out["weight_bytes"] = mx.nbytes()
+    out["workload"] = (f"batch 1, prompt {args.prompt}, {steps} timed steps per k, {args.mode}; MXFP8 copies of "
+                       f"every projection and the LM head (embedding bf16)")
+    out["pages_ratio"] = "MXFP8 over BF16 at batch 1 on a DGX Spark: 1.69x (in 2560 / out 300), 1.84x (in 128 / out 1024)"
+    h.close()
+    del mx
+    torch.cuda.empty_cache()
+    return out
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -583,6 +647,7 @@ def main():
                                "bytes_per_token": by, "ctx": ctx}
         aux["decode_k_sweep_last_loop" if args.mode == "last_loop" else "decode_k_sweep"] = sweep
         aux["sampling"], tok = sampling_leg(dory, torch, h, tok, args, mode)
+        aux["mxfp8_decode"] = mxfp8_leg(dory, torch, shape, dw, args, mode, sweep)
         # ---- end to end: every step copies its input token from pinned host
         # memory and reads the chosen token back, through the public API
         pin_in = torch.empty(1, dtype=torch.int32).pin_memory()

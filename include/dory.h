@@ -18,6 +18,10 @@
  *             정밀도로 공개": "Looped structure" (input re-injected every loop),
  *             "How to run" (loop count 1..4 chosen at inference; the
  *             recurrent KV cache mode switch last_loop / per-loop).
+ *   [trawling] trawling.dev/post/2766 "NVIDIA, 반복 연산형 4B 언어 모델 Dory
+ *             공개": "KV 캐시와 실행 환경" (KV cache and runtime: the
+ *             released weight formats BF16, MXFP8, NVFP4, Q5_K_M; MXFP8
+ *             decodes 1.69x to 1.84x faster than BF16 at batch 1).
  *   [review]  blog.secrett2633.cloud "[논문리뷰] Dory1.0-4B: A Looped
  *             Normalized-GPT", "1. Key Terms" (nGPT: L2-normalised states;
  *             last-loop KV caching keeps the footprint of one loop).
@@ -259,6 +263,72 @@ dory_status dory_gemm_bf16_noalloc(int32_t M, int32_t N, int32_t K, const void* 
  * The tensor-core GEMM streams packed weights with one bulk copy per pipeline
  * stage.  Queues work on `stream`. */
 dory_status dory_pack_weight_bf16(const void* src, void* dst, int32_t N, int32_t K, dory_stream stream);
+
+/* ---------------------------------------------------------------- MXFP8
+ * 8-bit weights for decoding.  The pages list MXFP8 among the released weight
+ * formats and measure it against BF16 at batch 1 ([trawling] "KV cache and
+ * runtime"; [news] "Training and variants": 1.69x to 1.84x on a DGX Spark).  The format is the OCP
+ * Microscaling Formats (MX) v1.0 MXFP8: FP8 E4M3 codes (bias 7, largest
+ * finite 448, subnormals m/8 * 2^-6) and one E8M0 scale byte
+ * (2^(byte - 127)) per 32 consecutive weights of a row.  Codes are
+ * row-major [N, K] bytes; scales are row-major [N, K/32] bytes.  The scale of
+ * weight (n, k) is scales[n*K/32 + k/32].
+ *
+ * Quantise a row-major bf16 weight w [N, K] (device, 16-byte aligned,
+ * K % 32 == 0).  For each block, shared = floor(log2(max |w|)) - 8, clamped
+ * to [-127, 127] (-127 for a block of zeros), and scale byte = shared + 127.
+ * Each code is E4M3(w * 2^-shared), rounded to nearest-even, with
+ * magnitudes above 448 clamped to 448; a value that rounds to zero keeps its
+ * sign.  q: device [N, K] bytes (16-byte aligned); scales: device [N, K/32]
+ * bytes.  w_deq (device, nullable, 16-byte aligned) receives the
+ * dequantised weights 2^shared * E4M3(code) rounded to bf16 [N, K], which
+ * is exact unless a block's scale is below 2^-120.  A non-finite weight sets
+ * *err_word (device int32, nullable); dory_synchronize then reports
+ * DORY_ERR_INVALID_ARG.  Queues work on `stream`. */
+dory_status dory_quantize_mxfp8(const void* w, int32_t N, int32_t K, void* q, void* scales, void* w_deq,
+                                int32_t* err_word, dory_stream stream);
+
+/* y[i, n] = sum_k x[i, k] * 2^(scales[n, k/32] - 127) * E4M3(q[n, k]) for
+ * i < M, n < N, in fp32.  x is bf16 [M, ldx] (device) and y is fp32
+ * [M, ldy] (device).  Each y[i, n] is summed in an order fixed by K alone,
+ * so its bits do not depend on M.  Requires K % 32 == 0, K <= 40960,
+ * ldx >= K, ldy >= N and q 16-byte aligned.  The supported range is
+ * |x| < 2^64 and scale bytes <= 198 (what the quantiser writes for
+ * |w| < 2^80).  An activation outside it sets *err_word (device, nullable).
+ * Queues work on `stream`. */
+dory_status dory_gemv_mxfp8(int32_t M, int32_t N, int32_t K, const void* x, int32_t ldx, const void* q,
+                            const void* scales, float* y, int32_t ldy, int32_t* err_word, dory_stream stream);
+
+/* MXFP8 copies of a handle's projection weights and LM head (device
+ * pointers, BORROWED: they must outlive the attachment).  The per-layer
+ * arrays are indexed by physical layer.  qkv_* and o_* entries are read for
+ * attention layers, gu_* and down_* entries for MLP layers.  An entry whose
+ * code and scale pointers are both NULL (or a NULL array) leaves that matrix
+ * in bf16. */
+typedef struct {
+  const void* lm_head_q;
+  const void* lm_head_s;
+  const void* const* qkv_q;
+  const void* const* qkv_s;
+  const void* const* o_q;
+  const void* const* o_s;
+  const void* const* gu_q;
+  const void* const* gu_s;
+  const void* const* down_q;
+  const void* const* down_s;
+} dory_mx_weights;
+
+/* Attach MXFP8 copies (mx != NULL) or detach them (mx == NULL).  While they
+ * are attached, the GEMMs of decode steps (plain, mixed-k and speculative)
+ * run dory_gemv_mxfp8 on the copies.  Prefill keeps the bf16 weights given
+ * to dory_create.  For a forward that is the dequantised model throughout,
+ * create the handle with the w_deq output of dory_quantize_mxfp8.  Attaching
+ * drops captured decode graphs and turns the L2 look-ahead off.  The handle
+ * must hold bf16 weights, and d_model, n_heads * head_dim and d_ff must be
+ * multiples of 32 (else DORY_ERR_UNSUPPORTED).  A copy with codes but no
+ * scales, or codes that are not 16-byte aligned, gives DORY_ERR_INVALID_ARG
+ * and leaves the previous attachment in place. */
+dory_status dory_attach_mxfp8(dory_handle* h, const dory_mx_weights* mx);
 
 /* Synchronise `stream` and report device-side errors (DORY_ERR_TIMEOUT when
  * a bounded wait in a kernel gave up; the handle stays usable). */

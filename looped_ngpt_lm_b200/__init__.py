@@ -37,7 +37,7 @@ SYMBOLS = ["dory_workspace_size", "dory_create", "dory_destroy", "dory_reset", "
            "dory_decode_step", "dory_decode_step_mixed", "dory_spec_decode", "dory_kv_bytes", "dory_seq_len", "dory_read_state",
            "dory_read_kv", "dory_synchronize", "dory_set_option", "dory_profile_read", "dory_profile_reset",
            "dory_last_error", "dory_gemm_bf16", "dory_gemm_bf16_noalloc", "dory_pack_weight_bf16",
-           "dory_set_sampling", "dory_sample"]
+           "dory_set_sampling", "dory_sample", "dory_quantize_mxfp8", "dory_gemv_mxfp8", "dory_attach_mxfp8"]
 
 
 class DoryError(RuntimeError):
@@ -57,6 +57,12 @@ class Weights(ctypes.Structure):
     _fields_ = [("embed", ctypes.c_void_p), ("lm_head", ctypes.c_void_p),
                 ("w_qkv", ctypes.POINTER(ctypes.c_void_p)), ("w_o", ctypes.POINTER(ctypes.c_void_p)),
                 ("w_gu", ctypes.POINTER(ctypes.c_void_p)), ("w_down", ctypes.POINTER(ctypes.c_void_p))]
+
+
+class MxWeightsC(ctypes.Structure):
+    _fields_ = [("lm_head_q", ctypes.c_void_p), ("lm_head_s", ctypes.c_void_p)] + [
+        (n, ctypes.POINTER(ctypes.c_void_p)) for n in (
+            "qkv_q", "qkv_s", "o_q", "o_s", "gu_q", "gu_s", "down_q", "down_s")]
 
 
 class SpecStats(ctypes.Structure):
@@ -92,6 +98,9 @@ def _load() -> ctypes.CDLL:
         "dory_pack_weight_bf16": [P, P, I32, I32, P],
         "dory_set_sampling": [P, ctypes.c_float, ctypes.c_float, ctypes.c_uint64],
         "dory_sample": [P, I32, I32, P, P, ctypes.c_float, ctypes.c_float, ctypes.c_uint64, P, P, P],
+        "dory_quantize_mxfp8": [P, I32, I32, P, P, P, P, P],
+        "dory_gemv_mxfp8": [I32, I32, I32, P, I32, P, P, P, I32, P, P],
+        "dory_attach_mxfp8": [P, ctypes.POINTER(MxWeightsC)],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -154,6 +163,30 @@ class DeviceWeights:
             else:
                 self.gu[l] = up(np.concatenate([weights[f"L{l}.wg"], weights[f"L{l}.wu"]]))
                 self.down[l] = up(weights[f"L{l}.wdown"])
+        self._bind()
+
+    @classmethod
+    def from_tensors(cls, shape, embed, lm_head, qkv, o, gu, down):
+        """Device weights from CUDA tensors already in the ABI layout."""
+        self = cls.__new__(cls)
+        self.shape = shape
+        self.bf16 = shape.dtype == "bf16"
+        self.tensors = {"embed": embed, "lm_head": lm_head}
+        self.qkv, self.o, self.gu, self.down = list(qkv), list(o), list(gu), list(down)
+        self._bind()
+        return self
+
+    def matrices(self):
+        """(name, tensor) of every projection matrix and the LM head."""
+        out = [("lm_head", self.tensors["lm_head"])]
+        for l in range(self.shape.n_layers):
+            for name, t in (("qkv", self.qkv[l]), ("o", self.o[l]), ("gu", self.gu[l]), ("down", self.down[l])):
+                if t is not None:
+                    out.append((f"{name}{l}", t))
+        return out
+
+    def _bind(self):
+        L = self.shape.n_layers
         arr = ctypes.c_void_p * L
         self._qkv = arr(*[_ptr(t) for t in self.qkv])
         self._o = arr(*[_ptr(t) for t in self.o])
@@ -203,6 +236,63 @@ def pack_weight_bf16(W, stream=None):
     return out
 
 
+def quantize_mxfp8(W, dequantised=True, err=None, stream=None):
+    """MXFP8 copy of a row-major [N, K] bf16 CUDA tensor: (codes uint8 [N, K],
+    scales uint8 [N, K/32], dequantised bf16 [N, K] or None)."""
+    import torch
+    N, K = W.shape
+    q = torch.empty((N, K), dtype=torch.uint8, device=W.device)
+    sc = torch.empty((N, K // 32), dtype=torch.uint8, device=W.device)
+    deq = torch.empty((N, K), dtype=torch.bfloat16, device=W.device) if dequantised else None
+    _check(lib.dory_quantize_mxfp8(ctypes.c_void_p(W.data_ptr()), N, K, ctypes.c_void_p(q.data_ptr()),
+                                   ctypes.c_void_p(sc.data_ptr()), ctypes.c_void_p(_ptr(deq)),
+                                   ctypes.c_void_p(_ptr(err)), _stream(stream)))
+    return q, sc, deq
+
+
+def gemv_mxfp8(X, q, scales, Y=None, err=None, stream=None):
+    """Y = X . dequantize(q, scales)^T through dory_gemv_mxfp8 (X bf16 [M, K])."""
+    import torch
+    M, K = X.shape
+    N = q.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float32, device=X.device)
+    _check(lib.dory_gemv_mxfp8(M, N, K, ctypes.c_void_p(X.data_ptr()), X.stride(0), ctypes.c_void_p(q.data_ptr()),
+                               ctypes.c_void_p(scales.data_ptr()), ctypes.c_void_p(Y.data_ptr()), Y.stride(0),
+                               ctypes.c_void_p(_ptr(err)), _stream(stream)))
+    return Y
+
+
+class MxWeights:
+    """MXFP8 copies of a DeviceWeights' projection matrices and LM head
+    (made on the GPU by dory_quantize_mxfp8), plus `dequantised`: a
+    DeviceWeights holding their exact bf16 dequantisation (same embedding)
+    for the handle's prefill GEMMs."""
+
+    def __init__(self, dw: DeviceWeights, stream=None):
+        self.shape = dw.shape
+        L = dw.shape.n_layers
+        self.q, self.s = {}, {}
+        deq = {}
+        for name, t in dw.matrices():
+            self.q[name], self.s[name], deq[name] = quantize_mxfp8(t, stream=stream)
+        pick = lambda kind: [deq.get(f"{kind}{l}") for l in range(L)]  # noqa: E731
+        self.dequantised = DeviceWeights.from_tensors(dw.shape, dw.tensors["embed"], deq["lm_head"], pick("qkv"),
+                                                      pick("o"), pick("gu"), pick("down"))
+        arr = ctypes.c_void_p * L
+
+        def ptrs(d, kind):
+            return arr(*[_ptr(d.get(f"{kind}{l}")) for l in range(L)])
+
+        self._keep = {f"{k}_{x}": ptrs(d, k) for k in ("qkv", "o", "gu", "down") for x, d in (("q", self.q),
+                                                                                                ("s", self.s))}
+        self.c = MxWeightsC(self.q["lm_head"].data_ptr(), self.s["lm_head"].data_ptr(),
+                            *[self._keep[f"{k}_{x}"] for k in ("qkv", "o", "gu", "down") for x in ("q", "s")])
+
+    def nbytes(self) -> int:
+        return sum(t.numel() for t in self.q.values()) + sum(t.numel() for t in self.s.values())
+
+
 def workspace_size(cfg: Config, alloc_mode=LAST_LOOP) -> int:
     n = ctypes.c_size_t()
     _check(lib.dory_workspace_size(ctypes.byref(cfg), MODES[alloc_mode], ctypes.byref(n)))
@@ -246,6 +336,11 @@ class Handle:
 
     def set_option(self, opt, value):
         _check(lib.dory_set_option(self.h, opt, int(value)))
+
+    def attach_mxfp8(self, mx: "MxWeights | None"):
+        """Decode GEMMs read these MXFP8 copies (None detaches)."""
+        self.mx = mx
+        _check(lib.dory_attach_mxfp8(self.h, ctypes.byref(mx.c) if mx is not None else None))
 
     def prefill(self, seq_ids, tokens, lens, k, mode, logits=None, next_tokens=None, stream=None):
         import torch

@@ -14,7 +14,8 @@ enum : int {
   DEV_ERR_NONE = 0,
   DEV_ERR_TIMEOUT = 1,   // a bounded wait gave up
   DEV_ERR_BAD_TOKEN = 2, // token id outside [0, vocab)
-  DEV_ERR_BAD_INDEX = 3  // a cache index check failed
+  DEV_ERR_BAD_INDEX = 3, // a cache index check failed
+  DEV_ERR_RANGE = 4      // a value outside a kernel's supported range (non-finite weight, |x| >= 2^64)
 };
 
 __device__ __forceinline__ float to_f(float v) { return v; }

@@ -18,6 +18,7 @@
 #include <cstdio>
 #include <cstring>
 #include <string>
+#include <unordered_map>
 #include <vector>
 
 #include "dory.h"
@@ -25,6 +26,7 @@
 #include "attn_prefill.cuh"
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
+#include "mxfp8.cuh"
 
 namespace dory {
 bool g_pdl = true;
@@ -102,6 +104,13 @@ struct dory_handle {
   const void* embed = nullptr;
   const void* head = nullptr;
   std::vector<const void*> w_qkv, w_o, w_gu, w_down;
+  // MXFP8 copies read by the decode / speculative GEMMs, keyed by the bf16
+  // weight they stand for (empty: none attached)
+  struct MxMat {
+    const uint8_t* q;
+    const uint8_t* s;
+  };
+  std::unordered_map<const void*, MxMat> mx;
   std::vector<int> attn_of;
   std::vector<AttnLayer> attn;
 
@@ -361,10 +370,21 @@ template <typename T>
 dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, const void* W, float* Y, int ldy,
                  size_t part_rows, int* S_out, size_t* ps_out, const char* name) {
   dory_handle* H = f.H;
-  double bytes = (double)N * K * sizeof(T) + (double)M * K * sizeof(T) + (double)M * N * 4;
-  Scope sc(H, f.st, name, bytes);
   *S_out = 1;
   *ps_out = 0;
+  if constexpr (sizeof(T) == 2) {
+    // decode and speculative rows read the MXFP8 copy when one is attached
+    if (f.invariant && !H->mx.empty()) {
+      auto it = H->mx.find(W);
+      if (it != H->mx.end()) {
+        Scope sc(H, f.st, name, (double)N * K * (1.0 + 1.0 / kMxBlock) + (double)M * K * 2 + (double)M * N * 4);
+        CK(launch_mx_gemv(M, N, K, (const bf16*)X, ldx, it->second.q, it->second.s, Y, ldy, H->err, f.st));
+        return DORY_OK;
+      }
+    }
+  }
+  double bytes = (double)N * K * sizeof(T) + (double)M * K * sizeof(T) + (double)M * N * 4;
+  Scope sc(H, f.st, name, bytes);
   if constexpr (sizeof(T) == 2) {
     if (H->gemm_impl != 1) {
       int S = 1;
@@ -659,7 +679,7 @@ dory_status prefill_t(dory_handle* H, int batch, const int32_t* seq_ids, const i
 // input block, k passes over the recurrent block, the output block, the LM
 // head.  Uploaded once per k (outside any graph capture).
 dory_status ensure_stream(dory_handle* H, int k, cudaStream_t st) {
-  if (H->pf_lead == 0 || !H->bf16 || H->gemm_impl == 1) return DORY_OK;
+  if (H->pf_lead == 0 || !H->bf16 || H->gemm_impl == 1 || !H->mx.empty()) return DORY_OK;
   if ((int)H->pf_host.size() <= k) {
     H->pf_host.resize(k + 1);
     H->pf_uploaded.resize(k + 1, 0);
@@ -699,7 +719,7 @@ dory_status ensure_stream(dory_handle* H, int k, cudaStream_t st) {
 // from its segment `pos` on (L2 look-ahead), when that stream is uploaded.
 template <typename T>
 void follow_stream(dory_handle* H, Fwd<T>& f, int k, int pos) {
-  const bool on = H->pf_lead > 0 && (int)H->pf_uploaded.size() > k && H->pf_uploaded[k];
+  const bool on = H->pf_lead > 0 && H->mx.empty() && (int)H->pf_uploaded.size() > k && H->pf_uploaded[k];
   f.pf_k = on ? k : 0;
   H->pf_pos = on ? pos : -1;
   H->pf_done = 0;
@@ -708,7 +728,7 @@ void follow_stream(dory_handle* H, Fwd<T>& f, int k, int pos) {
 template <typename T>
 dory_status decode_body(dory_handle* H, int batch, const int32_t* tokens_in, int k, int mode, int max_ctx,
                         float* logits, int32_t* next_tokens, cudaStream_t st) {
-  const bool pf = H->pf_lead > 0 && (int)H->pf_uploaded.size() > k && H->pf_uploaded[k];
+  const bool pf = H->pf_lead > 0 && H->mx.empty() && (int)H->pf_uploaded.size() > k && H->pf_uploaded[k];
   H->pf_pos = pf ? 0 : -1;
   H->pf_done = 0;
   CK(launch_plan_uniform(batch, 1, 0, H->seq_ids, H->seq_len, H->meta, st));
@@ -1158,6 +1178,7 @@ dory_status dory_synchronize(dory_handle* h, dory_stream stream) {
     if (err[0] == DEV_ERR_TIMEOUT) return fail(DORY_ERR_TIMEOUT, "a device-side wait timed out");
     if (err[0] == DEV_ERR_BAD_TOKEN) return fail(DORY_ERR_INVALID_ARG, "a token id was outside [0, vocab)");
     if (err[0] == DEV_ERR_BAD_INDEX) return fail(DORY_ERR_CAPACITY, "a cache position was outside max_seq");
+    if (err[0] == DEV_ERR_RANGE) return fail(DORY_ERR_INVALID_ARG, "a value was outside a kernel's supported range");
     return fail(DORY_ERR_CUDA, "device error code %d", err[0]);
   }
   return DORY_OK;
@@ -1190,6 +1211,66 @@ dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value) {
       return DORY_OK;
   }
   return fail(DORY_ERR_INVALID_ARG, "unknown option %d", opt);
+}
+
+dory_status dory_quantize_mxfp8(const void* w, int32_t n, int32_t k, void* q, void* scales, void* w_deq,
+                                int32_t* err_word, dory_stream stream) {
+  if (!w || !q || !scales || n < 1 || k < 1) return fail(DORY_ERR_INVALID_ARG, "bad quantiser arguments");
+  if (k % kMxBlock) return fail(DORY_ERR_UNSUPPORTED, "K must be a multiple of %d", kMxBlock);
+  if (((uintptr_t)w & 15) || ((uintptr_t)q & 15) || ((uintptr_t)w_deq & 15))
+    return fail(DORY_ERR_INVALID_ARG, "w, q and w_deq must be 16-byte aligned");
+  CK(launch_mx_quantize((const bf16*)w, n, k, (uint8_t*)q, (uint8_t*)scales, (bf16*)w_deq, err_word,
+                        (cudaStream_t)stream));
+  return DORY_OK;
+}
+
+dory_status dory_gemv_mxfp8(int32_t m, int32_t n, int32_t k, const void* x, int32_t ldx, const void* q,
+                            const void* scales, float* y, int32_t ldy, int32_t* err_word, dory_stream stream) {
+  if (!x || !q || !scales || !y || m < 1 || n < 1 || k < 1 || ldx < k || ldy < n)
+    return fail(DORY_ERR_INVALID_ARG, "bad GEMV arguments");
+  if (k % kMxBlock || k > 40960) return fail(DORY_ERR_UNSUPPORTED, "K must be a multiple of 32 and at most 40960");
+  if ((uintptr_t)q & 15) return fail(DORY_ERR_INVALID_ARG, "q must be 16-byte aligned");
+  CK(launch_mx_gemv(m, n, k, (const bf16*)x, ldx, (const uint8_t*)q, (const uint8_t*)scales, y, ldy, err_word,
+                    (cudaStream_t)stream));
+  return DORY_OK;
+}
+
+dory_status dory_attach_mxfp8(dory_handle* h, const dory_mx_weights* mx) {
+  if (!h) return fail(DORY_ERR_INVALID_ARG, "NULL handle");
+  std::unordered_map<const void*, dory_handle::MxMat> map;
+  if (mx) {
+    const dory_config& c = h->c;
+    if (!h->bf16) return fail(DORY_ERR_UNSUPPORTED, "MXFP8 copies stand for bf16 weights only");
+    if (c.d_model % kMxBlock || h->q_dim % kMxBlock || c.d_ff % kMxBlock)
+      return fail(DORY_ERR_UNSUPPORTED, "d_model, n_heads * head_dim and d_ff must be multiples of %d", kMxBlock);
+    bool ok = true;
+    auto add = [&](const void* w, const void* const* qs, const void* const* ss, int l) {
+      const void* q = qs ? qs[l] : nullptr;
+      const void* sc = ss ? ss[l] : nullptr;
+      if (!q && !sc) return;  // this matrix stays bf16
+      if (!q || !sc || ((uintptr_t)q & 15)) ok = false;
+      map[w] = {(const uint8_t*)q, (const uint8_t*)sc};
+    };
+    for (int l = 0; l < h->L; ++l) {
+      if (layer_is_attn(l)) {
+        add(h->w_qkv[l], mx->qkv_q, mx->qkv_s, l);
+        add(h->w_o[l], mx->o_q, mx->o_s, l);
+      } else {
+        add(h->w_gu[l], mx->gu_q, mx->gu_s, l);
+        add(h->w_down[l], mx->down_q, mx->down_s, l);
+      }
+    }
+    const void* hq[1] = {mx->lm_head_q};
+    const void* hs[1] = {mx->lm_head_s};
+    add(h->head, hq, hs, 0);
+    if (!ok) return fail(DORY_ERR_INVALID_ARG, "each MXFP8 copy needs codes (16-byte aligned) and scales");
+  }
+  // graphs captured with the other weights are dropped
+  for (auto& g : h->graphs_cache)
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+  h->graphs_cache.clear();
+  h->mx.swap(map);
+  return DORY_OK;
 }
 
 dory_status dory_set_sampling(dory_handle* h, float temperature, float top_p, uint64_t seed) {

@@ -2,8 +2,9 @@
 tests/, the smoke check and the bench's CPU legs use this package).
 
 The pages list MXFP8 among the released weight formats and measure its batch-1
-decode speed against BF16 (trawling.dev, section on the KV cache and the
-runtime; lucasainews, the formats article), but do not define the format.  The
+decode speed against BF16 ("NVIDIA, 반복 연산형 4B 언어 모델 Dory 공개",
+section "KV 캐시와 실행 환경"; the lucasainews formats article, section
+"학습 방식과 변형"), but do not define the format.  The
 reading taken here is the OCP Microscaling Formats (MX) Specification v1.0
 with FP8 E4M3 elements:
 

@@ -126,6 +126,37 @@ def test_argument_validation():
     lib.dory_destroy(h)
 
 
+def test_mxfp8_argument_validation():
+    F, F8 = ctypes.c_void_p(FAKE_WS), ctypes.c_void_p(FAKE_WS + 8)
+    G = lambda *a: status_name(lib.dory_gemv_mxfp8(*a, None, None))
+    assert G(1, 8, 48, F, 48, F, F, F, 8) == "DORY_ERR_UNSUPPORTED"    # K % 32
+    assert G(1, 8, 40992, F, 40992, F, F, F, 8) == "DORY_ERR_UNSUPPORTED"  # staged activations too large
+    assert G(1, 8, 64, F, 32, F, F, F, 8) == "DORY_ERR_INVALID_ARG"    # ldx < K
+    assert G(1, 8, 64, F, 64, F, F, F, 4) == "DORY_ERR_INVALID_ARG"    # ldy < N
+    assert G(1, 8, 64, F, 64, F8, F, F, 8) == "DORY_ERR_INVALID_ARG"   # codes not 16-byte aligned
+    assert G(0, 8, 64, F, 64, F, F, F, 8) == "DORY_ERR_INVALID_ARG"    # no rows
+    Q = lambda *a: status_name(lib.dory_quantize_mxfp8(*a, None, None))
+    assert Q(F, 4, 40, F, F, None) == "DORY_ERR_UNSUPPORTED"           # K % 32
+    assert Q(F8, 4, 64, F, F, None) == "DORY_ERR_INVALID_ARG"          # weights not 16-byte aligned
+    assert Q(F, 4, 64, F, F, F8) == "DORY_ERR_INVALID_ARG"             # dequantised output not aligned
+    assert Q(F, 0, 64, F, F, None) == "DORY_ERR_INVALID_ARG"
+    A = lambda h, mx: status_name(lib.dory_attach_mxfp8(h, mx))
+    h32, _, keep32 = fake_handle(synth.TINY)
+    L = synth.TINY.n_layers
+    arr = (ctypes.c_void_p * L)(*([FAKE_WS] * L))
+    full = dory.MxWeightsC(FAKE_WS, FAKE_WS, *([arr] * 8))
+    assert A(h32, full) == "DORY_ERR_UNSUPPORTED"  # fp32 weights
+    assert A(h32, None) == "DORY_OK"
+    hb, _, keepb = fake_handle(synth.TINY_BF16)
+    assert A(hb, dory.MxWeightsC(FAKE_WS, None, *([arr] * 8))) == "DORY_ERR_INVALID_ARG"  # codes without scales
+    assert A(hb, dory.MxWeightsC(FAKE_WS + 8, FAKE_WS, *([arr] * 8))) == "DORY_ERR_INVALID_ARG"  # misaligned
+    assert A(hb, full) == "DORY_OK"
+    assert A(hb, dory.MxWeightsC(None, None, None, None, None, None, None, None, None, None)) == "DORY_OK"
+    assert A(hb, None) == "DORY_OK"
+    lib.dory_destroy(h32)
+    lib.dory_destroy(hb)
+
+
 def test_create_rejects_bad_workspace_and_config():
     cfg = cfg_for(synth.TINY)
     n = dory.workspace_size(cfg, dory.LAST_LOOP)
