@@ -387,25 +387,28 @@ def mxfp8_leg(dory, torch, shape, dw, args, mode, bf16_sweep, steps=32):
     tok = h.prefill([0], prompt, [args.prompt], args.k, mode)
     bufs = [torch.empty(1, dtype=torch.int32, device="cuda") for _ in range(2)]
     out = {}
-    for kk in (1, 2, 4):
-        if args.mode == "per_loop" and kk != args.k:
-            continue
-        for i in range(3):
-            tok = h.decode_step([0], tok, kk, mode, next_tokens=bufs[i % 2])
-        torch.cuda.synchronize()
-        a, b = ev(), ev()
-        a.record()
-        for i in range(steps):
-            tok = h.decode_step([0], tok, kk, mode, next_tokens=bufs[i % 2])
-        b.record()
-        torch.cuda.synchronize()
-        ms = a.elapsed_time(b) / steps
-        r = {"tokens_per_s": round(1e3 / ms, 2), "ms_per_token": round(ms, 4), "ctx": h.seq_len(0)}
-        ref = (bf16_sweep or {}).get(f"k{kk}")
-        if ref:
-            r["speedup_vs_bf16"] = round(r["tokens_per_s"] / ref["tokens_per_s"], 3)
-        out[f"k{kk}"] = r
-    # the GEMV's own time: CUDA events around every launch of two steps
+    # impl 2: the tensor-core GEMV, at the bench's k only; then the default (CUDA cores) at every k
+    for impl, ks in ((2, (args.k,)), (0, (1, 2, 4))):
+        h.set_option(dory.OPT_MX_GEMV, impl)
+        for kk in ks:
+            if args.mode == "per_loop" and kk != args.k:
+                continue
+            for i in range(3):
+                tok = h.decode_step([0], tok, kk, mode, next_tokens=bufs[i % 2])
+            torch.cuda.synchronize()
+            a, b = ev(), ev()
+            a.record()
+            for i in range(steps):
+                tok = h.decode_step([0], tok, kk, mode, next_tokens=bufs[i % 2])
+            b.record()
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / steps
+            r = {"tokens_per_s": round(1e3 / ms, 2), "ms_per_token": round(ms, 4), "ctx": h.seq_len(0)}
+            ref = (bf16_sweep or {}).get(f"k{kk}")
+            if ref:
+                r["speedup_vs_bf16"] = round(r["tokens_per_s"] / ref["tokens_per_s"], 3)
+            out[f"k{kk}" if impl == 0 else f"k{kk}_tensor_core_gemv"] = r
+    # the (default) GEMV's own time: CUDA events around every launch of two steps
     h.profile_reset()
     h.set_option(dory.OPT_PROFILE, 1)
     for i in range(2):
@@ -484,9 +487,11 @@ def main():
     ap.add_argument("--mode", default="last_loop", choices=["last_loop", "per_loop"])
     ap.add_argument("--no-aux", action="store_true", help="skip the k sweep, e2e and CPU baseline legs")
     ap.add_argument("--profile-steps", type=int, default=3)
-    ap.add_argument("--kernel", default=None, choices=["gemm"],
+    ap.add_argument("--kernel", default=None, choices=["gemm", "mxgemv"],
                     help="time one kernel alone instead of the decode step (prints its own JSON line)")
-    ap.add_argument("--shape", default="qkv,o,gate_up,down,lm_head", help="GEMM shapes for --kernel gemm")
+    ap.add_argument("--shape", default="qkv,o,gate_up,down,lm_head", help="GEMM shapes for --kernel gemm / mxgemv")
+    ap.add_argument("--mx-impl", dest="mx_impl", type=int, default=1,
+                    help="--kernel mxgemv: 1 CUDA cores (default), 2 tensor cores")
     ap.add_argument("--m", type=int, default=1, help="token rows for --kernel gemm")
     ap.add_argument("--l2-lookahead-mb", dest="l2_mb", type=int, default=None,
                     help="bytes of upcoming weights each decode GEMM prefetches into L2 (MiB; 0 = off; "
@@ -505,6 +510,9 @@ def main():
         return
     if args.kernel == "gemm":
         gemm_probe(args)
+        return
+    if args.kernel == "mxgemv":
+        mx_gemv_probe(args)
         return
     if args.warmup < 3:
         args.warmup = 3
@@ -865,6 +873,67 @@ def gemm_probe(args):
                      "frac_of_measured": round(by / us / 1e3 / hbm, 4)}
         del Ws
     print(json.dumps({"kernel": "gemm_tc", "impl": args.gemm_variant, "m": args.m, "results": out,
+                      "note": "graph-replayed back-to-back launches, weights cold in L2"}))
+
+
+def mx_gemv_probe(args):
+    """The MXFP8 decode GEMV (dory_gemv_mxfp8) on the 4B decode shapes at M
+    token rows, each timed alone like --kernel gemm: graph-replayed launches
+    rotating through weight copies (> 2x L2) of random E4M3 codes (NaN codes
+    excluded) and scale bytes 110..124.  --mx-impl 1: CUDA cores, 2: tensor
+    cores."""
+    import ctypes
+    import torch
+    import looped_ngpt_lm_b200 as dory
+    import synth
+    s = synth.DORY_4B
+    shapes = {"qkv": (s.q_dim + 2 * s.kv_dim, s.d_model), "o": (s.d_model, s.q_dim),
+              "gate_up": (2 * s.d_ff, s.d_model), "down": (s.d_model, s.d_ff), "lm_head": (s.vocab, s.d_model)}
+    hbm = peaks()[0]
+    out = {}
+    for name in args.shape.split(","):
+        N, K = shapes[name]
+        wbytes = N * K + N * K // 32
+        copies = max(2, -(-300_000_000 // wbytes))
+        g = torch.Generator(device="cuda").manual_seed(0)
+        qs, ss = [], []
+        for _ in range(copies):
+            q = torch.randint(0, 0x7E, (N, K), generator=g, dtype=torch.uint8, device="cuda")
+            q |= torch.randint(0, 2, (N, K), generator=g, dtype=torch.uint8, device="cuda") << 7
+            qs.append(q)
+            ss.append(torch.randint(110, 125, (N, K // 32), generator=g, dtype=torch.uint8, device="cuda"))
+        X = (torch.randn((args.m, K), generator=g, device="cuda") / K ** 0.5).to(torch.bfloat16)
+        Y = torch.empty((args.m, N), dtype=torch.float32, device="cuda")
+
+        def one(i, st):
+            dory._check(dory.lib.dory_gemv_mxfp8(args.m, N, K, ctypes.c_void_p(X.data_ptr()), K,
+                                                  ctypes.c_void_p(qs[i].data_ptr()), ctypes.c_void_p(ss[i].data_ptr()),
+                                                  ctypes.c_void_p(Y.data_ptr()), N, args.mx_impl, None,
+                                                  ctypes.c_void_p(st.cuda_stream)))
+
+        for i in range(3):
+            one(i % copies, torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        iters = max(30, 3 * copies)
+        side = torch.cuda.Stream()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            for i in range(iters):
+                one(i % copies, side)
+        graph.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        graph.replay()
+        b.record()
+        torch.cuda.synchronize()
+        us = 1e3 * a.elapsed_time(b) / iters
+        by = wbytes + args.m * K * 2 + args.m * N * 4
+        out[name] = {"N": N, "K": K, "us": round(us, 2), "GBs": round(by / us / 1e3, 1),
+                     "frac_of_measured": round(by / us / 1e3 / hbm, 4)}
+        del qs, ss, graph
+        torch.cuda.empty_cache()
+    print(json.dumps({"kernel": "mx_gemv", "mx_impl": args.mx_impl, "m": args.m, "results": out,
                       "note": "graph-replayed back-to-back launches, weights cold in L2"}))
 
 

@@ -289,15 +289,21 @@ dory_status dory_quantize_mxfp8(const void* w, int32_t N, int32_t K, void* q, vo
                                 int32_t* err_word, dory_stream stream);
 
 /* y[i, n] = sum_k x[i, k] * 2^(scales[n, k/32] - 127) * E4M3(q[n, k]) for
- * i < M, n < N, in fp32.  x is bf16 [M, ldx] (device) and y is fp32
+ * i < M, n < N, with fp32 sums.  x is bf16 [M, ldx] (device) and y is fp32
  * [M, ldy] (device).  Each y[i, n] is summed in an order fixed by K alone,
- * so its bits do not depend on M.  Requires K % 32 == 0, K <= 40960,
- * ldx >= K, ldy >= N and q 16-byte aligned.  The supported range is
- * |x| < 2^64 and scale bytes <= 198 (what the quantiser writes for
- * |w| < 2^80).  An activation outside it sets *err_word (device, nullable).
- * Queues work on `stream`. */
+ * so its bits do not depend on M.  Requires K % 32 == 0, ldx >= K,
+ * ldy >= N and q 16-byte aligned.
+ *   impl 2: tensor cores.  mma.sync with f16 operands and fp32 accumulators;
+ *     one block's 32 products per accumulation, then the block scale.
+ *     K <= 10240.  Any finite x; |x| below 2^-124 adds nothing.
+ *   impl 1: CUDA cores.  K <= 40960; supported range |x| < 2^64 and scale
+ *     bytes <= 198 (what the quantiser writes for |w| < 2^80).
+ *   impl 0: 1 (measured faster than 2 at every 4B decode shape).
+ * An activation outside the range (non-finite for 2) sets *err_word (device,
+ * nullable).  Queues work on `stream`. */
 dory_status dory_gemv_mxfp8(int32_t M, int32_t N, int32_t K, const void* x, int32_t ldx, const void* q,
-                            const void* scales, float* y, int32_t ldy, int32_t* err_word, dory_stream stream);
+                            const void* scales, float* y, int32_t ldy, int32_t impl, int32_t* err_word,
+                            dory_stream stream);
 
 /* MXFP8 copies of a handle's projection weights and LM head (device
  * pointers, BORROWED: they must outlive the attachment).  The per-layer
@@ -348,7 +354,10 @@ enum {
    * past its own once its loads have landed (default 8 MiB; 0 turns the
    * look-ahead off).  Changes only when HBM reads happen, never what is
    * computed. */
-  DORY_OPT_L2_LOOKAHEAD = 7
+  DORY_OPT_L2_LOOKAHEAD = 7,
+  /* GEMV on attached MXFP8 copies (see dory_gemv_mxfp8's impl): 0 (default, = 1), 1 CUDA cores,
+     2 tensor cores */
+  DORY_OPT_MX_GEMV = 8
 };
 dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value);
 

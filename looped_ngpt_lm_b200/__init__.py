@@ -28,6 +28,7 @@ OPT_PDL = 4
 OPT_PREFILL_TC = 5
 OPT_ATTN_CLUSTER = 6
 OPT_L2_LOOKAHEAD = 7
+OPT_MX_GEMV = 8
 
 STATUS = {0: "DORY_OK", 1: "DORY_ERR_INVALID_ARG", 2: "DORY_ERR_CAPACITY", 3: "DORY_ERR_STATE",
           4: "DORY_ERR_WORKSPACE", 5: "DORY_ERR_CUDA", 6: "DORY_ERR_TIMEOUT", 7: "DORY_ERR_UNSUPPORTED"}
@@ -99,7 +100,7 @@ def _load() -> ctypes.CDLL:
         "dory_set_sampling": [P, ctypes.c_float, ctypes.c_float, ctypes.c_uint64],
         "dory_sample": [P, I32, I32, P, P, ctypes.c_float, ctypes.c_float, ctypes.c_uint64, P, P, P],
         "dory_quantize_mxfp8": [P, I32, I32, P, P, P, P, P],
-        "dory_gemv_mxfp8": [I32, I32, I32, P, I32, P, P, P, I32, P, P],
+        "dory_gemv_mxfp8": [I32, I32, I32, P, I32, P, P, P, I32, I32, P, P],
         "dory_attach_mxfp8": [P, ctypes.POINTER(MxWeightsC)],
     }
     for name, args in sig.items():
@@ -250,8 +251,9 @@ def quantize_mxfp8(W, dequantised=True, err=None, stream=None):
     return q, sc, deq
 
 
-def gemv_mxfp8(X, q, scales, Y=None, err=None, stream=None):
-    """Y = X . dequantize(q, scales)^T through dory_gemv_mxfp8 (X bf16 [M, K])."""
+def gemv_mxfp8(X, q, scales, Y=None, impl=0, err=None, stream=None):
+    """Y = X . dequantize(q, scales)^T through dory_gemv_mxfp8 (X bf16 [M, K];
+    impl 0 default (= 1), 1 CUDA cores, 2 tensor cores)."""
     import torch
     M, K = X.shape
     N = q.shape[0]
@@ -259,7 +261,7 @@ def gemv_mxfp8(X, q, scales, Y=None, err=None, stream=None):
         Y = torch.empty((M, N), dtype=torch.float32, device=X.device)
     _check(lib.dory_gemv_mxfp8(M, N, K, ctypes.c_void_p(X.data_ptr()), X.stride(0), ctypes.c_void_p(q.data_ptr()),
                                ctypes.c_void_p(scales.data_ptr()), ctypes.c_void_p(Y.data_ptr()), Y.stride(0),
-                               ctypes.c_void_p(_ptr(err)), _stream(stream)))
+                               impl, ctypes.c_void_p(_ptr(err)), _stream(stream)))
     return Y
 
 

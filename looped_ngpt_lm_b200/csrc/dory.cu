@@ -111,6 +111,7 @@ struct dory_handle {
     const uint8_t* s;
   };
   std::unordered_map<const void*, MxMat> mx;
+  int mx_impl = 0;  // GEMV on the copies: 0 default (CUDA cores), 1 CUDA cores, 2 tensor cores
   std::vector<int> attn_of;
   std::vector<AttnLayer> attn;
 
@@ -378,7 +379,8 @@ dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, cons
       auto it = H->mx.find(W);
       if (it != H->mx.end()) {
         Scope sc(H, f.st, name, (double)N * K * (1.0 + 1.0 / kMxBlock) + (double)M * K * 2 + (double)M * N * 4);
-        CK(launch_mx_gemv(M, N, K, (const bf16*)X, ldx, it->second.q, it->second.s, Y, ldy, H->err, f.st));
+        CK(launch_mx_gemv(M, N, K, (const bf16*)X, ldx, it->second.q, it->second.s, Y, ldy, H->err, f.st,
+                          H->mx_impl));
         return DORY_OK;
       }
     }
@@ -1205,6 +1207,15 @@ dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value) {
       }
       h->pf_lead = (unsigned long long)value & ~127ull;
       return DORY_OK;
+    case DORY_OPT_MX_GEMV:
+      if (value < 0 || value > 2) return fail(DORY_ERR_INVALID_ARG, "bad MXFP8 GEMV impl");
+      if (value != h->mx_impl) {
+        for (auto& g : h->graphs_cache)
+          if (g.exec) cudaGraphExecDestroy(g.exec);
+        h->graphs_cache.clear();
+      }
+      h->mx_impl = (int)value;
+      return DORY_OK;
     case DORY_OPT_GEMM_IMPL:
       if (value < 0 || value > 2) return fail(DORY_ERR_INVALID_ARG, "bad GEMM impl");
       h->gemm_impl = (int)value;
@@ -1225,13 +1236,15 @@ dory_status dory_quantize_mxfp8(const void* w, int32_t n, int32_t k, void* q, vo
 }
 
 dory_status dory_gemv_mxfp8(int32_t m, int32_t n, int32_t k, const void* x, int32_t ldx, const void* q,
-                            const void* scales, float* y, int32_t ldy, int32_t* err_word, dory_stream stream) {
-  if (!x || !q || !scales || !y || m < 1 || n < 1 || k < 1 || ldx < k || ldy < n)
+                            const void* scales, float* y, int32_t ldy, int32_t impl, int32_t* err_word,
+                            dory_stream stream) {
+  if (!x || !q || !scales || !y || m < 1 || n < 1 || k < 1 || ldx < k || ldy < n || impl < 0 || impl > 2)
     return fail(DORY_ERR_INVALID_ARG, "bad GEMV arguments");
-  if (k % kMxBlock || k > 40960) return fail(DORY_ERR_UNSUPPORTED, "K must be a multiple of 32 and at most 40960");
+  if (k % kMxBlock || k > (impl == 2 ? 10240 : 40960))
+    return fail(DORY_ERR_UNSUPPORTED, "K must be a multiple of 32 and at most %d", impl == 2 ? 10240 : 40960);
   if ((uintptr_t)q & 15) return fail(DORY_ERR_INVALID_ARG, "q must be 16-byte aligned");
   CK(launch_mx_gemv(m, n, k, (const bf16*)x, ldx, (const uint8_t*)q, (const uint8_t*)scales, y, ldy, err_word,
-                    (cudaStream_t)stream));
+                    (cudaStream_t)stream, impl));
   return DORY_OK;
 }
 

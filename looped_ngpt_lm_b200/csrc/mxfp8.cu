@@ -16,6 +16,7 @@
 #include <map>
 
 #include "mxfp8.cuh"
+#include "warp_mma.cuh"
 
 namespace dory {
 
@@ -244,6 +245,186 @@ cudaError_t run_gemv(int M, int N, int K, const bf16* X, int ldx, const uint8_t*
   return launch(k_mx_gemv<MT>, grid, GV_T, smem, st, M, N, K, X, ldx, q, s, Y, ldy, err);
 }
 
+// ------------------------------------------------------------------ GEMV on the tensor cores
+// One CTA computes 16 weight rows x up to 8 tokens at a time with
+// mma.sync m16n8k16 (f16 operands, fp32 accumulators); its 8 warps split K
+// into 8 fixed ranges of 32-weight blocks and their partial sums are added
+// in warp order.  Each k16 step stays inside one block, so a block's partial
+// product leaves the tensor core in fp32 and takes the block scale with one
+// FMA.  The E4M3 codes become f16 in registers (exact: every E4M3 value is
+// an f16 value); the activations are staged as f16 after a per-token
+// power-of-two scaling 2^p that puts the token's largest |x| in [2^14, 2^15),
+// exact for bf16 inputs whose magnitude is within 2^28 of that maximum, and
+// the result is scaled back by 2^-p.
+//
+// k permutation: thread t of a quad (lane & 3) holds codes 8t..8t+7 of the
+// block for its two rows (one 8-byte load each).  The MMA's k slots 2t, 2t+1
+// and 2t+8, 2t+9 take codes (0, 1) and (2, 3) in the first k16 step and
+// (4, 5), (6, 7) in the second; the activation fragment of the same thread
+// reads x[8t .. 8t+7] of its token (one 16-byte shared-memory load), which
+// applies the same permutation to x.  The dot product is unchanged.
+constexpr int TV_T = 256;  // threads per CTA
+constexpr int TV_W = TV_T / 32;
+constexpr int TV_U = 8;    // blocks per warp in flight
+
+__device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t two) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xFFFFu), __NV_E4M3);
+  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
+// 2^(byte - 127), E8M0 (byte 0 is 2^-127, a float subnormal)
+__device__ __forceinline__ float e8m0(uint32_t b) {
+  return __uint_as_float(b == 0u ? 0x00400000u : b << 23);
+}
+
+__global__ void __launch_bounds__(TV_T) k_mx_gemv_tc(int M, int N, int K, const bf16* __restrict__ X, int ldx,
+                                                     const uint8_t* __restrict__ q, const uint8_t* __restrict__ s,
+                                                     float* __restrict__ Y, int ldy, int* err) {
+  extern __shared__ __align__(16) unsigned char tv_smem[];
+  __half* xs = reinterpret_cast<__half*>(tv_smem);  // [mc][K] f16, x * 2^p
+  __shared__ float red[TV_W][32][4];
+  __shared__ int s_p[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int nb = K >> 5, ntile = (N + 15) >> 4;
+  const int kb0 = warp * nb / TV_W, kb1 = (warp + 1) * nb / TV_W;  // this warp's blocks
+
+  // the first tile's weights do not depend on earlier kernels: ask L2 now
+  if (blockIdx.x < ntile) {
+    const int r = blockIdx.x * 16 + (threadIdx.x & 15);
+    if (r < N) {
+      const char* row = reinterpret_cast<const char*>(q) + (size_t)r * K;
+      for (int a = (threadIdx.x >> 4) * 128; a < K; a += 16 * 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(row + a));
+    }
+  }
+  pdl_wait();
+
+  for (int m0 = 0; m0 < M; m0 += 8) {
+    const int mc = M - m0 < 8 ? M - m0 : 8;
+    if (m0 > 0) __syncthreads();  // every warp is done with the previous tokens
+    // per-token exponent p from the largest |x| (bf16 bits), warp w: token w
+    if (warp < mc) {
+      const unsigned short* xr = reinterpret_cast<const unsigned short*>(X + (size_t)(m0 + warp) * ldx);
+      uint32_t mx = 0;
+      for (int k = lane; k < K; k += 32) {
+        const uint32_t v = xr[k] & 0x7FFFu;
+        mx = v > mx ? v : mx;
+      }
+      mx = __reduce_max_sync(0xffffffffu, mx);
+      if (lane == 0) {
+        if (mx >= 0x7F80u) set_error(err, DEV_ERR_RANGE);  // inf or NaN
+        // |x| < 2^128 needs p >= -113; below 2^-124 f16 keeps no bits of x * 2^100
+        int p = mx == 0 ? 0 : 14 - ((int)(mx >> 7) - 127);
+        s_p[warp] = p < -113 ? -113 : (p > 100 ? 100 : p);
+      }
+    }
+    __syncthreads();
+    // stage x * 2^p as f16 pairs
+    const int K2 = K >> 1;
+    for (int e = threadIdx.x; e < mc * K2; e += TV_T) {
+      const int m = e / K2, k2 = e - m * K2;
+      const float sc = __uint_as_float((uint32_t)(s_p[m] + 127) << 23);
+      const bf16* xr = X + (size_t)(m0 + m) * ldx + 2 * k2;
+      reinterpret_cast<__half2*>(xs)[e] = __floats2half2_rn(__bfloat162float(xr[0]) * sc,
+                                                            __bfloat162float(xr[1]) * sc);
+    }
+    __syncthreads();
+    if (m0 == 0) pdl_trigger();
+
+    const bool hasx = g < mc;
+    const __half* xg = xs + (size_t)(hasx ? g : 0) * K + 8 * t;
+    for (int rt = blockIdx.x; rt < ntile; rt += gridDim.x) {
+      const int r0 = rt * 16 + g, r1 = r0 + 8;
+      // rows past N read row 0 (in bounds) and are never written
+      const uint8_t* q0 = q + (size_t)(r0 < N ? r0 : 0) * K + 8 * t;
+      const uint8_t* q1 = q + (size_t)(r1 < N ? r1 : 0) * K + 8 * t;
+      const uint8_t* s0 = s + (size_t)(r0 < N ? r0 : 0) * nb;
+      const uint8_t* s1 = s + (size_t)(r1 < N ? r1 : 0) * nb;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int b0 = kb0; b0 < kb1; b0 += TV_U) {
+        uint2 w0[TV_U], w1[TV_U];
+        uint32_t sa[TV_U], sb[TV_U];
+#pragma unroll
+        for (int u = 0; u < TV_U; ++u) {
+          const int b = b0 + u;
+          if (b < kb1) {
+            w0[u] = __ldcs(reinterpret_cast<const uint2*>(q0 + (size_t)b * 32));
+            w1[u] = __ldcs(reinterpret_cast<const uint2*>(q1 + (size_t)b * 32));
+            sa[u] = s0[b];
+            sb[u] = s1[b];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < TV_U; ++u) {
+          const int b = b0 + u;
+          if (b < kb1) {
+            const uint4 xv = hasx ? *reinterpret_cast<const uint4*>(xg + (size_t)b * 32) : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t a0[4] = {e4m3x2_f16x2(w0[u].x), e4m3x2_f16x2(w1[u].x), e4m3x2_f16x2(w0[u].x >> 16),
+                                    e4m3x2_f16x2(w1[u].x >> 16)};
+            const uint32_t a1[4] = {e4m3x2_f16x2(w0[u].y), e4m3x2_f16x2(w1[u].y), e4m3x2_f16x2(w0[u].y >> 16),
+                                    e4m3x2_f16x2(w1[u].y >> 16)};
+            float blk[4] = {0.f, 0.f, 0.f, 0.f};
+            wm::mma_f16(blk, a0, xv.x, xv.y);
+            wm::mma_f16(blk, a1, xv.z, xv.w);
+            const float sc0 = e8m0(sa[u]), sc1 = e8m0(sb[u]);
+            acc[0] = __fmaf_rn(blk[0], sc0, acc[0]);
+            acc[1] = __fmaf_rn(blk[1], sc0, acc[1]);
+            acc[2] = __fmaf_rn(blk[2], sc1, acc[2]);
+            acc[3] = __fmaf_rn(blk[3], sc1, acc[3]);
+          }
+        }
+      }
+      // add the 8 warps' partial sums in warp order
+#pragma unroll
+      for (int j = 0; j < 4; ++j) red[warp][lane][j] = acc[j];
+      __syncthreads();
+      if (warp == 0) {
+        float v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          v[j] = red[0][lane][j];
+#pragma unroll
+          for (int w = 1; w < TV_W; ++w) v[j] = __fadd_rn(v[j], red[w][lane][j]);
+        }
+        // thread t holds tokens 2t, 2t+1 of rows r0 (v0, v1) and r1 (v2, v3)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int m = 2 * t + j;
+          if (m < mc) {
+            const float un = __uint_as_float((uint32_t)(127 - s_p[m]) << 23);
+            if (r0 < N) Y[(size_t)(m0 + m) * ldy + r0] = v[j] * un;
+            if (r1 < N) Y[(size_t)(m0 + m) * ldy + r1] = v[2 + j] * un;
+          }
+        }
+      }
+      __syncthreads();  // red is reused by the next tile
+    }
+  }
+}
+
+cudaError_t run_gemv_tc(int M, int N, int K, const bf16* X, int ldx, const uint8_t* q, const uint8_t* s, float* Y,
+                        int ldy, int* err, cudaStream_t st) {
+  const int mc = M < 8 ? M : 8;
+  const int smem = mc * K * 2;
+  static int attr_smem = 0;
+  static std::map<int, int> per_sm;
+  if (smem > attr_smem) {
+    cudaError_t e = cudaFuncSetAttribute(k_mx_gemv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr_smem = smem;
+  }
+  auto it = per_sm.find(smem);
+  if (it == per_sm.end()) {
+    int b = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, k_mx_gemv_tc, TV_T, smem);
+    if (e != cudaSuccess) return e;
+    it = per_sm.emplace(smem, b < 1 ? 1 : b).first;
+  }
+  const long long want = ((long long)N + 15) / 16;
+  const long long cap = (long long)num_sms() * it->second;
+  const int grid = (int)(want < cap ? want : cap);
+  return launch(k_mx_gemv_tc, grid, TV_T, smem, st, M, N, K, X, ldx, q, s, Y, ldy, err);
+}
+
 }  // namespace
 
 cudaError_t launch_mx_quantize(const bf16* W, int N, int K, uint8_t* q, uint8_t* s, bf16* deq, int* err,
@@ -258,8 +439,13 @@ cudaError_t launch_mx_quantize(const bf16* W, int N, int K, uint8_t* q, uint8_t*
 }
 
 cudaError_t launch_mx_gemv(int M, int N, int K, const bf16* X, int ldx, const uint8_t* q, const uint8_t* s,
-                           float* Y, int ldy, int* err, cudaStream_t st) {
+                           float* Y, int ldy, int* err, cudaStream_t st, int impl) {
   if (M <= 0 || N <= 0 || K <= 0 || K % kMxBlock || ((uintptr_t)q & 15)) return cudaErrorNotSupported;
+  // the tensor-core kernel only by request: measured slower at every 4B decode shape
+  if (impl == 2) {
+    if (K * 16 > GV_SMEM_CAP) return cudaErrorNotSupported;  // 8 staged f16 tokens
+    return run_gemv_tc(M, N, K, X, ldx, q, s, Y, ldy, err, st);
+  }
   // tokens per pass: the smallest power of two covering M, up to 8, within
   // the staged-activation budget
   int cap = GV_SMEM_CAP / (K * 4);

@@ -21,12 +21,16 @@ cudaError_t launch_mx_quantize(const bf16* W, int N, int K, uint8_t* q, uint8_t*
 
 // Y[m, n] = sum_k X[m, k] * 2^(s[n, k/32] - 127) * E4M3(q[n, k]) for
 // m < M, n < N: bf16 activations X (row stride ldx), fp32 result Y (row
-// stride ldy), fp32 arithmetic.  Each Y[m, n] is computed in an order fixed
-// by K alone, so its bits do not depend on M.  Supported range: |X| < 2^64
-// (else DEV_ERR_RANGE in *err) and scale bytes <= 198 (the quantiser's output
-// for |w| < 2^80).  K % 32 == 0 and q 16-byte aligned, else
-// cudaErrorNotSupported.
+// stride ldy), fp32 sums.  Each Y[m, n] is computed in an order fixed by K
+// alone, so its bits do not depend on M.  K % 32 == 0 and q 16-byte aligned,
+// else cudaErrorNotSupported.
+// impl 2: tensor cores (mma.sync, f16 operands, fp32 accumulators; K <= 10240;
+//   finite X, else DEV_ERR_RANGE in *err; |x| below 2^-124 contributes
+//   nothing).
+// impl 1: CUDA cores (|X| < 2^64, else DEV_ERR_RANGE; scale bytes <= 198,
+//   the quantiser's output for |w| < 2^80; K <= 40960).
+// impl 0: 1 (the faster of the two at every 4B decode shape).
 cudaError_t launch_mx_gemv(int M, int N, int K, const bf16* X, int ldx, const uint8_t* q, const uint8_t* s,
-                           float* Y, int ldy, int* err, cudaStream_t st);
+                           float* Y, int ldy, int* err, cudaStream_t st, int impl = 0);
 
 }  // namespace dory

@@ -128,9 +128,11 @@ def test_argument_validation():
 
 def test_mxfp8_argument_validation():
     F, F8 = ctypes.c_void_p(FAKE_WS), ctypes.c_void_p(FAKE_WS + 8)
-    G = lambda *a: status_name(lib.dory_gemv_mxfp8(*a, None, None))
+    G = lambda *a, impl=0: status_name(lib.dory_gemv_mxfp8(*a, impl, None, None))
     assert G(1, 8, 48, F, 48, F, F, F, 8) == "DORY_ERR_UNSUPPORTED"    # K % 32
     assert G(1, 8, 40992, F, 40992, F, F, F, 8) == "DORY_ERR_UNSUPPORTED"  # staged activations too large
+    assert G(1, 8, 10272, F, 10272, F, F, F, 8, impl=2) == "DORY_ERR_UNSUPPORTED"  # tensor cores: K <= 10240
+    assert G(1, 8, 64, F, 64, F, F, F, 8, impl=3) == "DORY_ERR_INVALID_ARG"
     assert G(1, 8, 64, F, 32, F, F, F, 8) == "DORY_ERR_INVALID_ARG"    # ldx < K
     assert G(1, 8, 64, F, 64, F, F, F, 4) == "DORY_ERR_INVALID_ARG"    # ldy < N
     assert G(1, 8, 64, F, 64, F8, F, F, 8) == "DORY_ERR_INVALID_ARG"   # codes not 16-byte aligned

@@ -3,7 +3,8 @@
 * Quantiser: integer work on exact power-of-two scalings.  Codes, scale bytes
   and the bf16 dequantisation must equal the oracle's bit for bit, edge
   blocks included.
-* GEMV: fp32 sums.  |y - y_ref| <= 2e-5 * sum_k |x_k w_k| per element,
+* GEMV, both implementations (CUDA cores; tensor cores with f16 operands and
+  fp32 accumulators): |y - y_ref| <= 2e-5 * sum_k |x_k w_k| per element,
   where y_ref is the oracle's float64 product.  A row's bits must not depend
   on how many rows share the call.
 * Decode with MXFP8 copies attached must follow the oracle's forward on the
@@ -93,8 +94,9 @@ GEMV_CASES = [(1, 37, 256), (2, 1000, 1056), (3, 384, 2560), (5, 2560, 2560), (1
               (13, 300, 10240), (8, 4096, 2560)]
 
 
+@pytest.mark.parametrize("impl", [1, 2])
 @pytest.mark.parametrize("M,N,K", GEMV_CASES)
-def test_gemv_matches_oracle(M, N, K):
+def test_gemv_matches_oracle(M, N, K, impl):
     rng = np.random.default_rng(M * 7 + N + K)
     w = rng.standard_normal((N, K)).astype(np.float32)
     w /= np.linalg.norm(w, axis=1, keepdims=True)
@@ -103,7 +105,7 @@ def test_gemv_matches_oracle(M, N, K):
     xb = synth.f32_to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32) / np.sqrt(K))
     q, s, _ = dory.quantize_mxfp8(bf16_cuda(wb), dequantised=False)
     X = bf16_cuda(xb)
-    y = dory.gemv_mxfp8(X, q, s)
+    y = dory.gemv_mxfp8(X, q, s, impl=impl)
     torch.cuda.synchronize()
     codes, scales = MX.quantize(synth.bf16_bits_to_f32(wb))
     x64 = synth.bf16_bits_to_f32(xb).astype(np.float64)
@@ -113,11 +115,12 @@ def test_gemv_matches_oracle(M, N, K):
     assert np.all(np.abs(got - ref) <= bound), float(np.max(np.abs(got - ref) / bound))
     # each row's bits do not depend on M
     for m in sorted({0, M // 2, M - 1}):
-        one = dory.gemv_mxfp8(X[m:m + 1].contiguous(), q, s)
+        one = dory.gemv_mxfp8(X[m:m + 1].contiguous(), q, s, impl=impl)
         assert torch.equal(one[0], y[m])
 
 
-def test_gemv_strided_operands_and_range_flag():
+@pytest.mark.parametrize("impl", [1, 2])
+def test_gemv_strided_operands_and_range_flag(impl):
     rng = np.random.default_rng(5)
     K, N = 512, 96
     w = synth.f32_to_bf16_bits(rng.standard_normal((N, K)).astype(np.float32) * 0.04)
@@ -125,16 +128,33 @@ def test_gemv_strided_operands_and_range_flag():
     xfull = bf16_cuda(synth.f32_to_bf16_bits(rng.standard_normal((3, K + 64)).astype(np.float32)))
     X = xfull[:, 32:32 + K]  # row stride K + 64
     Y = torch.full((3, N + 8), 7.0, device="cuda")
-    dory.gemv_mxfp8(X, q, s, Y=Y[:, :N])
-    ref = dory.gemv_mxfp8(X.contiguous(), q, s)
+    dory.gemv_mxfp8(X, q, s, Y=Y[:, :N], impl=impl)
+    ref = dory.gemv_mxfp8(X.contiguous(), q, s, impl=impl)
     torch.cuda.synchronize()
     assert torch.equal(Y[:, :N], ref) and bool((Y[:, N:] == 7.0).all())
     err = torch.zeros(4, dtype=torch.int32, device="cuda")
     big = X.contiguous().clone()
-    big[1, 3] = 2.0 ** 70
-    dory.gemv_mxfp8(big, q, s, err=err)
+    big[1, 3] = 2.0 ** 70 if impl == 1 else float("inf")  # outside each kernel's range
+    dory.gemv_mxfp8(big, q, s, impl=impl, err=err)
     torch.cuda.synchronize()
     assert int(err[0]) == 4
+
+
+def test_tensor_core_gemv_scales_each_token():
+    # tokens of very different magnitudes in one call: each is staged with its own power of two
+    rng = np.random.default_rng(6)
+    K, N = 1024, 160
+    w = synth.f32_to_bf16_bits(rng.standard_normal((N, K)).astype(np.float32) * 0.03)
+    q, s, _ = dory.quantize_mxfp8(bf16_cuda(w), dequantised=False)
+    x = rng.standard_normal((4, K)).astype(np.float32)
+    x *= np.array([1e-20, 1.0, 3e10, 2.0 ** -60], np.float32)[:, None]
+    xb = synth.f32_to_bf16_bits(x)
+    y = dory.gemv_mxfp8(bf16_cuda(xb), q, s, impl=2).cpu().numpy()
+    codes, scales = MX.quantize(synth.bf16_bits_to_f32(w))
+    x64 = synth.bf16_bits_to_f32(xb).astype(np.float64)
+    ref = MX.gemv(x64, codes, scales)
+    bound = 2e-5 * (np.abs(x64) @ np.abs(MX.dequantize(codes, scales)).T)
+    assert np.all(np.abs(y - ref) <= bound)
 
 
 def mx_handle(shape, seed=0, alloc="per_loop"):
@@ -153,11 +173,13 @@ def mx_model(request):
     return shape, O.Model(shape, MX.quantized_weights(w)), h, mx
 
 
+@pytest.mark.parametrize("impl", [2, 1])
 @pytest.mark.parametrize("k", [1, 2, 4])
 @pytest.mark.parametrize("mode", ["last_loop", "per_loop"])
-def test_decode_with_mxfp8_matches_oracle(mx_model, k, mode):
+def test_decode_with_mxfp8_matches_oracle(mx_model, k, mode, impl):
     shape, model, h, _ = mx_model
     prompt = synth.make_prompt(3, 40, shape.vocab)
+    h.set_option(dory.OPT_MX_GEMV, impl)
     h.reset()
     om, cm = MODES[mode]
     toks, lg = gpu_generate(h, prompt, 13, k, cm)
@@ -166,6 +188,7 @@ def test_decode_with_mxfp8_matches_oracle(mx_model, k, mode):
     assert max(errs) <= 2e-2, errs
     tol = 4 * max(float(np.abs(lg[i] - ora[i]).max()) for i in range(len(toks)))
     check_tokens(toks, ora, tol)
+    h.set_option(dory.OPT_MX_GEMV, 0)
 
 
 def test_decode_reads_the_mxfp8_copies(mx_model):
@@ -183,8 +206,10 @@ def test_decode_reads_the_mxfp8_copies(mx_model):
     assert per_launch < 1.2 * n * kk  # 1 + 1/32 bytes per weight, not bf16's 2
 
 
-def test_graph_replay_and_speculative_decoding_with_mxfp8(mx_model):
+@pytest.mark.parametrize("impl", [2, 1])
+def test_graph_replay_and_speculative_decoding_with_mxfp8(mx_model, impl):
     shape, _, h, _ = mx_model
+    h.set_option(dory.OPT_MX_GEMV, impl)
     prompt = synth.make_prompt(5, 30, shape.vocab)
     tok = torch.tensor(prompt, dtype=torch.int32, device="cuda")
 
@@ -206,6 +231,7 @@ def test_graph_replay_and_speculative_decoding_with_mxfp8(mx_model):
     spec = [int(first[0])] + out[0].cpu().tolist()
     assert spec == ref  # per-loop speculative decoding is token-identical to plain k=4
     h.set_option(dory.OPT_CUDA_GRAPHS, 1)
+    h.set_option(dory.OPT_MX_GEMV, 0)
 
 
 def test_attach_validation():
