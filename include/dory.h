@@ -40,6 +40,12 @@
  *   - The library never allocates device memory: all device state lives in
  *     the caller-provided workspace.
  *   - A handle is not thread-safe; use one host thread per handle.
+ *   - Every entry point caches, per process, the kernel attributes,
+ *     occupancy figures and tensor maps of the launches it has made.  This
+ *     includes the functions without a handle (dory_gemm_bf16,
+ *     dory_gemm_bf16_noalloc, dory_pack_weight_bf16, dory_quantize_mxfp8,
+ *     dory_gemv_mxfp8, dory_sample).  Call the library from one host thread
+ *     at a time.
  */
 #ifndef DORY_H
 #define DORY_H
