@@ -1,0 +1,67 @@
+"""The Python binding's ctypes structures against the C header (CPU): a small
+C program compiled with the system compiler against include/dory.h prints
+sizeof and offsetof of every struct the ABI passes by pointer, the enum
+values the binding copies, and the option numbers; the binding must agree."""
+import ctypes
+import os
+import shutil
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+dory = pytest.importorskip("looped_ngpt_lm_b200")
+
+STRUCTS = {
+    "dory_config": (dory.Config, [f[0] for f in dory.Config._fields_]),
+    "dory_weights": (dory.Weights, [f[0] for f in dory.Weights._fields_]),
+    "dory_spec_stats": (dory.SpecStats, [f[0] for f in dory.SpecStats._fields_]),
+    "dory_mx_weights": (dory.MxWeightsC, [f[0] for f in dory.MxWeightsC._fields_]),
+}
+CONSTANTS = {
+    "DORY_LAST_LOOP": dory.LAST_LOOP, "DORY_PER_LOOP": dory.PER_LOOP, "DORY_F32": dory.F32,
+    "DORY_BF16": dory.BF16, "DORY_OPT_CUDA_GRAPHS": dory.OPT_CUDA_GRAPHS, "DORY_OPT_PROFILE": dory.OPT_PROFILE,
+    "DORY_OPT_GEMM_IMPL": dory.OPT_GEMM_IMPL, "DORY_OPT_PDL": dory.OPT_PDL, "DORY_OPT_PREFILL_TC": dory.OPT_PREFILL_TC,
+    "DORY_OPT_ATTN_CLUSTER": dory.OPT_ATTN_CLUSTER, "DORY_OPT_L2_LOOKAHEAD": dory.OPT_L2_LOOKAHEAD,
+    "DORY_OPT_MX_GEMV": dory.OPT_MX_GEMV,
+}
+
+
+@pytest.fixture(scope="module")
+def c_layout(tmp_path_factory):
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if not cc:
+        pytest.skip("no C compiler")
+    d = tmp_path_factory.mktemp("abi")
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "dory.h"', "int main(void) {"]
+    for name, (_, fields) in STRUCTS.items():
+        lines.append(f'  printf("{name} size %zu\\n", sizeof({name}));')
+        for f in fields:
+            lines.append(f'  printf("{name}.{f} %zu\\n", offsetof({name}, {f}));')
+    for k in CONSTANTS:
+        lines.append(f'  printf("{k} %d\\n", (int){k});')
+    for code, name in dory.STATUS.items():
+        lines.append(f'  printf("{name} %d\\n", (int){name});')
+    lines += ["  return 0;", "}"]
+    src = d / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = d / "layout"
+    subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src), "-o",
+                    str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout
+    return dict(line.rsplit(" ", 1) for line in out.strip().splitlines())
+
+
+@pytest.mark.parametrize("name", list(STRUCTS))
+def test_struct_layouts_match_the_header(c_layout, name):
+    cls, fields = STRUCTS[name]
+    assert int(c_layout[f"{name} size"]) == ctypes.sizeof(cls)
+    for f in fields:
+        assert int(c_layout[f"{name}.{f}"]) == getattr(cls, f).offset, f
+
+
+def test_constants_match_the_header(c_layout):
+    for k, v in CONSTANTS.items():
+        assert int(c_layout[k]) == v, k
+    for code, name in dory.STATUS.items():
+        assert int(c_layout[name]) == code, name
