@@ -65,3 +65,60 @@ def test_constants_match_the_header(c_layout):
         assert int(c_layout[k]) == v, k
     for code, name in dory.STATUS.items():
         assert int(c_layout[name]) == code, name
+
+
+def header_prototypes():
+    """name -> list of parameter declarations, from include/dory.h (comments removed;
+    balanced parentheses, so function-pointer-like parameters such as char (*names)[48] parse)."""
+    import re
+    text = open(os.path.join(ROOT, "include", "dory.h")).read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(?:dory_status|const char\*)\s+(dory_\w+)\s*\(", text):
+        i, depth = m.end(), 1
+        j = i
+        while depth:
+            depth += {"(": 1, ")": -1}.get(text[j], 0)
+            j += 1
+        body = text[i:j - 1]
+        params, depth, cur = [], 0, ""
+        for ch in body:
+            if ch == "," and depth == 0:
+                params.append(cur.strip())
+                cur = ""
+                continue
+            depth += {"(": 1, ")": -1, "[": 1, "]": -1}.get(ch, 0)
+            cur += ch
+        if cur.strip() and cur.strip() != "void":
+            params.append(cur.strip())
+        out[m.group(1)] = params
+    return out
+
+
+def c_class(decl: str) -> str:
+    d = " ".join(decl.split())
+    if "*" in d or d.startswith("dory_stream") or "[" in d:
+        return "ptr"
+    for t, c in (("int64_t", "i64"), ("uint64_t", "u64"), ("int32_t", "i32"), ("size_t", "u64"),
+                 ("float", "f32"), ("dory_cache_mode", "i32"), ("dory_dtype", "i32")):
+        if d.startswith(t + " ") or d.startswith("const " + t + " "):
+            return c
+    raise AssertionError(f"unclassified parameter {decl!r}")
+
+
+def py_class(t) -> str:
+    if t in (ctypes.c_void_p,) or isinstance(t, type) and issubclass(t, ctypes._Pointer):
+        return "ptr"
+    # size_t and uint64_t are both 64-bit unsigned here (ctypes makes them one type)
+    return {ctypes.c_int32: "i32", ctypes.c_int64: "i64", ctypes.c_uint64: "u64", ctypes.c_size_t: "u64",
+            ctypes.c_float: "f32"}[t]
+
+
+def test_argtypes_match_the_prototypes():
+    protos = header_prototypes()
+    assert sorted(protos) == sorted(dory.SYMBOLS)
+    for name, params in protos.items():
+        f = getattr(dory.lib, name)
+        want = [c_class(p) for p in params]
+        got = [py_class(t) for t in (f.argtypes or [])]
+        assert got == want, (name, got, want)
