@@ -1,15 +1,19 @@
 // MXFP8 weights (OCP Microscaling Formats v1.0: FP8 E4M3 elements, one E8M0
-// scale per 32 consecutive weights of a row): the quantiser, and the decode
-// GEMV that reads them.
+// scale per 32 consecutive weights of a row): the quantiser, and two decode
+// GEMVs that read them.
 //
 // The pages list MXFP8 among the released weight formats.  They measure it
 // against BF16 at batch 1, where decoding is bound by weight bytes
 // ("NVIDIA, 반복 연산형 4B 언어 모델 Dory 공개", section "KV 캐시와 실행 환경";
 // lucasainews formats article, section "학습 방식과 변형").  A decode step at
-// small batch is a matrix-vector product per weight matrix, bound by HBM, so
-// the GEMV runs on the CUDA cores.  Each warp streams one weight row at a
-// time in 16-byte chunks.  The activations, pre-scaled, are staged once per
-// CTA in shared memory.
+// small batch is a matrix-vector product per weight matrix, bound by HBM.
+//
+// k_mx_gemv (the default) runs on the CUDA cores.  Each warp streams one
+// weight row at a time in 16-byte chunks, against activations staged once
+// per CTA in shared memory.  k_mx_gemv_tc puts the products on the tensor
+// cores (mma.sync).  Measured on the 4B decode shapes, both are
+// latency-bound: each warp keeps its own loads in registers.  The
+// CUDA-core kernel is the faster of the two.
 #include <cuda_fp8.h>
 #include <float.h>
 
