@@ -67,6 +67,16 @@ def nucleus_threshold(q: np.ndarray, top_p: float) -> int:
     return int(desc[min(idx, len(desc) - 1)])
 
 
+def draw(seed: int, seq: int, pos: int, M: int) -> int:
+    """r = floor(u * M) for the draw u = (word >> 8) / 2^24 of (seq, pos)."""
+    return ((uniform_word(seed, seq, pos) >> 8) * int(M)) >> 24
+
+
+def choose(mass, r: int) -> int:
+    """The first index at which the running sum of `mass` exceeds r."""
+    return int(np.searchsorted(np.cumsum(mass), r, side="right"))
+
+
 def sample(logits, temperature: float, top_p: float, seed: int, seq: int, pos: int) -> int:
     """The token drawn for sequence `seq` at position `pos`.  Temperature and
     top_p are float32 parameters (rounded to float32 first)."""
@@ -74,6 +84,4 @@ def sample(logits, temperature: float, top_p: float, seed: int, seq: int, pos: i
     q = masses(logits, temperature)
     tau = nucleus_threshold(q, top_p)
     mass = np.where(q >= tau, q, 0)
-    M = int(mass.sum())
-    r = ((uniform_word(seed, seq, pos) >> 8) * M) >> 24
-    return int(np.searchsorted(np.cumsum(mass), r, side="right"))
+    return choose(mass, draw(seed, seq, pos, int(mass.sum())))

@@ -73,3 +73,39 @@ def test_draws_depend_only_on_seed_sequence_and_position():
     b = [S.sample(l, 1.0, 0.95, seed=7, seq=2, pos=i) for i in range(50)]
     c = [S.sample(l, 1.0, 0.95, seed=8, seq=2, pos=i) for i in range(50)]
     assert a == b and a != c
+
+
+@pytest.mark.parametrize("T", [0.5, 2.0])
+def test_temperature_frequencies_follow_softmax_of_scaled_logits(T):
+    l = np.array([0.0, 1.0, -0.5, 2.0, 0.3], np.float32)
+    p = np.exp(l / T - (l / T).max())
+    p /= p.sum()
+    n = 20000
+    counts = np.bincount([S.sample(l, T, 1.0, seed=21, seq=3, pos=i) for i in range(n)], minlength=len(l))
+    sd = np.sqrt(n * p * (1 - p))
+    assert np.all(np.abs(counts - n * p) <= 5 * sd + 1), (counts, n * p)
+
+
+def test_masses_closed_forms():
+    # the largest logit has mass 2^31; one T * ln 2 below it, exactly half (exp2(-1) = 0.5)
+    for T in (1.0, 0.5, 2.0):
+        l = np.array([3.0, 3.0 - T * math.log(2.0), -50.0], np.float32)
+        q = S.masses(l, T)
+        assert q[0] == 2 ** 31 and abs(int(q[1]) - 2 ** 30) <= 2 ** 31 * 2e-7 and q[2] >= 0
+
+
+def test_nucleus_mass_is_rounded_up():
+    # top_p * Q = 0.55 * 19 = 10.45: the nucleus must reach 10.45, so {10} (mass 10) is not enough
+    assert S.nucleus_threshold(np.array([10, 4, 4, 1], np.int64), 0.55) == 4
+
+
+def test_choice_rule_at_boundaries():
+    mass = np.array([5, 0, 3], np.int64)  # running sums 5, 5, 8
+    assert [S.choose(mass, r) for r in range(8)] == [0, 0, 0, 0, 0, 2, 2, 2]
+
+
+def test_worked_draw_from_the_philox_known_answer():
+    # seed 0, sequence 0, position 0: counter and key all zero, first output word 0x6627E8D5
+    # (the published known answer), so u = 0x6627E8 / 2^24 and r = floor(u * M)
+    assert S.draw(0, 0, 0, 2 ** 24) == 0x6627E8
+    assert S.draw(0, 0, 0, 1000) == (0x6627E8 * 1000) >> 24  # 399
