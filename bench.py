@@ -437,6 +437,15 @@ def mxfp8_leg(dory, torch, shape, dw, args, mode, bf16_sweep, steps=32):
     return out
 
 
+def leg(fn, *a):
+    """One auxiliary measurement.  An exception is recorded in the JSON line
+    (as {"error": ...}) instead of costing the headline."""
+    try:
+        return fn(*a)
+    except Exception as e:  # noqa: BLE001 - any failure of an extra leg is reported, not raised
+        return {"error": f"{type(e).__name__}: {e}"[:400]}
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -654,8 +663,12 @@ def main():
                                "hbm_frac_of_measured": round(by / (ms / 1e3) / 1e9 / hbm, 4),
                                "bytes_per_token": by, "ctx": ctx}
         aux["decode_k_sweep_last_loop" if args.mode == "last_loop" else "decode_k_sweep"] = sweep
-        aux["sampling"], tok = sampling_leg(dory, torch, h, tok, args, mode)
-        aux["mxfp8_decode"] = mxfp8_leg(dory, torch, shape, dw, args, mode, sweep)
+        r = leg(sampling_leg, dory, torch, h, tok, args, mode)
+        if isinstance(r, tuple):
+            aux["sampling"], tok = r
+        else:
+            aux["sampling"] = r
+        aux["mxfp8_decode"] = leg(mxfp8_leg, dory, torch, shape, dw, args, mode, sweep)
         # ---- end to end: every step copies its input token from pinned host
         # memory and reads the chosen token back, through the public API
         pin_in = torch.empty(1, dtype=torch.int32).pin_memory()
@@ -690,9 +703,9 @@ def main():
                        "sample": f"skipped: {host_mem_gb():.0f} GB host memory available, the fp32 oracle needs ~40"}
 
     if not args.no_aux and world == 1:
-        aux["k_mode_sweep"] = sweep_modes(dory, torch, shape, dw, args)
-        aux["spec_decode"] = spec_leg(dory, torch, shape, dw, args)
-        aux["mixed_k_decode"] = mixed_leg(dory, torch, shape, dw, args)
+        aux["k_mode_sweep"] = leg(sweep_modes, dory, torch, shape, dw, args)
+        aux["spec_decode"] = leg(spec_leg, dory, torch, shape, dw, args)
+        aux["mixed_k_decode"] = leg(mixed_leg, dory, torch, shape, dw, args)
 
     if rank == 0:
         line = {

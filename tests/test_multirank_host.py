@@ -46,3 +46,9 @@ def test_reference_arm_runs_on_rank_zero_only():
                        timeout=120)
     assert p.returncode == 0, p.stderr
     assert p.stdout.strip() == ""
+
+
+def test_a_failing_extra_leg_is_reported_not_raised():
+    import bench
+    assert bench.leg(lambda: 1 / 0) == {"error": "ZeroDivisionError: division by zero"}
+    assert bench.leg(lambda a, b: (a, b), 1, 2) == (1, 2)
