@@ -304,6 +304,11 @@ dory_status dory_quantize_mxfp8(const void* w, int32_t N, int32_t K, void* q, vo
  *     K <= 10240.  Any finite x; |x| below 2^-124 adds nothing.
  *   impl 1: CUDA cores.  K <= 40960; supported range |x| < 2^64 and scale
  *     bytes <= 198 (what the quantiser writes for |w| < 2^80).
+ *   impl 3: tcgen05 GEMM fed by TMA.  Converter warps expand the codes to
+ *     f16 in shared memory; each 32-weight block accumulates in its own TMEM
+ *     columns and takes its scale in the epilogue.  Requires M <= 16,
+ *     N % 128 == 0, K % 128 == 0, x 16-byte aligned, ldx % 8 == 0, scales
+ *     4-byte aligned (else DORY_ERR_UNSUPPORTED); |x| < 4.
  *   impl 0: 1 (measured faster than 2 at every 4B decode shape).
  * An activation outside the range (non-finite for 2) sets *err_word (device,
  * nullable).  Queues work on `stream`. */
@@ -361,8 +366,9 @@ enum {
    * look-ahead off).  Changes only when HBM reads happen, never what is
    * computed. */
   DORY_OPT_L2_LOOKAHEAD = 7,
-  /* GEMV on attached MXFP8 copies (see dory_gemv_mxfp8's impl): 0 (default, = 1), 1 CUDA cores,
-     2 tensor cores */
+  /* GEMM on attached MXFP8 copies (see dory_gemv_mxfp8's impl): 0 (default, = 1), 1 CUDA cores,
+     2 mma.sync, 3 TMA-fed tcgen05 with split-K slices (passes of at most 16 rows; larger passes
+     use 1, so row-count invariance then needs every pass to fit) */
   DORY_OPT_MX_GEMV = 8
 };
 dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value);

@@ -379,8 +379,21 @@ dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, cons
       auto it = H->mx.find(W);
       if (it != H->mx.end()) {
         Scope sc(H, f.st, name, (double)N * K * (1.0 + 1.0 / kMxBlock) + (double)M * K * 2 + (double)M * N * 4);
+        if (H->mx_impl == 3) {
+          // TMA-fed tensor-core GEMM with split-K slices; shapes it does not take use the CUDA-core GEMV
+          const int S = mx_gemm_splits(N, K);
+          const size_t ps = part_rows * (size_t)ldy;
+          cudaError_t e = launch_mx_gemm_tc(M, N, K, (const bf16*)X, ldx, it->second.q, it->second.s, Y, ldy, ps, S,
+                                            H->err, f.st);
+          if (e == cudaSuccess) {
+            *S_out = S;
+            *ps_out = ps;
+            return DORY_OK;
+          }
+          if (e != cudaErrorNotSupported) return fail(DORY_ERR_CUDA, "%s: %s", name, cudaGetErrorString(e));
+        }
         CK(launch_mx_gemv(M, N, K, (const bf16*)X, ldx, it->second.q, it->second.s, Y, ldy, H->err, f.st,
-                          H->mx_impl));
+                          H->mx_impl == 3 ? 1 : H->mx_impl));
         return DORY_OK;
       }
     }
@@ -1208,7 +1221,7 @@ dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value) {
       h->pf_lead = (unsigned long long)value & ~127ull;
       return DORY_OK;
     case DORY_OPT_MX_GEMV:
-      if (value < 0 || value > 2) return fail(DORY_ERR_INVALID_ARG, "bad MXFP8 GEMV impl");
+      if (value < 0 || value > 3) return fail(DORY_ERR_INVALID_ARG, "bad MXFP8 GEMV impl");
       if (value != h->mx_impl) {
         for (auto& g : h->graphs_cache)
           if (g.exec) cudaGraphExecDestroy(g.exec);
@@ -1238,8 +1251,10 @@ dory_status dory_quantize_mxfp8(const void* w, int32_t n, int32_t k, void* q, vo
 dory_status dory_gemv_mxfp8(int32_t m, int32_t n, int32_t k, const void* x, int32_t ldx, const void* q,
                             const void* scales, float* y, int32_t ldy, int32_t impl, int32_t* err_word,
                             dory_stream stream) {
-  if (!x || !q || !scales || !y || m < 1 || n < 1 || k < 1 || ldx < k || ldy < n || impl < 0 || impl > 2)
+  if (!x || !q || !scales || !y || m < 1 || n < 1 || k < 1 || ldx < k || ldy < n || impl < 0 || impl > 3)
     return fail(DORY_ERR_INVALID_ARG, "bad GEMV arguments");
+  if (impl == 3 && (m > 16 || n % 128 || k % 128 || ((uintptr_t)x & 15) || ldx % 8 || ((uintptr_t)scales & 3)))
+    return fail(DORY_ERR_UNSUPPORTED, "impl 3 needs M <= 16, N %% 128 == 0, K %% 128 == 0, aligned x and scales");
   if (k % kMxBlock || k > (impl == 2 ? 10240 : 40960))
     return fail(DORY_ERR_UNSUPPORTED, "K must be a multiple of 32 and at most %d", impl == 2 ? 10240 : 40960);
   if ((uintptr_t)q & 15) return fail(DORY_ERR_INVALID_ARG, "q must be 16-byte aligned");

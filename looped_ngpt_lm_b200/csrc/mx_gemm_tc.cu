@@ -1,0 +1,424 @@
+// MXFP8 decode GEMM on the tensor cores, fed by TMA (tcgen05, sm_100a).
+//
+// The 8-bit codes stream through a deep ring of raw 128-row x 128-code tiles
+// (TMA, no swizzle), as the bf16 decode GEMM streams its weights.  Four
+// converter warps turn each tile into the 128-byte-swizzled K-major f16
+// image the MMA reads (E4M3 -> f16 is exact), and turn the bf16 activations
+// into f16(x * 2^14) (exact for |x| < 4, else DEV_ERR_RANGE).  tcgen05.mma
+// kind::f16 then accumulates each 32-weight block into its own TMEM columns,
+// and four epilogue warps apply the block scale 2^(s - 127 - 14) with one FMA
+// and keep the sums in registers.  Warps: 0 TMA producer, 1 MMA issuer, 2-5
+// epilogue, 6-9 converters.  Every wait is bounded; on a timeout the kernel
+// sets DEV_ERR_TIMEOUT, drains its copies, frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+#include "mxfp8.cuh"
+#include "umma.cuh"
+
+namespace dory {
+namespace {
+
+using namespace tc;
+
+constexpr int BM = 128;         // weight rows per tile
+constexpr int MT = 16;          // tokens (MMA N)
+constexpr int CK = 128;         // K per chunk (4 scale blocks)
+constexpr int RAW_A = BM * CK;  // 16 KB of codes
+constexpr int RAW_B = MT * CK * 2;  // 4 KB of bf16 activations (2 SW128 boxes of 64 columns)
+constexpr int RAW_STAGE = RAW_A + RAW_B;
+constexpr int CONV_A = BM * CK * 2;  // 32 KB f16 (2 SW128 sub-tiles of 64 columns)
+constexpr int CONV_B = MT * CK * 2;  // 4 KB f16
+constexpr int CONV_STAGE = CONV_A + CONV_B;
+constexpr int RS = 7, CS = 2, TS = 4;  // raw, converted and TMEM-slot ring depths
+constexpr int TMEM_COLS = TS * 64;     // 4 blocks x 16 tokens per slot
+constexpr int NTH = 320;               // 0 producer, 1 MMA, 2-5 epilogue, 6-9 converters
+constexpr int SMEM = RS * RAW_STAGE + CS * CONV_STAGE + 1024 + 512;
+static_assert(SMEM <= 232448, "shared memory");
+constexpr float kXScale = 16384.f;  // activations are staged as f16(x * 2^14)
+
+__host__ __device__ constexpr uint32_t idesc_f16(int m, int n) {
+  // fp32 accumulator, A and B f16 (format 0), both K-major
+  return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t two) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xFFFFu), __NV_E4M3);
+  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
+// units: (n tile, split) with the split's chunk range fixed by (n chunks, S)
+struct Units {
+  int n_tiles, S, nch;
+  __device__ __forceinline__ void decode(int u, int& nt, int& s, int& c0, int& c1) const {
+    nt = u / S;
+    s = u - nt * S;
+    c0 = s * nch / S;
+    c1 = (s + 1) * nch / S;
+  }
+};
+
+__global__ void __launch_bounds__(NTH, 1)
+    k_mx_gemm(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapX,
+              const uint8_t* __restrict__ scales, int K, float* Y, int ldy, size_t part_stride, int M, Units un,
+              int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* raw = smem;                          // [RS][RAW_STAGE]
+  uint8_t* conv = smem + RS * RAW_STAGE;        // [CS][CONV_STAGE]
+  uint64_t* bars = (uint64_t*)(conv + CS * CONV_STAGE);
+  uint64_t* raw_full = bars;
+  uint64_t* raw_empty = raw_full + RS;
+  uint64_t* conv_full = raw_empty + RS;
+  uint64_t* conv_empty = conv_full + CS;
+  uint64_t* tfull = conv_empty + CS;
+  uint64_t* tempty = tfull + TS;
+  uint64_t* mma_done = tempty + TS;
+  uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nsb = K >> 5;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < RS; ++i) {
+      mbar_init(&raw_full[i], 1);
+      mbar_init(&raw_empty[i], 4);
+    }
+    for (int i = 0; i < CS; ++i) {
+      mbar_init(&conv_full[i], 4);
+      mbar_init(&conv_empty[i], 1);
+    }
+    for (int i = 0; i < TS; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 4);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int units = un.n_tiles * un.S;
+
+  if (threadIdx.x == 0) pdl_trigger();
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer.  The codes do not depend on earlier
+      // kernels: the first RS stages get their codes before the predecessor
+      // grid is waited for, their activations after.
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
+      int u = blockIdx.x, nt = 0, s = 0, c = 0, c1 = 0;
+      if (u < units) un.decode(u, nt, s, c, c1);
+      auto next = [&]() {
+        if (++c >= c1) {
+          u += gridDim.x;
+          if (u < units) un.decode(u, nt, s, c, c1);
+        }
+      };
+      int pre_c[RS];
+      int npre = 0;
+      while (npre < RS && u < units) {
+        mbar_expect_tx(&raw_full[npre], RAW_STAGE);
+        tma_load_2d(raw + npre * RAW_STAGE, &mapQ, &raw_full[npre], c * CK, nt * BM);
+        pre_c[npre++] = c;
+        next();
+      }
+      pdl_wait();
+      for (int i = 0; i < npre; ++i) {
+        tma_load_2d(raw + i * RAW_STAGE + RAW_A, &mapX, &raw_full[i], pre_c[i] * CK, 0);
+        tma_load_2d(raw + i * RAW_STAGE + RAW_A + RAW_B / 2, &mapX, &raw_full[i], pre_c[i] * CK + 64, 0);
+      }
+      issued = npre;
+      stage = npre % RS;
+      phase = npre == RS ? 1u : 0u;
+      while (u < units) {
+        if (!mbar_wait(&raw_empty[stage], phase ^ 1, abort_flag, err)) break;
+        uint8_t* dst = raw + stage * RAW_STAGE;
+        mbar_expect_tx(&raw_full[stage], RAW_STAGE);
+        tma_load_2d(dst, &mapQ, &raw_full[stage], c * CK, nt * BM);
+        tma_load_2d(dst + RAW_A, &mapX, &raw_full[stage], c * CK, 0);
+        tma_load_2d(dst + RAW_A + RAW_B / 2, &mapX, &raw_full[stage], c * CK + 64, 0);
+        ++issued;
+        if (++stage == RS) {
+          stage = 0;
+          phase ^= 1;
+        }
+        next();
+      }
+      {
+      int st = stage;
+      uint32_t ph = phase;
+      for (int i = 0; i < RS && i < issued; ++i) {
+        if (st == 0) {
+          st = RS;
+          ph ^= 1;
+        }
+        --st;
+        mbar_wait_drain(&raw_full[st], ph);
+      }
+    }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer: one TMEM slot (4 block accumulators) per chunk
+      constexpr uint32_t IDESC = idesc_f16(BM, MT);
+      int cst = 0, tsl = 0;
+      uint32_t cph = 0, tph = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        int nt, s, c0, c1;
+        un.decode(u, nt, s, c0, c1);
+        for (int c = c0; c < c1; ++c) {
+          if (!mbar_wait(&conv_full[cst], cph, abort_flag, err) || !mbar_wait(&tempty[tsl], tph ^ 1, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(conv + cst * CONV_STAGE), sb = sa + CONV_A;
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int q = b >> 1;
+            const uint64_t ad = sw128_desc(sa + q * (CONV_A / 2)), bd = sw128_desc(sb + q * (CONV_B / 2));
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+              const int kk = 2 * (b & 1) + k2;  // 16-column step inside the 64-column sub-tile
+              umma(tmem_base + tsl * 64 + b * 16, ad + 2 * kk, bd + 2 * kk, IDESC, k2);
+            }
+          }
+          umma_commit(&conv_empty[cst]);
+          umma_commit(&tfull[tsl]);
+          if (++cst == CS) {
+            cst = 0;
+            cph ^= 1;
+          }
+          if (++tsl == TS) {
+            tsl = 0;
+            tph ^= 1;
+          }
+        }
+      }
+      umma_commit(mma_done);
+      mbar_wait_drain(mma_done, 0);
+    }
+  } else if (warp < 6) {
+    // ---------------- epilogue: block accumulators -> scaled sums
+    pdl_wait();
+    const int lane_base = 32 * (warp & 3);
+    int tsl = 0;
+    uint32_t tph = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      int nt, s, c0, c1;
+      un.decode(u, nt, s, c0, c1);
+      const int n = nt * BM + lane_base + lane;
+      float acc[MT];
+#pragma unroll
+      for (int t = 0; t < MT; ++t) acc[t] = 0.f;
+      for (int c = c0; c < c1; ++c) {
+        const uint32_t sw = *reinterpret_cast<const uint32_t*>(scales + (size_t)n * nsb + c * 4);  // 4 blocks
+        if (!mbar_wait(&tfull[tsl], tph, abort_flag, err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          float v[16];
+          tmem_ld16(tmem_base + ((uint32_t)lane_base << 16) + tsl * 64 + b * 16, v);
+          const int e = (int)((sw >> (8 * b)) & 0xFFu) - 127 - 14;  // block scale and the activations' 2^14
+          const float sc = e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : ldexpf(1.f, e);
+#pragma unroll
+          for (int t = 0; t < MT; ++t) acc[t] = __fmaf_rn(v[t], sc, acc[t]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[tsl]);
+        if (++tsl == TS) {
+          tsl = 0;
+          tph ^= 1;
+        }
+      }
+      if (!ok) break;
+      float* out = Y + (size_t)s * part_stride + n;
+#pragma unroll
+      for (int t = 0; t < MT; ++t)
+        if (t < M) out[(size_t)t * ldy] = acc[t];
+    }
+  } else {
+    // ---------------- converters: raw E4M3 -> f16 tiles (128-byte swizzle), bf16 x -> f16(x * 2^14)
+    const int cw = warp - 6;
+    int rst = 0, cst = 0;
+    uint32_t rph = 0, cph = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      int nt, s, c0, c1;
+      un.decode(u, nt, s, c0, c1);
+      for (int c = c0; c < c1; ++c) {
+        if (!mbar_wait(&raw_full[rst], rph, abort_flag, err) || !mbar_wait(&conv_empty[cst], cph ^ 1, abort_flag, err)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* ra = raw + rst * RAW_STAGE;
+        uint8_t* ca = conv + cst * CONV_STAGE;
+        // A: this warp's 32 rows, 4 rows of 128 codes per warp instruction
+#pragma unroll 2
+        for (int it = 0; it < 8; ++it) {
+          const int r = 32 * cw + 4 * it + (lane >> 3), j = lane & 7;
+          const uint4 w = *reinterpret_cast<const uint4*>(ra + r * CK + j * 16);
+          const uint4 lo = make_uint4(e4m3x2_f16x2(w.x), e4m3x2_f16x2(w.x >> 16), e4m3x2_f16x2(w.y),
+                                      e4m3x2_f16x2(w.y >> 16));
+          const uint4 hi = make_uint4(e4m3x2_f16x2(w.z), e4m3x2_f16x2(w.z >> 16), e4m3x2_f16x2(w.w),
+                                      e4m3x2_f16x2(w.w >> 16));
+          uint8_t* sub = ca + (j >> 2) * (CONV_A / 2) + r * 128;  // codes 16j..16j+15: sub-tile j/4
+          const int ch = 2 * (j & 3);                               // 8-element chunks ch, ch+1 of the row
+          *reinterpret_cast<uint4*>(sub + ((ch ^ (r & 7)) << 4)) = lo;
+          *reinterpret_cast<uint4*>(sub + (((ch + 1) ^ (r & 7)) << 4)) = hi;
+        }
+        // B: 4 KB of swizzled bf16, same chunk positions in f16
+        bool bad = false;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int off = (cw * 32 + lane + 128 * i) * 16;
+          const uint4 w = *reinterpret_cast<const uint4*>(ra + RAW_A + off);
+          const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+          uint32_t o[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float a = __uint_as_float(in[q] << 16) * kXScale, b = __uint_as_float(in[q] & 0xFFFF0000u) * kXScale;
+            bad |= !(fabsf(a) < 65504.f && fabsf(b) < 65504.f);
+            const __half2 h = __floats2half2_rn(a, b);
+            o[q] = *reinterpret_cast<const uint32_t*>(&h);
+          }
+          *reinterpret_cast<uint4*>(ca + CONV_A + off) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        if (bad) set_error(err, DEV_ERR_RANGE);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&raw_empty[rst]);
+          mbar_arrive(&conv_full[cst]);
+        }
+        if (++rst == RS) {
+          rst = 0;
+          rph ^= 1;
+        }
+        if (++cst == CS) {
+          cst = 0;
+          cph ^= 1;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------------ host
+typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                             const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                             CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encode() {
+  static EncodeFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeFn)p;
+  }
+  return fn;
+}
+
+int num_sms_tc() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+}  // namespace
+
+int mx_gemm_splits(int N, int K) {
+  const int tiles = N / BM, nch = K / CK;
+  if (tiles <= 0 || nch <= 0) return 1;
+  int S = (num_sms_tc() + tiles - 1) / tiles;
+  S = S > 8 ? 8 : S;
+  return S > nch ? nch : (S < 1 ? 1 : S);
+}
+
+cudaError_t launch_mx_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const uint8_t* q, const uint8_t* scales,
+                              float* Y, int ldy, size_t part_stride, int S, int* err, cudaStream_t st) {
+  if (M < 1 || M > MT || N % BM || K % CK || ((uintptr_t)q & 15) || ((uintptr_t)X & 15) || (ldx * 2) % 16 ||
+      ((uintptr_t)scales & 3))
+    return cudaErrorNotSupported;
+  EncodeFn fn = encode();
+  if (!fn) return cudaErrorNotSupported;
+  CUtensorMap mq, mx;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N};
+    cuuint64_t strides[1] = {(cuuint64_t)K};
+    cuuint32_t box[2] = {CK, BM};
+    cuuint32_t es[2] = {1, 1};
+    if (fn(&mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(q), dims, strides, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorNotSupported;
+  }
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)ldx * 2};
+    cuuint32_t box[2] = {64, MT};
+    cuuint32_t es[2] = {1, 1};
+    if (fn(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<bf16*>(X), dims, strides, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorNotSupported;
+  }
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_mx_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int nch = K / CK;
+  if (S < 1) S = 1;
+  if (S > nch) S = nch;
+  Units un{N / BM, S, nch};
+  const int sms = num_sms_tc();
+  const int units = un.n_tiles * S;
+  const int grid = units < sms ? units : sms;
+  return launch(k_mx_gemm, grid, NTH, SMEM, st, mq, mx, scales, K, Y, ldy, part_stride, M, un, err);
+}
+
+}  // namespace dory

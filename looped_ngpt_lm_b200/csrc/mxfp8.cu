@@ -445,7 +445,8 @@ cudaError_t launch_mx_quantize(const bf16* W, int N, int K, uint8_t* q, uint8_t*
 cudaError_t launch_mx_gemv(int M, int N, int K, const bf16* X, int ldx, const uint8_t* q, const uint8_t* s,
                            float* Y, int ldy, int* err, cudaStream_t st, int impl) {
   if (M <= 0 || N <= 0 || K <= 0 || K % kMxBlock || ((uintptr_t)q & 15)) return cudaErrorNotSupported;
-  // the tensor-core kernel only by request: measured slower at every 4B decode shape
+  if (impl == 3) return launch_mx_gemm_tc(M, N, K, X, ldx, q, s, Y, ldy, 0, 1, err, st);
+  // the mma.sync kernel only by request: measured slower at every 4B decode shape
   if (impl == 2) {
     if (K * 16 > GV_SMEM_CAP) return cudaErrorNotSupported;  // 8 staged f16 tokens
     return run_gemv_tc(M, N, K, X, ldx, q, s, Y, ldy, err, st);

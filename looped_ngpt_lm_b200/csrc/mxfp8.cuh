@@ -29,8 +29,24 @@ cudaError_t launch_mx_quantize(const bf16* W, int N, int K, uint8_t* q, uint8_t*
 //   nothing).
 // impl 1: CUDA cores (|X| < 2^64, else DEV_ERR_RANGE; scale bytes <= 198,
 //   the quantiser's output for |w| < 2^80; K <= 40960).
-// impl 0: 1 (the faster of the two at every 4B decode shape).
+// impl 3: the TMA-fed tensor-core GEMM below, unsplit (M <= 16, N % 128 == 0,
+//   K % 128 == 0, X 16-byte aligned with ldx % 8 == 0, |X| < 4).
+// impl 0: 1 (the faster of 1 and 2 at every 4B decode shape).
 cudaError_t launch_mx_gemv(int M, int N, int K, const bf16* X, int ldx, const uint8_t* q, const uint8_t* s,
                            float* Y, int ldy, int* err, cudaStream_t st, int impl = 0);
+
+// MXFP8 decode GEMM on the tensor cores, fed by TMA (mx_gemm_tc.cu): S
+// partial products at Y + s * part_stride (row stride ldy) that the consumer
+// adds in order s = 0..S-1, for X [M, K] bf16 (row stride ldx).  The K range
+// of each split depends on (K, S) only and the tokens are independent MMA
+// columns, so a row's bits do not depend on M.  Limits: M <= 16,
+// N % 128 == 0, K % 128 == 0, X and q 16-byte aligned, ldx % 8 == 0, scales
+// 4-byte aligned (else cudaErrorNotSupported); |X| < 4 (else DEV_ERR_RANGE).
+cudaError_t launch_mx_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const uint8_t* q, const uint8_t* s,
+                              float* Y, int ldy, size_t part_stride, int S, int* err, cudaStream_t st);
+
+// Splits for launch_mx_gemm_tc: enough (N / 128, split) units to cover the
+// SMs, at most 8 and at most one per 128-column chunk.  Depends on (N, K).
+int mx_gemm_splits(int N, int K);
 
 }  // namespace dory

@@ -11,6 +11,8 @@
   dequantised weights, within the bf16 path's tolerances: logits relative L2
   <= 2e-2, and greedy tokens identical except at near ties.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -252,3 +254,61 @@ def test_attach_validation():
     with pytest.raises(dory.DoryError) as e:
         f32.attach_mxfp8(mx)
     assert e.value.status == 7
+
+
+# The TMA-fed tcgen05 GEMM (impl 3) runs only when opted in.
+opt_in = pytest.mark.skipif(os.environ.get("DORY_RUN_PENDING") != "1",
+                            reason="opt-in: set DORY_RUN_PENDING=1")
+
+
+@opt_in
+@pytest.mark.parametrize("M,N,K", [(1, 384, 256), (5, 2560, 2560), (16, 1024, 1024), (3, 128, 10240)])
+def test_tma_tcgen05_gemm_matches_oracle(M, N, K):
+    rng = np.random.default_rng(M + N + K)
+    w = rng.standard_normal((N, K)).astype(np.float32)
+    w /= np.linalg.norm(w, axis=1, keepdims=True)
+    w[0, 1:32] *= 1e-4
+    wb = synth.f32_to_bf16_bits(w)
+    xb = synth.f32_to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32) / np.sqrt(K))
+    q, s, _ = dory.quantize_mxfp8(bf16_cuda(wb), dequantised=False)
+    X = bf16_cuda(xb)
+    err = torch.zeros(4, dtype=torch.int32, device="cuda")
+    y = dory.gemv_mxfp8(X, q, s, impl=3, err=err)
+    torch.cuda.synchronize()
+    assert int(err[0]) == 0
+    codes, scales = MX.quantize(synth.bf16_bits_to_f32(wb))
+    x64 = synth.bf16_bits_to_f32(xb).astype(np.float64)
+    ref = MX.gemv(x64, codes, scales)
+    bound = 2e-5 * (np.abs(x64) @ np.abs(MX.dequantize(codes, scales)).T) + 1e-30
+    got = y.cpu().numpy()
+    assert np.all(np.abs(got - ref) <= bound), float(np.max(np.abs(got - ref) / bound))
+    for m in sorted({0, M - 1}):
+        one = dory.gemv_mxfp8(X[m:m + 1].contiguous(), q, s, impl=3)
+        assert torch.equal(one[0], y[m])
+
+
+@opt_in
+@pytest.mark.parametrize("k", [1, 4])
+def test_decode_with_tma_tcgen05_gemm_matches_oracle(mx_model, k):
+    shape, model, h, _ = mx_model
+    prompt = synth.make_prompt(7, 40, shape.vocab)
+    h.set_option(dory.OPT_MX_GEMV, 3)
+    h.reset()
+    toks, lg = gpu_generate(h, prompt, 9, k, dory.LAST_LOOP)
+    h.synchronize()
+    _, ora = O.generate(model, prompt, 9, k, O.LAST_LOOP, forced=toks[:-1])
+    errs = [rel_l2(lg[i], ora[i]) for i in range(len(toks))]
+    assert max(errs) <= 2e-2, errs
+    check_tokens(toks, ora, 4 * max(float(np.abs(lg[i] - ora[i]).max()) for i in range(len(toks))))
+    # per-loop speculative decoding stays token-identical (draft and verify passes fit 16 rows)
+    tok = torch.tensor(prompt[:30], dtype=torch.int32, device="cuda")
+    h.reset()
+    nxt = h.prefill([0], tok, [30], 4, dory.PER_LOOP)
+    plain = [int(nxt[0])]
+    for _ in range(7):
+        nxt = h.decode_step([0], nxt, 4, dory.PER_LOOP)
+        plain.append(int(nxt[0]))
+    first = h.prefill([1], tok, [30], 4, dory.PER_LOOP)
+    out, _, _ = h.spec_decode([1], first, 1, 4, 4, dory.PER_LOOP, 7)
+    assert [int(first[0])] + out[0].cpu().tolist() == plain
+    h.set_option(dory.OPT_MX_GEMV, 0)
