@@ -500,7 +500,7 @@ def main():
                     help="time one kernel alone instead of the decode step (prints its own JSON line)")
     ap.add_argument("--shape", default="qkv,o,gate_up,down,lm_head", help="GEMM shapes for --kernel gemm / mxgemv")
     ap.add_argument("--mx-impl", dest="mx_impl", type=int, default=1,
-                    help="--kernel mxgemv: 1 CUDA cores (default), 2 tensor cores")
+                    help="--kernel mxgemv: 1 CUDA cores (default), 2 mma.sync, 3 TMA-fed tcgen05 (one slice)")
     ap.add_argument("--m", type=int, default=1, help="token rows for --kernel gemm")
     ap.add_argument("--l2-lookahead-mb", dest="l2_mb", type=int, default=None,
                     help="bytes of upcoming weights each decode GEMM prefetches into L2 (MiB; 0 = off; "
@@ -893,8 +893,8 @@ def mx_gemv_probe(args):
     """The MXFP8 decode GEMV (dory_gemv_mxfp8) on the 4B decode shapes at M
     token rows, each timed alone like --kernel gemm: graph-replayed launches
     rotating through weight copies (> 2x L2) of random E4M3 codes (NaN codes
-    excluded) and scale bytes 110..124.  --mx-impl 1: CUDA cores, 2: tensor
-    cores."""
+    excluded) and scale bytes 110..124.  --mx-impl 1: CUDA cores, 2: mma.sync,
+    3: TMA-fed tcgen05 without split-K."""
     import ctypes
     import torch
     import looped_ngpt_lm_b200 as dory
