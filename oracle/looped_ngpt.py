@@ -44,9 +44,11 @@ Arithmetic is float64 by default; ``dtype=np.float32`` is accepted for the
 4B-shaped model, whose float64 weights would not fit in host memory.
 
 Pins (tests/test_oracle_pins.py) fix the pages' numbers, the invariants and
-the closed forms of the recurrence, the attention and the MLP.  Parity
-unpinned: the whole-model composition beyond them, because the pages print
-no worked example of a forward pass.
+the closed forms of the recurrence, the attention and the MLP, and the
+composition through relabelling invariances: renaming hidden units, MLP units
+or heads consistently must leave the logits unchanged.  No external
+reference value exists for a whole forward pass: the pages print no worked
+example.
 """
 from __future__ import annotations
 

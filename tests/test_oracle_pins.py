@@ -413,3 +413,64 @@ def test_unwritten_key_is_an_error(tiny, prompt):
 
 def test_norm_floor():
     assert np.array_equal(O.l2n(np.zeros((2, 3))), np.zeros((2, 3)))
+
+
+# ---------------------------------------------------------------- relabelling invariances
+def relabelled(model, perm_d=None, perm_ff=None, perm_kv=None, perm_in_group=None):
+    """The same network with its hidden units renamed: perm_d on the model width
+    (embedding and head columns, every input column and every output row onto
+    the residual stream), perm_ff on the MLP hidden units (gate and up rows,
+    down columns), perm_kv on the KV heads together with their query groups,
+    perm_in_group on the query heads inside every group.  The logits must not
+    change."""
+    s = model.shape
+    d, hd, G = s.d_model, s.head_dim, s.n_heads // s.n_kv_heads
+    w = {k: v.copy() for k, v in model.w.items()}
+    qh = np.arange(s.n_heads)
+    if perm_kv is not None or perm_in_group is not None:
+        kv = perm_kv if perm_kv is not None else np.arange(s.n_kv_heads)
+        ig = perm_in_group if perm_in_group is not None else np.arange(G)
+        qh = np.array([kv[h // G] * G + ig[h % G] for h in range(s.n_heads)])  # new head h <- old head qh[h]
+    else:
+        kv = np.arange(s.n_kv_heads)
+    q_rows = np.concatenate([np.arange(o * hd, (o + 1) * hd) for o in qh])
+    kv_rows = np.concatenate([np.arange(o * hd, (o + 1) * hd) for o in kv])
+    for l in range(s.n_layers):
+        if model.kind(l) == "attn":
+            w[f"L{l}.wq"] = w[f"L{l}.wq"][q_rows]
+            w[f"L{l}.wk"] = w[f"L{l}.wk"][kv_rows]
+            w[f"L{l}.wv"] = w[f"L{l}.wv"][kv_rows]
+            w[f"L{l}.wo"] = w[f"L{l}.wo"][:, q_rows]
+        elif perm_ff is not None:
+            w[f"L{l}.wg"] = w[f"L{l}.wg"][perm_ff]
+            w[f"L{l}.wu"] = w[f"L{l}.wu"][perm_ff]
+            w[f"L{l}.wdown"] = w[f"L{l}.wdown"][:, perm_ff]
+    if perm_d is not None:
+        for name in list(w):
+            if name in ("embed", "lm_head") or name.endswith((".wq", ".wk", ".wv", ".wg", ".wu")):
+                w[name] = w[name][:, perm_d]
+            elif name.endswith((".wo", ".wdown")):
+                w[name] = w[name][perm_d]
+    m = O.Model(s, {})
+    m.w = w
+    return m
+
+
+@pytest.mark.parametrize("what", ["width", "mlp_hidden", "kv_heads", "heads_in_group", "all"])
+@pytest.mark.parametrize("mode", [O.LAST_LOOP, O.PER_LOOP])
+def test_renaming_hidden_units_leaves_the_logits_unchanged(tiny, prompt, what, mode):
+    s = synth.TINY
+    rng = np.random.default_rng(11)
+    kw = {}
+    if what in ("width", "all"):
+        kw["perm_d"] = rng.permutation(s.d_model)
+    if what in ("mlp_hidden", "all"):
+        kw["perm_ff"] = rng.permutation(s.d_ff)
+    if what in ("kv_heads", "all"):  # a cyclic shift: never the identity
+        kw["perm_kv"] = np.roll(np.arange(s.n_kv_heads), 1)
+    if what in ("heads_in_group", "all"):
+        kw["perm_in_group"] = np.roll(np.arange(s.n_heads // s.n_kv_heads), 1)
+    other = relabelled(tiny, **kw)
+    a = O.forward_chunk(tiny, O.Cache(tiny, 40), prompt[:24], 2, mode, head="all")
+    b = O.forward_chunk(other, O.Cache(other, 40), prompt[:24], 2, mode, head="all")
+    assert np.abs(a - b).max() < 1e-12
