@@ -306,9 +306,9 @@ dory_status dory_quantize_mxfp8(const void* w, int32_t N, int32_t K, void* q, vo
  *     bytes <= 198 (what the quantiser writes for |w| < 2^80).
  *   impl 3: tcgen05 GEMM fed by TMA.  Converter warps expand the codes to
  *     f16 in shared memory; each 32-weight block accumulates in its own TMEM
- *     columns and takes its scale in the epilogue.  Requires M <= 16,
- *     N % 128 == 0, K % 128 == 0, x 16-byte aligned, ldx % 8 == 0, scales
- *     4-byte aligned (else DORY_ERR_UNSUPPORTED); |x| < 4.
+ *     columns and takes its scale in the epilogue.  Requires N % 128 == 0,
+ *     K % 128 == 0, x 16-byte aligned, ldx % 8 == 0 (else
+ *     DORY_ERR_UNSUPPORTED); |x| < 4.
  *   impl 0: 1 (measured faster than 2 at every 4B decode shape).
  * An activation outside the range (non-finite for 2) sets *err_word (device,
  * nullable).  Queues work on `stream`. */
@@ -347,6 +347,75 @@ typedef struct {
  * and leaves the previous attachment in place. */
 dory_status dory_attach_mxfp8(dory_handle* h, const dory_mx_weights* mx);
 
+/* ---------------------------------------------------------------- NVFP4
+ * 4-bit weights for decoding ([trawling] "KV cache and runtime"; [news]
+ * "Training and variants": 2.17x to 2.44x over BF16 at batch 1 on a DGX
+ * Spark).  The format is NVIDIA's NVFP4:
+ *   - FP4 E2M1 codes (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), two per byte,
+ *     the even k in the low nibble: q is [N, K/2] bytes;
+ *   - one FP8 E4M3 scale per 16 consecutive weights of a row: scales is
+ *     [N, K/16] bytes;
+ *   - one per-tensor float scale g.
+ *   w = E2M1(code) * E4M3(scale) * g.
+ *
+ * Quantise a row-major bf16 weight w [N, K] (device, 16-byte aligned,
+ * K % 16 == 0):
+ *   - g = the smallest power of two with 6 * 448 * g >= max |w|, written to
+ *     the device float *g;
+ *   - block scale = E4M3(amax_b / (6 g));
+ *   - code = E2M1(w / (scale * g)), both rounded to nearest-even and
+ *     saturating; codes are 0 for a block whose scale is 0, and a value that
+ *     rounds to zero keeps its sign.
+ * q is 8-byte aligned.  w_deq (nullable, 16-byte aligned) receives the exact
+ * bf16 dequantisation.  A non-finite weight sets *err_word.  Queues three
+ * launches on `stream`. */
+dory_status dory_quantize_nvfp4(const void* w, int32_t N, int32_t K, void* q, void* scales, float* g, void* w_deq,
+                                int32_t* err_word, dory_stream stream);
+
+/* y[i, n] = sum_k x[i, k] * E2M1(q[n, k]) * E4M3(scales[n, k/16]) * g, with
+ * fp32 sums, for x bf16 [M, ldx] (device) and y fp32 [M, ldy] (device).
+ * tcgen05 GEMM fed by TMA: converter warps expand the codes to f16; each
+ * 16-weight block accumulates in its own TMEM columns and takes its scale
+ * in the epilogue.  Each y[i, n] is summed in an order fixed by K alone.
+ * Requires N % 128 == 0, K % 256 == 0, x and q 16-byte aligned, ldx % 8 == 0
+ * (else DORY_ERR_UNSUPPORTED); |x| < 4 (else *err_word).  Queues work on
+ * `stream`. */
+dory_status dory_gemm_nvfp4(int32_t M, int32_t N, int32_t K, const void* x, int32_t ldx, const void* q,
+                            const void* scales, const float* g, float* y, int32_t ldy, int32_t* err_word,
+                            dory_stream stream);
+
+/* NVFP4 copies of a handle's projection weights and LM head (device
+ * pointers, BORROWED), indexed like dory_mx_weights, with each matrix's
+ * tensor scale as a device float. */
+typedef struct {
+  const void* lm_head_q;
+  const void* lm_head_s;
+  const float* lm_head_g;
+  const void* const* qkv_q;
+  const void* const* qkv_s;
+  const float* const* qkv_g;
+  const void* const* o_q;
+  const void* const* o_s;
+  const float* const* o_g;
+  const void* const* gu_q;
+  const void* const* gu_s;
+  const float* const* gu_g;
+  const void* const* down_q;
+  const void* const* down_s;
+  const float* const* down_g;
+} dory_nvfp4_weights;
+
+/* Attach NVFP4 copies (nv != NULL) or detach them (nv == NULL).  While
+ * attached, decode GEMMs (plain, mixed-k, speculative) run dory_gemm_nvfp4's
+ * kernel with split-K slices.  A handle holds one low-bit format at a time:
+ * attaching NVFP4 replaces attached MXFP8 copies and vice versa.  Needs bf16
+ * weights, and d_model, n_heads * head_dim and d_ff multiples of 256 (else
+ * DORY_ERR_UNSUPPORTED).  For a forward that is the dequantised model
+ * throughout, create the handle with the w_deq output of
+ * dory_quantize_nvfp4.  Drops captured decode graphs and turns the L2
+ * look-ahead off. */
+dory_status dory_attach_nvfp4(dory_handle* h, const dory_nvfp4_weights* nv);
+
 /* Synchronise `stream` and report device-side errors (DORY_ERR_TIMEOUT when
  * a bounded wait in a kernel gave up; the handle stays usable). */
 dory_status dory_synchronize(dory_handle* h, dory_stream stream);
@@ -367,8 +436,7 @@ enum {
    * computed. */
   DORY_OPT_L2_LOOKAHEAD = 7,
   /* GEMM on attached MXFP8 copies (see dory_gemv_mxfp8's impl): 0 (default, = 1), 1 CUDA cores,
-     2 mma.sync, 3 TMA-fed tcgen05 with split-K slices (passes of at most 16 rows; larger passes
-     use 1, so row-count invariance then needs every pass to fit) */
+     2 mma.sync, 3 TMA-fed tcgen05 with split-K slices (matrices whose N or K it does not take use 1) */
   DORY_OPT_MX_GEMV = 8
 };
 dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value);

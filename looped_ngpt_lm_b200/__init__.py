@@ -38,7 +38,8 @@ SYMBOLS = ["dory_workspace_size", "dory_create", "dory_destroy", "dory_reset", "
            "dory_decode_step", "dory_decode_step_mixed", "dory_spec_decode", "dory_kv_bytes", "dory_seq_len", "dory_read_state",
            "dory_read_kv", "dory_synchronize", "dory_set_option", "dory_profile_read", "dory_profile_reset",
            "dory_last_error", "dory_gemm_bf16", "dory_gemm_bf16_noalloc", "dory_pack_weight_bf16",
-           "dory_set_sampling", "dory_sample", "dory_quantize_mxfp8", "dory_gemv_mxfp8", "dory_attach_mxfp8"]
+           "dory_set_sampling", "dory_sample", "dory_quantize_mxfp8", "dory_gemv_mxfp8", "dory_attach_mxfp8",
+           "dory_quantize_nvfp4", "dory_gemm_nvfp4", "dory_attach_nvfp4"]
 
 
 class DoryError(RuntimeError):
@@ -64,6 +65,14 @@ class MxWeightsC(ctypes.Structure):
     _fields_ = [("lm_head_q", ctypes.c_void_p), ("lm_head_s", ctypes.c_void_p)] + [
         (n, ctypes.POINTER(ctypes.c_void_p)) for n in (
             "qkv_q", "qkv_s", "o_q", "o_s", "gu_q", "gu_s", "down_q", "down_s")]
+
+
+class NvWeightsC(ctypes.Structure):
+    _fields_ = [("lm_head_q", ctypes.c_void_p), ("lm_head_s", ctypes.c_void_p), ("lm_head_g", ctypes.c_void_p)]
+    for _n in ("qkv", "o", "gu", "down"):
+        _fields_ += [(f"{_n}_q", ctypes.POINTER(ctypes.c_void_p)), (f"{_n}_s", ctypes.POINTER(ctypes.c_void_p)),
+                     (f"{_n}_g", ctypes.POINTER(ctypes.c_void_p))]
+    del _n
 
 
 class SpecStats(ctypes.Structure):
@@ -102,6 +111,9 @@ def _load() -> ctypes.CDLL:
         "dory_quantize_mxfp8": [P, I32, I32, P, P, P, P, P],
         "dory_gemv_mxfp8": [I32, I32, I32, P, I32, P, P, P, I32, I32, P, P],
         "dory_attach_mxfp8": [P, ctypes.POINTER(MxWeightsC)],
+        "dory_quantize_nvfp4": [P, I32, I32, P, P, P, P, P, P],
+        "dory_gemm_nvfp4": [I32, I32, I32, P, I32, P, P, P, P, I32, P, P],
+        "dory_attach_nvfp4": [P, ctypes.POINTER(NvWeightsC)],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -295,6 +307,60 @@ class MxWeights:
         return sum(t.numel() for t in self.q.values()) + sum(t.numel() for t in self.s.values())
 
 
+def quantize_nvfp4(W, dequantised=True, err=None, stream=None):
+    """NVFP4 copy of a row-major [N, K] bf16 CUDA tensor: (code pairs uint8
+    [N, K/2], E4M3 scales uint8 [N, K/16], tensor scale float32 [1] on the
+    device, dequantised bf16 [N, K] or None)."""
+    import torch
+    N, K = W.shape
+    q = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    sc = torch.empty((N, K // 16), dtype=torch.uint8, device=W.device)
+    g = torch.empty(1, dtype=torch.float32, device=W.device)
+    deq = torch.empty((N, K), dtype=torch.bfloat16, device=W.device) if dequantised else None
+    _check(lib.dory_quantize_nvfp4(ctypes.c_void_p(W.data_ptr()), N, K, ctypes.c_void_p(q.data_ptr()),
+                                   ctypes.c_void_p(sc.data_ptr()), ctypes.c_void_p(g.data_ptr()),
+                                   ctypes.c_void_p(_ptr(deq)), ctypes.c_void_p(_ptr(err)), _stream(stream)))
+    return q, sc, g, deq
+
+
+def gemm_nvfp4(X, q, scales, g, Y=None, err=None, stream=None):
+    """Y = X . dequantize(q, scales, g)^T through dory_gemm_nvfp4 (X bf16 [M, K])."""
+    import torch
+    M, K = X.shape
+    N = q.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float32, device=X.device)
+    _check(lib.dory_gemm_nvfp4(M, N, K, ctypes.c_void_p(X.data_ptr()), X.stride(0), ctypes.c_void_p(q.data_ptr()),
+                               ctypes.c_void_p(scales.data_ptr()), ctypes.c_void_p(g.data_ptr()),
+                               ctypes.c_void_p(Y.data_ptr()), Y.stride(0), ctypes.c_void_p(_ptr(err)),
+                               _stream(stream)))
+    return Y
+
+
+class NvWeights:
+    """NVFP4 copies of a DeviceWeights' projection matrices and LM head, plus
+    `dequantised` (their exact bf16 dequantisation, same embedding)."""
+
+    def __init__(self, dw: DeviceWeights, stream=None):
+        self.shape = dw.shape
+        L = dw.shape.n_layers
+        self.q, self.s, self.g = {}, {}, {}
+        deq = {}
+        for name, t in dw.matrices():
+            self.q[name], self.s[name], self.g[name], deq[name] = quantize_nvfp4(t, stream=stream)
+        pick = lambda kind: [deq.get(f"{kind}{l}") for l in range(L)]  # noqa: E731
+        self.dequantised = DeviceWeights.from_tensors(dw.shape, dw.tensors["embed"], deq["lm_head"], pick("qkv"),
+                                                      pick("o"), pick("gu"), pick("down"))
+        arr = ctypes.c_void_p * L
+        self._keep = {f"{k}_{x}": arr(*[_ptr(d.get(f"{k}{l}")) for l in range(L)])
+                      for k in ("qkv", "o", "gu", "down") for x, d in (("q", self.q), ("s", self.s), ("g", self.g))}
+        self.c = NvWeightsC(self.q["lm_head"].data_ptr(), self.s["lm_head"].data_ptr(), self.g["lm_head"].data_ptr(),
+                            *[self._keep[f"{k}_{x}"] for k in ("qkv", "o", "gu", "down") for x in ("q", "s", "g")])
+
+    def nbytes(self) -> int:
+        return sum(t.numel() for d in (self.q, self.s) for t in d.values()) + 4 * len(self.g)
+
+
 def workspace_size(cfg: Config, alloc_mode=LAST_LOOP) -> int:
     n = ctypes.c_size_t()
     _check(lib.dory_workspace_size(ctypes.byref(cfg), MODES[alloc_mode], ctypes.byref(n)))
@@ -343,6 +409,11 @@ class Handle:
         """Decode GEMMs read these MXFP8 copies (None detaches)."""
         self.mx = mx
         _check(lib.dory_attach_mxfp8(self.h, ctypes.byref(mx.c) if mx is not None else None))
+
+    def attach_nvfp4(self, nv: "NvWeights | None"):
+        """Decode GEMMs read these NVFP4 copies (None detaches)."""
+        self.mx = nv
+        _check(lib.dory_attach_nvfp4(self.h, ctypes.byref(nv.c) if nv is not None else None))
 
     def prefill(self, seq_ids, tokens, lens, k, mode, logits=None, next_tokens=None, stream=None):
         import torch

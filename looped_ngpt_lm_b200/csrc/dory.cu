@@ -109,6 +109,8 @@ struct dory_handle {
   struct MxMat {
     const uint8_t* q;
     const uint8_t* s;
+    const float* g = nullptr;  // NVFP4 tensor scale (device)
+    int fmt = 0;               // 0 MXFP8, 1 NVFP4
   };
   std::unordered_map<const void*, MxMat> mx;
   int mx_impl = 0;  // GEMV on the copies: 0 default (CUDA cores), 1 CUDA cores, 2 tensor cores
@@ -377,10 +379,24 @@ dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, cons
     // decode and speculative rows read the MXFP8 copy when one is attached
     if (f.invariant && !H->mx.empty()) {
       auto it = H->mx.find(W);
+      if (it != H->mx.end() && it->second.fmt == 1) {
+        // NVFP4: the TMA-fed tensor-core GEMM with split-K slices
+        Scope sc(H, f.st, name, (double)N * K * (0.5 + 1.0 / 16) + (double)M * K * 2 + (double)M * N * 4);
+        const int S = nv_gemm_splits(N, K);
+        const size_t ps = part_rows * (size_t)ldy;
+        cudaError_t e = launch_nv_gemm_tc(M, N, K, (const bf16*)X, ldx, it->second.q, it->second.s, it->second.g, Y,
+                                          ldy, ps, S, H->err, f.st);
+        if (e == cudaErrorNotSupported) return fail(DORY_ERR_UNSUPPORTED, "%s: shape not supported by NVFP4", name);
+        if (e != cudaSuccess) return fail(DORY_ERR_CUDA, "%s: %s", name, cudaGetErrorString(e));
+        *S_out = S;
+        *ps_out = ps;
+        return DORY_OK;
+      }
       if (it != H->mx.end()) {
         Scope sc(H, f.st, name, (double)N * K * (1.0 + 1.0 / kMxBlock) + (double)M * K * 2 + (double)M * N * 4);
         if (H->mx_impl == 3) {
           // TMA-fed tensor-core GEMM with split-K slices; shapes it does not take use the CUDA-core GEMV
+          // (whose rows differ in their last bits, so a handle mixing the two loses row-count invariance)
           const int S = mx_gemm_splits(N, K);
           const size_t ps = part_rows * (size_t)ldy;
           cudaError_t e = launch_mx_gemm_tc(M, N, K, (const bf16*)X, ldx, it->second.q, it->second.s, Y, ldy, ps, S,
@@ -1253,8 +1269,8 @@ dory_status dory_gemv_mxfp8(int32_t m, int32_t n, int32_t k, const void* x, int3
                             dory_stream stream) {
   if (!x || !q || !scales || !y || m < 1 || n < 1 || k < 1 || ldx < k || ldy < n || impl < 0 || impl > 3)
     return fail(DORY_ERR_INVALID_ARG, "bad GEMV arguments");
-  if (impl == 3 && (m > 16 || n % 128 || k % 128 || ((uintptr_t)x & 15) || ldx % 8 || ((uintptr_t)scales & 3)))
-    return fail(DORY_ERR_UNSUPPORTED, "impl 3 needs M <= 16, N %% 128 == 0, K %% 128 == 0, aligned x and scales");
+  if (impl == 3 && (n % 128 || k % 128 || ((uintptr_t)x & 15) || ldx % 8))
+    return fail(DORY_ERR_UNSUPPORTED, "impl 3 needs N %% 128 == 0, K %% 128 == 0, x 16-byte aligned, ldx %% 8 == 0");
   if (k % kMxBlock || k > (impl == 2 ? 10240 : 40960))
     return fail(DORY_ERR_UNSUPPORTED, "K must be a multiple of 32 and at most %d", impl == 2 ? 10240 : 40960);
   if ((uintptr_t)q & 15) return fail(DORY_ERR_INVALID_ARG, "q must be 16-byte aligned");
@@ -1294,6 +1310,74 @@ dory_status dory_attach_mxfp8(dory_handle* h, const dory_mx_weights* mx) {
     if (!ok) return fail(DORY_ERR_INVALID_ARG, "each MXFP8 copy needs codes (16-byte aligned) and scales");
   }
   // graphs captured with the other weights are dropped
+  for (auto& g : h->graphs_cache)
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+  h->graphs_cache.clear();
+  h->mx.swap(map);
+  return DORY_OK;
+}
+
+dory_status dory_quantize_nvfp4(const void* w, int32_t n, int32_t k, void* q, void* scales, float* g, void* w_deq,
+                                int32_t* err_word, dory_stream stream) {
+  if (!w || !q || !scales || !g || n < 1 || k < 1) return fail(DORY_ERR_INVALID_ARG, "bad quantiser arguments");
+  if (k % 16) return fail(DORY_ERR_UNSUPPORTED, "K must be a multiple of 16");
+  if (((uintptr_t)w & 15) || ((uintptr_t)q & 7) || ((uintptr_t)w_deq & 15) || ((uintptr_t)g & 3))
+    return fail(DORY_ERR_INVALID_ARG, "w and w_deq must be 16-byte, q 8-byte and g 4-byte aligned");
+  CK(launch_nv_quantize((const bf16*)w, n, k, (uint8_t*)q, (uint8_t*)scales, g, (bf16*)w_deq, err_word,
+                        (cudaStream_t)stream));
+  return DORY_OK;
+}
+
+dory_status dory_gemm_nvfp4(int32_t m, int32_t n, int32_t k, const void* x, int32_t ldx, const void* q,
+                            const void* scales, const float* g, float* y, int32_t ldy, int32_t* err_word,
+                            dory_stream stream) {
+  if (!x || !q || !scales || !g || !y || m < 1 || n < 1 || k < 1 || ldx < k || ldy < n)
+    return fail(DORY_ERR_INVALID_ARG, "bad GEMM arguments");
+  if (n % 128 || k % 256 || ((uintptr_t)x & 15) || ldx % 8 || ((uintptr_t)q & 15))
+    return fail(DORY_ERR_UNSUPPORTED, "NVFP4 GEMM needs N %% 128 == 0, K %% 256 == 0, x and q 16-byte aligned, "
+                                      "ldx %% 8 == 0");
+  CK(launch_nv_gemm_tc(m, n, k, (const bf16*)x, ldx, (const uint8_t*)q, (const uint8_t*)scales, g, y, ldy, 0, 1,
+                       err_word, (cudaStream_t)stream));
+  return DORY_OK;
+}
+
+dory_status dory_attach_nvfp4(dory_handle* h, const dory_nvfp4_weights* nv) {
+  if (!h) return fail(DORY_ERR_INVALID_ARG, "NULL handle");
+  std::unordered_map<const void*, dory_handle::MxMat> map;
+  if (nv) {
+    const dory_config& c = h->c;
+    if (!h->bf16) return fail(DORY_ERR_UNSUPPORTED, "NVFP4 copies stand for bf16 weights only");
+    if (c.d_model % 256 || h->q_dim % 256 || c.d_ff % 256)
+      return fail(DORY_ERR_UNSUPPORTED, "d_model, n_heads * head_dim and d_ff must be multiples of 256");
+    bool ok = true;
+    auto add = [&](const void* w, const void* const* qs, const void* const* ss, const float* const* gs, int l) {
+      const void* q = qs ? qs[l] : nullptr;
+      const void* sc = ss ? ss[l] : nullptr;
+      const float* g = gs ? gs[l] : nullptr;
+      if (!q && !sc && !g) return;  // this matrix stays bf16
+      if (!q || !sc || !g || ((uintptr_t)q & 15)) ok = false;
+      dory_handle::MxMat m;
+      m.q = (const uint8_t*)q;
+      m.s = (const uint8_t*)sc;
+      m.g = g;
+      m.fmt = 1;
+      map[w] = m;
+    };
+    for (int l = 0; l < h->L; ++l) {
+      if (layer_is_attn(l)) {
+        add(h->w_qkv[l], nv->qkv_q, nv->qkv_s, nv->qkv_g, l);
+        add(h->w_o[l], nv->o_q, nv->o_s, nv->o_g, l);
+      } else {
+        add(h->w_gu[l], nv->gu_q, nv->gu_s, nv->gu_g, l);
+        add(h->w_down[l], nv->down_q, nv->down_s, nv->down_g, l);
+      }
+    }
+    const void* hq[1] = {nv->lm_head_q};
+    const void* hs[1] = {nv->lm_head_s};
+    const float* hg[1] = {nv->lm_head_g};
+    add(h->head, hq, hs, hg, 0);
+    if (!ok) return fail(DORY_ERR_INVALID_ARG, "each NVFP4 copy needs codes (16-byte aligned), scales and g");
+  }
   for (auto& g : h->graphs_cache)
     if (g.exec) cudaGraphExecDestroy(g.exec);
   h->graphs_cache.clear();

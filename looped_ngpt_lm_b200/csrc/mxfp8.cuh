@@ -29,24 +29,40 @@ cudaError_t launch_mx_quantize(const bf16* W, int N, int K, uint8_t* q, uint8_t*
 //   nothing).
 // impl 1: CUDA cores (|X| < 2^64, else DEV_ERR_RANGE; scale bytes <= 198,
 //   the quantiser's output for |w| < 2^80; K <= 40960).
-// impl 3: the TMA-fed tensor-core GEMM below, unsplit (M <= 16, N % 128 == 0,
+// impl 3: the TMA-fed tensor-core GEMM below, unsplit (N % 128 == 0,
 //   K % 128 == 0, X 16-byte aligned with ldx % 8 == 0, |X| < 4).
 // impl 0: 1 (the faster of 1 and 2 at every 4B decode shape).
 cudaError_t launch_mx_gemv(int M, int N, int K, const bf16* X, int ldx, const uint8_t* q, const uint8_t* s,
                            float* Y, int ldy, int* err, cudaStream_t st, int impl = 0);
 
-// MXFP8 decode GEMM on the tensor cores, fed by TMA (mx_gemm_tc.cu): S
+// Low-bit decode GEMMs on the tensor cores, fed by TMA (mx_gemm_tc.cu): S
 // partial products at Y + s * part_stride (row stride ldy) that the consumer
-// adds in order s = 0..S-1, for X [M, K] bf16 (row stride ldx).  The K range
-// of each split depends on (K, S) only and the tokens are independent MMA
-// columns, so a row's bits do not depend on M.  Limits: M <= 16,
-// N % 128 == 0, K % 128 == 0, X and q 16-byte aligned, ldx % 8 == 0, scales
-// 4-byte aligned (else cudaErrorNotSupported); |X| < 4 (else DEV_ERR_RANGE).
+// adds in order s = 0..S-1, for X [M, K] bf16 (row stride ldx), any M.  The
+// K range of each split depends on (K, S) only and the tokens are
+// independent MMA columns, so a row's bits do not depend on M.  Limits:
+// N % 128 == 0, K % 128 (MXFP8) or K % 256 (NVFP4) == 0, X and q 16-byte
+// aligned, ldx % 8 == 0 (else cudaErrorNotSupported); |X| < 4 (else
+// DEV_ERR_RANGE).
+// MXFP8: q [N, K] E4M3 codes, s [N, K/32] E8M0 scales.
 cudaError_t launch_mx_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const uint8_t* q, const uint8_t* s,
                               float* Y, int ldy, size_t part_stride, int S, int* err, cudaStream_t st);
+// NVFP4: q [N, K/2] E2M1 code pairs (even k in the low nibble), s [N, K/16]
+// E4M3 block scales, g the per-tensor scale (one device float).
+cudaError_t launch_nv_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const uint8_t* q, const uint8_t* s,
+                              const float* g, float* Y, int ldy, size_t part_stride, int S, int* err,
+                              cudaStream_t st);
 
-// Splits for launch_mx_gemm_tc: enough (N / 128, split) units to cover the
-// SMs, at most 8 and at most one per 128-column chunk.  Depends on (N, K).
+// NVFP4 copy of a row-major bf16 W [N, K] (K % 16 == 0): g (one device float)
+// receives the power-of-two tensor scale, q [N, K/2] the E2M1 code pairs, s
+// [N, K/16] the E4M3 block scales, deq (nullable) the exact bf16
+// dequantisation.  Three launches on st.  W, deq 16-byte aligned, q 8-byte
+// aligned.  A non-finite weight sets DEV_ERR_RANGE.
+cudaError_t launch_nv_quantize(const bf16* W, int N, int K, uint8_t* q, uint8_t* s, float* g, bf16* deq, int* err,
+                               cudaStream_t st);
+
+// Splits for the two GEMMs: enough (N / 128, split) units to cover the SMs,
+// at most 8 and at most one per chunk.  Depend on (N, K) only.
 int mx_gemm_splits(int N, int K);
+int nv_gemm_splits(int N, int K);
 
 }  // namespace dory

@@ -133,7 +133,6 @@ def test_mxfp8_argument_validation():
     assert G(1, 8, 40992, F, 40992, F, F, F, 8) == "DORY_ERR_UNSUPPORTED"  # staged activations too large
     assert G(1, 8, 10272, F, 10272, F, F, F, 8, impl=2) == "DORY_ERR_UNSUPPORTED"  # tensor cores: K <= 10240
     assert G(1, 8, 64, F, 64, F, F, F, 8, impl=4) == "DORY_ERR_INVALID_ARG"
-    assert G(17, 128, 128, F, 128, F, F, F, 128, impl=3) == "DORY_ERR_UNSUPPORTED"  # more than 16 rows
     assert G(1, 100, 128, F, 128, F, F, F, 100, impl=3) == "DORY_ERR_UNSUPPORTED"   # N % 128
     assert G(1, 128, 96, F, 96, F, F, F, 128, impl=3) == "DORY_ERR_UNSUPPORTED"    # K % 128
     assert G(1, 128, 128, F8, 128, F, F, F, 128, impl=3) == "DORY_ERR_UNSUPPORTED"  # x not 16-byte aligned
@@ -161,6 +160,21 @@ def test_mxfp8_argument_validation():
     assert A(hb, None) == "DORY_OK"
     assert lib.dory_set_option(hb, dory.OPT_MX_GEMV, 3) == 0
     assert lib.dory_set_option(hb, dory.OPT_MX_GEMV, 4) == 1
+    # NVFP4
+    NQ = lambda *a: status_name(lib.dory_quantize_nvfp4(*a, None, None))
+    assert NQ(F, 4, 40, F, F, F, None) == "DORY_ERR_UNSUPPORTED"       # K % 16
+    assert NQ(F8, 4, 64, F, F, F, None) == "DORY_ERR_INVALID_ARG"      # weights not 16-byte aligned
+    assert NQ(F, 4, 64, F, F, None, None) == "DORY_ERR_INVALID_ARG"    # no tensor scale
+    NG = lambda *a: status_name(lib.dory_gemm_nvfp4(*a, None, None))
+    assert NG(1, 100, 256, F, 256, F, F, F, F, 100) == "DORY_ERR_UNSUPPORTED"  # N % 128
+    assert NG(1, 128, 128, F, 128, F, F, F, F, 128) == "DORY_ERR_UNSUPPORTED"  # K % 256
+    assert NG(1, 128, 256, F, 256, F, F, None, F, 128) == "DORY_ERR_INVALID_ARG"  # no tensor scale
+    NA = lambda h, nv: status_name(lib.dory_attach_nvfp4(h, nv))
+    nv_full = dory.NvWeightsC(FAKE_WS, FAKE_WS, FAKE_WS, *([arr] * 12))
+    assert NA(h32, nv_full) == "DORY_ERR_UNSUPPORTED"  # fp32 weights
+    assert NA(hb, dory.NvWeightsC(FAKE_WS, FAKE_WS, None, *([arr] * 12))) == "DORY_ERR_INVALID_ARG"  # no g
+    assert NA(hb, nv_full) == "DORY_OK"
+    assert NA(hb, None) == "DORY_OK"
     lib.dory_destroy(h32)
     lib.dory_destroy(hb)
 

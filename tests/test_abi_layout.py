@@ -17,6 +17,7 @@ STRUCTS = {
     "dory_weights": (dory.Weights, [f[0] for f in dory.Weights._fields_]),
     "dory_spec_stats": (dory.SpecStats, [f[0] for f in dory.SpecStats._fields_]),
     "dory_mx_weights": (dory.MxWeightsC, [f[0] for f in dory.MxWeightsC._fields_]),
+    "dory_nvfp4_weights": (dory.NvWeightsC, [f[0] for f in dory.NvWeightsC._fields_]),
 }
 CONSTANTS = {
     "DORY_LAST_LOOP": dory.LAST_LOOP, "DORY_PER_LOOP": dory.PER_LOOP, "DORY_F32": dory.F32,

@@ -199,3 +199,29 @@ def test_converter_addressing_builds_the_swizzled_k_major_tile():
         for k in range(CK):
             c = (k % 64) // 8
             assert conv[(k // 64) * BM * 64 + r * 64 + ((c ^ (r % 8)) * 8) + k % 8] == ids[r][k]
+
+
+def test_nvfp4_converter_addressing_builds_the_swizzled_k_major_tile():
+    """NVFP4 tiles: a raw row is 128 bytes = 256 codes.  Lane l of converter warp w, pass it, holds
+    raw bytes 16j..16j+15 (j = l % 8) of row r = 32w + 4it + l/8, i.e. codes 32j..32j+31.  Its raw
+    word i (codes 32j+8i .. +7) becomes f16 chunk 4(j%2)+i of 64-column sub-tile j/2 at
+    r*128 + ((chunk ^ (r % 8)) * 16); read back through the swizzle rule every code is at (r, k)."""
+    BM, CK = 128, 256
+    ids = [[r * CK + k for k in range(CK)] for r in range(BM)]
+    conv = [None] * (4 * BM * 64)
+    for w in range(4):
+        for it in range(8):
+            for l in range(32):
+                r, j = 32 * w + 4 * it + (l >> 3), l & 7
+                base = (j >> 1) * BM * 64 + r * 64
+                for i in range(4):
+                    ch = 4 * (j & 1) + i
+                    for e in range(8):
+                        conv[base + ((ch ^ (r & 7)) * 8) + e] = ids[r][32 * j + 8 * i + e]
+    for r in range(BM):
+        for k in range(CK):
+            c = (k % 64) // 8
+            assert conv[(k // 64) * BM * 64 + r * 64 + ((c ^ (r % 8)) * 8) + k % 8] == ids[r][k]
+    # the MMA's block b (16 columns) is sub-tile b // 4, 16-column step b % 4
+    for b in range(16):
+        assert (b * 16) // 64 == b // 4 and ((b * 16) % 64) // 16 == b % 4
