@@ -496,7 +496,7 @@ def main():
     ap.add_argument("--mode", default="last_loop", choices=["last_loop", "per_loop"])
     ap.add_argument("--no-aux", action="store_true", help="skip the k sweep, e2e and CPU baseline legs")
     ap.add_argument("--profile-steps", type=int, default=3)
-    ap.add_argument("--kernel", default=None, choices=["gemm", "mxgemv"],
+    ap.add_argument("--kernel", default=None, choices=["gemm", "mxgemv", "nvgemm"],
                     help="time one kernel alone instead of the decode step (prints its own JSON line)")
     ap.add_argument("--shape", default="qkv,o,gate_up,down,lm_head", help="GEMM shapes for --kernel gemm / mxgemv")
     ap.add_argument("--mx-impl", dest="mx_impl", type=int, default=1,
@@ -520,7 +520,7 @@ def main():
     if args.kernel == "gemm":
         gemm_probe(args)
         return
-    if args.kernel == "mxgemv":
+    if args.kernel in ("mxgemv", "nvgemm"):
         mx_gemv_probe(args)
         return
     if args.warmup < 3:
@@ -894,7 +894,10 @@ def mx_gemv_probe(args):
     token rows, each timed alone like --kernel gemm: graph-replayed launches
     rotating through weight copies (> 2x L2) of random E4M3 codes (NaN codes
     excluded) and scale bytes 110..124.  --mx-impl 1: CUDA cores, 2: mma.sync,
-    3: TMA-fed tcgen05 without split-K."""
+    3: TMA-fed tcgen05 without split-K.  --kernel nvgemm: the NVFP4 GEMM
+    (dory_gemm_nvfp4) on random E2M1 code pairs, E4M3 scales 0x30..0x37 and
+    g = 2^-9."""
+    nv = args.kernel == "nvgemm"
     import ctypes
     import torch
     import looped_ngpt_lm_b200 as dory
@@ -906,11 +909,16 @@ def mx_gemv_probe(args):
     out = {}
     for name in args.shape.split(","):
         N, K = shapes[name]
-        wbytes = N * K + N * K // 32
+        wbytes = N * K // 2 + N * K // 16 if nv else N * K + N * K // 32
         copies = max(2, -(-300_000_000 // wbytes))
         g = torch.Generator(device="cuda").manual_seed(0)
         qs, ss = [], []
+        gscale = torch.tensor([2.0 ** -9], dtype=torch.float32, device="cuda")
         for _ in range(copies):
+            if nv:
+                qs.append(torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8, device="cuda"))
+                ss.append(torch.randint(0x30, 0x38, (N, K // 16), generator=g, dtype=torch.uint8, device="cuda"))
+                continue
             q = torch.randint(0, 0x7E, (N, K), generator=g, dtype=torch.uint8, device="cuda")
             q |= torch.randint(0, 2, (N, K), generator=g, dtype=torch.uint8, device="cuda") << 7
             qs.append(q)
@@ -919,6 +927,13 @@ def mx_gemv_probe(args):
         Y = torch.empty((args.m, N), dtype=torch.float32, device="cuda")
 
         def one(i, st):
+            if nv:
+                dory._check(dory.lib.dory_gemm_nvfp4(args.m, N, K, ctypes.c_void_p(X.data_ptr()), K,
+                                                      ctypes.c_void_p(qs[i].data_ptr()),
+                                                      ctypes.c_void_p(ss[i].data_ptr()),
+                                                      ctypes.c_void_p(gscale.data_ptr()), ctypes.c_void_p(Y.data_ptr()),
+                                                      N, None, ctypes.c_void_p(st.cuda_stream)))
+                return
             dory._check(dory.lib.dory_gemv_mxfp8(args.m, N, K, ctypes.c_void_p(X.data_ptr()), K,
                                                   ctypes.c_void_p(qs[i].data_ptr()), ctypes.c_void_p(ss[i].data_ptr()),
                                                   ctypes.c_void_p(Y.data_ptr()), N, args.mx_impl, None,
@@ -946,7 +961,8 @@ def mx_gemv_probe(args):
                      "frac_of_measured": round(by / us / 1e3 / hbm, 4)}
         del qs, ss, graph
         torch.cuda.empty_cache()
-    print(json.dumps({"kernel": "mx_gemv", "mx_impl": args.mx_impl, "m": args.m, "results": out,
+    print(json.dumps({"kernel": "nv_gemm" if nv else "mx_gemv", "mx_impl": None if nv else args.mx_impl,
+                      "m": args.m, "results": out,
                       "note": "graph-replayed back-to-back launches, weights cold in L2"}))
 
 
