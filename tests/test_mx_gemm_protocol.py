@@ -1,4 +1,4 @@
-"""The barrier protocol of the TMA-fed MXFP8 GEMM (csrc/mx_gemm_tc.cu), model-checked on
+"""The barrier protocol of the TMA-fed low-bit GEMM (csrc/mx_gemm_tc.cu, MXFP8 and NVFP4), model-checked on
 the CPU.
 
 The kernel's roles, each restated as a state machine:
