@@ -261,6 +261,15 @@ dory_status dory_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* X, const
 dory_status dory_gemm_bf16_noalloc(int32_t M, int32_t N, int32_t K, const void* X, const void* W, float* Y,
                                    int32_t batch_hint, dory_stream stream);
 
+/* Timeout report of dory_gemm_bf16_noalloc (no counterpart on the pages).
+ * Its GEMM's bounded waits give up after about a second; they then record
+ * the fact in a second word built into the library next to the scratch
+ * array, and every later call writes NaN into its Y until this function
+ * clears the word.  Synchronises `stream`, reads and clears the word, and
+ * returns DORY_ERR_TIMEOUT if a wait gave up since the last check
+ * (DORY_OK otherwise).  Allocates nothing. */
+dory_status dory_gemm_bf16_noalloc_status(dory_stream stream);
+
 /* Repack a row-major [N, K] bf16 weight (device src, 16-byte aligned,
  * N % 128 == 0, K % 64 == 0) into device dst (N*K*2 bytes, distinct from src)
  * in the packed tile layout: 128-row x 64-column tiles, each stored as its

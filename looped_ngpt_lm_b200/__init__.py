@@ -37,7 +37,8 @@ STATUS = {0: "DORY_OK", 1: "DORY_ERR_INVALID_ARG", 2: "DORY_ERR_CAPACITY", 3: "D
 SYMBOLS = ["dory_workspace_size", "dory_create", "dory_destroy", "dory_reset", "dory_prefill",
            "dory_decode_step", "dory_decode_step_mixed", "dory_spec_decode", "dory_kv_bytes", "dory_seq_len", "dory_read_state",
            "dory_read_kv", "dory_synchronize", "dory_set_option", "dory_profile_read", "dory_profile_reset",
-           "dory_last_error", "dory_gemm_bf16", "dory_gemm_bf16_noalloc", "dory_pack_weight_bf16",
+           "dory_last_error", "dory_gemm_bf16", "dory_gemm_bf16_noalloc", "dory_gemm_bf16_noalloc_status",
+           "dory_pack_weight_bf16",
            "dory_set_sampling", "dory_sample", "dory_quantize_mxfp8", "dory_gemv_mxfp8", "dory_attach_mxfp8",
            "dory_quantize_nvfp4", "dory_gemm_nvfp4", "dory_attach_nvfp4"]
 
@@ -105,6 +106,7 @@ def _load() -> ctypes.CDLL:
         "dory_profile_reset": [P],
         "dory_gemm_bf16": [I32, I32, I32, P, P, P, I32, I32, I32, IP, P, P],
         "dory_gemm_bf16_noalloc": [I32, I32, I32, P, P, P, I32, P],
+        "dory_gemm_bf16_noalloc_status": [P],
         "dory_pack_weight_bf16": [P, P, I32, I32, P],
         "dory_set_sampling": [P, ctypes.c_float, ctypes.c_float, ctypes.c_uint64],
         "dory_sample": [P, I32, I32, P, P, ctypes.c_float, ctypes.c_float, ctypes.c_uint64, P, P, P],

@@ -8,6 +8,16 @@ import synth
 
 MODES = {"last_loop": (O.LAST_LOOP, dory.LAST_LOOP), "per_loop": (O.PER_LOOP, dory.PER_LOOP)}
 
+# bf16 configurations must keep the logits within relative L2 2e-2 of the
+# oracle's.  Spread evenly, that error is about 2e-2 * rms(logits) per logit;
+# two logits moving that far in opposite directions can swap only when the
+# oracle's margin between them is below twice that.  A greedy choice that
+# differs from the oracle's argmax is accepted only under that margin.  The
+# threshold is fixed by the stated tolerance and the oracle's own logits; it
+# never grows with the error the run under test happens to make.
+BF16_LOGITS_TOL = 2e-2
+BF16_TIE_FRAC = 2 * BF16_LOGITS_TOL
+
 
 def make(shape, seed=0, alloc="per_loop", **cap):
     w = synth.make_weights(shape, seed)
@@ -33,19 +43,39 @@ def gpu_generate(h, prompt, n_new, k, mode, seq=0):
     return np.array(toks), np.stack(logits)
 
 
-def check_tokens(gpu_toks, ora_logits, tol):
-    """Every GPU choice must be the oracle's argmax, unless the oracle's best
-    and the GPU's choice are within `tol` (a near tie both sides may break
-    either way).  Returns the number of near-tie steps."""
-    ties = 0
+def top2_margin(row):
+    """Oracle logit of the best token minus that of the runner-up."""
+    part = np.partition(np.asarray(row, dtype=np.float64), -2)
+    return float(part[-1] - part[-2])
+
+
+def check_tokens(gpu_toks, ora_logits, tol=None, rel=None):
+    """Every GPU choice must be the oracle's argmax, except at a near tie:
+    the oracle's logit of its best token exceeds that of the GPU's choice by
+    at most `tol` (absolute) or `rel` * rms(oracle logits of that step).
+    Returns {"exempt": steps excused as near ties, "min_margin": smallest
+    top-2 margin of the oracle over the steps, "threshold": largest
+    threshold used}; the caller may assert on them."""
+    assert (tol is None) != (rel is None)
+    exempt, min_margin, thr_max = 0, float("inf"), 0.0
     for i, t in enumerate(gpu_toks):
-        best = int(np.argmax(ora_logits[i]))
-        if t == best:
+        row = np.asarray(ora_logits[i], dtype=np.float64)
+        thr = tol if tol is not None else rel * float(np.sqrt(np.mean(row * row)))
+        thr_max = max(thr_max, thr)
+        min_margin = min(min_margin, top2_margin(row))
+        best = int(np.argmax(row))
+        if int(t) == best:
             continue
-        gap = ora_logits[i][best] - ora_logits[i][t]
-        assert gap <= tol, f"step {i}: gpu chose {t}, oracle {best}, gap {gap}"
-        ties += 1
-    return ties
+        gap = float(row[best] - row[int(t)])
+        assert gap <= thr, (f"step {i}: gpu chose {int(t)}, oracle {best}; oracle margin {gap:.3e} "
+                            f"above the near-tie threshold {thr:.3e}")
+        exempt += 1
+    return {"exempt": exempt, "min_margin": min_margin, "threshold": thr_max}
+
+
+def check_bf16_tokens(gpu_toks, ora_logits):
+    """check_tokens at the bf16 near-tie threshold."""
+    return check_tokens(gpu_toks, ora_logits, rel=BF16_TIE_FRAC)
 
 
 def rel_l2(a, b):

@@ -16,7 +16,7 @@ if not torch.cuda.is_available():
     pytest.skip("needs a CUDA GPU", allow_module_level=True)
 
 import looped_ngpt_lm_b200 as dory  # noqa: E402
-from gpu_util import MODES, check_tokens, cosine_rows, gpu_generate, rel_l2  # noqa: E402
+from gpu_util import MODES, check_bf16_tokens, cosine_rows, gpu_generate, rel_l2  # noqa: E402
 
 SHAPE = synth.DORY_4B
 
@@ -42,8 +42,8 @@ def test_4b_decode_matches_oracle(model, k, mode, n_new):
     _, ora = O.generate(om, prompt, n_new, k, o_mode, forced=toks[:-1])
     errs = [rel_l2(lg[i], ora[i]) for i in range(n_new)]
     assert max(errs) <= 2e-2, errs
-    tol = 4 * max(float(np.abs(lg[i] - ora[i]).max()) for i in range(n_new))
-    check_tokens(toks, ora, tol)
+    ties = check_bf16_tokens(toks, ora)
+    print(f"4B k={k} {mode}: near-tie exemptions {ties}")
 
 
 @pytest.mark.parametrize("n", [64, 256])  # 256 rows: the warp-per-row add + norm

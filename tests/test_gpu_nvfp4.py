@@ -1,7 +1,5 @@
 """NVFP4 weights on the GPU against the oracle's format (oracle/nvfp4.py).
 
-The whole module is opt-in: set DORY_RUN_PENDING=1 to run it.
-
 * Quantiser: codes, block scales, the tensor scale and the bf16
   dequantisation must equal the oracle's bit for bit.  The oracle keeps one
   code per byte; the GPU packs two, the even k in the low nibble.
@@ -11,8 +9,6 @@ The whole module is opt-in: set DORY_RUN_PENDING=1 to run it.
   dequantised weights: logits relative L2 <= 2e-2, and greedy tokens
   identical except at near ties.
 """
-import os
-
 import numpy as np
 import pytest
 import torch
@@ -21,14 +17,13 @@ import oracle as O
 import synth
 from oracle import nvfp4 as F
 
-pytestmark = [pytest.mark.gpu, pytest.mark.skipif(os.environ.get("DORY_RUN_PENDING") != "1",
-                                                  reason="opt-in: set DORY_RUN_PENDING=1")]
+pytestmark = pytest.mark.gpu
 
 if not torch.cuda.is_available():
     pytest.skip("needs a CUDA GPU", allow_module_level=True)
 
 import looped_ngpt_lm_b200 as dory  # noqa: E402
-from gpu_util import check_tokens, gpu_generate, rel_l2  # noqa: E402
+from gpu_util import check_bf16_tokens, gpu_generate, rel_l2  # noqa: E402
 
 CAP = dict(max_batch=4, max_seq=160, k_max=4, gamma_max=4, max_chunk=128)
 
@@ -107,7 +102,7 @@ def test_decode_with_nvfp4_matches_oracle(nv_model, k, mode):
     _, ora = O.generate(model, prompt, 9, k, om, forced=toks[:-1])
     errs = [rel_l2(lg[i], ora[i]) for i in range(len(toks))]
     assert max(errs) <= 2e-2, errs
-    check_tokens(toks, ora, 4 * max(float(np.abs(lg[i] - ora[i]).max()) for i in range(len(toks))))
+    check_bf16_tokens(toks, ora)
 
 
 def test_speculative_decoding_with_nvfp4_is_token_identical(nv_model):

@@ -18,7 +18,7 @@ if not torch.cuda.is_available():
     pytest.skip("needs a CUDA GPU", allow_module_level=True)
 
 import looped_ngpt_lm_b200 as dory  # noqa: E402
-from gpu_util import MODES, check_tokens, cosine_rows, gpu_generate, make, rel_l2  # noqa: E402
+from gpu_util import MODES, check_bf16_tokens, check_tokens, cosine_rows, gpu_generate, make, rel_l2  # noqa: E402
 
 F32_TOL = 1e-4
 CAP = dict(max_batch=4, max_seq=160, k_max=4, gamma_max=4, max_chunk=128)
@@ -64,8 +64,8 @@ def test_tiny_bf16_matches_oracle(tiny_bf16, prompt, k, mode):
     _, ora = O.generate(model, prompt, 17, k, om, forced=toks[:-1])
     errs = [rel_l2(lg[i], ora[i]) for i in range(len(toks))]
     assert max(errs) <= 2e-2, errs
-    tol = 4 * max(float(np.abs(lg[i] - ora[i]).max()) for i in range(len(toks)))
-    check_tokens(toks, ora, tol)
+    ties = check_bf16_tokens(toks, ora)
+    print(f"tiny bf16 k={k} {mode}: near-tie exemptions {ties}")
     # final state of the prompt: rerun the prefill and read s_k for every row
     h.reset()
     tok = torch.tensor(prompt, dtype=torch.int32, device="cuda")
