@@ -446,7 +446,13 @@ enum {
   DORY_OPT_L2_LOOKAHEAD = 7,
   /* GEMM on attached MXFP8 copies (see dory_gemv_mxfp8's impl): 0 (default, = 1), 1 CUDA cores,
      2 mma.sync, 3 TMA-fed tcgen05 with split-K slices (matrices whose N or K it does not take use 1) */
-  DORY_OPT_MX_GEMV = 8
+  DORY_OPT_MX_GEMV = 8,
+  /* bf16 decode and speculative steps of at most this many rows (default 4,
+   * at most 16; 0 off): the add + L2 norm after a layer and the SwiGLU of a
+   * split gate-up product run inside the next projection GEMM, whose
+   * epilogue warps build its operand in shared memory, instead of as kernels
+   * of their own.  Same arithmetic, so the same bits, either way. */
+  DORY_OPT_FUSED_OPERANDS = 9
 };
 dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value);
 

@@ -126,14 +126,20 @@ struct dory_handle {
   int tiles_cap = 0;
   void* qh = nullptr;     // bf16 pre-scaled queries of long chunks
   RowMeta meta{};
-  float *h = nullptr, *x = nullptr, *s = nullptr, *q = nullptr, *part_qkv = nullptr, *part_y = nullptr,
-        *part_gu = nullptr, *attn_part = nullptr, *logits = nullptr;
+  // the state h lives in one of two buffers: a GEMM that applies the
+  // previous layer's update in its operand stage reads one and writes the other
+  float* hb[2] = {nullptr, nullptr};
+  int hc = 0;
+  float *x = nullptr, *s = nullptr, *q = nullptr, *part_qkv = nullptr, *part_y = nullptr, *part_gu = nullptr,
+        *attn_part = nullptr, *logits = nullptr;
   void *hop = nullptr, *ao = nullptr, *act = nullptr, *kscr = nullptr, *vscr = nullptr, *hop_head = nullptr;
   size_t part_rows = 0;      // rows of an unsplit GEMM output (prefill)
   size_t part_rows_dec = 0;  // rows per split slice on the decode / speculative path
   float *stash_x = nullptr, *stash_s = nullptr;
-  int *drafts = nullptr, *pending = nullptr, *vtok = nullptr, *out_len = nullptr, *all_done = nullptr;
+  int *drafts = nullptr, *pending = nullptr, *vtok = nullptr;
   unsigned long long* accepted = nullptr;
+  SpecIo* spec_io = nullptr;
+  int* spec_flags = nullptr;  // [0] all finished, [1] steps, [2] step bound hit
   unsigned* attn_counters = nullptr;  // [M_max * n_kv], zero between launches
   int nb_cap = 0;                     // key blocks per row the partial buffer holds
   int attn_rows = 0;                  // rows the partial buffer holds
@@ -163,12 +169,16 @@ struct dory_handle {
     long long key;
     int seen;
     cudaGraphExec_t exec;
+    int hc_end;  // state buffer holding h when the recorded step ends
   };
   std::vector<Graph> graphs_cache;
   cudaStream_t cap_stream = nullptr;  // private stream used only to record graphs
 
+  int fuse_rows = 4;  // operand stages for decode / speculative passes of at most this many rows (0 off)
+
   template <typename T>
   T* hop_t() const { return (T*)hop; }
+  float* hcur() const { return hb[hc]; }
 };
 
 namespace {
@@ -255,7 +265,8 @@ size_t layout(dory_handle* h) {
   h->meta.p0 = cv.take<int>(sizeof(int) * M);
   h->meta.base = cv.take<int>(sizeof(int) * M);
   h->meta.pend = cv.take<int>(sizeof(int) * M);
-  h->h = cv.take<float>(sizeof(float) * M * d);
+  h->hb[0] = cv.take<float>(sizeof(float) * M * d);
+  h->hb[1] = cv.take<float>(sizeof(float) * M * d);
   h->x = cv.take<float>(sizeof(float) * M * d);
   h->s = cv.take<float>(sizeof(float) * M * d);
   h->q = cv.take<float>(sizeof(float) * M * h->q_dim);
@@ -286,9 +297,9 @@ size_t layout(dory_handle* h) {
   h->drafts = cv.take<int>(sizeof(int) * c.max_batch * gc);
   h->pending = cv.take<int>(sizeof(int) * c.max_batch);
   h->vtok = cv.take<int>(sizeof(int) * c.max_batch * gc);
-  h->out_len = cv.take<int>(sizeof(int) * c.max_batch);
-  h->all_done = cv.take<int>(sizeof(int) * 4);
   h->accepted = cv.take<unsigned long long>(sizeof(unsigned long long) * 2);
+  h->spec_io = cv.take<SpecIo>(sizeof(SpecIo));
+  h->spec_flags = cv.take<int>(sizeof(int) * 4);
   // two GEMMs per physical layer per application, plus the LM head
   h->pf_nseg_max = 2 * (c.n_in + c.n_out + c.k_max * c.n_rec) + 1;
   h->pf_segs = cv.take<PfSeg>(sizeof(PfSeg) * (size_t)c.k_max * h->pf_nseg_max);
@@ -369,9 +380,11 @@ size_t prows(const Fwd<T>& f) {
 
 // Y (and, when the tensor-core kernel splits K, the slices after it) must
 // hold kMaxSplitK slices of part_rows rows of ldy floats.
+// prep: an operand stage the caller has checked with stage_ok (bf16
+// tensor-core decode GEMMs only); X is then unused.
 template <typename T>
 dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, const void* W, float* Y, int ldy,
-                 size_t part_rows, int* S_out, size_t* ps_out, const char* name) {
+                 size_t part_rows, int* S_out, size_t* ps_out, const char* name, const Prep* prep = nullptr) {
   dory_handle* H = f.H;
   *S_out = 1;
   *ps_out = 0;
@@ -445,12 +458,13 @@ dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, cons
         }
       }
       cudaError_t e = launch_gemm_tc(M, N, K, (const bf16*)X, ldx, (const bf16*)W, Y, ldy, part_rows,
-                                     H->err, f.batch, f.invariant, &S, &ps, f.st, 0, false, pp);
+                                     H->err, f.batch, f.invariant, &S, &ps, f.st, 0, false, pp, prep);
       if (e == cudaSuccess) {
         *S_out = S;
         *ps_out = ps;
         return DORY_OK;
       }
+      if (prep) return fail(DORY_ERR_CUDA, "%s: operand stage: %s", name, cudaGetErrorString(e));
       if (e != cudaErrorNotSupported) return fail(DORY_ERR_CUDA, "%s: %s", name, cudaGetErrorString(e));
       if (H->gemm_impl == 2) return fail(DORY_ERR_UNSUPPORTED, "%s: shape not supported by tcgen05 GEMM", name);
     }
@@ -465,20 +479,64 @@ dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, cons
     if (r_ != DORY_OK) return r_;       \
   } while (0)
 
+// Whether the GEMM of weight W ([N, K]) on this pass can take operand stage p.
+template <typename T>
+bool stage_ok(const Fwd<T>& f, int N, int K, const void* W, const Prep& p) {
+  const dory_handle* H = f.H;
+  if (sizeof(T) != 2 || !f.invariant || f.M > H->fuse_rows || H->gemm_impl == 1) return false;
+  if (!H->mx.empty() && H->mx.count(W)) return false;
+  return gemm_tc_prep_ok(f.M, N, K, f.batch, p);
+}
+
 // Apply physical layers l0..l1-1.  copy_last (if not NULL) also receives the
 // result of the last layer.
+//
+// Each layer ends with h <- N(h + y).  On decode and speculative passes of
+// few rows that update is carried to the next layer's first GEMM, which
+// applies it in its operand stage (reading h from one state buffer and
+// writing the other), and the SwiGLU of the gate-up product is applied by
+// the down projection's operand stage.  The last layer's update runs as its
+// own kernel, and so does any update the next GEMM cannot take.
 template <typename T>
 dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop, float* copy_last = nullptr) {
   dory_handle* H = f.H;
   const dory_config& c = H->c;
   const int M = f.M, d = c.d_model;
+  bool pend = false;  // h <- N(h + part_y) of the previous layer not yet applied
+  int S_pend = 1;
+  size_t ps_pend = 0;
+  auto flush = [&](float* copy) -> dory_status {
+    Scope sc(H, f.st, "addnorm", 0);
+    CK(launch_addnorm<T>(M, d, H->hcur(), H->hcur(), H->part_y, S_pend, ps_pend, d, H->hop_t<T>(), copy, f.st));
+    pend = false;
+    return DORY_OK;
+  };
+  // operand stage applying the pending update, or NULL after flushing it
+  auto take_pending = [&](int N, const void* W, Prep* p) -> const Prep* {
+    if (!pend) return nullptr;
+    p->mode = kPrepAddNorm;
+    p->h_in = H->hcur();
+    p->h_out = H->hb[H->hc ^ 1];
+    p->y = H->part_y;
+    p->S = S_pend;
+    p->ps = ps_pend;
+    p->ldy = d;
+    return stage_ok(f, N, d, W, *p) ? p : nullptr;
+  };
   for (int l = l0; l < l1; ++l) {
     int S;
     size_t ps;
     if (layer_is_attn(l)) {
       KVView kv = kv_view(H, l, loop, f.mode);
-      RET(gemm<T>(f, M, H->qkv_dim, d, H->hop_t<T>(), d, H->w_qkv[l], H->part_qkv, H->qkv_dim, prows(f), &S, &ps, "gemm_qkv"));
-      if (f.direct) {
+      Prep pq;
+      const Prep* pre = take_pending(H->qkv_dim, H->w_qkv[l], &pq);
+      if (pend && !pre) RET(flush(nullptr));
+      RET(gemm<T>(f, M, H->qkv_dim, d, H->hop_t<T>(), d, H->w_qkv[l], H->part_qkv, H->qkv_dim, prows(f), &S, &ps,
+                  pre ? "gemm_qkv_norm" : "gemm_qkv", pre));
+      if (pre) {
+        H->hc ^= 1;
+        pend = false;
+      }      if (f.direct) {
         // fused: q from the partials, own K/V into the cache, split-KV attention
         Scope sc(H, f.st, "attn_decode", 0);
         CK(launch_attn_decode<T>(M, c.n_heads, c.n_kv_heads, c.head_dim, H->part_qkv, S, ps, kv, H->meta, f.max_ctx,
@@ -523,6 +581,7 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop, float* copy_la
       if constexpr (sizeof(T) == 2) {
         // long chunks: gate-up GEMM with SwiGLU in its epilogue
         if (!f.invariant && H->gemm_impl != 1) {
+          if (pend) RET(flush(nullptr));
           Scope sc(H, f.st, "gemm_gate_up_glu", 4.0 * c.d_ff * d + 2.0 * M * d + 2.0 * M * c.d_ff);
           cudaError_t e = launch_gemm_glu(M, c.d_ff, d, (const bf16*)H->hop, d, (const bf16*)H->w_gu[l],
                                           (bf16*)H->act, H->err, f.st);
@@ -532,18 +591,40 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop, float* copy_la
             return fail(DORY_ERR_CUDA, "gemm_gate_up_glu: %s", cudaGetErrorString(e));
         }
       }
-      if (!fused) {
+      if (fused) {
+        RET(gemm<T>(f, M, d, c.d_ff, (const T*)H->act, c.d_ff, H->w_down[l], H->part_y, d, prows(f), &S, &ps,
+                    "gemm_down"));
+      } else {
+        Prep pg;
+        const Prep* pre = take_pending(2 * c.d_ff, H->w_gu[l], &pg);
+        if (pend && !pre) RET(flush(nullptr));
         RET(gemm<T>(f, M, 2 * c.d_ff, d, H->hop_t<T>(), d, H->w_gu[l], H->part_gu, 2 * c.d_ff, prows(f), &S, &ps,
-                    "gemm_gate_up"));
-        Scope sc(H, f.st, "swiglu", 0);
-        CK(launch_swiglu<T>(M, c.d_ff, H->part_gu, S, ps, (T*)H->act, f.st));
+                    pre ? "gemm_gate_up_norm" : "gemm_gate_up", pre));
+        if (pre) {
+          H->hc ^= 1;
+          pend = false;
+        }
+        // the down projection applies the SwiGLU in its operand stage when it can
+        Prep pd;
+        pd.mode = kPrepSwiglu;
+        pd.y = H->part_gu;
+        pd.S = S;
+        pd.ps = ps;
+        pd.ldy = 2 * c.d_ff;
+        const bool st_ok = stage_ok(f, d, c.d_ff, H->w_down[l], pd);
+        if (!st_ok) {
+          Scope sc(H, f.st, "swiglu", 0);
+          CK(launch_swiglu<T>(M, c.d_ff, H->part_gu, S, ps, (T*)H->act, f.st));
+        }
+        RET(gemm<T>(f, M, d, c.d_ff, (const T*)H->act, c.d_ff, H->w_down[l], H->part_y, d, prows(f), &S, &ps,
+                    st_ok ? "gemm_down_swiglu" : "gemm_down", st_ok ? &pd : nullptr));
       }
-      RET(gemm<T>(f, M, d, c.d_ff, (const T*)H->act, c.d_ff, H->w_down[l], H->part_y, d, prows(f), &S, &ps,
-                  "gemm_down"));
     }
-    Scope sc(H, f.st, "addnorm", 0);
-    CK(launch_addnorm<T>(M, d, H->h, H->part_y, S, ps, d, H->hop_t<T>(), l == l1 - 1 ? copy_last : nullptr, f.st));
+    pend = true;
+    S_pend = S;
+    ps_pend = ps;
   }
+  if (pend) RET(flush(copy_last));
   return DORY_OK;
 }
 
@@ -554,7 +635,8 @@ dory_status input_block(const Fwd<T>& f, const int* tokens) {
   const dory_config& c = H->c;
   {
     Scope sc(H, f.st, "embed", 0);
-    CK(launch_embed<T>(f.M, c.d_model, c.vocab, tokens, (const T*)H->embed, H->h, H->hop_t<T>(),
+    H->hc = 0;  // every pass starts its state in the first buffer
+    CK(launch_embed<T>(f.M, c.d_model, c.vocab, tokens, (const T*)H->embed, H->hcur(), H->hop_t<T>(),
                        c.n_in == 0 ? H->x : nullptr, H->err, f.st));
   }
   RET(run_layers<T>(f, 0, c.n_in, 0, H->x));
@@ -575,7 +657,7 @@ dory_status loops(const Fwd<T>& f, int t0, int k, int stash_col, int rps) {
     float* save = (t > 1 && t - 1 == 1 && stash_col >= 0) ? H->stash_s : nullptr;
     {
       Scope sc(H, f.st, "reinject", 0);
-      CK(launch_reinject<T>(f.M, d, H->h, H->x, src, H->s, true, H->hop_t<T>(), save, rps, gc,
+      CK(launch_reinject<T>(f.M, d, H->hcur(), H->x, src, H->s, true, H->hop_t<T>(), save, rps, gc,
                             stash_col < 0 ? 0 : stash_col, f.st));
     }
     RET(run_layers<T>(f, c.n_in, c.n_in + c.n_rec, t));
@@ -584,12 +666,12 @@ dory_status loops(const Fwd<T>& f, int t0, int k, int stash_col, int rps) {
   // or in the speculative stash when a stash column is given
   Scope sc(H, f.st, "reinject", 0);
   if (t0 > k) {
-    CK(launch_reinject<T>(f.M, d, H->h, H->x, 2, H->s, false, H->hop_t<T>(), nullptr, 1, 1, 0, f.st));
+    CK(launch_reinject<T>(f.M, d, H->hcur(), H->x, 2, H->s, false, H->hop_t<T>(), nullptr, 1, 1, 0, f.st));
   } else if (stash_col >= 0 && k == 1) {
-    CK(launch_reinject<T>(f.M, d, H->h, H->x, 1, nullptr, false, H->hop_t<T>(), H->stash_s, rps, gc, stash_col,
+    CK(launch_reinject<T>(f.M, d, H->hcur(), H->x, 1, nullptr, false, H->hop_t<T>(), H->stash_s, rps, gc, stash_col,
                           f.st));
   } else {
-    CK(launch_reinject<T>(f.M, d, H->h, H->x, 1, nullptr, false, H->hop_t<T>(), H->s, 1, 1, 0, f.st));
+    CK(launch_reinject<T>(f.M, d, H->hcur(), H->x, 1, nullptr, false, H->hop_t<T>(), H->s, 1, 1, 0, f.st));
   }
   return DORY_OK;
 }
@@ -793,7 +875,7 @@ dory_status decode_t(dory_handle* H, int batch, const int32_t* seq_ids, const in
     for (auto& e : H->graphs_cache)
       if (e.key == key) g = &e;
     if (!g) {
-      H->graphs_cache.push_back({key, 0, nullptr});
+      H->graphs_cache.push_back({key, 0, nullptr, 0});
       g = &H->graphs_cache.back();
     }
     CK(cudaMemcpyAsync(H->tokens, tokens_in, sizeof(int) * batch, cudaMemcpyDeviceToDevice, st));
@@ -821,8 +903,10 @@ dory_status decode_t(dory_handle* H, int batch, const int32_t* seq_ids, const in
           g->exec = nullptr;
           return fail(DORY_ERR_CUDA, "graph instantiate: %s", cudaGetErrorString(e));
         }
+        g->hc_end = H->hc;
       }
       CK(cudaGraphLaunch(g->exec, st));
+      H->hc = g->hc_end;
     }
     CK(cudaMemcpyAsync(next_tokens, H->next, sizeof(int) * batch, cudaMemcpyDeviceToDevice, st));
   }
@@ -858,13 +942,13 @@ dory_status decode_mixed_t(dory_handle* H, int batch, const int32_t* seq_ids, co
     {
       // u_t = N(s_{t-1} + x), s_0 = x, s_{t-1} = N(h)
       Scope sc(H, st, "reinject", 0);
-      CK(launch_reinject<T>(rows, d, H->h, H->x, t == 1 ? 0 : 1, H->s, true, H->hop_t<T>(), nullptr, 1, 1, 0, st));
+      CK(launch_reinject<T>(rows, d, H->hcur(), H->x, t == 1 ? 0 : 1, H->s, true, H->hop_t<T>(), nullptr, 1, 1, 0, st));
     }
     RET(run_layers<T>(g, c.n_in, c.n_in + c.n_rec, t));
   }
   {
     Scope sc(H, st, "reinject", 0);
-    CK(launch_reinject<T>(batch, d, H->h, H->x, 1, nullptr, false, H->hop_t<T>(), H->s, 1, 1, 0, st));
+    CK(launch_reinject<T>(batch, d, H->hcur(), H->x, 1, nullptr, false, H->hop_t<T>(), H->s, 1, 1, 0, st));
   }
   RET(output_and_head<T>(f, batch, nullptr, logits, next_tokens));
   CK(launch_advance(batch, H->seq_ids, H->seq_len, 1, st));
@@ -873,78 +957,154 @@ dory_status decode_mixed_t(dory_handle* H, int batch, const int32_t* seq_ids, co
   return DORY_OK;
 }
 
+// One step of self-speculative decoding for B sequences: gamma draft passes
+// at k = 1, the input block and loop 1 of d_gamma, the verify pass from loop
+// 2 at k_verify, then acceptance on the device.  cond: the graph conditional
+// the acceptance sets while another step is needed (0: none).
+template <typename T>
+dory_status spec_step(dory_handle* H, int B, int kv_, int gamma, int mode, int max_ctx, cudaStream_t st,
+                      unsigned long long cond) {
+  const dory_config& c = H->c;
+  const int gc = c.gamma_max + 1;
+  // drafts: y0, d1..d_{gamma-1} at k = 1, one token per sequence each
+  for (int i = 0; i < gamma; ++i) {
+    CK(launch_plan_uniform(B, 1, i, H->seq_ids, H->seq_len, H->meta, st));
+    Fwd<T> f{H, st, B, max_ctx, true, mode, 1, B, true};
+    follow_stream(H, f, 1, 0);  // a draft is a k = 1 step
+    const int* tok = i == 0 ? H->pending : H->drafts + (i - 1) * B;
+    RET(input_block<T>(f, tok));
+    CK(launch_stash_copy(B, c.d_model, H->x, H->stash_x, 1, gc, i, 0, st));
+    RET(loops<T>(f, 1, 1, i, 1));
+    RET(output_and_head<T>(f, B, nullptr, nullptr, H->drafts + i * B));
+  }
+  // d_gamma: input block and loop 1 only
+  {
+    CK(launch_plan_uniform(B, 1, gamma, H->seq_ids, H->seq_len, H->meta, st));
+    Fwd<T> f{H, st, B, max_ctx, true, mode, 1, B, true};
+    follow_stream(H, f, 1, 0);  // the first two blocks of a k = 1 step
+    RET(input_block<T>(f, H->drafts + (gamma - 1) * B));
+    CK(launch_stash_copy(B, c.d_model, H->x, H->stash_x, 1, gc, gamma, 0, st));
+    Scope sc(H, st, "reinject", 0);
+    CK(launch_reinject<T>(B, c.d_model, H->hcur(), H->x, 0, nullptr, true, H->hop_t<T>(), nullptr, 1, 1, 0, st));
+    RET(run_layers<T>(f, c.n_in, c.n_in + c.n_rec, 1));
+    CK(launch_reinject<T>(B, c.d_model, H->hcur(), H->x, 1, nullptr, false, H->hop_t<T>(), H->stash_s, 1, gc,
+                          gamma, st));
+  }
+  // verify [y0, d1..d_gamma] at k_verify from the stashed x and s_1
+  const int rps = gamma + 1, M = B * rps;
+  CK(launch_plan_uniform(B, rps, 0, H->seq_ids, H->seq_len, H->meta, st));
+  Fwd<T> f{H, st, M, max_ctx, true, mode, kv_, B, true};
+  follow_stream(H, f, kv_, 2 * (c.n_in + c.n_rec));  // a k_verify step from its loop 2 on
+  CK(launch_stash_copy(M, c.d_model, H->x, H->stash_x, rps, gc, 0, 1, st));
+  CK(launch_stash_copy(M, c.d_model, H->s, H->stash_s, rps, gc, 0, 1, st));
+  RET(loops<T>(f, 2, kv_, -1, rps));
+  RET(output_and_head<T>(f, M, nullptr, nullptr, H->vtok));
+  CK(launch_spec_accept(B, gamma, B, H->seq_ids, H->seq_len, H->drafts, H->vtok, H->pending, H->spec_io,
+                        H->accepted, H->spec_flags, H->err, cond, cond != 0, st));
+  H->last_rows = M;
+  return DORY_OK;
+}
+
+// The whole speculative loop as one CUDA graph: a conditional while node
+// whose body is one recorded step; the acceptance kernel decides on the
+// device whether the body runs again, so the host waits once, at the end.
+template <typename T>
+dory_status spec_graph(dory_handle* H, int B, int kv_, int gamma, int mode, cudaStream_t st, bool* built) {
+  *built = false;
+  const long long key = (1ll << 40) | ((long long)B << 16) | (gamma << 8) | (kv_ << 4) | mode;
+  dory_handle::Graph* g = nullptr;
+  for (auto& e : H->graphs_cache)
+    if (e.key == key) g = &e;
+  if (!g) {
+    if (!H->cap_stream) CK(cudaStreamCreateWithFlags(&H->cap_stream, cudaStreamNonBlocking));
+    cudaGraph_t graph = nullptr;
+    CK(cudaGraphCreate(&graph, 0));
+    cudaGraphConditionalHandle cond = 0;
+    cudaError_t e = cudaGraphConditionalHandleCreate(&cond, graph, 1, cudaGraphCondAssignDefault);
+    cudaGraphNodeParams np = {};
+    np.type = cudaGraphNodeTypeConditional;
+    np.conditional.handle = cond;
+    np.conditional.type = cudaGraphCondTypeWhile;
+    np.conditional.size = 1;
+    cudaGraphNode_t node = nullptr;
+    if (e == cudaSuccess) e = cudaGraphAddNode(&node, graph, nullptr, 0, &np);
+    if (e != cudaSuccess) {
+      cudaGraphDestroy(graph);
+      return DORY_OK;  // no conditional nodes here: the caller runs the host loop
+    }
+    cudaGraph_t body = np.conditional.phGraph_out[0];
+    const int hc0 = H->hc;
+    dory_status r = DORY_OK;
+    e = cudaStreamBeginCaptureToGraph(H->cap_stream, body, nullptr, nullptr, 0, cudaStreamCaptureModeThreadLocal);
+    if (e == cudaSuccess) {
+      r = spec_step<T>(H, B, kv_, gamma, mode, H->c.max_seq, H->cap_stream, (unsigned long long)cond);
+      cudaGraph_t out = nullptr;
+      e = cudaStreamEndCapture(H->cap_stream, &out);
+    }
+    cudaGraphExec_t exec = nullptr;
+    if (r == DORY_OK && e == cudaSuccess) e = cudaGraphInstantiate(&exec, graph, 0);
+    cudaGraphDestroy(graph);
+    cudaGetLastError();  // a refused capture or instantiation leaves no sticky error
+    if (r != DORY_OK) return r;
+    if (e != cudaSuccess) {
+      H->hc = hc0;
+      return DORY_OK;  // the caller runs the host loop
+    }
+    H->graphs_cache.push_back({key, 1, exec, H->hc});
+    g = &H->graphs_cache.back();
+  }
+  CK(cudaGraphLaunch(g->exec, st));
+  H->hc = g->hc_end;
+  *built = true;
+  return DORY_OK;
+}
+
 template <typename T>
 dory_status spec_t(dory_handle* H, int B, const int32_t* seq_ids, const int32_t* last_tokens, int kv_, int gamma,
                    int mode, int max_new, int32_t* out_tokens, int32_t* out_len, dory_spec_stats* stats,
                    cudaStream_t st) {
   const dory_config& c = H->c;
-  const int gc = c.gamma_max + 1;
   int max_ctx = 0;
   for (int i = 0; i < B; ++i) max_ctx = std::max(max_ctx, H->len[seq_ids[i]] + max_new + 2 * gamma + 1);
   RET(upload_ids(H, seq_ids, B, st));
   RET(ensure_stream(H, 1, st));
   RET(ensure_stream(H, kv_, st));
+  SpecIo io{out_tokens, out_len, max_new, 0};
+  CK(cudaMemcpyAsync(H->spec_io, &io, sizeof io, cudaMemcpyHostToDevice, st));
   CK(cudaMemcpyAsync(H->pending, last_tokens, sizeof(int) * B, cudaMemcpyDeviceToDevice, st));
   CK(cudaMemsetAsync(out_len, 0, sizeof(int) * B, st));
   CK(cudaMemsetAsync(H->accepted, 0, sizeof(unsigned long long), st));
-  int64_t steps = 0;
-  for (;;) {
-    // drafts: y0, d1..d_{gamma-1} at k = 1, one token per sequence each
-    for (int i = 0; i < gamma; ++i) {
-      CK(launch_plan_uniform(B, 1, i, H->seq_ids, H->seq_len, H->meta, st));
-      Fwd<T> f{H, st, B, max_ctx, true, mode, 1, B, true};
-      follow_stream(H, f, 1, 0);  // a draft is a k = 1 step
-      const int* tok = i == 0 ? H->pending : H->drafts + (i - 1) * B;
-      RET(input_block<T>(f, tok));
-      CK(launch_stash_copy(B, c.d_model, H->x, H->stash_x, 1, gc, i, 0, st));
-      RET(loops<T>(f, 1, 1, i, 1));
-      RET(output_and_head<T>(f, B, nullptr, nullptr, H->drafts + i * B));
+  CK(cudaMemsetAsync(H->spec_flags, 0, sizeof(int) * 4, st));
+  bool on_device = false;
+  if (H->graphs && !H->profile) RET(spec_graph<T>(H, B, kv_, gamma, mode, st, &on_device));
+  if (!on_device) {
+    // host loop: one step, then the host reads whether another is needed
+    for (int64_t steps = 0;; ++steps) {
+      RET(spec_step<T>(H, B, kv_, gamma, mode, max_ctx, st, 0));
+      int flags[4] = {0, 0, 0, 0};
+      CK(cudaMemcpyAsync(flags, H->spec_flags, sizeof flags, cudaMemcpyDeviceToHost, st));
+      CK(cudaStreamSynchronize(st));
+      if (flags[0] || flags[2]) break;
     }
-    // d_gamma: input block and loop 1 only
-    {
-      CK(launch_plan_uniform(B, 1, gamma, H->seq_ids, H->seq_len, H->meta, st));
-      Fwd<T> f{H, st, B, max_ctx, true, mode, 1, B, true};
-      follow_stream(H, f, 1, 0);  // the first two blocks of a k = 1 step
-      RET(input_block<T>(f, H->drafts + (gamma - 1) * B));
-      CK(launch_stash_copy(B, c.d_model, H->x, H->stash_x, 1, gc, gamma, 0, st));
-      Scope sc(H, st, "reinject", 0);
-      CK(launch_reinject<T>(B, c.d_model, H->h, H->x, 0, nullptr, true, H->hop_t<T>(), nullptr, 1, 1, 0, st));
-      RET(run_layers<T>(f, c.n_in, c.n_in + c.n_rec, 1));
-      CK(launch_reinject<T>(B, c.d_model, H->h, H->x, 1, nullptr, false, H->hop_t<T>(), H->stash_s, 1, gc, gamma,
-                            st));
-    }
-    // verify [y0, d1..d_gamma] at k_verify from the stashed x and s_1
-    {
-      const int rps = gamma + 1, M = B * rps;
-      CK(launch_plan_uniform(B, rps, 0, H->seq_ids, H->seq_len, H->meta, st));
-      Fwd<T> f{H, st, M, max_ctx, true, mode, kv_, B, true};
-      follow_stream(H, f, kv_, 2 * (c.n_in + c.n_rec));  // a k_verify step from its loop 2 on
-      CK(launch_stash_copy(M, c.d_model, H->x, H->stash_x, rps, gc, 0, 1, st));
-      CK(launch_stash_copy(M, c.d_model, H->s, H->stash_s, rps, gc, 0, 1, st));
-      RET(loops<T>(f, 2, kv_, -1, rps));
-      RET(output_and_head<T>(f, M, nullptr, nullptr, H->vtok));
-      CK(launch_spec_accept(B, gamma, B, H->seq_ids, H->seq_len, H->drafts, H->vtok, H->pending, out_tokens, out_len,
-                            max_new, H->accepted, H->all_done, st));
-      H->last_rows = M;
-    }
-    ++steps;
-    int done = 0;
-    CK(cudaMemcpyAsync(&done, H->all_done, sizeof(int), cudaMemcpyDeviceToHost, st));
-    CK(cudaStreamSynchronize(st));
-    if (done) break;
-    if (steps > (int64_t)max_new + 1) return fail(DORY_ERR_STATE, "speculative loop did not finish");
   }
+  // the one wait of the call: lengths, acceptance counts and step flags
   std::vector<int> lens(c.max_batch);
-  CK(cudaMemcpyAsync(lens.data(), H->seq_len, sizeof(int) * c.max_batch, cudaMemcpyDeviceToHost, st));
+  int flags[4] = {0, 0, 0, 0}, err[4] = {0, 0, 0, 0};
   unsigned long long acc = 0;
+  CK(cudaMemcpyAsync(lens.data(), H->seq_len, sizeof(int) * c.max_batch, cudaMemcpyDeviceToHost, st));
   CK(cudaMemcpyAsync(&acc, H->accepted, sizeof(acc), cudaMemcpyDeviceToHost, st));
+  CK(cudaMemcpyAsync(flags, H->spec_flags, sizeof flags, cudaMemcpyDeviceToHost, st));
+  CK(cudaMemcpyAsync(err, H->err, sizeof err, cudaMemcpyDeviceToHost, st));
   CK(cudaStreamSynchronize(st));
   for (int i = 0; i < B; ++i) H->len[seq_ids[i]] = lens[seq_ids[i]];
+  H->last_rows = B * (gamma + 1);
   if (stats) {
-    stats->steps = steps;
-    stats->drafted = steps * gamma * B;
+    stats->steps = flags[1];
+    stats->drafted = (int64_t)flags[1] * gamma * B;
     stats->accepted = (int64_t)acc;
   }
+  if (err[0] == DEV_ERR_TIMEOUT) return fail(DORY_ERR_TIMEOUT, "a device-side wait timed out during speculative decoding");
+  if (flags[2] || !flags[0]) return fail(DORY_ERR_STATE, "speculative loop did not finish");
   return DORY_OK;
 }
 
@@ -1139,7 +1299,7 @@ dory_status dory_seq_len(const dory_handle* h, int32_t seq, int32_t* len) {
 dory_status dory_read_state(dory_handle* h, int32_t which, float* dst, int32_t rows, dory_stream stream) {
   if (!h || !dst) return fail(DORY_ERR_INVALID_ARG, "NULL argument");
   if (rows < 1 || rows > h->last_rows) return fail(DORY_ERR_INVALID_ARG, "rows %d outside 1..%d", rows, h->last_rows);
-  const float* src = which == 0 ? h->x : which == 1 ? h->s : which == 2 ? h->h : nullptr;
+  const float* src = which == 0 ? h->x : which == 1 ? h->s : which == 2 ? h->hcur() : nullptr;
   if (!src) return fail(DORY_ERR_INVALID_ARG, "bad state selector");
   CK(cudaMemcpyAsync(dst, src, sizeof(float) * rows * h->c.d_model, cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
   return DORY_OK;
@@ -1248,6 +1408,15 @@ dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value) {
     case DORY_OPT_GEMM_IMPL:
       if (value < 0 || value > 2) return fail(DORY_ERR_INVALID_ARG, "bad GEMM impl");
       h->gemm_impl = (int)value;
+      return DORY_OK;
+    case DORY_OPT_FUSED_OPERANDS:
+      if (value < 0 || value > 16) return fail(DORY_ERR_INVALID_ARG, "fused operand rows must be in 0..16");
+      if (value != h->fuse_rows) {
+        for (auto& g : h->graphs_cache)
+          if (g.exec) cudaGraphExecDestroy(g.exec);
+        h->graphs_cache.clear();
+      }
+      h->fuse_rows = (int)value;
       return DORY_OK;
   }
   return fail(DORY_ERR_INVALID_ARG, "unknown option %d", opt);

@@ -21,10 +21,12 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 #include <unordered_map>
 
+#include "addnorm.cuh"
 #include "gemm_tc.cuh"
 #include "umma.cuh"
 
@@ -95,19 +97,24 @@ __device__ void l2_look_ahead(const PfCtl& pf, int lane) {
 // contiguous bytes of every weight row.
 // GLU: a unit's A operand is two 128-row tiles of one matrix, rows
 // [128 nt, +128) and [glu_rows + 128 nt, +128), with one accumulator each.
-template <int NG, int GN, int KSUB, int BUDGET = 216 * 1024, bool GLU = false>
+// PREP: the token operand is built in shared memory by the epilogue warps
+// (see Prep) in a resident region of BSUB 64-column sub-tiles; stages then
+// carry weights only.
+template <int NG, int GN, int KSUB, int BUDGET = 216 * 1024, bool GLU = false, int PREP = 0, int BSUB = 0>
 struct Tile {
   static constexpr int MT = NG * GN;                   // tokens per unit
   static constexpr int A_SUB = BM * BK * 2;            // 16 KB per sub-tile
   static constexpr int B_SUB = MT * BK * 2;
   static constexpr int NA = GLU ? 2 : 1;               // A tiles per unit
   static constexpr int A_BYTES = NA * KSUB * A_SUB;
-  static constexpr int B_BYTES = KSUB * B_SUB;
+  static constexpr int B_BYTES = PREP ? 0 : KSUB * B_SUB;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int STAGES = BUDGET / STAGE > 12 ? 12 : (BUDGET / STAGE < 1 ? 1 : BUDGET / STAGE);
+  static constexpr int B_RES = PREP ? BSUB * B_SUB : 0;  // resident token operand
+  static constexpr int STAGES = (BUDGET - B_RES) / STAGE > 12 ? 12
+                                : ((BUDGET - B_RES) / STAGE < 1 ? 1 : (BUDGET - B_RES) / STAGE);
   static constexpr int ACC = NA * MT;                  // TMEM columns per accumulator (pair)
   static constexpr int TMEM_COLS = 2 * ACC <= 32 ? 32 : 2 * ACC <= 64 ? 64 : 2 * ACC <= 128 ? 128 : 2 * ACC <= 256 ? 256 : 512;
-  static constexpr int SMEM = STAGES * STAGE + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int SMEM = STAGES * STAGE + B_RES + 1024 /*align*/ + 512 /*barriers*/;
 };
 
 // Units are (n tile, m tile, split).  Split boundaries are placed on groups
@@ -133,12 +140,114 @@ struct UnitMap {
 // bf16 (row stride ldy) from the pair of accumulators, where g and u are the
 // products with weight rows j and glu_rows + j: the SwiGLU of a concatenated
 // [gate; up] matrix, without its fp32 products ever reaching memory.
-template <int NG, int GN, int KSUB, int BUDGET, bool PACK, bool GLU = false>
+// The resident token operand of a PREP GEMM: the first CTA's units' K range
+// as 64-column sub-tiles [lo, hi) (every CTA's units share one range when
+// the host chose this path).
+struct SubRange {
+  int lo, hi;
+};
+
+__device__ __forceinline__ SubRange prep_range(const UnitMap& um, int ksub) {
+  SubRange r{1 << 30, -1};
+  for (int u = blockIdx.x; u < um.units; u += gridDim.x) {
+    int nt, mt, s, kb0, kb1;
+    um.decode(u, nt, mt, s, kb0, kb1);
+    r.lo = min(r.lo, kb0 * ksub);
+    r.hi = max(r.hi, kb1 * ksub);
+  }
+  return r;
+}
+
+__device__ __forceinline__ void bar_epi() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// The operand stage (see Prep), run by the 128 epilogue threads (t = 0..127)
+// into `breg`: sub-tile i of the region holds columns 64 (lo + i) .. + 63 of
+// the MT token rows, 128-byte swizzled K-major (row m's 16-byte chunk c at
+// m * 128 + (c ^ (m % 8)) * 16); rows >= M are zero.  K: the operand's width.
+template <int PREP, int MT>
+__device__ void prep_operand(const Prep& pp, int M, int K, SubRange rg, uint8_t* breg, float* red, int t) {
+  const int nsub = rg.hi - rg.lo, c_lo = rg.lo * BK, c_hi = rg.hi * BK;
+  // rows M..MT-1 of every sub-tile: bytes [M * 128, MT * 128)
+  for (int i = t; i < nsub * (MT - M) * 8; i += 128) {
+    const int sub = i / ((MT - M) * 8), off = i % ((MT - M) * 8);
+    *reinterpret_cast<uint4*>(breg + sub * (MT * 128) + M * 128 + off * 16) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  if constexpr (PREP == kPrepAddNorm) {
+    const int nc = K / 4;
+    for (int m = 0; m < M; ++m) {
+      const float* hr = pp.h_in + (size_t)m * K;
+      const float* yr = pp.y + (size_t)m * pp.ldy;
+      float4 v[AN_MAXC];
+      float ss = 0.f;
+#pragma unroll
+      for (int c = 0; c < AN_MAXC; ++c) {
+        const int j = t + c * AN_THREADS;
+        if (j < nc) {
+          v[c] = an_chunk(hr, yr, pp.S, pp.ps, j);
+          ss = an_squares(ss, v[c]);
+        }
+      }
+      const float inv = an_inv_norm(ss, red, t, [] { bar_epi(); });
+#pragma unroll
+      for (int c = 0; c < AN_MAXC; ++c) {
+        const int j = t + c * AN_THREADS;
+        if (j < nc) {
+          const float4 o = an_scale(v[c], inv);
+          if (blockIdx.x == 0) reinterpret_cast<float4*>(pp.h_out + (size_t)m * K)[j] = o;
+          const int col = 4 * j;
+          if (col >= c_lo && col < c_hi) {
+            const int cc = col - c_lo, sub = cc / BK, ch = (cc % BK) / 8;
+            const __nv_bfloat162 a = __floats2bfloat162_rn(o.x, o.y), b = __floats2bfloat162_rn(o.z, o.w);
+            *reinterpret_cast<uint2*>(breg + sub * (MT * 128) + m * 128 + ((ch ^ (m & 7)) << 4) + (cc % 8) * 2) =
+                make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
+          }
+        }
+      }
+    }
+  } else {
+    // SwiGLU: 16-byte chunks of 8 columns; gate columns j, up columns K + j
+    const int nch = nsub * (BK / 8);
+    for (int m = 0; m < M; ++m) {
+      const float* yr = pp.y + (size_t)m * pp.ldy;
+      for (int i = t; i < nch; i += 128) {
+        const int col = c_lo + 8 * i;
+        float g[8], u[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) g[e] = u[e] = 0.f;
+        for (int s = 0; s < pp.S; ++s) {
+          const float4* gp = reinterpret_cast<const float4*>(yr + s * pp.ps + col);
+          const float4* up = reinterpret_cast<const float4*>(yr + s * pp.ps + K + col);
+          const float4 g0 = __ldcg(gp), g1 = __ldcg(gp + 1), u0 = __ldcg(up), u1 = __ldcg(up + 1);
+          g[0] += g0.x; g[1] += g0.y; g[2] += g0.z; g[3] += g0.w;
+          g[4] += g1.x; g[5] += g1.y; g[6] += g1.z; g[7] += g1.w;
+          u[0] += u0.x; u[1] += u0.y; u[2] += u0.z; u[3] += u0.w;
+          u[4] += u1.x; u[5] += u1.y; u[6] += u1.z; u[7] += u1.w;
+        }
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a0 = g[2 * e] / (1.f + expf(-g[2 * e])) * u[2 * e];
+          const float a1 = g[2 * e + 1] / (1.f + expf(-g[2 * e + 1])) * u[2 * e + 1];
+          const __nv_bfloat162 p = __floats2bfloat162_rn(a0, a1);
+          w[e] = *reinterpret_cast<const uint32_t*>(&p);
+        }
+        const int sub = i / (BK / 8), ch = i % (BK / 8);
+        *reinterpret_cast<uint4*>(breg + sub * (MT * 128) + m * 128 + ((ch ^ (m & 7)) << 4)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  }
+  // generic-proxy writes -> visible to the tensor core's reads
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  bar_epi();
+}
+
+template <int NG, int GN, int KSUB, int BUDGET, bool PACK, bool GLU = false, int PREP = 0, int BSUB = 0>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, float* Y, int ldy,
               size_t part_stride, int M, UnitMap um, int* err, const uint8_t* Apack,
-              int k_tiles, PfCtl pf, bf16* act, int glu_rows) {
-  using TL = Tile<NG, GN, KSUB, BUDGET, GLU>;
+              int k_tiles, PfCtl pf, bf16* act, int glu_rows, Prep pp) {
+  using TL = Tile<NG, GN, KSUB, BUDGET, GLU, PREP, BSUB>;
   constexpr int STAGES = TL::STAGES;
   auto load_a = [&](uint8_t* sa, uint64_t* bar, int nt, int kb, uint64_t pol) {
     if constexpr (PACK) {
@@ -155,13 +264,16 @@ __global__ void __launch_bounds__(192, 1)
   };
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t* full = (uint64_t*)(smem + STAGES * TL::STAGE);
+  uint8_t* breg = smem + STAGES * TL::STAGE;  // PREP: resident token operand
+  uint64_t* full = (uint64_t*)(breg + TL::B_RES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
-  uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
+  uint64_t* b_ready = mma_done + 1;
+  uint32_t* tmem_slot = (uint32_t*)(b_ready + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  float* red = (float*)(tmem_slot + 4);  // 4 floats, 16-byte aligned
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -174,13 +286,14 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&tempty[i], 4);
     }
     mbar_init(mma_done, 1);
+    mbar_init(b_ready, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == 0 && lane == 0) {
     if (!PACK) asm volatile("prefetch.tensormap [%0];" ::"l"(&mapA) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(&mapB) : "memory");
+    if (!PREP) asm volatile("prefetch.tensormap [%0];" ::"l"(&mapB) : "memory");
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -220,12 +333,14 @@ __global__ void __launch_bounds__(192, 1)
         ++npre;
         next();
       }
-      pdl_wait();
-      for (int i = 0; i < npre; ++i)
+      if constexpr (!PREP) {
+        pdl_wait();
+        for (int i = 0; i < npre; ++i)
 #pragma unroll
-        for (int q = 0; q < KSUB; ++q)
-          tma_load_2d(smem + i * TL::STAGE + TL::A_BYTES + q * TL::B_SUB, &mapB, &full[i], (pre_kb[i] * KSUB + q) * BK,
-                      pre_mt[i] * TL::MT, pol_x);
+          for (int q = 0; q < KSUB; ++q)
+            tma_load_2d(smem + i * TL::STAGE + TL::A_BYTES + q * TL::B_SUB, &mapB, &full[i],
+                        (pre_kb[i] * KSUB + q) * BK, pre_mt[i] * TL::MT, pol_x);
+      }
       int stage = npre % STAGES, issued = npre;
       uint32_t phase = npre == STAGES ? 1u : 0u;
       while (u < um.units) {
@@ -234,9 +349,12 @@ __global__ void __launch_bounds__(192, 1)
         uint8_t* sa = smem + stage * TL::STAGE;
         mbar_expect_tx(&full[stage], TL::STAGE);
         load_a(sa, &full[stage], nt, kb, pol_w);
+        if constexpr (!PREP) {
 #pragma unroll
-        for (int q = 0; q < KSUB; ++q)
-          tma_load_2d(sa + TL::A_BYTES + q * TL::B_SUB, &mapB, &full[stage], (kb * KSUB + q) * BK, mt * TL::MT, pol_x);
+          for (int q = 0; q < KSUB; ++q)
+            tma_load_2d(sa + TL::A_BYTES + q * TL::B_SUB, &mapB, &full[stage], (kb * KSUB + q) * BK, mt * TL::MT,
+                        pol_x);
+        }
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1;
@@ -267,6 +385,12 @@ __global__ void __launch_bounds__(192, 1)
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
+      int sub_lo = 0;
+      if constexpr (PREP != 0) {
+        sub_lo = prep_range(um, KSUB).lo;
+        ok = mbar_wait(b_ready, 0, abort_flag, err) && !*abort_flag;
+        tc_fence_after();
+      }
       for (int u = blockIdx.x; u < um.units && ok; u += gridDim.x) {
         int nt, mt, s, kb0, kb1;
         um.decode(u, nt, mt, s, kb0, kb1);
@@ -283,7 +407,9 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int q = 0; q < KSUB; ++q) {
             const uint64_t adesc = sw128_desc(sa + q * TL::A_SUB);
-            const uint64_t bdesc = sw128_desc(sa + TL::A_BYTES + q * TL::B_SUB);
+            const uint64_t bdesc =
+                PREP ? sw128_desc(smem_u32(breg) + (uint32_t)((kb * KSUB + q - sub_lo) * TL::B_SUB))
+                     : sw128_desc(sa + TL::A_BYTES + q * TL::B_SUB);
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk) {
 #pragma unroll
@@ -318,6 +444,20 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     // ---------------- epilogue: warps 2..5 own TMEM lanes 32*(warp%4) ..
     pdl_wait();
+    if constexpr (PREP != 0) {
+      const int t = threadIdx.x - 64;
+      const SubRange rg = prep_range(um, KSUB);
+      if (rg.hi - rg.lo > BSUB || rg.hi <= rg.lo) {
+        // the host sizes the region for every CTA; this cannot happen
+        if (t == 0) {
+          set_error(err, DEV_ERR_RANGE);
+          *abort_flag = 1;
+        }
+      } else {
+        prep_operand<PREP, TL::MT>(pp, M, k_tiles * BK, rg, breg, red, t);
+      }
+      if (t == 0) mbar_arrive(b_ready);
+    }
     const int lane_base = 32 * (warp & 3);
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -436,23 +576,27 @@ int sm_count() {
   return n;
 }
 
-template <int NG, int GN, int KSUB, int BUDGET = kDecodeBudget, bool PACK = false, bool GLU = false>
+template <int NG, int GN, int KSUB, int BUDGET = kDecodeBudget, bool PACK = false, bool GLU = false, int PREP = 0,
+          int BSUB = 0>
 cudaError_t run(const CUtensorMap& ma, const bf16* X, int ldx, int M, int K, float* Y, int ldy, size_t ps,
                 UnitMap um, int* err, cudaStream_t st, const void* Apack = nullptr,
-                const PfCtl& pf = PfCtl{}, bf16* act = nullptr, int glu_rows = 0) {
-  using TL = Tile<NG, GN, KSUB, BUDGET, GLU>;
+                const PfCtl& pf = PfCtl{}, bf16* act = nullptr, int glu_rows = 0, const Prep& pp = Prep{}) {
+  using TL = Tile<NG, GN, KSUB, BUDGET, GLU, PREP, BSUB>;
+  auto kern = k_gemm_tc<NG, GN, KSUB, BUDGET, PACK, GLU, PREP, BSUB>;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<NG, GN, KSUB, BUDGET, PACK, GLU>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, TL::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TL::SMEM);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   CUtensorMap mb;
-  if (!make_map(&mb, X, M, K, ldx, TL::MT)) return cudaErrorInvalidValue;
+  if (PREP)
+    memset(&mb, 0, sizeof mb);  // the token operand is built in shared memory
+  else if (!make_map(&mb, X, M, K, ldx, TL::MT))
+    return cudaErrorInvalidValue;
   int grid = um.units < sm_count() ? um.units : sm_count();
-  return launch(k_gemm_tc<NG, GN, KSUB, BUDGET, PACK, GLU>, dim3(grid), dim3(192), TL::SMEM, st, ma, mb, Y, ldy,
-                ps, M, um, err, (const uint8_t*)Apack, K / BK, pf, act, glu_rows);
+  return launch(kern, dim3(grid), dim3(192), TL::SMEM, st, ma, mb, Y, ldy, ps, M, um, err, (const uint8_t*)Apack,
+                K / BK, pf, act, glu_rows, pp);
 }
 
 // Split factor for the decode tiles: chosen from (N, K, batch) only, never
@@ -522,13 +666,80 @@ cudaError_t launch_pack_weight(const bf16* W, void* dst, int N, int K, cudaStrea
   return cudaGetLastError();
 }
 
+// Largest 64-column sub-tile range one CTA's units span (the resident token
+// operand of an operand-stage GEMM), for a grid of min(units, SMs) CTAs.
+static int prep_span(const UnitMap& um, int ksub) {
+  const int grid = um.units < sm_count() ? um.units : sm_count();
+  int span = 0;
+  for (int b = 0; b < grid; ++b) {
+    int lo = 1 << 30, hi = -1;
+    for (int u = b; u < um.units; u += grid) {
+      const int s = u % um.S;
+      lo = std::min(lo, (s * um.KBg / um.S) * um.gran * ksub);
+      hi = std::max(hi, ((s + 1) * um.KBg / um.S) * um.gran * ksub);
+    }
+    span = std::max(span, hi - lo);
+  }
+  return span;
+}
+
+// Decode GEMM with an operand stage: 16-token tiles, 2 sub-tiles per stage,
+// the resident operand region sized for the widest CTA range.
+static cudaError_t run_prep(const CUtensorMap& ma, int M, int K, float* Y, int ldy, size_t ps, UnitMap um, int* err,
+                     cudaStream_t st, const PfCtl& pf, const Prep& pp) {
+  constexpr int KS = 2;
+  const int span = prep_span(um, KS);
+#define DORY_PREP(P, B)                                                                                       \
+  if (pp.mode == P && span <= B)                                                                             \
+  return run<1, 16, KS, kDecodeBudget, false, false, P, B>(ma, nullptr, 0, M, K, Y, ldy, ps, um, err, st, nullptr, \
+                                                           pf, nullptr, 0, pp)
+  DORY_PREP(kPrepAddNorm, 8);
+  DORY_PREP(kPrepAddNorm, 24);
+  DORY_PREP(kPrepAddNorm, 40);
+  DORY_PREP(kPrepSwiglu, 8);
+  DORY_PREP(kPrepSwiglu, 24);
+  DORY_PREP(kPrepSwiglu, 40);
+#undef DORY_PREP
+  return cudaErrorNotSupported;
+}
+
+bool gemm_tc_prep_ok(int M, int N, int K, int batch, const Prep& p) {
+  if (p.mode == kPrepNone || M < 1 || M > 16 || N % BM || K % (4 * BK) || K > 4 * AN_MAXC * AN_THREADS ||
+      p.S < 1 || p.S > AN_MAXS || p.ldy % 4 || p.ps % 4 || ((uintptr_t)p.y & 15))
+    return false;
+  if (p.mode == kPrepAddNorm &&
+      (p.h_in == p.h_out || ((uintptr_t)p.h_in & 15) || ((uintptr_t)p.h_out & 15) || p.ldy < K))
+    return false;
+  if (p.mode == kPrepSwiglu && p.ldy < 2 * K) return false;
+  UnitMap um;
+  um.n_tiles = N / BM;
+  um.KBg = K / (4 * BK);
+  um.gran = 2;
+  um.S = choose_split(N, K, batch, um.KBg);
+  if (um.S > um.KBg) return false;
+  um.m_tiles = 1;
+  um.units = um.n_tiles * um.S;
+  return prep_span(um, 2) <= 40;
+}
+
 cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf16* W, float* Y, int ldy,
                            size_t part_rows, int* err, int batch, bool invariant, int* S_out, size_t* ps_out,
-                           cudaStream_t st, int variant, bool packed, const PfCtl* pf) {
+                           cudaStream_t st, int variant, bool packed, const PfCtl* pf, const Prep* prep) {
   *S_out = 1;
   *ps_out = 0;
-  if (M <= 0 || N % BM || K % BK || ldx % 8 || (size_t)M > part_rows || ((uintptr_t)X & 15) || ((uintptr_t)W & 15))
+  const bool staged = prep && prep->mode != kPrepNone;
+  if (staged) {
+    // the operand stage: decode tiles of one 16-token group, weights by TMA
+    if (!invariant || packed || variant != 0 || M > 16 || N % BM || K % (4 * BK) || K > 4 * AN_MAXC * AN_THREADS ||
+        (size_t)M > part_rows || ((uintptr_t)W & 15) || prep->S < 1 || prep->S > AN_MAXS || prep->ldy % 4 ||
+        prep->ps % 4 || ((uintptr_t)prep->y & 15) ||
+        (prep->mode == kPrepAddNorm && (prep->h_in == prep->h_out || ((uintptr_t)prep->h_in & 15) ||
+                                        ((uintptr_t)prep->h_out & 15))))
+      return cudaErrorNotSupported;
+  } else if (M <= 0 || N % BM || K % BK || ldx % 8 || (size_t)M > part_rows || ((uintptr_t)X & 15) ||
+             ((uintptr_t)W & 15)) {
     return cudaErrorNotSupported;
+  }
   CUtensorMap ma;
   if (packed)
     memset(&ma, 0, sizeof ma);
@@ -544,7 +755,7 @@ cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf
     const bool g256 = K % (4 * BK) == 0;  // split on 256-column groups
     const int ksub = (variant == 1 || !g256) ? 1 : (NG >= 8 ? 1 : (NG >= 2 ? 2 : kDecodeKsub));
     um.KBg = g256 ? K / (4 * BK) : K / BK;
-    um.gran = g256 ? 4 / ksub : 1;
+    um.gran = g256 ? 4 / (staged ? 2 : ksub) : 1;
     const int S = choose_split(N, K, batch, um.KBg);
     if (S > um.KBg) return cudaErrorNotSupported;
     const size_t ps = part_rows * (size_t)ldy;
@@ -552,9 +763,17 @@ cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf
     const int MT = 16 * NG;
     um.m_tiles = (M + MT - 1) / MT;
     um.units = um.n_tiles * um.m_tiles * S;
+    const PfCtl pfc = pf ? *pf : PfCtl{};
+    if (staged) {
+      const cudaError_t e = run_prep(ma, M, K, Y, ldy, ps, um, err, st, pfc, *prep);
+      if (e == cudaSuccess) {
+        *S_out = S;
+        *ps_out = ps;
+      }
+      return e;
+    }
     *S_out = S;
     *ps_out = ps;
-    const PfCtl pfc = pf ? *pf : PfCtl{};
 #define DORY_RUN(NGV, KS)                                                                                 \
   return packed ? run<NGV, 16, KS, kDecodeBudget, true>(ma, X, ldx, M, K, Y, ldy, ps, um, err, st, W, pfc) \
                 : run<NGV, 16, KS>(ma, X, ldx, M, K, Y, ldy, ps, um, err, st, nullptr, pfc)

@@ -28,6 +28,27 @@ struct PfCtl {
   unsigned long long lo = 0, hi = 0;
 };
 
+// Operand stage of a decode GEMM (M <= 16 rows).  Instead of loading X by
+// TMA, the four epilogue warps build the bf16 operand in shared memory from
+// the previous kernel's fp32 outputs, so the elementwise step between two
+// GEMMs costs no launch of its own:
+//   kPrepAddNorm: X = N(h_in + sum_{s<S} y_s) (rows of d = K floats, the
+//                 arithmetic of addnorm.cuh); the first CTA also writes the
+//                 fp32 result to h_out (a buffer other than h_in);
+//   kPrepSwiglu:  X[m, j] = silu(sum_s y_s[m, j]) * sum_s y_s[m, K + j], the
+//                 SwiGLU of a split gate-up product (rows of ldy = 2K floats).
+// y_s = y + s * ps.  X and ldx are unused.
+enum : int { kPrepNone = 0, kPrepAddNorm = 1, kPrepSwiglu = 2 };
+struct Prep {
+  int mode = kPrepNone;
+  const float* h_in = nullptr;
+  float* h_out = nullptr;
+  const float* y = nullptr;
+  int S = 1;
+  size_t ps = 0;
+  int ldy = 0;
+};
+
 // Y = X . W^T for X [M, K] (row stride ldx) and W [N, K], both bf16, fp32
 // accumulation.  Writes S partial products to Y + s * (*part_stride)
 // (row stride ldy); the consumer adds them in order s = 0..S-1.
@@ -38,10 +59,15 @@ struct PfCtl {
 // handle (N % 128, K % 64, unaligned pointers).  variant 1 forces one
 // 64-column sub-tile per pipeline stage (for comparisons).
 // packed: W is in the packed tile layout below.  pf: L2 look-ahead (decode
-// tiles only; ignored for prefill tiles).
+// tiles only; ignored for prefill tiles).  prep (decode tiles, M <= 16): the
+// operand stage above; cudaErrorNotSupported when this shape cannot take it
+// (the caller then runs the elementwise step and a plain GEMM).  A GEMM with
+// an operand stage computes the same bits as the plain one on the operand
+// the standalone kernels would have written.
 cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf16* W, float* Y, int ldy,
                            size_t part_rows, int* err, int batch, bool invariant, int* S, size_t* part_stride,
-                           cudaStream_t st, int variant = 0, bool packed = false, const PfCtl* pf = nullptr);
+                           cudaStream_t st, int variant = 0, bool packed = false, const PfCtl* pf = nullptr,
+                           const Prep* prep = nullptr);
 
 // act[m, j] = silu(g) * u (bf16, row stride dff) with g = X[m] . Wgu[j] and
 // u = X[m] . Wgu[dff + j] for the concatenated [gate; up] weight Wgu
@@ -49,6 +75,10 @@ cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf
 // tensor-core GEMM (fp32 accumulation, no split).  dff % 128 == 0.
 cudaError_t launch_gemm_glu(int M, int dff, int K, const bf16* X, int ldx, const bf16* Wgu, bf16* act,
                             int* err, cudaStream_t st);
+
+// Whether a decode GEMM of this shape (M rows, `batch` sequences) can take
+// the operand stage `p` (the checks launch_gemm_tc makes, without launching).
+bool gemm_tc_prep_ok(int M, int N, int K, int batch, const Prep& p);
 
 // Repack a row-major [N, K] bf16 weight (N % 128 == 0, K % 64 == 0) into the
 // packed tile layout the tensor-core GEMM streams with bulk copies: 128 x 64

@@ -47,11 +47,12 @@ cudaError_t launch_advance_ragged(int n_seq, const int* seq_ids, const int* cu, 
 template <typename T>
 cudaError_t launch_embed(int M, int d, int vocab, const int* tokens, const T* E, float* h, T* hop, float* x,
                          int* err, cudaStream_t st);
-// h <- N(h + sum_{s<S} y[s]) ; hop <- (T)h ; copy_out (if not NULL) <- h.
-// y[s] = y + s*part_stride, rows of ldy.  S <= kMaxSplitK.
+// h_out <- N(h_in + sum_{s<S} y[s]) ; hop <- (T)h_out ; copy_out (if not NULL)
+// <- h_out (h_out may equal h_in).  y[s] = y + s*part_stride, rows of ldy.
+// S <= kMaxSplitK; d, ldy and part_stride multiples of 4.
 template <typename T>
-cudaError_t launch_addnorm(int M, int d, float* h, const float* y, int S, size_t part_stride, int ldy,
-                           T* hop, float* copy_out, cudaStream_t st);
+cudaError_t launch_addnorm(int M, int d, const float* h_in, float* h_out, const float* y, int S,
+                           size_t part_stride, int ldy, T* hop, float* copy_out, cudaStream_t st);
 // Loop boundary.  s_src: 0 -> s = x ; 1 -> s = N(h) ; 2 -> s = s_in.
 // If make_u: out = N(s + x), else out = s.  h <- out, hop <- (T)out.
 // If s_save: s_save <- s.  stash rows: when stash_x/stash_s are given, row r
@@ -110,13 +111,27 @@ cudaError_t launch_sample(int R, int V, const float* logits, uint32_t* qbuf, con
                           const int* pos, int pos_add, float temperature, float top_p, unsigned long long seed,
                           int* out, cudaStream_t st);
 
+// Caller buffers of a speculative decoding call (device copy, so a recorded
+// step reads each call's buffers).
+struct SpecIo {
+  int* out;      // [B, max_new] accepted tokens
+  int* out_len;  // [B]
+  int max_new;
+  int pad;
+};
+
 // Speculative acceptance for B sequences.  drafts[i * dstride + b] = d_{i+1},
-// vtok [B, gamma+1] verifier choices.  Appends accepted tokens to out
-// [B, max_new] at out_len, sets seq_len = p0 + n + 1 and pending = a_n for
-// unfinished sequences; adds n to *accepted (device int64).
+// vtok [B, gamma+1] verifier choices.  Appends accepted tokens to io->out
+// [B, max_new] at io->out_len, sets seq_len = p0 + n + 1 and pending = a_n
+// for unfinished sequences; adds n to *accepted (device int64).  flags[0] <-
+// every sequence finished; flags[1] counts steps; flags[2] <- 1 once more
+// steps ran than max_new (which always suffice).  With use_cond the kernel
+// sets graph conditional `cond` to 1 while another step is needed (no
+// sequence finished everything, no step bound hit, error word err clear).
 cudaError_t launch_spec_accept(int B, int gamma, int dstride, const int* seq_ids, int* seq_len,
-                               const int* drafts, const int* vtok, int* pending, int* out, int* out_len,
-                               int max_new, unsigned long long* accepted, int* all_done, cudaStream_t st);
+                               const int* drafts, const int* vtok, int* pending, const SpecIo* io,
+                               unsigned long long* accepted, int* flags, const int* err, unsigned long long cond,
+                               bool use_cond, cudaStream_t st);
 
 cudaError_t launch_fill_i32(int n, int* p, int v, cudaStream_t st);
 

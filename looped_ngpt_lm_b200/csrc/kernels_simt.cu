@@ -9,13 +9,13 @@
 // a row computes bit-identical results alone or inside a larger chunk.
 #include <float.h>
 
+#include "addnorm.cuh"
 #include "common.cuh"
 #include "kernels.cuh"
 #include "gemm_tc.cuh"
 
 namespace dory {
 
-constexpr int kMaxSplit = kMaxSplitK;
 
 // ------------------------------------------------------------------ planning
 __global__ void k_plan_uniform(int n_rows, int rps, int pos_offset, const int* seq_ids, const int* seq_len,
@@ -147,56 +147,50 @@ cudaError_t launch_embed(int M, int d, int vocab, const int* tokens, const T* E,
 }
 
 // ------------------------------------------------------------------ add + norm
-// One 512-thread block per row; thread t owns elements t, t+512, ...; the S
-// partial loads are independent (unrolled, predicated) so they overlap.
-constexpr int AN_THREADS = 512;
-constexpr int AN_CPT = 8;  // d <= 4096
+// One 128-thread block per row, 16-byte loads (the arithmetic of addnorm.cuh,
+// shared with the decode GEMM's operand stage).
 template <typename T>
-__global__ void __launch_bounds__(AN_THREADS) k_addnorm(int d, float* h, const float* __restrict__ y, int S,
-                                                        size_t ps, int ldy, T* hop, float* copy_out) {
+__global__ void __launch_bounds__(AN_THREADS) k_addnorm(int d, const float* h_in, float* h_out,
+                                                        const float* __restrict__ y, int S, size_t ps, int ldy,
+                                                        T* hop, float* copy_out) {
   pdl_wait();
   pdl_trigger();
-  __shared__ float red[33];
-  const int r = blockIdx.x;
-  float* hr = h + (size_t)r * d;
+  __shared__ float red[4];
+  const int r = blockIdx.x, t = threadIdx.x, nc = d / 4;
+  const float* hr = h_in + (size_t)r * d;
   const float* yr = y + (size_t)r * ldy;
-  float v[AN_CPT];
+  float4 v[AN_MAXC];
   float ss = 0.f;
 #pragma unroll
-  for (int c = 0; c < AN_CPT; ++c) {
-    const int i = threadIdx.x + c * AN_THREADS;
-    v[c] = 0.f;
-    if (i < d) {
-      float p[kMaxSplit];
-#pragma unroll
-      for (int s = 0; s < kMaxSplit; ++s) p[s] = s < S ? __ldcg(yr + s * ps + i) : 0.f;
-      float acc = 0.f;
-#pragma unroll
-      for (int s = 0; s < kMaxSplit; ++s)
-        if (s < S) acc += p[s];
-      v[c] = hr[i] + acc;
-      ss += v[c] * v[c];
+  for (int c = 0; c < AN_MAXC; ++c) {
+    const int j = t + c * AN_THREADS;
+    if (j < nc) {
+      v[c] = an_chunk(hr, yr, S, ps, j);
+      ss = an_squares(ss, v[c]);
     }
   }
-  ss = block_sum(ss, red);
-  const float inv = 1.f / fmaxf(sqrtf(ss), 1e-12f);
+  const float inv = an_inv_norm(ss, red, t, [] { __syncthreads(); });
 #pragma unroll
-  for (int c = 0; c < AN_CPT; ++c) {
-    const int i = threadIdx.x + c * AN_THREADS;
-    if (i < d) {
-      const float o = v[c] * inv;
-      hr[i] = o;
-      hop[(size_t)r * d + i] = from_f<T>(o);
-      if (copy_out) copy_out[(size_t)r * d + i] = o;
+  for (int c = 0; c < AN_MAXC; ++c) {
+    const int j = t + c * AN_THREADS;
+    if (j < nc) {
+      const float4 o = an_scale(v[c], inv);
+      reinterpret_cast<float4*>(h_out + (size_t)r * d)[j] = o;
+      if (copy_out) reinterpret_cast<float4*>(copy_out + (size_t)r * d)[j] = o;
+      T* dst = hop + (size_t)r * d + 4 * j;
+      dst[0] = from_f<T>(o.x);
+      dst[1] = from_f<T>(o.y);
+      dst[2] = from_f<T>(o.z);
+      dst[3] = from_f<T>(o.w);
     }
   }
 }
 
 template <typename T>
-cudaError_t launch_addnorm(int M, int d, float* h, const float* y, int S, size_t ps, int ldy, T* hop,
-                           float* copy_out, cudaStream_t st) {
-  if (d > AN_CPT * AN_THREADS || S > kMaxSplit) return cudaErrorInvalidValue;
-  return launch(k_addnorm<T>, dim3(M), dim3(AN_THREADS), 0, st, d, h, y, S, ps, ldy, hop, copy_out);
+cudaError_t launch_addnorm(int M, int d, const float* h_in, float* h_out, const float* y, int S, size_t ps, int ldy,
+                           T* hop, float* copy_out, cudaStream_t st) {
+  if (d % 4 || d > 4 * AN_MAXC * AN_THREADS || S > AN_MAXS || ldy % 4 || ps % 4) return cudaErrorInvalidValue;
+  return launch(k_addnorm<T>, dim3(M), dim3(AN_THREADS), 0, st, d, h_in, h_out, y, S, ps, ldy, hop, copy_out);
 }
 
 // ------------------------------------------------------------------ loop boundary
@@ -743,13 +737,16 @@ cudaError_t launch_argmax(int R, int V, const float* logits, int* out, cudaStrea
 
 // ------------------------------------------------------------------ speculative acceptance
 __global__ void k_spec_accept(int B, int gamma, int dstride, const int* seq_ids, int* seq_len, const int* drafts,
-                              const int* vtok, int* pending, int* out, int* out_len, int max_new,
-                              unsigned long long* accepted, int* all_done) {
+                              const int* vtok, int* pending, const SpecIo* io, unsigned long long* accepted,
+                              int* flags, const int* err, cudaGraphConditionalHandle cond, int use_cond) {
   pdl_wait();
   pdl_trigger();
   __shared__ int n_unfinished;
   if (threadIdx.x == 0) n_unfinished = 0;
   __syncthreads();
+  int* out = io->out;
+  int* out_len = io->out_len;
+  const int max_new = io->max_new;
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
     int ol = out_len[b];
     if (ol >= max_new) continue;  // finished: cache and length stay frozen
@@ -765,14 +762,24 @@ __global__ void k_spec_accept(int B, int gamma, int dstride, const int* seq_ids,
     if (ol < max_new) atomicAdd(&n_unfinished, 1);
   }
   __syncthreads();
-  if (threadIdx.x == 0) *all_done = (n_unfinished == 0);
+  if (threadIdx.x == 0) {
+    // every step gives each unfinished sequence at least one token, so
+    // max_new steps finish every sequence; one more means something is wrong
+    const int done = n_unfinished == 0, steps = flags[1] + 1;
+    const int overrun = !done && steps > max_new;
+    flags[0] = done;
+    flags[1] = steps;
+    if (overrun) flags[2] = 1;
+    if (use_cond) cudaGraphSetConditional(cond, (done || overrun || *(volatile const int*)err != 0) ? 0u : 1u);
+  }
 }
 
 cudaError_t launch_spec_accept(int B, int gamma, int dstride, const int* seq_ids, int* seq_len, const int* drafts,
-                               const int* vtok, int* pending, int* out, int* out_len, int max_new,
-                               unsigned long long* accepted, int* all_done, cudaStream_t st) {
-  launch(k_spec_accept, 1, 256, 0, st, B, gamma, dstride, seq_ids, seq_len, drafts, vtok, pending, out, out_len, max_new,
-                                   accepted, all_done);
+                               const int* vtok, int* pending, const SpecIo* io, unsigned long long* accepted,
+                               int* flags, const int* err, unsigned long long cond, bool use_cond,
+                               cudaStream_t st) {
+  launch(k_spec_accept, 1, 256, 0, st, B, gamma, dstride, seq_ids, seq_len, drafts, vtok, pending, io, accepted,
+         flags, err, (cudaGraphConditionalHandle)cond, use_cond ? 1 : 0);
   return cudaGetLastError();
 }
 
@@ -780,8 +787,8 @@ cudaError_t launch_spec_accept(int B, int gamma, int dstride, const int* seq_ids
 #define DORY_INST(T)                                                                                              \
   template cudaError_t launch_embed<T>(int, int, int, const int*, const T*, float*, T*, float*, int*,            \
                                        cudaStream_t);                                                             \
-  template cudaError_t launch_addnorm<T>(int, int, float*, const float*, int, size_t, int, T*, float*,            \
-                                         cudaStream_t);                                                           \
+  template cudaError_t launch_addnorm<T>(int, int, const float*, float*, const float*, int, size_t, int, T*,      \
+                                         float*, cudaStream_t);                                                   \
   template cudaError_t launch_reinject<T>(int, int, float*, const float*, int, const float*, bool, T*, float*,    \
                                           int, int, int, cudaStream_t);                                           \
   template cudaError_t launch_qkv_post<T>(int, int, int, int, const float*, int, size_t, float*, T*, T*, bool,    \

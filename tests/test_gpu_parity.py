@@ -258,3 +258,38 @@ def test_l2_look_ahead_changes_no_bits(tiny_bf16, prompt, lead_mib):
     h.set_option(dory.OPT_L2_LOOKAHEAD, 8 << 20)
     assert got[0] == ref[0] and got2[0] == ref[0]
     assert torch.equal(got[1], ref[1]) and torch.equal(got2[1], ref[1])
+
+
+@pytest.mark.parametrize("rows", [1, 3])
+def test_fused_operand_stages_change_no_bits(tiny_bf16, prompt, rows):
+    """The add + norm and SwiGLU steps folded into the next GEMM's operand
+    stage compute what the standalone kernels compute: tokens, logits and
+    the final state are bit-identical with the folding off, for one and for
+    several rows, eager and graph-replayed."""
+    _, _, h = tiny_bf16
+    V = synth.TINY_BF16.vocab
+    ids = list(range(rows))
+
+    def run(graphs):
+        h.set_option(dory.OPT_CUDA_GRAPHS, graphs)
+        h.reset()
+        tok = torch.tensor(np.concatenate([prompt[:30 + 3 * i] for i in ids]), dtype=torch.int32, device="cuda")
+        nxt = h.prefill(ids, tok, [30 + 3 * i for i in ids], 2, dory.LAST_LOOP)
+        toks = [nxt.cpu().numpy().copy()]
+        lg = torch.empty((rows, V), device="cuda")
+        for i in range(6):
+            nxt = h.decode_step(ids, nxt, 2, dory.LAST_LOOP, logits=lg if i == 0 else None)
+            toks.append(nxt.cpu().numpy().copy())
+        return np.stack(toks), lg.cpu(), h.read_state("s", rows).cpu(), h.read_state("out", rows).cpu()
+
+    h.set_option(dory.OPT_FUSED_OPERANDS, 0)
+    ref = run(0)
+    h.set_option(dory.OPT_FUSED_OPERANDS, 16)
+    got = run(0)
+    got_graph = run(1)
+    h.set_option(dory.OPT_FUSED_OPERANDS, 4)
+    h.set_option(dory.OPT_CUDA_GRAPHS, 1)
+    for g in (got, got_graph):
+        assert np.array_equal(g[0], ref[0])
+        assert torch.equal(g[2], ref[2]) and torch.equal(g[3], ref[3])
+    assert torch.equal(got[1], ref[1])
