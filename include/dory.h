@@ -99,6 +99,18 @@ typedef struct {
   int32_t k_max;                  /* largest loop count a call may use (1..4) */
   int32_t gamma_max;              /* largest speculative draft length (0 disables) */
   int32_t max_chunk;              /* most new tokens in one forward, summed over the batch */
+  /* Paged cache of the full-attention layers (the sliding-window layers keep
+   * a ring of swa_window + slack positions per sequence).  kv_page = 0: each
+   * sequence slot reserves max_seq positions in every full-attention layer.
+   * kv_page > 0 (a power of two in 16..4096): positions come in pages of
+   * kv_page, drawn on demand from a pool of kv_pages pages per layer and
+   * cache slot (0: enough for every slot to reach max_seq) and returned by
+   * dory_reset, so a few long sequences and many short ones share one pool
+   * (256K-token contexts without max_batch x 256K reservations).  A call
+   * that needs more pages than are free fails with DORY_ERR_CAPACITY before
+   * any work is queued. */
+  int32_t kv_page;
+  int32_t kv_pages;
 } dory_config;
 
 /* Device weight pointers, BORROWED (must outlive the handle).  All matrices
@@ -452,7 +464,11 @@ enum {
    * split gate-up product run inside the next projection GEMM, whose
    * epilogue warps build its operand in shared memory, instead of as kernels
    * of their own.  Same arithmetic, so the same bits, either way. */
-  DORY_OPT_FUSED_OPERANDS = 9
+  DORY_OPT_FUSED_OPERANDS = 9,
+  /* bf16 decode steps: bytes of upcoming weights each decode attention
+   * launch prefetches into L2 before waiting for its queries (default 0:
+   * none).  Changes only when HBM reads happen, never what is computed. */
+  DORY_OPT_ATTN_LOOKAHEAD = 10
 };
 dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value);
 

@@ -30,6 +30,7 @@ OPT_ATTN_CLUSTER = 6
 OPT_L2_LOOKAHEAD = 7
 OPT_MX_GEMV = 8
 OPT_FUSED_OPERANDS = 9
+OPT_ATTN_LOOKAHEAD = 10
 
 STATUS = {0: "DORY_OK", 1: "DORY_ERR_INVALID_ARG", 2: "DORY_ERR_CAPACITY", 3: "DORY_ERR_STATE",
           4: "DORY_ERR_WORKSPACE", 5: "DORY_ERR_CUDA", 6: "DORY_ERR_TIMEOUT", 7: "DORY_ERR_UNSUPPORTED"}
@@ -54,7 +55,7 @@ class Config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "d_model", "vocab", "n_heads", "head_dim", "n_kv_heads", "d_ff", "n_in", "n_rec", "n_out",
         "swa_window", "full_every", "full_phase", "dtype", "max_batch", "max_seq", "k_max", "gamma_max",
-        "max_chunk")]
+        "max_chunk", "kv_page", "kv_pages")]
 
 
 class Weights(ctypes.Structure):
@@ -135,12 +136,14 @@ def _check(status: int) -> None:
         raise DoryError(status, lib.dory_last_error().decode())
 
 
-def make_config(shape, max_batch=1, max_seq=256, k_max=4, gamma_max=4, max_chunk=None) -> Config:
-    """C config for a synth.Shape plus capacity."""
+def make_config(shape, max_batch=1, max_seq=256, k_max=4, gamma_max=4, max_chunk=None, kv_page=0,
+                kv_pages=0) -> Config:
+    """C config for a synth.Shape plus capacity (kv_page > 0: paged
+    full-attention cache with a pool of kv_pages pages)."""
     return Config(shape.d_model, shape.vocab, shape.n_heads, shape.head_dim, shape.n_kv_heads, shape.d_ff,
                   shape.n_in, shape.n_rec, shape.n_out, shape.swa_window, shape.full_every, shape.full_phase,
                   BF16 if shape.dtype == "bf16" else F32, max_batch, max_seq, k_max, gamma_max,
-                  max_chunk if max_chunk is not None else max_seq)
+                  max_chunk if max_chunk is not None else max_seq, kv_page, kv_pages)
 
 
 def _ptr(t) -> int:

@@ -96,14 +96,14 @@ __global__ void __launch_bounds__(256) k_attn_decode(int KV, const float* __rest
   const int klo = max(lo, kb), khi = min(pos, kb + DEC_BK - 1);
   const int H = KV * G, qd = H * HD, kvd = KV * HD, ld = qd + 2 * kvd;
   const int tid = threadIdx.x;
-  T* Kc = (T*)kv.K + ((size_t)seq * KV + g) * kv.cap * HD;
-  T* Vc = (T*)kv.V + ((size_t)seq * KV + g) * kv.cap * HD;
+  T* Kc = (T*)kv.K;
+  T* Vc = (T*)kv.V;
 
   // 1. cached keys -> shared memory (all copies in flight), chunk keys rebuilt
   const int cache_hi = min(khi, p0 - 1);  // last cached key of this block
   for (int i = tid; i < (cache_hi - klo + 1) * CH; i += blockDim.x) {
     const int jj = i / CH, c = i % CH;
-    const size_t src = (size_t)((klo + jj) % kv.cap) * HD;
+    const size_t src = kv_row(kv, seq, KV, g, klo + jj) * HD;
     cp16(saddr(&sm.k[klo - kb + jj][0]) + c * 16, (const uint8_t*)(Kc + src) + c * 16);
     cp16(saddr(&sm.v[klo - kb + jj][0]) + c * 16, (const uint8_t*)(Vc + src) + c * 16);
   }
@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(256) k_attn_decode(int KV, const float* __rest
     sm.q[h][d] = sum_splits(qkv + (size_t)r * ld + (g * G + h) * HD + d, S, ps) * scale_log2;
   }
   if (khi == pos) {
-    const size_t slot = (size_t)(pos % kv.cap) * HD;
+    const size_t slot = kv_row(kv, seq, KV, g, pos) * HD;
     for (int i = tid; i < 2 * HD; i += blockDim.x) {
       const int d = i % HD;
       const bool is_v = i >= HD;
@@ -318,8 +318,8 @@ __global__ void __launch_bounds__(256) k_attn_decode_cl(int KV, const float* __r
   const int klo = lo + rank * per, khi = row_ok ? min(pos, klo + per - 1) : klo - 1;  // empty when klo > khi
   const int H = KV * G, qd = H * HD, kvd = KV * HD, ld = qd + 2 * kvd;
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, sg = lane >> 3, dl = lane & 7;
-  T* Kc = (T*)kv.K + ((size_t)seq * KV + g) * kv.cap * HD;
-  T* Vc = (T*)kv.V + ((size_t)seq * KV + g) * kv.cap * HD;
+  T* Kc = (T*)kv.K;
+  T* Vc = (T*)kv.V;
 
   if (row_ok) {
     for (int i = tid; i < G * HD; i += blockDim.x) {
@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(256) k_attn_decode_cl(int KV, const float* __r
       sm.q[h][d] = sum_splits(qkv + (size_t)r * ld + (g * G + h) * HD + d, S, ps) * scale_log2;
     }
     if (klo <= pos && pos <= khi) {  // this block holds the row's own key
-      const size_t slot = (size_t)(pos % kv.cap) * HD;
+      const size_t slot = kv_row(kv, seq, KV, g, pos) * HD;
       for (int i = tid; i < 2 * HD; i += blockDim.x) {
         const int d = i % HD;
         const bool is_v = i >= HD;
@@ -354,7 +354,7 @@ __global__ void __launch_bounds__(256) k_attn_decode_cl(int KV, const float* __r
     const int cache_hi = min(c1, p0 - 1);
     for (int i = tid; i < (cache_hi - c0 + 1) * CH; i += blockDim.x) {
       const int jj = i / CH, c = i % CH;
-      const size_t src = (size_t)((c0 + jj) % kv.cap) * HD;
+      const size_t src = kv_row(kv, seq, KV, g, c0 + jj) * HD;
       cp16(saddr(&sm.k[jj][0]) + c * 16, (const uint8_t*)(Kc + src) + c * 16);
       cp16(saddr(&sm.v[jj][0]) + c * 16, (const uint8_t*)(Vc + src) + c * 16);
     }
@@ -529,7 +529,7 @@ inline int decode_cluster_size(int batch, int KV) {
 template <int HD, int G, int CS>
 __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __restrict__ qkv, int S, size_t ps,
                                                         KVView kv, RowMeta m, bf16* __restrict__ out,
-                                                        float scale_log2) {
+                                                        float scale_log2, PfCtl pf) {
   using namespace wm;
   constexpr int CH = HD / 8;  // 16-byte chunks per row
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -545,8 +545,9 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
   const int klo = lo + rank * per, khi = row_ok ? min(pos, klo + per - 1) : klo - 1;
   const int H = KV * G, qd = H * HD, kvd = KV * HD, ld = qd + 2 * kvd;
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, gq = lane >> 2, tig = lane & 3;
-  const bf16* Kc = (const bf16*)kv.K + ((size_t)seq * KV + g) * kv.cap * HD;
-  const bf16* Vc = (const bf16*)kv.V + ((size_t)seq * KV + g) * kv.cap * HD;
+  // linear or ring cache: this (sequence, KV head)'s rows; paged: the pools
+  const bf16* Kc = (const bf16*)kv.K + (kv.pt ? 0 : ((size_t)seq * KV + g) * kv.cap * HD);
+  const bf16* Vc = (const bf16*)kv.V + (kv.pt ? 0 : ((size_t)seq * KV + g) * kv.cap * HD);
 
   // chunk ci holds keys klo + ci * TC_KC .. in buffer ci & 1.  Cached keys
   // (positions < p0) and the zero padding up to 16 keys come by cp.async;
@@ -563,15 +564,26 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
     uint8_t* kb = sm.k[ci & 1];
     uint8_t* vb = sm.v[ci & 1];
     const int c = tid % CH;
-    int jj = tid / CH, slot = (c0 + jj) % kv.cap;
-    for (; jj < n16; jj += RS) {
-      if (c0 + jj <= cache_hi || jj >= n) {  // cached key, or zero padding up to 16 keys
-        const size_t src = (size_t)slot * HD + c * 8;
-        cp_async16(smem_addr(kb + swz<HD>(jj, c)), Kc + src, jj < n);
-        cp_async16(smem_addr(vb + swz<HD>(jj, c)), Vc + src, jj < n);
+    int jj = tid / CH;
+    if (kv.pt) {
+      for (; jj < n16; jj += RS) {
+        if (c0 + jj <= cache_hi || jj >= n) {  // cached key, or zero padding up to 16 keys
+          const size_t src = (jj < n ? kv_row(kv, seq, KV, g, c0 + jj) : 0) * HD + c * 8;
+          cp_async16(smem_addr(kb + swz<HD>(jj, c)), Kc + src, jj < n);
+          cp_async16(smem_addr(vb + swz<HD>(jj, c)), Vc + src, jj < n);
+        }
       }
-      slot += RS;
-      if (slot >= kv.cap) slot %= kv.cap;  // rare: only when the row wraps around the ring
+    } else {
+      int slot = (c0 + jj) % kv.cap;
+      for (; jj < n16; jj += RS) {
+        if (c0 + jj <= cache_hi || jj >= n) {  // cached key, or zero padding up to 16 keys
+          const size_t src = (size_t)slot * HD + c * 8;
+          cp_async16(smem_addr(kb + swz<HD>(jj, c)), Kc + src, jj < n);
+          cp_async16(smem_addr(vb + swz<HD>(jj, c)), Vc + src, jj < n);
+        }
+        slot += RS;
+        if (slot >= kv.cap) slot %= kv.cap;  // rare: only when the row wraps around the ring
+      }
     }
     cp_async_commit();
   };
@@ -592,6 +604,8 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
   };
   if (nchunk > 0) issue_cached(0);
   if (nchunk > 1) issue_cached(1);
+  // upcoming weights into L2 while this latency-bound kernel leaves HBM idle
+  if (pf.lo < pf.hi) l2_look_ahead(pf, tid, 256);
   pdl_wait();
 
   // Q tile: rows 0..G-1 = the G heads (pre-scaled, bf16), rows G..15 zero
@@ -604,9 +618,9 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
     *reinterpret_cast<bf16*>(sm.q + swz<HD>(h, d / 8) + (d % 8) * 2) = __float2bfloat16_rn(val);
   }
   if (row_ok && klo <= pos && pos <= khi) {  // this block holds the row's own key
-    bf16* Kw = (bf16*)kv.K + ((size_t)seq * KV + g) * kv.cap * HD;
-    bf16* Vw = (bf16*)kv.V + ((size_t)seq * KV + g) * kv.cap * HD;
-    const size_t slot = (size_t)(pos % kv.cap) * HD;
+    bf16* Kw = (bf16*)kv.K;
+    bf16* Vw = (bf16*)kv.V;
+    const size_t slot = kv_row(kv, seq, KV, g, pos) * HD;
     for (int i = tid; i < 2 * HD; i += blockDim.x) {
       const int d = i % HD;
       const bool is_v = i >= HD;
@@ -776,7 +790,7 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
 
 template <int HD, int G, int CS>
 cudaError_t dispatch_tc(int M, int KV, const float* qkv, int S, size_t ps, KVView kv, RowMeta m, bf16* out,
-                        cudaStream_t st) {
+                        cudaStream_t st, const PfCtl& pf) {
   constexpr int SMEM = (int)sizeof(TcSmem<HD, G, CS>);
   auto kern = k_attn_decode_tc<HD, G, CS>;
   static int state = 0;
@@ -818,7 +832,7 @@ cudaError_t dispatch_tc(int M, int KV, const float* qkv, int S, size_t ps, KVVie
   cfg.attrs = at;
   cfg.numAttrs = 2;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
-  return cudaLaunchKernelEx(&cfg, kern, KV, qkv, S, ps, kv, m, out, scale_log2);
+  return cudaLaunchKernelEx(&cfg, kern, KV, qkv, S, ps, kv, m, out, scale_log2, pf);
 }
 
 template <typename T, int HD, int G>
@@ -872,13 +886,13 @@ cudaError_t dispatch_cl(int M, int KV, const float* qkv, int S, size_t ps, KVVie
 template <typename T, int HD, int G>
 cudaError_t dispatch(int M, int KV, const float* qkv, int S, size_t ps, KVView kv, RowMeta m, int max_ctx,
                      float* part, int nb_cap, int part_rows, unsigned* counters, T* out, int batch,
-                     cudaStream_t st) {
+                     cudaStream_t st, const PfCtl& pf) {
   if constexpr (sizeof(T) == 2 && HD >= 64 && G <= 16) {
     if (g_attn_cluster) {
       const int cs = decode_cluster_size(batch, KV);
-      cudaError_t e = cs == 16  ? dispatch_tc<HD, G, 16>(M, KV, qkv, S, ps, kv, m, (bf16*)out, st)
-                      : cs == 8 ? dispatch_tc<HD, G, 8>(M, KV, qkv, S, ps, kv, m, (bf16*)out, st)
-                                : dispatch_tc<HD, G, 4>(M, KV, qkv, S, ps, kv, m, (bf16*)out, st);
+      cudaError_t e = cs == 16  ? dispatch_tc<HD, G, 16>(M, KV, qkv, S, ps, kv, m, (bf16*)out, st, pf)
+                      : cs == 8 ? dispatch_tc<HD, G, 8>(M, KV, qkv, S, ps, kv, m, (bf16*)out, st, pf)
+                                : dispatch_tc<HD, G, 4>(M, KV, qkv, S, ps, kv, m, (bf16*)out, st, pf);
       if (e != cudaErrorNotSupported) return e;
     }
   }
@@ -906,12 +920,12 @@ cudaError_t dispatch(int M, int KV, const float* qkv, int S, size_t ps, KVView k
 template <typename T>
 cudaError_t launch_attn_decode(int M, int H, int KV, int hd, const float* qkv, int S, size_t ps, KVView kv,
                                RowMeta m, int max_ctx, float* part, int nb_cap, int part_rows, unsigned* counters,
-                               T* out, int batch, cudaStream_t st) {
+                               T* out, int batch, cudaStream_t st, const PfCtl& pf) {
   const int G = H / KV;
 #define DORY_DEC_CASE(HDV, GV)                                                                                   \
   if (hd == HDV && G == GV)                                                                                      \
     return dispatch<T, HDV, GV>(M, KV, qkv, S, ps, kv, m, max_ctx, part, nb_cap, part_rows, counters, out, batch, \
-                                st);
+                                st, pf);
   DORY_DEC_CASE(32, 1) DORY_DEC_CASE(32, 2) DORY_DEC_CASE(32, 4) DORY_DEC_CASE(32, 5) DORY_DEC_CASE(32, 8)
   DORY_DEC_CASE(64, 1) DORY_DEC_CASE(64, 2) DORY_DEC_CASE(64, 4) DORY_DEC_CASE(64, 5) DORY_DEC_CASE(64, 8)
   DORY_DEC_CASE(128, 1) DORY_DEC_CASE(128, 2) DORY_DEC_CASE(128, 4) DORY_DEC_CASE(128, 5)
@@ -920,8 +934,9 @@ cudaError_t launch_attn_decode(int M, int H, int KV, int hd, const float* qkv, i
 }
 
 template cudaError_t launch_attn_decode<float>(int, int, int, int, const float*, int, size_t, KVView, RowMeta, int,
-                                               float*, int, int, unsigned*, float*, int, cudaStream_t);
+                                               float*, int, int, unsigned*, float*, int, cudaStream_t,
+                                               const PfCtl&);
 template cudaError_t launch_attn_decode<bf16>(int, int, int, int, const float*, int, size_t, KVView, RowMeta, int,
-                                              float*, int, int, unsigned*, bf16*, int, cudaStream_t);
+                                              float*, int, int, unsigned*, bf16*, int, cudaStream_t, const PfCtl&);
 
 }  // namespace dory

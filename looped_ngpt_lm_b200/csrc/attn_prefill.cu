@@ -98,8 +98,8 @@ __global__ void __launch_bounds__(128, 3) k_attn_prefill(int KV, int G, const bf
   const int pf = m.pos[r0], pl = m.pos[r1 - 1];
   const int lo_min = kv.window > 0 ? max(0, pf - kv.window + 1) : 0;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bf16* Kc = (const bf16*)kv.K + ((size_t)seq * KV + g) * kv.cap * HD;
-  const bf16* Vc = (const bf16*)kv.V + ((size_t)seq * KV + g) * kv.cap * HD;
+  const bf16* Kc = (const bf16*)kv.K;
+  const bf16* Vc = (const bf16*)kv.V;
 
   // Q tile -> shared memory (rows past r1 are zero)
   for (int i = tid; i < QT * CH; i += 128) {
@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(128, 3) k_attn_prefill(int KV, int G, const bf
         ks = kscr + o;
         vs = vscr + o;
       } else {
-        const size_t o = (size_t)((ok ? j : 0) % kv.cap) * HD + ch * 8;
+        const size_t o = (ok ? kv_row(kv, seq, KV, g, j) : 0) * HD + ch * 8;
         ks = Kc + o;
         vs = Vc + o;
       }

@@ -156,8 +156,8 @@ __global__ void __launch_bounds__(NTH, 2) k_attn_prefill_tc(int KV, int G, const
   const int seq = m.seq[r0], p0 = m.p0[r0], base = m.base[r0];
   const int pf = m.pos[r0], pl = m.pos[tile.y - 1];
   const int lo_min = kv.window > 0 ? max(0, pf - kv.window + 1) : 0;
-  const bf16* Kc = (const bf16*)kv.K + ((size_t)seq * KV + g) * kv.cap * HDT;
-  const bf16* Vc = (const bf16*)kv.V + ((size_t)seq * KV + g) * kv.cap * HDT;
+  const bf16* Kc = (const bf16*)kv.K;
+  const bf16* Vc = (const bf16*)kv.V;
 
   // Q tile (rows past the tile are zero)
   for (int i = tid; i < TQ * 16; i += NTH) {
@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(NTH, 2) k_attn_prefill_tc(int KV, int G, const
           ks = kscr + o;
           vs = vscr + o;
         } else if (ok) {
-          const size_t o = (size_t)(j % kv.cap) * HDT + lc * 8;
+          const size_t o = kv_row(kv, seq, KV, g, j) * HDT + lc * 8;
           ks = Kc + o;
           vs = Vc + o;
         }

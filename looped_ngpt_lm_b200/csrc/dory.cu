@@ -149,12 +149,19 @@ struct dory_handle {
 
   // host state
   std::vector<int> len, mode, kfix;  // per sequence; mode -1 = empty
+  // paged full-attention cache: device page table [max_batch][pt_stride],
+  // its host copy, the pages each sequence holds and the free pool
+  int* page_table = nullptr;
+  int pt_stride = 0, page_shift = 0, pool_pages = 0;
+  std::vector<int> pt_host, free_pages;
+  std::vector<std::vector<int>> seq_pages;
   std::vector<int> ids_on_device;     // seq ids last uploaded to seq_ids
   int last_rows = 0;
   bool graphs = true, profile = false;
   int prefill_tc = 2;  // long-chunk attention: 2 tcgen05 (head_dim 128), 1 mma.sync, 0 CUDA cores
   int gemm_impl = 0;
   unsigned long long pf_lead = 8ull << 20;   // 0: no L2 look-ahead
+  unsigned long long pf_attn = 0;            // bytes the decode attention prefetches (0: none)
   float temperature = 0.f, top_p = 1.f;      // temperature 0: greedy
   unsigned long long seed = 0;
   std::vector<std::vector<PfSeg>> pf_host;   // [k] -> stream of a k-loop decode step
@@ -206,6 +213,9 @@ dory_status check_config(const dory_config* c) {
   if (c->max_batch <= 0 || c->max_seq <= 0 || c->max_chunk <= 0) return fail(DORY_ERR_INVALID_ARG, "bad capacity");
   if (c->k_max < 1 || c->k_max > 8) return fail(DORY_ERR_INVALID_ARG, "k_max must be in 1..8");
   if (c->gamma_max < 0 || c->gamma_max > 16) return fail(DORY_ERR_INVALID_ARG, "gamma_max must be in 0..16");
+  if (c->kv_page != 0 && (c->kv_page < 16 || c->kv_page > 4096 || (c->kv_page & (c->kv_page - 1))))
+    return fail(DORY_ERR_INVALID_ARG, "kv_page must be 0 or a power of two in 16..4096");
+  if (c->kv_pages < 0) return fail(DORY_ERR_INVALID_ARG, "kv_pages must be >= 0");
   return DORY_OK;
 }
 
@@ -231,6 +241,12 @@ size_t layout(dory_handle* h) {
 
   h->attn.clear();
   h->attn_of.assign(h->L, -1);
+  if (c.kv_page > 0) {
+    h->pt_stride = (c.max_seq + c.kv_page - 1) / c.kv_page;
+    h->page_shift = 0;
+    while ((1 << h->page_shift) < c.kv_page) ++h->page_shift;
+    h->pool_pages = c.kv_pages > 0 ? c.kv_pages : c.max_batch * h->pt_stride;
+  }
   int j = 0;
   for (int l = 0; l < h->L; ++l) {
     if (!layer_is_attn(l)) continue;
@@ -241,6 +257,7 @@ size_t layout(dory_handle* h) {
     a.cap = a.full ? c.max_seq : std::min(c.max_seq, c.swa_window + h->slack);
     a.nslots = (h->alloc_mode == DORY_PER_LOOP && a.rec) ? c.k_max : 1;
     size_t bytes = (size_t)c.max_batch * c.n_kv_heads * a.cap * c.head_dim * e;
+    if (a.full && c.kv_page > 0) bytes = (size_t)h->pool_pages * c.n_kv_heads * c.kv_page * c.head_dim * e;
     for (int s = 0; s < a.nslots; ++s) {
       a.K[s] = cv.take<char>(bytes);
       a.V[s] = cv.take<char>(bytes);
@@ -250,6 +267,7 @@ size_t layout(dory_handle* h) {
     ++j;
   }
   const int d = c.d_model;
+  if (c.kv_page > 0) h->page_table = cv.take<int>(sizeof(int) * (size_t)c.max_batch * h->pt_stride);
   h->seq_len = cv.take<int>(sizeof(int) * c.max_batch);
   h->err = cv.take<int>(sizeof(int) * 4);
   h->seq_ids = cv.take<int>(sizeof(int) * M);
@@ -369,7 +387,47 @@ KVView kv_view(dory_handle* H, int l, int loop, int mode) {
   v.window = a.full ? 0 : H->c.swa_window;
   v.limit = H->c.max_seq;
   v.err = H->err;
+  if (a.full && H->page_table) {
+    v.pt = H->page_table;
+    v.pt_stride = H->pt_stride;
+    v.page_shift = H->page_shift;
+  }
   return v;
+}
+
+// Paged cache: give every listed sequence the pages that hold positions
+// 0 .. upto[i] - 1, and upload the new page-table entries.  Checks the free
+// pool first, so a refused call changes nothing.
+dory_status ensure_pages(dory_handle* H, int n, const int32_t* seq_ids, const int64_t* upto, cudaStream_t st) {
+  if (!H->page_table) return DORY_OK;
+  const int P = H->c.kv_page;
+  int64_t need = 0;
+  for (int i = 0; i < n; ++i)
+    need += std::max<int64_t>(0, (upto[i] + P - 1) / P - (int64_t)H->seq_pages[seq_ids[i]].size());
+  if (need > (int64_t)H->free_pages.size())
+    return fail(DORY_ERR_CAPACITY, "the paged cache needs %lld more pages, %zu are free", (long long)need,
+                H->free_pages.size());
+  for (int i = 0; i < n; ++i) {
+    const int sq = seq_ids[i];
+    std::vector<int>& mine = H->seq_pages[sq];
+    const int first = (int)mine.size(), want = (int)((upto[i] + P - 1) / P);
+    if (want <= first) continue;
+    for (int q = first; q < want; ++q) {
+      mine.push_back(H->free_pages.back());
+      H->free_pages.pop_back();
+      H->pt_host[(size_t)sq * H->pt_stride + q] = mine.back();
+    }
+    const size_t at = (size_t)sq * H->pt_stride + first;
+    CK(cudaMemcpyAsync(H->page_table + at, H->pt_host.data() + at, sizeof(int) * (want - first),
+                       cudaMemcpyHostToDevice, st));
+  }
+  return DORY_OK;
+}
+
+void release_pages(dory_handle* H, int seq) {
+  if (!H->page_table) return;
+  for (int p : H->seq_pages[seq]) H->free_pages.push_back(p);
+  H->seq_pages[seq].clear();
 }
 
 // Rows per split slice of a GEMM output buffer for this pass.
@@ -479,6 +537,28 @@ dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, cons
     if (r_ != DORY_OK) return r_;       \
   } while (0)
 
+// L2 look-ahead of a decode attention launch: the next pf_attn bytes of the
+// weight stream not yet handed out, starting at the next GEMM's weights (the
+// attention leaves HBM idle while it waits on latency).
+template <typename T>
+PfCtl attn_look_ahead(const Fwd<T>& f) {
+  dory_handle* H = f.H;
+  PfCtl pfc;
+  if (H->pf_attn == 0 || f.pf_k <= 0 || H->pf_pos < 0) return pfc;
+  const std::vector<PfSeg>& v = H->pf_host[f.pf_k];
+  if (H->pf_pos >= (int)v.size()) return pfc;
+  const unsigned long long total = v.back().off + v.back().bytes;
+  pfc.segs = H->pf_segs + (size_t)(f.pf_k - 1) * H->pf_nseg_max;
+  pfc.nseg = (int)v.size();
+  pfc.lo = std::max(H->pf_done, v[H->pf_pos].off);
+  pfc.hi = std::min(pfc.lo + H->pf_attn, total);
+  if (pfc.lo >= pfc.hi) return PfCtl{};
+  pfc.first = H->pf_pos;
+  while (pfc.first + 1 < pfc.nseg && v[pfc.first + 1].off <= pfc.lo) ++pfc.first;
+  H->pf_done = pfc.hi;
+  return pfc;
+}
+
 // Whether the GEMM of weight W ([N, K]) on this pass can take operand stage p.
 template <typename T>
 bool stage_ok(const Fwd<T>& f, int N, int K, const void* W, const Prep& p) {
@@ -539,9 +619,10 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop, float* copy_la
       }      if (f.direct) {
         // fused: q from the partials, own K/V into the cache, split-KV attention
         Scope sc(H, f.st, "attn_decode", 0);
+        const PfCtl apf = attn_look_ahead(f);
         CK(launch_attn_decode<T>(M, c.n_heads, c.n_kv_heads, c.head_dim, H->part_qkv, S, ps, kv, H->meta, f.max_ctx,
                                  H->attn_part, H->nb_cap, H->attn_rows, H->attn_counters, (T*)H->ao, f.batch,
-                                 f.st));
+                                 f.st, apf));
       } else {
         // long chunks: K/V into scratch, attention, then the cache commit
         const bool tc = f.n_tiles > 0;
@@ -1156,6 +1237,12 @@ dory_status dory_create(const dory_config* cfg, const dory_weights* w, dory_cach
   H->len.assign(cfg->max_batch, 0);
   H->mode.assign(cfg->max_batch, -1);
   H->kfix.assign(cfg->max_batch, 0);
+  if (H->page_table) {
+    H->pt_host.assign((size_t)cfg->max_batch * H->pt_stride, 0);
+    H->seq_pages.assign(cfg->max_batch, {});
+    H->free_pages.clear();
+    for (int p = H->pool_pages - 1; p >= 0; --p) H->free_pages.push_back(p);
+  }
   *out = H;
   return DORY_OK;
 }
@@ -1179,12 +1266,14 @@ dory_status dory_reset(dory_handle* h, int32_t seq, dory_stream stream) {
     CK(cudaMemsetAsync(h->attn_counters, 0, sizeof(unsigned) * (size_t)h->M_max * h->c.n_kv_heads, st));
     std::fill(h->len.begin(), h->len.end(), 0);
     std::fill(h->mode.begin(), h->mode.end(), -1);
+    for (int q = 0; q < h->c.max_batch; ++q) release_pages(h, q);
     return DORY_OK;
   }
   if (seq < 0 || seq >= h->c.max_batch) return fail(DORY_ERR_INVALID_ARG, "seq %d out of range", seq);
   CK(cudaMemsetAsync(h->seq_len + seq, 0, sizeof(int), st));
   h->len[seq] = 0;
   h->mode[seq] = -1;
+  release_pages(h, seq);
   return DORY_OK;
 }
 
@@ -1202,6 +1291,11 @@ dory_status dory_prefill(dory_handle* h, int32_t batch, const int32_t* seq_ids, 
       return fail(DORY_ERR_CAPACITY, "sequence %d would exceed max_seq", seq_ids[i]);
   }
   if (total > h->c.max_chunk) return fail(DORY_ERR_CAPACITY, "%lld tokens > max_chunk %d", (long long)total, h->c.max_chunk);
+  {
+    std::vector<int64_t> upto(batch);
+    for (int i = 0; i < batch; ++i) upto[i] = (int64_t)h->len[seq_ids[i]] + lens[i];
+    RET(ensure_pages(h, batch, seq_ids, upto.data(), (cudaStream_t)stream));
+  }
   dory_status r = h->bf16 ? prefill_t<bf16>(h, batch, seq_ids, tokens, lens, k, mode, last_logits, next_tokens,
                                              (cudaStream_t)stream)
                           : prefill_t<float>(h, batch, seq_ids, tokens, lens, k, mode, last_logits, next_tokens,
@@ -1219,6 +1313,11 @@ dory_status dory_decode_step(dory_handle* h, int32_t batch, const int32_t* seq_i
   for (int i = 0; i < batch; ++i)
     if (h->len[seq_ids[i]] + 1 > h->c.max_seq)
       return fail(DORY_ERR_CAPACITY, "sequence %d would exceed max_seq", seq_ids[i]);
+  {
+    std::vector<int64_t> upto(batch);
+    for (int i = 0; i < batch; ++i) upto[i] = (int64_t)h->len[seq_ids[i]] + 1;
+    RET(ensure_pages(h, batch, seq_ids, upto.data(), (cudaStream_t)stream));
+  }
   dory_status r = h->bf16 ? decode_t<bf16>(h, batch, seq_ids, tokens_in, k, mode, logits, next_tokens,
                                             (cudaStream_t)stream)
                           : decode_t<float>(h, batch, seq_ids, tokens_in, k, mode, logits, next_tokens,
@@ -1243,6 +1342,11 @@ dory_status dory_decode_step_mixed(dory_handle* h, int32_t batch, const int32_t*
       return fail(DORY_ERR_CAPACITY, "sequence %d would exceed max_seq", seq_ids[i]);
   }
   const cudaStream_t st = (cudaStream_t)stream;
+  {
+    std::vector<int64_t> upto(batch);
+    for (int i = 0; i < batch; ++i) upto[i] = (int64_t)h->len[seq_ids[i]] + 1;
+    RET(ensure_pages(h, batch, seq_ids, upto.data(), st));
+  }
   dory_status r = h->bf16 ? decode_mixed_t<bf16>(h, batch, seq_ids, tokens_in, ks, mode, logits, next_tokens, st)
                           : decode_mixed_t<float>(h, batch, seq_ids, tokens_in, ks, mode, logits, next_tokens, st);
   if (r == DORY_OK)
@@ -1269,6 +1373,11 @@ dory_status dory_spec_decode(dory_handle* h, int32_t batch, const int32_t* seq_i
     // still writes gamma positions past its length
     if ((int64_t)h->len[sq] + max_new + 2 * gamma + 1 > h->c.max_seq)
       return fail(DORY_ERR_CAPACITY, "sequence %d: len + max_new + 2*gamma + 1 exceeds max_seq", sq);
+  }
+  {
+    std::vector<int64_t> upto(batch);
+    for (int i = 0; i < batch; ++i) upto[i] = (int64_t)h->len[seq_ids[i]] + max_new + 2 * gamma + 1;
+    RET(ensure_pages(h, batch, seq_ids, upto.data(), (cudaStream_t)stream));
   }
   return h->bf16 ? spec_t<bf16>(h, batch, seq_ids, last_tokens, k_verify, gamma, mode, max_new, out_tokens, out_len,
                                 stats, (cudaStream_t)stream)
@@ -1321,6 +1430,10 @@ dory_status dory_read_kv(dory_handle* h, int32_t layer, int32_t slot, int32_t se
     int p = pos0 + i;
     for (int g = 0; g < KV; ++g) {
       size_t src = (((size_t)seq * KV + g) * a.cap + (p % a.cap)) * row;
+      if (a.full && h->page_table) {
+        const int P = h->c.kv_page;
+        src = (((size_t)h->pt_host[(size_t)seq * h->pt_stride + p / P] * KV + g) * P + p % P) * row;
+      }
       size_t dst = ((size_t)i * KV + g) * row;
       CK(cudaMemcpyAsync((char*)k_dst + dst, a.K[slot] + src, row, cudaMemcpyDeviceToDevice, st));
       CK(cudaMemcpyAsync((char*)v_dst + dst, a.V[slot] + src, row, cudaMemcpyDeviceToDevice, st));
@@ -1408,6 +1521,15 @@ dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value) {
     case DORY_OPT_GEMM_IMPL:
       if (value < 0 || value > 2) return fail(DORY_ERR_INVALID_ARG, "bad GEMM impl");
       h->gemm_impl = (int)value;
+      return DORY_OK;
+    case DORY_OPT_ATTN_LOOKAHEAD:
+      if (value < 0 || value > (1ll << 40)) return fail(DORY_ERR_INVALID_ARG, "bad look-ahead");
+      if ((unsigned long long)value != h->pf_attn) {
+        for (auto& g : h->graphs_cache)
+          if (g.exec) cudaGraphExecDestroy(g.exec);
+        h->graphs_cache.clear();
+      }
+      h->pf_attn = (unsigned long long)value & ~127ull;
       return DORY_OK;
     case DORY_OPT_FUSED_OPERANDS:
       if (value < 0 || value > 16) return fail(DORY_ERR_INVALID_ARG, "fused operand rows must be in 0..16");

@@ -74,25 +74,6 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
   return p;
 }
 
-// Prefetch this CTA's piece of the look-ahead range (see PfCtl) into L2;
-// called by all 32 lanes of one warp, each taking every 32nd 128-byte line.
-// Segment sizes and offsets are multiples of 128 bytes.
-__device__ void l2_look_ahead(const PfCtl& pf, int lane) {
-  const unsigned long long span = pf.hi - pf.lo;
-  const unsigned long long piece = ((span + gridDim.x - 1) / gridDim.x + 127) & ~127ull;
-  const unsigned long long a0 = pf.lo + piece * blockIdx.x;
-  const unsigned long long a1 = a0 + piece < pf.hi ? a0 + piece : pf.hi;
-  if (a0 >= a1) return;
-  for (int q = pf.first; q < pf.nseg && pf.segs[q].off < a1; ++q) {
-    const unsigned long long so = pf.segs[q].off, se = so + pf.segs[q].bytes;
-    if (se <= a0) continue;
-    const unsigned long long lo = a0 > so ? a0 : so, hi = a1 < se ? a1 : se;
-    const char* base = pf.segs[q].p - so;
-    for (unsigned long long a = (lo & ~127ull) + 128ull * lane; a < hi; a += 128ull * 32)
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(base + a));
-  }
-}
-
 // KSUB 64-column sub-tiles per pipeline stage: a stage reads KSUB*128
 // contiguous bytes of every weight row.
 // GLU: a unit's A operand is two 128-row tiles of one matrix, rows
@@ -376,7 +357,7 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
     __syncwarp();
-    if (pf.lo < pf.hi && !*abort_flag) l2_look_ahead(pf, lane);
+    if (pf.lo < pf.hi && !*abort_flag) l2_look_ahead(pf, lane, 32);
   } else if (warp == 1) {
     pdl_wait();
     if (lane == 0) {

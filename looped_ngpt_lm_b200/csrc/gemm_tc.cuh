@@ -49,6 +49,26 @@ struct Prep {
   int ldy = 0;
 };
 
+// Prefetch this CTA's piece of the look-ahead range into L2 (CTA b takes
+// the b-th of gridDim.x equal pieces); called by `nthreads` threads, thread
+// t taking every nthreads-th 128-byte line.  Segment sizes and offsets are
+// multiples of 128 bytes.
+__device__ __forceinline__ void l2_look_ahead(const PfCtl& pf, int t, int nthreads) {
+  const unsigned long long span = pf.hi - pf.lo;
+  const unsigned long long piece = ((span + gridDim.x - 1) / gridDim.x + 127) & ~127ull;
+  const unsigned long long a0 = pf.lo + piece * blockIdx.x;
+  const unsigned long long a1 = a0 + piece < pf.hi ? a0 + piece : pf.hi;
+  if (a0 >= a1) return;
+  for (int q = pf.first; q < pf.nseg && pf.segs[q].off < a1; ++q) {
+    const unsigned long long so = pf.segs[q].off, se = so + pf.segs[q].bytes;
+    if (se <= a0) continue;
+    const unsigned long long lo = a0 > so ? a0 : so, hi = a1 < se ? a1 : se;
+    const char* base = pf.segs[q].p - so;
+    for (unsigned long long a = (lo & ~127ull) + 128ull * t; a < hi; a += 128ull * nthreads)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(base + a));
+  }
+}
+
 // Y = X . W^T for X [M, K] (row stride ldx) and W [N, K], both bf16, fp32
 // accumulation.  Writes S partial products to Y + s * (*part_stride)
 // (row stride ldy); the consumer adds them in order s = 0..S-1.

@@ -24,6 +24,10 @@ struct RowMeta {
 // [max_batch][n_kv][cap][head_dim] in the storage type.  window == 0 means
 // full causal attention, otherwise keys p-window < j <= p.  Position j lives
 // at index j % cap (a ring for sliding-window layers, cap >= max_seq for full).
+//
+// Paged full-attention layers (pt != NULL): positions come in pages of
+// 2^page_shift; page table pt[seq * pt_stride + j >> page_shift] names the
+// page holding position j, and K, V are [pages][n_kv][2^page_shift][head_dim].
 struct KVView {
   void* K;
   void* V;
@@ -31,7 +35,20 @@ struct KVView {
   int window;
   int limit;  // max_seq: positions >= limit are rejected (error word set)
   int* err;   // device error word
+  const int* pt = nullptr;
+  int pt_stride = 0;
+  int page_shift = 0;
 };
+
+// Row index (in head_dim-element rows) of position j of sequence seq, KV
+// head g, in K or V of the layer.
+__device__ __forceinline__ size_t kv_row(const KVView& kv, int seq, int n_kv, int g, int j) {
+  if (kv.pt) {
+    const int page = kv.pt[(size_t)seq * kv.pt_stride + (j >> kv.page_shift)];
+    return (((size_t)page * n_kv + g) << kv.page_shift) + (size_t)(j & ((1 << kv.page_shift) - 1));
+  }
+  return ((size_t)seq * n_kv + g) * kv.cap + (size_t)(j % kv.cap);
+}
 
 // ---- chunk planning (device-side row metadata) ---------------------------
 cudaError_t launch_plan_uniform(int n_seq, int rows_per_seq, int pos_offset, const int* seq_ids,

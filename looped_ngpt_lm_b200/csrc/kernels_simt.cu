@@ -294,7 +294,6 @@ __global__ void k_qkv_post(int H, int KV, int hd, const float* qkv, int S, size_
     if (threadIdx.x == 0) set_error(kv.err, DEV_ERR_BAD_INDEX);
     return;
   }
-  const size_t ring = (size_t)(pos % kv.cap);
   for (int i = threadIdx.x; i < ld; i += blockDim.x) {
     float a = 0.f;
     for (int s = 0; s < S; ++s) a += src[s * ps + i];
@@ -310,7 +309,7 @@ __global__ void k_qkv_post(int H, int KV, int hd, const float* qkv, int S, size_
       T val = from_f<T>(a);
       if (direct) {
         int g = j / hd, e = j % hd;
-        size_t off = (((size_t)seq * KV + g) * kv.cap + ring) * hd + e;
+        size_t off = kv_row(kv, seq, KV, g, pos) * hd + e;
         (is_v ? (T*)kv.V : (T*)kv.K)[off] = val;
       } else {
         (is_v ? vscr : kscr)[(size_t)r * kvd + j] = val;
@@ -378,8 +377,8 @@ __global__ void __launch_bounds__(128) k_attn_partial(int KV, const float* __res
 #pragma unroll
     for (int e = 0; e < DL; ++e) acc[h][e] = 0.f;
   }
-  const T* Kc = (const T*)kv.K + ((size_t)seq * KV + g) * kv.cap * HD;
-  const T* Vc = (const T*)kv.V + ((size_t)seq * KV + g) * kv.cap * HD;
+  const T* Kc = (const T*)kv.K;
+  const T* Vc = (const T*)kv.V;
   const int kb = ab * ATTN_BK;
   for (int jq = kb + 4 * w; jq <= khi; jq += 16) {
     const int j = jq + sg;
@@ -392,7 +391,7 @@ __global__ void __launch_bounds__(128) k_attn_partial(int KV, const float* __res
         kp = kscr + row * kvd + g * HD;
         vp = vscr + row * kvd + g * HD;
       } else {
-        size_t idx = (size_t)(j % kv.cap) * HD;
+        size_t idx = kv_row(kv, seq, KV, g, j) * HD;
         kp = Kc + idx;
         vp = Vc + idx;
       }
@@ -565,10 +564,9 @@ __global__ void k_kv_commit(int KV, int hd, const T* kscr, const T* vscr, KVView
     return;
   }
   const int kvd = KV * hd;
-  const size_t ring = (size_t)(pos % kv.cap);
   for (int j = threadIdx.x; j < kvd; j += blockDim.x) {
     int g = j / hd, e = j % hd;
-    size_t off = (((size_t)seq * KV + g) * kv.cap + ring) * hd + e;
+    size_t off = kv_row(kv, seq, KV, g, pos) * hd + e;
     ((T*)kv.K)[off] = kscr[(size_t)r * kvd + j];
     ((T*)kv.V)[off] = vscr[(size_t)r * kvd + j];
   }

@@ -194,3 +194,44 @@ def test_create_rejects_bad_workspace_and_config():
     assert lib.dory_workspace_size(ctypes.byref(bad), 0, ctypes.byref(ctypes.c_size_t())) == 7
     bad = dory.make_config(synth.TINY.with_(n_kv_heads=3))
     assert lib.dory_workspace_size(ctypes.byref(bad), 0, ctypes.byref(ctypes.c_size_t())) == 1
+
+
+def test_paged_full_attention_cache_sizes_the_pool_not_every_slot():
+    """A page pool for the full-attention layers replaces max_batch linear
+    arrays of max_seq positions: 8 slots of 262,144 positions with a pool for
+    one such sequence (plus short ones) is several times smaller."""
+    s = synth.DORY_4B  # 9 full-attention layers, one cache slot each in last_loop mode
+    big = dict(max_batch=8, max_seq=262144, max_chunk=8192)
+    pages = 262144 // 64 + 7 * 64
+    linear = dory.workspace_size(cfg_for(s, **big), dory.LAST_LOOP)
+    paged = dory.workspace_size(cfg_for(s, kv_page=64, kv_pages=pages, **big), dory.LAST_LOOP)
+    full = dory.workspace_size(cfg_for(s, kv_page=64, **big), dory.LAST_LOOP)  # default pool: every slot full
+    per_pos = 2 * s.kv_dim * 2  # K and V bytes of one position in one layer
+    saved = 9 * (8 * 262144 - pages * 64) * per_pos
+    table = 8 * (262144 // 64) * 4
+    assert abs((linear - paged) - (saved - table)) < 64 * 1024
+    assert abs(full - linear - table) < 64 * 1024
+    assert paged < linear / 3
+
+
+@pytest.mark.parametrize("page", [8, 48, 8192])
+def test_bad_page_sizes_are_rejected(page):
+    cfg = cfg_for(synth.TINY, kv_page=page)
+    n = ctypes.c_size_t()
+    assert lib.dory_workspace_size(ctypes.byref(cfg), dory.LAST_LOOP, ctypes.byref(n)) == 1
+    assert b"kv_page" in lib.dory_last_error()
+
+
+def test_page_pool_exhaustion_is_a_capacity_error_before_any_work():
+    """Two 16-position pages for a 48-token prompt: refused before launch,
+    with nothing changed (the same call then fits after a reset frees pages)."""
+    h, cfg, keep = fake_handle(synth.TINY, kv_page=16, kv_pages=2)
+    ids = (ctypes.c_int32 * 1)(0)
+    lens = (ctypes.c_int32 * 1)(48)
+    st = lib.dory_prefill(h, 1, ids, ctypes.c_void_p(FAKE_WS), lens, 1, dory.LAST_LOOP, None,
+                          ctypes.c_void_p(FAKE_WS), None)
+    assert st == 2, lib.dory_last_error()
+    assert b"pages" in lib.dory_last_error()
+    n = ctypes.c_int32()
+    assert lib.dory_seq_len(h, 0, ctypes.byref(n)) == 0 and n.value == 0
+    lib.dory_destroy(h)

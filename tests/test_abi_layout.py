@@ -24,7 +24,8 @@ CONSTANTS = {
     "DORY_BF16": dory.BF16, "DORY_OPT_CUDA_GRAPHS": dory.OPT_CUDA_GRAPHS, "DORY_OPT_PROFILE": dory.OPT_PROFILE,
     "DORY_OPT_GEMM_IMPL": dory.OPT_GEMM_IMPL, "DORY_OPT_PDL": dory.OPT_PDL, "DORY_OPT_PREFILL_TC": dory.OPT_PREFILL_TC,
     "DORY_OPT_ATTN_CLUSTER": dory.OPT_ATTN_CLUSTER, "DORY_OPT_L2_LOOKAHEAD": dory.OPT_L2_LOOKAHEAD,
-    "DORY_OPT_MX_GEMV": dory.OPT_MX_GEMV,
+    "DORY_OPT_MX_GEMV": dory.OPT_MX_GEMV, "DORY_OPT_FUSED_OPERANDS": dory.OPT_FUSED_OPERANDS,
+    "DORY_OPT_ATTN_LOOKAHEAD": dory.OPT_ATTN_LOOKAHEAD,
 }
 
 
