@@ -375,6 +375,7 @@ struct Fwd {
   int n_tiles = 0;  // > 0: long-chunk attention on the tensor cores over H->tiles
   bool tc5 = false; // ... by the tcgen05 kernel (128-row tiles)
   int pf_k = 0;     // > 0: GEMMs follow the weight stream of a pf_k-loop decode step
+  bool stage = true;  // layer updates may run in the next GEMM's operand stage
 };
 
 KVView kv_view(dory_handle* H, int l, int loop, int mode) {
@@ -563,7 +564,7 @@ PfCtl attn_look_ahead(const Fwd<T>& f) {
 template <typename T>
 bool stage_ok(const Fwd<T>& f, int N, int K, const void* W, const Prep& p) {
   const dory_handle* H = f.H;
-  if (sizeof(T) != 2 || !f.invariant || f.M > H->fuse_rows || H->gemm_impl == 1) return false;
+  if (sizeof(T) != 2 || !f.stage || !f.invariant || f.M > H->fuse_rows || H->gemm_impl == 1) return false;
   if (!H->mx.empty() && H->mx.count(W)) return false;
   return gemm_tc_prep_ok(f.M, N, K, f.batch, p);
 }
@@ -1020,6 +1021,10 @@ dory_status decode_mixed_t(dory_handle* H, int batch, const int32_t* seq_ids, co
     while (rows < batch && ks[rows] >= t) ++rows;
     Fwd<T> g = f;
     g.M = rows;
+    // an operand stage writes the updated state of its rows to the other
+    // state buffer; rows that finished their loops would be left behind in
+    // this one, so a pass over part of the batch updates in place
+    g.stage = rows == batch;
     {
       // u_t = N(s_{t-1} + x), s_0 = x, s_{t-1} = N(h)
       Scope sc(H, st, "reinject", 0);

@@ -685,11 +685,11 @@ static cudaError_t run_prep(const CUtensorMap& ma, int M, int K, float* Y, int l
 }
 
 bool gemm_tc_prep_ok(int M, int N, int K, int batch, const Prep& p) {
-  if (p.mode == kPrepNone || M < 1 || M > 16 || N % BM || K % (4 * BK) || K > 4 * AN_MAXC * AN_THREADS ||
-      p.S < 1 || p.S > AN_MAXS || p.ldy % 4 || p.ps % 4 || ((uintptr_t)p.y & 15))
+  if (p.mode == kPrepNone || M < 1 || M > 16 || N % BM || K % (4 * BK) || p.S < 1 || p.S > AN_MAXS || p.ldy % 4 ||
+      p.ps % 4 || ((uintptr_t)p.y & 15))
     return false;
-  if (p.mode == kPrepAddNorm &&
-      (p.h_in == p.h_out || ((uintptr_t)p.h_in & 15) || ((uintptr_t)p.h_out & 15) || p.ldy < K))
+  if (p.mode == kPrepAddNorm && (K > 4 * AN_MAXC * AN_THREADS || p.h_in == p.h_out ||
+                                 ((uintptr_t)p.h_in & 15) || ((uintptr_t)p.h_out & 15) || p.ldy < K))
     return false;
   if (p.mode == kPrepSwiglu && p.ldy < 2 * K) return false;
   UnitMap um;
@@ -711,11 +711,8 @@ cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf
   const bool staged = prep && prep->mode != kPrepNone;
   if (staged) {
     // the operand stage: decode tiles of one 16-token group, weights by TMA
-    if (!invariant || packed || variant != 0 || M > 16 || N % BM || K % (4 * BK) || K > 4 * AN_MAXC * AN_THREADS ||
-        (size_t)M > part_rows || ((uintptr_t)W & 15) || prep->S < 1 || prep->S > AN_MAXS || prep->ldy % 4 ||
-        prep->ps % 4 || ((uintptr_t)prep->y & 15) ||
-        (prep->mode == kPrepAddNorm && (prep->h_in == prep->h_out || ((uintptr_t)prep->h_in & 15) ||
-                                        ((uintptr_t)prep->h_out & 15))))
+    if (!invariant || packed || variant != 0 || (size_t)M > part_rows || ((uintptr_t)W & 15) ||
+        !gemm_tc_prep_ok(M, N, K, batch, *prep))
       return cudaErrorNotSupported;
   } else if (M <= 0 || N % BM || K % BK || ldx % 8 || (size_t)M > part_rows || ((uintptr_t)X & 15) ||
              ((uintptr_t)W & 15)) {
