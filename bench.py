@@ -370,27 +370,33 @@ def sampling_leg(dory, torch, h, tok, args, mode, steps=64):
     return out, tok
 
 
-def mxfp8_leg(dory, torch, shape, dw, args, mode, bf16_sweep, steps=32):
-    """Batch-1 decode with MXFP8 weights (E4M3 codes, one E8M0 scale per 32
-    weights, quantised on the GPU from the bench's bf16 weights) at k = 1, 2,
-    4 on a handle of its own: prefill reads the exact bf16 dequantisation,
-    decode GEMMs the 8-bit copies.  Reports tokens/s, the speed-up over the
-    bf16 k sweep at the same context, and the GEMV's HBM roofline."""
+def lowbit_leg(dory, torch, shape, dw, args, mode, bf16_sweep, fmt, steps=32):
+    """Batch-1 decode with low-bit weight copies made on the GPU from the
+    bench's bf16 weights, at k = 1, 2, 4 on a handle of its own: prefill reads
+    the exact bf16 dequantisation, decode GEMMs the copies.  fmt "mxfp8":
+    E4M3 codes with one E8M0 scale per 32 weights, timed with the CUDA-core
+    GEMV (option 1) and the TMA-fed tcgen05 GEMM (option 3); fmt "nvfp4":
+    E2M1 codes, one E4M3 scale per 16 weights and a tensor scale, on the
+    tcgen05 GEMM.  Reports tokens/s, the speed-up over the bf16 k sweep at
+    the same context, and the low-bit GEMMs' HBM rate from a profiled pass."""
     import synth
     ev = lambda: torch.cuda.Event(enable_timing=True)
-    mx = dory.MxWeights(dw)
+    wq = dory.MxWeights(dw) if fmt == "mxfp8" else dory.NvWeights(dw)
     cfg = dory.make_config(shape, max_batch=1, max_seq=args.prompt + 8 * steps + 64, k_max=4, gamma_max=4,
                            max_chunk=args.prompt)
-    h = dory.Handle(cfg, mx.dequantised, dory.LAST_LOOP if args.mode == "last_loop" else dory.PER_LOOP)
-    h.attach_mxfp8(mx)
+    h = dory.Handle(cfg, wq.dequantised, dory.LAST_LOOP if args.mode == "last_loop" else dory.PER_LOOP)
+    (h.attach_mxfp8 if fmt == "mxfp8" else h.attach_nvfp4)(wq)
     prompt = torch.tensor(synth.make_prompt(1, args.prompt, shape.vocab), dtype=torch.int32, device="cuda")
     tok = h.prefill([0], prompt, [args.prompt], args.k, mode)
     bufs = [torch.empty(1, dtype=torch.int32, device="cuda") for _ in range(2)]
     out = {}
-    # impl 2: the tensor-core GEMV, at the bench's k only; then the default (CUDA cores) at every k
-    for impl, ks in ((2, (args.k,)), (0, (1, 2, 4))):
-        h.set_option(dory.OPT_MX_GEMV, impl)
-        for kk in ks:
+    impls = ((1, "cuda_core_gemv"), (3, "tcgen05_gemm")) if fmt == "mxfp8" else ((0, "tcgen05_gemm"),)
+    hbm = peaks()[0]
+    for impl, label in impls:
+        if fmt == "mxfp8":
+            h.set_option(dory.OPT_MX_GEMV, impl)
+        res = {}
+        for kk in (1, 2, 4):
             if args.mode == "per_loop" and kk != args.k:
                 continue
             for i in range(3):
@@ -407,32 +413,31 @@ def mxfp8_leg(dory, torch, shape, dw, args, mode, bf16_sweep, steps=32):
             ref = (bf16_sweep or {}).get(f"k{kk}")
             if ref:
                 r["speedup_vs_bf16"] = round(r["tokens_per_s"] / ref["tokens_per_s"], 3)
-            out[f"k{kk}" if impl == 0 else f"k{kk}_tensor_core_gemv"] = r
-    # the (default) GEMV's own time: CUDA events around every launch of two steps
-    h.profile_reset()
-    h.set_option(dory.OPT_PROFILE, 1)
-    for i in range(2):
-        tok = h.decode_step([0], tok, args.k, mode, next_tokens=bufs[i % 2])
-    prof = h.profile_read()
-    h.set_option(dory.OPT_PROFILE, 0)
-    gemv = {n: v for n, v in prof.items() if n.startswith("gemm")}
-    g_ms = sum(v["ms"] for v in gemv.values())
-    g_bytes = sum(v["bytes"] for v in gemv.values())
-    g_launch = sum(v["launches"] for v in gemv.values())
-    tot_ms = sum(v["ms"] for v in prof.values())
-    hbm = peaks()[0]
-    achieved = g_bytes / (g_ms / 1e3) / 1e9 if g_ms > 0 else 0.0
-    out["gemv_roofline"] = {"bound": "hbm", "kernel": "k_mx_gemv (decode projections + LM head, MXFP8)",
-                            "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                            "frac": round(achieved / hbm, 4), "bytes_per_launch": round(g_bytes / max(g_launch, 1)),
-                            "avg_launch_us": round(1e3 * g_ms / max(g_launch, 1), 2),
-                            "share_of_step": round(g_ms / tot_ms, 4) if tot_ms else None}
-    out["weight_bytes"] = mx.nbytes()
-    out["workload"] = (f"batch 1, prompt {args.prompt}, {steps} timed steps per k, {args.mode}; MXFP8 copies of "
+            res[f"k{kk}"] = r
+        # the low-bit GEMMs' own time: CUDA events around every launch of two steps
+        h.profile_reset()
+        h.set_option(dory.OPT_PROFILE, 1)
+        for i in range(2):
+            tok = h.decode_step([0], tok, args.k, mode, next_tokens=bufs[i % 2])
+        prof = h.profile_read()
+        h.set_option(dory.OPT_PROFILE, 0)
+        g = {n: v for n, v in prof.items() if n.startswith("gemm")}
+        g_ms = sum(v["ms"] for v in g.values())
+        g_bytes = sum(v["bytes"] for v in g.values())
+        g_launch = sum(v["launches"] for v in g.values())
+        tot_ms = sum(v["ms"] for v in prof.values())
+        achieved = g_bytes / (g_ms / 1e3) / 1e9 if g_ms > 0 else 0.0
+        res["gemm_hbm"] = {"achieved_GBs": round(achieved, 1), "frac": round(achieved / hbm, 4),
+                           "avg_launch_us": round(1e3 * g_ms / max(g_launch, 1), 2),
+                           "share_of_profiled_step": round(g_ms / tot_ms, 4) if tot_ms else None}
+        out[label] = res
+    out["weight_bytes"] = wq.nbytes()
+    out["workload"] = (f"batch 1, prompt {args.prompt}, {steps} timed steps per k, {args.mode}; {fmt} copies of "
                        f"every projection and the LM head (embedding bf16)")
-    out["pages_ratio"] = "MXFP8 over BF16 at batch 1 on a DGX Spark: 1.69x (in 2560 / out 300), 1.84x (in 128 / out 1024)"
+    out["pages_ratio"] = ("over BF16 at batch 1 on a DGX Spark: MXFP8 1.69x / NVFP4 2.17x (in 2560 / out 300), "
+                          "MXFP8 1.84x / NVFP4 2.44x (in 128 / out 1024)")
     h.close()
-    del mx
+    del wq
     torch.cuda.empty_cache()
     return out
 
@@ -556,6 +561,8 @@ def main():
     ap.add_argument("--fused-rows", dest="fused_rows", type=int, default=None,
                     help="operand stages for decode passes of at most this many rows (0 = off; default: the "
                          "library's)")
+    ap.add_argument("--attn-cluster", dest="attn_cluster", type=int, default=None,
+                    help="decode attention cluster size (4, 8, 16; 1 = chosen from the batch; 0 = none)")
     ap.add_argument("--batched", action="store_true",
                     help="run the batched workload instead (--batch sequences of --prompt-batched tokens, "
                          "chunked prefill, then --steps decode steps) and print its own JSON line")
@@ -616,6 +623,8 @@ def main():
         h.set_option(dory.OPT_ATTN_LOOKAHEAD, args.attn_mb << 20)
     if args.fused_rows is not None:
         h.set_option(dory.OPT_FUSED_OPERANDS, args.fused_rows)
+    if args.attn_cluster is not None:
+        h.set_option(dory.OPT_ATTN_CLUSTER, args.attn_cluster)
     mode = dory.MODES[args.mode]
     stream = torch.cuda.current_stream()
     prompt = torch.tensor(synth.make_prompt(1, args.prompt, shape.vocab), dtype=torch.int32, device="cuda")
@@ -732,7 +741,8 @@ def main():
             aux["sampling"], tok = r
         else:
             aux["sampling"] = r
-        aux["mxfp8_decode"] = leg(mxfp8_leg, dory, torch, shape, dw, args, mode, sweep)
+        aux["mxfp8_decode"] = leg(lowbit_leg, dory, torch, shape, dw, args, mode, sweep, "mxfp8")
+        aux["nvfp4_decode"] = leg(lowbit_leg, dory, torch, shape, dw, args, mode, sweep, "nvfp4")
         # ---- end to end: every step copies its input token from pinned host
         # memory and reads the chosen token back, through the public API
         pin_in = torch.empty(1, dtype=torch.int32).pin_memory()

@@ -450,7 +450,8 @@ enum {
   DORY_OPT_PREFILL_TC = 5,  /* bf16 long-chunk attention: 2 (default) tcgen05 with TMEM accumulators for
                                head_dim 128 (else as 1), 1 warp-level mma.sync, 0 CUDA cores */
   DORY_OPT_ATTN_CLUSTER = 6, /* 1 (default): decode attention as clusters of 16, 8 or 4 blocks per row and
-                                KV head, chosen from the number of sequences (process-wide) */
+                                KV head, chosen from the number of sequences; 4, 8, 16: that cluster size;
+                                0: no clusters (process-wide) */
   /* bf16 decode steps: bytes of upcoming weights each GEMM prefetches into L2
    * past its own once its loads have landed (default 8 MiB; 0 turns the
    * look-ahead off).  Changes only when HBM reads happen, never what is
@@ -459,11 +460,12 @@ enum {
   /* GEMM on attached MXFP8 copies (see dory_gemv_mxfp8's impl): 0 (default, = 1), 1 CUDA cores,
      2 mma.sync, 3 TMA-fed tcgen05 with split-K slices (matrices whose N or K it does not take use 1) */
   DORY_OPT_MX_GEMV = 8,
-  /* bf16 decode and speculative steps of at most this many rows (default 4,
-   * at most 16; 0 off): the add + L2 norm after a layer and the SwiGLU of a
+  /* bf16 decode and speculative steps of at most this many rows (default 0:
+   * off; at most 16): the add + L2 norm after a layer and the SwiGLU of a
    * split gate-up product run inside the next projection GEMM, whose
    * epilogue warps build its operand in shared memory, instead of as kernels
-   * of their own.  Same arithmetic, so the same bits, either way. */
+   * of their own.  Same arithmetic, so the same bits, either way.  Measured
+   * slower than the separate kernels at batch 1 on the 4B shape, hence off. */
   DORY_OPT_FUSED_OPERANDS = 9,
   /* bf16 decode steps: bytes of upcoming weights each decode attention
    * launch prefetches into L2 before waiting for its queries (default 0:

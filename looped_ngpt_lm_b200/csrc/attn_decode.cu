@@ -35,7 +35,7 @@ constexpr int NW = 8;  // warps per block
 
 }  // namespace
 
-bool g_attn_cluster = true;
+int g_attn_cluster = 1;
 
 namespace {
 
@@ -889,7 +889,7 @@ cudaError_t dispatch(int M, int KV, const float* qkv, int S, size_t ps, KVView k
                      cudaStream_t st, const PfCtl& pf) {
   if constexpr (sizeof(T) == 2 && HD >= 64 && G <= 16) {
     if (g_attn_cluster) {
-      const int cs = decode_cluster_size(batch, KV);
+      const int cs = g_attn_cluster >= 4 ? g_attn_cluster : decode_cluster_size(batch, KV);
       cudaError_t e = cs == 16  ? dispatch_tc<HD, G, 16>(M, KV, qkv, S, ps, kv, m, (bf16*)out, st, pf)
                       : cs == 8 ? dispatch_tc<HD, G, 8>(M, KV, qkv, S, ps, kv, m, (bf16*)out, st, pf)
                                 : dispatch_tc<HD, G, 4>(M, KV, qkv, S, ps, kv, m, (bf16*)out, st, pf);

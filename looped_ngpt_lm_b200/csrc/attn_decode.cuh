@@ -8,9 +8,11 @@ namespace dory {
 
 constexpr int DEC_BK = 128;  // keys per block (absolute-position aligned)
 
-// Use the cluster kernel (16 blocks per row and KV head, merged through
-// distributed shared memory) when the device can schedule it.
-extern bool g_attn_cluster;
+// Use the cluster kernels (blocks per row and KV head merged through
+// distributed shared memory) when the device can schedule them: 0 never,
+// 1 with the cluster size chosen from the number of sequences, 4 / 8 / 16
+// with that cluster size.
+extern int g_attn_cluster;
 
 // Attention of M rows whose K/V go straight into the cache.  qkv: the QKV
 // projection's S split-K partial slices (slice stride ps floats, rows of

@@ -181,7 +181,7 @@ struct dory_handle {
   std::vector<Graph> graphs_cache;
   cudaStream_t cap_stream = nullptr;  // private stream used only to record graphs
 
-  int fuse_rows = 4;  // operand stages for decode / speculative passes of at most this many rows (0 off)
+  int fuse_rows = 0;  // operand stages for decode / speculative passes of at most this many rows (0 off)
 
   template <typename T>
   T* hop_t() const { return (T*)hop; }
@@ -1503,7 +1503,16 @@ dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value) {
       if (value < 0 || value > 2) return fail(DORY_ERR_INVALID_ARG, "bad prefill attention kernel");
       h->prefill_tc = (int)value;
       return DORY_OK;
-    case DORY_OPT_ATTN_CLUSTER: dory::g_attn_cluster = value != 0; return DORY_OK;
+    case DORY_OPT_ATTN_CLUSTER:
+      if (value != 0 && value != 1 && value != 4 && value != 8 && value != 16)
+        return fail(DORY_ERR_INVALID_ARG, "attention cluster option must be 0, 1, 4, 8 or 16");
+      if (value != dory::g_attn_cluster) {
+        for (auto& g : h->graphs_cache)
+          if (g.exec) cudaGraphExecDestroy(g.exec);
+        h->graphs_cache.clear();
+      }
+      dory::g_attn_cluster = (int)value;
+      return DORY_OK;
     case DORY_OPT_L2_LOOKAHEAD:
       if (value < 0 || value > (1ll << 40)) return fail(DORY_ERR_INVALID_ARG, "bad look-ahead");
       if ((unsigned long long)value != h->pf_lead) {

@@ -287,7 +287,7 @@ def test_fused_operand_stages_change_no_bits(tiny_bf16, prompt, rows):
     h.set_option(dory.OPT_FUSED_OPERANDS, 16)
     got = run(0)
     got_graph = run(1)
-    h.set_option(dory.OPT_FUSED_OPERANDS, 4)
+    h.set_option(dory.OPT_FUSED_OPERANDS, 0)
     h.set_option(dory.OPT_CUDA_GRAPHS, 1)
     for g in (got, got_graph):
         assert np.array_equal(g[0], ref[0])
