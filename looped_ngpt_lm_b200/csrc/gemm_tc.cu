@@ -154,36 +154,35 @@ __device__ void prep_operand(const Prep& pp, int M, int K, SubRange rg, uint8_t*
     *reinterpret_cast<uint4*>(breg + sub * (MT * 128) + M * 128 + off * 16) = make_uint4(0u, 0u, 0u, 0u);
   }
   if constexpr (PREP == kPrepAddNorm) {
-    const int nc = K / 4;
+    // thread t runs virtual threads t + 128 j (j = 0..3): virtual warp
+    // warp(t) + 4 j, the same lane
     for (int m = 0; m < M; ++m) {
       const float* hr = pp.h_in + (size_t)m * K;
       const float* yr = pp.y + (size_t)m * pp.ldy;
-      float4 v[AN_MAXC];
-      float ss = 0.f;
+      float e[4][AN_CPT];
 #pragma unroll
-      for (int c = 0; c < AN_MAXC; ++c) {
-        const int j = t + c * AN_THREADS;
-        if (j < nc) {
-          v[c] = an_chunk(hr, yr, pp.S, pp.ps, j);
-          ss = an_squares(ss, v[c]);
-        }
+      for (int j = 0; j < 4; ++j) {
+        const float ss = an_warp_tree(an_load(hr, yr, pp.S, pp.ps, K, t + 128 * j, e[j]));
+        if ((t & 31) == 0) red[(t >> 5) + 4 * j] = ss;
       }
-      const float inv = an_inv_norm(ss, red, t, [] { bar_epi(); });
+      bar_epi();
+      const float inv = an_inv_from_warps(red);
+      bar_epi();  // red is written again for the next row
 #pragma unroll
-      for (int c = 0; c < AN_MAXC; ++c) {
-        const int j = t + c * AN_THREADS;
-        if (j < nc) {
-          const float4 o = an_scale(v[c], inv);
-          if (blockIdx.x == 0) reinterpret_cast<float4*>(pp.h_out + (size_t)m * K)[j] = o;
-          const int col = 4 * j;
-          if (col >= c_lo && col < c_hi) {
-            const int cc = col - c_lo, sub = cc / BK, ch = (cc % BK) / 8;
-            const __nv_bfloat162 a = __floats2bfloat162_rn(o.x, o.y), b = __floats2bfloat162_rn(o.z, o.w);
-            *reinterpret_cast<uint2*>(breg + sub * (MT * 128) + m * 128 + ((ch ^ (m & 7)) << 4) + (cc % 8) * 2) =
-                make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int c = 0; c < AN_CPT; ++c) {
+          const int i = t + 128 * j + c * AN_VT;
+          if (i < K) {
+            const float o = e[j][c] * inv;
+            if (blockIdx.x == 0) pp.h_out[(size_t)m * K + i] = o;
+            if (i >= c_lo && i < c_hi) {
+              const int cc = i - c_lo, sub = cc / BK, ch = (cc % BK) / 8;
+              *reinterpret_cast<bf16*>(breg + sub * (MT * 128) + m * 128 + ((ch ^ (m & 7)) << 4) + (cc % 8) * 2) =
+                  __float2bfloat16_rn(o);
+            }
           }
         }
-      }
     }
   } else {
     // SwiGLU: 16-byte chunks of 8 columns; gate columns j, up columns K + j
@@ -254,7 +253,7 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* b_ready = mma_done + 1;
   uint32_t* tmem_slot = (uint32_t*)(b_ready + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
-  float* red = (float*)(tmem_slot + 4);  // 4 floats, 16-byte aligned
+  float* red = (float*)(tmem_slot + 4);  // 16 floats (the operand stage's warp sums)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -688,7 +687,7 @@ bool gemm_tc_prep_ok(int M, int N, int K, int batch, const Prep& p) {
   if (p.mode == kPrepNone || M < 1 || M > 16 || N % BM || K % (4 * BK) || p.S < 1 || p.S > AN_MAXS || p.ldy % 4 ||
       p.ps % 4 || ((uintptr_t)p.y & 15))
     return false;
-  if (p.mode == kPrepAddNorm && (K > 4 * AN_MAXC * AN_THREADS || p.h_in == p.h_out ||
+  if (p.mode == kPrepAddNorm && (K > AN_CPT * AN_VT || p.h_in == p.h_out ||
                                  ((uintptr_t)p.h_in & 15) || ((uintptr_t)p.h_out & 15) || p.ldy < K))
     return false;
   if (p.mode == kPrepSwiglu && p.ldy < 2 * K) return false;

@@ -147,41 +147,29 @@ cudaError_t launch_embed(int M, int d, int vocab, const int* tokens, const T* E,
 }
 
 // ------------------------------------------------------------------ add + norm
-// One 128-thread block per row, 16-byte loads (the arithmetic of addnorm.cuh,
-// shared with the decode GEMM's operand stage).
+// One 512-thread block per row, one thread per virtual thread of the
+// arithmetic in addnorm.cuh (shared with the decode GEMM's operand stage).
 template <typename T>
-__global__ void __launch_bounds__(AN_THREADS) k_addnorm(int d, const float* h_in, float* h_out,
-                                                        const float* __restrict__ y, int S, size_t ps, int ldy,
-                                                        T* hop, float* copy_out) {
+__global__ void __launch_bounds__(AN_VT) k_addnorm(int d, const float* h_in, float* h_out,
+                                                   const float* __restrict__ y, int S, size_t ps, int ldy, T* hop,
+                                                   float* copy_out) {
   pdl_wait();
   pdl_trigger();
-  __shared__ float red[4];
-  const int r = blockIdx.x, t = threadIdx.x, nc = d / 4;
-  const float* hr = h_in + (size_t)r * d;
-  const float* yr = y + (size_t)r * ldy;
-  float4 v[AN_MAXC];
-  float ss = 0.f;
+  __shared__ float red[AN_VT / 32];
+  const int r = blockIdx.x, v = threadIdx.x;
+  float e[AN_CPT];
+  const float ss = an_warp_tree(an_load(h_in + (size_t)r * d, y + (size_t)r * ldy, S, ps, d, v, e));
+  if ((v & 31) == 0) red[v >> 5] = ss;
+  __syncthreads();
+  const float inv = an_inv_from_warps(red);
 #pragma unroll
-  for (int c = 0; c < AN_MAXC; ++c) {
-    const int j = t + c * AN_THREADS;
-    if (j < nc) {
-      v[c] = an_chunk(hr, yr, S, ps, j);
-      ss = an_squares(ss, v[c]);
-    }
-  }
-  const float inv = an_inv_norm(ss, red, t, [] { __syncthreads(); });
-#pragma unroll
-  for (int c = 0; c < AN_MAXC; ++c) {
-    const int j = t + c * AN_THREADS;
-    if (j < nc) {
-      const float4 o = an_scale(v[c], inv);
-      reinterpret_cast<float4*>(h_out + (size_t)r * d)[j] = o;
-      if (copy_out) reinterpret_cast<float4*>(copy_out + (size_t)r * d)[j] = o;
-      T* dst = hop + (size_t)r * d + 4 * j;
-      dst[0] = from_f<T>(o.x);
-      dst[1] = from_f<T>(o.y);
-      dst[2] = from_f<T>(o.z);
-      dst[3] = from_f<T>(o.w);
+  for (int c = 0; c < AN_CPT; ++c) {
+    const int i = v + c * AN_VT;
+    if (i < d) {
+      const float o = e[c] * inv;
+      h_out[(size_t)r * d + i] = o;
+      hop[(size_t)r * d + i] = from_f<T>(o);
+      if (copy_out) copy_out[(size_t)r * d + i] = o;
     }
   }
 }
@@ -189,8 +177,8 @@ __global__ void __launch_bounds__(AN_THREADS) k_addnorm(int d, const float* h_in
 template <typename T>
 cudaError_t launch_addnorm(int M, int d, const float* h_in, float* h_out, const float* y, int S, size_t ps, int ldy,
                            T* hop, float* copy_out, cudaStream_t st) {
-  if (d % 4 || d > 4 * AN_MAXC * AN_THREADS || S > AN_MAXS || ldy % 4 || ps % 4) return cudaErrorInvalidValue;
-  return launch(k_addnorm<T>, dim3(M), dim3(AN_THREADS), 0, st, d, h_in, h_out, y, S, ps, ldy, hop, copy_out);
+  if (d > AN_CPT * AN_VT || S > AN_MAXS) return cudaErrorInvalidValue;
+  return launch(k_addnorm<T>, dim3(M), dim3(AN_VT), 0, st, d, h_in, h_out, y, S, ps, ldy, hop, copy_out);
 }
 
 // ------------------------------------------------------------------ loop boundary
