@@ -467,9 +467,11 @@ enum {
    * of their own.  Same arithmetic, so the same bits, either way.  Measured
    * slower than the separate kernels at batch 1 on the 4B shape, hence off. */
   DORY_OPT_FUSED_OPERANDS = 9,
-  /* bf16 decode steps: bytes of upcoming weights each decode attention
-   * launch prefetches into L2 before waiting for its queries (default 0:
-   * none).  Changes only when HBM reads happen, never what is computed. */
+  /* bf16 decode steps: bytes of upcoming weights (past its own) that the O
+   * projection after each decode attention prefetches into L2 as soon as it
+   * is launched, before it waits for the attention, instead of the
+   * DORY_OPT_L2_LOOKAHEAD range after its loads (default 0: that range).
+   * Changes only when HBM reads happen, never what is computed. */
   DORY_OPT_ATTN_LOOKAHEAD = 10
 };
 dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value);

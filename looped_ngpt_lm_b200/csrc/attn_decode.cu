@@ -529,7 +529,7 @@ inline int decode_cluster_size(int batch, int KV) {
 template <int HD, int G, int CS>
 __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __restrict__ qkv, int S, size_t ps,
                                                         KVView kv, RowMeta m, bf16* __restrict__ out,
-                                                        float scale_log2, PfCtl pf) {
+                                                        float scale_log2) {
   using namespace wm;
   constexpr int CH = HD / 8;  // 16-byte chunks per row
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -604,8 +604,6 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
   };
   if (nchunk > 0) issue_cached(0);
   if (nchunk > 1) issue_cached(1);
-  // upcoming weights into L2 while this latency-bound kernel leaves HBM idle
-  if (pf.lo < pf.hi) l2_look_ahead(pf, tid, 256);
   pdl_wait();
 
   // Q tile: rows 0..G-1 = the G heads (pre-scaled, bf16), rows G..15 zero
@@ -790,7 +788,7 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
 
 template <int HD, int G, int CS>
 cudaError_t dispatch_tc(int M, int KV, const float* qkv, int S, size_t ps, KVView kv, RowMeta m, bf16* out,
-                        cudaStream_t st, const PfCtl& pf) {
+                        cudaStream_t st) {
   constexpr int SMEM = (int)sizeof(TcSmem<HD, G, CS>);
   auto kern = k_attn_decode_tc<HD, G, CS>;
   static int state = 0;
@@ -832,7 +830,7 @@ cudaError_t dispatch_tc(int M, int KV, const float* qkv, int S, size_t ps, KVVie
   cfg.attrs = at;
   cfg.numAttrs = 2;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
-  return cudaLaunchKernelEx(&cfg, kern, KV, qkv, S, ps, kv, m, out, scale_log2, pf);
+  return cudaLaunchKernelEx(&cfg, kern, KV, qkv, S, ps, kv, m, out, scale_log2);
 }
 
 template <typename T, int HD, int G>
@@ -886,13 +884,13 @@ cudaError_t dispatch_cl(int M, int KV, const float* qkv, int S, size_t ps, KVVie
 template <typename T, int HD, int G>
 cudaError_t dispatch(int M, int KV, const float* qkv, int S, size_t ps, KVView kv, RowMeta m, int max_ctx,
                      float* part, int nb_cap, int part_rows, unsigned* counters, T* out, int batch,
-                     cudaStream_t st, const PfCtl& pf) {
+                     cudaStream_t st) {
   if constexpr (sizeof(T) == 2 && HD >= 64 && G <= 16) {
     if (g_attn_cluster) {
       const int cs = g_attn_cluster >= 4 ? g_attn_cluster : decode_cluster_size(batch, KV);
-      cudaError_t e = cs == 16  ? dispatch_tc<HD, G, 16>(M, KV, qkv, S, ps, kv, m, (bf16*)out, st, pf)
-                      : cs == 8 ? dispatch_tc<HD, G, 8>(M, KV, qkv, S, ps, kv, m, (bf16*)out, st, pf)
-                                : dispatch_tc<HD, G, 4>(M, KV, qkv, S, ps, kv, m, (bf16*)out, st, pf);
+      cudaError_t e = cs == 16  ? dispatch_tc<HD, G, 16>(M, KV, qkv, S, ps, kv, m, (bf16*)out, st)
+                      : cs == 8 ? dispatch_tc<HD, G, 8>(M, KV, qkv, S, ps, kv, m, (bf16*)out, st)
+                                : dispatch_tc<HD, G, 4>(M, KV, qkv, S, ps, kv, m, (bf16*)out, st);
       if (e != cudaErrorNotSupported) return e;
     }
   }
@@ -920,12 +918,12 @@ cudaError_t dispatch(int M, int KV, const float* qkv, int S, size_t ps, KVView k
 template <typename T>
 cudaError_t launch_attn_decode(int M, int H, int KV, int hd, const float* qkv, int S, size_t ps, KVView kv,
                                RowMeta m, int max_ctx, float* part, int nb_cap, int part_rows, unsigned* counters,
-                               T* out, int batch, cudaStream_t st, const PfCtl& pf) {
+                               T* out, int batch, cudaStream_t st) {
   const int G = H / KV;
 #define DORY_DEC_CASE(HDV, GV)                                                                                   \
   if (hd == HDV && G == GV)                                                                                      \
     return dispatch<T, HDV, GV>(M, KV, qkv, S, ps, kv, m, max_ctx, part, nb_cap, part_rows, counters, out, batch, \
-                                st, pf);
+                                st);
   DORY_DEC_CASE(32, 1) DORY_DEC_CASE(32, 2) DORY_DEC_CASE(32, 4) DORY_DEC_CASE(32, 5) DORY_DEC_CASE(32, 8)
   DORY_DEC_CASE(64, 1) DORY_DEC_CASE(64, 2) DORY_DEC_CASE(64, 4) DORY_DEC_CASE(64, 5) DORY_DEC_CASE(64, 8)
   DORY_DEC_CASE(128, 1) DORY_DEC_CASE(128, 2) DORY_DEC_CASE(128, 4) DORY_DEC_CASE(128, 5)
@@ -934,9 +932,8 @@ cudaError_t launch_attn_decode(int M, int H, int KV, int hd, const float* qkv, i
 }
 
 template cudaError_t launch_attn_decode<float>(int, int, int, int, const float*, int, size_t, KVView, RowMeta, int,
-                                               float*, int, int, unsigned*, float*, int, cudaStream_t,
-                                               const PfCtl&);
+                                               float*, int, int, unsigned*, float*, int, cudaStream_t);
 template cudaError_t launch_attn_decode<bf16>(int, int, int, int, const float*, int, size_t, KVView, RowMeta, int,
-                                              float*, int, int, unsigned*, bf16*, int, cudaStream_t, const PfCtl&);
+                                              float*, int, int, unsigned*, bf16*, int, cudaStream_t);
 
 }  // namespace dory

@@ -1,7 +1,6 @@
 // Fused GQA attention for decode and speculative chunks.
 #pragma once
 
-#include "gemm_tc.cuh"
 #include "kernels.cuh"
 
 namespace dory {
@@ -21,11 +20,9 @@ extern int g_attn_cluster;
 // required); counters: [M * KV] zeros (left zero on return).  out: [M, H * hd]
 // in the storage type.  batch: sequences in the call (rows may be several
 // per sequence); selects how many blocks share one row's keys.
-// pf: upcoming weights the tensor-core kernel prefetches into L2 before it
-// waits for the QKV projection (see PfCtl; other variants ignore it).
 template <typename T>
 cudaError_t launch_attn_decode(int M, int H, int KV, int hd, const float* qkv, int S, size_t ps, KVView kv,
                                RowMeta m, int max_ctx, float* part, int nb_cap, int part_rows, unsigned* counters,
-                               T* out, int batch, cudaStream_t st, const PfCtl& pf);
+                               T* out, int batch, cudaStream_t st);
 
 }  // namespace dory

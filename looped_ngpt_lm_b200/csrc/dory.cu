@@ -161,7 +161,7 @@ struct dory_handle {
   int prefill_tc = 2;  // long-chunk attention: 2 tcgen05 (head_dim 128), 1 mma.sync, 0 CUDA cores
   int gemm_impl = 0;
   unsigned long long pf_lead = 8ull << 20;   // 0: no L2 look-ahead
-  unsigned long long pf_attn = 0;            // bytes the decode attention prefetches (0: none)
+  unsigned long long pf_attn = 0;            // early look-ahead of the GEMM after a decode attention (0: none)
   float temperature = 0.f, top_p = 1.f;      // temperature 0: greedy
   unsigned long long seed = 0;
   std::vector<std::vector<PfSeg>> pf_host;   // [k] -> stream of a k-loop decode step
@@ -441,9 +441,12 @@ size_t prows(const Fwd<T>& f) {
 // hold kMaxSplitK slices of part_rows rows of ldy floats.
 // prep: an operand stage the caller has checked with stage_ok (bf16
 // tensor-core decode GEMMs only); X is then unused.
+// after_attn: the GEMM follows a decode attention launch; its look-ahead
+// then covers pf_attn bytes and is issued before it waits (see PfCtl).
 template <typename T>
 dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, const void* W, float* Y, int ldy,
-                 size_t part_rows, int* S_out, size_t* ps_out, const char* name, const Prep* prep = nullptr) {
+                 size_t part_rows, int* S_out, size_t* ps_out, const char* name, const Prep* prep = nullptr,
+                 bool after_attn = false) {
   dory_handle* H = f.H;
   *S_out = 1;
   *ps_out = 0;
@@ -503,8 +506,10 @@ dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, cons
           pfc.segs = H->pf_segs + (size_t)(f.pf_k - 1) * H->pf_nseg_max;
           pfc.nseg = (int)v.size();
           pfc.first = H->pf_pos + 1;
+          const bool early = after_attn && H->pf_attn > 0;
+          pfc.early = early ? 1 : 0;
           pfc.lo = std::max(H->pf_done, end);
-          pfc.hi = std::min(end + H->pf_lead, total);
+          pfc.hi = std::min(end + (early ? H->pf_attn : H->pf_lead), total);
           if (pfc.lo < pfc.hi) {
             // start the segment walk at the segment holding lo
             while (pfc.first + 1 < pfc.nseg && v[pfc.first + 1].off <= pfc.lo) ++pfc.first;
@@ -537,28 +542,6 @@ dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, cons
     dory_status r_ = (x);               \
     if (r_ != DORY_OK) return r_;       \
   } while (0)
-
-// L2 look-ahead of a decode attention launch: the next pf_attn bytes of the
-// weight stream not yet handed out, starting at the next GEMM's weights (the
-// attention leaves HBM idle while it waits on latency).
-template <typename T>
-PfCtl attn_look_ahead(const Fwd<T>& f) {
-  dory_handle* H = f.H;
-  PfCtl pfc;
-  if (H->pf_attn == 0 || f.pf_k <= 0 || H->pf_pos < 0) return pfc;
-  const std::vector<PfSeg>& v = H->pf_host[f.pf_k];
-  if (H->pf_pos >= (int)v.size()) return pfc;
-  const unsigned long long total = v.back().off + v.back().bytes;
-  pfc.segs = H->pf_segs + (size_t)(f.pf_k - 1) * H->pf_nseg_max;
-  pfc.nseg = (int)v.size();
-  pfc.lo = std::max(H->pf_done, v[H->pf_pos].off);
-  pfc.hi = std::min(pfc.lo + H->pf_attn, total);
-  if (pfc.lo >= pfc.hi) return PfCtl{};
-  pfc.first = H->pf_pos;
-  while (pfc.first + 1 < pfc.nseg && v[pfc.first + 1].off <= pfc.lo) ++pfc.first;
-  H->pf_done = pfc.hi;
-  return pfc;
-}
 
 // Whether the GEMM of weight W ([N, K]) on this pass can take operand stage p.
 template <typename T>
@@ -620,10 +603,9 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop, float* copy_la
       }      if (f.direct) {
         // fused: q from the partials, own K/V into the cache, split-KV attention
         Scope sc(H, f.st, "attn_decode", 0);
-        const PfCtl apf = attn_look_ahead(f);
         CK(launch_attn_decode<T>(M, c.n_heads, c.n_kv_heads, c.head_dim, H->part_qkv, S, ps, kv, H->meta, f.max_ctx,
                                  H->attn_part, H->nb_cap, H->attn_rows, H->attn_counters, (T*)H->ao, f.batch,
-                                 f.st, apf));
+                                 f.st));
       } else {
         // long chunks: K/V into scratch, attention, then the cache commit
         const bool tc = f.n_tiles > 0;
@@ -657,7 +639,8 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop, float* copy_la
                                  f.st));
         }
       }
-      RET(gemm<T>(f, M, d, H->q_dim, (const T*)H->ao, H->q_dim, H->w_o[l], H->part_y, d, prows(f), &S, &ps, "gemm_o"));
+      RET(gemm<T>(f, M, d, H->q_dim, (const T*)H->ao, H->q_dim, H->w_o[l], H->part_y, d, prows(f), &S, &ps, "gemm_o",
+                  nullptr, f.direct));
     } else {
       bool fused = false;
       if constexpr (sizeof(T) == 2) {

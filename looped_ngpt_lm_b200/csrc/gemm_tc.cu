@@ -356,8 +356,9 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
     __syncwarp();
-    if (pf.lo < pf.hi && !*abort_flag) l2_look_ahead(pf, lane, 32);
+    if (!pf.early && pf.lo < pf.hi && !*abort_flag) l2_look_ahead(pf, lane, 32);
   } else if (warp == 1) {
+    if (pf.early && pf.lo < pf.hi) l2_look_ahead(pf, lane, 32);
     pdl_wait();
     if (lane == 0) {
       // ---------------- MMA issuer

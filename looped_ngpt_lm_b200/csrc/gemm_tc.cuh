@@ -21,11 +21,15 @@ struct PfSeg {
 // own loads have landed (CTA b takes the b-th of gridDim.x equal pieces).
 // The following attention, norms and the next GEMM's ramp-up then overlap
 // HBM reads of the weights that come next.  lo >= hi: off.
+// early: issued by the MMA warp before the launch waits for its predecessor
+// (a GEMM launched early next to a latency-bound kernel then streams the
+// following weights while HBM would idle), not after its own loads.
 struct PfCtl {
   const PfSeg* segs = nullptr;
   int nseg = 0;
   int first = 0;  // a segment at or before the one holding lo
   unsigned long long lo = 0, hi = 0;
+  int early = 0;
 };
 
 // Operand stage of a decode GEMM (M <= 16 rows).  Instead of loading X by
