@@ -92,6 +92,15 @@ def peaks():
 
 
 # ---------------------------------------------------------------- algorithmic work
+# DRAM bytes (read + write) per decode-GEMM launch from one ncu capture of the
+# decode GEMMs of a 2+2+2-layer model of the 4B width (every launch's counters,
+# weighted by the full step's launch counts: 56 each of QKV, O, gate-up, down
+# and one LM head).  Each launch's count includes the 8 MiB of the next
+# weights it prefetches into L2 (the look-ahead), which ncu's flush between
+# launches makes the next launch read again.
+GEMM_TRAFFIC_PER_LAUNCH = 58.40e6
+
+
 def weight_bytes(shape, k):
     """Weight bytes one decode step streams at loop count k (bf16)."""
     d, q, kv, f = shape.d_model, shape.q_dim, shape.kv_dim, shape.d_ff
@@ -701,7 +710,11 @@ def main():
     achieved = gs_bytes / (gs_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "kernel": "k_gemm_tc (decode projections + LM head, one token row)",
                 "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
-                "peak_source": peak_src, "traffic": None, "bytes_per_launch": round(gs_bytes / gs_n),
+                "peak_source": peak_src,
+                "traffic": GEMM_TRAFFIC_PER_LAUNCH if (shape.name == "dory4b" and args.k == 2) else None,
+                "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum per decode GEMM launch "
+                                "(algorithmic bytes + the 8 MiB L2 look-ahead of the next weights)",
+                "bytes_per_launch": round(gs_bytes / gs_n),
                 "avg_launch_us": round(1e3 * gs_ms / gs_n, 2), "launches_per_step": gs_n,
                 "gemm_ms_per_step": round(gs_ms, 4), "share_of_step": round(gs_ms / ms_step, 4),
                 "method": "the step's GEMM sequence (same weights, order, shapes and split choice) recorded into one "

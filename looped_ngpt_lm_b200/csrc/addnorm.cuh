@@ -21,29 +21,31 @@ constexpr int AN_VT = 512;   // virtual threads per row
 constexpr int AN_CPT = 8;    // elements per virtual thread: d <= 4096
 constexpr int AN_MAXS = 8;   // split-K slices
 
-// Element i of v = h + sum_{s<S} y_s for one row (y_s = y + s * ps).
-__device__ __forceinline__ float an_elem(const float* h, const float* y, int S, size_t ps, int i) {
-  float p[AN_MAXS];
-#pragma unroll
-  for (int s = 0; s < AN_MAXS; ++s) p[s] = s < S ? __ldcg(y + s * ps + i) : 0.f;
-  const float hv = __ldcg(h + i);
-  float a = 0.f;
-#pragma unroll
-  for (int s = 0; s < AN_MAXS; ++s)
-    if (s < S) a += p[s];
-  return hv + a;
-}
-
-// A virtual thread's elements and the sum of their squares.
+// A virtual thread's elements (element i of v = h + sum_{s<S} y_s, with
+// y_s = y + s * ps) and the sum of their squares.  Every load of every
+// element is issued before the first one is used (elements past d read
+// element 0 and are dropped), so a row costs one round trip to L2.
 __device__ __forceinline__ float an_load(const float* h, const float* y, int S, size_t ps, int d, int v,
                                          float (&e)[AN_CPT]) {
+  float p[AN_CPT][AN_MAXS], hv[AN_CPT];
+#pragma unroll
+  for (int c = 0; c < AN_CPT; ++c) {
+    const bool live = c * AN_VT < d;  // the same for every thread of the row
+    const int i = v + c * AN_VT < d ? v + c * AN_VT : 0;
+    hv[c] = live ? __ldcg(h + i) : 0.f;
+#pragma unroll
+    for (int s = 0; s < AN_MAXS; ++s) p[c][s] = live && s < S ? __ldcg(y + s * ps + i) : 0.f;
+  }
   float ss = 0.f;
 #pragma unroll
   for (int c = 0; c < AN_CPT; ++c) {
-    const int i = v + c * AN_VT;
+    float a = 0.f;
+#pragma unroll
+    for (int s = 0; s < AN_MAXS; ++s)
+      if (s < S) a += p[c][s];
     e[c] = 0.f;
-    if (i < d) {
-      e[c] = an_elem(h, y, S, ps, i);
+    if (v + c * AN_VT < d) {
+      e[c] = hv[c] + a;
       ss = __fmaf_rn(e[c], e[c], ss);
     }
   }

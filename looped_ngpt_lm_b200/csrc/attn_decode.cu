@@ -606,25 +606,48 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
   if (nchunk > 1) issue_cached(1);
   pdl_wait();
 
-  // Q tile: rows 0..G-1 = the G heads (pre-scaled, bf16), rows G..15 zero
-  // (unrolled: every partial load of the tile is in flight at once)
+  // Q tile: rows 0..G-1 = the G heads (pre-scaled, bf16), rows G..15 zero;
+  // the block holding the row's own position also writes the row's K and V
+  // into the cache.  Every split-K partial these need is requested before
+  // any is summed (one round trip to L2); each sum runs in slice order.
+  constexpr int QIT = (G * HD + 255) / 256;  // passes of the 256 threads that hold query elements
+  const bool own = row_ok && klo <= pos && pos <= khi;
+  float qp[QIT][kMaxSplitK], kp[kMaxSplitK];
+#pragma unroll
+  for (int it = 0; it < QIT; ++it) {
+    const int i = tid + it * 256, h = i / HD, d = i % HD;
+    const bool live = h < G && row_ok;
+    const float* src = qkv + (size_t)r * ld + (live ? (g * G + h) * HD + d : 0);
+#pragma unroll
+    for (int s = 0; s < kMaxSplitK; ++s) qp[it][s] = live && s < S ? __ldcg(src + s * ps) : 0.f;
+  }
+  {
+    const int d = tid % HD;
+    const bool live = own && tid < 2 * HD;
+    const float* src = qkv + (size_t)r * ld + (live ? qd + (tid >= HD ? kvd : 0) + g * HD + d : 0);
+#pragma unroll
+    for (int s = 0; s < kMaxSplitK; ++s) kp[s] = live && s < S ? __ldcg(src + s * ps) : 0.f;
+  }
 #pragma unroll
   for (int it = 0; it < 16 * HD / 256; ++it) {
     const int i = tid + it * 256, h = i / HD, d = i % HD;
     float val = 0.f;
-    if (h < G && row_ok) val = sum_splits(qkv + (size_t)r * ld + (g * G + h) * HD + d, S, ps) * scale_log2;
+    if (it < QIT && h < G && row_ok) {
+      float a = 0.f;
+#pragma unroll
+      for (int s = 0; s < kMaxSplitK; ++s)
+        if (s < S) a += qp[it < QIT ? it : 0][s];
+      val = a * scale_log2;
+    }
     *reinterpret_cast<bf16*>(sm.q + swz<HD>(h, d / 8) + (d % 8) * 2) = __float2bfloat16_rn(val);
   }
-  if (row_ok && klo <= pos && pos <= khi) {  // this block holds the row's own key
-    bf16* Kw = (bf16*)kv.K;
-    bf16* Vw = (bf16*)kv.V;
-    const size_t slot = kv_row(kv, seq, KV, g, pos) * HD;
-    for (int i = tid; i < 2 * HD; i += blockDim.x) {
-      const int d = i % HD;
-      const bool is_v = i >= HD;
-      const float a = sum_splits(qkv + (size_t)r * ld + qd + (is_v ? kvd : 0) + g * HD + d, S, ps);
-      (is_v ? Vw : Kw)[slot + d] = __float2bfloat16_rn(a);
-    }
+  if (own && tid < 2 * HD) {  // this block holds the row's own key
+    float a = 0.f;
+#pragma unroll
+    for (int s = 0; s < kMaxSplitK; ++s)
+      if (s < S) a += kp[s];
+    bf16* dst = (bf16*)(tid >= HD ? kv.V : kv.K);
+    dst[kv_row(kv, seq, KV, g, pos) * HD + tid % HD] = __float2bfloat16_rn(a);
   }
   __syncthreads();
   uint32_t qa[HD / 16][4];

@@ -74,6 +74,10 @@ namespace dory {
 // before touching anything an earlier kernel writes or reads.  pdl_trigger()
 // lets the next kernel in the stream start early (it still waits in its own
 // pdl_wait()).  Both are no-ops for a kernel launched without the attribute.
+// Small kernels trigger before they wait, so the projection GEMM that
+// follows them is scheduled while the GEMM before them drains and takes each
+// SM as soon as that GEMM's block there exits (a dependent grid launches only
+// once every block of this grid has started, so this cannot starve it).
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
