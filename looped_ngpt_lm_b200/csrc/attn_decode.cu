@@ -641,13 +641,24 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
     }
     *reinterpret_cast<bf16*>(sm.q + swz<HD>(h, d / 8) + (d % 8) * 2) = __float2bfloat16_rn(val);
   }
+  // a decode row's chunk holds one new key, its own: when that chunk sits in
+  // one of the first two buffers it is written from these sums (the same
+  // bits the cache gets) instead of being summed again by fill_new
+  const int ci_own = own ? (pos - klo) / TC_KC : -1;
+  const bool own_direct = own && p0 == pos && ci_own < 2;
   if (own && tid < 2 * HD) {  // this block holds the row's own key
     float a = 0.f;
 #pragma unroll
     for (int s = 0; s < kMaxSplitK; ++s)
       if (s < S) a += kp[s];
+    const bf16 b = __float2bfloat16_rn(a);
+    const int d = tid % HD;
     bf16* dst = (bf16*)(tid >= HD ? kv.V : kv.K);
-    dst[kv_row(kv, seq, KV, g, pos) * HD + tid % HD] = __float2bfloat16_rn(a);
+    dst[kv_row(kv, seq, KV, g, pos) * HD + d] = b;
+    if (own_direct) {
+      uint8_t* buf = tid >= HD ? sm.v[ci_own & 1] : sm.k[ci_own & 1];
+      *reinterpret_cast<bf16*>(buf + swz<HD>(pos - klo - ci_own * TC_KC, d / 8) + (d % 8) * 2) = b;
+    }
   }
   __syncthreads();
   uint32_t qa[HD / 16][4];
@@ -660,8 +671,8 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
   for (int i = 0; i < HD / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   float mrow[2] = {-FLT_MAX, -FLT_MAX}, lrow[2] = {0.f, 0.f};
 
-  if (nchunk > 0) fill_new(0);
-  if (nchunk > 1) fill_new(1);
+  if (nchunk > 0 && !(own_direct && ci_own == 0)) fill_new(0);
+  if (nchunk > 1 && !(own_direct && ci_own == 1)) fill_new(1);
 
 #pragma unroll 1
   for (int ci = 0; ci < nchunk; ++ci) {

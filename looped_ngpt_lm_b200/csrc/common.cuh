@@ -74,8 +74,15 @@ namespace dory {
 // before touching anything an earlier kernel writes or reads.  pdl_trigger()
 // lets the next kernel in the stream start early (it still waits in its own
 // pdl_wait()).  Both are no-ops for a kernel launched without the attribute.
-// Small kernels trigger before they wait, so the projection GEMM that
-// follows them is scheduled while the GEMM before them drains and takes each
+//
+// Ordering invariant.  The decode attention reads the row metadata (and the
+// cache) before its pdl_wait().  Kernels that wait before they trigger
+// guarantee that everything two launches back has completed when a kernel
+// launches; the kernels that open a pass (planning, embedding, stash copies,
+// loop re-injection) keep that order, so no attention launches before the
+// planning kernel of its pass has finished.  The add + norm and SwiGLU
+// kernels between two projection GEMMs trigger first instead: the GEMM that
+// follows is then scheduled while the GEMM before them drains and takes each
 // SM as soon as that GEMM's block there exits (a dependent grid launches only
 // once every block of this grid has started, so this cannot starve it).
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }

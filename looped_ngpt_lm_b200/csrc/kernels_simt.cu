@@ -20,8 +20,8 @@ namespace dory {
 // ------------------------------------------------------------------ planning
 __global__ void k_plan_uniform(int n_rows, int rps, int pos_offset, const int* seq_ids, const int* seq_len,
                                RowMeta m) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   int r = blockIdx.x * blockDim.x + threadIdx.x;
   if (r >= n_rows) return;
   int b = r / rps, i = r % rps;
@@ -42,8 +42,8 @@ cudaError_t launch_plan_uniform(int n_seq, int rps, int pos_offset, const int* s
 }
 
 __global__ void k_plan_ragged(int n_seq, const int* cu, const int* seq_ids, const int* seq_len, RowMeta m) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   int b = blockIdx.x;
   int seq = seq_ids[b];
   int r0 = cu[b], r1 = cu[b + 1];
@@ -65,8 +65,8 @@ cudaError_t launch_plan_ragged(int n_seq, int n_rows, const int* cu, const int* 
 }
 
 __global__ void k_advance(int n_seq, const int* seq_ids, int* seq_len, int delta) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < n_seq) seq_len[seq_ids[b]] += delta;
 }
@@ -77,8 +77,8 @@ cudaError_t launch_advance(int n_seq, const int* seq_ids, int* seq_len, int delt
 }
 
 __global__ void k_advance_ragged(int n_seq, const int* seq_ids, const int* cu, int* seq_len) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < n_seq) seq_len[seq_ids[b]] += cu[b + 1] - cu[b];
 }
@@ -89,8 +89,8 @@ cudaError_t launch_advance_ragged(int n_seq, const int* seq_ids, const int* cu, 
 }
 
 __global__ void k_fill_i32(int n, int* p, int v) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) p[i] = v;
 }
@@ -102,8 +102,8 @@ cudaError_t launch_fill_i32(int n, int* p, int v, cudaStream_t st) {
 }
 
 __global__ void k_split_reduce(size_t total, const float* part, int S, size_t ps, float* out) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
     float a = 0.f;
     for (int s = 0; s < S; ++s) a += part[s * ps + i];
@@ -122,8 +122,8 @@ cudaError_t launch_split_reduce(int M, int N, const float* part, int S, size_t p
 // ------------------------------------------------------------------ embedding
 template <typename T>
 __global__ void k_embed(int d, int vocab, const int* tokens, const T* E, float* h, T* hop, float* x, int* err) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   int r = blockIdx.x;
   int tok = tokens[r];
   if (tok < 0 || tok >= vocab) {
@@ -153,7 +153,7 @@ template <typename T>
 __global__ void __launch_bounds__(AN_VT) k_addnorm(int d, const float* h_in, float* h_out,
                                                    const float* __restrict__ y, int S, size_t ps, int ldy, T* hop,
                                                    float* copy_out) {
-  pdl_trigger();
+  pdl_trigger();  // see common.cuh: the next GEMM may take SMs as the last one drains
   pdl_wait();
   __shared__ float red[AN_VT / 32];
   const int r = blockIdx.x, v = threadIdx.x;
@@ -185,8 +185,8 @@ cudaError_t launch_addnorm(int M, int d, const float* h_in, float* h_out, const 
 template <typename T>
 __global__ void k_reinject(int d, float* h, const float* x, int s_src, const float* s_in, bool make_u, T* hop,
                            float* stash_s, int rps, int scols, int col0) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   __shared__ float red[33];
   const int r = blockIdx.x;
   float* hr = h + (size_t)r * d;
@@ -250,8 +250,8 @@ cudaError_t launch_reinject(int M, int d, float* h, const float* x, int s_src, c
 }
 
 __global__ void k_stash_copy(int d, float* state, float* stash, int rps, int scols, int col0, int dir) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x;
   size_t srow = (size_t)((r / rps) * scols + r % rps + col0) * d;
   for (int i = threadIdx.x; i < d; i += blockDim.x) {
@@ -272,8 +272,8 @@ cudaError_t launch_stash_copy(int M, int d, float* state, float* stash, int rps,
 template <typename T>
 __global__ void k_qkv_post(int H, int KV, int hd, const float* qkv, int S, size_t ps, float* q_out, T* kscr,
                            T* vscr, bool direct, KVView kv, RowMeta m, int max_batch, bf16* qh, float qscale) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x;
   const int qd = H * hd, kvd = KV * hd, ld = qd + 2 * kvd;
   const float* src = qkv + (size_t)r * ld;
@@ -327,8 +327,8 @@ template <typename T, int HD, int G>
 __global__ void __launch_bounds__(128) k_attn_partial(int KV, const float* __restrict__ q, const T* kscr,
                                                       const T* vscr, bool inchunk_scratch, KVView kv, RowMeta m,
                                                       float* __restrict__ part, int nb_max, float scale_log2) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   constexpr int DL = HD / 8;  // dims per lane
   __shared__ float sm_m[4][G], sm_l[4][G];
   __shared__ float sm_acc[4][G][HD];
@@ -466,8 +466,8 @@ __global__ void __launch_bounds__(128) k_attn_partial(int KV, const float* __res
 // One warp per (row, head): merge the row's key blocks in order.
 template <typename T, int HD>
 __global__ void k_attn_combine(int H, const float* __restrict__ part, int nb_max, KVView kv, RowMeta m, T* out) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x, head = blockIdx.y * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (head >= H) return;
   const int lane = threadIdx.x & 31;
@@ -542,8 +542,8 @@ cudaError_t launch_attention(int M, int H, int KV, int hd, const float* q, const
 
 template <typename T>
 __global__ void k_kv_commit(int KV, int hd, const T* kscr, const T* vscr, KVView kv, RowMeta m) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x;
   const int pos = m.pos[r], pend = m.pend[r], seq = m.seq[r];
   if (pos < pend - kv.cap) return;  // overwritten later in this chunk
@@ -570,7 +570,7 @@ cudaError_t launch_kv_commit(int M, int KV, int hd, const T* kscr, const T* vscr
 // ------------------------------------------------------------------ SwiGLU
 template <typename T>
 __global__ void k_swiglu(int dff, const float* gu, int S, size_t ps, T* act) {
-  pdl_trigger();
+  pdl_trigger();  // see common.cuh
   pdl_wait();
   const int r = blockIdx.y;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -594,8 +594,8 @@ cudaError_t launch_swiglu(int M, int dff, const float* gu, int S, size_t ps, T* 
 
 template <typename T>
 __global__ void k_gather_rows(int d, const int* rows, const T* src, T* dst) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x;
   const T* s = src + (size_t)rows[r] * d;
   for (int i = threadIdx.x; i < d; i += blockDim.x) dst[(size_t)r * d + i] = s[i];
@@ -613,8 +613,8 @@ cudaError_t launch_gather_rows(int R, int d, const int* rows, const T* src, T* d
 template <typename T>
 __global__ void __launch_bounds__(256) k_gemm_simt(int M, int N, int K, const T* __restrict__ X, int ldx,
                                                    const T* __restrict__ W, float* __restrict__ Y, int ldy) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   __shared__ float xs[16][64 + 4];
   __shared__ float ws[16][64 + 4];
   const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
@@ -676,8 +676,8 @@ __device__ __forceinline__ void am_take(float v, int i, float& best, int& bi) {
 }
 
 __global__ void __launch_bounds__(AM_THREADS) k_argmax(int V, const float* logits, int* out, bool vec) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   __shared__ float sv[AM_THREADS / 32];
   __shared__ int si[AM_THREADS / 32];
   const float* x = logits + (size_t)blockIdx.x * V;
@@ -725,8 +725,8 @@ cudaError_t launch_argmax(int R, int V, const float* logits, int* out, cudaStrea
 __global__ void k_spec_accept(int B, int gamma, int dstride, const int* seq_ids, int* seq_len, const int* drafts,
                               const int* vtok, int* pending, const SpecIo* io, unsigned long long* accepted,
                               int* flags, const int* err, cudaGraphConditionalHandle cond, int use_cond) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   __shared__ int n_unfinished;
   if (threadIdx.x == 0) n_unfinished = 0;
   __syncthreads();

@@ -60,8 +60,8 @@ __device__ unsigned long long block_sum_u64(unsigned long long v, unsigned long 
 __global__ void __launch_bounds__(SP_T) k_sample(int V, const float* logits, uint32_t* qbuf, const int* rows,
                                                  const int* seq, const int* pos, int pos_add, float scale,
                                                  double top_p, uint32_t k0, uint32_t k1, int* out, bool vec) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   extern __shared__ unsigned long long hist[];  // [SP_W][256] per-warp histograms
   __shared__ unsigned long long red[SP_W];
   __shared__ float redf[SP_W];
