@@ -174,10 +174,56 @@ __global__ void __launch_bounds__(AN_VT) k_addnorm(int d, const float* h_in, flo
   }
 }
 
+// The same arithmetic spread over a cluster of AN_CL blocks per row: block
+// rank q runs virtual threads 64q .. 64q + 63, so each SM reads an eighth
+// of the row's split-K slices (a lone block reading all of them competes on
+// its SM with the next GEMM's weight stream, which starts while it runs).
+// Every warp pushes its sum into all ranks' shared memory; after the
+// cluster barrier each rank adds the 16 sums in order.
+constexpr int AN_CL = 8;
+constexpr int AN_CL_T = AN_VT / AN_CL;
+
+__device__ __forceinline__ void an_push(float* local, unsigned rank, float v) {
+  uint32_t a = (uint32_t)__cvta_generic_to_shared(local), ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
+}
+
+template <typename T>
+__global__ void __cluster_dims__(AN_CL, 1, 1) __launch_bounds__(AN_CL_T)
+    k_addnorm_cl(int d, const float* h_in, float* h_out, const float* __restrict__ y, int S, size_t ps, int ldy,
+                 T* hop, float* copy_out) {
+  pdl_trigger();  // see common.cuh
+  pdl_wait();
+  __shared__ float red[AN_VT / 32];
+  unsigned rank;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
+  const int r = blockIdx.x / AN_CL, v = (int)rank * AN_CL_T + threadIdx.x;
+  float e[AN_CPT];
+  const float ss = an_warp_tree(an_load(h_in + (size_t)r * d, y + (size_t)r * ldy, S, ps, d, v, e));
+  if ((threadIdx.x & 31) == 0)
+    for (unsigned q = 0; q < AN_CL; ++q) an_push(&red[v >> 5], q, ss);
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  const float inv = an_inv_from_warps(red);
+#pragma unroll
+  for (int c = 0; c < AN_CPT; ++c) {
+    const int i = v + c * AN_VT;
+    if (i < d) {
+      const float o = e[c] * inv;
+      h_out[(size_t)r * d + i] = o;
+      hop[(size_t)r * d + i] = from_f<T>(o);
+      if (copy_out) copy_out[(size_t)r * d + i] = o;
+    }
+  }
+}
+
 template <typename T>
 cudaError_t launch_addnorm(int M, int d, const float* h_in, float* h_out, const float* y, int S, size_t ps, int ldy,
                            T* hop, float* copy_out, cudaStream_t st) {
   if (d > AN_CPT * AN_VT || S > AN_MAXS) return cudaErrorInvalidValue;
+  // decode-sized batches: a cluster per row; long chunks: one block per row
+  if (M <= 64) return launch(k_addnorm_cl<T>, dim3(M * AN_CL), dim3(AN_CL_T), 0, st, d, h_in, h_out, y, S, ps, ldy,
+                             hop, copy_out);
   return launch(k_addnorm<T>, dim3(M), dim3(AN_VT), 0, st, d, h_in, h_out, y, S, ps, ldy, hop, copy_out);
 }
 
