@@ -398,9 +398,9 @@ dory_status dory_quantize_nvfp4(const void* w, int32_t N, int32_t K, void* q, vo
  * tcgen05 GEMM fed by TMA: converter warps expand the codes to f16; each
  * 16-weight block accumulates in its own TMEM columns and takes its scale
  * in the epilogue.  Each y[i, n] is summed in an order fixed by K alone.
- * Requires N % 128 == 0, K % 256 == 0, x and q 16-byte aligned, ldx % 8 == 0
- * (else DORY_ERR_UNSUPPORTED); |x| < 4 (else *err_word).  Queues work on
- * `stream`. */
+ * Requires N % 128 == 0, K % 256 == 0, x, q and scales 16-byte aligned,
+ * ldx % 8 == 0 (else DORY_ERR_UNSUPPORTED); |x| < 4 (else *err_word).
+ * Queues work on `stream`. */
 dory_status dory_gemm_nvfp4(int32_t M, int32_t N, int32_t K, const void* x, int32_t ldx, const void* q,
                             const void* scales, const float* g, float* y, int32_t ldy, int32_t* err_word,
                             dory_stream stream);

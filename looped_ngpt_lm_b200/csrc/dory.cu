@@ -1621,9 +1621,9 @@ dory_status dory_gemm_nvfp4(int32_t m, int32_t n, int32_t k, const void* x, int3
                             dory_stream stream) {
   if (!x || !q || !scales || !g || !y || m < 1 || n < 1 || k < 1 || ldx < k || ldy < n)
     return fail(DORY_ERR_INVALID_ARG, "bad GEMM arguments");
-  if (n % 128 || k % 256 || ((uintptr_t)x & 15) || ldx % 8 || ((uintptr_t)q & 15))
-    return fail(DORY_ERR_UNSUPPORTED, "NVFP4 GEMM needs N %% 128 == 0, K %% 256 == 0, x and q 16-byte aligned, "
-                                      "ldx %% 8 == 0");
+  if (n % 128 || k % 256 || ((uintptr_t)x & 15) || ldx % 8 || ((uintptr_t)q & 15) || ((uintptr_t)scales & 15))
+    return fail(DORY_ERR_UNSUPPORTED, "NVFP4 GEMM needs N %% 128 == 0, K %% 256 == 0, x, q and scales 16-byte "
+                                      "aligned, ldx %% 8 == 0");
   CK(launch_nv_gemm_tc(m, n, k, (const bf16*)x, ldx, (const uint8_t*)q, (const uint8_t*)scales, g, y, ldy, 0, 1,
                        err_word, (cudaStream_t)stream));
   return DORY_OK;
@@ -1643,7 +1643,7 @@ dory_status dory_attach_nvfp4(dory_handle* h, const dory_nvfp4_weights* nv) {
       const void* sc = ss ? ss[l] : nullptr;
       const float* g = gs ? gs[l] : nullptr;
       if (!q && !sc && !g) return;  // this matrix stays bf16
-      if (!q || !sc || !g || ((uintptr_t)q & 15)) ok = false;
+      if (!q || !sc || !g || ((uintptr_t)q & 15) || ((uintptr_t)sc & 15)) ok = false;
       dory_handle::MxMat m;
       m.q = (const uint8_t*)q;
       m.s = (const uint8_t*)sc;
@@ -1664,7 +1664,7 @@ dory_status dory_attach_nvfp4(dory_handle* h, const dory_nvfp4_weights* nv) {
     const void* hs[1] = {nv->lm_head_s};
     const float* hg[1] = {nv->lm_head_g};
     add(h->head, hq, hs, hg, 0);
-    if (!ok) return fail(DORY_ERR_INVALID_ARG, "each NVFP4 copy needs codes (16-byte aligned), scales and g");
+    if (!ok) return fail(DORY_ERR_INVALID_ARG, "each NVFP4 copy needs codes and scales (16-byte aligned) and g");
   }
   for (auto& g : h->graphs_cache)
     if (g.exec) cudaGraphExecDestroy(g.exec);

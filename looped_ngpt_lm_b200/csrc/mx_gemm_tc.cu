@@ -95,16 +95,48 @@ struct Units {
   }
 };
 
-// The scale of block b of a chunk, times 2^-14 for the staged activations.
+// The scale bytes of one chunk of a weight row: 4 (MXFP8) or 16 (NVFP4).
 template <int FMT>
-__device__ __forceinline__ float block_scale(const uint8_t* srow, int c, int b, float g) {
+struct ChunkScales {
+  uint32_t w[FMT == 0 ? 1 : 4];
+};
+
+template <int FMT>
+__device__ __forceinline__ ChunkScales<FMT> load_scales(const uint8_t* srow, int c) {
+  ChunkScales<FMT> r;
   if constexpr (FMT == 0) {
-    const int e = (int)srow[c * 4 + b] - 127 - 14;
+    r.w[0] = __ldg(reinterpret_cast<const uint32_t*>(srow + c * 4));
+  } else {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(srow + c * 16));
+    r.w[0] = v.x;
+    r.w[1] = v.y;
+    r.w[2] = v.z;
+    r.w[3] = v.w;
+  }
+  return r;
+}
+
+// The scale of block b of a chunk (from its scale bytes), times 2^-14 for
+// the staged activations.
+template <int FMT>
+__device__ __forceinline__ float block_scale(const ChunkScales<FMT>& cs, int b, float g) {
+  const uint32_t byte = (cs.w[b >> 2] >> (8 * (b & 3))) & 0xFFu;
+  if constexpr (FMT == 0) {
+    const int e = (int)byte - 127 - 14;
     return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : ldexpf(1.f, e);
   } else {
-    const __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)srow[c * 16 + b], __NV_E4M3);
+    const __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)byte, __NV_E4M3);
     return __half2float(__half(h)) * g * (1.f / kXScale);
   }
+}
+
+// tcgen05.ld of 16 columns without the wait (the caller waits once for a group).
+__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
 }
 
 template <int FMT>
@@ -279,27 +311,50 @@ __global__ void __launch_bounds__(NTH, 1)
       float acc[MT];
 #pragma unroll
       for (int t = 0; t < MT; ++t) acc[t] = 0.f;
-      for (int c = c0; c < c1; ++c) {
-        if (!mbar_wait(&tfull[tsl], tph, abort_flag, err)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-#pragma unroll 4
-        for (int b = 0; b < F::NB; ++b) {
-          float v[16];
-          tmem_ld16(tmem_base + ((uint32_t)lane_base << 16) + tsl * F::SLOT + b * MT, v);
-          const float sc = block_scale<FMT>(srow, c, b, g);
+      // the row's scale bytes are fetched kSA chunks ahead (a ring in
+      // registers), so no chunk waits on a global load
+      constexpr int kSA = 4;
+      ChunkScales<FMT> ring[kSA];
 #pragma unroll
-          for (int t = 0; t < MT; ++t) acc[t] = __fmaf_rn(v[t], sc, acc[t]);
+      for (int j = 0; j < kSA; ++j)
+        if (c0 + j < c1) ring[j] = load_scales<FMT>(srow, c0 + j);
+      for (int c = c0; c < c1; c += kSA) {
+#pragma unroll
+        for (int j = 0; j < kSA; ++j) {
+          if (c + j >= c1) break;
+          const ChunkScales<FMT> cs = ring[j];
+          if (c + j + kSA < c1) ring[j] = load_scales<FMT>(srow, c + j + kSA);
+          if (!mbar_wait(&tfull[tsl], tph, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          // the chunk's block accumulators, four blocks per wait
+#pragma unroll
+          for (int b0 = 0; b0 < F::NB; b0 += 4) {
+            uint32_t v[4][16];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (b0 + q < F::NB)
+                tmem_ld16_nowait(tmem_base + ((uint32_t)lane_base << 16) + tsl * F::SLOT + (b0 + q) * MT, v[q]);
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (b0 + q >= F::NB) break;
+              const float sc = block_scale<FMT>(cs, b0 + q, g);
+#pragma unroll
+              for (int t = 0; t < MT; ++t) acc[t] = __fmaf_rn(__uint_as_float(v[q][t]), sc, acc[t]);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[tsl]);
+          if (++tsl == TS) {
+            tsl = 0;
+            tph ^= 1;
+          }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[tsl]);
-        if (++tsl == TS) {
-          tsl = 0;
-          tph ^= 1;
-        }
+        if (!ok) break;
       }
       if (!ok) break;
       float* out = Y + (size_t)s * part_stride + n;
@@ -430,7 +485,9 @@ cudaError_t run_lowbit(int M, int N, int K, const bf16* X, int ldx, const uint8_
                        const float* g, float* Y, int ldy, size_t part_stride, int S, int* err, cudaStream_t st) {
   using F = Fmt<FMT>;
   const long long row_bytes = FMT == 0 ? K : K / 2;
-  if (M < 1 || N % BM || K % F::CK || ((uintptr_t)q & 15) || ((uintptr_t)X & 15) || (ldx * 2) % 16)
+  // the epilogue reads a chunk's scale bytes as one 4-byte (MXFP8) or 16-byte (NVFP4) word
+  if (M < 1 || N % BM || K % F::CK || ((uintptr_t)q & 15) || ((uintptr_t)X & 15) || (ldx * 2) % 16 ||
+      ((uintptr_t)scales & (FMT == 0 ? 3 : 15)))
     return cudaErrorNotSupported;
   EncodeFn fn = encode();
   if (!fn) return cudaErrorNotSupported;
