@@ -508,7 +508,7 @@ struct TcSmem {
   float wm[NW][G], wl[NW][G];
   float wacc[NW][G][HD];
   float part[G][HD + 2];
-  float all[CS][G][HD + 2];  // rank 0: every rank's partial, pushed by the ranks
+  float all[CS][G][HD + 2];  // every rank's (max, sum) and this rank's dimensions of its accumulator
   float rw[CS][G];
   float rinv[G];
 };
@@ -791,13 +791,24 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
     sm.part[h][2 + d] = a;
   }
   __syncthreads();
-  // push this block's partial into rank 0's shared memory (stores only)
-  for (int i = tid; i < G * (HD + 2); i += blockDim.x) {
-    const int h = i / (HD + 2), c = i % (HD + 2);
-    dsmem_st(&sm.all[rank][h][c], 0, sm.part[h][c]);
+  // every rank merges HD / CS of the head dimensions: each block pushes its
+  // (max, sum) pair to every rank and each of its accumulator elements to
+  // the rank that owns that dimension (stores only), then, after one cluster
+  // barrier, each rank reads only its own shared memory and writes its slice
+  // of the output.  The merge runs in rank order, the same sums as a single
+  // merging block.
+  static_assert(HD % CS == 0, "head dimensions split evenly over the cluster");
+  constexpr int DS = HD / CS;  // head dimensions per rank
+  for (int i = tid; i < CS * G * 2; i += blockDim.x) {
+    const int q = i / (G * 2), e = i % (G * 2);
+    dsmem_st(&sm.all[rank][e >> 1][e & 1], q, sm.part[e >> 1][e & 1]);
   }
-  cluster_sync();  // every partial has landed in rank 0
-  if (rank == 0 && row_ok) {
+  for (int i = tid; i < G * HD; i += blockDim.x) {
+    const int h = i / HD, d = i % HD;
+    dsmem_st(&sm.all[rank][h][2 + d], d / DS, sm.part[h][2 + d]);
+  }
+  cluster_sync();  // every partial has landed where it is merged
+  if (row_ok) {
     if (tid < G) {
       float M = -FLT_MAX;
       for (int q = 0; q < CS; ++q) M = fmaxf(M, sm.all[q][tid][0]);
@@ -811,8 +822,8 @@ __global__ void __launch_bounds__(256) k_attn_decode_tc(int KV, const float* __r
       sm.rinv[tid] = 1.f / L;
     }
     __syncthreads();
-    for (int i = tid; i < G * HD; i += blockDim.x) {
-      const int h = i / HD, d = i % HD;
+    for (int i = tid; i < G * DS; i += blockDim.x) {
+      const int h = i / DS, d = rank * DS + i % DS;
       float a = 0.f;
       for (int q = 0; q < CS; ++q) a += sm.all[q][h][2 + d] * sm.rw[q][h];
       out[(size_t)r * qd + (g * G + h) * HD + d] = __float2bfloat16_rn(a * sm.rinv[h]);
@@ -969,5 +980,11 @@ template cudaError_t launch_attn_decode<float>(int, int, int, int, const float*,
                                                float*, int, int, unsigned*, float*, int, cudaStream_t);
 template cudaError_t launch_attn_decode<bf16>(int, int, int, int, const float*, int, size_t, KVView, RowMeta, int,
                                               float*, int, int, unsigned*, bf16*, int, cudaStream_t);
+
+int attn_decode_ctas(int batch, int KV, int hd, int G) {
+  if (!g_attn_cluster || hd < 64 || G > 16) return 0;
+  const int cs = g_attn_cluster >= 4 ? g_attn_cluster : decode_cluster_size(batch, KV);
+  return batch * KV * cs;
+}
 
 }  // namespace dory

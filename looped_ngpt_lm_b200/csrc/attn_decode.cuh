@@ -20,6 +20,10 @@ extern int g_attn_cluster;
 // required); counters: [M * KV] zeros (left zero on return).  out: [M, H * hd]
 // in the storage type.  batch: sequences in the call (rows may be several
 // per sequence); selects how many blocks share one row's keys.
+// Blocks the bf16 tensor-core decode attention runs for one row per
+// sequence of `batch` sequences (0 when it would not run).
+int attn_decode_ctas(int batch, int KV, int hd, int G);
+
 template <typename T>
 cudaError_t launch_attn_decode(int M, int H, int KV, int hd, const float* qkv, int S, size_t ps, KVView kv,
                                RowMeta m, int max_ctx, float* part, int nb_cap, int part_rows, unsigned* counters,

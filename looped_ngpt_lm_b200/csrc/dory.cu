@@ -521,8 +521,14 @@ dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, cons
           H->pf_pos = -1;  // the pass left the stream: no further look-ahead
         }
       }
+      // the projection after a decode attention leaves the attention's SMs free
+      int cap = 0;
+      if (after_attn && f.invariant) {
+        const int busy = attn_decode_ctas(f.batch, H->c.n_kv_heads, H->c.head_dim, H->c.n_heads / H->c.n_kv_heads);
+        cap = busy > 0 && busy < 148 ? 148 - busy : 0;
+      }
       cudaError_t e = launch_gemm_tc(M, N, K, (const bf16*)X, ldx, (const bf16*)W, Y, ldy, part_rows,
-                                     H->err, f.batch, f.invariant, &S, &ps, f.st, 0, false, pp, prep);
+                                     H->err, f.batch, f.invariant, &S, &ps, f.st, 0, false, pp, prep, cap);
       if (e == cudaSuccess) {
         *S_out = S;
         *ps_out = ps;
@@ -600,7 +606,8 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop, float* copy_la
       if (pre) {
         H->hc ^= 1;
         pend = false;
-      }      if (f.direct) {
+      }
+      if (f.direct) {
         // fused: q from the partials, own K/V into the cache, split-KV attention
         Scope sc(H, f.st, "attn_decode", 0);
         CK(launch_attn_decode<T>(M, c.n_heads, c.n_kv_heads, c.head_dim, H->part_qkv, S, ps, kv, H->meta, f.max_ctx,

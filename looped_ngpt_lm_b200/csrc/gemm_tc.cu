@@ -585,9 +585,15 @@ cudaError_t run(const CUtensorMap& ma, const bf16* X, int ldx, int M, int K, flo
 // dealt round-robin to one CTA per SM; the model charges the larger of the
 // whole GEMM at HBM speed and the busiest CTA at one SM's streaming rate,
 // plus the partial sums' HBM traffic.
-int choose_split(int N, int K, int batch, int kstages) {
+// cap > 0: prefer splits whose units fit in `cap` CTAs (see launch_gemm_tc).
+int choose_split(int N, int K, int batch, int kstages, int cap = 0) {
   const double hbm = 6.5e12, sm_bw = 5.5e10;
   const int tiles = N / BM, sms = sm_count();
+  if (cap > 0 && tiles <= cap) {
+    int S = 1;
+    while (S + 1 <= kMaxSplitK && S + 1 <= kstages && tiles * (S + 1) <= cap) ++S;
+    return S;
+  }
   // partial-sum traffic is charged for one row per sequence (plain decode);
   // a speculative verify chunk has gamma + 1 rows per sequence and pays more
   const double rows = batch;
@@ -705,7 +711,8 @@ bool gemm_tc_prep_ok(int M, int N, int K, int batch, const Prep& p) {
 
 cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf16* W, float* Y, int ldy,
                            size_t part_rows, int* err, int batch, bool invariant, int* S_out, size_t* ps_out,
-                           cudaStream_t st, int variant, bool packed, const PfCtl* pf, const Prep* prep) {
+                           cudaStream_t st, int variant, bool packed, const PfCtl* pf, const Prep* prep,
+                           int cta_cap) {
   *S_out = 1;
   *ps_out = 0;
   const bool staged = prep && prep->mode != kPrepNone;
@@ -734,7 +741,7 @@ cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf
     const int ksub = (variant == 1 || !g256) ? 1 : (NG >= 8 ? 1 : (NG >= 2 ? 2 : kDecodeKsub));
     um.KBg = g256 ? K / (4 * BK) : K / BK;
     um.gran = g256 ? 4 / (staged ? 2 : ksub) : 1;
-    const int S = choose_split(N, K, batch, um.KBg);
+    const int S = choose_split(N, K, batch, um.KBg, staged ? 0 : cta_cap);
     if (S > um.KBg) return cudaErrorNotSupported;
     const size_t ps = part_rows * (size_t)ldy;
     um.S = S;

@@ -88,10 +88,15 @@ __device__ __forceinline__ void l2_look_ahead(const PfCtl& pf, int t, int nthrea
 // (the caller then runs the elementwise step and a plain GEMM).  A GEMM with
 // an operand stage computes the same bits as the plain one on the operand
 // the standalone kernels would have written.
+// cta_cap (decode tiles): when the weight tiles allow it, split K only so
+// far that the units fit in this many CTAs, leaving the other SMs to a
+// kernel that runs alongside (the decode attention that precedes an O
+// projection: the whole projection then loads its weights while the
+// attention runs).  Depends on the number of sequences only, never on M.
 cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const bf16* W, float* Y, int ldy,
                            size_t part_rows, int* err, int batch, bool invariant, int* S, size_t* part_stride,
                            cudaStream_t st, int variant = 0, bool packed = false, const PfCtl* pf = nullptr,
-                           const Prep* prep = nullptr);
+                           const Prep* prep = nullptr, int cta_cap = 0);
 
 // act[m, j] = silu(g) * u (bf16, row stride dff) with g = X[m] . Wgu[j] and
 // u = X[m] . Wgu[dff + j] for the concatenated [gate; up] weight Wgu
