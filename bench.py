@@ -570,6 +570,8 @@ def main():
     ap.add_argument("--fused-rows", dest="fused_rows", type=int, default=None,
                     help="operand stages for decode passes of at most this many rows (0 = off; default: the "
                          "library's)")
+    ap.add_argument("--prefill-tc", dest="prefill_tc", type=int, default=None,
+                    help="prefill attention kernel (DORY_OPT_PREFILL_TC; default: the library's)")
     ap.add_argument("--attn-cluster", dest="attn_cluster", type=int, default=None,
                     help="decode attention cluster size (4, 8, 16; 1 = chosen from the batch; 0 = none)")
     ap.add_argument("--batched", action="store_true",
@@ -634,6 +636,8 @@ def main():
         h.set_option(dory.OPT_FUSED_OPERANDS, args.fused_rows)
     if args.attn_cluster is not None:
         h.set_option(dory.OPT_ATTN_CLUSTER, args.attn_cluster)
+    if args.prefill_tc is not None:
+        h.set_option(dory.OPT_PREFILL_TC, args.prefill_tc)
     mode = dory.MODES[args.mode]
     stream = torch.cuda.current_stream()
     prompt = torch.tensor(synth.make_prompt(1, args.prompt, shape.vocab), dtype=torch.int32, device="cuda")
@@ -856,6 +860,8 @@ def batched_leg(args):
     cfg = dory.make_config(shape, max_batch=B, max_seq=P + steps + warm + 64, k_max=2, gamma_max=0,
                            max_chunk=chunk)
     h = dory.Handle(cfg, dw, dory.LAST_LOOP)
+    if args.prefill_tc is not None:
+        h.set_option(dory.OPT_PREFILL_TC, args.prefill_tc)
     ws_gb = dory.workspace_size(cfg, dory.LAST_LOOP) / 1e9
     prompts = torch.tensor(synth.make_prompt(1, B * P, shape.vocab), dtype=torch.int32).view(B, P).cuda()
     ev = lambda: torch.cuda.Event(enable_timing=True)

@@ -447,8 +447,10 @@ enum {
   DORY_OPT_PROFILE = 2,     /* 1: time every launch with CUDA events (slow) */
   DORY_OPT_GEMM_IMPL = 3,   /* bf16 GEMM: 0 auto, 1 SIMT reference kernel, 2 tcgen05 */
   DORY_OPT_PDL = 4,         /* 1 (default): programmatic dependent launches (process-wide) */
-  DORY_OPT_PREFILL_TC = 5,  /* bf16 long-chunk attention: 2 (default) tcgen05 with TMEM accumulators for
-                               head_dim 128 (else as 1), 1 warp-level mma.sync, 0 CUDA cores */
+  DORY_OPT_PREFILL_TC = 5,  /* bf16 long-chunk attention, head_dim 128 (other widths as 1): 3 (default)
+                               warp-specialised tcgen05, two 128-row query slots per CTA sharing a
+                               TMA-fed key/value stream, P kept in TMEM; 2 tcgen05, one slot per CTA;
+                               1 warp-level mma.sync; 0 CUDA cores */
   DORY_OPT_ATTN_CLUSTER = 6, /* 1 (default): decode attention as clusters of 16, 8 or 4 blocks per row and
                                 KV head, chosen from the number of sequences; 4, 8, 16: that cluster size;
                                 0: no clusters (process-wide) */

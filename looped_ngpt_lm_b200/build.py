@@ -10,8 +10,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdory.so")
 SOURCES = ["dory.cu", "kernels_simt.cu", "gemm_tc.cu", "attn_decode.cu", "attn_prefill.cu", "attn_prefill_tc.cu",
-           "gemm_noalloc.cu", "sample.cu", "mxfp8.cu",
-           "mx_gemm_tc.cu", "nvfp4.cu"]
+           "attn_prefill_ws.cu", "gemm_noalloc.cu", "sample.cu", "mxfp8.cu", "mx_gemm_tc.cu", "nvfp4.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

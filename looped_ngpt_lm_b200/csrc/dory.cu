@@ -122,8 +122,10 @@ struct dory_handle {
   size_t ws_bytes = 0;
   int *seq_len = nullptr, *err = nullptr, *seq_ids = nullptr, *tokens = nullptr, *next = nullptr;
   int *cu = nullptr, *head_rows = nullptr;
-  int2* tiles = nullptr;  // prefill attention tiles (64 rows of one sequence)
+  int2* tiles = nullptr;  // prefill attention tiles (64 or 128 rows of one sequence)
   int tiles_cap = 0;
+  int4* pf_items = nullptr;  // warp-specialised prefill attention: CTA work items
+  int items_cap = 0;
   void* qh = nullptr;     // bf16 pre-scaled queries of long chunks
   RowMeta meta{};
   // the state h lives in one of two buffers: a GEMM that applies the
@@ -154,11 +156,13 @@ struct dory_handle {
   int* page_table = nullptr;
   int pt_stride = 0, page_shift = 0, pool_pages = 0;
   std::vector<int> pt_host, free_pages;
+  std::vector<int4> items_host;
   std::vector<std::vector<int>> seq_pages;
   std::vector<int> ids_on_device;     // seq ids last uploaded to seq_ids
   int last_rows = 0;
   bool graphs = true, profile = false;
-  int prefill_tc = 2;  // long-chunk attention: 2 tcgen05 (head_dim 128), 1 mma.sync, 0 CUDA cores
+  int prefill_tc = 3;  // long-chunk attention: 3 warp-specialised tcgen05, 2 one-slot tcgen05 (head_dim 128),
+                       // 1 mma.sync, 0 CUDA cores
   int gemm_impl = 0;
   unsigned long long pf_lead = 8ull << 20;   // 0: no L2 look-ahead
   unsigned long long pf_attn = 0;            // early look-ahead of the GEMM after a decode attention (0: none)
@@ -277,6 +281,8 @@ size_t layout(dory_handle* h) {
   h->head_rows = cv.take<int>(sizeof(int) * h->head_max);
   h->tiles_cap = M / 64 + c.max_batch + 1;
   h->tiles = cv.take<int2>(sizeof(int2) * h->tiles_cap);
+  h->items_cap = h->tiles_cap * c.n_heads;
+  h->pf_items = cv.take<int4>(sizeof(int4) * h->items_cap);
   h->qh = cv.take<char>(2 * (size_t)M * h->q_dim);
   h->meta.seq = cv.take<int>(sizeof(int) * M);
   h->meta.pos = cv.take<int>(sizeof(int) * M);
@@ -373,7 +379,8 @@ struct Fwd {
   int batch;    // sequences in the call (selects the GEMM split)
   bool invariant;  // decode / speculative rows: GEMM arithmetic independent of M
   int n_tiles = 0;  // > 0: long-chunk attention on the tensor cores over H->tiles
-  bool tc5 = false; // ... by the tcgen05 kernel (128-row tiles)
+  int tc5 = 0;      // ... by a tcgen05 kernel (128-row tiles): 2 one slot per CTA, 3 warp-specialised
+  int n_items = 0;  // work items of the warp-specialised kernel (H->pf_items)
   int pf_k = 0;     // > 0: GEMMs follow the weight stream of a pf_k-loop decode step
   bool stage = true;  // layer updates may run in the next GEMM's operand stage
 };
@@ -394,6 +401,13 @@ KVView kv_view(dory_handle* H, int l, int loop, int mode) {
     v.page_shift = H->page_shift;
   }
   return v;
+}
+
+// Rows of head_dim elements in one K (or V) buffer of layer l's cache.
+size_t kv_rows(dory_handle* H, int l) {
+  const AttnLayer& a = H->attn[H->attn_of[l]];
+  if (a.full && H->page_table) return (size_t)H->pool_pages * H->c.n_kv_heads * (1 << H->page_shift);
+  return (size_t)H->c.max_batch * H->c.n_kv_heads * a.cap;
 }
 
 // Paged cache: give every listed sequence the pages that hold positions
@@ -623,7 +637,11 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop, float* copy_la
         }
         if (tc) {
           Scope sc(H, f.st, "attn_prefill", 0);
-          if (f.tc5)
+          if (f.tc5 == 3)
+            CK(launch_attn_prefill_ws(f.n_items, H->pf_items, H->tiles, M, c.n_heads, c.n_kv_heads, c.head_dim,
+                                      (const bf16*)H->qh, (const bf16*)H->kscr, (const bf16*)H->vscr, kv,
+                                      kv_rows(H, l), H->meta, (bf16*)H->ao, f.st));
+          else if (f.tc5 == 2)
             CK(launch_attn_prefill_tc(f.n_tiles, H->tiles, c.n_heads, c.n_kv_heads, c.head_dim, (const bf16*)H->qh,
                                       (const bf16*)H->kscr, (const bf16*)H->vscr, kv, H->meta, (bf16*)H->ao, f.st));
           else
@@ -843,12 +861,27 @@ dory_status prefill_t(dory_handle* H, int batch, const int32_t* seq_ids, const i
   // whose split-KV partials hold attn_rows rows)
   Fwd<T> f{H, st, M, max_ctx, max_len <= H->slack + 1 && M <= H->attn_rows, mode, k, batch, false};
   if (!f.direct && H->bf16 && attn_prefill_supported(c.head_dim) && H->prefill_tc) {
-    f.tc5 = H->prefill_tc >= 2 && attn_prefill_tc_supported(c.head_dim);
+    f.tc5 = H->prefill_tc >= 2 && attn_prefill_tc_supported(c.head_dim) ? H->prefill_tc : 0;
     std::vector<int2> tl(H->tiles_cap);
     const int n = prefill_tiles(batch, cu.data(), tl.data(), H->tiles_cap, f.tc5 ? 128 : 64);
     if (n < 0) return fail(DORY_ERR_CAPACITY, "too many prefill attention tiles");
     CK(cudaMemcpyAsync(H->tiles, tl.data(), sizeof(int2) * n, cudaMemcpyHostToDevice, st));
     f.n_tiles = n;
+    if (f.tc5 == 3) {
+      // each tile's sequence and last position, for pairing and ordering
+      std::vector<int> last(n), sq(n);
+      for (int t = 0, b = 0; t < n; ++t) {
+        while (tl[t].x >= cu[b + 1]) ++b;
+        sq[t] = b;
+        last[t] = H->len[seq_ids[b]] + (tl[t].y - 1 - cu[b]);
+      }
+      H->items_host.resize(H->items_cap);
+      const int ni = prefill_ws_items(n, last.data(), sq.data(), c.n_heads, c.n_kv_heads, H->items_host.data(),
+                                      H->items_cap);
+      if (ni < 0) return fail(DORY_ERR_CAPACITY, "too many prefill attention items");
+      CK(cudaMemcpyAsync(H->pf_items, H->items_host.data(), sizeof(int4) * ni, cudaMemcpyHostToDevice, st));
+      f.n_items = ni;
+    }
   }
   RET(input_block<T>(f, tokens));
   RET(loops<T>(f, 1, k, -1, 1));
@@ -1490,7 +1523,7 @@ dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value) {
     case DORY_OPT_PROFILE: h->profile = value != 0; return DORY_OK;
     case DORY_OPT_PDL: dory::g_pdl = value != 0; return DORY_OK;
     case DORY_OPT_PREFILL_TC:
-      if (value < 0 || value > 2) return fail(DORY_ERR_INVALID_ARG, "bad prefill attention kernel");
+      if (value < 0 || value > 3) return fail(DORY_ERR_INVALID_ARG, "bad prefill attention kernel");
       h->prefill_tc = (int)value;
       return DORY_OK;
     case DORY_OPT_ATTN_CLUSTER:

@@ -55,7 +55,7 @@ def test_small128_chunked_prefill_and_decode(small, k, mode):
     check_bf16_tokens(toks, ora)
 
 
-@pytest.mark.parametrize("tc", [0, 1, 2])  # CUDA cores, mma.sync, tcgen05
+@pytest.mark.parametrize("tc", [0, 1, 2, 3])  # CUDA cores, mma.sync, tcgen05 one slot, warp-specialised
 def test_small128_prefill_state_both_attention_kernels(small, tc):
     model, _, h = small
     prompt = synth.make_prompt(6, 150, SHAPE.vocab)
@@ -63,7 +63,7 @@ def test_small128_prefill_state_both_attention_kernels(small, tc):
     h.reset()
     h.prefill([0], torch.tensor(prompt, dtype=torch.int32, device="cuda"), [150], 2, dory.LAST_LOOP)
     s = h.read_state("s", 150).cpu().numpy()
-    h.set_option(dory.OPT_PREFILL_TC, 2)
+    h.set_option(dory.OPT_PREFILL_TC, 3)
     tr = {}
     O.forward_chunk(model, O.Cache(model, 160), prompt, 2, O.LAST_LOOP, trace=tr)
     assert cosine_rows(s, tr["s"][-1]).min() >= 0.999
