@@ -111,6 +111,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
       "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // D (TMEM) (+)= A (TMEM, M x 16 bf16 as 8 columns of pairs) * B (shared memory descriptor).
@@ -153,8 +161,8 @@ struct Slot {
   int r0, nrows, head, pf, pl, a, b;  // a..b: key tiles this slot reads (relative to kt0)
 };
 
-// 320 threads x 200 registers fit one CTA per SM.
-__global__ void __maxnreg__(200)
+// Ten warps: three share a scheduler, whose 16K registers cap a thread at 168.
+__global__ void __launch_bounds__(NTH, 1)
     k_attn_prefill_ws(int KV, int G, const __grid_constant__ CUtensorMap map_q,
                       const __grid_constant__ CUtensorMap map_ks, const __grid_constant__ CUtensorMap map_vs,
                       const __grid_constant__ CUtensorMap map_kc, const __grid_constant__ CUtensorMap map_vc,
@@ -430,16 +438,16 @@ __global__ void __maxnreg__(200)
       l *= factor;
       float rs = 0.f;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {  // P over the first 64 columns of S, 32 columns (64 keys) at a time
-        uint32_t pk[32];
+      for (int h = 0; h < 4; ++h) {  // P over the first 64 columns of S, 16 columns (32 keys) at a time
+        uint32_t pk[16];
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float x0 = ex2(__uint_as_float(r[64 * h + c]) - m_used);
-          const float x1 = ex2(__uint_as_float(r[64 * h + c + 1]) - m_used);
+        for (int c = 0; c < 32; c += 2) {
+          const float x0 = ex2(__uint_as_float(r[32 * h + c]) - m_used);
+          const float x1 = ex2(__uint_as_float(r[32 * h + c + 1]) - m_used);
           rs += x0 + x1;
           pk[c / 2] = pack2(x0, x1);
         }
-        tmem_st32(lane_addr + s_col + 32 * h, pk);
+        tmem_st16(lane_addr + s_col + 16 * h, pk);
       }
       l += rs;
       tmem_wait_st();
