@@ -9,6 +9,10 @@
 //   warp 9     loader: Q once, then K and V tiles of 128 keys into a
 //              two-stage ring, by TMA when a tile is one run of rows of the
 //              chunk scratch or of the cache, else by cp.async row by row
+//   warps 10-11 idle (they complete the third warpgroup)
+// The CTA launches with 168 registers a thread; the third warpgroup gives
+// back all but 72 and the softmax warpgroups take them (216 each), enough to
+// hold a row of S.
 //
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
 // Per key tile j the MMA lane issues, for each slot q in turn,
@@ -50,7 +54,9 @@ constexpr int HDT = 128;               // head dimensions
 constexpr int TQ = 128;                // query rows per slot
 constexpr int TK = 128;                // keys per tile
 constexpr int NS = 2;                  // K/V ring stages
-constexpr int NTH = 320;               // 10 warps
+constexpr int NTH = 384;               // 12 warps, three warpgroups
+constexpr int REG_SOFTMAX = 216, REG_OTHER = 72;  // 2 x 128 x 216 + 128 x 72 = 384 x 168
+static_assert(2 * 128 * REG_SOFTMAX + 128 * REG_OTHER <= NTH * 168, "register split exceeds the launch's registers");
 constexpr int PANEL = 128 * 128;       // 64 head dims x 128 rows, bytes
 constexpr int TILE = 2 * PANEL;        // one Q, K or V tile, bytes
 constexpr float kLazy = 8.f;
@@ -145,6 +151,44 @@ __device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr, uint32_t panel
   return d;
 }
 
+// Packed fp32 pairs (one instruction for two lanes of arithmetic):
+// (x, y) = (a0 - b, a1 - b) and (x, y) += (a0, a1).
+__device__ __forceinline__ void sub2(float& x, float& y, float a0, float a1, float b) {
+  asm("{.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %4};\n\tsub.rn.f32x2 d, a, b;\n\t"
+      "mov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(x), "=f"(y)
+      : "f"(a0), "f"(a1), "f"(b));
+}
+__device__ __forceinline__ void add2(float& x, float& y, float a0, float a1) {
+  asm("{.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tadd.rn.f32x2 d, a, b;\n\t"
+      "mov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(x), "=f"(y)
+      : "f"(x), "f"(y), "f"(a0), "f"(a1));
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Maximum of a row of 128 values held as bits, by three-input maxima.
+__device__ __forceinline__ float row_max(const uint32_t (&r)[128]) {
+  float m[43];
+#pragma unroll
+  for (int i = 0; i < 42; ++i)
+    m[i] = max3(__uint_as_float(r[3 * i]), __uint_as_float(r[3 * i + 1]), __uint_as_float(r[3 * i + 2]));
+  m[42] = fmaxf(__uint_as_float(r[126]), __uint_as_float(r[127]));
+  float n[15];
+#pragma unroll
+  for (int i = 0; i < 14; ++i) n[i] = max3(m[3 * i], m[3 * i + 1], m[3 * i + 2]);
+  n[14] = m[42];
+  float p[5];
+#pragma unroll
+  for (int i = 0; i < 5; ++i) p[i] = max3(n[3 * i], n[3 * i + 1], n[3 * i + 2]);
+  return fmaxf(max3(p[0], p[1], p[2]), fmaxf(p[3], p[4]));
+}
+
 // A bounded wait taken by every lane of a warp, with one outcome for all of
 // them (the warp-wide TMEM accesses and __syncwarp that follow need every lane).
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err) {
@@ -161,7 +205,8 @@ struct Slot {
   int r0, nrows, head, pf, pl, a, b;  // a..b: key tiles this slot reads (relative to kt0)
 };
 
-// Ten warps: three share a scheduler, whose 16K registers cap a thread at 168.
+// 12 warps: three share a scheduler, whose 16K registers cap a thread at 168
+// at launch.
 __global__ void __launch_bounds__(NTH, 1)
     k_attn_prefill_ws(int KV, int G, const __grid_constant__ CUtensorMap map_q,
                       const __grid_constant__ CUtensorMap map_ks, const __grid_constant__ CUtensorMap map_vs,
@@ -249,7 +294,9 @@ __global__ void __launch_bounds__(NTH, 1)
   const int seq = m.seq[r_ref], p0 = m.p0[r_ref], base = m.base[r_ref];
   const int k_last = max(sl[0].pl, nslot == 2 ? sl[1].pl : 0);  // last key position any slot reads
 
-  if (warp == 9) {
+  if (warp >= 8) {
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_OTHER));
+   if (warp == 9) {
     // ------------------------------------------------------------ loader
     const bf16* Kc = (const bf16*)kv.K;
     const bf16* Vc = (const bf16*)kv.V;
@@ -390,14 +437,16 @@ __global__ void __launch_bounds__(NTH, 1)
       mbar_wait_drain(o_full, 0);  // no MMA may still write TMEM when it is freed
     }
     __syncwarp();
-  } else if (warp / 4 < nslot) {
+   }
+  } else {
+   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REG_SOFTMAX));
+   if (warp / 4 < nslot) {
     // ------------------------------------------------------------ softmax
     const int q = warp >> 2, row = tid & 127;
     const Slot s = q ? sl[1] : sl[0];
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t s_col = q * 128, o_col = 256 + q * 128;
     const int pr = s.pf + row;
-    const int lo_r = kv.window > 0 ? pr - kv.window + 1 : INT_MIN;
     float m_used = -1e30f, l = 0.f;
     bool ok = true;
     for (int j = s.a; j <= s.b; ++j) {
@@ -409,15 +458,15 @@ __global__ void __launch_bounds__(NTH, 1)
       for (int c = 0; c < TK; c += 32) tmem_ld32(lane_addr + s_col + c, r + c);
       tmem_wait_ld();
       const int kt = kt0 + j * TK;
+      // a tile every row of the slot sees whole needs no mask
       const bool open = kt + TK - 1 <= s.pf && (kv.window == 0 || kt >= s.pl - kv.window + 1);
-      float mt = -INFINITY;
+      if (!open) {  // key kt + c is visible iff c_lo <= c <= c_hi
+        const int c_hi = pr - kt, c_lo = kv.window > 0 ? pr - kv.window + 1 - kt : -1;
 #pragma unroll
-      for (int c = 0; c < TK; ++c) {
-        float v = __uint_as_float(r[c]);
-        if (!open && !(kt + c <= pr && kt + c >= lo_r)) v = -INFINITY;
-        r[c] = __float_as_uint(v);
-        mt = fmaxf(mt, v);
+        for (int c = 0; c < TK; ++c)
+          if (c > c_hi || c < c_lo) r[c] = __float_as_uint(-INFINITY);
       }
+      const float mt = row_max(r);
       const bool grow = mt > m_used + kLazy;
       float factor = 1.f;
       if (grow) {
@@ -436,20 +485,24 @@ __global__ void __launch_bounds__(NTH, 1)
         }
       }
       l *= factor;
-      float rs = 0.f;
+      // P = 2^(s - m) as bf16 pairs over the first 64 columns of S, 16
+      // columns (32 keys) at a time; two running sums (even, odd keys)
+      float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {  // P over the first 64 columns of S, 16 columns (32 keys) at a time
+      for (int h = 0; h < 4; ++h) {
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
-          const float x0 = ex2(__uint_as_float(r[32 * h + c]) - m_used);
-          const float x1 = ex2(__uint_as_float(r[32 * h + c + 1]) - m_used);
-          rs += x0 + x1;
+          float x0, x1;
+          sub2(x0, x1, __uint_as_float(r[32 * h + c]), __uint_as_float(r[32 * h + c + 1]), m_used);
+          x0 = ex2(x0);
+          x1 = ex2(x1);
+          add2(rs0, rs1, x0, x1);
           pk[c / 2] = pack2(x0, x1);
         }
         tmem_st16(lane_addr + s_col + 16 * h, pk);
       }
-      l += rs;
+      l += rs0 + rs1;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[q]);
@@ -477,6 +530,7 @@ __global__ void __launch_bounds__(NTH, 1)
         }
       }
     }
+  }
   }
   tc_fence_before();
   __syncthreads();
