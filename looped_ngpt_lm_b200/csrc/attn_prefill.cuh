@@ -28,9 +28,10 @@ cudaError_t launch_attn_prefill_tc(int n_tiles, const int2* tiles, int H, int KV
 // The warp-specialised tcgen05 kernel (head_dim 128, 128-row tiles): each
 // CTA runs one work item, two query slots that share a key/value stream over
 // a range of key tiles.  a = {tile, head, tile, head} (second tile -1: one
-// slot); b = {first key tile, end key tile, merge unit, pieces}: an item cut
-// into `pieces` key ranges has one CTA per range; they merge through the
-// partial buffer (unit -1: not cut, range [0, INT_MAX)).
+// slot); b = {first key tile, end key tile, merge unit, pieces | piece << 8}:
+// an item cut into `pieces` key ranges has one CTA per range; they merge
+// through the partial buffer, units unit .. unit + pieces - 1 (unit -1: not
+// cut, range [0, INT_MAX)).
 struct PfItem {
   int4 a, b;
 };
@@ -41,7 +42,7 @@ constexpr int kPfMaxPieces = 4;
 // KV group pair on the same tile (an odd head left over pairs consecutive
 // tiles of one sequence); items longer than the per-SM share of all key
 // tiles are cut into up to kPfMaxPieces key ranges while merge units
-// (pieces - 1 each) last; items come largest first.  tile_first_pos,
+// (one per piece) last; items come largest first.  tile_first_pos,
 // tile_last_pos, tile_seq: each tile's first and last position and sequence.
 // Returns the count (and the merge units used in *units), or -1 past `cap`.
 int prefill_ws_items(int n_tiles, const int* tile_first_pos, const int* tile_last_pos, const int* tile_seq, int H,

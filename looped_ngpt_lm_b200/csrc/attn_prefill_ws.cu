@@ -573,15 +573,17 @@ __global__ void __launch_bounds__(NTH, 1)
         }
       } else {
         // a piece of a cut item: the first pieces to finish leave (O, max,
-        // sum) in the partial buffer; the last one merges them with its own
-        const int unit = rng.z, pieces = rng.w;
+        // sum) in the partial buffer, each in its piece's place; the last one
+        // to finish merges all of them with its own in piece order (the same
+        // bits whichever piece finishes last)
+        const int unit = rng.z, pieces = rng.w & 0xff, mine = rng.w >> 8;
         volatile int* s_arrival = abort_flag + 1;
         named_sync(nthr);
         if (tid == 0) *s_arrival = atomicAdd(&counters[unit], 1);
         named_sync(nthr);
         const int k = *s_arrival;
         if (k < pieces - 1) {
-          float* pr_row = part + (((size_t)(unit + k) * 2 + q) * TQ + row) * kPfPartStride;
+          float* pr_row = part + (((size_t)(unit + mine) * 2 + q) * TQ + row) * kPfPartStride;
 #pragma unroll 1
           for (int c = 0; c < HDT; c += 32) {
             uint32_t o[32];
@@ -597,12 +599,13 @@ __global__ void __launch_bounds__(NTH, 1)
           __stcg(reinterpret_cast<float4*>(pr_row + HDT), make_float4(m_used, l, 0.f, 0.f));
           __threadfence();
           named_sync(nthr);
-          if (tid == 0) atomicExch(&counters[max_units + unit + k], 1);
+          if (tid == 0) atomicExch(&counters[max_units + unit + mine], 1);
         } else {
           // every earlier piece has arrived, so each one's flag comes soon
           if (tid == 0) {
             bool got = true;
-            for (int p = 0; p < pieces - 1 && got; ++p) {
+            for (int p = 0; p < pieces && got; ++p) {
+              if (p == mine) continue;
               const long long t0 = clock64();
               while (atomicAdd(&counters[max_units + unit + p], 0) == 0)
                 if (clock64() - t0 > kWaitCycles) {
@@ -617,21 +620,22 @@ __global__ void __launch_bounds__(NTH, 1)
           named_sync(nthr);
           if (*s_arrival) {
             float mp[kPfMaxPieces], wp[kPfMaxPieces];
-            float mx = m_used;
+            float mx = -INFINITY;
 #pragma unroll
-            for (int p = 0; p < kPfMaxPieces - 1; ++p)
-              if (p < pieces - 1) {
-                const float2 ml = __ldcg(reinterpret_cast<const float2*>(
-                    part + (((size_t)(unit + p) * 2 + q) * TQ + row) * kPfPartStride + HDT));
+            for (int p = 0; p < kPfMaxPieces; ++p)
+              if (p < pieces) {
+                float2 ml = make_float2(m_used, l);
+                if (p != mine)
+                  ml = __ldcg(reinterpret_cast<const float2*>(
+                      part + (((size_t)(unit + p) * 2 + q) * TQ + row) * kPfPartStride + HDT));
                 mp[p] = ml.x;
                 wp[p] = ml.y;  // the piece's sum for now
                 mx = fmaxf(mx, ml.x);
               }
-            const float w_self = ex2(m_used - mx);
-            float lt = l * w_self;
+            float lt = 0.f;
 #pragma unroll
-            for (int p = 0; p < kPfMaxPieces - 1; ++p)
-              if (p < pieces - 1) {
+            for (int p = 0; p < kPfMaxPieces; ++p)
+              if (p < pieces) {
                 const float w = ex2(mp[p] - mx);
                 lt += wp[p] * w;
                 wp[p] = w;
@@ -639,31 +643,37 @@ __global__ void __launch_bounds__(NTH, 1)
             const float inv = lt > 0.f ? 1.f / lt : 0.f;
 #pragma unroll 1
             for (int c = 0; c < HDT; c += 32) {
-              uint32_t o[32];
+              uint32_t o[32], acc[32];
               tmem_ld32(lane_addr + o_col + c, o);
               tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(empty ? 0.f : __uint_as_float(o[e]) * w_self);
+              for (int e = 0; e < 32; ++e) acc[e] = __float_as_uint(0.f);
 #pragma unroll
-              for (int p = 0; p < kPfMaxPieces - 1; ++p)
-                if (p < pieces - 1) {
-                  const float* src = part + (((size_t)(unit + p) * 2 + q) * TQ + row) * kPfPartStride + c;
+              for (int p = 0; p < kPfMaxPieces; ++p)
+                if (p < pieces) {
+                  if (p == mine) {
 #pragma unroll
-                  for (int e = 0; e < 32; e += 4) {
-                    const float4 v = __ldcg(reinterpret_cast<const float4*>(src + e));
-                    o[e] = __float_as_uint(__uint_as_float(o[e]) + v.x * wp[p]);
-                    o[e + 1] = __float_as_uint(__uint_as_float(o[e + 1]) + v.y * wp[p]);
-                    o[e + 2] = __float_as_uint(__uint_as_float(o[e + 2]) + v.z * wp[p]);
-                    o[e + 3] = __float_as_uint(__uint_as_float(o[e + 3]) + v.w * wp[p]);
+                    for (int e = 0; e < 32; ++e)
+                      acc[e] = __float_as_uint(__uint_as_float(acc[e]) + (empty ? 0.f : __uint_as_float(o[e]) * wp[p]));
+                  } else {
+                    const float* src = part + (((size_t)(unit + p) * 2 + q) * TQ + row) * kPfPartStride + c;
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4) {
+                      const float4 v = __ldcg(reinterpret_cast<const float4*>(src + e));
+                      acc[e] = __float_as_uint(__uint_as_float(acc[e]) + v.x * wp[p]);
+                      acc[e + 1] = __float_as_uint(__uint_as_float(acc[e + 1]) + v.y * wp[p]);
+                      acc[e + 2] = __float_as_uint(__uint_as_float(acc[e + 2]) + v.z * wp[p]);
+                      acc[e + 3] = __float_as_uint(__uint_as_float(acc[e + 3]) + v.w * wp[p]);
+                    }
                   }
                 }
-              if (row < s.nrows) store_row32(dst + c, o, inv);
+              if (row < s.nrows) store_row32(dst + c, acc, inv);
             }
           }
           named_sync(nthr);  // every partial read: the unit's words go back to zero
           if (tid == 0) {
             counters[unit] = 0;
-            for (int p = 0; p < pieces - 1; ++p) counters[max_units + unit + p] = 0;
+            for (int p = 0; p < pieces; ++p) counters[max_units + unit + p] = 0;
           }
         }
       }
@@ -794,16 +804,16 @@ int prefill_ws_items(int n_tiles, const int* tile_first_pos, const int* tile_las
     const Base& b = base[i];
     const int cost = b.hi - b.lo + 1;
     int pieces = std::min(kPfMaxPieces, (cost + share - 1) / share);
-    if (pieces > 1 && used + pieces - 1 > max_units) pieces = 1;
+    if (pieces > 1 && used + pieces > max_units) pieces = 1;
     if (pieces == 1) {
       list.push_back({{b.a, make_int4(0, INT_MAX, -1, 1)}, cost});
       continue;
     }
     for (int p = 0; p < pieces; ++p) {
       const int k0 = b.lo + (int)((long long)cost * p / pieces), k1 = b.lo + (int)((long long)cost * (p + 1) / pieces);
-      list.push_back({{b.a, make_int4(k0, k1, used, pieces)}, k1 - k0});
+      list.push_back({{b.a, make_int4(k0, k1, used, pieces | (p << 8))}, k1 - k0});
     }
-    used += pieces - 1;
+    used += pieces;
   }
   if ((int)list.size() > cap) return -1;
   std::stable_sort(list.begin(), list.end(), [](const Item& x, const Item& y) { return x.cost > y.cost; });
