@@ -637,7 +637,7 @@ __global__ void __launch_bounds__(NTH, 1)
             for (int p = 0; p < kPfMaxPieces; ++p)
               if (p < pieces) {
                 const float w = ex2(mp[p] - mx);
-                lt += wp[p] * w;
+                lt = __fmaf_rn(wp[p], w, lt);
                 wp[p] = w;
               }
             const float inv = lt > 0.f ? 1.f / lt : 0.f;
@@ -651,20 +651,22 @@ __global__ void __launch_bounds__(NTH, 1)
 #pragma unroll
               for (int p = 0; p < kPfMaxPieces; ++p)
                 if (p < pieces) {
-                  if (p == mine) {
+                  // one explicit FMA per term whichever piece it comes from,
+                  // so the bits do not depend on which piece merges
+                  const float* src = part + (((size_t)(unit + p) * 2 + q) * TQ + row) * kPfPartStride + c;
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                      acc[e] = __float_as_uint(__uint_as_float(acc[e]) + (empty ? 0.f : __uint_as_float(o[e]) * wp[p]));
-                  } else {
-                    const float* src = part + (((size_t)(unit + p) * 2 + q) * TQ + row) * kPfPartStride + c;
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4) {
-                      const float4 v = __ldcg(reinterpret_cast<const float4*>(src + e));
-                      acc[e] = __float_as_uint(__uint_as_float(acc[e]) + v.x * wp[p]);
-                      acc[e + 1] = __float_as_uint(__uint_as_float(acc[e + 1]) + v.y * wp[p]);
-                      acc[e + 2] = __float_as_uint(__uint_as_float(acc[e + 2]) + v.z * wp[p]);
-                      acc[e + 3] = __float_as_uint(__uint_as_float(acc[e + 3]) + v.w * wp[p]);
-                    }
+                  for (int e = 0; e < 32; e += 4) {
+                    float4 v;
+                    if (p == mine)
+                      v = empty ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                : make_float4(__uint_as_float(o[e]), __uint_as_float(o[e + 1]),
+                                              __uint_as_float(o[e + 2]), __uint_as_float(o[e + 3]));
+                    else
+                      v = __ldcg(reinterpret_cast<const float4*>(src + e));
+                    acc[e] = __float_as_uint(__fmaf_rn(v.x, wp[p], __uint_as_float(acc[e])));
+                    acc[e + 1] = __float_as_uint(__fmaf_rn(v.y, wp[p], __uint_as_float(acc[e + 1])));
+                    acc[e + 2] = __float_as_uint(__fmaf_rn(v.z, wp[p], __uint_as_float(acc[e + 2])));
+                    acc[e + 3] = __float_as_uint(__fmaf_rn(v.w, wp[p], __uint_as_float(acc[e + 3])));
                   }
                 }
               if (row < s.nrows) store_row32(dst + c, acc, inv);

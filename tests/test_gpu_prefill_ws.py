@@ -12,7 +12,9 @@ itself.  The kernel must follow the oracle within the bf16 bar (logits
 relative L2 <= 2e-2, final-state cosine >= 0.999, greedy tokens identical up
 to near ties), agree with the one-slot tcgen05 kernel within the same bar,
 and give the same bits whether a full layer's cache is linear or paged
-(pages of 128 positions are copied by TMA, pages of 64 row by row).
+(pages of 128 positions are copied by TMA, pages of 64 row by row).  On this
+small model every item longer than two key tiles is cut into key ranges (up
+to four) whose partial results are merged, so each test also covers the merge.
 """
 import numpy as np
 import pytest
@@ -121,3 +123,19 @@ def test_ws_paged_cache_same_bits(g5, page):
     _, ora = O.generate(model, prompt, len(out[1][0]), 2, O.LAST_LOOP, chunks=chunks, forced=out[1][0][:-1])
     assert max(rel_l2(out[1][1][i], ora[i]) for i in range(len(out[1][0]))) <= 2e-2
     pag.close()
+
+
+def test_ws_cut_items_deterministic(g5):
+    """Long items are cut into key ranges merged by whichever piece finishes
+    last; the merge runs in piece order, so repeated prefills agree bit for
+    bit."""
+    _, _, h = g5
+    h.set_option(dory.OPT_PREFILL_TC, 3)
+    prompt = synth.make_prompt(34, 640, G5.vocab)
+    outs = []
+    for _ in range(3):
+        h.reset()
+        lg = torch.empty((1, G5.vocab), device="cuda")
+        h.prefill([0], torch.tensor(prompt, dtype=torch.int32, device="cuda"), [640], 2, dory.LAST_LOOP, logits=lg)
+        outs.append(np.concatenate([lg.cpu().numpy().ravel(), h.read_state("s", 640).cpu().numpy().ravel()]))
+    assert all(np.array_equal(outs[0], o) for o in outs[1:])
