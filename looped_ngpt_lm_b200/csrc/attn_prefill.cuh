@@ -26,33 +26,16 @@ cudaError_t launch_attn_prefill_tc(int n_tiles, const int2* tiles, int H, int KV
                                    cudaStream_t st);
 
 // The warp-specialised tcgen05 kernel (head_dim 128, 128-row tiles): each
-// CTA runs one work item, two query slots that share a key/value stream over
-// a range of key tiles.  a = {tile, head, tile, head} (second tile -1: one
-// slot); b = {first key tile, end key tile, merge unit, pieces | piece << 8}:
-// an item cut into `pieces` key ranges has one CTA per range; they merge
-// through the partial buffer, units unit .. unit + pieces - 1 (unit -1: not
-// cut, range [0, INT_MAX)).
-struct PfItem {
-  int4 a, b;
-};
-// Partial rows of a cut item: fp32 O (128) then the running max and sum.
-constexpr int kPfPartStride = 132;
-constexpr int kPfMaxPieces = 4;
-// Host: work items for one layer kind (window 0: full causal).  Heads of a
-// KV group pair on the same tile (an odd head left over pairs consecutive
-// tiles of one sequence); items longer than the per-SM share of all key
-// tiles are cut into up to kPfMaxPieces key ranges while merge units
-// (one per piece) last; items come largest first.  tile_first_pos,
-// tile_last_pos, tile_seq: each tile's first and last position and sequence.
-// Returns the count (and the merge units used in *units), or -1 past `cap`.
-int prefill_ws_items(int n_tiles, const int* tile_first_pos, const int* tile_last_pos, const int* tile_seq, int H,
-                     int KV, int window, int n_sm, int max_units, PfItem* items, int cap, int* units);
-// kv_rows: rows of head_dim elements in each of kv.K, kv.V.  counters
-// (2 x max_units ints, zero) and part (max_units x 2 x 128 x kPfPartStride
-// floats) serve the cut items; a launch that completes leaves counters at zero.
-cudaError_t launch_attn_prefill_ws(int n_items, const PfItem* items, const int2* tiles, int M, int H, int KV, int hd,
+// CTA runs one work item of two query slots that share a key/value stream.
+// prefill_ws_items (host) pairs the heads of each KV group on the same tile
+// (an odd head left over pairs consecutive tiles of one sequence) and orders
+// the items by their number of key tiles, largest first; tile_last_pos[t] and
+// tile_seq[t] are tile t's last position and sequence.  Returns the count, or
+// -1 past `cap`.  kv_rows: rows of head_dim elements in each of kv.K, kv.V.
+int prefill_ws_items(int n_tiles, const int* tile_last_pos, const int* tile_seq, int H, int KV, int4* items,
+                     int cap);
+cudaError_t launch_attn_prefill_ws(int n_items, const int4* items, const int2* tiles, int M, int H, int KV, int hd,
                                    const bf16* qh, const bf16* kscr, const bf16* vscr, KVView kv, size_t kv_rows,
-                                   RowMeta m, int* counters, int max_units, float* part, bf16* out,
-                                   cudaStream_t st);
+                                   RowMeta m, bf16* out, cudaStream_t st);
 
 }  // namespace dory

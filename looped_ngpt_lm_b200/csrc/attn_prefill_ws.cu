@@ -189,40 +189,6 @@ __device__ __forceinline__ float row_max(const uint32_t (&r)[128]) {
   return fmaxf(max3(p[0], p[1], p[2]), fmaxf(p[3], p[4]));
 }
 
-// 2^x for x <= 8 on the FMA pipe (Cody-Waite style reduction: x = n + f,
-// n the nearest integer, |f| <= 1/2, by adding 1.5 * 2^23; 2^f by a cubic
-// fitted to minimise the relative error on [-1/2, 1/2] (7.5e-5, below the
-// 2^-9 half-ulp of the bf16 that P is rounded to); 2^n added to the
-// exponent field).  x is clamped at -125 so the result stays a normal
-// number: fully masked keys give about 2^-125 instead of 0, below anything
-// a bf16 sum of 128-key tiles resolves.
-constexpr int kPolyEvery = 4;  // one key pair in kPolyEvery takes this path
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.f);
-  const float y = x + 12582912.f;
-  const float f = x - (y - 12582912.f);
-  float p = fmaf(0.05517155f, f, 0.24261096f);
-  p = fmaf(p, f, 0.69326097f);
-  p = fmaf(p, f, 0.99992806f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(y) << 23));
-}
-
-// Barrier among the first `n` threads (the softmax warps of the active slots).
-__device__ __forceinline__ void named_sync(int n) { asm volatile("bar.sync 1, %0;" ::"r"(n) : "memory"); }
-
-// 32 values of a row of O times `inv`, as bf16, to global memory.
-__device__ __forceinline__ void store_row32(bf16* dst, const uint32_t* o, float inv) {
-#pragma unroll
-  for (int e = 0; e < 32; e += 8) {
-    uint4 u;
-    u.x = pack2(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
-    u.y = pack2(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
-    u.z = pack2(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
-    u.w = pack2(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
-    *reinterpret_cast<uint4*>(dst + e) = u;
-  }
-}
-
 // A bounded wait taken by every lane of a warp, with one outcome for all of
 // them (the warp-wide TMEM accesses and __syncwarp that follow need every lane).
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err) {
@@ -246,8 +212,7 @@ __global__ void __launch_bounds__(NTH, 1)
                       const __grid_constant__ CUtensorMap map_ks, const __grid_constant__ CUtensorMap map_vs,
                       const __grid_constant__ CUtensorMap map_kc, const __grid_constant__ CUtensorMap map_vc,
                       const bf16* __restrict__ kscr, const bf16* __restrict__ vscr, KVView kv, RowMeta m,
-                      const int2* __restrict__ tiles, const PfItem* __restrict__ items, int* __restrict__ counters,
-                      int max_units, float* __restrict__ part, bf16* __restrict__ out) {
+                      const int2* __restrict__ tiles, const int4* __restrict__ items, bf16* __restrict__ out) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sb = smem_u32(smem);
@@ -295,8 +260,7 @@ __global__ void __launch_bounds__(NTH, 1)
   pdl_trigger();
 
   // ---- the work item: one or two slots of one KV group and one sequence
-  const int4 it = items[blockIdx.x].a;
-  const int4 rng = items[blockIdx.x].b;  // key tiles [rng.x, rng.y); merge unit rng.z of rng.w pieces
+  const int4 it = items[blockIdx.x];
   const int nslot = it.z >= 0 ? 2 : 1;
   const int H = KV * G, qd = H * HDT;
   const int g = it.y / G;
@@ -319,14 +283,12 @@ __global__ void __launch_bounds__(NTH, 1)
       hi_t = max(hi_t, s.b);
     }
   }
-  lo_t = max(lo_t, rng.x);
-  hi_t = min(hi_t, rng.y - 1);
   const int n_tiles = hi_t - lo_t + 1;
   const int kt0 = lo_t * TK;
 #pragma unroll
-  for (int q = 0; q < 2; ++q) {  // a slot's range may be empty in one piece of a cut item (a > b)
-    sl[q].a = max(sl[q].a, lo_t) - lo_t;
-    sl[q].b = min(sl[q].b, hi_t) - lo_t;
+  for (int q = 0; q < 2; ++q) {
+    sl[q].a -= lo_t;
+    sl[q].b -= lo_t;
   }
   const int r_ref = sl[0].r0;
   const int seq = m.seq[r_ref], p0 = m.p0[r_ref], base = m.base[r_ref];
@@ -434,7 +396,7 @@ __global__ void __launch_bounds__(NTH, 1)
         tc_fence_after();
 #pragma unroll
         for (int q = 0; q < 2; ++q)
-          if (q < nslot && sl[q].a == 0 && sl[q].b >= 0) s_mma(q, 0);
+          if (q < nslot && sl[q].a == 0) s_mma(q, 0);
         umma_commit(&k_empty[0]);
       }
       for (int j = 0; j < n_tiles && ok; ++j) {
@@ -533,13 +495,8 @@ __global__ void __launch_bounds__(NTH, 1)
         for (int c = 0; c < 32; c += 2) {
           float x0, x1;
           sub2(x0, x1, __uint_as_float(r[32 * h + c]), __uint_as_float(r[32 * h + c + 1]), m_used);
-          if ((c / 2) % kPolyEvery == kPolyEvery - 1) {  // on the FMA pipe: the MUFU is the busier unit
-            x0 = exp2_poly(x0);
-            x1 = exp2_poly(x1);
-          } else {
-            x0 = ex2(x0);
-            x1 = ex2(x1);
-          }
+          x0 = ex2(x0);
+          x1 = ex2(x1);
           add2(rs0, rs1, x0, x1);
           pk[c / 2] = pack2(x0, x1);
         }
@@ -550,132 +507,25 @@ __global__ void __launch_bounds__(NTH, 1)
       tc_fence_before();
       mbar_arrive(&p_full[q]);
     }
-    // every product of this CTA complete: normalise and store this row of O.
-    // Every softmax thread of the active slots gets here; one waits for the
-    // products and all take its outcome (the barriers below need them all).
-    const int nthr = nslot * TQ;
-    volatile int* s_go = abort_flag + 2;
-    named_sync(nthr);
-    if (tid == 0) *s_go = ok && !*abort_flag && mbar_wait(o_full, 0, abort_flag, kv.err);
-    named_sync(nthr);
-    if (*s_go) {
+    // every product of this CTA complete: normalise and store this row of O
+    if (ok && warp_wait(o_full, 0, abort_flag, kv.err)) {
       tc_fence_after();
-      const bool empty = s.a > s.b;  // no key tile of this piece: O was never written
+      const float inv = l > 0.f ? 1.f / l : 0.f;
       bf16* dst = out + (size_t)(s.r0 + row) * qd + s.head * HDT;
-      if (rng.z < 0) {
-        const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
-        for (int c = 0; c < HDT; c += 32) {
-          uint32_t o[32];
-          tmem_ld32(lane_addr + o_col + c, o);
-          tmem_wait_ld();
-          if (row < s.nrows) store_row32(dst + c, o, inv);
-        }
-      } else {
-        // a piece of a cut item: the first pieces to finish leave (O, max,
-        // sum) in the partial buffer, each in its piece's place; the last one
-        // to finish merges all of them with its own in piece order (the same
-        // bits whichever piece finishes last)
-        const int unit = rng.z, pieces = rng.w & 0xff, mine = rng.w >> 8;
-        volatile int* s_arrival = abort_flag + 1;
-        named_sync(nthr);
-        if (tid == 0) *s_arrival = atomicAdd(&counters[unit], 1);
-        named_sync(nthr);
-        const int k = *s_arrival;
-        if (k < pieces - 1) {
-          float* pr_row = part + (((size_t)(unit + mine) * 2 + q) * TQ + row) * kPfPartStride;
-#pragma unroll 1
-          for (int c = 0; c < HDT; c += 32) {
-            uint32_t o[32];
-            tmem_ld32(lane_addr + o_col + c, o);
-            tmem_wait_ld();
+      for (int c = 0; c < HDT; c += 32) {
+        uint32_t o[32];
+        tmem_ld32(lane_addr + o_col + c, o);
+        tmem_wait_ld();
+        if (row < s.nrows) {
 #pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              __stcg(reinterpret_cast<float4*>(pr_row + c + e),
-                     empty ? make_float4(0.f, 0.f, 0.f, 0.f)
-                           : make_float4(__uint_as_float(o[e]), __uint_as_float(o[e + 1]),
-                                         __uint_as_float(o[e + 2]), __uint_as_float(o[e + 3])));
-          }
-          __stcg(reinterpret_cast<float4*>(pr_row + HDT), make_float4(m_used, l, 0.f, 0.f));
-          __threadfence();
-          named_sync(nthr);
-          if (tid == 0) atomicExch(&counters[max_units + unit + mine], 1);
-        } else {
-          // every earlier piece has arrived, so each one's flag comes soon
-          if (tid == 0) {
-            bool got = true;
-            for (int p = 0; p < pieces && got; ++p) {
-              if (p == mine) continue;
-              const long long t0 = clock64();
-              while (atomicAdd(&counters[max_units + unit + p], 0) == 0)
-                if (clock64() - t0 > kWaitCycles) {
-                  got = false;
-                  set_error(kv.err, DEV_ERR_TIMEOUT);
-                  break;
-                }
-            }
-            __threadfence();
-            *s_arrival = got ? 1 : 0;
-          }
-          named_sync(nthr);
-          if (*s_arrival) {
-            float mp[kPfMaxPieces], wp[kPfMaxPieces];
-            float mx = -INFINITY;
-#pragma unroll
-            for (int p = 0; p < kPfMaxPieces; ++p)
-              if (p < pieces) {
-                float2 ml = make_float2(m_used, l);
-                if (p != mine)
-                  ml = __ldcg(reinterpret_cast<const float2*>(
-                      part + (((size_t)(unit + p) * 2 + q) * TQ + row) * kPfPartStride + HDT));
-                mp[p] = ml.x;
-                wp[p] = ml.y;  // the piece's sum for now
-                mx = fmaxf(mx, ml.x);
-              }
-            float lt = 0.f;
-#pragma unroll
-            for (int p = 0; p < kPfMaxPieces; ++p)
-              if (p < pieces) {
-                const float w = ex2(mp[p] - mx);
-                lt = __fmaf_rn(wp[p], w, lt);
-                wp[p] = w;
-              }
-            const float inv = lt > 0.f ? 1.f / lt : 0.f;
-#pragma unroll 1
-            for (int c = 0; c < HDT; c += 32) {
-              uint32_t o[32], acc[32];
-              tmem_ld32(lane_addr + o_col + c, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) acc[e] = __float_as_uint(0.f);
-#pragma unroll
-              for (int p = 0; p < kPfMaxPieces; ++p)
-                if (p < pieces) {
-                  // one explicit FMA per term whichever piece it comes from,
-                  // so the bits do not depend on which piece merges
-                  const float* src = part + (((size_t)(unit + p) * 2 + q) * TQ + row) * kPfPartStride + c;
-#pragma unroll
-                  for (int e = 0; e < 32; e += 4) {
-                    float4 v;
-                    if (p == mine)
-                      v = empty ? make_float4(0.f, 0.f, 0.f, 0.f)
-                                : make_float4(__uint_as_float(o[e]), __uint_as_float(o[e + 1]),
-                                              __uint_as_float(o[e + 2]), __uint_as_float(o[e + 3]));
-                    else
-                      v = __ldcg(reinterpret_cast<const float4*>(src + e));
-                    acc[e] = __float_as_uint(__fmaf_rn(v.x, wp[p], __uint_as_float(acc[e])));
-                    acc[e + 1] = __float_as_uint(__fmaf_rn(v.y, wp[p], __uint_as_float(acc[e + 1])));
-                    acc[e + 2] = __float_as_uint(__fmaf_rn(v.z, wp[p], __uint_as_float(acc[e + 2])));
-                    acc[e + 3] = __float_as_uint(__fmaf_rn(v.w, wp[p], __uint_as_float(acc[e + 3])));
-                  }
-                }
-              if (row < s.nrows) store_row32(dst + c, acc, inv);
-            }
-          }
-          named_sync(nthr);  // every partial read: the unit's words go back to zero
-          if (tid == 0) {
-            counters[unit] = 0;
-            for (int p = 0; p < pieces; ++p) counters[max_units + unit + p] = 0;
+          for (int e = 0; e < 32; e += 8) {
+            uint4 u;
+            u.x = pack2(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
+            u.y = pack2(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+            u.z = pack2(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
+            u.w = pack2(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
+            *reinterpret_cast<uint4*>(dst + c + e) = u;
           }
         }
       }
@@ -748,86 +598,42 @@ bool map_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint6
 
 }  // namespace
 
-int prefill_ws_items(int n_tiles, const int* tile_first_pos, const int* tile_last_pos, const int* tile_seq, int H,
-                     int KV, int window, int n_sm, int max_units, PfItem* items, int cap, int* units) {
+int prefill_ws_items(int n_tiles, const int* tile_last_pos, const int* tile_seq, int H, int KV, int4* items,
+                     int cap) {
   const int G = H / KV;
-  struct Base {
-    int4 a;
-    int lo, hi;  // key tiles of the union of the slots' ranges
+  struct Item {
+    int4 v;
+    int cost;
   };
-  auto range = [&](int t, int& lo, int& hi) {
-    const int first = window > 0 ? std::max(0, tile_first_pos[t] - window + 1) : 0;
-    lo = first / TK;
-    hi = tile_last_pos[t] / TK;
-  };
-  std::vector<Base> base;
-  base.reserve((size_t)n_tiles * H);
-  auto add = [&](int t0, int h0, int t1, int h1) {
-    int lo, hi;
-    range(t0, lo, hi);
-    if (t1 >= 0) {
-      int lo1, hi1;
-      range(t1, lo1, hi1);
-      lo = std::min(lo, lo1);
-      hi = std::max(hi, hi1);
-    }
-    base.push_back({make_int4(t0, h0, t1, h1), lo, hi});
-  };
+  std::vector<Item> list;
+  list.reserve((size_t)n_tiles * H);
   for (int g = 0; g < KV; ++g) {
-    for (int t = 0; t < n_tiles; ++t)  // head pairs on the same rows
-      for (int h = g * G; h + 1 < (g + 1) * G; h += 2) add(t, h, t, h + 1);
+    // head pairs on the same rows
+    for (int t = 0; t < n_tiles; ++t)
+      for (int h = g * G; h + 1 < (g + 1) * G; h += 2)
+        list.push_back({make_int4(t, h, t, h + 1), tile_last_pos[t] / TK + 1});
     if (G % 2 == 0) continue;
-    const int h = (g + 1) * G - 1;  // the odd head: consecutive row tiles of one sequence
+    // the odd head: consecutive row tiles of one sequence
+    const int h = (g + 1) * G - 1;
     for (int t = 0; t < n_tiles;) {
       if (t + 1 < n_tiles && tile_seq[t + 1] == tile_seq[t]) {
-        add(t, h, t + 1, h);
+        list.push_back({make_int4(t, h, t + 1, h), tile_last_pos[t + 1] / TK + 1});
         t += 2;
       } else {
-        add(t, h, -1, -1);
+        list.push_back({make_int4(t, h, -1, -1), tile_last_pos[t] / TK + 1});
         t += 1;
       }
     }
   }
-  // cut items longer than every SM's share of the key tiles
-  long long total = 0;
-  for (const Base& b : base) total += b.hi - b.lo + 1;
-  const int share = (int)std::max<long long>(2, (total + n_sm - 1) / std::max(1, n_sm));
-  std::vector<int> order(base.size());
-  for (size_t i = 0; i < order.size(); ++i) order[i] = (int)i;
-  std::stable_sort(order.begin(), order.end(),
-                   [&](int x, int y) { return base[x].hi - base[x].lo > base[y].hi - base[y].lo; });
-  struct Item {
-    PfItem v;
-    int cost;
-  };
-  std::vector<Item> list;
-  int used = 0;
-  for (int i : order) {
-    const Base& b = base[i];
-    const int cost = b.hi - b.lo + 1;
-    int pieces = std::min(kPfMaxPieces, (cost + share - 1) / share);
-    if (pieces > 1 && used + pieces > max_units) pieces = 1;
-    if (pieces == 1) {
-      list.push_back({{b.a, make_int4(0, INT_MAX, -1, 1)}, cost});
-      continue;
-    }
-    for (int p = 0; p < pieces; ++p) {
-      const int k0 = b.lo + (int)((long long)cost * p / pieces), k1 = b.lo + (int)((long long)cost * (p + 1) / pieces);
-      list.push_back({{b.a, make_int4(k0, k1, used, pieces | (p << 8))}, k1 - k0});
-    }
-    used += pieces;
-  }
   if ((int)list.size() > cap) return -1;
-  std::stable_sort(list.begin(), list.end(), [](const Item& x, const Item& y) { return x.cost > y.cost; });
+  std::stable_sort(list.begin(), list.end(), [](const Item& a, const Item& b) { return a.cost > b.cost; });
   for (size_t i = 0; i < list.size(); ++i) items[i] = list[i].v;
-  if (units) *units = used;
   return (int)list.size();
 }
 
-cudaError_t launch_attn_prefill_ws(int n_items, const PfItem* items, const int2* tiles, int M, int H, int KV, int hd,
+cudaError_t launch_attn_prefill_ws(int n_items, const int4* items, const int2* tiles, int M, int H, int KV, int hd,
                                    const bf16* qh, const bf16* kscr, const bf16* vscr, KVView kv, size_t kv_rows,
-                                   RowMeta m, int* counters, int max_units, float* part, bf16* out,
-                                   cudaStream_t st) {
+                                   RowMeta m, bf16* out, cudaStream_t st) {
   if (hd != HDT || H % KV) return cudaErrorNotSupported;
   if (n_items == 0) return cudaSuccess;
   static bool attr = false;
@@ -843,7 +649,7 @@ cudaError_t launch_attn_prefill_ws(int n_items, const PfItem* items, const int2*
       !map_2d(&mvc, kv.V, kv_rows, HDT, HDT))
     return cudaErrorInvalidValue;
   return launch(k_attn_prefill_ws, dim3(n_items), dim3(NTH), SMEM_BYTES, st, KV, H / KV, mq, mks, mvs, mkc, mvc, kscr,
-                vscr, kv, m, tiles, items, counters, max_units, part, out);
+                vscr, kv, m, tiles, items, out);
 }
 
 }  // namespace dory

@@ -124,12 +124,8 @@ struct dory_handle {
   int *cu = nullptr, *head_rows = nullptr;
   int2* tiles = nullptr;  // prefill attention tiles (64 or 128 rows of one sequence)
   int tiles_cap = 0;
-  PfItem* pf_items[2] = {nullptr, nullptr};  // warp-specialised prefill attention work items:
-                                             // [0] sliding-window layers, [1] full layers
+  int4* pf_items = nullptr;  // warp-specialised prefill attention: CTA work items
   int items_cap = 0;
-  int pf_units = 0;             // merge units for cut items
-  int* pf_counters = nullptr;   // [2 * pf_units], zero between launches
-  float* pf_part = nullptr;     // [pf_units][2][128][kPfPartStride]
   void* qh = nullptr;     // bf16 pre-scaled queries of long chunks
   RowMeta meta{};
   // the state h lives in one of two buffers: a GEMM that applies the
@@ -160,7 +156,7 @@ struct dory_handle {
   int* page_table = nullptr;
   int pt_stride = 0, page_shift = 0, pool_pages = 0;
   std::vector<int> pt_host, free_pages;
-  std::vector<PfItem> items_host;
+  std::vector<int4> items_host;
   std::vector<std::vector<int>> seq_pages;
   std::vector<int> ids_on_device;     // seq ids last uploaded to seq_ids
   int last_rows = 0;
@@ -285,11 +281,8 @@ size_t layout(dory_handle* h) {
   h->head_rows = cv.take<int>(sizeof(int) * h->head_max);
   h->tiles_cap = M / 64 + c.max_batch + 1;
   h->tiles = cv.take<int2>(sizeof(int2) * h->tiles_cap);
-  h->items_cap = h->tiles_cap * c.n_heads * kPfMaxPieces;
-  for (int i = 0; i < 2; ++i) h->pf_items[i] = cv.take<PfItem>(sizeof(PfItem) * h->items_cap);
-  h->pf_units = std::min(256, h->tiles_cap * c.n_heads);
-  h->pf_counters = cv.take<int>(sizeof(int) * 2 * h->pf_units);
-  h->pf_part = cv.take<float>(sizeof(float) * (size_t)h->pf_units * 2 * 128 * kPfPartStride);
+  h->items_cap = h->tiles_cap * c.n_heads;
+  h->pf_items = cv.take<int4>(sizeof(int4) * h->items_cap);
   h->qh = cv.take<char>(2 * (size_t)M * h->q_dim);
   h->meta.seq = cv.take<int>(sizeof(int) * M);
   h->meta.pos = cv.take<int>(sizeof(int) * M);
@@ -387,7 +380,7 @@ struct Fwd {
   bool invariant;  // decode / speculative rows: GEMM arithmetic independent of M
   int n_tiles = 0;  // > 0: long-chunk attention on the tensor cores over H->tiles
   int tc5 = 0;      // ... by a tcgen05 kernel (128-row tiles): 2 one slot per CTA, 3 warp-specialised
-  int n_items[2] = {0, 0};  // work items of the warp-specialised kernel (H->pf_items)
+  int n_items = 0;  // work items of the warp-specialised kernel (H->pf_items)
   int pf_k = 0;     // > 0: GEMMs follow the weight stream of a pf_k-loop decode step
   bool stage = true;  // layer updates may run in the next GEMM's operand stage
 };
@@ -408,14 +401,6 @@ KVView kv_view(dory_handle* H, int l, int loop, int mode) {
     v.page_shift = H->page_shift;
   }
   return v;
-}
-
-// Streaming multiprocessors of the current device.
-int device_sms() {
-  int dev = 0, n = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
 }
 
 // Rows of head_dim elements in one K (or V) buffer of layer l's cache.
@@ -652,13 +637,10 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop, float* copy_la
         }
         if (tc) {
           Scope sc(H, f.st, "attn_prefill", 0);
-          if (f.tc5 == 3) {
-            const int full = kv.window > 0 ? 0 : 1;
-            CK(launch_attn_prefill_ws(f.n_items[full], H->pf_items[full], H->tiles, M, c.n_heads, c.n_kv_heads,
-                                      c.head_dim, (const bf16*)H->qh, (const bf16*)H->kscr, (const bf16*)H->vscr,
-                                      kv, kv_rows(H, l), H->meta, H->pf_counters, H->pf_units, H->pf_part,
-                                      (bf16*)H->ao, f.st));
-          }
+          if (f.tc5 == 3)
+            CK(launch_attn_prefill_ws(f.n_items, H->pf_items, H->tiles, M, c.n_heads, c.n_kv_heads, c.head_dim,
+                                      (const bf16*)H->qh, (const bf16*)H->kscr, (const bf16*)H->vscr, kv,
+                                      kv_rows(H, l), H->meta, (bf16*)H->ao, f.st));
           else if (f.tc5 == 2)
             CK(launch_attn_prefill_tc(f.n_tiles, H->tiles, c.n_heads, c.n_kv_heads, c.head_dim, (const bf16*)H->qh,
                                       (const bf16*)H->kscr, (const bf16*)H->vscr, kv, H->meta, (bf16*)H->ao, f.st));
@@ -886,26 +868,19 @@ dory_status prefill_t(dory_handle* H, int batch, const int32_t* seq_ids, const i
     CK(cudaMemcpyAsync(H->tiles, tl.data(), sizeof(int2) * n, cudaMemcpyHostToDevice, st));
     f.n_tiles = n;
     if (f.tc5 == 3) {
-      // each tile's sequence and positions, for pairing, cutting and ordering;
-      // one item table for the sliding-window layers and one for the full ones
-      std::vector<int> first(n), last(n), sq(n);
+      // each tile's sequence and last position, for pairing and ordering
+      std::vector<int> last(n), sq(n);
       for (int t = 0, b = 0; t < n; ++t) {
         while (tl[t].x >= cu[b + 1]) ++b;
         sq[t] = b;
-        first[t] = H->len[seq_ids[b]] + (tl[t].x - cu[b]);
         last[t] = H->len[seq_ids[b]] + (tl[t].y - 1 - cu[b]);
       }
       H->items_host.resize(H->items_cap);
-      for (int full = 0; full < 2; ++full) {
-        int units = 0;
-        const int ni = prefill_ws_items(n, first.data(), last.data(), sq.data(), c.n_heads, c.n_kv_heads,
-                                        full ? 0 : c.swa_window, device_sms(), H->pf_units, H->items_host.data(),
-                                        H->items_cap, &units);
-        if (ni < 0) return fail(DORY_ERR_CAPACITY, "too many prefill attention items");
-        CK(cudaMemcpyAsync(H->pf_items[full], H->items_host.data(), sizeof(PfItem) * ni, cudaMemcpyHostToDevice,
-                           st));
-        f.n_items[full] = ni;
-      }
+      const int ni = prefill_ws_items(n, last.data(), sq.data(), c.n_heads, c.n_kv_heads, H->items_host.data(),
+                                      H->items_cap);
+      if (ni < 0) return fail(DORY_ERR_CAPACITY, "too many prefill attention items");
+      CK(cudaMemcpyAsync(H->pf_items, H->items_host.data(), sizeof(int4) * ni, cudaMemcpyHostToDevice, st));
+      f.n_items = ni;
     }
   }
   RET(input_block<T>(f, tokens));
@@ -1317,7 +1292,6 @@ dory_status dory_reset(dory_handle* h, int32_t seq, dory_stream stream) {
     CK(cudaMemsetAsync(h->seq_len, 0, sizeof(int) * h->c.max_batch, st));
     CK(cudaMemsetAsync(h->err, 0, sizeof(int) * 4, st));
     CK(cudaMemsetAsync(h->attn_counters, 0, sizeof(unsigned) * (size_t)h->M_max * h->c.n_kv_heads, st));
-    CK(cudaMemsetAsync(h->pf_counters, 0, sizeof(int) * 2 * h->pf_units, st));
     std::fill(h->len.begin(), h->len.end(), 0);
     std::fill(h->mode.begin(), h->mode.end(), -1);
     for (int q = 0; q < h->c.max_batch; ++q) release_pages(h, q);
