@@ -60,6 +60,7 @@ static_assert(2 * 128 * REG_SOFTMAX + 128 * REG_OTHER <= NTH * 168, "register sp
 constexpr int PANEL = 128 * 128;       // 64 head dims x 128 rows, bytes
 constexpr int TILE = 2 * PANEL;        // one Q, K or V tile, bytes
 constexpr float kLazy = 8.f;
+constexpr float kSingleTime = 0.55f;  // time of a one-slot item against a two-slot item of the same key tiles
 
 constexpr int Q_OFF = 0;                       // 2 slots
 constexpr int K_OFF = Q_OFF + 2 * TILE;        // NS stages
@@ -598,35 +599,51 @@ bool map_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint6
 
 }  // namespace
 
-int prefill_ws_items(int n_tiles, const int* tile_last_pos, const int* tile_seq, int H, int KV, int4* items,
-                     int cap) {
+int prefill_ws_items(int n_tiles, const int* tile_last_pos, const int* tile_seq, int H, int KV, int n_sm,
+                     int4* items, int cap) {
   const int G = H / KV;
   struct Item {
     int4 v;
-    int cost;
+    float time;  // in key tiles of a two-slot item
   };
-  std::vector<Item> list;
-  list.reserve((size_t)n_tiles * H);
+  auto tiles_of = [&](int t) { return tile_last_pos[t] / TK + 1; };
+  std::vector<Item> pairs;
+  pairs.reserve((size_t)n_tiles * H);
   for (int g = 0; g < KV; ++g) {
     // head pairs on the same rows
     for (int t = 0; t < n_tiles; ++t)
-      for (int h = g * G; h + 1 < (g + 1) * G; h += 2)
-        list.push_back({make_int4(t, h, t, h + 1), tile_last_pos[t] / TK + 1});
+      for (int h = g * G; h + 1 < (g + 1) * G; h += 2) pairs.push_back({make_int4(t, h, t, h + 1), (float)tiles_of(t)});
     if (G % 2 == 0) continue;
     // the odd head: consecutive row tiles of one sequence
     const int h = (g + 1) * G - 1;
     for (int t = 0; t < n_tiles;) {
       if (t + 1 < n_tiles && tile_seq[t + 1] == tile_seq[t]) {
-        list.push_back({make_int4(t, h, t + 1, h), tile_last_pos[t + 1] / TK + 1});
+        pairs.push_back({make_int4(t, h, t + 1, h), (float)tiles_of(t + 1)});
         t += 2;
       } else {
-        list.push_back({make_int4(t, h, -1, -1), tile_last_pos[t] / TK + 1});
+        pairs.push_back({make_int4(t, h, -1, -1), kSingleTime * tiles_of(t)});
         t += 1;
       }
     }
   }
+  // a two-slot item longer than every SM's share of the work runs as two
+  // one-slot items: a slot alone goes through its key tiles in about half
+  // the time, so the longest items no longer set the end of the launch
+  double total = 0;
+  for (const Item& it : pairs) total += it.time;
+  const double share = total / std::max(1, n_sm);
+  std::vector<Item> list;
+  list.reserve(pairs.size() * 2);
+  for (const Item& it : pairs) {
+    if (it.v.z >= 0 && it.time > share) {
+      list.push_back({make_int4(it.v.x, it.v.y, -1, -1), kSingleTime * tiles_of(it.v.x)});
+      list.push_back({make_int4(it.v.z, it.v.w, -1, -1), kSingleTime * tiles_of(it.v.z)});
+    } else {
+      list.push_back(it);
+    }
+  }
   if ((int)list.size() > cap) return -1;
-  std::stable_sort(list.begin(), list.end(), [](const Item& a, const Item& b) { return a.cost > b.cost; });
+  std::stable_sort(list.begin(), list.end(), [](const Item& a, const Item& b) { return a.time > b.time; });
   for (size_t i = 0; i < list.size(); ++i) items[i] = list[i].v;
   return (int)list.size();
 }

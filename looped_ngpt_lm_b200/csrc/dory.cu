@@ -403,6 +403,14 @@ KVView kv_view(dory_handle* H, int l, int loop, int mode) {
   return v;
 }
 
+// Streaming multiprocessors of the current device.
+int device_sms() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
 // Rows of head_dim elements in one K (or V) buffer of layer l's cache.
 size_t kv_rows(dory_handle* H, int l) {
   const AttnLayer& a = H->attn[H->attn_of[l]];
@@ -876,7 +884,7 @@ dory_status prefill_t(dory_handle* H, int batch, const int32_t* seq_ids, const i
         last[t] = H->len[seq_ids[b]] + (tl[t].y - 1 - cu[b]);
       }
       H->items_host.resize(H->items_cap);
-      const int ni = prefill_ws_items(n, last.data(), sq.data(), c.n_heads, c.n_kv_heads, H->items_host.data(),
+      const int ni = prefill_ws_items(n, last.data(), sq.data(), c.n_heads, c.n_kv_heads, device_sms(), H->items_host.data(),
                                       H->items_cap);
       if (ni < 0) return fail(DORY_ERR_CAPACITY, "too many prefill attention items");
       CK(cudaMemcpyAsync(H->pf_items, H->items_host.data(), sizeof(int4) * ni, cudaMemcpyHostToDevice, st));
