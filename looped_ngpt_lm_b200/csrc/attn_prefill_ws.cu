@@ -2,26 +2,34 @@
 // (bf16, head_dim 128).  Each CTA runs one work item: 128 query rows of one
 // head, over the key tiles its rows see.
 //
-//   warps 0-3  softmax, one query row per thread (= TMEM lane)
-//   warp 4     allocates TMEM; one lane issues every MMA and commit
-//   warp 5     loader: Q once, then K and V tiles of 128 keys into a
+//   warps 0-3  softmax of the even key tiles, one query row per thread
+//              (= TMEM lane)
+//   warps 4-7  softmax of the odd key tiles, the same rows
+//   warp 8     allocates TMEM; one lane issues every MMA and commit
+//   warp 9     loader: Q once, then K and V tiles of 128 keys into a
 //              three-stage ring, by TMA when a tile is one run of rows of
 //              the chunk scratch or of the cache, else by cp.async row by row
+//   warps 10-11 idle (they complete the third warpgroup)
+// The CTA launches with 168 registers a thread; the third warpgroup gives
+// back all but 72 and the softmax warpgroups take them (216 each), enough to
+// hold a row of S.
 //
-// TMEM (512 columns): S buffers 0 and 1 at [0,128) and [128,256), O at
-// [256,384).  S(j) = Q K(j)^T goes to buffer j % 2, so the tensor core
-// computes S(j+1) while the softmax works on S(j), and the softmax runs from
-// one tile to the next without waiting for a product.  The softmax writes
-// P(j) as bf16 pairs over the first 64 columns of S(j)'s buffer; the MMA lane
-// then issues O += P(j) V(j) (P from TMEM) and S(j+2) into the same buffer
-// (the tensor core runs one lane's products in order, so P(j) is read before
-// S(j+2) overwrites it).  V stays as loaded (keys x head dims): the P V
-// product reads it as an MN-major operand, so nothing is transposed.
+// TMEM (512 columns): S buffers 0 and 1 at [0,128) and [128,256), O0 at
+// [256,384), O1 at [384,512).  Key tile j belongs to half b = j % 2: S(j) =
+// Q K(j)^T goes to buffer b, the softmax warpgroup b turns it into P(j)
+// (bf16 pairs over the first 64 columns of the buffer) and O_b += P(j) V(j).
+// Each half keeps its own running maximum, sum and O, so the two warpgroups
+// work on consecutive tiles at the same time; the halves are merged once at
+// the end.  The MMA lane issues, per tile j, O_b += P(j) V(j) (P from TMEM)
+// and then S(j+2) into the same buffer (the tensor core runs one lane's
+// products in order, so P(j) is read before S(j+2) overwrites it; the commit
+// after S(j+2) covers O_b += P(j) V(j), so a warpgroup that sees S(j+2) may
+// rescale O_b).  V stays as loaded (keys x head dims): the P V product reads
+// it as an MN-major operand, so nothing is transposed.
 //
 // Softmax in base 2 (Q is pre-scaled by log2(e)/sqrt(head_dim)) with a lazy
 // running maximum: O and the row sum are rescaled only when a row maximum
-// grows by more than 8 (P = 2^(s - m) then stays below 256).  A rescale waits
-// for the product that last added to O.
+// grows by more than 8 (P = 2^(s - m) then stays below 256).
 //
 // Every mbarrier wait is bounded; on expiry the CTA sets the device error
 // word, every role stops, the loader waits (bounded) for its copies in flight
@@ -48,7 +56,9 @@ constexpr int HDT = 128;               // head dimensions
 constexpr int TQ = 128;                // query rows per item
 constexpr int TK = 128;                // keys per tile
 constexpr int NS = 3;                  // K/V ring stages
-constexpr int NTH = 192;               // 6 warps
+constexpr int NTH = 384;               // 12 warps, three warpgroups
+constexpr int REG_SOFTMAX = 216, REG_OTHER = 72;  // 2 x 128 x 216 + 128 x 72 = 384 x 168
+static_assert(2 * 128 * REG_SOFTMAX + 128 * REG_OTHER <= NTH * 168, "register split exceeds the launch's registers");
 constexpr int PANEL = 128 * 128;       // 64 head dims x 128 rows, bytes
 constexpr int TILE = 2 * PANEL;        // one Q, K or V tile, bytes
 constexpr float kLazy = 8.f;
@@ -58,8 +68,9 @@ constexpr int K_OFF = Q_OFF + TILE;            // NS stages
 constexpr int V_OFF = K_OFF + NS * TILE;       // NS stages
 constexpr int BAR_OFF = V_OFF + NS * TILE;     // mbarriers, TMEM slot, flags
 constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
 constexpr int TMEM_COLS = 512;
-constexpr uint32_t O_COL = 256;
+constexpr uint32_t O_COL = 256;  // O_b at O_COL + 128 b
 
 __device__ __forceinline__ uint32_t sw(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 
@@ -208,11 +219,13 @@ __global__ void __launch_bounds__(NTH, 1)
   uint64_t* k_empty = v_full + NS;        // [NS]
   uint64_t* v_empty = k_empty + NS;       // [NS]
   uint64_t* s_full = v_empty + NS;        // [2]: S(j) in buffer j % 2
-  uint64_t* p_full = s_full + 2;          // P(j) written (all 128 rows)
-  uint64_t* pv_done = p_full + 1;         // O += P(j) V(j) complete, once per tile
-  uint64_t* o_full = pv_done + 1;         // every product complete
+  uint64_t* p_full = s_full + 2;          // [2]: P(j) written (all 128 rows of half j % 2)
+  uint64_t* o_full = p_full + 2;          // every product complete
   uint32_t* tmem_slot = (uint32_t*)(o_full + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  // [2][128]: each half's (max, sum) per row, written over Q once every S
+  // product is complete
+  float2* half_ml = (float2*)(smem + Q_OFF);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
@@ -223,15 +236,15 @@ __global__ void __launch_bounds__(NTH, 1)
       mbar_init(&k_empty[i], 1);
       mbar_init(&v_empty[i], 1);
     }
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    mbar_init(p_full, TQ);
-    mbar_init(pv_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], TQ);
+    }
     mbar_init(o_full, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 4) {
+  if (warp == 8) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(TMEM_COLS)
                  : "memory");
@@ -257,7 +270,9 @@ __global__ void __launch_bounds__(NTH, 1)
   const int n_tiles = pl / TK - lo / TK + 1;
   const int seq = m.seq[r0], p0 = m.p0[r0], base = m.base[r0];
 
-  if (warp == 5) {
+  if (warp >= 8) {
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_OTHER));
+   if (warp == 9) {
     // ------------------------------------------------------------ loader
     const bf16* Kc = (const bf16*)kv.K;
     const bf16* Vc = (const bf16*)kv.V;
@@ -335,7 +350,7 @@ __global__ void __launch_bounds__(NTH, 1)
         mbar_wait_drain(&v_full[j % NS], (j / NS) & 1);
       }
     }
-  } else if (warp == 4) {
+   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
       auto s_mma = [&](int j) {  // S(j) = Q K(j)^T into buffer j % 2
@@ -359,15 +374,14 @@ __global__ void __launch_bounds__(NTH, 1)
       for (int j = 0; j < n_tiles && ok; ++j) {
         const int st = j % NS;
         ok = mbar_wait(&v_full[st], (j / NS) & 1, abort_flag, kv.err) &&
-             mbar_wait(p_full, j & 1, abort_flag, kv.err);
+             mbar_wait(&p_full[j & 1], (j >> 1) & 1, abort_flag, kv.err);
         if (!ok) break;
         tc_fence_after();
         const uint32_t va = sb + V_OFF + st * TILE;
 #pragma unroll
         for (int kk = 0; kk < TK / 16; ++kk)
-          umma_ts(tmem + O_COL, tmem + (j & 1) * 128 + kk * 8, sw128_mn_desc(va + kk * 2048, PANEL), kIdescO,
-                  (j > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(pv_done);
+          umma_ts(tmem + O_COL + (j & 1) * 128, tmem + (j & 1) * 128 + kk * 8, sw128_mn_desc(va + kk * 2048, PANEL),
+                  kIdescO, (j > 1 || kk > 0) ? 1u : 0u);
         umma_commit(&v_empty[st]);
         if (j + 2 < n_tiles) {
           ok = mbar_wait(&k_full[(j + 2) % NS], ((j + 2) / NS) & 1, abort_flag, kv.err);
@@ -380,18 +394,22 @@ __global__ void __launch_bounds__(NTH, 1)
       mbar_wait_drain(o_full, 0);  // no MMA may still write TMEM when it is freed
     }
     __syncwarp();
-  } else if (warp < 4) {
+   }
+  } else {
+   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REG_SOFTMAX));
+   {
     // ------------------------------------------------------------ softmax
-    const int row = tid;
-    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const int half = warp >> 2, row = tid & 127;
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t o_col = O_COL + half * 128;
     const int pr = pf + row;
     float m_used = -1e30f, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
-      ok = warp_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag, kv.err);
+    for (int j = half; j < n_tiles; j += 2) {
+      ok = warp_wait(&s_full[half], (j >> 1) & 1, abort_flag, kv.err);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t s_col = (j & 1) * 128;
+      const uint32_t s_col = half * 128;
       uint32_t r[TK];
 #pragma unroll
       for (int c = 0; c < TK; c += 32) tmem_ld32(lane_addr + s_col + c, r + c);
@@ -412,23 +430,19 @@ __global__ void __launch_bounds__(NTH, 1)
         factor = ex2(m_used - mt);
         m_used = mt;
       }
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        // O holds tiles up to j - 1: wait for that product, rescale this row
-        ok = warp_wait(pv_done, (j - 1) & 1, abort_flag, kv.err);
-        if (!ok) break;
-        tc_fence_after();
+      if (j > 1 && __any_sync(0xffffffffu, grow)) {  // O_b holds this half's earlier tiles: rescale the row
 #pragma unroll 1
         for (int c = 0; c < HDT; c += 32) {
           uint32_t o[32];
-          tmem_ld32(lane_addr + O_COL + c, o);
+          tmem_ld32(lane_addr + o_col + c, o);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-          tmem_st32(lane_addr + O_COL + c, o);
+          tmem_st32(lane_addr + o_col + c, o);
         }
       }
       l *= factor;
-      // P = 2^(s - m) as bf16 pairs over the first 64 columns of S(j)'s
+      // P = 2^(s - m) as bf16 pairs over the first 64 columns of the
       // buffer, 16 columns (32 keys) at a time; two running sums
       float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
@@ -448,35 +462,51 @@ __global__ void __launch_bounds__(NTH, 1)
       l += rs0 + rs1;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[half]);
     }
-    // every product complete: normalise and store this row of O
+    // every product complete: merge the halves and store this row of O, the
+    // even half's warps the first 64 head dimensions, the odd half's the rest.
+    // Both halves are past their last tile, so every S product (the only
+    // readers of Q) is complete and Q's space takes the (max, sum) pairs.
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    half_ml[half * TQ + row] = make_float2(m_used, l);
+    asm volatile("bar.sync 1, 256;" ::: "memory");
     if (ok && warp_wait(o_full, 0, abort_flag, kv.err)) {
       tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float2 a = half_ml[row], b = half_ml[TQ + row];
+      const bool two = n_tiles > 1;  // O1 holds a product only when there are two tiles
+      const float mx = two ? fmaxf(a.x, b.x) : a.x;
+      const float w0 = ex2(a.x - mx), w1 = two ? ex2(b.x - mx) : 0.f;
+      const float lt = __fmaf_rn(a.y, w0, b.y * w1);
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
       bf16* dst = out + (size_t)(r0 + row) * qd + head * HDT;
 #pragma unroll 1
-      for (int c = 0; c < HDT; c += 32) {
-        uint32_t o[32];
-        tmem_ld32(lane_addr + O_COL + c, o);
+      for (int c = half * 64; c < half * 64 + 64; c += 32) {
+        uint32_t o0[32], o1[32];
+        tmem_ld32(lane_addr + O_COL + c, o0);
+        tmem_ld32(lane_addr + O_COL + 128 + c, o1);
         tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          o0[e] = __float_as_uint(__fmaf_rn(__uint_as_float(o0[e]), w0, two ? __uint_as_float(o1[e]) * w1 : 0.f));
         if (row < nrows) {
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
             uint4 u;
-            u.x = pack2(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
-            u.y = pack2(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
-            u.z = pack2(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
-            u.w = pack2(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
+            u.x = pack2(__uint_as_float(o0[e]) * inv, __uint_as_float(o0[e + 1]) * inv);
+            u.y = pack2(__uint_as_float(o0[e + 2]) * inv, __uint_as_float(o0[e + 3]) * inv);
+            u.z = pack2(__uint_as_float(o0[e + 4]) * inv, __uint_as_float(o0[e + 5]) * inv);
+            u.w = pack2(__uint_as_float(o0[e + 6]) * inv, __uint_as_float(o0[e + 7]) * inv);
             *reinterpret_cast<uint4*>(dst + c + e) = u;
           }
         }
       }
     }
+   }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 8) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
   }
