@@ -25,16 +25,16 @@ cudaError_t launch_attn_prefill_tc(int n_tiles, const int2* tiles, int H, int KV
                                    const bf16* kscr, const bf16* vscr, KVView kv, RowMeta m, bf16* out,
                                    cudaStream_t st);
 
-// The warp-specialised tcgen05 kernel (head_dim 128, 128-row tiles): one CTA
-// per work item {tile, head}.  prefill_ws_items (host) lists every (tile,
-// head), the heads of a tile next to each other, ordered by their number of
-// key tiles, largest first; tile_last_pos[t] is tile t's last position and
-// tile_window_first[t] the first position its first row sees (0 for full
-// attention).  Returns the count, or -1 past `cap`.  kv_rows: rows of
-// head_dim elements in each of kv.K, kv.V.
-int prefill_ws_items(int n_tiles, const int* tile_last_pos, const int* tile_window_first, int H, int2* items,
+// The warp-specialised tcgen05 kernel (head_dim 128, 128-row tiles): each
+// CTA runs one work item of two query slots that share a key/value stream.
+// prefill_ws_items (host) pairs the heads of each KV group on the same tile
+// (an odd head left over pairs consecutive tiles of one sequence) and orders
+// the items by their number of key tiles, largest first; tile_last_pos[t] and
+// tile_seq[t] are tile t's last position and sequence.  Returns the count, or
+// -1 past `cap`.  kv_rows: rows of head_dim elements in each of kv.K, kv.V.
+int prefill_ws_items(int n_tiles, const int* tile_last_pos, const int* tile_seq, int H, int KV, int4* items,
                      int cap);
-cudaError_t launch_attn_prefill_ws(int n_items, const int2* items, const int2* tiles, int M, int H, int KV, int hd,
+cudaError_t launch_attn_prefill_ws(int n_items, const int4* items, const int2* tiles, int M, int H, int KV, int hd,
                                    const bf16* qh, const bf16* kscr, const bf16* vscr, KVView kv, size_t kv_rows,
                                    RowMeta m, bf16* out, cudaStream_t st);
 

@@ -1,35 +1,33 @@
 // Prefill attention, warp-specialised for the 5th-generation tensor cores
-// (bf16, head_dim 128).  Each CTA runs one work item: 128 query rows of one
-// head, over the key tiles its rows see.
+// (bf16, head_dim 128).  Each CTA runs two query slots of 128 rows that share
+// one key/value stream: two query heads of one KV group on the same rows, or
+// one head on two consecutive row tiles of the same sequence.
 //
-//   warps 0-3  softmax of the even key tiles, one query row per thread
-//              (= TMEM lane)
-//   warps 4-7  softmax of the odd key tiles, the same rows
+//   warps 0-3  softmax of slot 0, one query row per thread (= TMEM lane)
+//   warps 4-7  softmax of slot 1
 //   warp 8     allocates TMEM; one lane issues every MMA and commit
 //   warp 9     loader: Q once, then K and V tiles of 128 keys into a
-//              three-stage ring, by TMA when a tile is one run of rows of
-//              the chunk scratch or of the cache, else by cp.async row by row
+//              two-stage ring, by TMA when a tile is one run of rows of the
+//              chunk scratch or of the cache, else by cp.async row by row
 //   warps 10-11 idle (they complete the third warpgroup)
 // The CTA launches with 168 registers a thread; the third warpgroup gives
 // back all but 72 and the softmax warpgroups take them (216 each), enough to
 // hold a row of S.
 //
-// TMEM (512 columns): S buffers 0 and 1 at [0,128) and [128,256), O0 at
-// [256,384), O1 at [384,512).  Key tile j belongs to half b = j % 2: S(j) =
-// Q K(j)^T goes to buffer b, the softmax warpgroup b turns it into P(j)
-// (bf16 pairs over the first 64 columns of the buffer) and O_b += P(j) V(j).
-// Each half keeps its own running maximum, sum and O, so the two warpgroups
-// work on consecutive tiles at the same time; the halves are merged once at
-// the end.  The MMA lane issues, per tile j, O_b += P(j) V(j) (P from TMEM)
-// and then S(j+2) into the same buffer (the tensor core runs one lane's
-// products in order, so P(j) is read before S(j+2) overwrites it; the commit
-// after S(j+2) covers O_b += P(j) V(j), so a warpgroup that sees S(j+2) may
-// rescale O_b).  V stays as loaded (keys x head dims): the P V product reads
-// it as an MN-major operand, so nothing is transposed.
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
+// Per key tile j the MMA lane issues, for each slot q in turn,
+//   O_q += P_q(j) V(j)      (P_q from TMEM, written over the first 64
+//                            columns of S_q by the softmax as bf16 pairs)
+//   S_q(j+1) = Q_q K(j+1)^T
+// so one slot's softmax runs while the tensor core works on the other's
+// products.  The commit after S_q(j+1) also covers O_q += P_q(j): when the
+// softmax sees S_q(j+1) the slot's O is complete up to tile j and may be
+// rescaled.  V stays as loaded (keys x head dims); the P V product reads it
+// as an MN-major operand, so nothing is transposed.
 //
-// Softmax in base 2 (Q is pre-scaled by log2(e)/sqrt(head_dim)) with a lazy
-// running maximum: O and the row sum are rescaled only when a row maximum
-// grows by more than 8 (P = 2^(s - m) then stays below 256).
+// Softmax in base 2 (Q is pre-scaled by log2(e)/sqrt(head_dim)) with the
+// lazy running maximum of the single-tile kernel: O and the row sum are
+// rescaled only when a row maximum grows by more than 8.
 //
 // Every mbarrier wait is bounded; on expiry the CTA sets the device error
 // word, every role stops, the loader waits (bounded) for its copies in flight
@@ -53,9 +51,9 @@ namespace {
 using namespace tc;
 
 constexpr int HDT = 128;               // head dimensions
-constexpr int TQ = 128;                // query rows per item
+constexpr int TQ = 128;                // query rows per slot
 constexpr int TK = 128;                // keys per tile
-constexpr int NS = 3;                  // K/V ring stages
+constexpr int NS = 2;                  // K/V ring stages
 constexpr int NTH = 384;               // 12 warps, three warpgroups
 constexpr int REG_SOFTMAX = 216, REG_OTHER = 72;  // 2 x 128 x 216 + 128 x 72 = 384 x 168
 static_assert(2 * 128 * REG_SOFTMAX + 128 * REG_OTHER <= NTH * 168, "register split exceeds the launch's registers");
@@ -63,14 +61,12 @@ constexpr int PANEL = 128 * 128;       // 64 head dims x 128 rows, bytes
 constexpr int TILE = 2 * PANEL;        // one Q, K or V tile, bytes
 constexpr float kLazy = 8.f;
 
-constexpr int Q_OFF = 0;
-constexpr int K_OFF = Q_OFF + TILE;            // NS stages
+constexpr int Q_OFF = 0;                       // 2 slots
+constexpr int K_OFF = Q_OFF + 2 * TILE;        // NS stages
 constexpr int V_OFF = K_OFF + NS * TILE;       // NS stages
 constexpr int BAR_OFF = V_OFF + NS * TILE;     // mbarriers, TMEM slot, flags
 constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
 constexpr int TMEM_COLS = 512;
-constexpr uint32_t O_COL = 256;  // O_b at O_COL + 128 b
 
 __device__ __forceinline__ uint32_t sw(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 
@@ -203,12 +199,20 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 constexpr uint32_t kIdescS = idesc_bf16(TQ, TK);                // Q K^T: both K-major
 constexpr uint32_t kIdescO = idesc_bf16(TQ, HDT) | (1u << 16);  // P V: B (V) MN-major
 
+// Per-slot geometry shared by every role (all computed from the row
+// metadata, so each role takes the same decisions).
+struct Slot {
+  int r0, nrows, head, pf, pl, a, b;  // a..b: key tiles this slot reads (relative to kt0)
+};
+
+// 12 warps: three share a scheduler, whose 16K registers cap a thread at 168
+// at launch.
 __global__ void __launch_bounds__(NTH, 1)
     k_attn_prefill_ws(int KV, int G, const __grid_constant__ CUtensorMap map_q,
                       const __grid_constant__ CUtensorMap map_ks, const __grid_constant__ CUtensorMap map_vs,
                       const __grid_constant__ CUtensorMap map_kc, const __grid_constant__ CUtensorMap map_vc,
                       const bf16* __restrict__ kscr, const bf16* __restrict__ vscr, KVView kv, RowMeta m,
-                      const int2* __restrict__ tiles, const int2* __restrict__ items, bf16* __restrict__ out) {
+                      const int2* __restrict__ tiles, const int4* __restrict__ items, bf16* __restrict__ out) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sb = smem_u32(smem);
@@ -218,14 +222,11 @@ __global__ void __launch_bounds__(NTH, 1)
   uint64_t* v_full = k_full + NS;         // [NS]
   uint64_t* k_empty = v_full + NS;        // [NS]
   uint64_t* v_empty = k_empty + NS;       // [NS]
-  uint64_t* s_full = v_empty + NS;        // [2]: S(j) in buffer j % 2
-  uint64_t* p_full = s_full + 2;          // [2]: P(j) written (all 128 rows of half j % 2)
-  uint64_t* o_full = p_full + 2;          // every product complete
+  uint64_t* s_full = v_empty + NS;        // [2]
+  uint64_t* p_full = s_full + 2;          // [2]
+  uint64_t* o_full = p_full + 2;
   uint32_t* tmem_slot = (uint32_t*)(o_full + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
-  // [2][128]: each half's (max, sum) per row, written over Q once every S
-  // product is complete
-  float2* half_ml = (float2*)(smem + Q_OFF);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
@@ -258,17 +259,40 @@ __global__ void __launch_bounds__(NTH, 1)
   pdl_wait();  // queries, chunk keys and row metadata come from earlier kernels
   pdl_trigger();
 
-  // ---- the work item: 128 rows (one tile of one sequence) of one head
-  const int2 it = items[blockIdx.x];  // {tile, head}
+  // ---- the work item: one or two slots of one KV group and one sequence
+  const int4 it = items[blockIdx.x];
+  const int nslot = it.z >= 0 ? 2 : 1;
   const int H = KV * G, qd = H * HDT;
-  const int head = it.y, g = head / G;
-  const int2 tl = tiles[it.x];
-  const int r0 = tl.x, nrows = tl.y - tl.x;
-  const int pf = m.pos[r0], pl = m.pos[tl.y - 1];
-  const int lo = kv.window > 0 ? max(0, pf - kv.window + 1) : 0;
-  const int kt0 = (lo / TK) * TK;
-  const int n_tiles = pl / TK - lo / TK + 1;
-  const int seq = m.seq[r0], p0 = m.p0[r0], base = m.base[r0];
+  const int g = it.y / G;
+  Slot sl[2];
+  int lo_t = INT_MAX, hi_t = 0;
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const int2 tl = tiles[q == 0 ? it.x : (nslot == 2 ? it.z : it.x)];
+    Slot& s = sl[q];
+    s.r0 = tl.x;
+    s.nrows = tl.y - tl.x;
+    s.head = q == 0 ? it.y : it.w;
+    s.pf = m.pos[tl.x];
+    s.pl = m.pos[tl.y - 1];
+    const int lo = kv.window > 0 ? max(0, s.pf - kv.window + 1) : 0;
+    s.a = lo / TK;
+    s.b = s.pl / TK;
+    if (q < nslot) {
+      lo_t = min(lo_t, s.a);
+      hi_t = max(hi_t, s.b);
+    }
+  }
+  const int n_tiles = hi_t - lo_t + 1;
+  const int kt0 = lo_t * TK;
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    sl[q].a -= lo_t;
+    sl[q].b -= lo_t;
+  }
+  const int r_ref = sl[0].r0;
+  const int seq = m.seq[r_ref], p0 = m.p0[r_ref], base = m.base[r_ref];
+  const int k_last = max(sl[0].pl, nslot == 2 ? sl[1].pl : 0);  // last key position any slot reads
 
   if (warp >= 8) {
    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_OTHER));
@@ -278,9 +302,12 @@ __global__ void __launch_bounds__(NTH, 1)
     const bf16* Vc = (const bf16*)kv.V;
     const int page = kv.pt ? (1 << kv.page_shift) : 0;
     if (lane == 0) {
-      mbar_expect_tx(q_full, TILE);
-      tma2d(sb + Q_OFF, &map_q, q_full, head * HDT, r0);
-      tma2d(sb + Q_OFF + PANEL, &map_q, q_full, head * HDT + 64, r0);
+      mbar_expect_tx(q_full, (uint32_t)(nslot * TILE));
+#pragma unroll
+      for (int q = 0; q < 2; ++q)
+        if (q < nslot)
+          for (int p = 0; p < 2; ++p)
+            tma2d(sb + Q_OFF + q * TILE + p * PANEL, &map_q, q_full, sl[q].head * HDT + p * 64, sl[q].r0);
     }
     int issued = 0;
     bool ok = true;
@@ -296,7 +323,8 @@ __global__ void __launch_bounds__(NTH, 1)
       // one run of rows: the chunk scratch, or the cache without a ring wrap
       // or page change inside the tile
       const bool scr = kt >= p0;
-      const bool cache_run = !scr && kt + TK - 1 < p0 && (kv.pt ? page >= TK : (kt % kv.cap) + TK <= kv.cap);
+      const bool cache_run = !scr && kt + TK - 1 < p0 &&
+                             (kv.pt ? page >= TK : (kt % kv.cap) + TK <= kv.cap);
       if (scr || cache_run) {
         if (lane == 0) {
           const CUtensorMap* mk = scr ? &map_ks : &map_kc;
@@ -311,12 +339,12 @@ __global__ void __launch_bounds__(NTH, 1)
           tma2d(dv + PANEL, mv, &v_full[st], x0 + 64, y);
         }
       } else {
-        // row by row: positions past the tile's last row are zero
+        // row by row: positions past the last key any slot reads are zero
         const int kvd = KV * HDT;
         for (int i = lane; i < TK * 16; i += 32) {
           const int row = i >> 4, c = i & 15;
           const int jp = kt + row;
-          const bool valid = jp <= pl;
+          const bool valid = jp <= k_last;
           const bf16 *ks = kscr, *vs = vscr;
           if (valid && jp >= p0) {
             const size_t o = (size_t)(base + jp - p0) * kvd + g * HDT + c * 8;
@@ -350,45 +378,60 @@ __global__ void __launch_bounds__(NTH, 1)
         mbar_wait_drain(&v_full[j % NS], (j / NS) & 1);
       }
     }
-   } else if (warp == 8) {
+  } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
-      auto s_mma = [&](int j) {  // S(j) = Q K(j)^T into buffer j % 2
-        const uint32_t ka = sb + K_OFF + (j % NS) * TILE;
+      auto s_mma = [&](int q, int st) {
+        const uint32_t qa = sb + Q_OFF + q * TILE, ka = sb + K_OFF + st * TILE;
 #pragma unroll
         for (int kk = 0; kk < HDT / 16; ++kk) {
-          const uint64_t a = sw128_desc(sb + Q_OFF + (kk >> 2) * PANEL) + 2 * (kk & 3);
+          const uint64_t a = sw128_desc(qa + (kk >> 2) * PANEL) + 2 * (kk & 3);
           const uint64_t b = sw128_desc(ka + (kk >> 2) * PANEL) + 2 * (kk & 3);
-          umma(tmem + (j & 1) * 128, a, b, kIdescS, kk > 0 ? 1u : 0u);
+          umma(tmem + q * 128, a, b, kIdescS, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&s_full[j & 1]);
-        umma_commit(&k_empty[j % NS]);
+        umma_commit(&s_full[q]);
       };
-      bool ok = mbar_wait(q_full, 0, abort_flag, kv.err);
-      for (int j = 0; j < 2 && j < n_tiles && ok; ++j) {
-        ok = mbar_wait(&k_full[j % NS], (j / NS) & 1, abort_flag, kv.err);
-        if (!ok) break;
+      bool ok = mbar_wait(q_full, 0, abort_flag, kv.err) && mbar_wait(&k_full[0], 0, abort_flag, kv.err);
+      if (ok) {
         tc_fence_after();
-        s_mma(j);
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+          if (q < nslot && sl[q].a == 0) s_mma(q, 0);
+        umma_commit(&k_empty[0]);
       }
       for (int j = 0; j < n_tiles && ok; ++j) {
         const int st = j % NS;
-        ok = mbar_wait(&v_full[st], (j / NS) & 1, abort_flag, kv.err) &&
-             mbar_wait(&p_full[j & 1], (j >> 1) & 1, abort_flag, kv.err);
+        ok = mbar_wait(&v_full[st], (j / NS) & 1, abort_flag, kv.err);
         if (!ok) break;
-        tc_fence_after();
-        const uint32_t va = sb + V_OFF + st * TILE;
+        const int j1 = j + 1, st1 = j1 % NS;
+        bool k_next = false;
 #pragma unroll
-        for (int kk = 0; kk < TK / 16; ++kk)
-          umma_ts(tmem + O_COL + (j & 1) * 128, tmem + (j & 1) * 128 + kk * 8, sw128_mn_desc(va + kk * 2048, PANEL),
-                  kIdescO, (j > 1 || kk > 0) ? 1u : 0u);
-        umma_commit(&v_empty[st]);
-        if (j + 2 < n_tiles) {
-          ok = mbar_wait(&k_full[(j + 2) % NS], ((j + 2) / NS) & 1, abort_flag, kv.err);
-          if (!ok) break;
-          tc_fence_after();
-          s_mma(j + 2);
+        for (int q = 0; q < 2; ++q) {
+          if (q >= nslot || !ok) break;
+          const Slot& s = sl[q];
+          if (j >= s.a && j <= s.b) {
+            ok = mbar_wait(&p_full[q], (j - s.a) & 1, abort_flag, kv.err);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t va = sb + V_OFF + st * TILE;
+#pragma unroll
+            for (int kk = 0; kk < TK / 16; ++kk)
+              umma_ts(tmem + 256 + q * 128, tmem + q * 128 + kk * 8, sw128_mn_desc(va + kk * 2048, PANEL),
+                      kIdescO, (j > s.a || kk > 0) ? 1u : 0u);
+          }
+          if (j1 >= s.a && j1 <= s.b) {
+            if (!k_next) {
+              ok = mbar_wait(&k_full[st1], (j1 / NS) & 1, abort_flag, kv.err);
+              if (!ok) break;
+              tc_fence_after();
+              k_next = true;
+            }
+            s_mma(q, st1);
+          }
         }
+        if (!ok) break;
+        umma_commit(&v_empty[st]);
+        if (j1 < n_tiles) umma_commit(&k_empty[st1]);
       }
       umma_commit(o_full);
       mbar_wait_drain(o_full, 0);  // no MMA may still write TMEM when it is freed
@@ -397,26 +440,26 @@ __global__ void __launch_bounds__(NTH, 1)
    }
   } else {
    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REG_SOFTMAX));
-   {
+   if (warp / 4 < nslot) {
     // ------------------------------------------------------------ softmax
-    const int half = warp >> 2, row = tid & 127;
+    const int q = warp >> 2, row = tid & 127;
+    const Slot s = q ? sl[1] : sl[0];
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    const uint32_t o_col = O_COL + half * 128;
-    const int pr = pf + row;
+    const uint32_t s_col = q * 128, o_col = 256 + q * 128;
+    const int pr = s.pf + row;
     float m_used = -1e30f, l = 0.f;
     bool ok = true;
-    for (int j = half; j < n_tiles; j += 2) {
-      ok = warp_wait(&s_full[half], (j >> 1) & 1, abort_flag, kv.err);
+    for (int j = s.a; j <= s.b; ++j) {
+      ok = warp_wait(&s_full[q], (j - s.a) & 1, abort_flag, kv.err);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t s_col = half * 128;
       uint32_t r[TK];
 #pragma unroll
       for (int c = 0; c < TK; c += 32) tmem_ld32(lane_addr + s_col + c, r + c);
       tmem_wait_ld();
       const int kt = kt0 + j * TK;
-      // a tile every row of the item sees whole needs no mask
-      const bool open = kt + TK - 1 <= pf && (kv.window == 0 || kt >= pl - kv.window + 1);
+      // a tile every row of the slot sees whole needs no mask
+      const bool open = kt + TK - 1 <= s.pf && (kv.window == 0 || kt >= s.pl - kv.window + 1);
       if (!open) {  // key kt + c is visible iff c_lo <= c <= c_hi
         const int c_hi = pr - kt, c_lo = kv.window > 0 ? pr - kv.window + 1 - kt : -1;
 #pragma unroll
@@ -430,7 +473,7 @@ __global__ void __launch_bounds__(NTH, 1)
         factor = ex2(m_used - mt);
         m_used = mt;
       }
-      if (j > 1 && __any_sync(0xffffffffu, grow)) {  // O_b holds this half's earlier tiles: rescale the row
+      if (j > s.a && __any_sync(0xffffffffu, grow)) {  // O holds earlier tiles: rescale this row
 #pragma unroll 1
         for (int c = 0; c < HDT; c += 32) {
           uint32_t o[32];
@@ -442,8 +485,8 @@ __global__ void __launch_bounds__(NTH, 1)
         }
       }
       l *= factor;
-      // P = 2^(s - m) as bf16 pairs over the first 64 columns of the
-      // buffer, 16 columns (32 keys) at a time; two running sums
+      // P = 2^(s - m) as bf16 pairs over the first 64 columns of S, 16
+      // columns (32 keys) at a time; two running sums (even, odd keys)
       float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
@@ -462,47 +505,32 @@ __global__ void __launch_bounds__(NTH, 1)
       l += rs0 + rs1;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[half]);
+      mbar_arrive(&p_full[q]);
     }
-    // every product complete: merge the halves and store this row of O, the
-    // even half's warps the first 64 head dimensions, the odd half's the rest.
-    // Both halves are past their last tile, so every S product (the only
-    // readers of Q) is complete and Q's space takes the (max, sum) pairs.
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    half_ml[half * TQ + row] = make_float2(m_used, l);
-    asm volatile("bar.sync 1, 256;" ::: "memory");
+    // every product of this CTA complete: normalise and store this row of O
     if (ok && warp_wait(o_full, 0, abort_flag, kv.err)) {
       tc_fence_after();
-      const float2 a = half_ml[row], b = half_ml[TQ + row];
-      const bool two = n_tiles > 1;  // O1 holds a product only when there are two tiles
-      const float mx = two ? fmaxf(a.x, b.x) : a.x;
-      const float w0 = ex2(a.x - mx), w1 = two ? ex2(b.x - mx) : 0.f;
-      const float lt = __fmaf_rn(a.y, w0, b.y * w1);
-      const float inv = lt > 0.f ? 1.f / lt : 0.f;
-      bf16* dst = out + (size_t)(r0 + row) * qd + head * HDT;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      bf16* dst = out + (size_t)(s.r0 + row) * qd + s.head * HDT;
 #pragma unroll 1
-      for (int c = half * 64; c < half * 64 + 64; c += 32) {
-        uint32_t o0[32], o1[32];
-        tmem_ld32(lane_addr + O_COL + c, o0);
-        tmem_ld32(lane_addr + O_COL + 128 + c, o1);
+      for (int c = 0; c < HDT; c += 32) {
+        uint32_t o[32];
+        tmem_ld32(lane_addr + o_col + c, o);
         tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          o0[e] = __float_as_uint(__fmaf_rn(__uint_as_float(o0[e]), w0, two ? __uint_as_float(o1[e]) * w1 : 0.f));
-        if (row < nrows) {
+        if (row < s.nrows) {
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
             uint4 u;
-            u.x = pack2(__uint_as_float(o0[e]) * inv, __uint_as_float(o0[e + 1]) * inv);
-            u.y = pack2(__uint_as_float(o0[e + 2]) * inv, __uint_as_float(o0[e + 3]) * inv);
-            u.z = pack2(__uint_as_float(o0[e + 4]) * inv, __uint_as_float(o0[e + 5]) * inv);
-            u.w = pack2(__uint_as_float(o0[e + 6]) * inv, __uint_as_float(o0[e + 7]) * inv);
+            u.x = pack2(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
+            u.y = pack2(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+            u.z = pack2(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
+            u.w = pack2(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
             *reinterpret_cast<uint4*>(dst + c + e) = u;
           }
         }
       }
     }
-   }
+  }
   }
   tc_fence_before();
   __syncthreads();
@@ -570,26 +598,40 @@ bool map_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint6
 
 }  // namespace
 
-int prefill_ws_items(int n_tiles, const int* tile_last_pos, const int* tile_window_first, int H, int2* items,
+int prefill_ws_items(int n_tiles, const int* tile_last_pos, const int* tile_seq, int H, int KV, int4* items,
                      int cap) {
+  const int G = H / KV;
   struct Item {
-    int2 v;
+    int4 v;
     int cost;
   };
   std::vector<Item> list;
   list.reserve((size_t)n_tiles * H);
-  // heads of one tile next to each other: a KV group's heads read the same
-  // key tiles at about the same time, from L2
-  for (int t = 0; t < n_tiles; ++t)
-    for (int h = 0; h < H; ++h)
-      list.push_back({make_int2(t, h), tile_last_pos[t] / TK - tile_window_first[t] / TK + 1});
+  for (int g = 0; g < KV; ++g) {
+    // head pairs on the same rows
+    for (int t = 0; t < n_tiles; ++t)
+      for (int h = g * G; h + 1 < (g + 1) * G; h += 2)
+        list.push_back({make_int4(t, h, t, h + 1), tile_last_pos[t] / TK + 1});
+    if (G % 2 == 0) continue;
+    // the odd head: consecutive row tiles of one sequence
+    const int h = (g + 1) * G - 1;
+    for (int t = 0; t < n_tiles;) {
+      if (t + 1 < n_tiles && tile_seq[t + 1] == tile_seq[t]) {
+        list.push_back({make_int4(t, h, t + 1, h), tile_last_pos[t + 1] / TK + 1});
+        t += 2;
+      } else {
+        list.push_back({make_int4(t, h, -1, -1), tile_last_pos[t] / TK + 1});
+        t += 1;
+      }
+    }
+  }
   if ((int)list.size() > cap) return -1;
   std::stable_sort(list.begin(), list.end(), [](const Item& a, const Item& b) { return a.cost > b.cost; });
   for (size_t i = 0; i < list.size(); ++i) items[i] = list[i].v;
   return (int)list.size();
 }
 
-cudaError_t launch_attn_prefill_ws(int n_items, const int2* items, const int2* tiles, int M, int H, int KV, int hd,
+cudaError_t launch_attn_prefill_ws(int n_items, const int4* items, const int2* tiles, int M, int H, int KV, int hd,
                                    const bf16* qh, const bf16* kscr, const bf16* vscr, KVView kv, size_t kv_rows,
                                    RowMeta m, bf16* out, cudaStream_t st) {
   if (hd != HDT || H % KV) return cudaErrorNotSupported;

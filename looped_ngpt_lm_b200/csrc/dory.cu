@@ -124,8 +124,7 @@ struct dory_handle {
   int *cu = nullptr, *head_rows = nullptr;
   int2* tiles = nullptr;  // prefill attention tiles (64 or 128 rows of one sequence)
   int tiles_cap = 0;
-  int2* pf_items[2] = {nullptr, nullptr};  // warp-specialised prefill attention work items:
-                                           // [0] sliding-window layers, [1] full layers
+  int4* pf_items = nullptr;  // warp-specialised prefill attention: CTA work items
   int items_cap = 0;
   void* qh = nullptr;     // bf16 pre-scaled queries of long chunks
   RowMeta meta{};
@@ -157,7 +156,7 @@ struct dory_handle {
   int* page_table = nullptr;
   int pt_stride = 0, page_shift = 0, pool_pages = 0;
   std::vector<int> pt_host, free_pages;
-  std::vector<int2> items_host;
+  std::vector<int4> items_host;
   std::vector<std::vector<int>> seq_pages;
   std::vector<int> ids_on_device;     // seq ids last uploaded to seq_ids
   int last_rows = 0;
@@ -283,7 +282,7 @@ size_t layout(dory_handle* h) {
   h->tiles_cap = M / 64 + c.max_batch + 1;
   h->tiles = cv.take<int2>(sizeof(int2) * h->tiles_cap);
   h->items_cap = h->tiles_cap * c.n_heads;
-  for (int i = 0; i < 2; ++i) h->pf_items[i] = cv.take<int2>(sizeof(int2) * h->items_cap);
+  h->pf_items = cv.take<int4>(sizeof(int4) * h->items_cap);
   h->qh = cv.take<char>(2 * (size_t)M * h->q_dim);
   h->meta.seq = cv.take<int>(sizeof(int) * M);
   h->meta.pos = cv.take<int>(sizeof(int) * M);
@@ -381,7 +380,7 @@ struct Fwd {
   bool invariant;  // decode / speculative rows: GEMM arithmetic independent of M
   int n_tiles = 0;  // > 0: long-chunk attention on the tensor cores over H->tiles
   int tc5 = 0;      // ... by a tcgen05 kernel (128-row tiles): 2 one slot per CTA, 3 warp-specialised
-  int n_items[2] = {0, 0};  // work items of the warp-specialised kernel (H->pf_items)
+  int n_items = 0;  // work items of the warp-specialised kernel (H->pf_items)
   int pf_k = 0;     // > 0: GEMMs follow the weight stream of a pf_k-loop decode step
   bool stage = true;  // layer updates may run in the next GEMM's operand stage
 };
@@ -638,12 +637,10 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop, float* copy_la
         }
         if (tc) {
           Scope sc(H, f.st, "attn_prefill", 0);
-          if (f.tc5 == 3) {
-            const int full = kv.window > 0 ? 0 : 1;
-            CK(launch_attn_prefill_ws(f.n_items[full], H->pf_items[full], H->tiles, M, c.n_heads, c.n_kv_heads,
-                                      c.head_dim, (const bf16*)H->qh, (const bf16*)H->kscr, (const bf16*)H->vscr,
-                                      kv, kv_rows(H, l), H->meta, (bf16*)H->ao, f.st));
-          }
+          if (f.tc5 == 3)
+            CK(launch_attn_prefill_ws(f.n_items, H->pf_items, H->tiles, M, c.n_heads, c.n_kv_heads, c.head_dim,
+                                      (const bf16*)H->qh, (const bf16*)H->kscr, (const bf16*)H->vscr, kv,
+                                      kv_rows(H, l), H->meta, (bf16*)H->ao, f.st));
           else if (f.tc5 == 2)
             CK(launch_attn_prefill_tc(f.n_tiles, H->tiles, c.n_heads, c.n_kv_heads, c.head_dim, (const bf16*)H->qh,
                                       (const bf16*)H->kscr, (const bf16*)H->vscr, kv, H->meta, (bf16*)H->ao, f.st));
@@ -871,22 +868,19 @@ dory_status prefill_t(dory_handle* H, int batch, const int32_t* seq_ids, const i
     CK(cudaMemcpyAsync(H->tiles, tl.data(), sizeof(int2) * n, cudaMemcpyHostToDevice, st));
     f.n_tiles = n;
     if (f.tc5 == 3) {
-      // each tile's last position and the first position its first row sees:
-      // one item table for the sliding-window layers and one for the full ones
-      std::vector<int> last(n), first(n);
-      for (int w = 0; w < 2; ++w) {
-        for (int t = 0, b = 0; t < n; ++t) {
-          while (tl[t].x >= cu[b + 1]) ++b;
-          const int p_first = H->len[seq_ids[b]] + (tl[t].x - cu[b]);
-          last[t] = H->len[seq_ids[b]] + (tl[t].y - 1 - cu[b]);
-          first[t] = w == 0 && c.swa_window > 0 ? std::max(0, p_first - c.swa_window + 1) : 0;
-        }
-        H->items_host.resize(H->items_cap);
-        const int ni = prefill_ws_items(n, last.data(), first.data(), c.n_heads, H->items_host.data(), H->items_cap);
-        if (ni < 0) return fail(DORY_ERR_CAPACITY, "too many prefill attention items");
-        CK(cudaMemcpyAsync(H->pf_items[w], H->items_host.data(), sizeof(int2) * ni, cudaMemcpyHostToDevice, st));
-        f.n_items[w] = ni;
+      // each tile's sequence and last position, for pairing and ordering
+      std::vector<int> last(n), sq(n);
+      for (int t = 0, b = 0; t < n; ++t) {
+        while (tl[t].x >= cu[b + 1]) ++b;
+        sq[t] = b;
+        last[t] = H->len[seq_ids[b]] + (tl[t].y - 1 - cu[b]);
       }
+      H->items_host.resize(H->items_cap);
+      const int ni = prefill_ws_items(n, last.data(), sq.data(), c.n_heads, c.n_kv_heads, H->items_host.data(),
+                                      H->items_cap);
+      if (ni < 0) return fail(DORY_ERR_CAPACITY, "too many prefill attention items");
+      CK(cudaMemcpyAsync(H->pf_items, H->items_host.data(), sizeof(int4) * ni, cudaMemcpyHostToDevice, st));
+      f.n_items = ni;
     }
   }
   RET(input_block<T>(f, tokens));
