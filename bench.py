@@ -570,6 +570,8 @@ def main():
     ap.add_argument("--fused-rows", dest="fused_rows", type=int, default=None,
                     help="operand stages for decode passes of at most this many rows (0 = off; default: the "
                          "library's)")
+    ap.add_argument("--l2-own", dest="l2_own", type=int, default=None,
+                    help="own weight tiles each decode GEMM CTA prefetches into L2 before its wait (DORY_OPT_L2_OWN)")
     ap.add_argument("--prefill-tc", dest="prefill_tc", type=int, default=None,
                     help="prefill attention kernel (DORY_OPT_PREFILL_TC; default: the library's)")
     ap.add_argument("--attn-cluster", dest="attn_cluster", type=int, default=None,
@@ -638,6 +640,8 @@ def main():
         h.set_option(dory.OPT_ATTN_CLUSTER, args.attn_cluster)
     if args.prefill_tc is not None:
         h.set_option(dory.OPT_PREFILL_TC, args.prefill_tc)
+    if args.l2_own is not None:
+        h.set_option(dory.OPT_L2_OWN, args.l2_own)
     mode = dory.MODES[args.mode]
     stream = torch.cuda.current_stream()
     prompt = torch.tensor(synth.make_prompt(1, args.prompt, shape.vocab), dtype=torch.int32, device="cuda")

@@ -474,7 +474,12 @@ enum {
    * is launched, before it waits for the attention, instead of the
    * DORY_OPT_L2_LOOKAHEAD range after its loads (default 0: that range).
    * Changes only when HBM reads happen, never what is computed. */
-  DORY_OPT_ATTN_LOOKAHEAD = 10
+  DORY_OPT_ATTN_LOOKAHEAD = 10,
+  /* bf16 decode GEMMs: before waiting for the previous kernel, each CTA asks
+   * L2 for up to this many of its own weight tiles past those its
+   * shared-memory ring takes (TMA prefetch; 0 turns it off).  Changes only
+   * when HBM reads happen, never what is computed. */
+  DORY_OPT_L2_OWN = 11
 };
 dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value);
 

@@ -31,6 +31,7 @@ OPT_L2_LOOKAHEAD = 7
 OPT_MX_GEMV = 8
 OPT_FUSED_OPERANDS = 9
 OPT_ATTN_LOOKAHEAD = 10
+OPT_L2_OWN = 11
 
 STATUS = {0: "DORY_OK", 1: "DORY_ERR_INVALID_ARG", 2: "DORY_ERR_CAPACITY", 3: "DORY_ERR_STATE",
           4: "DORY_ERR_WORKSPACE", 5: "DORY_ERR_CUDA", 6: "DORY_ERR_TIMEOUT", 7: "DORY_ERR_UNSUPPORTED"}

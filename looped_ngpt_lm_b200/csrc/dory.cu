@@ -166,6 +166,7 @@ struct dory_handle {
   int gemm_impl = 0;
   unsigned long long pf_lead = 8ull << 20;   // 0: no L2 look-ahead
   unsigned long long pf_attn = 0;            // early look-ahead of the GEMM after a decode attention (0: none)
+  int pf_own = 0;                            // own weight tiles a decode GEMM CTA prefetches before its wait
   float temperature = 0.f, top_p = 1.f;      // temperature 0: greedy
   unsigned long long seed = 0;
   std::vector<std::vector<PfSeg>> pf_host;   // [k] -> stream of a k-loop decode step
@@ -512,6 +513,10 @@ dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, cons
       // L2 look-ahead while this GEMM is the next one of the weight stream
       PfCtl pfc;
       const PfCtl* pp = nullptr;
+      if (f.invariant && H->pf_own > 0) {
+        pfc.own = H->pf_own;
+        pp = &pfc;
+      }
       if (f.pf_k > 0 && H->pf_pos >= 0) {
         const std::vector<PfSeg>& v = H->pf_host[f.pf_k];
         if (H->pf_pos < (int)v.size() && v[H->pf_pos].p == (const char*)W) {
@@ -1558,6 +1563,15 @@ dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value) {
     case DORY_OPT_GEMM_IMPL:
       if (value < 0 || value > 2) return fail(DORY_ERR_INVALID_ARG, "bad GEMM impl");
       h->gemm_impl = (int)value;
+      return DORY_OK;
+    case DORY_OPT_L2_OWN:
+      if (value < 0 || value > (1 << 20)) return fail(DORY_ERR_INVALID_ARG, "bad own-tile prefetch count");
+      if (value != h->pf_own) {
+        for (auto& g : h->graphs_cache)
+          if (g.exec) cudaGraphExecDestroy(g.exec);
+        h->graphs_cache.clear();
+      }
+      h->pf_own = (int)value;
       return DORY_OK;
     case DORY_OPT_ATTN_LOOKAHEAD:
       if (value < 0 || value > (1ll << 40)) return fail(DORY_ERR_INVALID_ARG, "bad look-ahead");

@@ -53,6 +53,17 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// A TMA box of a 2-D tensor map, global -> L2 only.
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
+               : "memory");
+}
+
+// Bytes at a 16-byte aligned address (a multiple of 16), global -> L2 only.
+__device__ __forceinline__ void bulk_prefetch(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Untiled bulk copy global -> shared (16-byte aligned, size a multiple of 16).
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t policy) {
   asm volatile(
@@ -312,6 +323,27 @@ __global__ void __launch_bounds__(192, 1)
         pre_mt[npre] = mt;
         ++npre;
         next();
+      }
+      if (pf.own > 0) {
+        // ask L2 for the CTA's next weight tiles while the previous kernel
+        // still runs (the ring above holds the first STAGES of them)
+        int u2 = u, nt2 = nt, mt2 = mt, s2 = s, kb2 = kb, kb12 = kb1;
+        for (int c = 0; c < pf.own && u2 < um.units; ++c) {
+          if constexpr (PACK) {
+            bulk_prefetch(Apack + ((size_t)nt2 * k_tiles + (size_t)kb2 * KSUB) * TL::A_SUB, TL::A_BYTES);
+          } else {
+#pragma unroll
+            for (int q = 0; q < KSUB; ++q) tma_prefetch_2d(&mapA, (kb2 * KSUB + q) * BK, nt2 * BM);
+            if constexpr (GLU) {
+#pragma unroll
+              for (int q = 0; q < KSUB; ++q) tma_prefetch_2d(&mapA, (kb2 * KSUB + q) * BK, glu_rows + nt2 * BM);
+            }
+          }
+          if (++kb2 >= kb12) {
+            u2 += gridDim.x;
+            if (u2 < um.units) um.decode(u2, nt2, mt2, s2, kb2, kb12);
+          }
+        }
       }
       if constexpr (!PREP) {
         pdl_wait();

@@ -30,6 +30,10 @@ struct PfCtl {
   int first = 0;  // a segment at or before the one holding lo
   unsigned long long lo = 0, hi = 0;
   int early = 0;
+  // decode tiles: before waiting for the previous kernel, the producer asks
+  // L2 for up to `own` more of this CTA's own weight tiles past those its
+  // shared-memory ring takes (0: none)
+  int own = 0;
 };
 
 // Operand stage of a decode GEMM (M <= 16 rows).  Instead of loading X by

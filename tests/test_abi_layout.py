@@ -26,6 +26,7 @@ CONSTANTS = {
     "DORY_OPT_ATTN_CLUSTER": dory.OPT_ATTN_CLUSTER, "DORY_OPT_L2_LOOKAHEAD": dory.OPT_L2_LOOKAHEAD,
     "DORY_OPT_MX_GEMV": dory.OPT_MX_GEMV, "DORY_OPT_FUSED_OPERANDS": dory.OPT_FUSED_OPERANDS,
     "DORY_OPT_ATTN_LOOKAHEAD": dory.OPT_ATTN_LOOKAHEAD,
+    "DORY_OPT_L2_OWN": dory.OPT_L2_OWN,
 }
 
 
