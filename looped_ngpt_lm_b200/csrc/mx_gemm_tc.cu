@@ -529,21 +529,28 @@ cudaError_t run_lowbit(int M, int N, int K, const bf16* X, int ldx, const uint8_
 
 }  // namespace
 
-int mx_gemm_splits(int N, int K) {
-  const int tiles = N / BM, nch = K / Fmt<0>::CK;
+// Split count S in 1..min(8, chunks) with the shortest launch: units
+// (tiles x S) run in ceil(units / SMs) rounds of 1/S of a tile's chunks each;
+// ties go to the smaller S (fewer partial slices to add).  A count just above
+// the SMs doubles the launch (160 units on 148 SMs: two rounds of one tile).
+int lowbit_splits(int tiles, int nch) {
   if (tiles <= 0 || nch <= 0) return 1;
-  int S = (num_sms_tc() + tiles - 1) / tiles;
-  S = S > 8 ? 8 : S;
-  return S > nch ? nch : (S < 1 ? 1 : S);
+  const int sms = num_sms_tc();
+  int best = 1;
+  double best_t = 1e30;
+  for (int S = 1; S <= 8 && S <= nch; ++S) {
+    const double t = (double)((tiles * S + sms - 1) / sms) / S;
+    if (t < best_t - 1e-9) {
+      best_t = t;
+      best = S;
+    }
+  }
+  return best;
 }
 
-int nv_gemm_splits(int N, int K) {
-  const int tiles = N / BM, nch = K / Fmt<1>::CK;
-  if (tiles <= 0 || nch <= 0) return 1;
-  int S = (num_sms_tc() + tiles - 1) / tiles;
-  S = S > 8 ? 8 : S;
-  return S > nch ? nch : (S < 1 ? 1 : S);
-}
+int mx_gemm_splits(int N, int K) { return lowbit_splits(N / BM, K / Fmt<0>::CK); }
+
+int nv_gemm_splits(int N, int K) { return lowbit_splits(N / BM, K / Fmt<1>::CK); }
 
 cudaError_t launch_mx_gemm_tc(int M, int N, int K, const bf16* X, int ldx, const uint8_t* q, const uint8_t* scales,
                               float* Y, int ldy, size_t part_stride, int S, int* err, cudaStream_t st) {
