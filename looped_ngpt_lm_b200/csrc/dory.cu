@@ -498,8 +498,13 @@ dory_status gemm(const Fwd<T>& f, int M, int N, int K, const T* X, int ldx, cons
           }
           if (e != cudaErrorNotSupported) return fail(DORY_ERR_CUDA, "%s: %s", name, cudaGetErrorString(e));
         }
-        CK(launch_mx_gemv(M, N, K, (const bf16*)X, ldx, it->second.q, it->second.s, Y, ldy, H->err, f.st,
-                          H->mx_impl == 3 ? 1 : H->mx_impl));
+        const int impl = H->mx_impl == 3 ? 1 : H->mx_impl;
+        const int S = impl == 2 ? 1 : mx_gemv_splits(N, K);
+        const size_t ps = part_rows * (size_t)ldy;
+        CK(launch_mx_gemv(M, N, K, (const bf16*)X, ldx, it->second.q, it->second.s, Y, ldy, H->err, f.st, impl, S,
+                          ps));
+        *S_out = S;
+        *ps_out = ps;
         return DORY_OK;
       }
     }

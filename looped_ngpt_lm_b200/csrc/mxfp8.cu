@@ -128,21 +128,29 @@ __device__ __forceinline__ float block_scale(uint32_t sb) {
   return __uint_as_float((e < 255u ? e : 255u) << 23);  // +inf past the supported range
 }
 
+// Split-K: blockIdx.y = split s takes weights [s Ks, (s + 1) Ks) of every
+// row and writes its partial dot products to Y + s * part_stride.
 template <int MT>
 __global__ void __launch_bounds__(GV_T) k_mx_gemv(int M, int N, int K, const bf16* __restrict__ X, int ldx,
                                                   const uint8_t* __restrict__ q, const uint8_t* __restrict__ s,
-                                                  float* __restrict__ Y, int ldy, int* err) {
+                                                  float* __restrict__ Y, int ldy, int* err, int Ks,
+                                                  size_t part_stride) {
   extern __shared__ float4 xs[];  // [MT][4][nch]: float4 i of chunk c of token m at (m*4 + i)*nch + c
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nch = K >> 4, nsb = K >> 5, K4 = K >> 2;
+  const int k0 = blockIdx.y * Ks;
+  const int nch = Ks >> 4, nsb = K >> 5, K4 = Ks >> 2;
   const int gw = blockIdx.x * GV_W + warp, nw = gridDim.x * GV_W;
+  q += k0;
+  s += k0 >> 5;
+  X += k0;
+  Y += blockIdx.y * part_stride;
 
   // The weights do not depend on earlier kernels: ask L2 for this warp's
   // first row while the previous kernel finishes.
   if (gw < N) {
     const char* row = reinterpret_cast<const char*>(q) + (size_t)gw * K;
-    for (int a = lane * 128; a < K; a += 32 * 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(row + a));
-    if (lane * 128 < nsb) asm volatile("prefetch.global.L2 [%0];" ::"l"(s + (size_t)gw * nsb + lane * 128));
+    for (int a = lane * 128; a < Ks; a += 32 * 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(row + a));
+    if (lane * 128 < (Ks >> 5)) asm volatile("prefetch.global.L2 [%0];" ::"l"(s + (size_t)gw * nsb + lane * 128));
   }
   pdl_wait();
 
@@ -227,8 +235,9 @@ __global__ void __launch_bounds__(GV_T) k_mx_gemv(int M, int N, int K, const bf1
 
 template <int MT>
 cudaError_t run_gemv(int M, int N, int K, const bf16* X, int ldx, const uint8_t* q, const uint8_t* s, float* Y,
-                     int ldy, int* err, cudaStream_t st) {
-  const int smem = MT * K * 4;
+                     int ldy, int* err, cudaStream_t st, int S, size_t part_stride) {
+  const int Ks = K / S;
+  const int smem = MT * Ks * 4;
   static int attr_smem = 0;
   static std::map<int, int> per_sm;  // dynamic shared memory -> resident CTAs per SM
   if (smem > attr_smem) {
@@ -244,9 +253,11 @@ cudaError_t run_gemv(int M, int N, int K, const bf16* X, int ldx, const uint8_t*
     it = per_sm.emplace(smem, b < 1 ? 1 : b).first;
   }
   const long long want = ((long long)N + GV_W - 1) / GV_W;
-  const long long cap = (long long)num_sms() * it->second;
+  long long cap = (long long)num_sms() * it->second / S;
+  if (cap < 1) cap = 1;
   const int grid = (int)(want < cap ? want : cap);
-  return launch(k_mx_gemv<MT>, grid, GV_T, smem, st, M, N, K, X, ldx, q, s, Y, ldy, err);
+  return launch(k_mx_gemv<MT>, dim3(grid, S), dim3(GV_T), smem, st, M, N, K, X, ldx, q, s, Y, ldy, err, Ks,
+                part_stride);
 }
 
 // ------------------------------------------------------------------ GEMV on the tensor cores
@@ -442,9 +453,16 @@ cudaError_t launch_mx_quantize(const bf16* W, int N, int K, uint8_t* q, uint8_t*
   return cudaGetLastError();
 }
 
+int mx_gemv_splits(int N, int K) {
+  int S = 1;
+  while (S < 8 && (long long)N * S < 48LL * num_sms() && K % (2 * S * kMxBlock) == 0 && K / (2 * S) >= 512) S *= 2;
+  return S;
+}
+
 cudaError_t launch_mx_gemv(int M, int N, int K, const bf16* X, int ldx, const uint8_t* q, const uint8_t* s,
-                           float* Y, int ldy, int* err, cudaStream_t st, int impl) {
+                           float* Y, int ldy, int* err, cudaStream_t st, int impl, int S, size_t part_stride) {
   if (M <= 0 || N <= 0 || K <= 0 || K % kMxBlock || ((uintptr_t)q & 15)) return cudaErrorNotSupported;
+  if (S < 1 || K % (S * kMxBlock) || (S > 1 && impl != 0 && impl != 1)) return cudaErrorNotSupported;
   if (impl == 3) return launch_mx_gemm_tc(M, N, K, X, ldx, q, s, Y, ldy, 0, 1, err, st);
   // the mma.sync kernel only by request: measured slower at every 4B decode shape
   if (impl == 2) {
@@ -453,15 +471,15 @@ cudaError_t launch_mx_gemv(int M, int N, int K, const bf16* X, int ldx, const ui
   }
   // tokens per pass: the smallest power of two covering M, up to 8, within
   // the staged-activation budget
-  int cap = GV_SMEM_CAP / (K * 4);
+  int cap = GV_SMEM_CAP / ((K / S) * 4);
   if (cap < 1) return cudaErrorNotSupported;
   int MT = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8;
   while (MT > cap) MT >>= 1;
   switch (MT) {
-    case 1: return run_gemv<1>(M, N, K, X, ldx, q, s, Y, ldy, err, st);
-    case 2: return run_gemv<2>(M, N, K, X, ldx, q, s, Y, ldy, err, st);
-    case 4: return run_gemv<4>(M, N, K, X, ldx, q, s, Y, ldy, err, st);
-    default: return run_gemv<8>(M, N, K, X, ldx, q, s, Y, ldy, err, st);
+    case 1: return run_gemv<1>(M, N, K, X, ldx, q, s, Y, ldy, err, st, S, part_stride);
+    case 2: return run_gemv<2>(M, N, K, X, ldx, q, s, Y, ldy, err, st, S, part_stride);
+    case 4: return run_gemv<4>(M, N, K, X, ldx, q, s, Y, ldy, err, st, S, part_stride);
+    default: return run_gemv<8>(M, N, K, X, ldx, q, s, Y, ldy, err, st, S, part_stride);
   }
 }
 

@@ -32,8 +32,16 @@ cudaError_t launch_mx_quantize(const bf16* W, int N, int K, uint8_t* q, uint8_t*
 // impl 3: the TMA-fed tensor-core GEMM below, unsplit (N % 128 == 0,
 //   K % 128 == 0, X 16-byte aligned with ldx % 8 == 0, |X| < 4).
 // impl 0: 1 (the faster of 1 and 2 at every 4B decode shape).
+// S > 1 (impl 0 / 1 only, K % (32 S) == 0): split K into S equal ranges;
+// split s writes its partial products to Y + s * part_stride and the
+// consumer adds them in order s = 0..S-1.
 cudaError_t launch_mx_gemv(int M, int N, int K, const bf16* X, int ldx, const uint8_t* q, const uint8_t* s,
-                           float* Y, int ldy, int* err, cudaStream_t st, int impl = 0);
+                           float* Y, int ldy, int* err, cudaStream_t st, int impl = 0, int S = 1,
+                           size_t part_stride = 0);
+// Splits for the CUDA-core GEMV inside a decode step: doubled while the rows
+// fill fewer than 48 warps per SM, at most 8, each split at least 512
+// weights.  Depends on (N, K) only.
+int mx_gemv_splits(int N, int K);
 
 // Low-bit decode GEMMs on the tensor cores, fed by TMA (mx_gemm_tc.cu): S
 // partial products at Y + s * part_stride (row stride ldy) that the consumer
