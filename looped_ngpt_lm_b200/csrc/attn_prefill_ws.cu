@@ -512,25 +512,23 @@ __global__ void __launch_bounds__(NTH, 1)
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       bf16* dst = out + (size_t)(s.r0 + row) * qd + s.head * HDT;
-#pragma unroll 1
-      for (int c = 0; c < HDT; c += 32) {
-        uint32_t o[32];
-        tmem_ld32(lane_addr + o_col + c, o);
-        tmem_wait_ld();
-        if (row < s.nrows) {
+      uint32_t o[HDT];  // the whole row of O with one wait
 #pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            uint4 u;
-            u.x = pack2(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
-            u.y = pack2(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
-            u.z = pack2(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
-            u.w = pack2(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
-            *reinterpret_cast<uint4*>(dst + c + e) = u;
-          }
+      for (int c = 0; c < HDT; c += 32) tmem_ld32(lane_addr + o_col + c, o + c);
+      tmem_wait_ld();
+      if (row < s.nrows) {
+#pragma unroll
+        for (int e = 0; e < HDT; e += 8) {
+          uint4 u;
+          u.x = pack2(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
+          u.y = pack2(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+          u.z = pack2(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
+          u.w = pack2(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
+          *reinterpret_cast<uint4*>(dst + e) = u;
         }
       }
     }
-  }
+   }
   }
   tc_fence_before();
   __syncthreads();
