@@ -1068,7 +1068,9 @@ def mx_gemv_probe(args):
         torch.cuda.empty_cache()
     print(json.dumps({"kernel": "nv_gemm" if nv else "mx_gemv", "mx_impl": None if nv else args.mx_impl,
                       "m": args.m, "results": out,
-                      "note": "graph-replayed back-to-back launches, weights cold in L2"}))
+                      "note": "graph-replayed back-to-back launches, weights cold in L2; one K split (S = 1), "
+                              "which a decode step does not use for the QKV, O and down shapes (it splits K: "
+                              "see the mxfp8_decode / nvfp4_decode legs for the in-step kernels)"}))
 
 
 def run_reference(args, shape, workload):
