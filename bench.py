@@ -384,7 +384,8 @@ def lowbit_leg(dory, torch, shape, dw, args, mode, bf16_sweep, fmt, steps=32):
     bench's bf16 weights, at k = 1, 2, 4 on a handle of its own: prefill reads
     the exact bf16 dequantisation, decode GEMMs the copies.  fmt "mxfp8":
     E4M3 codes with one E8M0 scale per 32 weights, timed with the CUDA-core
-    GEMV (option 1) and the TMA-fed tcgen05 GEMM (option 3); fmt "nvfp4":
+    GEMV (option 1), the same GEMV fed by bulk copies (option 4) and the
+    TMA-fed tcgen05 GEMM (option 3); fmt "nvfp4":
     E2M1 codes, one E4M3 scale per 16 weights and a tensor scale, on the
     tcgen05 GEMM.  Reports tokens/s, the speed-up over the bf16 k sweep at
     the same context, and the low-bit GEMMs' HBM rate from a profiled pass."""
@@ -399,7 +400,8 @@ def lowbit_leg(dory, torch, shape, dw, args, mode, bf16_sweep, fmt, steps=32):
     tok = h.prefill([0], prompt, [args.prompt], args.k, mode)
     bufs = [torch.empty(1, dtype=torch.int32, device="cuda") for _ in range(2)]
     out = {}
-    impls = ((1, "cuda_core_gemv"), (3, "tcgen05_gemm")) if fmt == "mxfp8" else ((0, "tcgen05_gemm"),)
+    impls = (((1, "cuda_core_gemv"), (4, "cuda_core_gemv_bulk_fed"), (3, "tcgen05_gemm")) if fmt == "mxfp8"
+             else ((0, "tcgen05_gemm"),))
     hbm = peaks()[0]
     for impl, label in impls:
         if fmt == "mxfp8":

@@ -330,6 +330,9 @@ dory_status dory_quantize_mxfp8(const void* w, int32_t N, int32_t K, void* q, vo
  *     columns and takes its scale in the epilogue.  Requires N % 128 == 0,
  *     K % 128 == 0, x 16-byte aligned, ldx % 8 == 0 (else
  *     DORY_ERR_UNSUPPORTED); |x| < 4.
+ *   impl 4: impl 1's arithmetic (the same bits) with the weight rows
+ *     streamed into shared memory by bulk copies; shapes it does not take
+ *     (N % 16, more than 48 KB of weights per 16 rows, M > 8) run as 1.
  *   impl 0: 1 (measured faster than 2 at every 4B decode shape).
  * An activation outside the range (non-finite for 2) sets *err_word (device,
  * nullable).  Queues work on `stream`. */
@@ -460,7 +463,8 @@ enum {
    * computed. */
   DORY_OPT_L2_LOOKAHEAD = 7,
   /* GEMM on attached MXFP8 copies (see dory_gemv_mxfp8's impl): 0 (default, = 1), 1 CUDA cores,
-     2 mma.sync, 3 TMA-fed tcgen05 with split-K slices (matrices whose N or K it does not take use 1) */
+     2 mma.sync, 3 TMA-fed tcgen05 with split-K slices (matrices whose N or K it does not take use 1),
+     4 CUDA cores fed by bulk copies (the same bits as 1; shapes it does not take use 1) */
   DORY_OPT_MX_GEMV = 8,
   /* bf16 decode and speculative steps of at most this many rows (default 0:
    * off; at most 16): the add + L2 norm after a layer and the SwiGLU of a

@@ -1557,7 +1557,7 @@ dory_status dory_set_option(dory_handle* h, int32_t opt, int64_t value) {
       h->pf_lead = (unsigned long long)value & ~127ull;
       return DORY_OK;
     case DORY_OPT_MX_GEMV:
-      if (value < 0 || value > 3) return fail(DORY_ERR_INVALID_ARG, "bad MXFP8 GEMV impl");
+      if (value < 0 || value > 4) return fail(DORY_ERR_INVALID_ARG, "bad MXFP8 GEMV impl");
       if (value != h->mx_impl) {
         for (auto& g : h->graphs_cache)
           if (g.exec) cudaGraphExecDestroy(g.exec);
@@ -1614,7 +1614,7 @@ dory_status dory_quantize_mxfp8(const void* w, int32_t n, int32_t k, void* q, vo
 dory_status dory_gemv_mxfp8(int32_t m, int32_t n, int32_t k, const void* x, int32_t ldx, const void* q,
                             const void* scales, float* y, int32_t ldy, int32_t impl, int32_t* err_word,
                             dory_stream stream) {
-  if (!x || !q || !scales || !y || m < 1 || n < 1 || k < 1 || ldx < k || ldy < n || impl < 0 || impl > 3)
+  if (!x || !q || !scales || !y || m < 1 || n < 1 || k < 1 || ldx < k || ldy < n || impl < 0 || impl > 4)
     return fail(DORY_ERR_INVALID_ARG, "bad GEMV arguments");
   if (impl == 3 && (n % 128 || k % 128 || ((uintptr_t)x & 15) || ldx % 8))
     return fail(DORY_ERR_UNSUPPORTED, "impl 3 needs N %% 128 == 0, K %% 128 == 0, x 16-byte aligned, ldx %% 8 == 0");

@@ -20,6 +20,7 @@
 #include <map>
 
 #include "mxfp8.cuh"
+#include "umma.cuh"
 #include "warp_mma.cuh"
 
 namespace dory {
@@ -231,6 +232,187 @@ __global__ void __launch_bounds__(GV_T) k_mx_gemv(int M, int N, int K, const bf1
       }
     }
   }
+}
+
+// ------------------------------------------------------------------ GEMV fed by bulk copies
+// The same per-row arithmetic as k_mx_gemv (lane l takes the 16-weight
+// chunks l, l + 32, ... of its row, in that order), with the weight rows
+// streamed into shared memory by bulk copies instead of each warp's own
+// loads: one producer warp keeps a ring of RG_STAGES units of 16 rows in
+// flight (the weights do not depend on earlier kernels, so it starts before
+// the predecessor grid has finished), and eight consumer warps take two rows
+// each.  blockIdx.y is the K split, as in k_mx_gemv.  Every mbarrier wait is
+// bounded; on expiry the CTA sets the error word, stops, and the producer
+// waits (bounded) for its copies in flight.
+constexpr int RG_RPU = 16;               // weight rows per unit
+constexpr int RG_NC = 8;                 // consumer warps, two rows each
+constexpr int RG_T = (RG_NC + 1) * 32;   // + the producer warp
+constexpr int RG_MAX_STAGES = 4;
+constexpr int RG_STAGE_CAP = 48 * 1024;  // weight bytes of one unit (16 rows x the split's K range)
+constexpr int RG_SMEM_CAP = 227 * 1024;
+
+__device__ __forceinline__ void rg_bulk(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(tc::smem_u32(bar))
+               : "memory");
+}
+
+template <int MT>
+__global__ void __launch_bounds__(RG_T) k_mx_gemv_ring(int M, int N, int K, const bf16* __restrict__ X, int ldx,
+                                                       const uint8_t* __restrict__ q,
+                                                       const uint8_t* __restrict__ s, float* __restrict__ Y,
+                                                       int ldy, int* err, int Ks, size_t part_stride, int stages) {
+  using namespace tc;
+  extern __shared__ __align__(128) uint8_t rg_smem[];
+  const int unit_bytes = RG_RPU * Ks;
+  uint8_t* wbuf = rg_smem;                                              // [stages][16 rows][Ks]
+  float4* xs = reinterpret_cast<float4*>(rg_smem + stages * unit_bytes);  // [MT][4][nch]
+  uint64_t* full = reinterpret_cast<uint64_t*>(rg_smem + stages * unit_bytes + MT * Ks * 4);
+  uint64_t* empty = full + RG_MAX_STAGES;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + RG_MAX_STAGES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k0 = blockIdx.y * Ks;
+  const int nch = Ks >> 4, nsb = K >> 5, K4 = Ks >> 2;
+  const int n_units = N / RG_RPU;
+  q += k0;
+  s += k0 >> 5;
+  X += k0;
+  Y += blockIdx.y * part_stride;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < stages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], RG_NC);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  if (warp == RG_NC) {
+    // ---------------- producer: weights need nothing from earlier kernels
+    if (lane == 0) {
+      int i = 0;
+      for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++i) {
+        const int st = i % stages;
+        if (i >= stages && !mbar_wait(&empty[st], ((i / stages) + 1) & 1, abort_flag, err)) break;
+        const uint32_t dst = smem_u32(wbuf + (size_t)st * unit_bytes);
+        mbar_expect_tx(&full[st], (uint32_t)unit_bytes);
+        if (Ks == K) {
+          rg_bulk(dst, q + (size_t)u * RG_RPU * K, (uint32_t)unit_bytes, &full[st]);
+        } else {
+          for (int r = 0; r < RG_RPU; ++r)
+            rg_bulk(dst + r * Ks, q + ((size_t)u * RG_RPU + r) * K, (uint32_t)Ks, &full[st]);
+        }
+      }
+      // copies still in flight land before the CTA can exit
+      for (int j = i - stages < 0 ? 0 : i - stages; j < i; ++j) mbar_wait_drain(&full[j % stages], (j / stages) & 1);
+    }
+    return;
+  }
+
+  // ---------------- consumers
+  pdl_wait();
+  for (int m0 = 0; m0 < M; m0 += MT) {
+    const int mc = M - m0 < MT ? M - m0 : MT;
+    if (m0 > 0) asm volatile("bar.sync 1, %0;" ::"r"(RG_NC * 32) : "memory");  // done with the previous tokens
+    bool bad = false;
+    for (int e = threadIdx.x; e < MT * K4; e += RG_NC * 32) {
+      const int m = e / K4, r = e - m * K4;  // elements 4r..4r+3 of token m
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (m < mc) {
+        const bf16* xr = X + (size_t)(m0 + m) * ldx + 4 * r;
+        v.x = __bfloat162float(xr[0]) * 0x1p64f;
+        v.y = __bfloat162float(xr[1]) * 0x1p64f;
+        v.z = __bfloat162float(xr[2]) * 0x1p64f;
+        v.w = __bfloat162float(xr[3]) * 0x1p64f;
+        bad |= !(fabsf(v.x) <= FLT_MAX && fabsf(v.y) <= FLT_MAX && fabsf(v.z) <= FLT_MAX && fabsf(v.w) <= FLT_MAX);
+      }
+      xs[((m << 2) + (r & 3)) * nch + (r >> 2)] = v;
+    }
+    if (bad) set_error(err, DEV_ERR_RANGE);
+    asm volatile("bar.sync 1, %0;" ::"r"(RG_NC * 32) : "memory");
+    if (m0 == 0 && threadIdx.x == 0) pdl_trigger();
+
+    int i = 0;
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++i) {
+      const int st = i % stages;
+      // launches have M <= MT: one token pass, each unit streamed once
+      if (!mbar_wait(&full[st], (i / stages) & 1, abort_flag, err)) break;
+#pragma unroll 1
+      for (int rr = 0; rr < 2; ++rr) {
+        const int rl = warp * 2 + rr, n = u * RG_RPU + rl;
+        const uint4* qrow = reinterpret_cast<const uint4*>(wbuf + (size_t)st * unit_bytes + (size_t)rl * Ks);
+        const uint8_t* srow = s + (size_t)n * nsb;
+        float acc[MT];
+#pragma unroll
+        for (int m = 0; m < MT; ++m) acc[m] = 0.f;
+        for (int c = lane; c < nch; c += 32) {
+          const uint4 w = qrow[c];
+          const uint32_t sb = __ldg(srow + (c >> 1));
+          float f[16];
+          const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            f[4 * j] = e4m3_scaled(wd[j] << 24);
+            f[4 * j + 1] = e4m3_scaled(wd[j] << 16);
+            f[4 * j + 2] = e4m3_scaled(wd[j] << 8);
+            f[4 * j + 3] = e4m3_scaled(wd[j]);
+          }
+          const float sc = block_scale(sb);
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            const float4* xp = xs + (m << 2) * nch + c;
+            float p[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float4 a = xp[j * nch];
+              float t = __fmul_rn(f[4 * j], a.x);
+              t = __fmaf_rn(f[4 * j + 1], a.y, t);
+              t = __fmaf_rn(f[4 * j + 2], a.z, t);
+              p[j] = __fmaf_rn(f[4 * j + 3], a.w, t);
+            }
+            acc[m] = __fmaf_rn(__fadd_rn(__fadd_rn(p[0], p[1]), __fadd_rn(p[2], p[3])), sc, acc[m]);
+          }
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          const float v = warp_sum(acc[m]);
+          if (lane == 0 && m < mc) Y[(size_t)(m0 + m) * ldy + n] = v;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+    }
+  }
+}
+
+// Launches k_mx_gemv_ring when its shapes fit (16-row units whose split of K
+// is at most RG_STAGE_CAP bytes, at least two stages in shared memory, one
+// token pass); cudaErrorNotSupported otherwise.
+template <int MT>
+cudaError_t run_gemv_ring(int M, int N, int K, const bf16* X, int ldx, const uint8_t* q, const uint8_t* s, float* Y,
+                          int ldy, int* err, cudaStream_t st, int S, size_t part_stride) {
+  const int Ks = K / S;
+  if (N % RG_RPU || M > MT || Ks % 16 || ((uintptr_t)q & 15) || RG_RPU * Ks > RG_STAGE_CAP)
+    return cudaErrorNotSupported;
+  const int fixed = MT * Ks * 4 + 2 * RG_MAX_STAGES * 8 + 16;
+  int stages = (RG_SMEM_CAP - fixed) / (RG_RPU * Ks);
+  if (stages > RG_MAX_STAGES) stages = RG_MAX_STAGES;
+  if (stages < 2) return cudaErrorNotSupported;
+  const int smem = stages * RG_RPU * Ks + fixed;
+  static int attr_smem = 0;
+  if (smem > attr_smem) {
+    cudaError_t e = cudaFuncSetAttribute(k_mx_gemv_ring<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, RG_SMEM_CAP);
+    if (e != cudaSuccess) return e;
+    attr_smem = RG_SMEM_CAP;
+  }
+  const int units = N / RG_RPU;
+  int gx = num_sms() / S;
+  if (gx < 1) gx = 1;
+  if (gx > units) gx = units;
+  return launch(k_mx_gemv_ring<MT>, dim3(gx, S), dim3(RG_T), smem, st, M, N, K, X, ldx, q, s, Y, ldy, err, Ks,
+                part_stride, stages);
 }
 
 template <int MT>
@@ -462,7 +644,7 @@ int mx_gemv_splits(int N, int K) {
 cudaError_t launch_mx_gemv(int M, int N, int K, const bf16* X, int ldx, const uint8_t* q, const uint8_t* s,
                            float* Y, int ldy, int* err, cudaStream_t st, int impl, int S, size_t part_stride) {
   if (M <= 0 || N <= 0 || K <= 0 || K % kMxBlock || ((uintptr_t)q & 15)) return cudaErrorNotSupported;
-  if (S < 1 || K % (S * kMxBlock) || (S > 1 && impl != 0 && impl != 1)) return cudaErrorNotSupported;
+  if (S < 1 || K % (S * kMxBlock) || (S > 1 && impl != 0 && impl != 1 && impl != 4)) return cudaErrorNotSupported;
   if (impl == 3) return launch_mx_gemm_tc(M, N, K, X, ldx, q, s, Y, ldy, 0, 1, err, st);
   // the mma.sync kernel only by request: measured slower at every 4B decode shape
   if (impl == 2) {
@@ -475,6 +657,17 @@ cudaError_t launch_mx_gemv(int M, int N, int K, const bf16* X, int ldx, const ui
   if (cap < 1) return cudaErrorNotSupported;
   int MT = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8;
   while (MT > cap) MT >>= 1;
+  if (impl == 4 && M <= MT) {
+    // the same arithmetic with the rows streamed by bulk copies, where it fits
+    cudaError_t e = cudaErrorNotSupported;
+    switch (MT) {
+      case 1: e = run_gemv_ring<1>(M, N, K, X, ldx, q, s, Y, ldy, err, st, S, part_stride); break;
+      case 2: e = run_gemv_ring<2>(M, N, K, X, ldx, q, s, Y, ldy, err, st, S, part_stride); break;
+      case 4: e = run_gemv_ring<4>(M, N, K, X, ldx, q, s, Y, ldy, err, st, S, part_stride); break;
+      default: e = run_gemv_ring<8>(M, N, K, X, ldx, q, s, Y, ldy, err, st, S, part_stride); break;
+    }
+    if (e != cudaErrorNotSupported) return e;
+  }
   switch (MT) {
     case 1: return run_gemv<1>(M, N, K, X, ldx, q, s, Y, ldy, err, st, S, part_stride);
     case 2: return run_gemv<2>(M, N, K, X, ldx, q, s, Y, ldy, err, st, S, part_stride);

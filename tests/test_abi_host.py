@@ -132,7 +132,7 @@ def test_mxfp8_argument_validation():
     assert G(1, 8, 48, F, 48, F, F, F, 8) == "DORY_ERR_UNSUPPORTED"    # K % 32
     assert G(1, 8, 40992, F, 40992, F, F, F, 8) == "DORY_ERR_UNSUPPORTED"  # staged activations too large
     assert G(1, 8, 10272, F, 10272, F, F, F, 8, impl=2) == "DORY_ERR_UNSUPPORTED"  # tensor cores: K <= 10240
-    assert G(1, 8, 64, F, 64, F, F, F, 8, impl=4) == "DORY_ERR_INVALID_ARG"
+    assert G(1, 8, 64, F, 64, F, F, F, 8, impl=5) == "DORY_ERR_INVALID_ARG"
     assert G(1, 100, 128, F, 128, F, F, F, 100, impl=3) == "DORY_ERR_UNSUPPORTED"   # N % 128
     assert G(1, 128, 96, F, 96, F, F, F, 128, impl=3) == "DORY_ERR_UNSUPPORTED"    # K % 128
     assert G(1, 128, 128, F8, 128, F, F, F, 128, impl=3) == "DORY_ERR_UNSUPPORTED"  # x not 16-byte aligned
@@ -159,7 +159,8 @@ def test_mxfp8_argument_validation():
     assert A(hb, dory.MxWeightsC(None, None, None, None, None, None, None, None, None, None)) == "DORY_OK"
     assert A(hb, None) == "DORY_OK"
     assert lib.dory_set_option(hb, dory.OPT_MX_GEMV, 3) == 0
-    assert lib.dory_set_option(hb, dory.OPT_MX_GEMV, 4) == 1
+    assert lib.dory_set_option(hb, dory.OPT_MX_GEMV, 4) == 0
+    assert lib.dory_set_option(hb, dory.OPT_MX_GEMV, 5) == 1
     # NVFP4
     NQ = lambda *a: status_name(lib.dory_quantize_nvfp4(*a, None, None))
     assert NQ(F, 4, 40, F, F, F, None) == "DORY_ERR_UNSUPPORTED"       # K % 16

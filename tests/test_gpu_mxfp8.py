@@ -95,7 +95,7 @@ GEMV_CASES = [(1, 37, 256), (2, 1000, 1056), (3, 384, 2560), (5, 2560, 2560), (1
               (13, 300, 10240), (8, 4096, 2560)]
 
 
-@pytest.mark.parametrize("impl", [1, 2])
+@pytest.mark.parametrize("impl", [1, 2, 4])
 @pytest.mark.parametrize("M,N,K", GEMV_CASES)
 def test_gemv_matches_oracle(M, N, K, impl):
     rng = np.random.default_rng(M * 7 + N + K)
@@ -118,6 +118,19 @@ def test_gemv_matches_oracle(M, N, K, impl):
     for m in sorted({0, M // 2, M - 1}):
         one = dory.gemv_mxfp8(X[m:m + 1].contiguous(), q, s, impl=impl)
         assert torch.equal(one[0], y[m])
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 3584, 2560), (3, 512, 2048), (8, 4096, 2560), (2, 272, 640)])
+def test_gemv_bulk_fed_same_bits_as_cuda_cores(M, N, K):
+    """impl 4 streams the rows by bulk copies but keeps impl 1's arithmetic:
+    the same bits."""
+    rng = np.random.default_rng(M + N + K)
+    w = rng.standard_normal((N, K)).astype(np.float32)
+    w /= np.linalg.norm(w, axis=1, keepdims=True)
+    xb = synth.f32_to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32) / np.sqrt(K))
+    q, s, _ = dory.quantize_mxfp8(bf16_cuda(synth.f32_to_bf16_bits(w)), dequantised=False)
+    X = bf16_cuda(xb)
+    assert torch.equal(dory.gemv_mxfp8(X, q, s, impl=4), dory.gemv_mxfp8(X, q, s, impl=1))
 
 
 @pytest.mark.parametrize("impl", [1, 2])
@@ -174,7 +187,7 @@ def mx_model(request):
     return shape, O.Model(shape, MX.quantized_weights(w)), h, mx
 
 
-@pytest.mark.parametrize("impl", [2, 1])
+@pytest.mark.parametrize("impl", [2, 1, 4])
 @pytest.mark.parametrize("k", [1, 2, 4])
 @pytest.mark.parametrize("mode", ["last_loop", "per_loop"])
 def test_decode_with_mxfp8_matches_oracle(mx_model, k, mode, impl):
@@ -206,7 +219,7 @@ def test_decode_reads_the_mxfp8_copies(mx_model):
     assert per_launch < 1.2 * n * kk  # 1 + 1/32 bytes per weight, not bf16's 2
 
 
-@pytest.mark.parametrize("impl", [2, 1])
+@pytest.mark.parametrize("impl", [2, 1, 4])
 def test_graph_replay_and_speculative_decoding_with_mxfp8(mx_model, impl):
     shape, _, h, _ = mx_model
     h.set_option(dory.OPT_MX_GEMV, impl)
