@@ -392,8 +392,10 @@ def lowbit_leg(dory, torch, shape, dw, args, mode, bf16_sweep, fmt, steps=32):
     import synth
     ev = lambda: torch.cuda.Event(enable_timing=True)
     wq = dory.MxWeights(dw) if fmt == "mxfp8" else dory.NvWeights(dw)
-    cfg = dory.make_config(shape, max_batch=1, max_seq=args.prompt + 8 * steps + 64, k_max=4, gamma_max=4,
-                           max_chunk=args.prompt)
+    n_impl = 3 if fmt == "mxfp8" else 1
+    # every implementation decodes (3 warm-up + steps) tokens at each k, then 2 profiled steps
+    cfg = dory.make_config(shape, max_batch=1, max_seq=args.prompt + n_impl * (3 * (steps + 3) + 2) + 64, k_max=4,
+                           gamma_max=4, max_chunk=args.prompt)
     h = dory.Handle(cfg, wq.dequantised, dory.LAST_LOOP if args.mode == "last_loop" else dory.PER_LOOP)
     (h.attach_mxfp8 if fmt == "mxfp8" else h.attach_nvfp4)(wq)
     prompt = torch.tensor(synth.make_prompt(1, args.prompt, shape.vocab), dtype=torch.int32, device="cuda")
