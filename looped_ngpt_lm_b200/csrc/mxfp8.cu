@@ -238,18 +238,18 @@ __global__ void __launch_bounds__(GV_T) k_mx_gemv(int M, int N, int K, const bf1
 // The same per-row arithmetic as k_mx_gemv (lane l takes the 16-weight
 // chunks l, l + 32, ... of its row, in that order), with the weight rows
 // streamed into shared memory by bulk copies instead of each warp's own
-// loads: one producer warp keeps a ring of RG_STAGES units of 16 rows in
+// loads: one producer warp keeps a ring of RG_MAX_STAGES units of 8 rows in
 // flight (the weights do not depend on earlier kernels, so it starts before
-// the predecessor grid has finished), and eight consumer warps take two rows
-// each.  blockIdx.y is the K split, as in k_mx_gemv.  Every mbarrier wait is
+// the predecessor grid has finished), and eight consumer warps take one row
+// each; three CTAs share an SM.  blockIdx.y is the K split, as in k_mx_gemv.  Every mbarrier wait is
 // bounded; on expiry the CTA sets the error word, stops, and the producer
 // waits (bounded) for its copies in flight.
-constexpr int RG_RPU = 16;               // weight rows per unit
-constexpr int RG_NC = 8;                 // consumer warps, two rows each
+constexpr int RG_RPU = 8;                // weight rows per unit
+constexpr int RG_NC = 8;                 // consumer warps, one row each
 constexpr int RG_T = (RG_NC + 1) * 32;   // + the producer warp
-constexpr int RG_MAX_STAGES = 4;
-constexpr int RG_STAGE_CAP = 48 * 1024;  // weight bytes of one unit (16 rows x the split's K range)
-constexpr int RG_SMEM_CAP = 227 * 1024;
+constexpr int RG_MAX_STAGES = 3;
+constexpr int RG_STAGE_CAP = 24 * 1024;  // weight bytes of one unit (8 rows x the split's K range)
+constexpr int RG_SMEM_CAP = 75 * 1024;   // three CTAs per SM
 
 __device__ __forceinline__ void rg_bulk(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(RG_T) k_mx_gemv_ring(int M, int N, int K, cons
   using namespace tc;
   extern __shared__ __align__(128) uint8_t rg_smem[];
   const int unit_bytes = RG_RPU * Ks;
-  uint8_t* wbuf = rg_smem;                                              // [stages][16 rows][Ks]
+  uint8_t* wbuf = rg_smem;                                              // [stages][8 rows][Ks]
   float4* xs = reinterpret_cast<float4*>(rg_smem + stages * unit_bytes);  // [MT][4][nch]
   uint64_t* full = reinterpret_cast<uint64_t*>(rg_smem + stages * unit_bytes + MT * Ks * 4);
   uint64_t* empty = full + RG_MAX_STAGES;
@@ -339,9 +339,8 @@ __global__ void __launch_bounds__(RG_T) k_mx_gemv_ring(int M, int N, int K, cons
       const int st = i % stages;
       // launches have M <= MT: one token pass, each unit streamed once
       if (!mbar_wait(&full[st], (i / stages) & 1, abort_flag, err)) break;
-#pragma unroll 1
-      for (int rr = 0; rr < 2; ++rr) {
-        const int rl = warp * 2 + rr, n = u * RG_RPU + rl;
+      {
+        const int rl = warp, n = u * RG_RPU + rl;
         const uint4* qrow = reinterpret_cast<const uint4*>(wbuf + (size_t)st * unit_bytes + (size_t)rl * Ks);
         const uint8_t* srow = s + (size_t)n * nsb;
         float acc[MT];
@@ -387,7 +386,7 @@ __global__ void __launch_bounds__(RG_T) k_mx_gemv_ring(int M, int N, int K, cons
   }
 }
 
-// Launches k_mx_gemv_ring when its shapes fit (16-row units whose split of K
+// Launches k_mx_gemv_ring when its shapes fit (8-row units whose split of K
 // is at most RG_STAGE_CAP bytes, at least two stages in shared memory, one
 // token pass); cudaErrorNotSupported otherwise.
 template <int MT>
@@ -408,7 +407,7 @@ cudaError_t run_gemv_ring(int M, int N, int K, const bf16* X, int ldx, const uin
     attr_smem = RG_SMEM_CAP;
   }
   const int units = N / RG_RPU;
-  int gx = num_sms() / S;
+  int gx = 3 * num_sms() / S;
   if (gx < 1) gx = 1;
   if (gx > units) gx = units;
   return launch(k_mx_gemv_ring<MT>, dim3(gx, S), dim3(RG_T), smem, st, M, N, K, X, ldx, q, s, Y, ldy, err, Ks,
