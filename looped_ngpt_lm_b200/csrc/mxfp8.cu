@@ -249,6 +249,7 @@ constexpr int RG_NC = 8;                 // consumer warps, one row each
 constexpr int RG_T = (RG_NC + 1) * 32;   // + the producer warp
 constexpr int RG_MAX_STAGES = 3;
 constexpr int RG_STAGE_CAP = 24 * 1024;  // weight bytes of one unit (8 rows x the split's K range)
+constexpr int RG_MAXC = RG_STAGE_CAP / RG_RPU / 16 / 32;  // 16-weight chunks of a row per lane: 6
 constexpr int RG_SMEM_CAP = 75 * 1024;   // three CTAs per SM
 
 __device__ __forceinline__ void rg_bulk(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -337,18 +338,28 @@ __global__ void __launch_bounds__(RG_T) k_mx_gemv_ring(int M, int N, int K, cons
     int i = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++i) {
       const int st = i % stages;
+      const int rl = warp, n = u * RG_RPU + rl;
+      // this lane's scale bytes, requested before the weights are waited for
+      const uint8_t* srow = s + (size_t)n * nsb;
+      uint32_t sbv[RG_MAXC];
+#pragma unroll
+      for (int t = 0; t < RG_MAXC; ++t) {
+        const int c = lane + 32 * t;
+        sbv[t] = c < nch ? __ldg(srow + (c >> 1)) : 0u;
+      }
       // launches have M <= MT: one token pass, each unit streamed once
       if (!mbar_wait(&full[st], (i / stages) & 1, abort_flag, err)) break;
       {
-        const int rl = warp, n = u * RG_RPU + rl;
         const uint4* qrow = reinterpret_cast<const uint4*>(wbuf + (size_t)st * unit_bytes + (size_t)rl * Ks);
-        const uint8_t* srow = s + (size_t)n * nsb;
         float acc[MT];
 #pragma unroll
         for (int m = 0; m < MT; ++m) acc[m] = 0.f;
-        for (int c = lane; c < nch; c += 32) {
+#pragma unroll
+        for (int t = 0; t < RG_MAXC; ++t) {
+          const int c = lane + 32 * t;
+          if (c >= nch) break;
           const uint4 w = qrow[c];
-          const uint32_t sb = __ldg(srow + (c >> 1));
+          const uint32_t sb = sbv[t];
           float f[16];
           const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
