@@ -334,7 +334,8 @@ dory_status dory_quantize_mxfp8(const void* w, int32_t N, int32_t K, void* q, vo
  *     streamed into shared memory by bulk copies; shapes it does not take
  *     (N % 8, more than 24 KB of weights per 8 rows, too many rows M for
  *     the staged activations) run as 1.
- *   impl 0: 1 (measured faster than 2 at every 4B decode shape).
+ *   impl 0: 4 where it takes the shape, else 1 (the same bits; measured
+ *     faster than 1 and 2 in a 4B decode step).
  * An activation outside the range (non-finite for 2) sets *err_word (device,
  * nullable).  Queues work on `stream`. */
 dory_status dory_gemv_mxfp8(int32_t M, int32_t N, int32_t K, const void* x, int32_t ldx, const void* q,
@@ -463,7 +464,7 @@ enum {
    * look-ahead off).  Changes only when HBM reads happen, never what is
    * computed. */
   DORY_OPT_L2_LOOKAHEAD = 7,
-  /* GEMM on attached MXFP8 copies (see dory_gemv_mxfp8's impl): 0 (default, = 1), 1 CUDA cores,
+  /* GEMM on attached MXFP8 copies (see dory_gemv_mxfp8's impl): 0 (default: 4 where it fits, else 1), 1 CUDA cores,
      2 mma.sync, 3 TMA-fed tcgen05 with split-K slices (matrices whose N or K it does not take use 1),
      4 CUDA cores fed by bulk copies (the same bits as 1; shapes it does not take use 1) */
   DORY_OPT_MX_GEMV = 8,

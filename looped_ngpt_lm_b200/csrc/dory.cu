@@ -113,7 +113,8 @@ struct dory_handle {
     int fmt = 0;               // 0 MXFP8, 1 NVFP4
   };
   std::unordered_map<const void*, MxMat> mx;
-  int mx_impl = 0;  // GEMV on the copies: 0 default (CUDA cores), 1 CUDA cores, 2 tensor cores
+  int mx_impl = 0;  // GEMV on the copies: 0 default (4 where it fits, else 1), 1 CUDA cores, 2 tensor cores,
+                    // 3 tcgen05 GEMM, 4 CUDA cores fed by bulk copies
   std::vector<int> attn_of;
   std::vector<AttnLayer> attn;
 

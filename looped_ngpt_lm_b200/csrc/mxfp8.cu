@@ -667,7 +667,7 @@ cudaError_t launch_mx_gemv(int M, int N, int K, const bf16* X, int ldx, const ui
   if (cap < 1) return cudaErrorNotSupported;
   int MT = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8;
   while (MT > cap) MT >>= 1;
-  if (impl == 4 && M <= MT) {
+  if ((impl == 4 || impl == 0) && M <= MT) {
     // the same arithmetic with the rows streamed by bulk copies, where it fits
     cudaError_t e = cudaErrorNotSupported;
     switch (MT) {

@@ -35,7 +35,8 @@ cudaError_t launch_mx_quantize(const bf16* W, int N, int K, uint8_t* q, uint8_t*
 //   into shared memory by bulk copies (8-row units, N % 8 == 0, at most
 //   24 KB of weights per unit, the staged activations and two units within
 //   75 KB); other shapes take impl 1.
-// impl 0: 1 (the faster of 1 and 2 at every 4B decode shape).
+// impl 0: 4 where it takes the shape, else 1 (the same bits either way;
+//   measured faster than 1 and 2 in a 4B decode step).
 // S > 1 (impl 0 / 1 only, K % (32 S) == 0): split K into S equal ranges;
 // split s writes its partial products to Y + s * part_stride and the
 // consumer adds them in order s = 0..S-1.
