@@ -332,8 +332,8 @@ dory_status dory_quantize_mxfp8(const void* w, int32_t N, int32_t K, void* q, vo
  *     DORY_ERR_UNSUPPORTED); |x| < 4.
  *   impl 4: impl 1's arithmetic (the same bits) with the weight rows
  *     streamed into shared memory by bulk copies; shapes it does not take
- *     (N % 16, more than 48 KB of weights per 16 rows, too many rows M
- *     for the staged activations) run as 1.
+ *     (N % 8, more than 24 KB of weights per 8 rows, too many rows M for
+ *     the staged activations) run as 1.
  *   impl 0: 4 where it takes the shape, else 1 (the same bits; measured
  *     faster than 1 and 2 in a 4B decode step).
  * An activation outside the range (non-finite for 2) sets *err_word (device,

@@ -238,19 +238,19 @@ __global__ void __launch_bounds__(GV_T) k_mx_gemv(int M, int N, int K, const bf1
 // The same per-row arithmetic as k_mx_gemv (lane l takes the 16-weight
 // chunks l, l + 32, ... of its row, in that order), with the weight rows
 // streamed into shared memory by bulk copies instead of each warp's own
-// loads: one producer warp keeps a ring of RG_MAX_STAGES units of 16 rows in
+// loads: one producer warp keeps a ring of RG_MAX_STAGES units of 8 rows in
 // flight (the weights do not depend on earlier kernels, so it starts before
-// the predecessor grid has finished), and eight consumer warps take two rows
-// each, reading each activation chunk once for both; two CTAs share an SM.  blockIdx.y is the K split, as in k_mx_gemv.  Every mbarrier wait is
+// the predecessor grid has finished), and eight consumer warps take one row
+// each; three CTAs share an SM.  blockIdx.y is the K split, as in k_mx_gemv.  Every mbarrier wait is
 // bounded; on expiry the CTA sets the error word, stops, and the producer
 // waits (bounded) for its copies in flight.
-constexpr int RG_RPU = 16;               // weight rows per unit
-constexpr int RG_NC = 8;                 // consumer warps, two rows each
+constexpr int RG_RPU = 8;                // weight rows per unit
+constexpr int RG_NC = 8;                 // consumer warps, one row each
 constexpr int RG_T = (RG_NC + 1) * 32;   // + the producer warp
-constexpr int RG_MAX_STAGES = 2;
-constexpr int RG_STAGE_CAP = 48 * 1024;  // weight bytes of one unit (16 rows x the split's K range)
+constexpr int RG_MAX_STAGES = 3;
+constexpr int RG_STAGE_CAP = 24 * 1024;  // weight bytes of one unit (8 rows x the split's K range)
 constexpr int RG_MAXC = RG_STAGE_CAP / RG_RPU / 16 / 32;  // 16-weight chunks of a row per lane: 6
-constexpr int RG_SMEM_CAP = 110 * 1024;  // two CTAs per SM
+constexpr int RG_SMEM_CAP = 75 * 1024;   // three CTAs per SM
 
 __device__ __forceinline__ void rg_bulk(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(RG_T) k_mx_gemv_ring(int M, int N, int K, cons
   using namespace tc;
   extern __shared__ __align__(128) uint8_t rg_smem[];
   const int unit_bytes = RG_RPU * Ks;
-  uint8_t* wbuf = rg_smem;                                              // [stages][16 rows][Ks]
+  uint8_t* wbuf = rg_smem;                                              // [stages][8 rows][Ks]
   float4* xs = reinterpret_cast<float4*>(rg_smem + stages * unit_bytes);  // [MT][4][nch]
   uint64_t* full = reinterpret_cast<uint64_t*>(rg_smem + stages * unit_bytes + MT * Ks * 4);
   uint64_t* empty = full + RG_MAX_STAGES;
@@ -338,70 +338,57 @@ __global__ void __launch_bounds__(RG_T) k_mx_gemv_ring(int M, int N, int K, cons
     int i = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++i) {
       const int st = i % stages;
-      const int rl = warp * 2, n = u * RG_RPU + rl;
-      // this lane's scale bytes of both rows, requested before the weights are waited for
-      const uint8_t* srow0 = s + (size_t)n * nsb;
-      const uint8_t* srow1 = srow0 + nsb;
-      uint32_t sbv0[RG_MAXC], sbv1[RG_MAXC];
+      const int rl = warp, n = u * RG_RPU + rl;
+      // this lane's scale bytes, requested before the weights are waited for
+      const uint8_t* srow = s + (size_t)n * nsb;
+      uint32_t sbv[RG_MAXC];
 #pragma unroll
       for (int t = 0; t < RG_MAXC; ++t) {
         const int c = lane + 32 * t;
-        sbv0[t] = c < nch ? __ldg(srow0 + (c >> 1)) : 0u;
-        sbv1[t] = c < nch ? __ldg(srow1 + (c >> 1)) : 0u;
+        sbv[t] = c < nch ? __ldg(srow + (c >> 1)) : 0u;
       }
       // launches have M <= MT: one token pass, each unit streamed once
       if (!mbar_wait(&full[st], (i / stages) & 1, abort_flag, err)) break;
       {
-        const uint4* qrow0 = reinterpret_cast<const uint4*>(wbuf + (size_t)st * unit_bytes + (size_t)rl * Ks);
-        const uint4* qrow1 = qrow0 + (Ks >> 4);
-        float acc0[MT], acc1[MT];
+        const uint4* qrow = reinterpret_cast<const uint4*>(wbuf + (size_t)st * unit_bytes + (size_t)rl * Ks);
+        float acc[MT];
 #pragma unroll
-        for (int m = 0; m < MT; ++m) acc0[m] = acc1[m] = 0.f;
+        for (int m = 0; m < MT; ++m) acc[m] = 0.f;
 #pragma unroll
         for (int t = 0; t < RG_MAXC; ++t) {
           const int c = lane + 32 * t;
           if (c >= nch) break;
-          const uint4 wa = qrow0[c], wb = qrow1[c];
-          float f0[16], f1[16];
-          const uint32_t wd0[4] = {wa.x, wa.y, wa.z, wa.w}, wd1[4] = {wb.x, wb.y, wb.z, wb.w};
+          const uint4 w = qrow[c];
+          const uint32_t sb = sbv[t];
+          float f[16];
+          const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            f0[4 * j] = e4m3_scaled(wd0[j] << 24);
-            f0[4 * j + 1] = e4m3_scaled(wd0[j] << 16);
-            f0[4 * j + 2] = e4m3_scaled(wd0[j] << 8);
-            f0[4 * j + 3] = e4m3_scaled(wd0[j]);
-            f1[4 * j] = e4m3_scaled(wd1[j] << 24);
-            f1[4 * j + 1] = e4m3_scaled(wd1[j] << 16);
-            f1[4 * j + 2] = e4m3_scaled(wd1[j] << 8);
-            f1[4 * j + 3] = e4m3_scaled(wd1[j]);
+            f[4 * j] = e4m3_scaled(wd[j] << 24);
+            f[4 * j + 1] = e4m3_scaled(wd[j] << 16);
+            f[4 * j + 2] = e4m3_scaled(wd[j] << 8);
+            f[4 * j + 3] = e4m3_scaled(wd[j]);
           }
-          const float sc0 = block_scale(sbv0[t]), sc1 = block_scale(sbv1[t]);
+          const float sc = block_scale(sb);
 #pragma unroll
           for (int m = 0; m < MT; ++m) {
             const float4* xp = xs + (m << 2) * nch + c;
-            float p0[4], p1[4];
+            float p[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const float4 a = xp[j * nch];
-              float t0 = __fmul_rn(f0[4 * j], a.x), t1 = __fmul_rn(f1[4 * j], a.x);
-              t0 = __fmaf_rn(f0[4 * j + 1], a.y, t0);
-              t1 = __fmaf_rn(f1[4 * j + 1], a.y, t1);
-              t0 = __fmaf_rn(f0[4 * j + 2], a.z, t0);
-              t1 = __fmaf_rn(f1[4 * j + 2], a.z, t1);
-              p0[j] = __fmaf_rn(f0[4 * j + 3], a.w, t0);
-              p1[j] = __fmaf_rn(f1[4 * j + 3], a.w, t1);
+              float t = __fmul_rn(f[4 * j], a.x);
+              t = __fmaf_rn(f[4 * j + 1], a.y, t);
+              t = __fmaf_rn(f[4 * j + 2], a.z, t);
+              p[j] = __fmaf_rn(f[4 * j + 3], a.w, t);
             }
-            acc0[m] = __fmaf_rn(__fadd_rn(__fadd_rn(p0[0], p0[1]), __fadd_rn(p0[2], p0[3])), sc0, acc0[m]);
-            acc1[m] = __fmaf_rn(__fadd_rn(__fadd_rn(p1[0], p1[1]), __fadd_rn(p1[2], p1[3])), sc1, acc1[m]);
+            acc[m] = __fmaf_rn(__fadd_rn(__fadd_rn(p[0], p[1]), __fadd_rn(p[2], p[3])), sc, acc[m]);
           }
         }
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
-          const float v0 = warp_sum(acc0[m]), v1 = warp_sum(acc1[m]);
-          if (lane == 0 && m < mc) {
-            Y[(size_t)(m0 + m) * ldy + n] = v0;
-            Y[(size_t)(m0 + m) * ldy + n + 1] = v1;
-          }
+          const float v = warp_sum(acc[m]);
+          if (lane == 0 && m < mc) Y[(size_t)(m0 + m) * ldy + n] = v;
         }
       }
       __syncwarp();
@@ -410,7 +397,7 @@ __global__ void __launch_bounds__(RG_T) k_mx_gemv_ring(int M, int N, int K, cons
   }
 }
 
-// Launches k_mx_gemv_ring when its shapes fit (16-row units whose split of K
+// Launches k_mx_gemv_ring when its shapes fit (8-row units whose split of K
 // is at most RG_STAGE_CAP bytes, at least two stages in shared memory, one
 // token pass); cudaErrorNotSupported otherwise.
 template <int MT>
@@ -431,7 +418,7 @@ cudaError_t run_gemv_ring(int M, int N, int K, const bf16* X, int ldx, const uin
     attr_smem = RG_SMEM_CAP;
   }
   const int units = N / RG_RPU;
-  int gx = 2 * num_sms() / S;
+  int gx = 3 * num_sms() / S;
   if (gx < 1) gx = 1;
   if (gx > units) gx = units;
   return launch(k_mx_gemv_ring<MT>, dim3(gx, S), dim3(RG_T), smem, st, M, N, K, X, ldx, q, s, Y, ldy, err, Ks,

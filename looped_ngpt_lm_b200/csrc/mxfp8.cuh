@@ -32,9 +32,9 @@ cudaError_t launch_mx_quantize(const bf16* W, int N, int K, uint8_t* q, uint8_t*
 // impl 3: the TMA-fed tensor-core GEMM below, unsplit (N % 128 == 0,
 //   K % 128 == 0, X 16-byte aligned with ldx % 8 == 0, |X| < 4).
 // impl 4: impl 1's arithmetic (the same bits) with the weight rows streamed
-//   into shared memory by bulk copies (16-row units, N % 16 == 0, at most
-//   48 KB of weights per unit, the staged activations and two units within
-//   110 KB); other shapes take impl 1.
+//   into shared memory by bulk copies (8-row units, N % 8 == 0, at most
+//   24 KB of weights per unit, the staged activations and two units within
+//   75 KB); other shapes take impl 1.
 // impl 0: 4 where it takes the shape, else 1 (the same bits either way;
 //   measured faster than 1 and 2 in a 4B decode step).
 // S > 1 (impl 0 / 1 only, K % (32 S) == 0): split K into S equal ranges;
