@@ -602,7 +602,8 @@ dory_status run_layers(const Fwd<T>& f, int l0, int l1, int loop, float* copy_la
   size_t ps_pend = 0;
   auto flush = [&](float* copy) -> dory_status {
     Scope sc(H, f.st, "addnorm", 0);
-    CK(launch_addnorm<T>(M, d, H->hcur(), H->hcur(), H->part_y, S_pend, ps_pend, d, H->hop_t<T>(), copy, f.st));
+    CK(launch_addnorm<T>(M, d, H->hcur(), H->hcur(), H->part_y, S_pend, ps_pend, d, H->hop_t<T>(), copy, f.st,
+                         !f.invariant));
     pend = false;
     return DORY_OK;
   };

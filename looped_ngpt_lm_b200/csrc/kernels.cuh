@@ -66,10 +66,14 @@ cudaError_t launch_embed(int M, int d, int vocab, const int* tokens, const T* E,
                          int* err, cudaStream_t st);
 // h_out <- N(h_in + sum_{s<S} y[s]) ; hop <- (T)h_out ; copy_out (if not NULL)
 // <- h_out (h_out may equal h_in).  y[s] = y + s*part_stride, rows of ldy.
-// S <= kMaxSplitK; d, ldy and part_stride multiples of 4.
+// S <= kMaxSplitK; d, ldy and part_stride multiples of 4.  Rows take the
+// 512-virtual-thread arithmetic of addnorm.cuh (the bits a decode row and
+// the same row of a speculative chunk share) unless any_order: then long
+// batches of rows (prefill chunks) may use a faster summation order.
 template <typename T>
 cudaError_t launch_addnorm(int M, int d, const float* h_in, float* h_out, const float* y, int S,
-                           size_t part_stride, int ldy, T* hop, float* copy_out, cudaStream_t st);
+                           size_t part_stride, int ldy, T* hop, float* copy_out, cudaStream_t st,
+                           bool any_order = false);
 // Loop boundary.  s_src: 0 -> s = x ; 1 -> s = N(h) ; 2 -> s = s_in.
 // If make_u: out = N(s + x), else out = s.  h <- out, hop <- (T)out.
 // If s_save: s_save <- s.  stash rows: when stash_x/stash_s are given, row r

@@ -174,6 +174,69 @@ __global__ void __launch_bounds__(AN_VT) k_addnorm(int d, const float* h_in, flo
   }
 }
 
+// Long prefill chunks: one warp per row, 16-byte loads and stores.  The same
+// mathematics (v = h + sum_s y_s in slice order, h <- v / max(||v||, 1e-12))
+// in another summation order: prefill rows never have to match the bits of
+// decode rows (those take the 512-virtual-thread arithmetic above).
+constexpr int ANR_ROWS = 8;   // rows (warps) per block
+constexpr int ANR_V4 = 24;    // float4 per lane: d <= 3072
+
+template <typename T>
+__global__ void __launch_bounds__(ANR_ROWS * 32) k_addnorm_rows(int M, int d, const float* h_in, float* h_out,
+                                                               const float* __restrict__ y, int S, size_t ps,
+                                                               int ldy, T* hop, float* copy_out) {
+  pdl_trigger();  // see common.cuh
+  pdl_wait();
+  const int r = blockIdx.x * ANR_ROWS + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (r >= M) return;
+  const int d4 = d >> 2;
+  const float4* hr = reinterpret_cast<const float4*>(h_in + (size_t)r * d);
+  float4 v[ANR_V4];
+  float ss = 0.f;
+#pragma unroll
+  for (int c = 0; c < ANR_V4; ++c) {
+    const int i = lane + 32 * c;
+    v[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i < d4) {
+      float4 a = __ldcg(hr + i);
+      for (int sl = 0; sl < S; ++sl) {
+        const float4 b = __ldcg(reinterpret_cast<const float4*>(y + sl * ps + (size_t)r * ldy) + i);
+        a.x += b.x;
+        a.y += b.y;
+        a.z += b.z;
+        a.w += b.w;
+      }
+      v[c] = a;
+      ss = __fmaf_rn(a.x, a.x, ss);
+      ss = __fmaf_rn(a.y, a.y, ss);
+      ss = __fmaf_rn(a.z, a.z, ss);
+      ss = __fmaf_rn(a.w, a.w, ss);
+    }
+  }
+  ss = warp_sum(ss);
+  const float inv = 1.f / fmaxf(sqrtf(ss), 1e-12f);
+  float4* ho = reinterpret_cast<float4*>(h_out + (size_t)r * d);
+  float4* co = copy_out ? reinterpret_cast<float4*>(copy_out + (size_t)r * d) : nullptr;
+#pragma unroll
+  for (int c = 0; c < ANR_V4; ++c) {
+    const int i = lane + 32 * c;
+    if (i < d4) {
+      const float4 o = make_float4(v[c].x * inv, v[c].y * inv, v[c].z * inv, v[c].w * inv);
+      ho[i] = o;
+      if (co) co[i] = o;
+      if constexpr (sizeof(T) == 2) {
+        const __nv_bfloat162 a = __floats2bfloat162_rn(o.x, o.y), b = __floats2bfloat162_rn(o.z, o.w);
+        uint2 u;
+        u.x = *reinterpret_cast<const uint32_t*>(&a);
+        u.y = *reinterpret_cast<const uint32_t*>(&b);
+        reinterpret_cast<uint2*>(hop + (size_t)r * d)[i] = u;
+      } else {
+        reinterpret_cast<float4*>(hop + (size_t)r * d)[i] = o;
+      }
+    }
+  }
+}
+
 // The same arithmetic spread over a cluster of AN_CL blocks per row: block
 // rank q runs virtual threads 64q .. 64q + 63, so each SM reads an eighth
 // of the row's split-K slices (a lone block reading all of them competes on
@@ -219,8 +282,12 @@ __global__ void __cluster_dims__(AN_CL, 1, 1) __launch_bounds__(AN_CL_T)
 
 template <typename T>
 cudaError_t launch_addnorm(int M, int d, const float* h_in, float* h_out, const float* y, int S, size_t ps, int ldy,
-                           T* hop, float* copy_out, cudaStream_t st) {
+                           T* hop, float* copy_out, cudaStream_t st, bool any_order) {
   if (d > AN_CPT * AN_VT || S > AN_MAXS) return cudaErrorInvalidValue;
+  // prefill rows: a warp per row with 16-byte accesses
+  if (any_order && M > 64 && d % 4 == 0 && d <= 4 * 32 * ANR_V4 && ldy % 4 == 0 && ps % 4 == 0)
+    return launch(k_addnorm_rows<T>, dim3((M + ANR_ROWS - 1) / ANR_ROWS), dim3(ANR_ROWS * 32), 0, st, M, d, h_in,
+                  h_out, y, S, ps, ldy, hop, copy_out);
   // decode-sized batches: a cluster per row; long chunks: one block per row
   if (M <= 64) return launch(k_addnorm_cl<T>, dim3(M * AN_CL), dim3(AN_CL_T), 0, st, d, h_in, h_out, y, S, ps, ldy,
                              hop, copy_out);
@@ -820,7 +887,7 @@ cudaError_t launch_spec_accept(int B, int gamma, int dstride, const int* seq_ids
   template cudaError_t launch_embed<T>(int, int, int, const int*, const T*, float*, T*, float*, int*,            \
                                        cudaStream_t);                                                             \
   template cudaError_t launch_addnorm<T>(int, int, const float*, float*, const float*, int, size_t, int, T*,      \
-                                         float*, cudaStream_t);                                                   \
+                                         float*, cudaStream_t, bool);                                             \
   template cudaError_t launch_reinject<T>(int, int, float*, const float*, int, const float*, bool, T*, float*,    \
                                           int, int, int, cudaStream_t);                                           \
   template cudaError_t launch_qkv_post<T>(int, int, int, int, const float*, int, size_t, float*, T*, T*, bool,    \
