@@ -191,27 +191,36 @@ __global__ void __launch_bounds__(ANR_ROWS * 32) k_addnorm_rows(int M, int d, co
   if (r >= M) return;
   const int d4 = d >> 2;
   const float4* hr = reinterpret_cast<const float4*>(h_in + (size_t)r * d);
+  // every load of a slice is issued before any is used
   float4 v[ANR_V4];
-  float ss = 0.f;
 #pragma unroll
   for (int c = 0; c < ANR_V4; ++c) {
     const int i = lane + 32 * c;
-    v[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (i < d4) {
-      float4 a = __ldcg(hr + i);
-      for (int sl = 0; sl < S; ++sl) {
-        const float4 b = __ldcg(reinterpret_cast<const float4*>(y + sl * ps + (size_t)r * ldy) + i);
-        a.x += b.x;
-        a.y += b.y;
-        a.z += b.z;
-        a.w += b.w;
-      }
-      v[c] = a;
-      ss = __fmaf_rn(a.x, a.x, ss);
-      ss = __fmaf_rn(a.y, a.y, ss);
-      ss = __fmaf_rn(a.z, a.z, ss);
-      ss = __fmaf_rn(a.w, a.w, ss);
+    v[c] = i < d4 ? __ldcg(hr + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int sl = 0; sl < S; ++sl) {
+    const float4* yr = reinterpret_cast<const float4*>(y + sl * ps + (size_t)r * ldy);
+    float4 b[ANR_V4];
+#pragma unroll
+    for (int c = 0; c < ANR_V4; ++c) {
+      const int i = lane + 32 * c;
+      b[c] = i < d4 ? __ldcg(yr + i) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
+#pragma unroll
+    for (int c = 0; c < ANR_V4; ++c) {
+      v[c].x += b[c].x;
+      v[c].y += b[c].y;
+      v[c].z += b[c].z;
+      v[c].w += b[c].w;
+    }
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int c = 0; c < ANR_V4; ++c) {
+    ss = __fmaf_rn(v[c].x, v[c].x, ss);
+    ss = __fmaf_rn(v[c].y, v[c].y, ss);
+    ss = __fmaf_rn(v[c].z, v[c].z, ss);
+    ss = __fmaf_rn(v[c].w, v[c].w, ss);
   }
   ss = warp_sum(ss);
   const float inv = 1.f / fmaxf(sqrtf(ss), 1e-12f);
