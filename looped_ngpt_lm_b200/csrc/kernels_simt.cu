@@ -404,26 +404,41 @@ __global__ void k_qkv_post(int H, int KV, int hd, const float* qkv, int S, size_
     if (threadIdx.x == 0) set_error(kv.err, DEV_ERR_BAD_INDEX);
     return;
   }
-  for (int i = threadIdx.x; i < ld; i += blockDim.x) {
-    float a = 0.f;
-    for (int s = 0; s < S; ++s) a += src[s * ps + i];
+  // four consecutive elements per thread (hd, and so every segment of the
+  // row, is a multiple of 4; the row and slice strides keep 16-byte alignment)
+  for (int i = 4 * threadIdx.x; i < ld; i += 4 * blockDim.x) {
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < S; ++s) {
+      const float4 b = *reinterpret_cast<const float4*>(src + s * ps + i);
+      a[0] += b.x;
+      a[1] += b.y;
+      a[2] += b.z;
+      a[3] += b.w;
+    }
     if (i < qd) {
-      if (qh)  // the tensor-core attention reads only the scaled bf16 copy
-        qh[(size_t)r * qd + i] = __float2bfloat16_rn(a * qscale);
-      else
-        q_out[(size_t)r * qd + i] = a;
+      if (qh) {  // the tensor-core attention reads only the scaled bf16 copy
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(a[0] * qscale, a[1] * qscale);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(a[2] * qscale, a[3] * qscale);
+        uint2 u;
+        u.x = *reinterpret_cast<const uint32_t*>(&lo);
+        u.y = *reinterpret_cast<const uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(qh + (size_t)r * qd + i) = u;
+      } else {
+        *reinterpret_cast<float4*>(q_out + (size_t)r * qd + i) = make_float4(a[0], a[1], a[2], a[3]);
+      }
     } else {
       int j = i - qd;
-      bool is_v = j >= kvd;
+      const bool is_v = j >= kvd;
       if (is_v) j -= kvd;
-      T val = from_f<T>(a);
+      T* dst;
       if (direct) {
-        int g = j / hd, e = j % hd;
-        size_t off = kv_row(kv, seq, KV, g, pos) * hd + e;
-        (is_v ? (T*)kv.V : (T*)kv.K)[off] = val;
+        const int g = j / hd, e = j % hd;
+        dst = (is_v ? (T*)kv.V : (T*)kv.K) + kv_row(kv, seq, KV, g, pos) * hd + e;
       } else {
-        (is_v ? vscr : kscr)[(size_t)r * kvd + j] = val;
+        dst = (is_v ? vscr : kscr) + (size_t)r * kvd + j;
       }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) dst[e] = from_f<T>(a[e]);
     }
   }
   (void)max_batch;
@@ -434,6 +449,7 @@ cudaError_t launch_qkv_post(int M, int H, int KV, int hd, const float* qkv, int 
                             T* kscr, T* vscr, bool direct, KVView kv, RowMeta m, int max_batch, bf16* qh,
                             cudaStream_t st) {
   const float qscale = 1.4426950408889634f / sqrtf((float)hd);
+  if (hd % 4 || ps % 4) return cudaErrorInvalidValue;
   launch(k_qkv_post<T>, M, 256, 0, st, H, KV, hd, qkv, S, ps, q_out, kscr, vscr, direct, kv, m, max_batch, qh,
          qscale);
   return cudaGetLastError();
