@@ -27,7 +27,7 @@
  *             last-loop KV caching keeps the footprint of one loop).
  *
  * Conventions for every entry point:
- *   - Return DORY_OK or an error status; dory_last_error() gives the message.
+ *   - Return DORY_OK or an error status; dory_last_error(h) gives the message.
  *   - Arguments are validated before any work is queued: an error leaves the
  *     handle and its caches unchanged.
  *   - Pointers marked "device" are CUDA device pointers, "host" are host
@@ -516,8 +516,10 @@ dory_status dory_profile_read(dory_handle* h, int32_t n, char (*names)[48], int6
                               double* total_ms, double* bytes, int32_t* count);
 dory_status dory_profile_reset(dory_handle* h);
 
-/* Message of the last failed call on this host thread ("" if none). */
-const char* dory_last_error(void);
+/* Message of the last failed call on this host thread ("" if none), valid
+ * until the next call on the thread.  h (nullable) is not read: the message
+ * is kept per thread, whichever handle the failing call used. */
+const char* dory_last_error(const dory_handle* h);
 
 #ifdef __cplusplus
 }

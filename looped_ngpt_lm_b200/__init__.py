@@ -124,7 +124,7 @@ def _load() -> ctypes.CDLL:
         f = getattr(lib, name)
         f.argtypes = args
         f.restype = ctypes.c_int
-    lib.dory_last_error.argtypes = []
+    lib.dory_last_error.argtypes = [ctypes.c_void_p]
     lib.dory_last_error.restype = ctypes.c_char_p
     return lib
 
@@ -134,7 +134,7 @@ lib = _load()
 
 def _check(status: int) -> None:
     if status != 0:
-        raise DoryError(status, lib.dory_last_error().decode())
+        raise DoryError(status, lib.dory_last_error(None).decode())
 
 
 def make_config(shape, max_batch=1, max_seq=256, k_max=4, gamma_max=4, max_chunk=None, kv_page=0,

@@ -1234,7 +1234,7 @@ dory_status spec_t(dory_handle* H, int B, const int32_t* seq_ids, const int32_t*
 // ====================================================================== C ABI
 extern "C" {
 
-const char* dory_last_error(void) { return g_last_error.c_str(); }
+const char* dory_last_error(const dory_handle*) { return g_last_error.c_str(); }
 
 dory_status dory_workspace_size(const dory_config* cfg, dory_cache_mode alloc_mode, size_t* bytes) {
   RET(check_config(cfg));

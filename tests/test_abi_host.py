@@ -46,7 +46,7 @@ def fake_handle(shape, alloc=dory.PER_LOOP, **kw):
     w = dory.Weights(FAKE_WS, FAKE_WS, fake, fake, fake, fake)
     h = ctypes.c_void_p()
     st = lib.dory_create(ctypes.byref(cfg), ctypes.byref(w), alloc, ctypes.c_void_p(FAKE_WS), n, ctypes.byref(h))
-    assert st == 0, lib.dory_last_error()
+    assert st == 0, lib.dory_last_error(None)
     return h, cfg, (cfg, w, fake)
 
 
@@ -122,7 +122,7 @@ def test_argument_validation():
     n = ctypes.c_int32()
     assert lib.dory_seq_len(h, 0, ctypes.byref(n)) == 0 and n.value == 0
     assert lib.dory_read_state(h, 0, ctypes.c_void_p(FAKE_WS), 1, None) == 1  # nothing computed yet
-    assert b"rows" in lib.dory_last_error()
+    assert b"rows" in lib.dory_last_error(None)
     lib.dory_destroy(h)
 
 
@@ -220,7 +220,7 @@ def test_bad_page_sizes_are_rejected(page):
     cfg = cfg_for(synth.TINY, kv_page=page)
     n = ctypes.c_size_t()
     assert lib.dory_workspace_size(ctypes.byref(cfg), dory.LAST_LOOP, ctypes.byref(n)) == 1
-    assert b"kv_page" in lib.dory_last_error()
+    assert b"kv_page" in lib.dory_last_error(None)
 
 
 def test_page_pool_exhaustion_is_a_capacity_error_before_any_work():
@@ -231,8 +231,8 @@ def test_page_pool_exhaustion_is_a_capacity_error_before_any_work():
     lens = (ctypes.c_int32 * 1)(48)
     st = lib.dory_prefill(h, 1, ids, ctypes.c_void_p(FAKE_WS), lens, 1, dory.LAST_LOOP, None,
                           ctypes.c_void_p(FAKE_WS), None)
-    assert st == 2, lib.dory_last_error()
-    assert b"pages" in lib.dory_last_error()
+    assert st == 2, lib.dory_last_error(None)
+    assert b"pages" in lib.dory_last_error(None)
     n = ctypes.c_int32()
     assert lib.dory_seq_len(h, 0, ctypes.byref(n)) == 0 and n.value == 0
     lib.dory_destroy(h)

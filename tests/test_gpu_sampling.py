@@ -31,7 +31,7 @@ def gpu_sample(logits, seq, pos, T, p, seed):
     out = torch.full((R,), -1, dtype=torch.int32, device="cuda")
     st = dory.lib.dory_sample(lg.data_ptr(), R, V, sq.data_ptr(), ps.data_ptr(), T, p, seed, scratch.data_ptr(),
                               out.data_ptr(), None)
-    assert st == 0, dory.lib.dory_last_error()
+    assert st == 0, dory.lib.dory_last_error(None)
     torch.cuda.synchronize()
     return out.cpu().numpy()
 

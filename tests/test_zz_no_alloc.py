@@ -44,10 +44,10 @@ def test_noalloc_matches_allocating_entry_point(M, N, K):
         X = torch.randn((M, K), generator=g, device="cuda").to(torch.bfloat16)
         ref, splits = dory.gemm_bf16(X, W, batch_hint=1, invariant=True, impl=2)
         Y = torch.full((M, N), float("nan"), device="cuda")
-        assert noalloc(X, W, Y) == 0, dory.lib.dory_last_error()
+        assert noalloc(X, W, Y) == 0, dory.lib.dory_last_error(None)
         torch.cuda.synchronize()
         assert torch.equal(Y, ref), (call, splits, (Y - ref).abs().max().item())
-    assert status() == 0, dory.lib.dory_last_error()
+    assert status() == 0, dory.lib.dory_last_error(None)
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
@@ -55,5 +55,5 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     W = torch.zeros((131072, 2560), dtype=torch.bfloat16, device="cuda")
     Y = torch.zeros((64, 131072), device="cuda")
     assert noalloc(X, W, Y) == 2  # DORY_ERR_CAPACITY, before any work is queued
-    assert b"2097152" in dory.lib.dory_last_error()
+    assert b"2097152" in dory.lib.dory_last_error(None)
     assert status() == 0
