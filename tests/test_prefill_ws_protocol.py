@@ -115,14 +115,14 @@ def simulate(n_tiles, ranges, paths, NS=2, seed=0, timeout_at=None, bug=None):
         issued, ok = 0, True
         for j in range(n_tiles):
             s, use = j % NS, j // NS
-            if j >= NS:
+            if j >= NS and bug != "loader_no_k_wait":
                 ok = yield ("wait", k_empty[s], (use + 1) & 1)
                 if not ok:
                     break
-                if bug != "loader_no_v_wait":
-                    ok = yield ("wait", v_empty[s], (use + 1) & 1)
-                    if not ok:
-                        break
+            if j >= NS and bug != "loader_no_v_wait":
+                ok = yield ("wait", v_empty[s], (use + 1) & 1)
+                if not ok:
+                    break
             if paths[j] == "tma":
                 k_full[s].arrive_expect_tx(2)
                 inflight.extend([("k", s, j, k_full[s])] * 2)
@@ -422,3 +422,14 @@ def test_p_columns_and_v_rows_meet_at_the_same_keys():
                     key_a = key
             v_row = (2048 * kk + 128 * e) // 128
             assert key_a == v_row == 16 * kk + e
+
+
+def test_k_empty_wait_is_implied_by_v_empty_wait():
+    """The V release of tile j is committed after the S product of every slot
+    that reads K of tile j, so a loader waiting only for V's stage to empty
+    would still never overwrite K in use."""
+    rng = random.Random(5)
+    for t in range(300):
+        n, ranges = random_item(rng)
+        simulate(n, ranges, paths_for(rng, n), NS=rng.choice([2, 3]), seed=t,
+                 timeout_at=rng.randint(1, 120) if t % 3 == 0 else None, bug="loader_no_k_wait")
