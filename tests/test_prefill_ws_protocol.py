@@ -11,9 +11,7 @@ The kernel's roles, each restated as a state machine:
 The asynchronous units are modelled too: the tensor core runs the MMA lane's
 products and commits in issue order at times of its own choosing, and each
 TMA copy lands (and completes its bytes on the stage's barrier) whenever it
-likes.  The mbarrier model: a phase completes when all its arrivals are in
-and its transaction bytes are all complete; try_wait.parity(p) succeeds when
-the completed-phase count's parity differs from p.
+likes (the barrier model is in protocol_model.py).
 
 Random schedules over random slot geometries must finish without deadlock,
 every read (of shared-memory stages, of S, P and O in tensor memory) must see
@@ -26,44 +24,10 @@ import random
 
 import pytest
 
+from protocol_model import Bar, Hazard, check, run_schedule
+
 TK = 128
 WARPS = 4  # softmax warps per slot; each arrives with its 32 lanes at once
-
-
-class Bar:
-    def __init__(self, count, name):
-        self.count, self.name = count, name
-        self.arrived, self.tx, self.phase = 0, 0, 0
-
-    def _complete(self):
-        if self.arrived == self.count and self.tx == 0:
-            self.arrived, self.phase = 0, self.phase + 1
-
-    def arrive(self):
-        self.arrived += 1
-        assert self.arrived <= self.count, f"{self.name}: arrivals past the count"
-        self._complete()
-
-    def arrive_expect_tx(self, nbytes):
-        self.tx += nbytes
-        self.arrive()
-
-    def complete_tx(self, nbytes):
-        self.tx -= nbytes
-        assert self.tx >= 0, f"{self.name}: bytes completed that were never expected"
-        self._complete()
-
-    def try_wait(self, parity):
-        return (self.phase & 1) != parity
-
-
-class Hazard(AssertionError):
-    pass
-
-
-def check(cond, msg):
-    if not cond:
-        raise Hazard(msg)
 
 
 def simulate(n_tiles, ranges, paths, NS=2, seed=0, timeout_at=None, bug=None):
@@ -257,48 +221,12 @@ def simulate(n_tiles, ranges, paths, NS=2, seed=0, timeout_at=None, bug=None):
         bar.complete_tx(1)
 
     # -------------------------------------------------------- scheduler
+    def async_actions():
+        acts = [tensor_core_step] if queue else []
+        return acts + [lambda i=i: land(i) for i in range(len(inflight))]
+
     roles = [loader(), mma()] + [softmax(q, w) for q in range(nslot) for w in range(WARPS)]
-    req = [("step",)] * len(roles)
-    sent = [None] * len(roles)
-    done = [False] * len(roles)
-    steps = 0
-    lazy = rng.random() < 0.5
-    while not all(done):
-        steps += 1
-        choices = []
-        blocked = []
-        for i, r in enumerate(req):
-            if done[i]:
-                continue
-            if r[0] == "step" or r[1].try_wait(r[2]):
-                choices.append(("role", i, True))
-            elif r[0] == "wait" and st["abort"]:
-                choices.append(("role", i, False))
-            elif r[0] == "wait":
-                blocked.append(i)
-        if timeout_at is not None and steps >= timeout_at and blocked and not st["abort"]:
-            i = rng.choice(blocked)
-            st["abort"] = True
-            choices = [("role", i, False)]
-        # in some runs the asynchronous units lag far behind the roles
-        if not choices or not lazy or rng.random() < 0.05:
-            if queue:
-                choices.append(("tc",))
-            choices += [("land", i) for i in range(len(inflight))]
-        if not choices:
-            raise RuntimeError(f"deadlock: {[r[:1] + (r[1].name,) if len(r) > 1 else r for r in req]}")
-        c = rng.choice(choices)
-        if c[0] == "tc":
-            tensor_core_step()
-        elif c[0] == "land":
-            land(c[1])
-        else:
-            i, res = c[1], c[2]
-            try:
-                req[i] = roles[i].send(res if req[i][0] == "wait" else None) if sent[i] else next(roles[i])
-                sent[i] = True
-            except StopIteration:
-                done[i] = True
+    run_schedule(roles, async_actions, rng, st, timeout_at)
     # the CTA frees TMEM and exits: nothing may still run
     check(not queue, f"products still queued at exit: {queue}")
     check(not inflight, f"copies still in flight at exit: {inflight}")
