@@ -564,7 +564,8 @@ def main():
                     help="time one kernel alone instead of the decode step (prints its own JSON line)")
     ap.add_argument("--shape", default="qkv,o,gate_up,down,lm_head", help="GEMM shapes for --kernel gemm / mxgemv")
     ap.add_argument("--mx-impl", dest="mx_impl", type=int, default=1,
-                    help="--kernel mxgemv: 1 CUDA cores (default), 2 mma.sync, 3 TMA-fed tcgen05 (one slice)")
+                    help="--kernel mxgemv: 1 CUDA cores (default), 2 mma.sync, 3 TMA-fed tcgen05 (one slice), "
+                         "4 CUDA cores fed by bulk copies")
     ap.add_argument("--m", type=int, default=1, help="token rows for --kernel gemm")
     ap.add_argument("--l2-lookahead-mb", dest="l2_mb", type=int, default=None,
                     help="bytes of upcoming weights each decode GEMM prefetches into L2 (MiB; 0 = off; "
