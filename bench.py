@@ -759,7 +759,7 @@ def main():
             ctx = h.seq_len(0)
             by = weight_bytes(shape, kk) + kv_read_bytes(shape, kk, ctx)
             sweep[f"k{kk}"] = {"tokens_per_s": round(1e3 / ms, 2), "ms_per_token": round(ms, 4),
-                               "hbm_frac_of_measured": round(by / (ms / 1e3) / 1e9 / hbm, 4),
+                               "hbm_frac_of_peak": round(by / (ms / 1e3) / 1e9 / hbm, 4),
                                "bytes_per_token": by, "ctx": ctx}
         aux["decode_k_sweep_last_loop" if args.mode == "last_loop" else "decode_k_sweep"] = sweep
         r = leg(sampling_leg, dory, torch, h, tok, args, mode)
@@ -826,12 +826,12 @@ def main():
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "inputs larger than L2: each step streams ~11 GB of weights"},
             "hbm": {"bytes_per_step": step_bytes, "achieved_GBs": round(step_bytes / (ms_step / 1e3) / 1e9, 1),
-                    "frac_of_measured": round(step_bytes / (ms_step / 1e3) / 1e9 / hbm, 4),
+                    "frac_of_peak": round(step_bytes / (ms_step / 1e3) / 1e9 / hbm, 4),
                     "frac_of_8TBs": round(step_bytes / (ms_step / 1e3) / 8e12, 4)},
             "prefill": {"tokens": args.prompt, "ms": round(pre_ms, 3),
                         "wall_tflops": round((pf + af) / (pre_ms / 1e3) / 1e12, 2),
                         "proj_tflops": round(pf / (proj_ms / 1e3) / 1e12, 2),
-                        "proj_frac_of_measured_bf16": round(pf / (proj_ms / 1e3) / 1e12 / tc, 4),
+                        "proj_frac_of_peak_bf16": round(pf / (proj_ms / 1e3) / 1e12 / tc, 4),
                         "attn_tflops": round(af / (attn_ms / 1e3) / 1e12, 2),
                         "proj_tflop": round(pf / 1e12, 3), "attn_tflop": round(af / 1e12, 3),
                         "note": "proj/attn TFLOP/s: algorithmic FLOPs over the event-timed GEMM / attention "
@@ -934,7 +934,7 @@ def batched_leg(args):
         "prefill": {"tokens": B * P, "s": round(pre_ms / 1e3, 3),
                     "wall_tflops": round(B * (pf1 + af1) / (pre_ms / 1e3) / 1e12, 2),
                     "proj_tflops": round(pf1 / (proj_ms / 1e3) / 1e12, 2),
-                    "proj_frac_of_measured_bf16": round(pf1 / (proj_ms / 1e3) / 1e12 / tc, 4),
+                    "proj_frac_of_peak_bf16": round(pf1 / (proj_ms / 1e3) / 1e12 / tc, 4),
                     "attn_tflops": round(af1 / (attn_ms / 1e3) / 1e12, 2),
                     "pflop": round(B * (pf1 + af1) / 1e15, 3),
                     "kernel_ms_one_sequence": {n_: round(v["ms"], 2) for n_, v in
@@ -943,7 +943,7 @@ def batched_leg(args):
                    "tokens_per_s": round(B * steps / (dec_ms / 1e3), 1),
                    "bytes_per_step": step_bytes,
                    "hbm_GBs": round(step_bytes / (ms_step / 1e3) / 1e9, 1),
-                   "hbm_frac_of_measured": round(step_bytes / (ms_step / 1e3) / 1e9 / hbm, 4)},
+                   "hbm_frac_of_peak": round(step_bytes / (ms_step / 1e3) / 1e9 / hbm, 4)},
         "peaks": {"hbm_GBs": hbm, "bf16_tflops": tc, "source": peak_src},
         "clocks": clk,
     }
@@ -993,9 +993,10 @@ def gemm_probe(args):
         us = 1e3 * a.elapsed_time(b) / iters
         by = wbytes + args.m * K * 2 + S * args.m * N * 4
         out[name] = {"N": N, "K": K, "splits": S, "us": round(us, 2), "GBs": round(by / us / 1e3, 1),
-                     "frac_of_measured": round(by / us / 1e3 / hbm, 4)}
+                     "frac_of_peak": round(by / us / 1e3 / hbm, 4)}
         del Ws
     print(json.dumps({"kernel": "gemm_tc", "impl": args.gemm_variant, "m": args.m, "results": out,
+                      "hbm_peak_GBs": hbm, "peak_source": peaks()[3],
                       "note": "graph-replayed back-to-back launches, weights cold in L2"}))
 
 
@@ -1068,11 +1069,11 @@ def mx_gemv_probe(args):
         us = 1e3 * a.elapsed_time(b) / iters
         by = wbytes + args.m * K * 2 + args.m * N * 4
         out[name] = {"N": N, "K": K, "us": round(us, 2), "GBs": round(by / us / 1e3, 1),
-                     "frac_of_measured": round(by / us / 1e3 / hbm, 4)}
+                     "frac_of_peak": round(by / us / 1e3 / hbm, 4)}
         del qs, ss, graph
         torch.cuda.empty_cache()
     print(json.dumps({"kernel": "nv_gemm" if nv else "mx_gemv", "mx_impl": None if nv else args.mx_impl,
-                      "m": args.m, "results": out,
+                      "m": args.m, "results": out, "hbm_peak_GBs": hbm, "peak_source": peaks()[3],
                       "note": "graph-replayed back-to-back launches, weights cold in L2; one K split (S = 1), "
                               "which a decode step does not use for the QKV, O and down shapes (it splits K: "
                               "see the mxfp8_decode / nvfp4_decode legs for the in-step kernels)"}))
