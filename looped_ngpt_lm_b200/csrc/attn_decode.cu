@@ -1,6 +1,15 @@
 // Fused GQA attention for decode and speculative chunks (K/V written straight
 // into the cache).
 //
+// What is computed: causal attention in sliding-window and full layers,
+// three of the first to one of the second (Dory1.0-4B digest,
+// onedev.kr/papers/1692, "How it works"); under last-loop caching (same
+// digest, "Premises & limits") a recurrent-block query of loop t sees the
+// loop-t keys of its own chunk and the final-loop keys cached by earlier
+// calls.  The pages give neither the window rule nor the head layout; this
+// library reads them as keys p - W < j <= p and as groups of query heads
+// sharing one K/V head (20 query heads over 4 K/V heads at the 4B shape).
+//
 // One 256-thread block per (row, KV head g, absolute key block of DEC_BK
 // positions):
 //   1. stage the block's cached keys and values in shared memory with cp.async

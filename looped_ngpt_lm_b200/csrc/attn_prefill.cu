@@ -1,6 +1,15 @@
 // Prefill attention on the tensor cores (bf16 mma.sync, fp32 accumulate),
 // flash-attention style, for chunks whose K/V sit in the chunk scratch.
 //
+// What is computed: causal attention in sliding-window and full layers,
+// three of the first to one of the second (Dory1.0-4B digest,
+// onedev.kr/papers/1692, "How it works"); under last-loop caching (same
+// digest, "Premises & limits") a recurrent-block query of loop t sees the
+// loop-t keys of its own chunk and the final-loop keys cached by earlier
+// calls.  The pages give neither the window rule nor the head layout; this
+// library reads them as keys p - W < j <= p and as groups of query heads
+// sharing one K/V head (20 query heads over 4 K/V heads at the 4B shape).
+//
 // One 128-thread block per (64-row query tile of one sequence, query head).
 // Each warp owns 16 query rows; Q fragments stay in registers.  Key tiles of
 // 64 absolute positions stream through a double-buffered shared-memory ring

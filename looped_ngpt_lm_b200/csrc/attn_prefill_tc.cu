@@ -1,6 +1,15 @@
 // Prefill attention on the 5th-generation tensor cores (bf16, head_dim 128):
 // S = Q K^T and O += P V as tcgen05 MMAs with fp32 accumulators in TMEM.
 //
+// What is computed: causal attention in sliding-window and full layers,
+// three of the first to one of the second (Dory1.0-4B digest,
+// onedev.kr/papers/1692, "How it works"); under last-loop caching (same
+// digest, "Premises & limits") a recurrent-block query of loop t sees the
+// loop-t keys of its own chunk and the final-loop keys cached by earlier
+// calls.  The pages give neither the window rule nor the head layout; this
+// library reads them as keys p - W < j <= p and as groups of query heads
+// sharing one K/V head (20 query heads over 4 K/V heads at the 4B shape).
+//
 // One CTA per (128 query rows of one sequence, query head); 6 warps.
 //   warps 0-3  one query row per thread (= TMEM lane): read S from TMEM,
 //              mask, online softmax in base 2 (Q is pre-scaled by

@@ -3,6 +3,15 @@
 // one key/value stream: two query heads of one KV group on the same rows, or
 // one head on two consecutive row tiles of the same sequence.
 //
+// What is computed: causal attention in sliding-window and full layers,
+// three of the first to one of the second (Dory1.0-4B digest,
+// onedev.kr/papers/1692, "How it works"); under last-loop caching (same
+// digest, "Premises & limits") a recurrent-block query of loop t sees the
+// loop-t keys of its own chunk and the final-loop keys cached by earlier
+// calls.  The pages give neither the window rule nor the head layout; this
+// library reads them as keys p - W < j <= p and as groups of query heads
+// sharing one K/V head (20 query heads over 4 K/V heads at the 4B shape).
+//
 //   warps 0-3  softmax of slot 0, one query row per thread (= TMEM lane)
 //   warps 4-7  softmax of slot 1
 //   warp 8     allocates TMEM; one lane issues every MMA and commit

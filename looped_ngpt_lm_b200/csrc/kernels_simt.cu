@@ -4,6 +4,12 @@
 // and a reference SIMT GEMM (fp32 storage, or bf16 before the tensor-core
 // path takes over).
 //
+// What is computed: the layer update h <- N(h + sublayer(h)) with N the L2
+// normalisation that keeps states on the unit sphere (review of "Dory1.0-4B:
+// A Looped Normalized-GPT", blog.secrett2633.cloud, "1. Key Terms"), and
+// the loop boundary u_t = N(s_{t-1} + x), s_0 = x, of the shared recurrent
+// block (Dory1.0-4B digest, onedev.kr/papers/1692, "How it works").
+//
 // Every reduction here runs in a fixed order that depends only on the row's
 // own data and absolute positions, never on how many rows share a launch, so
 // a row computes bit-identical results alone or inside a larger chunk.

@@ -1,4 +1,7 @@
-// Temperature / top-p sampling, one 1024-thread block per row.
+// Temperature / top-p sampling, one 1024-thread block per row.  The released
+// model's settings are temperature 1.0 and top-p 0.95 (lucasainews.com,
+// "NVIDIA, 루프 구조 4B 모델 Dory1.0-4B 4가지 정밀도로 공개", "How to run");
+// the pages give no procedure, and the one below is this library's reading.
 //
 // The draw for a row is Philox4x32 with 10 rounds (Salmon, Moraes, Dror and
 // Shaw, "Parallel random numbers: as easy as 1, 2, 3", SC 2011), key = the
