@@ -5,8 +5,9 @@
 // path takes over).
 //
 // What is computed: the layer update h <- N(h + sublayer(h)) with N the L2
-// normalisation that keeps states on the unit sphere (review of "Dory1.0-4B:
-// A Looped Normalized-GPT", blog.secrett2633.cloud, "1. Key Terms"), and
+// normalisation of the nGPT backbone (review of "Dory1.0-4B: A Looped
+// Normalized-GPT", blog.secrett2633.cloud, "1. Key Terms"; the update rule
+// itself is this library's reading), and
 // the loop boundary u_t = N(s_{t-1} + x), s_0 = x, of the shared recurrent
 // block (Dory1.0-4B digest, onedev.kr/papers/1692, "How it works").
 //
