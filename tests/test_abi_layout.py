@@ -125,3 +125,21 @@ def test_argtypes_match_the_prototypes():
         want = [c_class(p) for p in params]
         got = [py_class(t) for t in (f.argtypes or [])]
         assert got == want, (name, got, want)
+
+
+def test_readme_c_example_compiles_against_the_header(tmp_path):
+    """The C usage example in the README uses the header's names and
+    signatures as they are (compiled, not run)."""
+    import re
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    cuda_inc = "/usr/local/cuda/include"
+    if not cc or not os.path.exists(os.path.join(cuda_inc, "cuda_runtime.h")):
+        pytest.skip("no C compiler or CUDA headers")
+    text = open(os.path.join(ROOT, "README.md")).read()
+    blocks = re.findall(r"```c\n(.*?)```", text, re.S)
+    assert blocks, "README has no C example"
+    src = tmp_path / "example.c"
+    src.write_text(blocks[0])
+    subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-c", "-I", os.path.join(ROOT, "include"), "-I", cuda_inc,
+                    str(src), "-o", str(tmp_path / "example.o")], check=True)
