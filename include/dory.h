@@ -160,8 +160,10 @@ dory_status dory_destroy(dory_handle* h);
 dory_status dory_reset(dory_handle* h, int32_t seq, dory_stream stream);
 
 /* Prefill: append lens[i] tokens to sequence seq_ids[i] for i < batch, as one
- * forward chunk per sequence at loop count k, and choose the next token of
- * each sequence (greedy, lowest id on ties).
+ * forward chunk per sequence at loop count k (the input block once, the
+ * recurrent block k times on u_t = N(s_{t-1} + x), the output block and the
+ * LM head: [digest] "How it works"), and choose the next token of each
+ * sequence (greedy, lowest id on ties).
  *   seq_ids      host int32[batch], distinct, in [0, max_batch)
  *   tokens       device int32[sum(lens)], the sequences' tokens concatenated
  *   lens         host int32[batch], each >= 1; sum(lens) <= max_chunk
@@ -178,7 +180,9 @@ dory_status dory_prefill(dory_handle* h, int32_t batch, const int32_t* seq_ids, 
                          int32_t* next_tokens, dory_stream stream);
 
 /* One decode step: append tokens_in[i] to sequence seq_ids[i] and choose its
- * next token.  seq_ids host int32[batch]; tokens_in device int32[batch];
+ * next token (the same forward as dory_prefill on a one-token chunk; under
+ * LAST_LOOP the recurrent layers overwrite their one cache slot in every
+ * loop, [digest] "Premises & limits").  seq_ids host int32[batch]; tokens_in device int32[batch];
  * logits device float[batch, vocab] or NULL; next_tokens device int32[batch]. */
 dory_status dory_decode_step(dory_handle* h, int32_t batch, const int32_t* seq_ids, const int32_t* tokens_in,
                              int32_t k, dory_cache_mode mode, float* logits, int32_t* next_tokens,
